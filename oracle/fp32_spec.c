@@ -1,0 +1,152 @@
+/*
+ * fp32 weight-map specification, restated in plain C.
+ *
+ * TEST INFRASTRUCTURE ONLY: only tests/ (through oracle/spec.py) load this.
+ * It shares no code with the CUDA path; the GPU map must reproduce its output
+ * bit for bit on the same fp32 scores.
+ *
+ * Compile with -O2 -ffp-contract=off and without -ffast-math: every a*b+c
+ * below is two correctly rounded operations unless written as fmaf().
+ *
+ * The maps are the ones named on the pages ("Pretraining Transformers with
+ * Quantized Softmax in Attention", abstract: K-interval attention with K+1 grid
+ * values, per-row calibration, interpolation vs hard rounding; "Approximating
+ * Softmax in Pretrained LLMs", abstract: Rowmax-PoT, power-of-two weights
+ * anchored at the row maximum).  The fp32 operation order is this library's
+ * own specification (the pages fix none):
+ *
+ *   hi = max s, lo_obs = min s over the valid keys (exact in fp32)
+ *   EXACT      w = spec_exp(s - hi)
+ *   ROWMAX_POT x = fmaf(s, -L2E, hi*L2E);  n = rne(min(x, N))  (clamp)
+ *              or n = rne(min(x, N+1)), flushed when n > N      (flush)
+ *              w = 2^-n built from exponent bits
+ *   KINTERVAL  lo = lo_obs (min-max) or hi - W (fixed-window)
+ *              a = hi - lo; degenerate when !(a > 0): u = K
+ *              inv = K / a; b = -(lo*inv); u = fmaf(s, inv, b)
+ *              flushed when below_policy == 1, fixed-window and u < 0
+ *              uc = min(max(u, 0), K)
+ *              step = a / K (min-max) or W / K (fixed-window)
+ *              g[k] = spec_exp(-(K-k) * step), d[k] = g[k+1] - g[k]
+ *              hard   n = rne(uc), w = g[n]
+ *              interp k = min(floor(uc), K-1), f = uc - k, w = fmaf(f, d[k], g[k])
+ *   rne(x) = (x + 1.5*2^23) - 1.5*2^23  (round half to even, |x| < 2^22)
+ *
+ *   spec_exp(x): Cody-Waite reduction x = n*ln2 + r with n = rne(x*log2 e),
+ *   ln2 split into a 16-bit head and a tail; e^r by the degree-7 Taylor
+ *   polynomial (coefficients 1/k! rounded to fp32) in Horner form with fmaf;
+ *   scaled by 2^n through the exponent bits; 0 when n < -125.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define MODE_EXACT 0
+#define MODE_KINTERVAL 1
+#define MODE_POT 2
+#define CAL_MINMAX 0
+#define CAL_FIXED 1
+#define RND_INTERP 0
+#define RND_HARD 1
+
+static const float MAGIC = 12582912.0f;          /* 1.5 * 2^23 */
+static const float L2E = 1.44269502162933349609375f;   /* fp32(log2 e) */
+static const float LN2_HEAD = 0.693145751953125f;      /* ln 2, 16 bits */
+static const float LN2_TAIL = 1.428606765330187e-06f;  /* ln 2 - head   */
+
+static float bits2f(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t f2bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+static float rne(float x) { float t = x + MAGIC; return t - MAGIC; }
+
+float spec_exp(float x) {
+    float n = rne(x * L2E);
+    if (n < -125.0f) return 0.0f;
+    float r = fmaf(n, -LN2_HEAD, x);
+    r = fmaf(n, -LN2_TAIL, r);
+    float p = 1.98412701138295233249664306640625e-4f;  /* 1/7! */
+    p = fmaf(p, r, 1.38888892251998186111450195312500e-3f); /* 1/6! */
+    p = fmaf(p, r, 8.33333376795053482055664062500000e-3f); /* 1/5! */
+    p = fmaf(p, r, 4.16666679084300994873046875000000e-2f); /* 1/4! */
+    p = fmaf(p, r, 1.66666671633720397949218750000000e-1f); /* 1/3! */
+    p = fmaf(p, r, 0.5f);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int32_t e = (int32_t)n;                  /* exact: n is integral */
+    return p * bits2f((uint32_t)(e + 127) << 23);
+}
+
+/*
+ * Map `rows` rows of `cols` fp32 scores.  valid_len[r] keys (a prefix) are
+ * valid in row r.  Outputs w [rows*cols] (0 where masked) and idx
+ * [rows*cols] (node / lower node / exponent; -1 masked, -2 flushed), and the
+ * per-row hi and lo (lo = the calibrated lower end for K-interval, the observed
+ * minimum otherwise).
+ */
+void spec_map_rows(const float *s, int rows, int cols, const int *valid_len,
+                   int mode, int K, int calib, int rounding, float window,
+                   int pot_floor, int below_policy, float *w, int *idx,
+                   float *hi_out, float *lo_out) {
+    float g[257], d[257];
+    for (int r = 0; r < rows; ++r) {
+        const float *sr = s + (size_t)r * cols;
+        float *wr = w + (size_t)r * cols;
+        int *ir = idx + (size_t)r * cols;
+        int L = valid_len[r];
+        float hi = -INFINITY, lo = INFINITY;
+        for (int j = 0; j < L; ++j) {
+            if (sr[j] > hi) hi = sr[j];
+            if (sr[j] < lo) lo = sr[j];
+        }
+        for (int j = L; j < cols; ++j) { wr[j] = 0.0f; ir[j] = -1; }
+        if (mode == MODE_EXACT) {
+            for (int j = 0; j < L; ++j) { wr[j] = spec_exp(sr[j] - hi); ir[j] = 0; }
+        } else if (mode == MODE_POT) {
+            float hl = hi * L2E;
+            float cap = below_policy ? (float)(pot_floor + 1) : (float)pot_floor;
+            for (int j = 0; j < L; ++j) {
+                float x = fmaf(sr[j], -L2E, hl);
+                float t = fminf(x, cap) + MAGIC;
+                int32_t n = (int32_t)f2bits(t) - (int32_t)f2bits(MAGIC);
+                if (n > pot_floor) { wr[j] = 0.0f; ir[j] = -2; continue; }
+                wr[j] = bits2f((uint32_t)(127 - n) << 23);
+                ir[j] = n;
+            }
+        } else {
+            float lc = (calib == CAL_MINMAX) ? lo : hi - window;
+            float a = hi - lc;
+            int degenerate = !(a > 0.0f);
+            float Kf = (float)K;
+            float step = (calib == CAL_MINMAX) ? a / Kf : window / Kf;
+            for (int k = 0; k <= K; ++k) g[k] = spec_exp(-(float)(K - k) * step);
+            for (int k = 0; k < K; ++k) d[k] = g[k + 1] - g[k];
+            float inv = degenerate ? 0.0f : Kf / a;
+            float b = -(lc * inv);
+            lo = lc;
+            for (int j = 0; j < L; ++j) {
+                float u = degenerate ? Kf : fmaf(sr[j], inv, b);
+                if (below_policy == 1 && calib == CAL_FIXED && u < 0.0f) {
+                    wr[j] = 0.0f; ir[j] = -2; continue;
+                }
+                float uc = fminf(fmaxf(u, 0.0f), Kf);
+                if (rounding == RND_HARD) {
+                    int32_t n = (int32_t)f2bits(uc + MAGIC) - (int32_t)f2bits(MAGIC);
+                    wr[j] = g[n];
+                    ir[j] = n;
+                } else {
+                    float kf = fminf(floorf(uc), Kf - 1.0f);
+                    float f = uc - kf;
+                    int k = (int)kf;
+                    wr[j] = fmaf(f, d[k], g[k]);
+                    ir[j] = k;
+                }
+            }
+        }
+        hi_out[r] = hi;
+        lo_out[r] = lo;
+    }
+}
+
+/* Vector form of spec_exp, for the accuracy pins. */
+void spec_exp_vec(const float *x, float *y, int n) {
+    for (int i = 0; i < n; ++i) y[i] = spec_exp(x[i]);
+}

@@ -1,0 +1,171 @@
+"""Pins for the oracle's backward rules.
+
+Each rule in ``oracle.attn_bwd`` claims to be the exact gradient of a stated
+surrogate graph with the forward's integer decisions frozen ("Pretraining
+Transformers with Quantized Softmax in Attention", abstract: backward rules
+including calibration derivatives; straight-through surrogate before or after
+normalization).  The tests below re-state each surrogate graph as a plain
+forward function (written here, not taken from the oracle) and compare central
+finite differences of it against the oracle's dQ, dK, dV.  Exact mode and the
+post-normalization surrogate with detached extrema are also checked against
+torch autograd of ordinary softmax attention.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as A
+
+
+def _frozen(s, K, calib, rounding, W):
+    """Decisions of the forward map, taken independently of the oracle."""
+    R, S = s.shape
+    hi = s.max(1)
+    lo = s.min(1)
+    amax = s.argmax(1)
+    amin = s.argmin(1)
+    lo_c = lo if calib == A.MINMAX else hi - W
+    d = (hi - lo_c) / K
+    u = (s - lo_c[:, None]) / d[:, None]
+    below = u < 0
+    uc = np.clip(u, 0, K)
+    if rounding == A.HARD:
+        node = np.rint(uc).astype(int)
+    else:
+        node = np.minimum(np.floor(uc), K - 1).astype(int)
+    return dict(amax=amax, amin=amin, below=below, node=node, s0=s.copy(), hi0=hi.copy(),
+                lo0=lo_c.copy())
+
+
+def _F(sv, hi, lo, fr, K, rounding):
+    """Forward map with frozen decisions, live in (sv, hi, lo); no clamping."""
+    a = hi - lo
+    d = a / K
+    R, S = sv.shape
+    rows = np.arange(R)[:, None]
+    kk = np.arange(K + 1)
+    g = np.exp(-(K - kk)[None, :] * d[:, None])
+    if rounding == A.HARD:
+        w = g[rows, fr["node"]]
+    else:
+        u = (sv - lo[:, None]) / d[:, None]
+        k = fr["node"]
+        f = u - k
+        w = (1 - f) * g[rows, k] + f * g[rows, k + 1]
+    return np.where(fr["below"], g[:, :1], w)
+
+
+def _surrogate_loss(q, k, v, dO, fr, K, calib, rounding, surrogate, detach, W, c):
+    s = c * (q @ k.T)
+    R = s.shape[0]
+    r = np.arange(R)
+    if detach:
+        hi, lo = fr["hi0"], fr["lo0"]
+    else:
+        hi = s[r, fr["amax"]]
+        lo = s[r, fr["amin"]] if calib == A.MINMAX else hi - W
+    if surrogate == A.SURR_NONE:
+        w = _F(s, hi, lo, fr, K, rounding)
+        p = w / w.sum(1, keepdims=True)
+    elif surrogate == A.SURR_PRE:
+        w = _F(fr["s0"], hi, lo, fr, K, rounding) + np.exp(s - fr["hi0"][:, None]) \
+            - np.exp(fr["s0"] - fr["hi0"][:, None])
+        p = w / w.sum(1, keepdims=True)
+    else:
+        w = _F(fr["s0"], hi, lo, fr, K, rounding)
+        sm = np.exp(s - s.max(1, keepdims=True))
+        sm /= sm.sum(1, keepdims=True)
+        sm0 = np.exp(fr["s0"] - fr["s0"].max(1, keepdims=True))
+        sm0 /= sm0.sum(1, keepdims=True)
+        p = w / w.sum(1, keepdims=True) + sm - sm0
+    return float((dO * (p @ v)).sum())
+
+
+CASES = [(K, cal, rnd, sur, det) for K in (4, 16) for cal in (0, 1) for rnd in (0, 1)
+         for sur in (0, 1, 2) for det in (False, True)]
+
+
+@pytest.mark.parametrize("K,calib,rounding,surrogate,detach", CASES)
+def test_finite_differences_of_surrogate_graph(K, calib, rounding, surrogate, detach):
+    rng = np.random.default_rng(100 + K + 7 * calib + 3 * rounding + 11 * surrogate + int(detach))
+    S, D = 9, 4
+    W = 2.5
+    q = rng.normal(size=(S, D))
+    k = rng.normal(size=(S, D))
+    v = rng.normal(size=(S, D))
+    dO = rng.normal(size=(S, D))
+    c = 1 / math.sqrt(D)
+    res = oracle.attn_bwd(q[None, None], k[None, None], v[None, None], dO[None, None], False,
+                          A.KINTERVAL, K=K, calib=calib, rounding=rounding,
+                          surrogate=surrogate, detach_extrema=detach, window=W)
+    fr = _frozen(c * (q @ k.T), K, calib, rounding, W)
+    h = 1e-6
+    for name, X, G in (("q", q, res["dQ"]), ("k", k, res["dK"]), ("v", v, res["dV"])):
+        for (i, d) in [(0, 0), (3, 1), (5, 2), (8, 3), (int(fr["amax"][2]), 0),
+                       (int(fr["amin"][4]), 1)]:
+            Xp = X.copy(); Xp[i, d] += h
+            Xm = X.copy(); Xm[i, d] -= h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = Xp
+            lp = _surrogate_loss(args["q"], args["k"], args["v"], dO, fr, K, calib, rounding,
+                                 surrogate, detach, W, c)
+            args[name] = Xm
+            lm = _surrogate_loss(args["q"], args["k"], args["v"], dO, fr, K, calib, rounding,
+                                 surrogate, detach, W, c)
+            fd = (lp - lm) / (2 * h)
+            an = G[0, 0, i, d]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, i, d, fd, an)
+
+
+@pytest.mark.parametrize("rounding", [0, 1])
+def test_shift_invariance_sum_of_ds_is_zero(rounding):
+    rng = np.random.default_rng(8)
+    s = rng.normal(size=(6, 20))
+    v = rng.normal(size=(20, 5))
+    dO = rng.normal(size=(6, 5))
+    ds, _, _ = A.attn_bwd_rows(s, np.ones_like(s, bool), v, dO, A.KINTERVAL, 4, A.MINMAX,
+                               rounding, A.SURR_NONE, False, 8.0)
+    np.testing.assert_allclose(ds.sum(1), 0.0, atol=1e-13)
+
+
+def _torch_softmax_grads(q, k, v, dO, causal):
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal)
+    (o * torch.tensor(dO)).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_backward_is_autograd(causal):
+    rng = np.random.default_rng(9)
+    B, H, S, D = 1, 2, 17, 8
+    q, k, v, dO = (rng.normal(size=(B, H, S, D)) for _ in range(4))
+    res = oracle.attn_bwd(q, k, v, dO, causal, A.EXACT)
+    gq, gk, gv = _torch_softmax_grads(q, k, v, dO, causal)
+    np.testing.assert_allclose(res["dQ"], gq, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(res["dK"], gk, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(res["dV"], gv, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("calib,rounding", [(0, 0), (0, 1), (1, 0), (1, 1)])
+def test_post_detached_is_softmax_backward_for_q_and_k(causal, calib, rounding):
+    rng = np.random.default_rng(10)
+    B, H, S, D = 1, 1, 15, 8
+    q, k, v, dO = (rng.normal(size=(B, H, S, D)) for _ in range(4))
+    res = oracle.attn_bwd(q, k, v, dO, causal, A.KINTERVAL, K=4, calib=calib,
+                          rounding=rounding, surrogate=A.SURR_POST, detach_extrema=True,
+                          window=3.0)
+    gq, gk, _ = _torch_softmax_grads(q, k, v, dO, causal)
+    np.testing.assert_allclose(res["dQ"], gq, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(res["dK"], gk, rtol=1e-10, atol=1e-12)
+    # dV uses the forward's approximate probabilities
+    P = np.eye(S)[None, None]
+    ident = oracle.attn_fwd(q, k, P, causal, A.KINTERVAL, K=4, calib=calib,
+                            rounding=rounding, window=3.0)["O"]
+    np.testing.assert_allclose(res["dV"], np.swapaxes(ident, -1, -2) @ dO, rtol=1e-10,
+                               atol=1e-12)
