@@ -14,6 +14,6 @@ __all__ = ["inputs", "qsm"]
 
 def __getattr__(name):
     if name == "qsm":
-        from . import qsm as _q
-        return _q
+        import importlib
+        return importlib.import_module(__name__ + ".qsm")
     raise AttributeError(name)

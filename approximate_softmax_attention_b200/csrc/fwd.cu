@@ -1,0 +1,620 @@
+// fwd.cu -- fused approximate-softmax attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (b, h) and sweeps the key/value
+// tiles of 128 rows ("QK tile -> row max -> power-of-two weights -> PV matmul
+// -> output", the tile loop of "Approximating Softmax in Pretrained LLMs",
+// wiki flowchart).  Roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, then K (statistics sweep) and
+//               K, V (main sweep) through a ring of shared-memory stages.
+//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (tcgen05, both
+//               operands in shared memory) and O += P V with P read from TMEM.
+//   warps 4-7   map group for query tile 0, one thread per row (TMEM lane).
+//   warps 8-11  map group for query tile 1.
+// TMEM (512 columns): S0 at 0, S1 at 128, O0 at 256, O1 at 384.  P (bf16 or
+// e4m3, packed) overwrites the S columns it was computed from.  During the
+// statistics sweep the O columns double as second S buffers.
+//
+// Approximate maps are defined against the row's final maximum (and minimum),
+// so they run a statistics sweep first (S tiles, max/min/argmax/argmin only,
+// no PV), then the main sweep with the row constants fixed.  The exact map
+// needs no such sweep: it rescales online, and rescales O only when the
+// running maximum grew by more than 2^8 in weight.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "internal.h"
+#include "sm100.cuh"
+#include "wmap.cuh"
+
+namespace qsm {
+
+enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
+
+struct FwdParams {
+  int S, nqt, nqb;
+  int causal;
+  int K;
+  int fixed_window;
+  int flush;        // below_policy == 1
+  int pot_floor;
+  float c;          // score scale
+  float cL2E;       // c * log2(e), exact map
+  float window;
+  float out_scale;  // v_descale / pscale
+  float pscale;     // P is stored as w * pscale (FP8 approximate maps: 64)
+  int num_stages;
+  uint32_t table_off, bar_off;
+  __nv_bfloat16 *O;
+  float *LSE, *hi, *lo;
+  int32_t *amax, *amin;
+  int8_t *dbg;
+  int32_t *status;
+  int debug_flags;
+};
+
+template <int D, bool FP8>
+struct Geo {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int ELEM = FP8 ? 1 : 2;
+  static constexpr int EPC = 128 / ELEM;                // elements per 128-byte swizzle row
+  static constexpr int CHUNKS = (D * ELEM) / 128;       // swizzle columns per tile
+  static constexpr int CHUNK_BYTES = 128 * 128;         // 128 rows x 128 bytes
+  static constexpr int TILE_BYTES = BM * D * ELEM;
+  static constexpr int MMA_K = FP8 ? 32 : 16;           // K of one MMA instruction
+  static constexpr int KSTEPS_QK = D / MMA_K;
+  static constexpr int KSTEPS_PV = BN / MMA_K;
+  static constexpr uint32_t FMT = FP8 ? 0u : 1u;        // e4m3 / bf16 format code
+  static constexpr uint32_t IDESC_QK = instr_desc(FMT, false, 128, BN);
+  static constexpr uint32_t IDESC_PV = instr_desc(FMT, true, 128, D);
+  static constexpr int P_COLS_PER_CHUNK = FP8 ? 8 : 16; // TMEM columns per 32 P values
+};
+
+constexpr int kThreads = 384;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+// barrier slots (uint64 each) after the stage barriers
+struct Bars {
+  uint64_t *kv_full, *kv_empty;   // [stages]
+  uint64_t *q_full;               // 1
+  uint64_t *s_full;               // [2 tiles][2 buffers]
+  uint64_t *s_empty;              // [2][2]
+  uint64_t *p_full;               // [2]
+  uint64_t *o_full;               // [2]
+  uint64_t *drain;                // 1
+  uint32_t *tmem_slot;
+  int *abort;
+};
+
+__device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
+  Bars b;
+  uint64_t *p = reinterpret_cast<uint64_t *>(base);
+  b.kv_full = p;
+  b.kv_empty = p + ns;
+  b.q_full = p + 2 * ns;
+  b.s_full = b.q_full + 1;
+  b.s_empty = b.s_full + 4;
+  b.p_full = b.s_empty + 4;
+  b.o_full = b.p_full + 2;
+  b.drain = b.o_full + 2;
+  b.tmem_slot = reinterpret_cast<uint32_t *>(b.drain + 1);
+  b.abort = reinterpret_cast<int *>(b.tmem_slot + 1);
+  return b;
+}
+
+template <int D, bool FP8, int MAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    qsm_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using G = Geo<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int qb = p.causal ? (p.nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  const int ns = p.num_stages;
+
+  uint8_t *sQ = smem;                                   // 2 tiles
+  uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages
+  float *sTab = reinterpret_cast<float *>(smem + p.table_off);
+  Bars bars = carve_bars(smem + p.bar_off, ns);
+  volatile int *abort = bars.abort;
+
+  const int nkvt = (p.S + 127) / 128;
+  int qi[2], nt[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    qi[t] = 2 * qb + t;
+    const bool exists = qi[t] < p.nqt;
+    nt[t] = exists ? (p.causal ? min(nkvt, qi[t] + 1) : nkvt) : 0;
+  }
+  const int nkv = max(nt[0], nt[1]);
+  constexpr bool kTwoPass = MAP != MAP_EXACT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ns; ++i) {
+      mbar_init(&bars.kv_full[i], 1);
+      mbar_init(&bars.kv_empty[i], 1);
+    }
+    mbar_init(bars.q_full, 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_empty[i], 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.p_full[i], 128);
+      mbar_init(&bars.o_full[i], 1);
+    }
+    mbar_init(bars.drain, 1);
+    *bars.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(bars.tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *bars.tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !(p.debug_flags & 1)) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const int nq = (nt[0] > 0) + (nt[1] > 0);
+      mbar_expect_tx(bars.q_full, nq * G::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        if (nt[t] > 0)
+          for (int ch = 0; ch < G::CHUNKS; ++ch)
+            tma_load_3d(sQ + t * G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmQ, bars.q_full,
+                        ch * G::EPC, qi[t] * 128, bh);
+      int it = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap *m, int kvt) {
+        const int st = it % ns;
+        if (it >= ns) ok = ok && mbar_wait(&bars.kv_empty[st], ((it / ns) & 1) ^ 1, abort);
+        if (!ok) return;
+        mbar_expect_tx(&bars.kv_full[st], G::TILE_BYTES);
+        for (int ch = 0; ch < G::CHUNKS; ++ch)
+          tma_load_3d(sKV + st * G::TILE_BYTES + ch * G::CHUNK_BYTES, m, &bars.kv_full[st],
+                      ch * G::EPC, kvt * 128, bh);
+        ++it;
+      };
+      if (kTwoPass)
+        for (int j = 0; j < nkv && ok; ++j) load(&tmK, j);
+      for (int j = 0; j < nkv && ok; ++j) {
+        load(&tmK, j);
+        load(&tmV, j);
+      }
+      // let every load issued so far land before the CTA may exit
+      mbar_wait(bars.q_full, 0, abort);
+      for (int st = 0; st < ns && st < it; ++st) {
+        const int fills = (it - st + ns - 1) / ns;  // loads issued into stage st
+        mbar_wait(&bars.kv_full[st], (fills - 1) & 1, abort);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t qaddr0 = smem_u32(sQ);
+      const uint32_t kvaddr0 = smem_u32(sKV);
+      int it = 0;
+      bool ok = mbar_wait(bars.q_full, 0, abort);
+      tc_fence_after();
+      auto acquire = [&]() -> int {
+        const int st = it % ns;
+        ok = ok && mbar_wait(&bars.kv_full[st], (it / ns) & 1, abort);
+        ++it;
+        tc_fence_after();
+        return st;
+      };
+      auto issue_qk = [&](int t, int st, uint32_t scol) {
+        const uint32_t qa = qaddr0 + t * G::TILE_BYTES;
+        const uint32_t ka = kvaddr0 + st * G::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < G::KSTEPS_QK; ++kk) {
+          const int e = kk * G::MMA_K;
+          const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * G::ELEM;
+          const uint64_t ad = smem_desc(qa + off, 16, 1024);
+          const uint64_t bd = smem_desc(ka + off, 16, 1024);
+          if (FP8)
+            mma_ss_f8(tmem + scol, ad, bd, G::IDESC_QK, kk > 0);
+          else
+            mma_ss_f16(tmem + scol, ad, bd, G::IDESC_QK, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t va = kvaddr0 + st * G::TILE_BYTES;
+        const uint32_t pcol = t * 128;
+        const uint32_t ocol = 256 + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
+          const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
+          const uint32_t at = tmem + pcol + kk * 8;
+          if (FP8)
+            mma_ts_f8(tmem + ocol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+          else
+            mma_ts_f16(tmem + ocol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      if (kTwoPass) {
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int st = acquire();
+          if (!ok) break;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= nt[t]) continue;
+            const int b = j & 1, use = j >> 1;
+            if (use >= 1) {
+              ok = mbar_wait(&bars.s_empty[t * 2 + b], (use - 1) & 1, abort);
+              tc_fence_after();
+              if (!ok) break;
+            }
+            issue_qk(t, st, t * 128 + b * 256);
+            mma_commit(&bars.s_full[t * 2 + b]);
+          }
+          mma_commit(&bars.kv_empty[st]);
+        }
+        // both S buffers of each tile must be read out before the main sweep
+        for (int t = 0; t < 2 && ok; ++t) {
+          const int u0 = (nt[t] + 1) / 2, u1 = nt[t] / 2;
+          if (u0 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 0], (u0 - 1) & 1, abort);
+          if (u1 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 1], (u1 - 1) & 1, abort);
+        }
+        tc_fence_after();
+      }
+      if (ok && nkv > 0) {
+        const int k0 = acquire();
+        if (ok) {
+          for (int t = 0; t < 2; ++t)
+            if (nt[t] > 0) {
+              issue_qk(t, k0, t * 128);
+              mma_commit(&bars.s_full[t * 2 + 0]);
+            }
+          mma_commit(&bars.kv_empty[k0]);
+        }
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int vst = acquire();
+          const bool has_next = j + 1 < nkv;
+          const int knext = has_next ? acquire() : -1;
+          if (!ok) break;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j < nt[t]) {
+              ok = mbar_wait(&bars.p_full[t], j & 1, abort);
+              tc_fence_after();
+              if (!ok) break;
+              issue_pv(t, vst, j > 0);
+            }
+            if (has_next && j + 1 < nt[t]) {
+              issue_qk(t, knext, t * 128);
+              mma_commit(&bars.s_full[t * 2 + 0]);
+            }
+          }
+          mma_commit(&bars.kv_empty[vst]);
+          if (has_next) mma_commit(&bars.kv_empty[knext]);
+        }
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] > 0) mma_commit(&bars.o_full[t]);
+      }
+      // every MMA issued must finish before TMEM is released
+      mma_commit(bars.drain);
+      mbar_wait(bars.drain, 0, abort);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ map groups
+    const int t = (warp - 4) >> 2;
+    const int row = threadIdx.x - 128 - t * 128;         // 0..127 == TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int qrow = qi[t] * 128 + row;
+    const bool row_ok = qrow < p.S;
+    const int L = p.causal ? min(qrow + 1, p.S) : p.S;   // valid keys of the row
+    const int n_t = nt[t];
+    if (n_t > 0) {
+      uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
+      bool ok = true;
+      float rmax = -INFINITY, rmin = INFINITY;
+      int amax = 0, amin = 0;
+      const bool want_arg = p.amax != nullptr || p.amin != nullptr;
+      const bool want_min =
+          ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window) || p.lo != nullptr;
+
+      // ------------------------------------------------ statistics sweep
+      if (kTwoPass) {
+        for (int j = 0; j < n_t && ok; ++j) {
+          const int b = j & 1;
+          ok = mbar_wait(&bars.s_full[t * 2 + b], (b ? sf_cnt1 : sf_cnt0) & 1, abort);
+          if (b) ++sf_cnt1; else ++sf_cnt0;
+          if (!ok) break;
+          tc_fence_after();
+          const int lim = L - 128 * j;
+          const uint32_t base = lane_base + t * 128 + b * 256;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(base + 32 * cc, v);
+            tmem_wait_ld();
+            const int c0 = 32 * cc;
+            if (want_arg) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(v[i]);
+                const bool valid = c0 + i < lim;
+                if (valid && x > rmax) { rmax = x; amax = 128 * j + c0 + i; }
+                if (valid && x < rmin) { rmin = x; amin = 128 * j + c0 + i; }
+              }
+            } else if (lim >= c0 + 32) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(v[i]);
+                rmax = fmaxf(rmax, x);
+                if (want_min) rmin = fminf(rmin, x);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(v[i]);
+                if (c0 + i < lim) {
+                  rmax = fmaxf(rmax, x);
+                  if (want_min) rmin = fminf(rmin, x);
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&bars.s_empty[t * 2 + b]);
+        }
+      }
+
+      // ------------------------------------------------------ main sweep
+      float Z = 0.0f;
+      float hi = 0.0f, lo = 0.0f;
+      float m_used = -INFINITY, m_run = -INFINITY;        // exact map, raw units
+      RowMap rm;
+      float *tab = sTab + t * (p.K + 1) * 128;
+      const float Kf = static_cast<float>(p.K);
+      const float cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
+      if (kTwoPass && ok) {
+        hi = __fmul_rn(p.c, rmax);
+        lo = __fmul_rn(p.c, rmin);
+        rm = make_rowmap(hi, lo, p.K, p.fixed_window != 0, p.window);
+        if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP)
+          for (int n = 0; n <= p.K; ++n) tab[n * 128 + row] = grid_value(rm, p.K, n);
+        lo = (MAP == MAP_POT) ? lo : rm.lo;
+      }
+      int8_t *dbg_row = (p.dbg != nullptr && row_ok)
+                            ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
+                            : nullptr;
+      for (int j = 0; j < n_t && ok; ++j) {
+        ok = mbar_wait(&bars.s_full[t * 2 + 0], sf_cnt0 & 1, abort);
+        ++sf_cnt0;
+        if (!ok) break;
+        tc_fence_after();
+        const int lim = L - 128 * j;
+        const uint32_t sbase = lane_base + t * 128;
+        if (MAP == MAP_EXACT) {
+          float mt = -INFINITY;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(sbase + 32 * cc, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (32 * cc + i < lim) mt = fmaxf(mt, __uint_as_float(v[i]));
+          }
+          m_run = fmaxf(m_run, mt);
+          if (m_used == -INFINITY || (m_run - m_used) * p.cL2E > kRescaleLog2) {
+            if (m_used != -INFINITY) {
+              const float alpha = ex2_approx((m_used - m_run) * p.cL2E);
+              Z *= alpha;
+              const uint32_t obase = lane_base + 256 + t * 128;
+#pragma unroll 1
+              for (int dc = 0; dc < D / 32; ++dc) {
+                uint32_t v[32];
+                tmem_ld32(obase + 32 * dc, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                tmem_st32(obase + 32 * dc, v);
+              }
+            }
+            m_used = m_run;
+          }
+        }
+        const float mb = m_used * p.cL2E;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(sbase + 32 * cc, v);
+          tmem_wait_ld();
+          float w[32];
+          int dn[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(v[i]);
+            const bool valid = 32 * cc + i < lim;
+            float wi;
+            int n = 0;
+            if (MAP == MAP_EXACT) {
+              wi = ex2_approx(__fmaf_rn(x, p.cL2E, -mb));
+            } else {
+              const float s = __fmul_rn(x, p.c);
+              if (MAP == MAP_POT) {
+                wi = pot_weight(s, rm.hiL2E, cap, p.pot_floor, p.flush != 0, n);
+              } else {
+                const float u = kint_u(s, rm, Kf);
+                if (p.flush && p.fixed_window && u < 0.0f) {
+                  wi = 0.0f;
+                  n = -2;
+                } else if (MAP == MAP_KI_HARD) {
+                  n = kint_hard_node(u, Kf);
+                  wi = tab[n * 128 + row];
+                } else {
+                  float f;
+                  n = kint_interp_node(u, Kf, f);
+                  wi = kint_interp_weight(f, tab[n * 128 + row], tab[(n + 1) * 128 + row]);
+                }
+              }
+            }
+            w[i] = valid ? wi : 0.0f;
+            dn[i] = valid ? n : -1;
+            Z += w[i];
+          }
+          if (FP8) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              pk[i] = pack_e4m3x4(w[4 * i] * p.pscale, w[4 * i + 1] * p.pscale,
+                                  w[4 * i + 2] * p.pscale, w[4 * i + 3] * p.pscale);
+            tmem_st8(sbase + cc * 8, pk);
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
+            tmem_st16(sbase + cc * 16, pk);
+          }
+          if (dbg_row != nullptr) {
+            const int kv0 = 128 * j + 32 * cc;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (kv0 + i < p.S) dbg_row[kv0 + i] = static_cast<int8_t>(dn[i]);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars.p_full[t]);
+      }
+
+      // -------------------------------------------------------- epilogue
+      if (ok) ok = mbar_wait(&bars.o_full[t], 0, abort);
+      if (ok) {
+        tc_fence_after();
+        if (MAP == MAP_EXACT) hi = p.c * m_run;
+        const float oscale = p.out_scale / Z;
+        const uint32_t obase = lane_base + 256 + t * 128;
+        __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D;
+#pragma unroll 1
+        for (int dc = 0; dc < D / 32; ++dc) {
+          uint32_t v[32];
+          tmem_ld32(obase + 32 * dc, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * oscale,
+                                __uint_as_float(v[2 * i + 1]) * oscale);
+          if (row_ok) {
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * dc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+        if (row_ok) {
+          const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
+          const float anchor = (MAP == MAP_EXACT) ? p.c * m_used : hi;
+          p.LSE[ri] = anchor + logf(Z);
+          if (p.hi) p.hi[ri] = hi;
+          if (MAP != MAP_EXACT) {          // the exact map runs no statistics sweep
+            if (p.lo) p.lo[ri] = lo;
+            if (p.amax) p.amax[ri] = amax;
+            if (p.amin) p.amin[ri] = amin;
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (threadIdx.x == 0 && *bars.abort && p.status != nullptr) atomicExch(p.status, QSM_ERR_TIMEOUT);
+}
+
+// ------------------------------------------------------------------- host
+
+template <int D, bool FP8, int MAP>
+static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                           const CUtensorMap &mv) {
+  using G = Geo<D, FP8>;
+  FwdParams p{};
+  p.S = a.S;
+  p.nqt = (a.S + 127) / 128;
+  p.nqb = (p.nqt + 1) / 2;
+  p.causal = a.causal;
+  p.K = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) ? a.Kint : 1;
+  p.fixed_window = a.calib == QSM_CALIB_FIXED_WINDOW;
+  p.flush = a.below_policy == 1;
+  p.pot_floor = a.pot_floor;
+  p.c = a.c;
+  p.cL2E = a.c * 1.4426950408889634f;
+  p.window = a.window;
+  p.pscale = (FP8 && MAP != MAP_EXACT) ? 64.0f : 1.0f;
+  p.out_scale = a.v_descale / p.pscale;
+  p.O = static_cast<__nv_bfloat16 *>(a.O);
+  p.LSE = a.LSE;
+  p.hi = a.row_hi;
+  p.lo = a.row_lo;
+  p.amax = a.row_argmax;
+  p.amin = a.row_argmin;
+  p.dbg = a.debug_idx;
+  p.status = a.status_dev;
+  p.debug_flags = a.debug_flags;
+
+  const size_t table_bytes = static_cast<size_t>(2) * (p.K + 1) * 128 * sizeof(float);
+  const size_t bar_bytes = 256;
+  const size_t max_smem = 232448;                        // 227 KB opt-in per CTA
+  const size_t fixed = 1024 + 2 * G::TILE_BYTES + table_bytes + bar_bytes;
+  int ns = static_cast<int>((max_smem - fixed) / G::TILE_BYTES);
+  if (ns > 4) ns = 4;
+  if (ns < 2) return QSM_ERR_UNSUPPORTED;
+  p.num_stages = ns;
+  p.table_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * G::TILE_BYTES);
+  p.bar_off = static_cast<uint32_t>((p.table_off + table_bytes + 15) & ~static_cast<size_t>(15));
+  size_t smem = 1024 + p.bar_off + bar_bytes;
+  // one CTA per SM: the kernel allocates all 512 TMEM columns
+  if (smem < 120 * 1024) smem = 120 * 1024;
+
+  auto kern = qsm_fwd_kernel<D, FP8, MAP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return QSM_ERR_CUDA;
+  dim3 grid(p.nqb, a.B * a.H);
+  kern<<<grid, kThreads, smem, a.stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+}
+
+template <int D, bool FP8>
+static qsm_status launch_d(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                           const CUtensorMap &mv) {
+  if (a.mode == QSM_MODE_EXACT) return launch_t<D, FP8, MAP_EXACT>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_ROWMAX_POT) return launch_t<D, FP8, MAP_POT>(a, mq, mk, mv);
+  if (a.rounding == QSM_ROUND_HARD) return launch_t<D, FP8, MAP_KI_HARD>(a, mq, mk, mv);
+  return launch_t<D, FP8, MAP_KI_INTERP>(a, mq, mk, mv);
+}
+
+qsm_status launch_fwd(const FwdArgs &a) {
+  alignas(64) CUtensorMap mq, mk, mv;
+  const int bh = a.B * a.H;
+  if (!make_tmap_3d(&mq, a.Q, a.fp8, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&mk, a.K, a.fp8, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&mv, a.V, a.fp8, a.D, a.S, bh, 128))
+    return QSM_ERR_CUDA;
+  if (a.fp8) {
+    if (a.D == 128) return launch_d<128, true>(a, mq, mk, mv);
+    return QSM_ERR_UNSUPPORTED;
+  }
+  if (a.D == 128) return launch_d<128, false>(a, mq, mk, mv);
+  if (a.D == 64) return launch_d<64, false>(a, mq, mk, mv);
+  return QSM_ERR_UNSUPPORTED;
+}
+
+}  // namespace qsm

@@ -1,0 +1,72 @@
+// internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/qsm.h"
+
+namespace qsm {
+
+// Everything a forward launch needs, validated by the C entry point.
+struct FwdArgs {
+  const void *Q, *K, *V;
+  void *O;
+  float *LSE;
+  int B, H, S, D;
+  int causal;
+  int mode, Kint, calib, rounding;
+  int fp8;
+  float c;          // scale * q_descale * k_descale
+  float v_descale;
+  float window;
+  int pot_floor, below_policy;
+  float *row_hi, *row_lo;
+  int32_t *row_argmax, *row_argmin;
+  int8_t *debug_idx;
+  int32_t *status_dev;
+  int debug_flags;
+  cudaStream_t stream;
+};
+
+qsm_status launch_fwd(const FwdArgs &a);
+
+struct MapArgs {
+  const float *scores;
+  const int32_t *valid_len;
+  int rows, cols;
+  int mode, Kint, calib, rounding;
+  float window;
+  int pot_floor, below_policy;
+  float *w;
+  int32_t *idx;
+  float *hi, *lo;
+  cudaStream_t stream;
+};
+
+qsm_status launch_weight_map(const MapArgs &a);
+
+struct BwdArgs {
+  const void *Q, *K, *V, *O, *dO;
+  const float *LSE;
+  void *dQ, *dK, *dV;
+  int B, H, S, D, causal;
+  int mode, Kint, calib, rounding, surrogate, detach;
+  float c, window;
+  int below_policy;
+  const float *row_hi, *row_lo;
+  const int32_t *row_argmax, *row_argmin;
+  void *workspace;
+  size_t workspace_bytes;
+  int32_t *status_dev;
+  cudaStream_t stream;
+};
+
+qsm_status launch_bwd(const BwdArgs &a);
+size_t bwd_workspace_bytes(int B, int H, int S, int D);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+bool make_tmap_3d(void *map_out, const void *base, bool fp8, int D, int S, int BH, int box_rows);
+
+}  // namespace qsm

@@ -1,0 +1,233 @@
+"""GPU parity of the forward path against the CPU oracle, through the C ABI.
+
+Tolerances (stated for the maps in "Approximating Softmax in Pretrained
+LLMs" / "Pretraining Transformers with Quantized Softmax in Attention", as
+readings of the forward they describe):
+  * the weight map on given fp32 scores is bit-exact with the C fp32 spec;
+  * bf16 attention output: max abs <= 1e-2, mean abs <= 1e-3 against fp64;
+  * e4m3 attention output: max abs <= 5e-2;
+  * grid node / PoT exponent agreement >= 99.9 %, every mismatch within 1e-3
+    (coordinate units) of a rounding boundary.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import spec
+from oracle import attention as A
+from approximate_softmax_attention_b200 import inputs, qsm
+
+from _helpers import boundary_distance_rows, err_stats
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _gpu(x):
+    return x.to(DEV).contiguous()
+
+
+# ------------------------------------------------------------ weight map
+
+MAP_CASES = [(0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1)] + \
+    [(1, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
+    [(1, 4, 1, 1, 1), (1, 16, 1, 0, 1)]
+
+
+@pytest.mark.parametrize("mode,K,calib,rounding,below", MAP_CASES)
+def test_weight_map_bit_exact(mode, K, calib, rounding, below):
+    rows, cols = 300, 517
+    s = inputs.scores_fp32(rows, cols, seed=40 + K + 3 * mode + calib + 7 * rounding).numpy()
+    rng = np.random.default_rng(K + mode)
+    vl = rng.integers(1, cols + 1, size=rows).astype(np.int32)
+    vl[:3] = [1, 2, cols]
+    s[5, :] = 0.5                                   # degenerate row
+    # adversarial: scores placed on and next to node boundaries of row 6
+    hi, lo = s[6].max(), s[6].min()
+    step = (hi - lo) / K
+    for i in range(40):
+        base = lo + (i % (K + 1)) * step + (0.5 * step if rounding == 1 else 0.0)
+        toward = (-np.inf, base, np.inf)[i % 3]
+        s[6, 10 + i] = np.nextafter(np.float32(base), np.float32(toward))
+    window = 6.0
+    w_ref, i_ref, hi_ref, lo_ref = spec.spec_map(s, vl, mode, K=K, calib=calib,
+                                                 rounding=rounding, window=window,
+                                                 pot_floor=15, below_policy=below)
+    S = _gpu(torch.from_numpy(s))
+    VL = _gpu(torch.from_numpy(vl))
+    W = torch.empty_like(S)
+    I = torch.empty(rows, cols, dtype=torch.int32, device=DEV)
+    HI = torch.empty(rows, dtype=torch.float32, device=DEV)
+    LO = torch.empty(rows, dtype=torch.float32, device=DEV)
+    opts = qsm.make_opts(window=window, pot_floor=15, below_policy=below)
+    st = qsm.qsm_weight_map(S, VL, mode, K, calib, rounding, opts, W, I, HI, LO)
+    assert st == qsm.QSM_OK
+    torch.cuda.synchronize()
+    assert np.array_equal(W.cpu().numpy().view(np.uint32), w_ref.view(np.uint32))
+    assert np.array_equal(I.cpu().numpy(), i_ref)
+    assert np.array_equal(HI.cpu().numpy().view(np.uint32), hi_ref.view(np.uint32))
+    assert np.array_equal(LO.cpu().numpy().view(np.uint32), lo_ref.view(np.uint32))
+
+
+# ------------------------------------------------------------- forward
+
+def _run_fwd(d, causal, mode, K, calib, rounding, window=8.0, below=0, debug=False):
+    q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    B, H, S, D = q.shape
+    dbg = torch.full((B, H, S, S), -7, dtype=torch.int8, device=DEV) if debug else None
+    O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rounding,
+                                       q_descale=d["q_descale"], k_descale=d["k_descale"],
+                                       v_descale=d["v_descale"], window=window,
+                                       below_policy=below, stats=True, debug_idx=dbg)
+    torch.cuda.synchronize()
+    out = dict(O=O.float().cpu().numpy(), LSE=LSE.cpu().numpy(),
+               hi=st["hi"].cpu().numpy(), lo=st["lo"].cpu().numpy(),
+               argmax=st["argmax"].cpu().numpy(), argmin=st["argmin"].cpu().numpy())
+    if debug:
+        out["idx"] = dbg.cpu().numpy()
+    return out
+
+
+def _oracle(d, causal, mode, K, calib, rounding, window=8.0, below=0, want_idx=False,
+            heads=None, rows=None):
+    return oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, K=K, calib=calib,
+                           rounding=rounding, q_descale=d["q_descale"],
+                           k_descale=d["k_descale"], v_descale=d["v_descale"], window=window,
+                           below_policy=below, want_idx=want_idx, heads=heads, rows=rows)
+
+
+def _check_idx(d, got_idx, ref_idx, causal, mode, K, calib, rounding, window):
+    if mode == A.EXACT:
+        return
+    q = d["q"].double().numpy() * d["q_descale"]
+    k = d["k"].double().numpy() * d["k_descale"]
+    B, H, S, D = q.shape
+    total = 0
+    bad = 0
+    for b in range(B):
+        for h in range(H):
+            s = (q[b, h] @ k[b, h].T) / math.sqrt(D)
+            valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal \
+                else np.ones((S, S), bool)
+            dist = boundary_distance_rows(s, valid, mode, K, calib, rounding, window)
+            g = got_idx[b, h].astype(np.int64)
+            r = ref_idx[b, h].astype(np.int64)
+            assert np.all(g[~valid] == -1)
+            mism = (g != r) & valid
+            assert np.all(dist[mism] <= 1e-3), (b, h, np.argwhere(mism & (dist > 1e-3))[:5])
+            bad += int(mism.sum())
+            total += int(valid.sum())
+    assert bad <= 1e-3 * total, (bad, total)
+
+
+MODES_FWD = [(0, 4, 0, 1), (2, 4, 0, 1), (1, 4, 0, 1), (1, 4, 0, 0), (1, 4, 1, 1),
+             (1, 16, 1, 0), (1, 16, 0, 0)]
+
+
+def test_tiny_config_all_modes():
+    """B=1, H=2, S=128, D=64 bf16, non-causal, seed 0: exact, K-interval K=4
+    (min-max, hard) and Rowmax-PoT against the oracle, with decision dumps."""
+    w = inputs.WORKLOADS["tiny"]
+    d = inputs.draw_workload(w)
+    for (mode, K, calib, rnd) in w.modes:
+        got = _run_fwd(d, w.causal, mode, K, calib, rnd, debug=True)
+        ref = _oracle(d, w.causal, mode, K, calib, rnd, want_idx=True)
+        mx, mean = err_stats(got["O"], ref["O"])
+        assert mx <= 1e-2 and mean <= 1e-3, (mode, mx, mean)
+        np.testing.assert_allclose(got["LSE"], ref["LSE"], atol=2e-3, rtol=1e-4)
+        np.testing.assert_allclose(got["hi"], ref["hi"], atol=1e-4, rtol=1e-5)
+        if mode != 0:
+            assert np.array_equal(got["argmax"], ref["argmax"])
+            assert np.array_equal(got["argmin"], ref["argmin"])
+        _check_idx(d, got["idx"], ref["idx"], w.causal, mode, K, calib, rnd, 8.0)
+
+
+@pytest.mark.parametrize("S,D,causal", [(1, 64, False), (77, 64, True), (200, 128, False),
+                                        (384, 128, True), (520, 64, True), (300, 128, True)])
+@pytest.mark.parametrize("mode,K,calib,rounding", MODES_FWD)
+def test_fwd_bf16_shapes(S, D, causal, mode, K, calib, rounding):
+    d = inputs.draw(1, 2, S, D, seed=S + D, peaked=S > 100)
+    got = _run_fwd(d, causal, mode, K, calib, rounding, window=6.0, debug=S <= 384)
+    ref = _oracle(d, causal, mode, K, calib, rounding, window=6.0, want_idx=S <= 384)
+    mx, mean = err_stats(got["O"], ref["O"])
+    assert mx <= 1e-2 and mean <= 1e-3, (mx, mean)
+    np.testing.assert_allclose(got["LSE"], ref["LSE"], atol=2e-3, rtol=1e-4)
+    if S <= 384:
+        _check_idx(d, got["idx"], ref["idx"], causal, mode, K, calib, rounding, 6.0)
+
+
+@pytest.mark.parametrize("below", [0, 1])
+def test_fwd_below_policy(below):
+    d = inputs.draw(1, 2, 256, 64, seed=9, peaked=True)
+    # a narrow window pushes many keys below it
+    for (mode, K, calib, rnd) in [(1, 4, 1, 1), (1, 4, 1, 0), (2, 4, 0, 1)]:
+        got = _run_fwd(d, True, mode, K, calib, rnd, window=1.5, below=below, debug=True)
+        ref = oracle.attn_fwd(d["q"], d["k"], d["v"], True, mode, K=K, calib=calib,
+                              rounding=rnd, window=1.5, pot_floor=15, below_policy=below,
+                              want_idx=True)
+        mx, mean = err_stats(got["O"], ref["O"])
+        assert mx <= 1e-2 and mean <= 1e-3, (mode, mx, mean)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("mode,K,calib,rounding", [(0, 4, 1, 1), (2, 4, 1, 1), (1, 4, 1, 1),
+                                                  (1, 16, 0, 0)])
+def test_fwd_fp8(causal, mode, K, calib, rounding):
+    d = inputs.draw(1, 2, 640, 128, seed=3, peaked=True, dtype="fp8")
+    got = _run_fwd(d, causal, mode, K, calib, rounding, debug=True)
+    ref = _oracle(d, causal, mode, K, calib, rounding, want_idx=True)
+    mx, mean = err_stats(got["O"], ref["O"])
+    assert mx <= 5e-2, (mx, mean)
+    _check_idx(d, got["idx"], ref["idx"], causal, mode, K, calib, rounding, 8.0)
+
+
+def _sampled_check(name, tol_max, tol_mean, nheads=3, nrows=96):
+    w = inputs.WORKLOADS[name]
+    d = inputs.draw_workload(w)
+    rng = np.random.default_rng(0)
+    heads = [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(nheads)]
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, w.S - 1],
+                                     rng.integers(0, w.S, size=nrows)]))
+    for (mode, K, calib, rnd) in w.modes:
+        got = _run_fwd(d, w.causal, mode, K, calib, rnd)
+        ref = _oracle(d, w.causal, mode, K, calib, rnd, heads=heads, rows=rows)
+        for (b, h) in heads:
+            mx, mean = err_stats(got["O"][b, h, rows], ref["O"][b, h, rows])
+            assert mx <= tol_max and mean <= tol_mean, (name, mode, b, h, mx, mean)
+            np.testing.assert_allclose(got["LSE"][b, h, rows], ref["LSE"][b, h, rows],
+                                       atol=5e-3, rtol=1e-4)
+        assert np.isfinite(got["O"]).all()
+
+
+def test_full_size_s2k_bf16_causal_sampled():
+    """B=4, H=16, S=2048, D=128 bf16 causal, peaked keys: the bench workload,
+    launched as the bench launches it, checked on sampled rows."""
+    _sampled_check("s2k_bf16_causal", 1e-2, 1e-3)
+
+
+@pytest.mark.parametrize("name", ["s8k_fp8", "s8k_fp8_causal"])
+def test_full_size_s8k_fp8_sampled(name):
+    _sampled_check(name, 5e-2, 5e-3, nheads=2, nrows=48)
+
+
+def test_timeout_path_reports_status_and_context_survives():
+    d = inputs.draw(1, 1, 256, 64, seed=1)
+    q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    O = torch.empty(1, 1, 256, 64, dtype=torch.bfloat16, device=DEV)
+    LSE = torch.empty(1, 1, 256, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    opts = qsm.make_opts(status_dev=status, debug_flags=1)
+    assert qsm.qsm_attn_fwd(q, k, v, O, LSE, False, qsm.MODE_ROWMAX_POT, 4, 0, 1, 0,
+                            opts) == qsm.QSM_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) == qsm.QSM_ERR_TIMEOUT
+    # the context is still usable
+    O2, _ = qsm.attention_forward(q, k, v, False, qsm.MODE_EXACT)
+    torch.cuda.synchronize()
+    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], False, A.EXACT)
+    assert err_stats(O2.float().cpu().numpy(), ref["O"])[0] <= 1e-2
