@@ -1,0 +1,450 @@
+"""Benchmark of the approximate-softmax attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): the forward of the B=4, H=16, S=2048, D=128 bf16 causal
+problem with peaked keys (1% of keys shifted +3 along a per-head unit
+direction), once per map: exact softmax, Rowmax-PoT, and K-interval K=16
+(min-max calibration, interpolation).  ``value`` is the step's algorithmic
+TFLOP/s (4*B*H*S^2*D per call, halved for causal; the statistics sweep of
+the approximate maps is not counted), whole job, inputs resident in HBM.
+Inputs rotate over three device copies (3 x 100 MB > the 126 MB L2), so no
+call starts with its operands in L2.
+
+The line also carries per-map TFLOP/s, the roofline of the dominant kernel
+(CUDA events on the launching stream), the oracle timed on the host cores on
+a bounded sample, an end-to-end number through host buffers, sampled SM
+clocks, and secondary per-map figures for the 8K / 16K problems.
+
+With --gpus N (launched under torchrun) every rank runs the same per-rank
+problem on its own GPU (data-parallel over independent batches; there is no
+exchange step), timing is the max over ranks and ``value`` sums all ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+MAIN_WORKLOAD = "s2k_bf16_causal"
+EXTRA_WORKLOADS = ("s8k_fp8", "s8k_bf16", "s8k_fp8_causal")
+MODE_NAMES = {0: "exact", 1: "kinterval", 2: "rowmax_pot"}
+CALIB_NAMES = {0: "minmax", 1: "fixed_window"}
+ROUND_NAMES = {0: "interp", 1: "hard"}
+KERNEL_SOURCE = os.path.join(ROOT, "approximate_softmax_attention_b200", "csrc", "fwd.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+
+
+def mode_label(m):
+    mode, K, cal, rnd = m
+    if mode == 1:
+        return "kinterval_K%d_%s_%s" % (K, CALIB_NAMES[cal], ROUND_NAMES[rnd])
+    return MODE_NAMES[mode]
+
+
+def fwd_flops(w):
+    f = 4.0 * w.B * w.H * w.S * w.S * w.D
+    return f / 2 if w.causal else f
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(bf16=d["bf16_tflops"], bf16_sustained=d.get("bf16_tflops_sustained",
+                                                                  d["bf16_tflops"]),
+                    hbm=d["hbm_gbs"], source="measured")
+    return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "qsm_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu),
+                                          "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def traffic_for(workload_name, label):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    with open(KERNEL_SOURCE, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    if d.get("kernel_source_sha256_16") != h:
+        return None
+    e = d.get("entries", {}).get("%s/%s" % (workload_name, label))
+    return None if e is None else e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_sample(w, modes, budget_s=12.0, min_heads=1):
+    """Time the CPU oracle on a bounded sample (whole heads of the workload)."""
+    import numpy as np
+    import oracle
+    from approximate_softmax_attention_b200 import inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    d = inputs.draw(1, 1, w.S, w.D, seed=w.seed, peaked=w.peaked, dtype=w.dtype)
+    q, k, v = d["q"], d["k"], d["v"]
+    per_head_flops = fwd_flops(w) / (w.B * w.H)
+    done_flops, t_total, heads = 0.0, 0.0, 0
+    per_budget = budget_s / len(modes)
+    for m in modes:
+        mode, K, cal, rnd = m
+        t_mode, n = 0.0, 0
+        while n < min_heads or t_mode < per_budget * 0.5:
+            t0 = time.perf_counter()
+            oracle.attn_fwd(q, k, v, w.causal, mode, K=K, calib=cal, rounding=rnd,
+                            q_descale=d["q_descale"], k_descale=d["k_descale"],
+                            v_descale=d["v_descale"])
+            dt = time.perf_counter() - t0
+            t_mode += dt
+            n += 1
+            if t_mode + dt > per_budget:
+                break
+        t_total += t_mode
+        heads += n
+        done_flops += n * per_head_flops
+    return {"value": done_flops / t_total / 1e12, "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle",
+            "sample": "%d whole (b,h) heads of %s (S=%d, D=%d), split over the %d maps of the "
+                      "step; %.1f s of host time" % (heads, w.name, w.S, w.D, len(modes),
+                                                      t_total),
+            "seconds": t_total}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from approximate_softmax_attention_b200 import inputs, qsm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+
+    w = inputs.WORKLOADS[args.workload]
+    d = inputs.draw_workload(w)
+    ncopy = 3
+    qs = [d["q"].to(dev) for _ in range(ncopy)]
+    ks = [d["k"].to(dev) for _ in range(ncopy)]
+    vs = [d["v"].to(dev) for _ in range(ncopy)]
+    B, H, S, D = w.shape
+    O = torch.empty(B, H, S, D, dtype=torch.bfloat16, device=dev)
+    LSE = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    opts = qsm.make_opts(dtype=qsm.DTYPE_FP8_E4M3 if w.dtype == "fp8" else qsm.DTYPE_BF16,
+                         q_descale=d["q_descale"], k_descale=d["k_descale"],
+                         v_descale=d["v_descale"])
+    modes = list(w.modes)
+
+    def call(m, i):
+        mode, K, cal, rnd = m
+        st = qsm.qsm_attn_fwd(qs[i], ks[i], vs[i], O, LSE, w.causal, mode, K, cal, rnd, 0, opts,
+                              stream)
+        if st != 0:
+            raise RuntimeError("qsm_attn_fwd: " + qsm.qsm_status_string(st))
+
+    nev = args.steps * len(modes)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(nev)]
+    cnt = 0
+    for _ in range(args.warmup):
+        for m in modes:
+            call(m, cnt % ncopy)
+            cnt += 1
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    e = 0
+    for _ in range(args.steps):
+        for m in modes:
+            ev[e][0].record(stream)
+            call(m, cnt % ncopy)
+            ev[e][1].record(stream)
+            cnt += 1
+            e += 1
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    ck = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+        dist.barrier()
+    per_mode = {}
+    for j, m in enumerate(modes):
+        ms = [ev[s * len(modes) + j][0].elapsed_time(ev[s * len(modes) + j][1])
+              for s in range(args.steps)]
+        avg = sum(ms) / len(ms)
+        tf = fwd_flops(w) / (avg * 1e-3) / 1e12
+        pk = peaks["bf16_sustained"] * (2.0 if w.dtype == "fp8" else 1.0)
+        per_mode[mode_label(m)] = {"ms": round(avg, 4), "tflops": round(tf, 1),
+                                   "frac_of_dtype_peak": round(tf / pk, 4),
+                                   "frac_of_bf16_peak": round(tf / peaks["bf16_sustained"], 4)}
+    step_flops = fwd_flops(w) * len(modes)
+    ms_step = ms_total / args.steps
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    # dominant kernel: the map with the largest time share
+    dom_label = max(per_mode, key=lambda k: per_mode[k]["ms"])
+    dom = per_mode[dom_label]
+    pk = peaks["bf16_sustained"] * (2.0 if w.dtype == "fp8" else 1.0)
+    roof = {"bound": "tensor", "kernel": "qsm_fwd_kernel (%s)" % dom_label,
+            "achieved": dom["tflops"], "peak": round(pk, 1), "unit": "TFLOP/s",
+            "frac": round(dom["tflops"] / pk, 4),
+            "peak_source": "%s bf16 sustained (MEASURED_PEAKS.json)%s" % (
+                peaks["source"], "; x2 nominal e4m3/bf16 ratio" if w.dtype == "fp8" else ""),
+            "algorithmic_flops_per_launch": fwd_flops(w),
+            "traffic": traffic_for(w.name, dom_label)}
+
+    # end to end through host buffers: pinned inputs in, every map's O out
+    e2e = None
+    if not args.no_e2e:
+        hq = d["q"].pin_memory()
+        hk = d["k"].pin_memory()
+        hv = d["v"].pin_memory()
+        hO = [torch.empty(B, H, S, D, dtype=torch.bfloat16).pin_memory() for _ in modes]
+        Os = [torch.empty(B, H, S, D, dtype=torch.bfloat16, device=dev) for _ in modes]
+
+        def e2e_step():
+            qd = hq.to(dev, non_blocking=True)
+            kd = hk.to(dev, non_blocking=True)
+            vd = hv.to(dev, non_blocking=True)
+            for j, m in enumerate(modes):
+                mode, K, cal, rnd = m
+                st = qsm.qsm_attn_fwd(qd, kd, vd, Os[j], LSE, w.causal, mode, K, cal, rnd, 0,
+                                      opts, stream)
+                if st != 0:
+                    raise RuntimeError(qsm.qsm_status_string(st))
+                hO[j].copy_(Os[j], non_blocking=True)
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = a.elapsed_time(b_) / args.steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": round(world * step_flops / (ms_e2e * 1e-3) / 1e12, 2),
+               "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
+               "h2d_bytes_per_step": 3 * B * H * S * D * d["q"].element_size(),
+               "d2h_bytes_per_step": len(modes) * B * H * S * D * 2}
+
+    # secondary problems (per-map TFLOP/s only; not part of value)
+    extras = {}
+    if not args.no_extra and rank == 0:
+        for name in EXTRA_WORKLOADS:
+            ew = inputs.WORKLOADS[name]
+            ed = inputs.draw_workload(ew)
+            eq, ek, evv = ed["q"].to(dev), ed["k"].to(dev), ed["v"].to(dev)
+            eO = torch.empty(ew.shape, dtype=torch.bfloat16, device=dev)
+            eL = torch.empty(ew.shape[:3], dtype=torch.float32, device=dev)
+            eopts = qsm.make_opts(dtype=qsm.DTYPE_FP8_E4M3 if ew.dtype == "fp8" else 0,
+                                  q_descale=ed["q_descale"], k_descale=ed["k_descale"],
+                                  v_descale=ed["v_descale"])
+            res = {}
+            for m in ew.modes:
+                mode, K, cal, rnd = m
+                for _ in range(3):
+                    qsm.qsm_attn_fwd(eq, ek, evv, eO, eL, ew.causal, mode, K, cal, rnd, 0, eopts,
+                                     stream)
+                x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                x0.record(stream)
+                for _ in range(reps):
+                    qsm.qsm_attn_fwd(eq, ek, evv, eO, eL, ew.causal, mode, K, cal, rnd, 0, eopts,
+                                     stream)
+                x1.record(stream)
+                torch.cuda.synchronize()
+                ms = x0.elapsed_time(x1) / reps
+                tf = fwd_flops(ew) / (ms * 1e-3) / 1e12
+                dpk = peaks["bf16_sustained"] * (2.0 if ew.dtype == "fp8" else 1.0)
+                res[mode_label(m)] = {"ms": round(ms, 4), "tflops": round(tf, 1),
+                                      "frac_of_dtype_peak": round(tf / dpk, 4),
+                                      "frac_of_bf16_peak": round(tf / peaks["bf16_sustained"], 4)}
+            extras[name] = {"shape": list(ew.shape), "dtype": ew.dtype, "causal": ew.causal,
+                            "per_mode": res, "l2": "inputs %.0f MB, back-to-back calls" % (
+                                3 * ew.B * ew.H * ew.S * ew.D * (1 if ew.dtype == "fp8" else 2)
+                                / 1e6)}
+            del eq, ek, evv, eO, eL
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(w, modes, budget_s=args.cpu_budget)
+        cpu.pop("seconds", None)
+
+    if rank == 0:
+        line = {
+            "metric": "attn fwd TFLOPS & % of B200 tensor peak per softmax mode, "
+                      "causal/non-causal 2K-16K",
+            "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded randn, peaked keys)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                       "causal": w.causal, "maps": [mode_label(m) for m in modes],
+                       "step": "one forward per map", "parallelism": "dp%d" % world,
+                       "l2": "inputs rotate over 3 device copies (%.0f MB > 126 MB L2)" % (
+                           3 * 3 * B * H * S * D * 2 / 1e6)},
+            "per_mode": per_mode,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps * len(modes),
+            "clocks": ck,
+            "extra": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args):
+    from approximate_softmax_attention_b200 import inputs
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[args.workload]
+    modes = list(w.modes)
+    budget = max(3.0, min(30.0, args.ref_budget / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, modes, budget_s=budget / 4)
+    vals, secs, last = [], 0.0, None
+    for _ in range(args.steps):
+        r = oracle_sample(w, modes, budget_s=budget)
+        vals.append(r["value"])
+        secs += r["seconds"]
+        last = r
+    value = sum(vals) / len(vals)
+    step_flops = fwd_flops(w) * len(modes)
+    line = {
+        "impl": "reference",
+        "metric": "attn fwd TFLOPS & % of B200 tensor peak per softmax mode, "
+                  "causal/non-causal 2K-16K",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_flops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded randn, peaked keys)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D,
+                   "causal": w.causal, "maps": [mode_label(m) for m in modes],
+                   "step": "one forward per map (bounded sample of whole heads per step)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=MAIN_WORKLOAD)
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

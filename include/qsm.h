@@ -100,7 +100,8 @@ typedef struct {
   /* Row statistics [B,H,S], optional in the forward (written when non-NULL)
    * and required by the K-interval backward: hi = row max of s, lo = row min
    * of s (min-max) or hi - window, argmax/argmin = lowest key index of the
-   * row max / min.  Device pointers. */
+   * row max / min.  Device pointers.  The exact map runs no statistics
+   * sweep: it writes row_hi only and leaves the other three untouched. */
   float *row_hi, *row_lo;
   int32_t *row_argmax, *row_argmin;
   /* Backward scratch, at least qsm_attn_bwd_workspace_size() bytes, device,
@@ -110,7 +111,10 @@ typedef struct {
   int32_t *status_dev;    /* optional device word; a timeout writes QSM_ERR_TIMEOUT */
   int8_t *debug_idx;      /* optional [B,H,S,S] dump of the per-element decision:
                              grid node (hard), lower node (interp), PoT
-                             exponent, 0 (exact); -1 masked, -2 flushed */
+                             exponent, 0 (exact); -1 masked, -2 flushed.
+                             Key tiles wholly above the causal diagonal are
+                             never visited and their entries are left as they
+                             were. */
   int debug_flags;        /* test hooks, 0 in normal use; bit 0: the forward's
                              load warp issues no loads, so every consumer wait
                              runs out (exercises the timeout path) */
