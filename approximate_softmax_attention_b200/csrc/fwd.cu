@@ -44,8 +44,9 @@ struct FwdParams {
   float c;          // score scale
   float cL2E;       // c * log2(e), exact map
   float window;
-  float out_scale;  // v_descale / pscale
+  float v_descale;
   float pscale;     // P is stored as w * pscale (FP8 approximate maps: 64)
+  int tab_stride;   // floats of grid table per query tile
   int num_stages;
   uint32_t table_off, bar_off;
   __nv_bfloat16 *O;
@@ -74,6 +75,9 @@ struct Geo {
 };
 
 constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;   // 65536 / 384 rounded down to a multiple of 8
+constexpr int kCtrlRegs = 80;
+constexpr int kMapRegs = 200;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -104,6 +108,431 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   b.tmem_slot = reinterpret_cast<uint32_t *>(b.drain + 1);
   b.abort = reinterpret_cast<int *>(b.tmem_slot + 1);
   return b;
+}
+
+// Per-row constants of the fused map, with the score scale folded in: the
+// map consumes the raw fp32 accumulator r = q.k of the MMA.
+//   PoT:        x = fma(r, -c*log2e, hi*log2e), w = 2^-rne(min(x, cap)) * pscale
+//   K-interval: u = fma(r, c*K/(hi-lo), -lo*K/(hi-lo)), table look-up as in
+//               wmap.cuh (grid values pre-multiplied by pscale)
+struct MapRow {
+  float a, b;        // coordinate = fma(r, a, b)
+  float cap, Kf, Km1;
+  uint32_t tab;      // shared address bias of this row's table column
+  uint32_t pow_bias; // bits of pscale (PoT)
+};
+
+template <int MAP>
+__device__ __forceinline__ float map_raw(float r, const MapRow &m) {
+  if (MAP == MAP_POT) {
+    const float x = __fmaf_rn(r, m.a, m.b);
+    const float t = __fadd_rn(fminf(x, m.cap), kMagic);
+    // 2^-n * pscale from the exponent field: bits(t) = kMagicBits + n and
+    // kMagicBits << 23 == 0 (mod 2^32), so -(bits(t) << 23) == -(n << 23)
+    return __uint_as_float(__float_as_uint(t) * 0xFF800000u + m.pow_bias);
+  } else if (MAP == MAP_KI_HARD) {
+    const float u = __fmaf_rn(r, m.a, m.b);
+    const float uc = fminf(fmaxf(u, 0.0f), m.Kf);
+    const uint32_t tb = __float_as_uint(__fadd_rn(uc, kMagic));
+    return lds_f32(tb * 512u + m.tab);
+  } else {
+    const float u = __fmaf_rn(r, m.a, m.b);
+    const float uc = fminf(fmaxf(u, 0.0f), m.Kf);
+    // floor(uc) for 0 <= uc < 2^23: add 2^23 rounding toward -inf
+    const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), m.Km1);
+    const float f = __fsub_rn(uc, kf);
+    const uint32_t tb = __float_as_uint(__fadd_rn(kf, kMagic));
+    const float2 gd = lds_f32x2(tb * 1024u + m.tab);
+    return __fmaf_rn(f, gd.y, gd.x);
+  }
+}
+
+// Decision index of one element (debug dump only; same arithmetic).
+template <int MAP>
+__device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flush, int N) {
+  if (MAP == MAP_EXACT) return 0;
+  const float x = __fmaf_rn(r, m.a, m.b);
+  if (MAP == MAP_POT) {
+    const int n = static_cast<int>(__float_as_uint(__fadd_rn(fminf(x, m.cap), kMagic)) -
+                                   kMagicBits);
+    return (flush && n > N) ? -2 : n;
+  }
+  const float uc = fminf(fmaxf(x, 0.0f), m.Kf);
+  if (MAP == MAP_KI_HARD)
+    return static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+  const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), m.Km1);
+  return static_cast<int>(kf);
+}
+
+// Weights of one 32-column chunk, packed for the PV MMA and stored to TMEM;
+// FULL: every column valid.
+template <int MAP, bool FULL, bool FP8>
+__device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow &m, int c0,
+                                          int lim, bool flush_below, float (&z)[8],
+                                          uint32_t taddr_p, int cc) {
+  auto wt = [&](int i) {
+    const float r = __uint_as_float(v[i]);
+    float wi = map_raw<MAP>(r, m);
+    if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
+      // fixed-window flush: coordinate below the window
+      if (flush_below && __fmaf_rn(r, m.a, m.b) < 0.0f) wi = 0.0f;
+    }
+    if (!FULL) wi = (c0 + i < lim) ? wi : 0.0f;
+    z[i & 7] += wi;
+    return wi;
+  };
+  if (FP8) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float a = wt(4 * i), b = wt(4 * i + 1), c = wt(4 * i + 2), d = wt(4 * i + 3);
+      pk[i] = pack_e4m3x4(a, b, c, d);
+    }
+    tmem_st8(taddr_p + cc * 8, pk);
+  } else {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float a = wt(2 * i), b = wt(2 * i + 1);
+      pk[i] = pack_bf16x2(a, b);
+    }
+    tmem_st16(taddr_p + cc * 16, pk);
+  }
+}
+
+// Decision dump of one chunk (debug option).
+template <int MAP>
+__device__ __forceinline__ void debug_chunk(int8_t *dbg_row, const uint32_t (&v)[32],
+                                            const MapRow &m, int kv0, int c0, int lim,
+                                            const FwdParams &p, bool flush_below) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (dbg_row != nullptr && kv0 + i < p.S) {
+      const float r = __uint_as_float(v[i]);
+      int n = map_raw_index<MAP>(r, m, p.flush != 0, p.pot_floor);
+      if (flush_below && __fmaf_rn(r, m.a, m.b) < 0.0f) n = -2;
+      dbg_row[kv0 + i] = static_cast<int8_t>((c0 + i < lim) ? n : -1);
+    }
+  }
+}
+
+// Every tcgen05.ld / tcgen05.st below is .sync.aligned: the 32 lanes of a
+// warp must reach it together.  Branches around them therefore depend only on
+// warp-uniform values (tile-level flags, votes), never on a row's own data.
+// Key tile j is valid in every column for every row of query tile qi (a
+// tile-level fact, so the same for all 128 threads of the group).
+__device__ __forceinline__ bool full_tile(const FwdParams &p, int qi, int j) {
+  return 128 * (j + 1) <= p.S && (!p.causal || j < qi);
+}
+
+__device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
+__device__ __forceinline__ bool warp_any(bool x) { return __any_sync(0xffffffffu, x); }
+
+// One map warp group: 128 threads, thread `row` owns query row qi*128+row of
+// the CTA's tile t and TMEM lane `row`.
+template <int D, bool FP8, int MAP>
+__device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, int t, int row,
+                                          uint32_t lane_base, int qi, int n_t, int bh,
+                                          float *tab, volatile int *abort) {
+  constexpr bool kTwoPass = MAP != MAP_EXACT;
+  const int qrow = qi * 128 + row;
+  const bool row_ok = qrow < p.S;
+  const int L = p.causal ? min(qrow + 1, p.S) : p.S;   // valid keys of the row
+  if (n_t <= 0) return;
+  uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
+  bool ok = true;
+  float rmax = -INFINITY, rmin = INFINITY;
+  int amax = 0, amin = 0;
+  const bool want_arg = p.amax != nullptr || p.amin != nullptr;
+  const bool want_min =
+      ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window) || p.lo != nullptr;
+
+  // -------------------------------------------------- statistics sweep
+  if (kTwoPass) {
+    float mx[8], mn[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { mx[i] = -INFINITY; mn[i] = INFINITY; }
+    for (int j = 0; j < n_t && ok; ++j) {
+      const int b = j & 1;
+      ok = warp_all(mbar_wait(&bars.s_full[t * 2 + b], (b ? sf_cnt1 : sf_cnt0) & 1, abort));
+      if (b) ++sf_cnt1; else ++sf_cnt0;
+      if (!ok) break;
+      tc_fence_after();
+      const int lim = L - 128 * j;
+      const bool full = full_tile(p, qi, j);
+      const uint32_t base = lane_base + t * 128 + b * 256;
+      if (want_arg) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld32_sync(base + 32 * cc, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(v[i]);
+            const bool valid = 32 * cc + i < lim;
+            if (valid && x > rmax) { rmax = x; amax = 128 * j + 32 * cc + i; }
+            if (valid && x < rmin) { rmin = x; amin = 128 * j + 32 * cc + i; }
+          }
+        }
+      } else {
+        uint32_t va[32], vb[32];
+        auto step = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
+          if (cc < 3) tmem_ld32(base + 32 * (cc + 1), nxt);
+          if (full) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(cur[i]);
+              mx[i & 7] = fmaxf(mx[i & 7], x);
+              if (want_min) mn[i & 7] = fminf(mn[i & 7], x);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = __uint_as_float(cur[i]);
+              const bool valid = 32 * cc + i < lim;
+              mx[i & 7] = fmaxf(mx[i & 7], valid ? x : -INFINITY);
+              if (want_min) mn[i & 7] = fminf(mn[i & 7], valid ? x : INFINITY);
+            }
+          }
+          if (cc < 3) {
+            tmem_wait_ld();
+            reg_fence32(nxt);
+          }
+        };
+        tmem_ld32(base, va);
+        tmem_wait_ld();
+        reg_fence32(va);
+        step(va, vb, 0);
+        step(vb, va, 1);
+        step(va, vb, 2);
+        step(vb, va, 3);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.s_empty[t * 2 + b]);
+    }
+    if (!want_arg) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        rmax = fmaxf(rmax, mx[i]);
+        rmin = fminf(rmin, mn[i]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------ main sweep
+  float z[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) z[i] = 0.0f;
+  float hi = 0.0f, lo = 0.0f;
+  float m_used = -INFINITY, m_run = -INFINITY;      // exact map, raw units
+  MapRow mr;
+  mr.a = mr.b = 0.0f;
+  mr.cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
+  mr.Kf = static_cast<float>(p.K);
+  mr.Km1 = static_cast<float>(p.K - 1);
+  mr.tab = 0;
+  mr.pow_bias = __float_as_uint(p.pscale);
+  const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush &&
+                           p.fixed_window;
+  if (kTwoPass && ok) {
+    hi = __fmul_rn(p.c, rmax);
+    lo = __fmul_rn(p.c, rmin);
+    RowMap rm = make_rowmap(hi, lo, p.K, p.fixed_window != 0, p.window);
+    if (MAP == MAP_POT) {
+      mr.a = -p.cL2E;
+      mr.b = rm.hiL2E;
+    } else {
+      mr.a = __fmul_rn(p.c, rm.inv);
+      mr.b = rm.b;
+      if (rm.degenerate) {           // every key sits at the top node
+        mr.a = 0.0f;
+        mr.b = mr.Kf;
+      }
+      lo = rm.lo;
+      const uint32_t tb = smem_u32(tab);
+      if (MAP == MAP_KI_HARD) {
+        for (int n = 0; n <= p.K; ++n) tab[n * 128 + row] = grid_value(rm, p.K, n) * p.pscale;
+        mr.tab = tb + row * 4 - kMagicBits * 512u;
+      } else {
+        float gk = grid_value(rm, p.K, 0);
+        for (int n = 0; n < p.K; ++n) {
+          const float gk1 = grid_value(rm, p.K, n + 1);
+          tab[(n * 128 + row) * 2 + 0] = gk * p.pscale;
+          tab[(n * 128 + row) * 2 + 1] = __fsub_rn(gk1, gk) * p.pscale;
+          gk = gk1;
+        }
+        mr.tab = tb + row * 8 - kMagicBits * 1024u;
+      }
+    }
+  }
+  int8_t *dbg_row = (p.dbg != nullptr && row_ok)
+                        ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
+                        : nullptr;
+  const uint32_t pbase = lane_base + t * 128;
+
+  for (int j = 0; j < n_t && ok; ++j) {
+    ok = warp_all(mbar_wait(&bars.s_full[t * 2 + 0], sf_cnt0 & 1, abort));
+    ++sf_cnt0;
+    if (!ok) break;
+    tc_fence_after();
+    const int lim = L - 128 * j;
+    const bool full = full_tile(p, qi, j);
+    const uint32_t sbase = lane_base + t * 128;
+    if (MAP == MAP_EXACT) {
+      // tile maximum, then (lazily) move the anchor and rescale O
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+      uint32_t va[32], vb[32];
+      auto mstep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
+        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x = __uint_as_float(cur[i]);
+          mx[i & 7] = fmaxf(mx[i & 7], (full || 32 * cc + i < lim) ? x : -INFINITY);
+        }
+        if (cc < 3) {
+          tmem_wait_ld();
+          reg_fence32(nxt);
+        }
+      };
+      tmem_ld32(sbase, va);
+      tmem_wait_ld();
+      reg_fence32(va);
+      mstep(va, vb, 0);
+      mstep(vb, va, 1);
+      mstep(va, vb, 2);
+      mstep(vb, va, 3);
+      float mt = mx[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) mt = fmaxf(mt, mx[i]);
+      m_run = fmaxf(m_run, mt);
+      // move this row's anchor on its first tile, or when the running max grew
+      // by more than 2^8 in weight; O is rescaled in TMEM when any row of the
+      // warp moved (rows that did not move use alpha = 1)
+      const bool first = m_used == -INFINITY;
+      const bool move = first || (m_run - m_used) * p.cL2E > kRescaleLog2;
+      const float alpha = (move && !first) ? ex2_approx((m_used - m_run) * p.cL2E) : 1.0f;
+      if (move) m_used = m_run;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) z[i] *= alpha;
+      if (j > 0 && warp_any(move)) {
+        const uint32_t obase = lane_base + 256 + t * 128;
+#pragma unroll 1
+        for (int dc = 0; dc < D / 32; ++dc) {
+          uint32_t v[32];
+          tmem_ld32_sync(obase + 32 * dc, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(obase + 32 * dc, v);
+        }
+      }
+      const float mb = m_used * p.cL2E;
+      auto estep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
+        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
+        auto ex = [&](int i) {
+          const float e = ex2_approx(__fmaf_rn(__uint_as_float(cur[i]), p.cL2E, -mb));
+          const float wi = (full || 32 * cc + i < lim) ? e : 0.0f;
+          z[i & 7] += wi;
+          return wi;
+        };
+        if (FP8) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float a = ex(4 * i), b = ex(4 * i + 1), c = ex(4 * i + 2), d = ex(4 * i + 3);
+            pk[i] = pack_e4m3x4(a, b, c, d);
+          }
+          tmem_st8(pbase + cc * 8, pk);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = ex(2 * i), b = ex(2 * i + 1);
+            pk[i] = pack_bf16x2(a, b);
+          }
+          tmem_st16(pbase + cc * 16, pk);
+        }
+        if (cc < 3) {
+          tmem_wait_ld();
+          reg_fence32(nxt);
+        }
+      };
+      tmem_ld32(sbase, va);
+      tmem_wait_ld();
+      reg_fence32(va);
+      estep(va, vb, 0);
+      estep(vb, va, 1);
+      estep(va, vb, 2);
+      estep(vb, va, 3);
+    } else {
+      uint32_t va[32], vb[32];
+      auto wstep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
+        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
+        if (full)
+          map_chunk<MAP, true, FP8>(cur, mr, 32 * cc, lim, flush_below, z, pbase, cc);
+        else
+          map_chunk<MAP, false, FP8>(cur, mr, 32 * cc, lim, flush_below, z, pbase, cc);
+        if (p.dbg != nullptr)
+          debug_chunk<MAP>(dbg_row, cur, mr, 128 * j + 32 * cc, 32 * cc, lim, p, flush_below);
+        if (cc < 3) {
+          tmem_wait_ld();
+          reg_fence32(nxt);
+        }
+      };
+      tmem_ld32(sbase, va);
+      tmem_wait_ld();
+      reg_fence32(va);
+      wstep(va, vb, 0);
+      wstep(vb, va, 1);
+      wstep(va, vb, 2);
+      wstep(vb, va, 3);
+    }
+    if (MAP == MAP_EXACT && dbg_row != nullptr) {
+      const int kv0 = 128 * j;
+      for (int i = 0; i < 128 && kv0 + i < p.S; ++i) dbg_row[kv0 + i] = (i < lim) ? 0 : -1;
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&bars.p_full[t]);
+  }
+
+  // ---------------------------------------------------------- epilogue
+  if (ok) ok = warp_all(mbar_wait(&bars.o_full[t], 0, abort));
+  if (!ok) return;
+  tc_fence_after();
+  float Z = ((z[0] + z[1]) + (z[2] + z[3])) + ((z[4] + z[5]) + (z[6] + z[7]));
+  if (MAP == MAP_EXACT) hi = p.c * m_run;
+  const float oscale = p.v_descale / Z;          // pscale cancels: P and Z both carry it
+  const uint32_t obase = lane_base + 256 + t * 128;
+  __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D;
+#pragma unroll 1
+  for (int dc = 0; dc < D / 32; ++dc) {
+    uint32_t v[32];
+    tmem_ld32_sync(obase + 32 * dc, v);
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * oscale,
+                          __uint_as_float(v[2 * i + 1]) * oscale);
+    if (row_ok) {
+      uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * dc);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+    }
+  }
+  if (row_ok) {
+    const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
+    const float anchor = (MAP == MAP_EXACT) ? p.c * m_used : hi;
+    p.LSE[ri] = anchor + logf(Z / p.pscale);
+    if (p.hi) p.hi[ri] = hi;
+    if (MAP != MAP_EXACT) {          // the exact map runs no statistics sweep
+      if (p.lo) p.lo[ri] = lo;
+      if (p.amax) p.amax[ri] = amax;
+      if (p.amin) p.amin[ri] = amin;
+    }
+  }
 }
 
 template <int D, bool FP8, int MAP>
@@ -161,6 +590,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
+  // The CTA launches with kThreads x kLaunchRegs registers; the control warp
+  // group (producer, MMA issuer, two idle warps) gives most of its share to
+  // the two map groups: 128 x kCtrlRegs + 256 x kMapRegs <= 384 x kLaunchRegs
+  // (an increase beyond what the decrease freed would wait forever).
+  static_assert(128 * kCtrlRegs + 256 * kMapRegs <= kThreads * kLaunchRegs,
+                "register split must equal the launch allocation");
+  if (warp < 4) {
+    regs_dec<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !(p.debug_flags & 1)) {
@@ -306,229 +743,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ map groups
+  }
+  } else {
+    regs_inc<kMapRegs>();
     const int t = (warp - 4) >> 2;
-    const int row = threadIdx.x - 128 - t * 128;         // 0..127 == TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int qrow = qi[t] * 128 + row;
-    const bool row_ok = qrow < p.S;
-    const int L = p.causal ? min(qrow + 1, p.S) : p.S;   // valid keys of the row
-    const int n_t = nt[t];
-    if (n_t > 0) {
-      uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
-      bool ok = true;
-      float rmax = -INFINITY, rmin = INFINITY;
-      int amax = 0, amin = 0;
-      const bool want_arg = p.amax != nullptr || p.amin != nullptr;
-      const bool want_min =
-          ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window) || p.lo != nullptr;
-
-      // ------------------------------------------------ statistics sweep
-      if (kTwoPass) {
-        for (int j = 0; j < n_t && ok; ++j) {
-          const int b = j & 1;
-          ok = mbar_wait(&bars.s_full[t * 2 + b], (b ? sf_cnt1 : sf_cnt0) & 1, abort);
-          if (b) ++sf_cnt1; else ++sf_cnt0;
-          if (!ok) break;
-          tc_fence_after();
-          const int lim = L - 128 * j;
-          const uint32_t base = lane_base + t * 128 + b * 256;
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(base + 32 * cc, v);
-            tmem_wait_ld();
-            const int c0 = 32 * cc;
-            if (want_arg) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(v[i]);
-                const bool valid = c0 + i < lim;
-                if (valid && x > rmax) { rmax = x; amax = 128 * j + c0 + i; }
-                if (valid && x < rmin) { rmin = x; amin = 128 * j + c0 + i; }
-              }
-            } else if (lim >= c0 + 32) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(v[i]);
-                rmax = fmaxf(rmax, x);
-                if (want_min) rmin = fminf(rmin, x);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(v[i]);
-                if (c0 + i < lim) {
-                  rmax = fmaxf(rmax, x);
-                  if (want_min) rmin = fminf(rmin, x);
-                }
-              }
-            }
-          }
-          tc_fence_before();
-          mbar_arrive(&bars.s_empty[t * 2 + b]);
-        }
-      }
-
-      // ------------------------------------------------------ main sweep
-      float Z = 0.0f;
-      float hi = 0.0f, lo = 0.0f;
-      float m_used = -INFINITY, m_run = -INFINITY;        // exact map, raw units
-      RowMap rm;
-      float *tab = sTab + t * (p.K + 1) * 128;
-      const float Kf = static_cast<float>(p.K);
-      const float cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
-      if (kTwoPass && ok) {
-        hi = __fmul_rn(p.c, rmax);
-        lo = __fmul_rn(p.c, rmin);
-        rm = make_rowmap(hi, lo, p.K, p.fixed_window != 0, p.window);
-        if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP)
-          for (int n = 0; n <= p.K; ++n) tab[n * 128 + row] = grid_value(rm, p.K, n);
-        lo = (MAP == MAP_POT) ? lo : rm.lo;
-      }
-      int8_t *dbg_row = (p.dbg != nullptr && row_ok)
-                            ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
-                            : nullptr;
-      for (int j = 0; j < n_t && ok; ++j) {
-        ok = mbar_wait(&bars.s_full[t * 2 + 0], sf_cnt0 & 1, abort);
-        ++sf_cnt0;
-        if (!ok) break;
-        tc_fence_after();
-        const int lim = L - 128 * j;
-        const uint32_t sbase = lane_base + t * 128;
-        if (MAP == MAP_EXACT) {
-          float mt = -INFINITY;
-#pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(sbase + 32 * cc, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (32 * cc + i < lim) mt = fmaxf(mt, __uint_as_float(v[i]));
-          }
-          m_run = fmaxf(m_run, mt);
-          if (m_used == -INFINITY || (m_run - m_used) * p.cL2E > kRescaleLog2) {
-            if (m_used != -INFINITY) {
-              const float alpha = ex2_approx((m_used - m_run) * p.cL2E);
-              Z *= alpha;
-              const uint32_t obase = lane_base + 256 + t * 128;
-#pragma unroll 1
-              for (int dc = 0; dc < D / 32; ++dc) {
-                uint32_t v[32];
-                tmem_ld32(obase + 32 * dc, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-                tmem_st32(obase + 32 * dc, v);
-              }
-            }
-            m_used = m_run;
-          }
-        }
-        const float mb = m_used * p.cL2E;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(sbase + 32 * cc, v);
-          tmem_wait_ld();
-          float w[32];
-          int dn[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(v[i]);
-            const bool valid = 32 * cc + i < lim;
-            float wi;
-            int n = 0;
-            if (MAP == MAP_EXACT) {
-              wi = ex2_approx(__fmaf_rn(x, p.cL2E, -mb));
-            } else {
-              const float s = __fmul_rn(x, p.c);
-              if (MAP == MAP_POT) {
-                wi = pot_weight(s, rm.hiL2E, cap, p.pot_floor, p.flush != 0, n);
-              } else {
-                const float u = kint_u(s, rm, Kf);
-                if (p.flush && p.fixed_window && u < 0.0f) {
-                  wi = 0.0f;
-                  n = -2;
-                } else if (MAP == MAP_KI_HARD) {
-                  n = kint_hard_node(u, Kf);
-                  wi = tab[n * 128 + row];
-                } else {
-                  float f;
-                  n = kint_interp_node(u, Kf, f);
-                  wi = kint_interp_weight(f, tab[n * 128 + row], tab[(n + 1) * 128 + row]);
-                }
-              }
-            }
-            w[i] = valid ? wi : 0.0f;
-            dn[i] = valid ? n : -1;
-            Z += w[i];
-          }
-          if (FP8) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              pk[i] = pack_e4m3x4(w[4 * i] * p.pscale, w[4 * i + 1] * p.pscale,
-                                  w[4 * i + 2] * p.pscale, w[4 * i + 3] * p.pscale);
-            tmem_st8(sbase + cc * 8, pk);
-          } else {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
-            tmem_st16(sbase + cc * 16, pk);
-          }
-          if (dbg_row != nullptr) {
-            const int kv0 = 128 * j + 32 * cc;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (kv0 + i < p.S) dbg_row[kv0 + i] = static_cast<int8_t>(dn[i]);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars.p_full[t]);
-      }
-
-      // -------------------------------------------------------- epilogue
-      if (ok) ok = mbar_wait(&bars.o_full[t], 0, abort);
-      if (ok) {
-        tc_fence_after();
-        if (MAP == MAP_EXACT) hi = p.c * m_run;
-        const float oscale = p.out_scale / Z;
-        const uint32_t obase = lane_base + 256 + t * 128;
-        __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D;
-#pragma unroll 1
-        for (int dc = 0; dc < D / 32; ++dc) {
-          uint32_t v[32];
-          tmem_ld32(obase + 32 * dc, v);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * oscale,
-                                __uint_as_float(v[2 * i + 1]) * oscale);
-          if (row_ok) {
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * dc);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
-        if (row_ok) {
-          const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
-          const float anchor = (MAP == MAP_EXACT) ? p.c * m_used : hi;
-          p.LSE[ri] = anchor + logf(Z);
-          if (p.hi) p.hi[ri] = hi;
-          if (MAP != MAP_EXACT) {          // the exact map runs no statistics sweep
-            if (p.lo) p.lo[ri] = lo;
-            if (p.amax) p.amax[ri] = amax;
-            if (p.amin) p.amin[ri] = amin;
-          }
-        }
-      }
-    }
+    map_group<D, FP8, MAP>(p, bars, t, threadIdx.x - 128 - t * 128,
+                           tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi[t], nt[t],
+                           bh, sTab + t * p.tab_stride, abort);
   }
 
   __syncwarp();
@@ -558,7 +779,7 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.cL2E = a.c * 1.4426950408889634f;
   p.window = a.window;
   p.pscale = (FP8 && MAP != MAP_EXACT) ? 64.0f : 1.0f;
-  p.out_scale = a.v_descale / p.pscale;
+  p.v_descale = a.v_descale;
   p.O = static_cast<__nv_bfloat16 *>(a.O);
   p.LSE = a.LSE;
   p.hi = a.row_hi;
@@ -569,7 +790,10 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.status = a.status_dev;
   p.debug_flags = a.debug_flags;
 
-  const size_t table_bytes = static_cast<size_t>(2) * (p.K + 1) * 128 * sizeof(float);
+  // grid table per query tile: [K+1][128] values (hard) or [K][128] (value,
+  // difference) pairs (interpolation)
+  p.tab_stride = (MAP == MAP_KI_INTERP) ? p.K * 128 * 2 : (p.K + 1) * 128;
+  const size_t table_bytes = static_cast<size_t>(2) * p.tab_stride * sizeof(float);
   const size_t bar_bytes = 256;
   const size_t max_smem = 232448;                        // 227 KB opt-in per CTA
   const size_t fixed = 1024 + 2 * G::TILE_BYTES + table_bytes + bar_bytes;
