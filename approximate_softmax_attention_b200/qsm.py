@@ -212,3 +212,30 @@ def attention_forward(q, k, v, causal=False, mode=MODE_EXACT, Kint=4,
 
 def default_scale(D):
     return 1.0 / math.sqrt(D)
+
+
+def attention_backward(q, k, v, O, dO, LSE, stats, causal=False, mode=MODE_KINTERVAL, Kint=4,
+                       calibration=CALIB_MINMAX, rounding=ROUND_HARD, surrogate=SURR_NONE, *,
+                       detach_extrema=False, scale=None, window=8.0, below_policy=0,
+                       workspace=None, stream=None):
+    """Allocate dQ, dK, dV (and the workspace, unless given) with torch and run
+    ``qsm_attn_bwd``.  ``stats`` is the dict returned by attention_forward(...,
+    stats=True)."""
+    B, H, S, D = q.shape
+    dev = q.device
+    dQ = torch.empty_like(q)
+    dK = torch.empty_like(k)
+    dV = torch.empty_like(v)
+    need = qsm_attn_bwd_workspace_size(B, H, S, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    kw = dict(scale=0.0 if scale is None else float(scale), window=float(window),
+              below_policy=int(below_policy), detach_extrema=int(bool(detach_extrema)),
+              workspace=workspace, workspace_bytes=int(workspace.numel()))
+    if stats is not None:
+        kw.update(row_hi=stats["hi"], row_lo=stats["lo"], row_argmax=stats["argmax"],
+                  row_argmin=stats["argmin"])
+    opts = make_opts(**kw)
+    _check(qsm_attn_bwd(q, k, v, O, dO, LSE, dQ, dK, dV, causal, mode, Kint, calibration,
+                        rounding, surrogate, opts, stream), "qsm_attn_bwd")
+    return dQ, dK, dV

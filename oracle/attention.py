@@ -105,9 +105,15 @@ def kint_grid(K: int, delta: np.ndarray) -> np.ndarray:
 
 
 def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
-              below_policy):
+              below_policy, frozen=None):
     """Apply one weight map to a block of rows; returns a dict of per-row and
     per-element quantities (everything the backward needs, decisions frozen).
+
+    ``frozen`` (optional, [R, S] ints): K-interval node decisions to use
+    instead of rounding the fp64 coordinate (node for hard rounding, lower
+    node for interpolation; entries < 0 are ignored).  The backward rules are
+    defined with the forward's decisions held fixed; passing the decisions a
+    forward actually took evaluates those rules at that forward.
     """
     hi, lo, amax, amin = row_stats(s, valid)
     R, S = s.shape
@@ -144,11 +150,15 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
     rows = np.arange(R)[:, None]
     if rounding == HARD:
         n = np.rint(u).astype(np.int64)
+        if frozen is not None:
+            n = np.where(valid & (frozen >= 0), frozen, n)
         w = g[rows, n]
         kidx = n
         f = np.zeros_like(u)
     elif rounding == INTERP:
         kidx = np.minimum(np.floor(u), K - 1).astype(np.int64)
+        if frozen is not None:
+            kidx = np.where(valid & (frozen >= 0), frozen, kidx)
         f = u - kidx
         w = (1.0 - f) * g[rows, kidx] + f * g[rows, kidx + 1]
     else:
@@ -241,7 +251,7 @@ def attn_fwd(q, k, v, causal, mode, K=4, calib=MINMAX, rounding=HARD,
 
 def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
                   surrogate=SURR_NONE, detach_extrema=False, window=8.0,
-                  below_policy=0):
+                  below_policy=0, frozen=None):
     """Backward of one block of query rows against all keys.
 
     Returns (dS [R,S], P [R,S], O [R,D]): dS is dL/ds (before the factor c
@@ -249,7 +259,7 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
     exact gradients of the surrogate graphs named in the module docstring.
     """
     m = _map_rows(s, valid, mode, K, calib, rounding, window, 15,
-                  below_policy)
+                  below_policy, frozen)
     w = m["w"]
     Z = w.sum(axis=1)
     P = w / Z[:, None]
@@ -330,10 +340,13 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
 
 def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
              surrogate=SURR_NONE, detach_extrema=False, scale=None,
-             window=8.0, below_policy=0, heads=None, row_block=512):
+             window=8.0, below_policy=0, heads=None, row_block=512,
+             decisions=None):
     """Gradients dQ, dK, dV [B,H,S,D] (float64) of the attention forward.
 
     ``heads`` restricts the work to a list of (b, h); other heads are NaN.
+    ``decisions`` (optional, [B,H,S,S] ints, the forward's per-element node
+    decisions) freezes the K-interval decisions at those values.
     """
     q, k, v, dO = _as64(q), _as64(k), _as64(v), _as64(dO)
     B, H, S, D = q.shape
@@ -351,9 +364,10 @@ def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
         for r0 in range(0, S, row_block):
             rr = np.arange(r0, min(S, r0 + row_block))
             s, valid = row_scores(q[b, h, rr], k[b, h], c, r0, causal)
+            fz = None if decisions is None else np.asarray(decisions[b, h, rr], dtype=np.int64)
             ds, P, _ = attn_bwd_rows(s, valid, v[b, h], dO[b, h, rr], mode,
                                      K, calib, rounding, surrogate,
-                                     detach_extrema, window, below_policy)
+                                     detach_extrema, window, below_policy, fz)
             dQ[b, h, rr] = c * (ds @ k[b, h])
             dK[b, h] += c * (ds.T @ q[b, h, rr])
             dV[b, h] += P.T @ dO[b, h, rr]

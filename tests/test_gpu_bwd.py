@@ -1,0 +1,97 @@
+"""GPU parity of the backward (K-interval and exact maps, bf16, D = 64)
+against the CPU oracle, through the C ABI.
+
+The rules are the oracle's ("Pretraining Transformers with Quantized Softmax
+in Attention", abstract: backward rules including calibration derivatives;
+straight-through surrogate before or after normalization), whose own pins
+are in test_oracle_bwd.py.  Tolerance (bf16 gradients): max abs <= 1e-2 beyond the rounding of the
+exact value to the bf16 output (gradients of the first keys of a causal row
+reach magnitudes above 4, where half a bf16 ulp alone is 0.0078-0.0156),
+mean abs <= 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from approximate_softmax_attention_b200 import inputs, qsm
+
+from _helpers import check_decisions, err_stats_bf16_out
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0):
+    q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
+    B, H, S, D = q.shape
+    dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV)
+    O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rnd, window=window,
+                                       stats=True, debug_idx=dbg)
+    dQ, dK, dV = qsm.attention_backward(q, k, v, O, dO, LSE, st, causal, mode, K, calib, rnd,
+                                        surr, detach_extrema=detach, window=window)
+    torch.cuda.synchronize()
+    return (dQ.float().cpu().numpy(), dK.float().cpu().numpy(), dV.float().cpu().numpy(),
+            dbg.cpu().numpy())
+
+
+def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None, dec=None):
+    """The oracle's backward, with the node decisions the kernel's forward
+    took (they agree with fp64 rounding except within 1e-3 of a boundary,
+    checked by check_decisions; the rules hold the forward's decisions
+    fixed, so the gradients are compared at those decisions)."""
+    if dec is not None and mode == 1:
+        check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads)
+    return oracle.attn_bwd(d["q"], d["k"], d["v"], d["dO"], causal, mode, K=K, calib=calib,
+                           rounding=rnd, surrogate=surr, detach_extrema=detach, window=window,
+                           heads=heads, decisions=dec if mode == 1 else None)
+
+
+def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3):
+    for g, name in zip(got, ("dQ", "dK", "dV")):
+        r = ref[name]
+        if heads is not None:
+            g = np.stack([g[b, h] for (b, h) in heads])
+            r = np.stack([r[b, h] for (b, h) in heads])
+        mx, mean = err_stats_bf16_out(g, r)
+        assert mx <= tol_max and mean <= tol_mean, (name, mx, mean)
+
+
+COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
+          for s in (0, 1, 2) for det in (False, True)]
+
+
+@pytest.mark.parametrize("K,calib,rnd,surr,detach", COMBOS)
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
+def test_bwd_kinterval_small(S, causal, K, calib, rnd, surr, detach):
+    d = inputs.draw(1, 2, S, 64, seed=50 + S, with_dO=True)
+    *got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
+    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, dec=dec)
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False), (77, True), (384, False)])
+def test_bwd_exact(S, causal):
+    d = inputs.draw(1, 2, S, 64, seed=7 + S, with_dO=True)
+    *got, _ = _run(d, causal, 0, 4, 0, 1, 0, False)
+    ref = _oracle(d, causal, 0, 4, 0, 1, 0, False)
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("mode,K,calib,rnd", [(1, 4, 0, 1), (1, 16, 0, 0), (1, 4, 1, 1),
+                                             (1, 16, 1, 0)])
+@pytest.mark.parametrize("surr,detach", [(0, False), (1, False), (2, False), (1, True),
+                                         (2, True)])
+def test_bwd_training_shape_sampled(mode, K, calib, rnd, surr, detach):
+    """B=8, H=12, S=1024, D=64 bf16 causal (124M-GPT attention shape), the
+    launch the bench times; the oracle checks three whole heads."""
+    w = inputs.WORKLOADS["train_s1k"]
+    d = inputs.draw_workload(w)
+    heads = [(0, 0), (3, 7), (7, 11)]
+    *got, dec = _run(d, True, mode, K, calib, rnd, surr, detach)
+    ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads, dec=dec)
+    _check(got, ref, heads=heads)
+    for g in got:
+        assert np.isfinite(g).all()

@@ -169,3 +169,46 @@ def test_post_detached_is_softmax_backward_for_q_and_k(causal, calib, rounding):
                             rounding=rounding, window=3.0)["O"]
     np.testing.assert_allclose(res["dV"], np.swapaxes(ident, -1, -2) @ dO, rtol=1e-10,
                                atol=1e-12)
+
+
+@pytest.mark.parametrize("K,calib,rounding,surrogate", [(4, 0, 0, 0), (16, 0, 0, 1), (4, 0, 1, 2),
+                                                       (16, 1, 0, 0), (4, 1, 1, 1)])
+def test_frozen_decisions_input(K, calib, rounding, surrogate):
+    """The optional decisions input: its own decisions reproduce the default
+    result exactly, and a decision moved to the neighbouring node gives the
+    exact gradient of the surrogate graph frozen at the moved decision
+    (central finite differences of the graph re-stated above)."""
+    rng = np.random.default_rng(77 + K + calib + rounding + surrogate)
+    S, D, W = 9, 4, 2.5
+    q, k, v, dO = (rng.normal(size=(S, D)) for _ in range(4))
+    c = 1 / math.sqrt(D)
+    fr = _frozen(c * (q @ k.T), K, calib, rounding, W)
+    args = (q[None, None], k[None, None], v[None, None], dO[None, None], False, A.KINTERVAL)
+    kw = dict(K=K, calib=calib, rounding=rounding, surrogate=surrogate, window=W)
+    base = oracle.attn_bwd(*args, **kw)
+    same = oracle.attn_bwd(*args, decisions=fr["node"][None, None], **kw)
+    for n in ("dQ", "dK", "dV"):
+        assert np.array_equal(base[n], same[n])
+    # move one interior decision by one node (as a boundary-near element may)
+    node = fr["node"].copy()
+    i, j = 3, 5
+    if j in (fr["amax"][i], fr["amin"][i]):
+        j = 6
+    node[i, j] = node[i, j] + 1 if node[i, j] < K - (1 if rounding == 0 else 0) else node[i, j] - 1
+    moved = oracle.attn_bwd(*args, decisions=node[None, None], **kw)
+    fr2 = dict(fr)
+    fr2["node"] = node
+    h = 1e-6
+    for name, X, G in (("q", q, moved["dQ"]), ("k", k, moved["dK"]), ("v", v, moved["dV"])):
+        for (a, d) in [(3, 1), (5, 2), (0, 0)]:
+            Xp = X.copy(); Xp[a, d] += h
+            Xm = X.copy(); Xm[a, d] -= h
+            ar = {"q": q, "k": k, "v": v}
+            ar[name] = Xp
+            lp = _surrogate_loss(ar["q"], ar["k"], ar["v"], dO, fr2, K, calib, rounding,
+                                 surrogate, False, W, c)
+            ar[name] = Xm
+            lm = _surrogate_loss(ar["q"], ar["k"], ar["v"], dO, fr2, K, calib, rounding,
+                                 surrogate, False, W, c)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - G[0, 0, a, d]) <= 1e-6 * max(1.0, abs(fd)), (name, a, d)
