@@ -177,6 +177,25 @@ def oracle_sample(w, modes, budget_s=12.0, min_heads=1):
             "seconds": t_total}
 
 
+# ------------------------------------------------------- multi-rank logic
+
+def max_over_ranks(x, world, device="cpu"):
+    """The slowest rank's value (every rank calls this, in the same order)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_rank_step, ms_per_step_max, world):
+    """Whole-job TFLOP/s: every rank runs its own problem of the same size
+    (independent batches), the job takes as long as the slowest rank."""
+    return world * flops_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- GPU arm
 
 def run_ours(args):
@@ -244,11 +263,8 @@ def run_ours(args):
     t_end.record(stream)
     torch.cuda.synchronize()
     ck = clocks.stop()
-    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
         dist.barrier()
     per_mode = {}
     for j, m in enumerate(modes):
@@ -262,7 +278,7 @@ def run_ours(args):
                                    "frac_of_bf16_peak": round(tf / peaks["bf16_sustained"], 4)}
     step_flops = fwd_flops(w) * len(modes)
     ms_step = ms_total / args.steps
-    value = world * step_flops / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(step_flops, ms_step, world)
 
     # dominant kernel: the map with the largest time share
     dom_label = max(per_mode, key=lambda k: per_mode[k]["ms"])
@@ -305,12 +321,8 @@ def run_ours(args):
             e2e_step()
         b_.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = a.elapsed_time(b_) / args.steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": round(world * step_flops / (ms_e2e * 1e-3) / 1e12, 2),
+        ms_e2e = max_over_ranks(a.elapsed_time(b_) / args.steps, world, dev)
+        e2e = {"value": round(weak_scaling_value(step_flops, ms_e2e, world), 2),
                "unit": "TFLOP/s", "ms_per_step": round(ms_e2e, 3),
                "h2d_bytes_per_step": 3 * B * H * S * D * d["q"].element_size(),
                "d2h_bytes_per_step": len(modes) * B * H * S * D * 2}
