@@ -27,7 +27,8 @@ SURR_NONE, SURR_PRE, SURR_POST = 0, 1, 2
 DTYPE_BF16, DTYPE_FP8_E4M3 = 0, 1
 
 EXPORTED = ("qsm_opts_default", "qsm_attn_fwd", "qsm_attn_bwd", "qsm_attn_bwd_workspace_size",
-            "qsm_weight_map", "qsm_status_string", "qsm_version")
+            "qsm_attn_bwd_noalloc", "qsm_weight_map", "qsm_status_string", "qsm_version")
+NOALLOC_SCRATCH_BYTES = 16 << 20     # QSM_NOALLOC_SCRATCH_BYTES
 
 
 class QsmOpts(ctypes.Structure):
@@ -81,6 +82,8 @@ def lib():
     L.qsm_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
                                ci, ci, ci, ctypes.POINTER(QsmOpts), vp]
     L.qsm_attn_bwd.restype = ci
+    L.qsm_attn_bwd_noalloc.argtypes = list(L.qsm_attn_bwd.argtypes)
+    L.qsm_attn_bwd_noalloc.restype = ci
     L.qsm_attn_bwd_workspace_size.argtypes = [ci, ci, ci, ci]
     L.qsm_attn_bwd_workspace_size.restype = ctypes.c_size_t
     L.qsm_weight_map.argtypes = [vp, vp, ci, ci, ci, ci, ci, ci, ctypes.POINTER(QsmOpts), vp, vp,
@@ -155,6 +158,20 @@ def qsm_attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, mode, Kint=4,
                               _ptr(dK), _ptr(dV), B, H, S, D, int(causal), int(mode), int(Kint),
                               int(calibration), int(rounding), int(surrogate),
                               ctypes.byref(opts) if opts is not None else None, _stream(stream))
+
+
+def qsm_attn_bwd_noalloc(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, mode, Kint=4,
+                         calibration=CALIB_MINMAX, rounding=ROUND_HARD, surrogate=SURR_NONE,
+                         opts=None, stream=None) -> int:
+    """qsm_attn_bwd with the library's static scratch instead of a workspace
+    (for callers that cannot allocate device memory at call time)."""
+    B, H, S, D = Q.shape
+    return lib().qsm_attn_bwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                      _ptr(dQ), _ptr(dK), _ptr(dV), B, H, S, D, int(causal),
+                                      int(mode), int(Kint), int(calibration), int(rounding),
+                                      int(surrogate),
+                                      ctypes.byref(opts) if opts is not None else None,
+                                      _stream(stream))
 
 
 def qsm_attn_bwd_workspace_size(B, H, S, D) -> int:

@@ -151,6 +151,36 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
 /* Bytes of opts->workspace that qsm_attn_bwd needs for this shape. */
 size_t qsm_attn_bwd_workspace_size(int B, int H, int S, int D);
 
+/* Size of the library's own backward scratch array (16 MiB). */
+#define QSM_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* qsm_attn_bwd without a caller-provided workspace.  (The papers have no
+ * counterpart: this is a convenience of the library.)
+ *
+ * For callers that cannot allocate device memory at the time of the call,
+ * such as a plugin whose host framework owns every device allocation through
+ * its own pool, or a latency-critical loop that cannot take cudaMalloc's
+ * implicit synchronisation.  The backward's scratch comes instead from one
+ * static device array of QSM_NOALLOC_SCRATCH_BYTES bytes inside the library,
+ * which every GPU that loads the library holds until the process exits.  This
+ * call allocates and frees nothing.
+ *
+ * Arguments and results are those of qsm_attn_bwd; opts->workspace and
+ * opts->workspace_bytes are ignored.  Returns QSM_ERR_INVALID_ARG when
+ * qsm_attn_bwd_workspace_size(B, H, S, D) exceeds QSM_NOALLOC_SCRATCH_BYTES
+ * (for D = 64, about 30 000 query rows B*H*S), before any launch.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call uses the same array, so calls whose work overlaps on a GPU
+ * (different streams or host threads) race; serialise them. */
+qsm_status qsm_attn_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O,
+                                const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
+                                int B, int H, int S, int D, int causal, qsm_mode mode, int Kint,
+                                qsm_calib calibration, qsm_rounding rounding,
+                                qsm_surrogate surrogate, const qsm_opts *opts,
+                                qsm_stream_t stream);
+
 /* The weight map alone on given fp32 scores (bit-exact with the library's
  * fp32 specification of the maps).
  *  scores:    device [rows, cols] fp32.
