@@ -35,7 +35,7 @@ namespace qsm {
 enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
 
 struct FwdParams {
-  int S, nqt, nqb;
+  int S, nqt, nqb, BH;
   int causal;
   int K;
   int fixed_window;
@@ -275,9 +275,18 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
           }
         }
       } else {
-        uint32_t va[32], vb[32];
-        auto step = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
-          if (cc < 3) tmem_ld32(base + 32 * (cc + 1), nxt);
+        // all four 32-column loads in flight, one wait
+        uint32_t v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(base, v0);
+        tmem_ld32(base + 32, v1);
+        tmem_ld32(base + 64, v2);
+        tmem_ld32(base + 96, v3);
+        tmem_wait_ld();
+        reg_fence32(v0);
+        reg_fence32(v1);
+        reg_fence32(v2);
+        reg_fence32(v3);
+        auto reduce = [&](const uint32_t(&cur)[32], int cc) {
           if (full) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -294,18 +303,11 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
               if (want_min) mn[i & 7] = fminf(mn[i & 7], valid ? x : INFINITY);
             }
           }
-          if (cc < 3) {
-            tmem_wait_ld();
-            reg_fence32(nxt);
-          }
         };
-        tmem_ld32(base, va);
-        tmem_wait_ld();
-        reg_fence32(va);
-        step(va, vb, 0);
-        step(vb, va, 1);
-        step(va, vb, 2);
-        step(vb, va, 3);
+        reduce(v0, 0);
+        reduce(v1, 1);
+        reduce(v2, 2);
+        reduce(v3, 3);
       }
       tc_fence_before();
       mbar_arrive(&bars.s_empty[t * 2 + b]);
@@ -483,10 +485,11 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
       tmem_ld32(sbase, va);
       tmem_wait_ld();
       reg_fence32(va);
-      wstep(va, vb, 0);
-      wstep(vb, va, 1);
-      wstep(va, vb, 2);
-      wstep(vb, va, 3);
+#pragma unroll 1
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        wstep(va, vb, c2);
+        wstep(vb, va, c2 + 1);
+      }
     }
     if (MAP == MAP_EXACT && dbg_row != nullptr) {
       const int kv0 = 128 * j;
@@ -545,8 +548,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int qb = p.causal ? (p.nqb - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+  // Work order: non-causal CTAs sweep one head's query blocks after another
+  // (the running CTAs share few heads' K/V in L2); causal CTAs go heaviest
+  // first over all heads (longest-processing-time order, so the lightest
+  // blocks form the tail).
+  int bh, qb;
+  if (p.causal) {
+    const int rank = static_cast<int>(blockIdx.x) / p.BH;
+    bh = static_cast<int>(blockIdx.x) - rank * p.BH;
+    qb = p.nqb - 1 - rank;
+  } else {
+    qb = static_cast<int>(blockIdx.x) % p.nqb;
+    bh = static_cast<int>(blockIdx.x) / p.nqb;
+  }
   const int ns = p.num_stages;
 
   uint8_t *sQ = smem;                                   // 2 tiles
@@ -770,6 +784,7 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.S = a.S;
   p.nqt = (a.S + 127) / 128;
   p.nqb = (p.nqt + 1) / 2;
+  p.BH = a.B * a.H;
   p.causal = a.causal;
   p.K = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) ? a.Kint : 1;
   p.fixed_window = a.calib == QSM_CALIB_FIXED_WINDOW;
@@ -811,7 +826,7 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return QSM_ERR_CUDA;
-  dim3 grid(p.nqb, a.B * a.H);
+  dim3 grid(p.nqb * a.B * a.H);
   kern<<<grid, kThreads, smem, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }

@@ -365,6 +365,38 @@ def run_ours(args):
                                 / 1e6)}
             del eq, ek, evv, eO, eL
 
+    # training shape: forward with statistics, then the backward (2.5 x the
+    # forward's algorithmic FLOPs), secondary figure
+    if not args.no_extra and rank == 0:
+        tw = inputs.WORKLOADS["train_s1k"]
+        td = inputs.draw_workload(tw)
+        tq, tk, tv, tdo = (td[n].to(dev) for n in ("q", "k", "v", "dO"))
+        res = {}
+        for (mode, K, cal, rnd) in tw.modes:
+            for surr in (qsm.SURR_PRE, qsm.SURR_POST):
+                O_, L_, st_ = qsm.attention_forward(tq, tk, tv, True, mode, K, cal, rnd, stats=True)
+                ws = torch.empty(qsm.qsm_attn_bwd_workspace_size(*tw.shape), dtype=torch.uint8,
+                                 device=dev)
+                for _ in range(3):
+                    qsm.attention_backward(tq, tk, tv, O_, tdo, L_, st_, True, mode, K, cal, rnd,
+                                           surr, workspace=ws)
+                x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                x0.record(stream)
+                for _ in range(reps):
+                    qsm.attention_backward(tq, tk, tv, O_, tdo, L_, st_, True, mode, K, cal, rnd,
+                                           surr, workspace=ws)
+                x1.record(stream)
+                torch.cuda.synchronize()
+                ms = x0.elapsed_time(x1) / reps
+                tf = 2.5 * fwd_flops(tw) / (ms * 1e-3) / 1e12
+                lab = "%s_%s" % (mode_label((mode, K, cal, rnd)),
+                                 {1: "pre", 2: "post"}[surr])
+                res[lab] = {"bwd_ms": round(ms, 4), "bwd_tflops": round(tf, 1),
+                            "frac_of_bf16_peak": round(tf / peaks["bf16_sustained"], 4)}
+        extras["train_s1k_bwd"] = {"shape": list(tw.shape), "dtype": "bf16", "causal": True,
+                                   "flops": "2.5 x 4*B*H*S^2*D/2", "per_mode": res}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(w, modes, budget_s=args.cpu_budget)
