@@ -76,8 +76,14 @@ struct Geo {
 
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;   // 65536 / 384 rounded down to a multiple of 8
-constexpr int kCtrlRegs = 80;
-constexpr int kMapRegs = 200;
+// Register split (see the kernel): 104 for the control warps (their longest
+// MMA-issue loop, the two-sweep maps, spills below that) and 192 for the map
+// warps; 128 x 104 + 256 x 192 = 62464 <= 384 x 168.
+template <int MAP>
+struct RegSplit {
+  static constexpr int ctrl = 104;
+  static constexpr int map = 192;
+};
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -113,8 +119,10 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
 // Per-row constants of the fused map, with the score scale folded in: the
 // map consumes the raw fp32 accumulator r = q.k of the MMA.
 //   PoT:        x = fma(r, -c*log2e, hi*log2e), w = 2^-rne(min(x, cap)) * pscale
-//   K-interval: u = fma(r, c*K/(hi-lo), -lo*K/(hi-lo)), table look-up as in
-//               wmap.cuh (grid values pre-multiplied by pscale)
+//   K-interval: u = fma(r, c*K/(hi-lo), -lo*K/(hi-lo)); hard: g[rne(u)];
+//               interpolation: u d_k + c_k at k = floor(u) (grid values
+//               pre-multiplied by pscale).  Same decisions as the library's
+//               fp32 map up to the rounding of the folded scale.
 struct MapRow {
   float a, b;        // coordinate = fma(r, a, b)
   float cap, Kf, Km1;
@@ -131,19 +139,20 @@ __device__ __forceinline__ float map_raw(float r, const MapRow &m) {
     // kMagicBits << 23 == 0 (mod 2^32), so -(bits(t) << 23) == -(n << 23)
     return __uint_as_float(__float_as_uint(t) * 0xFF800000u + m.pow_bias);
   } else if (MAP == MAP_KI_HARD) {
-    const float u = __fmaf_rn(r, m.a, m.b);
-    const float uc = fminf(fmaxf(u, 0.0f), m.Kf);
-    const uint32_t tb = __float_as_uint(__fadd_rn(uc, kMagic));
+    // the clamp to [0, K] bounds the table index for every input (masked
+    // keys, ragged rows, near-degenerate rows, inf and NaN included)
+    const float u = fminf(fmaxf(__fmaf_rn(r, m.a, m.b), 0.0f), m.Kf);
+    const uint32_t tb = __float_as_uint(__fadd_rn(u, kMagic));
     return lds_f32(tb * 512u + m.tab);
   } else {
-    const float u = __fmaf_rn(r, m.a, m.b);
-    const float uc = fminf(fmaxf(u, 0.0f), m.Kf);
-    // floor(uc) for 0 <= uc < 2^23: add 2^23 rounding toward -inf
-    const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), m.Km1);
-    const float f = __fsub_rn(uc, kf);
-    const uint32_t tb = __float_as_uint(__fadd_rn(kf, kMagic));
-    const float2 gd = lds_f32x2(tb * 1024u + m.tab);
-    return __fmaf_rn(f, gd.y, gd.x);
+    // interpolation as one FMA: w = g_k + (u - k) d_k = u d_k + c_k with
+    // c_k = g_k - k d_k; k = floor(u) in [0, K] (the clamp bounds the index)
+    // through a round-down add of 2^23; the table entry at k = K repeats
+    // k = K - 1, which is the interpolation's value at u = K
+    const float u = fminf(fmaxf(__fmaf_rn(r, m.a, m.b), 0.0f), m.Kf);
+    const uint32_t tb = __float_as_uint(__fadd_rd(u, 8388608.0f));
+    const float2 cd = lds_f32x2(tb * 1024u + m.tab);
+    return __fmaf_rn(u, cd.y, cd.x);
   }
 }
 
@@ -356,14 +365,22 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
         for (int n = 0; n <= p.K; ++n) tab[n * 128 + row] = grid_value(rm, p.K, n) * p.pscale;
         mr.tab = tb + row * 4 - kMagicBits * 512u;
       } else {
+        // entries k = 0 .. K: (c_k, d_k); entry K repeats entry K - 1
         float gk = grid_value(rm, p.K, 0);
         for (int n = 0; n < p.K; ++n) {
           const float gk1 = grid_value(rm, p.K, n + 1);
-          tab[(n * 128 + row) * 2 + 0] = gk * p.pscale;
-          tab[(n * 128 + row) * 2 + 1] = __fsub_rn(gk1, gk) * p.pscale;
+          const float d = __fsub_rn(gk1, gk) * p.pscale;
+          const float c = __fmaf_rn(-static_cast<float>(n), d, gk * p.pscale);
+          tab[(n * 128 + row) * 2 + 0] = c;
+          tab[(n * 128 + row) * 2 + 1] = d;
+          if (n == p.K - 1) {
+            tab[(p.K * 128 + row) * 2 + 0] = c;
+            tab[(p.K * 128 + row) * 2 + 1] = d;
+          }
           gk = gk1;
         }
-        mr.tab = tb + row * 8 - kMagicBits * 1024u;
+        // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
+        mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
       }
     }
   }
@@ -608,6 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // group (producer, MMA issuer, two idle warps) gives most of its share to
   // the two map groups: 128 x kCtrlRegs + 256 x kMapRegs <= 384 x kLaunchRegs
   // (an increase beyond what the decrease freed would wait forever).
+  constexpr int kCtrlRegs = RegSplit<MAP>::ctrl;
+  constexpr int kMapRegs = RegSplit<MAP>::map;
   static_assert(128 * kCtrlRegs + 256 * kMapRegs <= kThreads * kLaunchRegs,
                 "register split must equal the launch allocation");
   if (warp < 4) {
@@ -805,9 +824,9 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.status = a.status_dev;
   p.debug_flags = a.debug_flags;
 
-  // grid table per query tile: [K+1][128] values (hard) or [K][128] (value,
-  // difference) pairs (interpolation)
-  p.tab_stride = (MAP == MAP_KI_INTERP) ? p.K * 128 * 2 : (p.K + 1) * 128;
+  // grid table per query tile: [K+1][128] values (hard) or [K+1][128]
+  // (c_k, d_k) pairs (interpolation)
+  p.tab_stride = (MAP == MAP_KI_INTERP) ? (p.K + 1) * 128 * 2 : (p.K + 1) * 128;
   const size_t table_bytes = static_cast<size_t>(2) * p.tab_stride * sizeof(float);
   const size_t bar_bytes = 256;
   const size_t max_smem = 232448;                        // 227 KB opt-in per CTA
