@@ -48,7 +48,7 @@ struct FwdParams {
   float pscale;     // P is stored as w * pscale (FP8 approximate maps: 64)
   int tab_stride;   // floats of grid table per query tile
   int num_stages;
-  uint32_t table_off, bar_off;
+  uint32_t table_off, bar_off, xch_off;
   __nv_bfloat16 *O;
   float *LSE, *hi, *lo;
   int32_t *amax, *amin;
@@ -74,15 +74,14 @@ struct Geo {
   static constexpr int P_COLS_PER_CHUNK = FP8 ? 8 : 16; // TMEM columns per 32 P values
 };
 
-constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;   // 65536 / 384 rounded down to a multiple of 8
-// Register split (see the kernel): 104 for the control warps (their longest
-// MMA-issue loop, the two-sweep maps, spills below that) and 192 for the map
-// warps; 128 x 104 + 256 x 192 = 62464 <= 384 x 168.
+constexpr int kThreads = 640;      // 4 control warps + 4 map warp groups
+constexpr int kLaunchRegs = 96;    // 65536 / 640 rounded down to a multiple of 8
+// Register split (see the kernel): with sixteen map warps every warp keeps
+// the launch allocation of 96 (no reallocation).
 template <int MAP>
 struct RegSplit {
-  static constexpr int ctrl = 104;
-  static constexpr int map = 192;
+  static constexpr int ctrl = 96;
+  static constexpr int map = 96;
 };
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
@@ -96,6 +95,7 @@ struct Bars {
   uint64_t *p_full;               // [2]
   uint64_t *o_full;               // [2]
   uint64_t *drain;                // 1
+  uint64_t *xstat, *xtile, *xz;   // [2 tiles] each: the halves' exchanges
   uint32_t *tmem_slot;
   int *abort;
 };
@@ -111,7 +111,10 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   b.p_full = b.s_empty + 4;
   b.o_full = b.p_full + 2;
   b.drain = b.o_full + 2;
-  b.tmem_slot = reinterpret_cast<uint32_t *>(b.drain + 1);
+  b.xstat = b.drain + 1;
+  b.xtile = b.xstat + 2;
+  b.xz = b.xtile + 2;
+  b.tmem_slot = reinterpret_cast<uint32_t *>(b.xz + 2);
   b.abort = reinterpret_cast<int *>(b.tmem_slot + 1);
   return b;
 }
@@ -178,7 +181,7 @@ __device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flus
 template <int MAP, bool FULL, bool FP8>
 __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow &m, int c0,
                                           int lim, bool flush_below, float (&z)[8],
-                                          uint32_t taddr_p, int cc) {
+                                          uint32_t taddr_pc) {
   auto wt = [&](int i) {
     const float r = __uint_as_float(v[i]);
     float wi = map_raw<MAP>(r, m);
@@ -197,7 +200,7 @@ __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow 
       const float a = wt(4 * i), b = wt(4 * i + 1), c = wt(4 * i + 2), d = wt(4 * i + 3);
       pk[i] = pack_e4m3x4(a, b, c, d);
     }
-    tmem_st8(taddr_p + cc * 8, pk);
+    tmem_st8(taddr_pc, pk);
   } else {
     uint32_t pk[16];
 #pragma unroll
@@ -205,7 +208,7 @@ __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow 
       const float a = wt(2 * i), b = wt(2 * i + 1);
       pk[i] = pack_bf16x2(a, b);
     }
-    tmem_st16(taddr_p + cc * 16, pk);
+    tmem_st16(taddr_pc, pk);
   }
 }
 
@@ -237,17 +240,31 @@ __device__ __forceinline__ bool full_tile(const FwdParams &p, int qi, int j) {
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
 __device__ __forceinline__ bool warp_any(bool x) { return __any_sync(0xffffffffu, x); }
 
-// One map warp group: 128 threads, thread `row` owns query row qi*128+row of
-// the CTA's tile t and TMEM lane `row`.
+// Per-row values the two halves of a query tile exchange through shared
+// memory (see map_half).
+struct Xch {
+  float4 *stats;      // [2 tiles][2 halves][128]: max, min, argmax, argmin
+  float *tilemax;     // [2 tiles][2 slots][2 halves][128]  (exact map)
+  float *zsum;        // [2 tiles][2 halves][128]
+};
+
+// One map warp group: 128 threads own half h (64 of the 128 key columns) of
+// every S tile of query tile t; thread `row` owns query row qi*128+row (TMEM
+// lane `row`).  The group that owns the other half shares the row: the two
+// combine row statistics, the exact map's tile maxima and the row sums
+// through shared memory behind bounded-wait barriers.  P of half h goes to
+// TMEM columns 64h.. of the tile's S buffer, which only this group reads.
 template <int D, bool FP8, int MAP>
-__device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, int t, int row,
-                                          uint32_t lane_base, int qi, int n_t, int bh,
-                                          float *tab, volatile int *abort) {
+__device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, int t, int h,
+                                         int row, uint32_t lane_base, int qi, int n_t, int bh,
+                                         float *tab, const Xch &xc, volatile int *abort) {
   constexpr bool kTwoPass = MAP != MAP_EXACT;
+  constexpr int PCOLS = FP8 ? 8 : 16;                  // TMEM columns per 32 P values
   const int qrow = qi * 128 + row;
   const bool row_ok = qrow < p.S;
   const int L = p.causal ? min(qrow + 1, p.S) : p.S;   // valid keys of the row
   if (n_t <= 0) return;
+  const int c_off = 64 * h;                            // first key column of this half
   uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
   bool ok = true;
   float rmax = -INFINITY, rmin = INFINITY;
@@ -267,35 +284,28 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
       if (b) ++sf_cnt1; else ++sf_cnt0;
       if (!ok) break;
       tc_fence_after();
-      const int lim = L - 128 * j;
+      const int lim = L - 128 * j - c_off;             // valid columns of this half
       const bool full = full_tile(p, qi, j);
-      const uint32_t base = lane_base + t * 128 + b * 256;
+      const uint32_t base = lane_base + t * 128 + b * 256 + c_off;
       if (want_arg) {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t v[32];
-          tmem_ld32_sync(base + 32 * cc, v);
+        auto scan = [&](const uint32_t(&cur)[32], int c0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(v[i]);
-            const bool valid = 32 * cc + i < lim;
-            if (valid && x > rmax) { rmax = x; amax = 128 * j + 32 * cc + i; }
-            if (valid && x < rmin) { rmin = x; amin = 128 * j + 32 * cc + i; }
+            const float x = __uint_as_float(cur[i]);
+            const bool valid = c0 + i < lim;
+            const int col = 128 * j + c_off + c0 + i;
+            if (valid && x > rmax) { rmax = x; amax = col; }
+            if (valid && x < rmin) { rmin = x; amin = col; }
           }
+        };
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(base + 32 * c, v);
+          scan(v, 32 * c);
         }
       } else {
-        // all four 32-column loads in flight, one wait
-        uint32_t v0[32], v1[32], v2[32], v3[32];
-        tmem_ld32(base, v0);
-        tmem_ld32(base + 32, v1);
-        tmem_ld32(base + 64, v2);
-        tmem_ld32(base + 96, v3);
-        tmem_wait_ld();
-        reg_fence32(v0);
-        reg_fence32(v1);
-        reg_fence32(v2);
-        reg_fence32(v3);
-        auto reduce = [&](const uint32_t(&cur)[32], int cc) {
+        auto reduce = [&](const uint32_t(&cur)[32], int c0) {
           if (full) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -307,16 +317,18 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float x = __uint_as_float(cur[i]);
-              const bool valid = 32 * cc + i < lim;
+              const bool valid = c0 + i < lim;
               mx[i & 7] = fmaxf(mx[i & 7], valid ? x : -INFINITY);
               if (want_min) mn[i & 7] = fminf(mn[i & 7], valid ? x : INFINITY);
             }
           }
         };
-        reduce(v0, 0);
-        reduce(v1, 1);
-        reduce(v2, 2);
-        reduce(v3, 3);
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(base + 32 * c, v);
+          reduce(v, 32 * c);
+        }
       }
       tc_fence_before();
       mbar_arrive(&bars.s_empty[t * 2 + b]);
@@ -327,6 +339,19 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
         rmax = fmaxf(rmax, mx[i]);
         rmin = fminf(rmin, mn[i]);
       }
+    }
+    // combine the two halves (ties: the lower key index)
+    if (ok) {
+      xc.stats[(t * 2 + h) * 128 + row] =
+          make_float4(rmax, rmin, __int_as_float(amax), __int_as_float(amin));
+      mbar_arrive(&bars.xstat[t]);
+      ok = warp_all(mbar_wait(&bars.xstat[t], 0, abort));
+    }
+    if (ok) {
+      const float4 o = xc.stats[(t * 2 + (h ^ 1)) * 128 + row];
+      const int oamax = __float_as_int(o.z), oamin = __float_as_int(o.w);
+      if (o.x > rmax || (o.x == rmax && oamax < amax)) { rmax = o.x; amax = oamax; }
+      if (o.y < rmin || (o.y == rmin && oamin < amin)) { rmin = o.y; amin = oamin; }
     }
   }
 
@@ -361,74 +386,69 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
       }
       lo = rm.lo;
       const uint32_t tb = smem_u32(tab);
+      // the two halves build alternate entries of this row's grid table
       if (MAP == MAP_KI_HARD) {
-        for (int n = 0; n <= p.K; ++n) tab[n * 128 + row] = grid_value(rm, p.K, n) * p.pscale;
+        for (int n = h; n <= p.K; n += 2) tab[n * 128 + row] = grid_value(rm, p.K, n) * p.pscale;
         mr.tab = tb + row * 4 - kMagicBits * 512u;
       } else {
-        // entries k = 0 .. K: (c_k, d_k); entry K repeats entry K - 1
-        float gk = grid_value(rm, p.K, 0);
-        for (int n = 0; n < p.K; ++n) {
-          const float gk1 = grid_value(rm, p.K, n + 1);
+        // entries k = 0 .. K: (c_k, d_k) with d_k = g_{k+1} - g_k and
+        // c_k = g_k - k d_k; entry K repeats entry K - 1
+        for (int n = h; n <= p.K; n += 2) {
+          const int k = n < p.K ? n : p.K - 1;
+          const float gk = grid_value(rm, p.K, k);
+          const float gk1 = grid_value(rm, p.K, k + 1);
           const float d = __fsub_rn(gk1, gk) * p.pscale;
-          const float c = __fmaf_rn(-static_cast<float>(n), d, gk * p.pscale);
-          tab[(n * 128 + row) * 2 + 0] = c;
+          tab[(n * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, gk * p.pscale);
           tab[(n * 128 + row) * 2 + 1] = d;
-          if (n == p.K - 1) {
-            tab[(p.K * 128 + row) * 2 + 0] = c;
-            tab[(p.K * 128 + row) * 2 + 1] = d;
-          }
-          gk = gk1;
         }
         // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
         mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
       }
+      // the table is complete before either half reads it
+      mbar_arrive(&bars.xstat[t]);
+      ok = warp_all(mbar_wait(&bars.xstat[t], 1, abort));
     }
   }
   int8_t *dbg_row = (p.dbg != nullptr && row_ok)
                         ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
                         : nullptr;
-  const uint32_t pbase = lane_base + t * 128;
+  const uint32_t pbase = lane_base + t * 128 + c_off;       // P columns of this half
 
   for (int j = 0; j < n_t && ok; ++j) {
     ok = warp_all(mbar_wait(&bars.s_full[t * 2 + 0], sf_cnt0 & 1, abort));
     ++sf_cnt0;
     if (!ok) break;
     tc_fence_after();
-    const int lim = L - 128 * j;
+    const int lim = L - 128 * j - c_off;
     const bool full = full_tile(p, qi, j);
-    const uint32_t sbase = lane_base + t * 128;
+    const uint32_t sbase = lane_base + t * 128 + c_off;
     if (MAP == MAP_EXACT) {
-      // tile maximum, then (lazily) move the anchor and rescale O
       float mx[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
-      uint32_t va[32], vb[32];
-      auto mstep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
-        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(sbase + 32 * c, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = __uint_as_float(cur[i]);
-          mx[i & 7] = fmaxf(mx[i & 7], (full || 32 * cc + i < lim) ? x : -INFINITY);
-        }
-        if (cc < 3) {
-          tmem_wait_ld();
-          reg_fence32(nxt);
-        }
-      };
-      tmem_ld32(sbase, va);
-      tmem_wait_ld();
-      reg_fence32(va);
-      mstep(va, vb, 0);
-      mstep(vb, va, 1);
-      mstep(va, vb, 2);
-      mstep(vb, va, 3);
+        for (int i = 0; i < 32; ++i)
+          mx[i & 7] = fmaxf(mx[i & 7], (full || 32 * c + i < lim) ? __uint_as_float(v[i]) : -INFINITY);
+      }
       float mt = mx[0];
 #pragma unroll
       for (int i = 1; i < 8; ++i) mt = fmaxf(mt, mx[i]);
+      // the tile maximum of the whole row
+      float *slot = xc.tilemax + ((t * 2 + (j & 1)) * 2) * 128;
+      slot[h * 128 + row] = mt;
+      mbar_arrive(&bars.xtile[t]);
+      ok = warp_all(mbar_wait(&bars.xtile[t], j & 1, abort));
+      if (!ok) break;
+      mt = fmaxf(mt, slot[(h ^ 1) * 128 + row]);
       m_run = fmaxf(m_run, mt);
       // move this row's anchor on its first tile, or when the running max grew
       // by more than 2^8 in weight; O is rescaled in TMEM when any row of the
-      // warp moved (rows that did not move use alpha = 1)
+      // warp moved (rows that did not move use alpha = 1).  Both halves take
+      // the same decisions (same rows, same combined maxima).
       const bool first = m_used == -INFINITY;
       const bool move = first || (m_run - m_used) * p.cL2E > kRescaleLog2;
       const float alpha = (move && !first) ? ex2_approx((m_used - m_run) * p.cL2E) : 1.0f;
@@ -436,9 +456,9 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
 #pragma unroll
       for (int i = 0; i < 8; ++i) z[i] *= alpha;
       if (j > 0 && warp_any(move)) {
-        const uint32_t obase = lane_base + 256 + t * 128;
+        const uint32_t obase = lane_base + 256 + t * 128 + h * (D / 2);
 #pragma unroll 1
-        for (int dc = 0; dc < D / 32; ++dc) {
+        for (int dc = 0; dc < D / 64; ++dc) {
           uint32_t v[32];
           tmem_ld32_sync(obase + 32 * dc, v);
 #pragma unroll
@@ -447,11 +467,10 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
         }
       }
       const float mb = m_used * p.cL2E;
-      auto estep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
-        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
-        auto ex = [&](int i) {
-          const float e = ex2_approx(__fmaf_rn(__uint_as_float(cur[i]), p.cL2E, -mb));
-          const float wi = (full || 32 * cc + i < lim) ? e : 0.0f;
+      auto ex = [&](const uint32_t(&cur)[32], int c0, uint32_t taddr) {
+        auto e = [&](int i) {
+          const float w = ex2_approx(__fmaf_rn(__uint_as_float(cur[i]), p.cL2E, -mb));
+          const float wi = (full || c0 + i < lim) ? w : 0.0f;
           z[i & 7] += wi;
           return wi;
         };
@@ -459,58 +478,45 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float a = ex(4 * i), b = ex(4 * i + 1), c = ex(4 * i + 2), d = ex(4 * i + 3);
+            const float a = e(4 * i), b = e(4 * i + 1), c = e(4 * i + 2), d = e(4 * i + 3);
             pk[i] = pack_e4m3x4(a, b, c, d);
           }
-          tmem_st8(pbase + cc * 8, pk);
+          tmem_st8(taddr, pk);
         } else {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = ex(2 * i), b = ex(2 * i + 1);
+            const float a = e(2 * i), b = e(2 * i + 1);
             pk[i] = pack_bf16x2(a, b);
           }
-          tmem_st16(pbase + cc * 16, pk);
-        }
-        if (cc < 3) {
-          tmem_wait_ld();
-          reg_fence32(nxt);
+          tmem_st16(taddr, pk);
         }
       };
-      tmem_ld32(sbase, va);
-      tmem_wait_ld();
-      reg_fence32(va);
-      estep(va, vb, 0);
-      estep(vb, va, 1);
-      estep(va, vb, 2);
-      estep(vb, va, 3);
-    } else {
-      uint32_t va[32], vb[32];
-      auto wstep = [&](uint32_t(&cur)[32], uint32_t(&nxt)[32], int cc) {
-        if (cc < 3) tmem_ld32(sbase + 32 * (cc + 1), nxt);
-        if (full)
-          map_chunk<MAP, true, FP8>(cur, mr, 32 * cc, lim, flush_below, z, pbase, cc);
-        else
-          map_chunk<MAP, false, FP8>(cur, mr, 32 * cc, lim, flush_below, z, pbase, cc);
-        if (p.dbg != nullptr)
-          debug_chunk<MAP>(dbg_row, cur, mr, 128 * j + 32 * cc, 32 * cc, lim, p, flush_below);
-        if (cc < 3) {
-          tmem_wait_ld();
-          reg_fence32(nxt);
-        }
-      };
-      tmem_ld32(sbase, va);
-      tmem_wait_ld();
-      reg_fence32(va);
 #pragma unroll 1
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        wstep(va, vb, c2);
-        wstep(vb, va, c2 + 1);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(sbase + 32 * c, v);
+        ex(v, 32 * c, pbase + c * PCOLS);
       }
-    }
-    if (MAP == MAP_EXACT && dbg_row != nullptr) {
-      const int kv0 = 128 * j;
-      for (int i = 0; i < 128 && kv0 + i < p.S; ++i) dbg_row[kv0 + i] = (i < lim) ? 0 : -1;
+      if (dbg_row != nullptr) {
+        for (int i = 0; i < 64; ++i) {
+          const int kv = 128 * j + c_off + i;
+          if (kv < p.S) dbg_row[kv] = (i < lim) ? 0 : -1;
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(sbase + 32 * c, v);
+        if (full)
+          map_chunk<MAP, true, FP8>(v, mr, 32 * c, lim, flush_below, z, pbase + c * PCOLS);
+        else
+          map_chunk<MAP, false, FP8>(v, mr, 32 * c, lim, flush_below, z, pbase + c * PCOLS);
+        if (p.dbg != nullptr)
+          debug_chunk<MAP>(dbg_row, v, mr, 128 * j + c_off + 32 * c, 32 * c, lim, p,
+                           flush_below);
+      }
     }
     tmem_wait_st();
     tc_fence_before();
@@ -522,12 +528,16 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
   if (!ok) return;
   tc_fence_after();
   float Z = ((z[0] + z[1]) + (z[2] + z[3])) + ((z[4] + z[5]) + (z[6] + z[7]));
+  xc.zsum[(t * 2 + h) * 128 + row] = Z;
+  mbar_arrive(&bars.xz[t]);
+  if (!warp_all(mbar_wait(&bars.xz[t], 0, abort))) return;
+  Z += xc.zsum[(t * 2 + (h ^ 1)) * 128 + row];
   if (MAP == MAP_EXACT) hi = p.c * m_run;
   const float oscale = p.v_descale / Z;          // pscale cancels: P and Z both carry it
-  const uint32_t obase = lane_base + 256 + t * 128;
-  __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D;
+  const uint32_t obase = lane_base + 256 + t * 128 + h * (D / 2);
+  __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D + h * (D / 2);
 #pragma unroll 1
-  for (int dc = 0; dc < D / 32; ++dc) {
+  for (int dc = 0; dc < D / 64; ++dc) {
     uint32_t v[32];
     tmem_ld32_sync(obase + 32 * dc, v);
     uint32_t pk[16];
@@ -542,7 +552,7 @@ __device__ __forceinline__ void map_group(const FwdParams &p, const Bars &bars, 
         dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
     }
   }
-  if (row_ok) {
+  if (row_ok && h == 0) {
     const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
     const float anchor = (MAP == MAP_EXACT) ? p.c * m_used : hi;
     p.LSE[ri] = anchor + logf(Z / p.pscale);
@@ -584,17 +594,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages
   float *sTab = reinterpret_cast<float *>(smem + p.table_off);
   Bars bars = carve_bars(smem + p.bar_off, ns);
+  Xch xc;
+  xc.stats = reinterpret_cast<float4 *>(smem + p.xch_off);
+  xc.tilemax = reinterpret_cast<float *>(smem + p.xch_off + 4 * 128 * 16);
+  xc.zsum = xc.tilemax + 8 * 128;
   volatile int *abort = bars.abort;
 
   const int nkvt = (p.S + 127) / 128;
-  int qi[2], nt[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    qi[t] = 2 * qb + t;
-    const bool exists = qi[t] < p.nqt;
-    nt[t] = exists ? (p.causal ? min(nkvt, qi[t] + 1) : nkvt) : 0;
-  }
-  const int nkv = max(nt[0], nt[1]);
+  // per query tile: index and number of key tiles (scalars, so the control
+  // loops never index a local array)
+  const int qi0 = 2 * qb, qi1 = 2 * qb + 1;
+  const int nt0 = p.causal ? min(nkvt, qi0 + 1) : nkvt;
+  const int nt1 = qi1 < p.nqt ? (p.causal ? min(nkvt, qi1 + 1) : nkvt) : 0;
+  auto NT = [&](int t) { return t ? nt1 : nt0; };
+  auto QI = [&](int t) { return t ? qi1 : qi0; };
+  const int nkv = max(nt0, nt1);
   constexpr bool kTwoPass = MAP != MAP_EXACT;
 
   if (threadIdx.x == 0) {
@@ -605,11 +619,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bars.q_full, 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_empty[i], 128);
+      mbar_init(&bars.s_empty[i], 256);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.p_full[i], 128);
+      mbar_init(&bars.p_full[i], 256);
       mbar_init(&bars.o_full[i], 1);
+      mbar_init(&bars.xstat[i], 256);
+      mbar_init(&bars.xtile[i], 256);
+      mbar_init(&bars.xz[i], 256);
     }
     mbar_init(bars.drain, 1);
     *bars.abort = 0;
@@ -623,38 +640,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // The CTA launches with kThreads x kLaunchRegs registers; the control warp
   // group (producer, MMA issuer, two idle warps) gives most of its share to
-  // the two map groups: 128 x kCtrlRegs + 256 x kMapRegs <= 384 x kLaunchRegs
+  // the four map groups: 128 x kCtrlRegs + 512 x kMapRegs <= 640 x kLaunchRegs
   // (an increase beyond what the decrease freed would wait forever).
   constexpr int kCtrlRegs = RegSplit<MAP>::ctrl;
   constexpr int kMapRegs = RegSplit<MAP>::map;
-  static_assert(128 * kCtrlRegs + 256 * kMapRegs <= kThreads * kLaunchRegs,
+  static_assert(128 * kCtrlRegs + 512 * kMapRegs <= kThreads * kLaunchRegs,
                 "register split must equal the launch allocation");
   if (warp < 4) {
-    regs_dec<kCtrlRegs>();
+    if (kCtrlRegs < kLaunchRegs) regs_dec<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && !(p.debug_flags & 1)) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int nq = (nt[0] > 0) + (nt[1] > 0);
+      const int nq = (nt0 > 0) + (nt1 > 0);
       mbar_expect_tx(bars.q_full, nq * G::TILE_BYTES);
       for (int t = 0; t < 2; ++t)
-        if (nt[t] > 0)
+        if (NT(t) > 0)
           for (int ch = 0; ch < G::CHUNKS; ++ch)
             tma_load_3d(sQ + t * G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmQ, bars.q_full,
-                        ch * G::EPC, qi[t] * 128, bh);
-      int it = 0;
+                        ch * G::EPC, QI(t) * 128, bh);
+      int it = 0, st = 0;
+      uint32_t ph = 0;                  // completed passes over the ring
       bool ok = true;
       auto load = [&](const CUtensorMap *m, int kvt) {
-        const int st = it % ns;
-        if (it >= ns) ok = ok && mbar_wait(&bars.kv_empty[st], ((it / ns) & 1) ^ 1, abort);
+        if (it >= ns) ok = ok && mbar_wait(&bars.kv_empty[st], ph ^ 1, abort);
         if (!ok) return;
         mbar_expect_tx(&bars.kv_full[st], G::TILE_BYTES);
         for (int ch = 0; ch < G::CHUNKS; ++ch)
           tma_load_3d(sKV + st * G::TILE_BYTES + ch * G::CHUNK_BYTES, m, &bars.kv_full[st],
                       ch * G::EPC, kvt * 128, bh);
         ++it;
+        if (++st == ns) {
+          st = 0;
+          ph ^= 1;
+        }
       };
       if (kTwoPass)
         for (int j = 0; j < nkv && ok; ++j) load(&tmK, j);
@@ -664,9 +685,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // let every load issued so far land before the CTA may exit
       mbar_wait(bars.q_full, 0, abort);
-      for (int st = 0; st < ns && st < it; ++st) {
-        const int fills = (it - st + ns - 1) / ns;  // loads issued into stage st
-        mbar_wait(&bars.kv_full[st], (fills - 1) & 1, abort);
+      for (int s = 0; s < ns && s < it; ++s) {
+        const int fills = (it - s + ns - 1) / ns;  // loads issued into stage s
+        mbar_wait(&bars.kv_full[s], (fills - 1) & 1, abort);
       }
     }
   } else if (warp == 1) {
@@ -674,13 +695,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t qaddr0 = smem_u32(sQ);
       const uint32_t kvaddr0 = smem_u32(sKV);
-      int it = 0;
+      int cst = 0;                      // next ring stage to consume
+      uint32_t cph = 0;                 // its phase parity
       bool ok = mbar_wait(bars.q_full, 0, abort);
       tc_fence_after();
       auto acquire = [&]() -> int {
-        const int st = it % ns;
-        ok = ok && mbar_wait(&bars.kv_full[st], (it / ns) & 1, abort);
-        ++it;
+        const int st = cst;
+        ok = ok && mbar_wait(&bars.kv_full[st], cph, abort);
+        if (++cst == ns) {
+          cst = 0;
+          cph ^= 1;
+        }
         tc_fence_after();
         return st;
       };
@@ -706,7 +731,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
           const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
-          const uint32_t at = tmem + pcol + kk * 8;
+          // keys 64h.. of the tile sit at TMEM columns 64h.. (each map half
+          // writes its P into its own S columns), 8 columns per k-step
+          const int key0 = kk * G::MMA_K;
+          const uint32_t at = tmem + pcol + 64 * (key0 / 64) + ((key0 % 64) / G::MMA_K) * 8;
           if (FP8)
             mma_ts_f8(tmem + ocol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
           else
@@ -719,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = acquire();
           if (!ok) break;
           for (int t = 0; t < 2 && ok; ++t) {
-            if (j >= nt[t]) continue;
+            if (j >= NT(t)) continue;
             const int b = j & 1, use = j >> 1;
             if (use >= 1) {
               ok = mbar_wait(&bars.s_empty[t * 2 + b], (use - 1) & 1, abort);
@@ -733,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // both S buffers of each tile must be read out before the main sweep
         for (int t = 0; t < 2 && ok; ++t) {
-          const int u0 = (nt[t] + 1) / 2, u1 = nt[t] / 2;
+          const int u0 = (NT(t) + 1) / 2, u1 = NT(t) / 2;
           if (u0 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 0], (u0 - 1) & 1, abort);
           if (u1 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 1], (u1 - 1) & 1, abort);
         }
@@ -743,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = acquire();
         if (ok) {
           for (int t = 0; t < 2; ++t)
-            if (nt[t] > 0) {
+            if (NT(t) > 0) {
               issue_qk(t, k0, t * 128);
               mma_commit(&bars.s_full[t * 2 + 0]);
             }
@@ -755,13 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int knext = has_next ? acquire() : -1;
           if (!ok) break;
           for (int t = 0; t < 2 && ok; ++t) {
-            if (j < nt[t]) {
+            if (j < NT(t)) {
               ok = mbar_wait(&bars.p_full[t], j & 1, abort);
               tc_fence_after();
               if (!ok) break;
               issue_pv(t, vst, j > 0);
             }
-            if (has_next && j + 1 < nt[t]) {
+            if (has_next && j + 1 < NT(t)) {
               issue_qk(t, knext, t * 128);
               mma_commit(&bars.s_full[t * 2 + 0]);
             }
@@ -770,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (has_next) mma_commit(&bars.kv_empty[knext]);
         }
         for (int t = 0; t < 2; ++t)
-          if (nt[t] > 0) mma_commit(&bars.o_full[t]);
+          if (NT(t) > 0) mma_commit(&bars.o_full[t]);
       }
       // every MMA issued must finish before TMEM is released
       mma_commit(bars.drain);
@@ -778,11 +806,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    regs_inc<kMapRegs>();
-    const int t = (warp - 4) >> 2;
-    map_group<D, FP8, MAP>(p, bars, t, threadIdx.x - 128 - t * 128,
-                           tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi[t], nt[t],
-                           bh, sTab + t * p.tab_stride, abort);
+    if (kMapRegs > kLaunchRegs) regs_inc<kMapRegs>();
+    const int g = (warp - 4) >> 2;                 // map group 0..3
+    const int t = g >> 1, h = g & 1;               // query tile, key-column half
+    map_half<D, FP8, MAP>(p, bars, t, h, threadIdx.x - 128 - g * 128,
+                          tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), QI(t), NT(t),
+                          bh, sTab + t * p.tab_stride, xc, abort);
   }
 
   __syncwarp();
@@ -828,16 +857,22 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   // (c_k, d_k) pairs (interpolation)
   p.tab_stride = (MAP == MAP_KI_INTERP) ? (p.K + 1) * 128 * 2 : (p.K + 1) * 128;
   const size_t table_bytes = static_cast<size_t>(2) * p.tab_stride * sizeof(float);
-  const size_t bar_bytes = 256;
+  // Bars: 2 per ring stage + 20 fixed mbarriers, then tmem_slot and abort;
+  // sized for the deepest ring allowed below
+  constexpr int kMaxStages = 8;
+  const size_t bar_bytes = ((2 * kMaxStages + 20) * 8 + 8 + 15) & ~static_cast<size_t>(15);
   const size_t max_smem = 232448;                        // 227 KB opt-in per CTA
-  const size_t fixed = 1024 + 2 * G::TILE_BYTES + table_bytes + bar_bytes;
+  const size_t fixed = 1024 + 2 * G::TILE_BYTES + table_bytes + bar_bytes +
+                       (4 * 128 * 16 + 8 * 128 * 4 + 4 * 128 * 4);
   int ns = static_cast<int>((max_smem - fixed) / G::TILE_BYTES);
-  if (ns > 4) ns = 4;
+  if (ns > kMaxStages) ns = kMaxStages;
   if (ns < 2) return QSM_ERR_UNSUPPORTED;
   p.num_stages = ns;
   p.table_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * G::TILE_BYTES);
   p.bar_off = static_cast<uint32_t>((p.table_off + table_bytes + 15) & ~static_cast<size_t>(15));
-  size_t smem = 1024 + p.bar_off + bar_bytes;
+  p.xch_off = p.bar_off + static_cast<uint32_t>(bar_bytes);
+  const size_t xch_bytes = 4 * 128 * 16 + 8 * 128 * 4 + 4 * 128 * 4;
+  size_t smem = 1024 + p.xch_off + xch_bytes;
   // one CTA per SM: the kernel allocates all 512 TMEM columns
   if (smem < 120 * 1024) smem = 120 * 1024;
 
