@@ -1,24 +1,33 @@
 // fwd.cu -- fused approximate-softmax attention forward for sm_100a.
 //
-// One CTA owns two 128-row query tiles of one (b, h) and sweeps the key/value
+// One CTA owns one 128-row query tile of one (b, h) and sweeps the key/value
 // tiles of 128 rows ("QK tile -> row max -> power-of-two weights -> PV matmul
 // -> output", the tile loop of "Approximating Softmax in Pretrained LLMs",
-// wiki flowchart).  Roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, then K (statistics sweep) and
+// wiki flowchart).  Roles (20 warps):
+//   warp 0      TMA producer: the Q tile once, then K (statistics sweep) and
 //               K, V (main sweep) through a ring of shared-memory stages.
-//   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (tcgen05, both
-//               operands in shared memory) and O += P V with P read from TMEM.
-//   warps 4-7   map group for query tile 0, one thread per row (TMEM lane).
-//   warps 8-11  map group for query tile 1.
-// TMEM (512 columns): S0 at 0, S1 at 128, O0 at 256, O1 at 384.  P (bf16 or
-// e4m3, packed) overwrites the S columns it was computed from.  During the
-// statistics sweep the O columns double as second S buffers.
+//   warp 1      QK issuer (one thread): S = Q K^T into TMEM (tcgen05, both
+//               operands in shared memory).
+//   warp 2      PV issuer (one thread): O += P V with P read from TMEM.
+//   warps 4-19  four map groups of four warps (one thread per query row, the
+//               row's TMEM lane), paired: pair 0 (warps 4-11) maps the even
+//               key tiles, pair 1 (warps 12-19) the odd ones, so the two
+//               pairs work on consecutive tiles at once; within a pair each
+//               group owns 64 of the tile's 128 key columns.
+// TMEM (512 columns): three S buffers at 0, 128, 256 and O at 384.  P (bf16
+// or e4m3, packed) overwrites the S columns it was computed from, so the QK
+// issuer runs up to two key tiles ahead of the map.  During the statistics
+// sweep the O columns serve as a fourth S buffer.  Splitting the MMA stream
+// over two issuers on different SM sub-partitions halves the instructions
+// each must issue per key tile; the statistics sweep alternates key tiles
+// between them.
 //
-// Approximate maps are defined against the row's final maximum (and minimum),
-// so they run a statistics sweep first (S tiles, max/min/argmax/argmin only,
-// no PV), then the main sweep with the row constants fixed.  The exact map
-// needs no such sweep: it rescales online, and rescales O only when the
-// running maximum grew by more than 2^8 in weight.
+// The approximate maps are defined against the row's final maximum (and
+// minimum), so every map runs a statistics sweep first (S tiles, max / min /
+// argmax / argmin only, no PV), then the main sweep with the row constants
+// fixed.  The exact map uses the same two sweeps: softmax against the true
+// row maximum, so O is never rescaled and the maps differ only in the weight
+// arithmetic.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,7 +44,7 @@ namespace qsm {
 enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
 
 struct FwdParams {
-  int S, nqt, nqb, BH;
+  int S, nqt, BH;
   int causal;
   int K;
   int fixed_window;
@@ -46,7 +55,7 @@ struct FwdParams {
   float window;
   float v_descale;
   float pscale;     // P is stored as w * pscale (FP8 approximate maps: 64)
-  int tab_stride;   // floats of grid table per query tile
+  int tab_stride;   // floats of grid table
   int num_stages;
   uint32_t table_off, bar_off, xch_off;
   __nv_bfloat16 *O;
@@ -71,34 +80,52 @@ struct Geo {
   static constexpr uint32_t FMT = FP8 ? 0u : 1u;        // e4m3 / bf16 format code
   static constexpr uint32_t IDESC_QK = instr_desc(FMT, false, 128, BN);
   static constexpr uint32_t IDESC_PV = instr_desc(FMT, true, 128, D);
-  static constexpr int P_COLS_PER_CHUNK = FP8 ? 8 : 16; // TMEM columns per 32 P values
 };
 
 constexpr int kThreads = 640;      // 4 control warps + 4 map warp groups
-constexpr int kLaunchRegs = 96;    // 65536 / 640 rounded down to a multiple of 8
-// Register split (see the kernel): with sixteen map warps every warp keeps
-// the launch allocation of 96 (no reallocation).
-template <int MAP>
-struct RegSplit {
-  static constexpr int ctrl = 96;
-  static constexpr int map = 96;
-};
+// Every warp keeps the launch allocation of 96 registers (65536 / 640).
+constexpr int kGroups = 4;         // map warp groups
+constexpr int kHalfCols = 64;     // key columns per map group and tile
+constexpr int kMapThreads = 128 * kGroups;
+constexpr int kPairThreads = 256;  // two groups map one key tile
+constexpr int kSBufs = 3;          // S / P buffers of the main sweep
+constexpr int kStatBufs = 4;       // S buffers of the statistics sweep
+constexpr uint32_t kOCol = 384;    // first TMEM column of O
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.0f;
+constexpr int kMaxStages = 8;
+// Statistics-sweep issuers: warps 1 and 2 take alternate key tiles, so each
+// S buffer (tile j % 4) is always fed by the same issuer; a buffer shared by
+// two issuers could see a later tile's wait pass on an older phase of the
+// same parity.
+constexpr int kStatIssuers = 2;
+static_assert(kStatBufs % kStatIssuers == 0, "each statistics buffer needs a single issuer");
+constexpr int kLead = 3;           // K tiles enter the ring this far ahead of V
 
-// barrier slots (uint64 each) after the stage barriers
+// Main-sweep ring order: K_0 .. K_{kLead-1}, then V_0, K_kLead, V_1,
+// K_kLead+1, ..., and the V tiles left over at the end.  K runs ahead because
+// S = Q K^T is issued up to two tiles before the PV product that needs V.
+__device__ __forceinline__ int ring_pos_k(int j) { return j < kLead ? j : 2 * j - kLead + 1; }
+__device__ __forceinline__ int ring_pos_v(int j, int n) {
+  return j < n - kLead ? kLead + 2 * j : n + j;
+}
+
+// mbarriers: two per ring stage, then the fixed ones
 struct Bars {
-  uint64_t *kv_full, *kv_empty;   // [stages]
-  uint64_t *q_full;               // 1
-  uint64_t *s_full;               // [2 tiles][2 buffers]
-  uint64_t *s_empty;              // [2][2]
-  uint64_t *p_full;               // [2]
-  uint64_t *o_full;               // [2]
-  uint64_t *drain;                // 1
-  uint64_t *xstat, *xtile, *xz;   // [2 tiles] each: the halves' exchanges
+  uint64_t *kv_full, *kv_empty;          // [stages]
+  uint64_t *q_full;                      // 1
+  uint64_t *st_full, *st_empty;          // [kStatBufs] statistics sweep
+  uint64_t *s_full, *p_full, *s_free;    // [kSBufs] main sweep
+  uint64_t *o_full;                      // 1
+  uint64_t *drain;                       // 1
+  uint64_t *xstat, *xz;                  // 1 each: the map groups' exchanges
   uint32_t *tmem_slot;
   int *abort;
 };
+constexpr int kFixedBars = 1 + 2 * kStatBufs + 3 * kSBufs + 2 + 2;
+
+__host__ __device__ constexpr size_t bar_bytes_for(int ns) {
+  return ((2 * static_cast<size_t>(ns) + kFixedBars) * 8 + 8 + 15) & ~static_cast<size_t>(15);
+}
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   Bars b;
@@ -106,15 +133,16 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   b.kv_full = p;
   b.kv_empty = p + ns;
   b.q_full = p + 2 * ns;
-  b.s_full = b.q_full + 1;
-  b.s_empty = b.s_full + 4;
-  b.p_full = b.s_empty + 4;
-  b.o_full = b.p_full + 2;
-  b.drain = b.o_full + 2;
+  b.st_full = b.q_full + 1;
+  b.st_empty = b.st_full + kStatBufs;
+  b.s_full = b.st_empty + kStatBufs;
+  b.p_full = b.s_full + kSBufs;
+  b.s_free = b.p_full + kSBufs;
+  b.o_full = b.s_free + kSBufs;
+  b.drain = b.o_full + 1;
   b.xstat = b.drain + 1;
-  b.xtile = b.xstat + 2;
-  b.xz = b.xtile + 2;
-  b.tmem_slot = reinterpret_cast<uint32_t *>(b.xz + 2);
+  b.xz = b.xstat + 1;
+  b.tmem_slot = reinterpret_cast<uint32_t *>(b.xz + 1);
   b.abort = reinterpret_cast<int *>(b.tmem_slot + 1);
   return b;
 }
@@ -129,33 +157,75 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
 struct MapRow {
   float a, b;        // coordinate = fma(r, a, b)
   float cap, Kf, Km1;
+  float flush_t;     // PoT flush: kMagic + floor (t above it: exponent past the floor)
   uint32_t tab;      // shared address bias of this row's table column
   uint32_t pow_bias; // bits of pscale (PoT)
 };
 
-template <int MAP>
-__device__ __forceinline__ float map_raw(float r, const MapRow &m) {
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE round-to-nearest
+// (or round-down) operations per instruction, the same results as the
+// scalar forms).
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_from(uint64_t r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(r);
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(r);
+}
+__device__ __forceinline__ float2 add2_rd(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(r);
+}
+
+// Weights of two scores (the map's arithmetic on a pair; FLUSH: Rowmax-PoT
+// with the below-floor policy "flush", exponents above the floor give 0).
+template <int MAP, bool FLUSH>
+__device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
+  const float2 x = fma2_rn(r, make_float2(m.a, m.a), make_float2(m.b, m.b));
   if (MAP == MAP_POT) {
-    const float x = __fmaf_rn(r, m.a, m.b);
-    const float t = __fadd_rn(fminf(x, m.cap), kMagic);
+    const float2 t =
+        add2_rn(make_float2(fminf(x.x, m.cap), fminf(x.y, m.cap)), make_float2(kMagic, kMagic));
     // 2^-n * pscale from the exponent field: bits(t) = kMagicBits + n and
     // kMagicBits << 23 == 0 (mod 2^32), so -(bits(t) << 23) == -(n << 23)
-    return __uint_as_float(__float_as_uint(t) * 0xFF800000u + m.pow_bias);
+    float2 w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + m.pow_bias),
+                           __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + m.pow_bias));
+    if (FLUSH) {
+      // t is kMagic + n exactly: n > floor  <=>  t > kMagic + floor
+      if (t.x > m.flush_t) w.x = 0.0f;
+      if (t.y > m.flush_t) w.y = 0.0f;
+    }
+    return w;
   } else if (MAP == MAP_KI_HARD) {
     // the clamp to [0, K] bounds the table index for every input (masked
     // keys, ragged rows, near-degenerate rows, inf and NaN included)
-    const float u = fminf(fmaxf(__fmaf_rn(r, m.a, m.b), 0.0f), m.Kf);
-    const uint32_t tb = __float_as_uint(__fadd_rn(u, kMagic));
-    return lds_f32(tb * 512u + m.tab);
+    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
+    const float2 t = add2_rn(u, make_float2(kMagic, kMagic));
+    return make_float2(lds_f32(__float_as_uint(t.x) * 512u + m.tab),
+                       lds_f32(__float_as_uint(t.y) * 512u + m.tab));
   } else {
     // interpolation as one FMA: w = g_k + (u - k) d_k = u d_k + c_k with
     // c_k = g_k - k d_k; k = floor(u) in [0, K] (the clamp bounds the index)
     // through a round-down add of 2^23; the table entry at k = K repeats
     // k = K - 1, which is the interpolation's value at u = K
-    const float u = fminf(fmaxf(__fmaf_rn(r, m.a, m.b), 0.0f), m.Kf);
-    const uint32_t tb = __float_as_uint(__fadd_rd(u, 8388608.0f));
-    const float2 cd = lds_f32x2(tb * 1024u + m.tab);
-    return __fmaf_rn(u, cd.y, cd.x);
+    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
+    const float2 t = add2_rd(u, make_float2(8388608.0f, 8388608.0f));
+    const float2 c0 = lds_f32x2(__float_as_uint(t.x) * 1024u + m.tab);
+    const float2 c1 = lds_f32x2(__float_as_uint(t.y) * 1024u + m.tab);
+    return make_float2(__fmaf_rn(u.x, c0.y, c0.x), __fmaf_rn(u.y, c1.y, c1.x));
   }
 }
 
@@ -177,36 +247,42 @@ __device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flus
 }
 
 // Weights of one 32-column chunk, packed for the PV MMA and stored to TMEM;
-// FULL: every column valid.
-template <int MAP, bool FULL, bool FP8>
+// FULL: every column valid.  z holds eight partial row sums as four pairs.
+template <int MAP, bool FULL, bool FP8, bool FLUSH>
 __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow &m, int c0,
-                                          int lim, bool flush_below, float (&z)[8],
+                                          int lim, bool flush_below, float2 (&z)[4],
                                           uint32_t taddr_pc) {
-  auto wt = [&](int i) {
-    const float r = __uint_as_float(v[i]);
-    float wi = map_raw<MAP>(r, m);
+  auto wt = [&](int i) {          // weights of columns 2i, 2i+1
+    const float2 r = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+    float2 w = map_pair<MAP, FLUSH>(r, m);
     if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
       // fixed-window flush: coordinate below the window
-      if (flush_below && __fmaf_rn(r, m.a, m.b) < 0.0f) wi = 0.0f;
+      if (flush_below) {
+        if (__fmaf_rn(r.x, m.a, m.b) < 0.0f) w.x = 0.0f;
+        if (__fmaf_rn(r.y, m.a, m.b) < 0.0f) w.y = 0.0f;
+      }
     }
-    if (!FULL) wi = (c0 + i < lim) ? wi : 0.0f;
-    z[i & 7] += wi;
-    return wi;
+    if (!FULL) {
+      w.x = (c0 + 2 * i < lim) ? w.x : 0.0f;
+      w.y = (c0 + 2 * i + 1 < lim) ? w.y : 0.0f;
+    }
+    z[i & 3] = add2_rn(z[i & 3], w);
+    return w;
   };
   if (FP8) {
     uint32_t pk[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float a = wt(4 * i), b = wt(4 * i + 1), c = wt(4 * i + 2), d = wt(4 * i + 3);
-      pk[i] = pack_e4m3x4(a, b, c, d);
+      const float2 a = wt(2 * i), b = wt(2 * i + 1);
+      pk[i] = pack_e4m3x4(a.x, a.y, b.x, b.y);
     }
     tmem_st8(taddr_pc, pk);
   } else {
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const float a = wt(2 * i), b = wt(2 * i + 1);
-      pk[i] = pack_bf16x2(a, b);
+      const float2 a = wt(i);
+      pk[i] = pack_bf16x2(a.x, a.y);
     }
     tmem_st16(taddr_pc, pk);
   }
@@ -240,32 +316,106 @@ __device__ __forceinline__ bool full_tile(const FwdParams &p, int qi, int j) {
 __device__ __forceinline__ bool warp_all(bool x) { return __all_sync(0xffffffffu, x); }
 __device__ __forceinline__ bool warp_any(bool x) { return __any_sync(0xffffffffu, x); }
 
-// Per-row values the two halves of a query tile exchange through shared
-// memory (see map_half).
+// Per-row values the map groups exchange through shared memory (see
+// map_half).
 struct Xch {
-  float4 *stats;      // [2 tiles][2 halves][128]: max, min, argmax, argmin
-  float *tilemax;     // [2 tiles][2 slots][2 halves][128]  (exact map)
-  float *zsum;        // [2 tiles][2 halves][128]
+  float4 *stats;      // [kGroups][128]: max, min, argmax, argmin
+  float *zsum;        // [kGroups][128]
 };
+constexpr size_t kXchBytes = kGroups * 128 * 16 + kGroups * 128 * 4;
 
-// One map warp group: 128 threads own half h (64 of the 128 key columns) of
-// every S tile of query tile t; thread `row` owns query row qi*128+row (TMEM
-// lane `row`).  The group that owns the other half shares the row: the two
-// combine row statistics, the exact map's tile maxima and the row sums
-// through shared memory behind bounded-wait barriers.  P of half h goes to
-// TMEM columns 64h.. of the tile's S buffer, which only this group reads.
+// Three-input fp32 maximum / minimum (one instruction on sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Scale this group's O columns, pack to bf16 and store the row's slice.
+template <int OC>
+__device__ __forceinline__ void o_store(uint32_t taddr, float oscale, __nv_bfloat16 *dst,
+                                        bool row_ok) {
+  uint32_t v[OC];
+  if constexpr (OC == 32)
+    tmem_ld32_sync(taddr, v);
+  else
+    tmem_ld16_sync(taddr, v);
+  uint32_t pk[OC / 2];
+#pragma unroll
+  for (int i = 0; i < OC / 2; ++i)
+    pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * oscale, __uint_as_float(v[2 * i + 1]) * oscale);
+  if (row_ok) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < OC / 8; ++i)
+      d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  }
+}
+
+// Exact weights of one 32-column chunk against the row maximum, packed and
+// stored to TMEM like map_chunk.
+template <bool FULL, bool FP8>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], float cL2E, float mL2E, int c0,
+                                          int lim, float2 (&z)[4], uint32_t taddr_pc) {
+  auto e = [&](int i) {           // weights of columns 2i, 2i+1
+    const float2 x = fma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                             make_float2(cL2E, cL2E), make_float2(-mL2E, -mL2E));
+    float2 w = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    if (!FULL) {
+      w.x = (c0 + 2 * i < lim) ? w.x : 0.0f;
+      w.y = (c0 + 2 * i + 1 < lim) ? w.y : 0.0f;
+    }
+    z[i & 3] = add2_rn(z[i & 3], w);
+    return w;
+  };
+  if (FP8) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 a = e(2 * i), b = e(2 * i + 1);
+      pk[i] = pack_e4m3x4(a.x, a.y, b.x, b.y);
+    }
+    tmem_st8(taddr_pc, pk);
+  } else {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 a = e(i);
+      pk[i] = pack_bf16x2(a.x, a.y);
+    }
+    tmem_st16(taddr_pc, pk);
+  }
+}
+
+// One map warp group: group g = 2 * pair + half.  The pair takes key tiles
+// j = pair, pair + 2, ... (the two pairs work on consecutive tiles at once);
+// the half owns key columns 64 * half .. 64 * half + 63 of each of them.
+// Thread `row` owns query row qi*128+row (TMEM lane `row`).  The four groups
+// share each row: they combine the row statistics and the row sums through
+// shared memory behind bounded-wait barriers, and build the row's grid table
+// together.  P of the group's columns goes to the first 16 (e4m3) or 32
+// (bf16) of its own S columns.
+//
+// Every map runs two sweeps: the statistics sweep finds the row's maximum
+// (and minimum, arguments) over all keys, then the main sweep maps each score
+// against those final values.  For the exact map this is softmax against the
+// true row maximum, with no online rescaling of O.
 template <int D, bool FP8, int MAP>
-__device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, int t, int h,
-                                         int row, uint32_t lane_base, int qi, int n_t, int bh,
-                                         float *tab, const Xch &xc, volatile int *abort) {
-  constexpr bool kTwoPass = MAP != MAP_EXACT;
+__device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, int g, int row,
+                                         uint32_t lane_base, int qi, int n, int bh, float *tab,
+                                         const Xch &xc, volatile int *abort) {
+  constexpr int OC = D / kGroups;                      // O columns of this group
   constexpr int PCOLS = FP8 ? 8 : 16;                  // TMEM columns per 32 P values
+  const int pair = g >> 1, h = g & 1;
   const int qrow = qi * 128 + row;
   const bool row_ok = qrow < p.S;
   const int L = p.causal ? min(qrow + 1, p.S) : p.S;   // valid keys of the row
-  if (n_t <= 0) return;
-  const int c_off = 64 * h;                            // first key column of this half
-  uint32_t sf_cnt0 = 0, sf_cnt1 = 0;
+  const int c_off = kHalfCols * h;                     // first key column of this group
   bool ok = true;
   float rmax = -INFINITY, rmin = INFINITY;
   int amax = 0, amin = 0;
@@ -274,93 +424,96 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
       ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window) || p.lo != nullptr;
 
   // -------------------------------------------------- statistics sweep
-  if (kTwoPass) {
-    float mx[8], mn[8];
+  {
+    float mx[4], mn[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { mx[i] = -INFINITY; mn[i] = INFINITY; }
-    for (int j = 0; j < n_t && ok; ++j) {
-      const int b = j & 1;
-      ok = warp_all(mbar_wait(&bars.s_full[t * 2 + b], (b ? sf_cnt1 : sf_cnt0) & 1, abort));
-      if (b) ++sf_cnt1; else ++sf_cnt0;
+    for (int i = 0; i < 4; ++i) { mx[i] = -INFINITY; mn[i] = INFINITY; }
+    for (int j = pair; j < n && ok; j += 2) {
+      const int b = j & 3;                             // S buffer of tile j
+      ok = warp_all(mbar_wait(&bars.st_full[b], (j >> 2) & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      const int lim = L - 128 * j - c_off;             // valid columns of this half
+      const int lim = L - 128 * j - c_off;             // valid columns of this group
       const bool full = full_tile(p, qi, j);
-      const uint32_t base = lane_base + t * 128 + b * 256 + c_off;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lane_base + b * 128 + c_off, v0);
+      tmem_ld32(lane_base + b * 128 + c_off + 32, v1);
+      tmem_wait_ld();
+      reg_fence32(v0);
+      reg_fence32(v1);
+      // the values are in registers: hand the buffer back before the reduction
+      tc_fence_before();
+      mbar_arrive(&bars.st_empty[b]);
       if (want_arg) {
-        auto scan = [&](const uint32_t(&cur)[32], int c0) {
+        auto scan = [&](const uint32_t(&v)[32], int c0) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(cur[i]);
+            const float x = __uint_as_float(v[i]);
             const bool valid = c0 + i < lim;
             const int col = 128 * j + c_off + c0 + i;
             if (valid && x > rmax) { rmax = x; amax = col; }
             if (valid && x < rmin) { rmin = x; amin = col; }
           }
         };
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tmem_ld32_sync(base + 32 * c, v);
-          scan(v, 32 * c);
+        scan(v0, 0);
+        scan(v1, 32);
+      } else if (full) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a0 = __uint_as_float(v0[2 * i]), a1 = __uint_as_float(v0[2 * i + 1]);
+          const float b0 = __uint_as_float(v1[2 * i]), b1 = __uint_as_float(v1[2 * i + 1]);
+          mx[i & 1] = max3f(mx[i & 1], a0, a1);
+          mx[2 + (i & 1)] = max3f(mx[2 + (i & 1)], b0, b1);
+          if (want_min) {
+            mn[i & 1] = min3f(mn[i & 1], a0, a1);
+            mn[2 + (i & 1)] = min3f(mn[2 + (i & 1)], b0, b1);
+          }
         }
       } else {
-        auto reduce = [&](const uint32_t(&cur)[32], int c0) {
-          if (full) {
+        auto red = [&](const uint32_t(&v)[32], int c0, int k) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(cur[i]);
-              mx[i & 7] = fmaxf(mx[i & 7], x);
-              if (want_min) mn[i & 7] = fminf(mn[i & 7], x);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = __uint_as_float(cur[i]);
-              const bool valid = c0 + i < lim;
-              mx[i & 7] = fmaxf(mx[i & 7], valid ? x : -INFINITY);
-              if (want_min) mn[i & 7] = fminf(mn[i & 7], valid ? x : INFINITY);
-            }
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+            const bool va = c0 + 2 * i < lim, vb = c0 + 2 * i + 1 < lim;
+            mx[k + (i & 1)] = max3f(mx[k + (i & 1)], va ? a0 : -INFINITY, vb ? a1 : -INFINITY);
+            if (want_min)
+              mn[k + (i & 1)] = min3f(mn[k + (i & 1)], va ? a0 : INFINITY, vb ? a1 : INFINITY);
           }
         };
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tmem_ld32_sync(base + 32 * c, v);
-          reduce(v, 32 * c);
-        }
+        red(v0, 0, 0);
+        red(v1, 32, 2);
       }
-      tc_fence_before();
-      mbar_arrive(&bars.s_empty[t * 2 + b]);
     }
     if (!want_arg) {
+      rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+      rmin = min3f(mn[0], mn[1], fminf(mn[2], mn[3]));
+    }
+    // combine the four groups in a fixed order (ties: the lower key index), so
+    // every group ends with the same row statistics
+    if (ok) {
+      xc.stats[g * 128 + row] = make_float4(rmax, rmin, __int_as_float(amax), __int_as_float(amin));
+      mbar_arrive(bars.xstat);
+      ok = warp_all(mbar_wait(bars.xstat, 0, abort));
+    }
+    if (ok) {
+      rmax = -INFINITY;
+      rmin = INFINITY;
+      amax = amin = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        rmax = fmaxf(rmax, mx[i]);
-        rmin = fminf(rmin, mn[i]);
+      for (int gg = 0; gg < kGroups; ++gg) {
+        const float4 o = xc.stats[gg * 128 + row];
+        const int oamax = __float_as_int(o.z), oamin = __float_as_int(o.w);
+        if (o.x > rmax || (o.x == rmax && oamax < amax)) { rmax = o.x; amax = oamax; }
+        if (o.y < rmin || (o.y == rmin && oamin < amin)) { rmin = o.y; amin = oamin; }
       }
-    }
-    // combine the two halves (ties: the lower key index)
-    if (ok) {
-      xc.stats[(t * 2 + h) * 128 + row] =
-          make_float4(rmax, rmin, __int_as_float(amax), __int_as_float(amin));
-      mbar_arrive(&bars.xstat[t]);
-      ok = warp_all(mbar_wait(&bars.xstat[t], 0, abort));
-    }
-    if (ok) {
-      const float4 o = xc.stats[(t * 2 + (h ^ 1)) * 128 + row];
-      const int oamax = __float_as_int(o.z), oamin = __float_as_int(o.w);
-      if (o.x > rmax || (o.x == rmax && oamax < amax)) { rmax = o.x; amax = oamax; }
-      if (o.y < rmin || (o.y == rmin && oamin < amin)) { rmin = o.y; amin = oamin; }
     }
   }
 
   // ------------------------------------------------------ main sweep
-  float z[8];
+  float2 z[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) z[i] = 0.0f;
+  for (int i = 0; i < 4; ++i) z[i] = make_float2(0.0f, 0.0f);
   float hi = 0.0f, lo = 0.0f;
-  float m_used = -INFINITY, m_run = -INFINITY;      // exact map, raw units
   MapRow mr;
   mr.a = mr.b = 0.0f;
   mr.cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
@@ -368,11 +521,16 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   mr.Km1 = static_cast<float>(p.K - 1);
   mr.tab = 0;
   mr.pow_bias = __float_as_uint(p.pscale);
+  mr.flush_t = kMagic + static_cast<float>(p.pot_floor);
+  const bool pot_flush = MAP == MAP_POT && p.flush;
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush &&
                            p.fixed_window;
-  if (kTwoPass && ok) {
+  const float mL2E = rmax * p.cL2E;                 // exact map: the anchor in log2 units
+  if (ok) {
     hi = __fmul_rn(p.c, rmax);
     lo = __fmul_rn(p.c, rmin);
+  }
+  if (MAP != MAP_EXACT && ok) {
     RowMap rm = make_rowmap(hi, lo, p.K, p.fixed_window != 0, p.window);
     if (MAP == MAP_POT) {
       mr.a = -p.cL2E;
@@ -386,133 +544,70 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
       }
       lo = rm.lo;
       const uint32_t tb = smem_u32(tab);
-      // the two halves build alternate entries of this row's grid table
+      // the four groups build interleaved entries of this row's grid table
       if (MAP == MAP_KI_HARD) {
-        for (int n = h; n <= p.K; n += 2) tab[n * 128 + row] = grid_value(rm, p.K, n) * p.pscale;
+        for (int nn = g; nn <= p.K; nn += kGroups)
+          tab[nn * 128 + row] = grid_value(rm, p.K, nn) * p.pscale;
         mr.tab = tb + row * 4 - kMagicBits * 512u;
       } else {
         // entries k = 0 .. K: (c_k, d_k) with d_k = g_{k+1} - g_k and
         // c_k = g_k - k d_k; entry K repeats entry K - 1
-        for (int n = h; n <= p.K; n += 2) {
-          const int k = n < p.K ? n : p.K - 1;
+        for (int nn = g; nn <= p.K; nn += kGroups) {
+          const int k = nn < p.K ? nn : p.K - 1;
           const float gk = grid_value(rm, p.K, k);
           const float gk1 = grid_value(rm, p.K, k + 1);
           const float d = __fsub_rn(gk1, gk) * p.pscale;
-          tab[(n * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, gk * p.pscale);
-          tab[(n * 128 + row) * 2 + 1] = d;
+          tab[(nn * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, gk * p.pscale);
+          tab[(nn * 128 + row) * 2 + 1] = d;
         }
         // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
         mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
       }
-      // the table is complete before either half reads it
-      mbar_arrive(&bars.xstat[t]);
-      ok = warp_all(mbar_wait(&bars.xstat[t], 1, abort));
+      // the table is complete before any group reads it
+      mbar_arrive(bars.xstat);
+      ok = warp_all(mbar_wait(bars.xstat, 1, abort));
     }
   }
   int8_t *dbg_row = (p.dbg != nullptr && row_ok)
                         ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
                         : nullptr;
-  const uint32_t pbase = lane_base + t * 128 + c_off;       // P columns of this half
 
-  for (int j = 0; j < n_t && ok; ++j) {
-    ok = warp_all(mbar_wait(&bars.s_full[t * 2 + 0], sf_cnt0 & 1, abort));
-    ++sf_cnt0;
+  for (int j = pair; j < n && ok; j += 2) {
+    const int b = j % kSBufs;                        // S / P buffer of tile j
+    ok = warp_all(mbar_wait(&bars.s_full[b], (j / kSBufs) & 1, abort));
     if (!ok) break;
     tc_fence_after();
     const int lim = L - 128 * j - c_off;
     const bool full = full_tile(p, qi, j);
-    const uint32_t sbase = lane_base + t * 128 + c_off;
-    if (MAP == MAP_EXACT) {
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = -INFINITY;
+    const uint32_t sb = lane_base + b * 128 + c_off;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(sbase + 32 * c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          mx[i & 7] = fmaxf(mx[i & 7], (full || 32 * c + i < lim) ? __uint_as_float(v[i]) : -INFINITY);
-      }
-      float mt = mx[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i) mt = fmaxf(mt, mx[i]);
-      // the tile maximum of the whole row
-      float *slot = xc.tilemax + ((t * 2 + (j & 1)) * 2) * 128;
-      slot[h * 128 + row] = mt;
-      mbar_arrive(&bars.xtile[t]);
-      ok = warp_all(mbar_wait(&bars.xtile[t], j & 1, abort));
-      if (!ok) break;
-      mt = fmaxf(mt, slot[(h ^ 1) * 128 + row]);
-      m_run = fmaxf(m_run, mt);
-      // move this row's anchor on its first tile, or when the running max grew
-      // by more than 2^8 in weight; O is rescaled in TMEM when any row of the
-      // warp moved (rows that did not move use alpha = 1).  Both halves take
-      // the same decisions (same rows, same combined maxima).
-      const bool first = m_used == -INFINITY;
-      const bool move = first || (m_run - m_used) * p.cL2E > kRescaleLog2;
-      const float alpha = (move && !first) ? ex2_approx((m_used - m_run) * p.cL2E) : 1.0f;
-      if (move) m_used = m_run;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) z[i] *= alpha;
-      if (j > 0 && warp_any(move)) {
-        const uint32_t obase = lane_base + 256 + t * 128 + h * (D / 2);
-#pragma unroll 1
-        for (int dc = 0; dc < D / 64; ++dc) {
-          uint32_t v[32];
-          tmem_ld32_sync(obase + 32 * dc, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-          tmem_st32(obase + 32 * dc, v);
-        }
-      }
-      const float mb = m_used * p.cL2E;
-      auto ex = [&](const uint32_t(&cur)[32], int c0, uint32_t taddr) {
-        auto e = [&](int i) {
-          const float w = ex2_approx(__fmaf_rn(__uint_as_float(cur[i]), p.cL2E, -mb));
-          const float wi = (full || c0 + i < lim) ? w : 0.0f;
-          z[i & 7] += wi;
-          return wi;
-        };
-        if (FP8) {
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float a = e(4 * i), b = e(4 * i + 1), c = e(4 * i + 2), d = e(4 * i + 3);
-            pk[i] = pack_e4m3x4(a, b, c, d);
-          }
-          tmem_st8(taddr, pk);
-        } else {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a = e(2 * i), b = e(2 * i + 1);
-            pk[i] = pack_bf16x2(a, b);
-          }
-          tmem_st16(taddr, pk);
-        }
-      };
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(sbase + 32 * c, v);
-        ex(v, 32 * c, pbase + c * PCOLS);
-      }
-      if (dbg_row != nullptr) {
-        for (int i = 0; i < 64; ++i) {
-          const int kv = 128 * j + c_off + i;
-          if (kv < p.S) dbg_row[kv] = (i < lim) ? 0 : -1;
-        }
-      }
-    } else {
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(sbase + 32 * c, v);
+    for (int c = 0; c < 2; ++c) {
+      uint32_t v[32];
+      tmem_ld32_sync(sb + 32 * c, v);
+      // P of chunk c lands in columns this group has already read
+      const uint32_t pc = sb + c * PCOLS;
+      if (MAP == MAP_EXACT) {
         if (full)
-          map_chunk<MAP, true, FP8>(v, mr, 32 * c, lim, flush_below, z, pbase + c * PCOLS);
+          exp_chunk<true, FP8>(v, p.cL2E, mL2E, 32 * c, lim, z, pc);
         else
-          map_chunk<MAP, false, FP8>(v, mr, 32 * c, lim, flush_below, z, pbase + c * PCOLS);
+          exp_chunk<false, FP8>(v, p.cL2E, mL2E, 32 * c, lim, z, pc);
+        if (dbg_row != nullptr) {
+          for (int i = 0; i < 32; ++i) {
+            const int kv = 128 * j + c_off + 32 * c + i;
+            if (kv < p.S) dbg_row[kv] = (32 * c + i < lim) ? 0 : -1;
+          }
+        }
+      } else {
+        if (pot_flush) {
+          if (full)
+            map_chunk<MAP, true, FP8, true>(v, mr, 32 * c, lim, false, z, pc);
+          else
+            map_chunk<MAP, false, FP8, true>(v, mr, 32 * c, lim, false, z, pc);
+        } else if (full) {
+          map_chunk<MAP, true, FP8, false>(v, mr, 32 * c, lim, flush_below, z, pc);
+        } else {
+          map_chunk<MAP, false, FP8, false>(v, mr, 32 * c, lim, flush_below, z, pc);
+        }
         if (p.dbg != nullptr)
           debug_chunk<MAP>(dbg_row, v, mr, 128 * j + c_off + 32 * c, 32 * c, lim, p,
                            flush_below);
@@ -520,48 +615,28 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
     }
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&bars.p_full[t]);
+    mbar_arrive(&bars.p_full[b]);
   }
 
   // ---------------------------------------------------------- epilogue
-  if (ok) ok = warp_all(mbar_wait(&bars.o_full[t], 0, abort));
+  if (ok) ok = warp_all(mbar_wait(bars.o_full, 0, abort));
   if (!ok) return;
   tc_fence_after();
-  float Z = ((z[0] + z[1]) + (z[2] + z[3])) + ((z[4] + z[5]) + (z[6] + z[7]));
-  xc.zsum[(t * 2 + h) * 128 + row] = Z;
-  mbar_arrive(&bars.xz[t]);
-  if (!warp_all(mbar_wait(&bars.xz[t], 0, abort))) return;
-  Z += xc.zsum[(t * 2 + (h ^ 1)) * 128 + row];
-  if (MAP == MAP_EXACT) hi = p.c * m_run;
+  const float Zg = ((z[0].x + z[0].y) + (z[1].x + z[1].y)) + ((z[2].x + z[2].y) + (z[3].x + z[3].y));
+  xc.zsum[g * 128 + row] = Zg;
+  mbar_arrive(bars.xz);
+  if (!warp_all(mbar_wait(bars.xz, 0, abort))) return;
+  const float Z = (xc.zsum[row] + xc.zsum[128 + row]) + (xc.zsum[256 + row] + xc.zsum[384 + row]);
   const float oscale = p.v_descale / Z;          // pscale cancels: P and Z both carry it
-  const uint32_t obase = lane_base + 256 + t * 128 + h * (D / 2);
-  __nv_bfloat16 *orow = p.O + (static_cast<size_t>(bh) * p.S + qrow) * D + h * (D / 2);
-#pragma unroll 1
-  for (int dc = 0; dc < D / 64; ++dc) {
-    uint32_t v[32];
-    tmem_ld32_sync(obase + 32 * dc, v);
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * oscale,
-                          __uint_as_float(v[2 * i + 1]) * oscale);
-    if (row_ok) {
-      uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * dc);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-    }
-  }
-  if (row_ok && h == 0) {
+  o_store<OC>(lane_base + kOCol + g * OC, oscale,
+              p.O + (static_cast<size_t>(bh) * p.S + qrow) * D + g * OC, row_ok);
+  if (row_ok && g == 0) {
     const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
-    const float anchor = (MAP == MAP_EXACT) ? p.c * m_used : hi;
-    p.LSE[ri] = anchor + logf(Z / p.pscale);
+    p.LSE[ri] = hi + logf(Z / p.pscale);
     if (p.hi) p.hi[ri] = hi;
-    if (MAP != MAP_EXACT) {          // the exact map runs no statistics sweep
-      if (p.lo) p.lo[ri] = lo;
-      if (p.amax) p.amax[ri] = amax;
-      if (p.amin) p.amin[ri] = amin;
-    }
+    if (p.lo) p.lo[ri] = lo;
+    if (p.amax) p.amax[ri] = amax;
+    if (p.amin) p.amin[ri] = amin;
   }
 }
 
@@ -575,41 +650,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Work order: non-causal CTAs sweep one head's query blocks after another
+  // Work order: non-causal CTAs sweep one head's query tiles after another
   // (the running CTAs share few heads' K/V in L2); causal CTAs go heaviest
   // first over all heads (longest-processing-time order, so the lightest
-  // blocks form the tail).
-  int bh, qb;
+  // tiles form the tail).
+  int bh, qi;
   if (p.causal) {
     const int rank = static_cast<int>(blockIdx.x) / p.BH;
     bh = static_cast<int>(blockIdx.x) - rank * p.BH;
-    qb = p.nqb - 1 - rank;
+    qi = p.nqt - 1 - rank;
   } else {
-    qb = static_cast<int>(blockIdx.x) % p.nqb;
-    bh = static_cast<int>(blockIdx.x) / p.nqb;
+    qi = static_cast<int>(blockIdx.x) % p.nqt;
+    bh = static_cast<int>(blockIdx.x) / p.nqt;
   }
   const int ns = p.num_stages;
 
-  uint8_t *sQ = smem;                                   // 2 tiles
-  uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages
+  uint8_t *sQ = smem;                                   // the query tile
+  uint8_t *sKV = smem + G::TILE_BYTES;                  // ns stages
   float *sTab = reinterpret_cast<float *>(smem + p.table_off);
   Bars bars = carve_bars(smem + p.bar_off, ns);
   Xch xc;
   xc.stats = reinterpret_cast<float4 *>(smem + p.xch_off);
-  xc.tilemax = reinterpret_cast<float *>(smem + p.xch_off + 4 * 128 * 16);
-  xc.zsum = xc.tilemax + 8 * 128;
+  xc.zsum = reinterpret_cast<float *>(smem + p.xch_off + kGroups * 128 * 16);
   volatile int *abort = bars.abort;
 
   const int nkvt = (p.S + 127) / 128;
-  // per query tile: index and number of key tiles (scalars, so the control
-  // loops never index a local array)
-  const int qi0 = 2 * qb, qi1 = 2 * qb + 1;
-  const int nt0 = p.causal ? min(nkvt, qi0 + 1) : nkvt;
-  const int nt1 = qi1 < p.nqt ? (p.causal ? min(nkvt, qi1 + 1) : nkvt) : 0;
-  auto NT = [&](int t) { return t ? nt1 : nt0; };
-  auto QI = [&](int t) { return t ? qi1 : qi0; };
-  const int nkv = max(nt0, nt1);
-  constexpr bool kTwoPass = MAP != MAP_EXACT;
+  const int n = p.causal ? min(nkvt, qi + 1) : nkvt;    // key tiles of this query tile
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
@@ -617,18 +683,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.kv_empty[i], 1);
     }
     mbar_init(bars.q_full, 1);
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kStatBufs; ++i) {
+      mbar_init(&bars.st_full[i], 1);
+      mbar_init(&bars.st_empty[i], kPairThreads);
+    }
+    for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_empty[i], 256);
+      mbar_init(&bars.p_full[i], kPairThreads);
+      mbar_init(&bars.s_free[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.p_full[i], 256);
-      mbar_init(&bars.o_full[i], 1);
-      mbar_init(&bars.xstat[i], 256);
-      mbar_init(&bars.xtile[i], 256);
-      mbar_init(&bars.xz[i], 256);
-    }
-    mbar_init(bars.drain, 1);
+    mbar_init(bars.o_full, 1);
+    mbar_init(bars.drain, kStatIssuers);       // one commit per issuer
+    mbar_init(bars.xstat, kMapThreads);
+    mbar_init(bars.xz, kMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
   }
@@ -638,29 +705,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
-  // The CTA launches with kThreads x kLaunchRegs registers; the control warp
-  // group (producer, MMA issuer, two idle warps) gives most of its share to
-  // the four map groups: 128 x kCtrlRegs + 512 x kMapRegs <= 640 x kLaunchRegs
-  // (an increase beyond what the decrease freed would wait forever).
-  constexpr int kCtrlRegs = RegSplit<MAP>::ctrl;
-  constexpr int kMapRegs = RegSplit<MAP>::map;
-  static_assert(128 * kCtrlRegs + 512 * kMapRegs <= kThreads * kLaunchRegs,
-                "register split must equal the launch allocation");
-  if (warp < 4) {
-    if (kCtrlRegs < kLaunchRegs) regs_dec<kCtrlRegs>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // ring positions: statistics sweep K_0 .. K_{n-1}, then the main sweep in
+    // the order of ring_pos_k / ring_pos_v
     if (lane == 0 && !(p.debug_flags & 1)) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const int nq = (nt0 > 0) + (nt1 > 0);
-      mbar_expect_tx(bars.q_full, nq * G::TILE_BYTES);
-      for (int t = 0; t < 2; ++t)
-        if (NT(t) > 0)
-          for (int ch = 0; ch < G::CHUNKS; ++ch)
-            tma_load_3d(sQ + t * G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmQ, bars.q_full,
-                        ch * G::EPC, QI(t) * 128, bh);
+      mbar_expect_tx(bars.q_full, G::TILE_BYTES);
+      for (int ch = 0; ch < G::CHUNKS; ++ch)
+        tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qi * 128, bh);
       int it = 0, st = 0;
       uint32_t ph = 0;                  // completed passes over the ring
       bool ok = true;
@@ -677,11 +732,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           ph ^= 1;
         }
       };
-      if (kTwoPass)
-        for (int j = 0; j < nkv && ok; ++j) load(&tmK, j);
-      for (int j = 0; j < nkv && ok; ++j) {
-        load(&tmK, j);
+      for (int j = 0; j < n && ok; ++j) load(&tmK, j);
+      for (int j = 0; j < kLead && j < n && ok; ++j) load(&tmK, j);
+      for (int j = 0; j < n && ok; ++j) {
         load(&tmV, j);
+        if (j + kLead < n) load(&tmK, j + kLead);
       }
       // let every load issued so far land before the CTA may exit
       mbar_wait(bars.q_full, 0, abort);
@@ -690,128 +745,130 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&bars.kv_full[s], (fills - 1) & 1, abort);
       }
     }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------------- MMA
+  } else if (warp <= kStatIssuers) {
+    // ---------------------------------------------------------------- MMA
+    // Warp 1 issues S = Q K^T, warp 2 issues O += P V (main sweep); in the
+    // statistics sweep they take alternate key tiles.  Each ring position is
+    // consumed, and released by an MMA commit, by exactly one of them.
     if (lane == 0) {
-      const uint32_t qaddr0 = smem_u32(sQ);
+      const bool qk_role = warp == 1;
+      const bool pv_role = warp == 2;
+      const uint32_t qaddr = smem_u32(sQ);
       const uint32_t kvaddr0 = smem_u32(sKV);
-      int cst = 0;                      // next ring stage to consume
-      uint32_t cph = 0;                 // its phase parity
+      int pos = 0, pst = 0;             // ring position, its stage
+      uint32_t pph = 0;                 // and the parity of its fill
       bool ok = mbar_wait(bars.q_full, 0, abort);
       tc_fence_after();
-      auto acquire = [&]() -> int {
-        const int st = cst;
-        ok = ok && mbar_wait(&bars.kv_full[st], cph, abort);
-        if (++cst == ns) {
-          cst = 0;
-          cph ^= 1;
+      auto acquire = [&](int target) -> int {
+        while (pos < target) {
+          ++pos;
+          if (++pst == ns) {
+            pst = 0;
+            pph ^= 1;
+          }
         }
+        ok = ok && mbar_wait(&bars.kv_full[pst], pph, abort);
         tc_fence_after();
-        return st;
+        return pst;
       };
-      auto issue_qk = [&](int t, int st, uint32_t scol) {
-        const uint32_t qa = qaddr0 + t * G::TILE_BYTES;
+      auto issue_qk = [&](int st, uint32_t col) {
         const uint32_t ka = kvaddr0 + st * G::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < G::KSTEPS_QK; ++kk) {
           const int e = kk * G::MMA_K;
           const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * G::ELEM;
-          const uint64_t ad = smem_desc(qa + off, 16, 1024);
+          const uint64_t ad = smem_desc(qaddr + off, 16, 1024);
           const uint64_t bd = smem_desc(ka + off, 16, 1024);
           if (FP8)
-            mma_ss_f8(tmem + scol, ad, bd, G::IDESC_QK, kk > 0);
+            mma_ss_f8(tmem + col, ad, bd, G::IDESC_QK, kk > 0);
           else
-            mma_ss_f16(tmem + scol, ad, bd, G::IDESC_QK, kk > 0);
+            mma_ss_f16(tmem + col, ad, bd, G::IDESC_QK, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
+      auto issue_pv = [&](int st, uint32_t pcol, bool acc) {
         const uint32_t va = kvaddr0 + st * G::TILE_BYTES;
-        const uint32_t pcol = t * 128;
-        const uint32_t ocol = 256 + t * 128;
 #pragma unroll
         for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
           const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
-          // keys 64h.. of the tile sit at TMEM columns 64h.. (each map half
-          // writes its P into its own S columns), 8 columns per k-step
+          // keys 64h .. 64h+63 of the tile sit, packed, from TMEM column 64h
+          // (the map group owning that half writes its P into the first of
+          // its own S columns): 8 columns per k-step
           const int key0 = kk * G::MMA_K;
-          const uint32_t at = tmem + pcol + 64 * (key0 / 64) + ((key0 % 64) / G::MMA_K) * 8;
+          const uint32_t at = tmem + pcol + kHalfCols * (key0 / kHalfCols) +
+                              ((key0 % kHalfCols) / G::MMA_K) * 8;
           if (FP8)
-            mma_ts_f8(tmem + ocol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            mma_ts_f8(tmem + kOCol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
           else
-            mma_ts_f16(tmem + ocol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            mma_ts_f16(tmem + kOCol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
       };
 
-      if (kTwoPass) {
-        for (int j = 0; j < nkv && ok; ++j) {
-          const int st = acquire();
+      {
+        // key tile j: issuer warp 1 + j % 2, S buffer j % 4
+        for (int j = warp - 1; j < n && ok; j += kStatIssuers) {
+          const int st = acquire(j);
           if (!ok) break;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (j >= NT(t)) continue;
-            const int b = j & 1, use = j >> 1;
-            if (use >= 1) {
-              ok = mbar_wait(&bars.s_empty[t * 2 + b], (use - 1) & 1, abort);
-              tc_fence_after();
-              if (!ok) break;
-            }
-            issue_qk(t, st, t * 128 + b * 256);
-            mma_commit(&bars.s_full[t * 2 + b]);
+          const int b = j & 3, u = j >> 2;
+          if (u >= 1) {
+            ok = mbar_wait(&bars.st_empty[b], (u - 1) & 1, abort);
+            tc_fence_after();
+            if (!ok) break;
           }
+          issue_qk(st, b * 128);
+          mma_commit(&bars.st_full[b]);
           mma_commit(&bars.kv_empty[st]);
         }
-        // both S buffers of each tile must be read out before the main sweep
-        for (int t = 0; t < 2 && ok; ++t) {
-          const int u0 = (NT(t) + 1) / 2, u1 = NT(t) / 2;
-          if (u0 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 0], (u0 - 1) & 1, abort);
-          if (u1 >= 1) ok = ok && mbar_wait(&bars.s_empty[t * 2 + 1], (u1 - 1) & 1, abort);
-        }
-        tc_fence_after();
-      }
-      if (ok && nkv > 0) {
-        const int k0 = acquire();
-        if (ok) {
-          for (int t = 0; t < 2; ++t)
-            if (NT(t) > 0) {
-              issue_qk(t, k0, t * 128);
-              mma_commit(&bars.s_full[t * 2 + 0]);
-            }
-          mma_commit(&bars.kv_empty[k0]);
-        }
-        for (int j = 0; j < nkv && ok; ++j) {
-          const int vst = acquire();
-          const bool has_next = j + 1 < nkv;
-          const int knext = has_next ? acquire() : -1;
-          if (!ok) break;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (j < NT(t)) {
-              ok = mbar_wait(&bars.p_full[t], j & 1, abort);
-              tc_fence_after();
-              if (!ok) break;
-              issue_pv(t, vst, j > 0);
-            }
-            if (has_next && j + 1 < NT(t)) {
-              issue_qk(t, knext, t * 128);
-              mma_commit(&bars.s_full[t * 2 + 0]);
-            }
+        // the main sweep writes S into buffers 0-2 (QK issuer) and O into
+        // buffer 3 (PV issuer): wait until their last statistics tile is read
+        if (qk_role || pv_role) {
+          for (int b = qk_role ? 0 : 3; b < (qk_role ? 3 : 4); ++b) {
+            const int uses = n > b ? (n - b + 3) / 4 : 0;
+            if (uses >= 1) ok = ok && mbar_wait(&bars.st_empty[b], (uses - 1) & 1, abort);
           }
-          mma_commit(&bars.kv_empty[vst]);
-          if (has_next) mma_commit(&bars.kv_empty[knext]);
+          tc_fence_after();
         }
-        for (int t = 0; t < 2; ++t)
-          if (NT(t) > 0) mma_commit(&bars.o_full[t]);
+      }
+      const int base = n;                              // first main-sweep position
+      int b = 0;
+      uint32_t ph = 0;                                 // buffer j % 3, parity of its use
+      if (qk_role) {
+        for (int j = 0; j < n && ok; ++j) {
+          const int st = acquire(base + ring_pos_k(j));
+          if (!ok) break;
+          if (j >= kSBufs) {
+            // tile j-3's P has gone through its PV product
+            ok = mbar_wait(&bars.s_free[b], ph ^ 1, abort);
+            tc_fence_after();
+            if (!ok) break;
+          }
+          issue_qk(st, b * 128);
+          mma_commit(&bars.s_full[b]);
+          mma_commit(&bars.kv_empty[st]);
+          if (++b == kSBufs) { b = 0; ph ^= 1; }
+        }
+      } else if (pv_role) {
+        for (int j = 0; j < n && ok; ++j) {
+          const int st = acquire(base + ring_pos_v(j, n));
+          if (!ok) break;
+          ok = mbar_wait(&bars.p_full[b], ph, abort);
+          tc_fence_after();
+          if (!ok) break;
+          issue_pv(st, b * 128, j > 0);
+          mma_commit(&bars.s_free[b]);
+          mma_commit(&bars.kv_empty[st]);
+          if (++b == kSBufs) { b = 0; ph ^= 1; }
+        }
+        if (ok) mma_commit(bars.o_full);
       }
       // every MMA issued must finish before TMEM is released
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
     }
-  }
-  } else {
-    if (kMapRegs > kLaunchRegs) regs_inc<kMapRegs>();
+  } else if (warp >= 4) {
     const int g = (warp - 4) >> 2;                 // map group 0..3
-    const int t = g >> 1, h = g & 1;               // query tile, key-column half
-    map_half<D, FP8, MAP>(p, bars, t, h, threadIdx.x - 128 - g * 128,
-                          tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), QI(t), NT(t),
-                          bh, sTab + t * p.tab_stride, xc, abort);
+    map_half<D, FP8, MAP>(p, bars, g, threadIdx.x - 128 - g * 128,
+                           tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh,
+                           sTab, xc, abort);
   }
 
   __syncwarp();
@@ -831,7 +888,6 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   FwdParams p{};
   p.S = a.S;
   p.nqt = (a.S + 127) / 128;
-  p.nqb = (p.nqt + 1) / 2;
   p.BH = a.B * a.H;
   p.causal = a.causal;
   p.K = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) ? a.Kint : 1;
@@ -853,34 +909,30 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.status = a.status_dev;
   p.debug_flags = a.debug_flags;
 
-  // grid table per query tile: [K+1][128] values (hard) or [K+1][128]
-  // (c_k, d_k) pairs (interpolation)
+  // grid table: [K+1][128] values (hard) or [K+1][128] (c_k, d_k) pairs
+  // (interpolation)
   p.tab_stride = (MAP == MAP_KI_INTERP) ? (p.K + 1) * 128 * 2 : (p.K + 1) * 128;
-  const size_t table_bytes = static_cast<size_t>(2) * p.tab_stride * sizeof(float);
-  // Bars: 2 per ring stage + 20 fixed mbarriers, then tmem_slot and abort;
-  // sized for the deepest ring allowed below
-  constexpr int kMaxStages = 8;
-  const size_t bar_bytes = ((2 * kMaxStages + 20) * 8 + 8 + 15) & ~static_cast<size_t>(15);
+  const size_t table_bytes = static_cast<size_t>(p.tab_stride) * sizeof(float);
+  const size_t bar_bytes = bar_bytes_for(kMaxStages);
   const size_t max_smem = 232448;                        // 227 KB opt-in per CTA
-  const size_t fixed = 1024 + 2 * G::TILE_BYTES + table_bytes + bar_bytes +
-                       (4 * 128 * 16 + 8 * 128 * 4 + 4 * 128 * 4);
+  const size_t fixed = 1024 + G::TILE_BYTES + table_bytes + 16 + bar_bytes + kXchBytes;
   int ns = static_cast<int>((max_smem - fixed) / G::TILE_BYTES);
   if (ns > kMaxStages) ns = kMaxStages;
   if (ns < 2) return QSM_ERR_UNSUPPORTED;
   p.num_stages = ns;
-  p.table_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * G::TILE_BYTES);
+  p.table_off = static_cast<uint32_t>(G::TILE_BYTES + ns * G::TILE_BYTES);
   p.bar_off = static_cast<uint32_t>((p.table_off + table_bytes + 15) & ~static_cast<size_t>(15));
   p.xch_off = p.bar_off + static_cast<uint32_t>(bar_bytes);
-  const size_t xch_bytes = 4 * 128 * 16 + 8 * 128 * 4 + 4 * 128 * 4;
-  size_t smem = 1024 + p.xch_off + xch_bytes;
+  size_t smem = 1024 + p.xch_off + kXchBytes;
   // one CTA per SM: the kernel allocates all 512 TMEM columns
   if (smem < 120 * 1024) smem = 120 * 1024;
+  if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
   auto kern = qsm_fwd_kernel<D, FP8, MAP>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return QSM_ERR_CUDA;
-  dim3 grid(p.nqb * a.B * a.H);
+  dim3 grid(p.nqt * a.B * a.H);
   kern<<<grid, kThreads, smem, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
