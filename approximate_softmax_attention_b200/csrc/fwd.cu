@@ -649,7 +649,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
   // Work order: non-causal CTAs sweep one head's query tiles after another
   // (the running CTAs share few heads' K/V in L2); causal CTAs go heaviest
   // first over all heads (longest-processing-time order, so the lightest
@@ -709,23 +708,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     // ring positions: statistics sweep K_0 .. K_{n-1}, then the main sweep in
     // the order of ring_pos_k / ring_pos_v
-    if (lane == 0 && !(p.debug_flags & 1)) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
-      mbar_expect_tx(bars.q_full, G::TILE_BYTES);
-      for (int ch = 0; ch < G::CHUNKS; ++ch)
-        tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qi * 128, bh);
+    if (!(p.debug_flags & 1)) {
+      const bool leader = elect_one();
+      if (leader) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+        mbar_expect_tx(bars.q_full, G::TILE_BYTES);
+        for (int ch = 0; ch < G::CHUNKS; ++ch)
+          tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qi * 128, bh);
+      }
+      __syncwarp();
       int it = 0, st = 0;
       uint32_t ph = 0;                  // completed passes over the ring
       bool ok = true;
       auto load = [&](const CUtensorMap *m, int kvt) {
-        if (it >= ns) ok = ok && mbar_wait(&bars.kv_empty[st], ph ^ 1, abort);
+        if (it >= ns) ok = ok && warp_all(mbar_wait(&bars.kv_empty[st], ph ^ 1, abort));
         if (!ok) return;
-        mbar_expect_tx(&bars.kv_full[st], G::TILE_BYTES);
-        for (int ch = 0; ch < G::CHUNKS; ++ch)
-          tma_load_3d(sKV + st * G::TILE_BYTES + ch * G::CHUNK_BYTES, m, &bars.kv_full[st],
-                      ch * G::EPC, kvt * 128, bh);
+        if (leader) {
+          mbar_expect_tx(&bars.kv_full[st], G::TILE_BYTES);
+          for (int ch = 0; ch < G::CHUNKS; ++ch)
+            tma_load_3d(sKV + st * G::TILE_BYTES + ch * G::CHUNK_BYTES, m, &bars.kv_full[st],
+                        ch * G::EPC, kvt * 128, bh);
+        }
+        __syncwarp();
         ++it;
         if (++st == ns) {
           st = 0;
@@ -749,121 +755,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- MMA
     // Warp 1 issues S = Q K^T, warp 2 issues O += P V (main sweep); in the
     // statistics sweep they take alternate key tiles.  Each ring position is
-    // consumed, and released by an MMA commit, by exactly one of them.
-    if (lane == 0) {
-      const bool qk_role = warp == 1;
-      const bool pv_role = warp == 2;
-      const uint32_t qaddr = smem_u32(sQ);
-      const uint32_t kvaddr0 = smem_u32(sKV);
-      int pos = 0, pst = 0;             // ring position, its stage
-      uint32_t pph = 0;                 // and the parity of its fill
-      bool ok = mbar_wait(bars.q_full, 0, abort);
-      tc_fence_after();
-      auto acquire = [&](int target) -> int {
-        while (pos < target) {
-          ++pos;
-          if (++pst == ns) {
-            pst = 0;
-            pph ^= 1;
-          }
+    // consumed, and released by an MMA commit, by exactly one of them.  The
+    // whole warp runs the loop; the elected lane issues every MMA and every
+    // commit (a commit tracks the MMAs of the thread that issues it).
+    const bool leader = elect_one();
+    const bool qk_role = warp == 1;
+    const bool pv_role = warp == 2;
+    const uint32_t qaddr = smem_u32(sQ);
+    const uint32_t kvaddr0 = smem_u32(sKV);
+    int pos = 0, pst = 0;               // ring position, its stage
+    uint32_t pph = 0;                   // and the parity of its fill
+    bool ok = warp_all(mbar_wait(bars.q_full, 0, abort));
+    tc_fence_after();
+    auto acquire = [&](int target) -> int {
+      while (pos < target) {
+        ++pos;
+        if (++pst == ns) {
+          pst = 0;
+          pph ^= 1;
         }
-        ok = ok && mbar_wait(&bars.kv_full[pst], pph, abort);
-        tc_fence_after();
-        return pst;
-      };
-      auto issue_qk = [&](int st, uint32_t col) {
-        const uint32_t ka = kvaddr0 + st * G::TILE_BYTES;
+      }
+      ok = ok && warp_all(mbar_wait(&bars.kv_full[pst], pph, abort));
+      tc_fence_after();
+      return pst;
+    };
+    auto commit = [&](uint64_t *bar) {
+      if (leader) mma_commit(bar);
+      __syncwarp();
+    };
+    auto issue_qk = [&](int st, uint32_t col) {
+      const uint32_t ka = kvaddr0 + st * G::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < G::KSTEPS_QK; ++kk) {
-          const int e = kk * G::MMA_K;
-          const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * G::ELEM;
-          const uint64_t ad = smem_desc(qaddr + off, 16, 1024);
-          const uint64_t bd = smem_desc(ka + off, 16, 1024);
+      for (int kk = 0; kk < G::KSTEPS_QK; ++kk) {
+        const int e = kk * G::MMA_K;
+        const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * G::ELEM;
+        const uint64_t ad = smem_desc(qaddr + off, 16, 1024);
+        const uint64_t bd = smem_desc(ka + off, 16, 1024);
+        if (leader) {
           if (FP8)
             mma_ss_f8(tmem + col, ad, bd, G::IDESC_QK, kk > 0);
           else
             mma_ss_f16(tmem + col, ad, bd, G::IDESC_QK, kk > 0);
         }
-      };
-      auto issue_pv = [&](int st, uint32_t pcol, bool acc) {
-        const uint32_t va = kvaddr0 + st * G::TILE_BYTES;
+      }
+      __syncwarp();
+    };
+    auto issue_pv = [&](int st, uint32_t pcol, bool acc) {
+      const uint32_t va = kvaddr0 + st * G::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
-          const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
-          // keys 64h .. 64h+63 of the tile sit, packed, from TMEM column 64h
-          // (the map group owning that half writes its P into the first of
-          // its own S columns): 8 columns per k-step
-          const int key0 = kk * G::MMA_K;
-          const uint32_t at = tmem + pcol + kHalfCols * (key0 / kHalfCols) +
-                              ((key0 % kHalfCols) / G::MMA_K) * 8;
+      for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
+        const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
+        // keys 64h .. 64h+63 of the tile sit, packed, from TMEM column 64h
+        // (the map group owning that half writes its P into the first of
+        // its own S columns): 8 columns per k-step
+        const int key0 = kk * G::MMA_K;
+        const uint32_t at = tmem + pcol + kHalfCols * (key0 / kHalfCols) +
+                            ((key0 % kHalfCols) / G::MMA_K) * 8;
+        if (leader) {
           if (FP8)
             mma_ts_f8(tmem + kOCol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
           else
             mma_ts_f16(tmem + kOCol, at, bd, G::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
-      };
+      }
+      __syncwarp();
+    };
 
-      {
-        // key tile j: issuer warp 1 + j % 2, S buffer j % 4
-        for (int j = warp - 1; j < n && ok; j += kStatIssuers) {
-          const int st = acquire(j);
-          if (!ok) break;
-          const int b = j & 3, u = j >> 2;
-          if (u >= 1) {
-            ok = mbar_wait(&bars.st_empty[b], (u - 1) & 1, abort);
-            tc_fence_after();
-            if (!ok) break;
-          }
-          issue_qk(st, b * 128);
-          mma_commit(&bars.st_full[b]);
-          mma_commit(&bars.kv_empty[st]);
-        }
-        // the main sweep writes S into buffers 0-2 (QK issuer) and O into
-        // buffer 3 (PV issuer): wait until their last statistics tile is read
-        if (qk_role || pv_role) {
-          for (int b = qk_role ? 0 : 3; b < (qk_role ? 3 : 4); ++b) {
-            const int uses = n > b ? (n - b + 3) / 4 : 0;
-            if (uses >= 1) ok = ok && mbar_wait(&bars.st_empty[b], (uses - 1) & 1, abort);
-          }
-          tc_fence_after();
-        }
-      }
-      const int base = n;                              // first main-sweep position
-      int b = 0;
-      uint32_t ph = 0;                                 // buffer j % 3, parity of its use
-      if (qk_role) {
-        for (int j = 0; j < n && ok; ++j) {
-          const int st = acquire(base + ring_pos_k(j));
-          if (!ok) break;
-          if (j >= kSBufs) {
-            // tile j-3's P has gone through its PV product
-            ok = mbar_wait(&bars.s_free[b], ph ^ 1, abort);
-            tc_fence_after();
-            if (!ok) break;
-          }
-          issue_qk(st, b * 128);
-          mma_commit(&bars.s_full[b]);
-          mma_commit(&bars.kv_empty[st]);
-          if (++b == kSBufs) { b = 0; ph ^= 1; }
-        }
-      } else if (pv_role) {
-        for (int j = 0; j < n && ok; ++j) {
-          const int st = acquire(base + ring_pos_v(j, n));
-          if (!ok) break;
-          ok = mbar_wait(&bars.p_full[b], ph, abort);
+    {
+      // statistics sweep: key tile j goes to issuer warp 1 + j % 2, S buffer j % 4
+      for (int j = warp - 1; j < n && ok; j += kStatIssuers) {
+        const int st = acquire(j);
+        if (!ok) break;
+        const int b = j & 3, u = j >> 2;
+        if (u >= 1) {
+          ok = warp_all(mbar_wait(&bars.st_empty[b], (u - 1) & 1, abort));
           tc_fence_after();
           if (!ok) break;
-          issue_pv(st, b * 128, j > 0);
-          mma_commit(&bars.s_free[b]);
-          mma_commit(&bars.kv_empty[st]);
-          if (++b == kSBufs) { b = 0; ph ^= 1; }
         }
-        if (ok) mma_commit(bars.o_full);
+        issue_qk(st, b * 128);
+        commit(&bars.st_full[b]);
+        commit(&bars.kv_empty[st]);
       }
-      // every MMA issued must finish before TMEM is released
-      mma_commit(bars.drain);
-      mbar_wait(bars.drain, 0, abort);
+      // the main sweep writes S into buffers 0-2 (QK issuer) and O into
+      // buffer 3 (PV issuer): wait until their last statistics tile is read
+      if (qk_role || pv_role) {
+        for (int b = qk_role ? 0 : 3; b < (qk_role ? 3 : 4); ++b) {
+          const int uses = n > b ? (n - b + 3) / 4 : 0;
+          if (uses >= 1) ok = ok && warp_all(mbar_wait(&bars.st_empty[b], (uses - 1) & 1, abort));
+        }
+        tc_fence_after();
+      }
     }
+    const int base = n;                              // first main-sweep position
+    int b = 0;
+    uint32_t ph = 0;                                 // buffer j % 3, parity of its use
+    if (qk_role) {
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = acquire(base + ring_pos_k(j));
+        if (!ok) break;
+        if (j >= kSBufs) {
+          // tile j-3's P has gone through its PV product
+          ok = warp_all(mbar_wait(&bars.s_free[b], ph ^ 1, abort));
+          tc_fence_after();
+          if (!ok) break;
+        }
+        issue_qk(st, b * 128);
+        commit(&bars.s_full[b]);
+        commit(&bars.kv_empty[st]);
+        if (++b == kSBufs) { b = 0; ph ^= 1; }
+      }
+    } else if (pv_role) {
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = acquire(base + ring_pos_v(j, n));
+        if (!ok) break;
+        ok = warp_all(mbar_wait(&bars.p_full[b], ph, abort));
+        tc_fence_after();
+        if (!ok) break;
+        issue_pv(st, b * 128, j > 0);
+        commit(&bars.s_free[b]);
+        commit(&bars.kv_empty[st]);
+        if (++b == kSBufs) { b = 0; ph ^= 1; }
+      }
+      if (ok) commit(bars.o_full);
+    }
+    // every MMA issued must finish before TMEM is released
+    commit(bars.drain);
+    mbar_wait(bars.drain, 0, abort);
   } else if (warp >= 4) {
     const int g = (warp - 4) >> 2;                 // map group 0..3
     map_half<D, FP8, MAP>(p, bars, g, threadIdx.x - 128 - g * 128,

@@ -46,8 +46,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same test, but a thread whose phase has not completed is suspended
+// until it completes or about hint_ns nanoseconds pass, so waiting warps
+// take no issue slots from the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Cycle budget of one wait: about one second at the B200's clocks.
 constexpr long long kWaitCycles = 2000000000LL;
+// Suspend hint of one test inside a wait (the abort flag and the cycle budget
+// are checked between tests).
+constexpr uint32_t kWaitHintNs = 100000;
 
 // Bounded wait for the phase with the given parity.  Returns false (and
 // raises *abort) when the budget runs out or another thread has already
@@ -57,13 +76,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitHintNs)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitCycles) {
       *abort = 1;
       return false;
     }
   }
+}
+
+// One lane of a converged warp: the control warps run their loops on all 32
+// lanes (warp-uniform state) and let this lane issue the single-thread
+// operations (TMA, tcgen05.mma, tcgen05.commit).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(e));
+  return e != 0;
 }
 
 // --------------------------------------------------------------------- TMA
