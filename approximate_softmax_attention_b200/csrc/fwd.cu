@@ -114,6 +114,7 @@ struct Bars {
   uint64_t *kv_full, *kv_empty;          // [stages]
   uint64_t *q_full;                      // 1
   uint64_t *st_full, *st_empty;          // [kStatBufs] statistics sweep
+  uint64_t *st_done;                     // 1: every map thread finished the statistics sweep
   uint64_t *s_full, *p_full, *s_free;    // [kSBufs] main sweep
   uint64_t *o_full;                      // 1
   uint64_t *drain;                       // 1
@@ -121,7 +122,7 @@ struct Bars {
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr int kFixedBars = 1 + 2 * kStatBufs + 3 * kSBufs + 2 + 2;
+constexpr int kFixedBars = 1 + 2 * kStatBufs + 1 + 3 * kSBufs + 2 + 2;
 
 __host__ __device__ constexpr size_t bar_bytes_for(int ns) {
   return ((2 * static_cast<size_t>(ns) + kFixedBars) * 8 + 8 + 15) & ~static_cast<size_t>(15);
@@ -135,7 +136,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   b.q_full = p + 2 * ns;
   b.st_full = b.q_full + 1;
   b.st_empty = b.st_full + kStatBufs;
-  b.s_full = b.st_empty + kStatBufs;
+  b.st_done = b.st_empty + kStatBufs;
+  b.s_full = b.st_done + 1;
   b.p_full = b.s_full + kSBufs;
   b.s_free = b.p_full + kSBufs;
   b.o_full = b.s_free + kSBufs;
@@ -484,6 +486,10 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
         red(v1, 32, 2);
       }
     }
+    // this thread has read every statistics tile it owns (a single-use
+    // barrier: an issuer must not wait on another issuer's buffers by
+    // parity, whose phases may still be two or more behind)
+    mbar_arrive(bars.st_done);
     if (!want_arg) {
       rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
       rmin = min3f(mn[0], mn[1], fminf(mn[2], mn[3]));
@@ -686,6 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.st_full[i], 1);
       mbar_init(&bars.st_empty[i], kPairThreads);
     }
+    mbar_init(bars.st_done, kMapThreads);
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], kPairThreads);
@@ -837,12 +844,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         commit(&bars.kv_empty[st]);
       }
       // the main sweep writes S into buffers 0-2 (QK issuer) and O into
-      // buffer 3 (PV issuer): wait until their last statistics tile is read
+      // buffer 3 (PV issuer): wait until every statistics tile is read (the
+      // map threads report that once, on a single-use barrier)
       if (qk_role || pv_role) {
-        for (int b = qk_role ? 0 : 3; b < (qk_role ? 3 : 4); ++b) {
-          const int uses = n > b ? (n - b + 3) / 4 : 0;
-          if (uses >= 1) ok = ok && warp_all(mbar_wait(&bars.st_empty[b], (uses - 1) & 1, abort));
-        }
+        ok = ok && warp_all(mbar_wait(bars.st_done, 0, abort));
         tc_fence_after();
       }
     }
