@@ -45,7 +45,11 @@ namespace qsm {
 
 namespace {
 
-constexpr int kBwdThreads = 256;        // warp 0 TMA, warp 1 MMA, warps 4-7 map
+constexpr int kBwdThreads = 256;        // rows kernel: warp 0 TMA, warp 1 MMA, warps 4-7 map
+// main kernel: warp 0 TMA, warp 1 MMA, warps 4-19 four map groups, group g
+// owning query columns 32g .. 32g+31 of every S^T / dP^T tile
+constexpr int kMainThreads = 640;
+constexpr int kMainMapThreads = 512;
 constexpr uint32_t kBwdTmemCols = 512;
 constexpr int kRowWs = 8;               // floats per row in the row workspace
 enum RowWs { RW_DELTA = 0, RW_DHI = 1, RW_DLO = 2, RW_LSESTAR = 3, RW_DELTASTAR = 4 };
@@ -105,6 +109,21 @@ __device__ __forceinline__ void mma_tn(uint32_t d_tmem, uint32_t a_tmem, uint32_
   for (int kk = 0; kk < G::KSTEPS_N; ++kk)
     mma_ts_f16(d_tmem, a_tmem + kk * 8, smem_desc(b_saddr + kk * 16 * 128, G::CHUNK_BYTES, 1024),
                G::IDESC_TS, (acc || kk > 0) ? 1u : 0u);
+}
+
+// acc (+)= A[tmem, 128 x 128, group layout] B[smem, 128 x D, MN-major]: the
+// bf16 values of K-columns 32g .. 32g+31 of A sit in TMEM columns 32g ..
+// 32g+15 (each map group writes its P^T / dS^T into the first half of its own
+// S^T / dP^T columns), 8 TMEM columns per k-step of 16.
+template <int D>
+__device__ __forceinline__ void mma_tn_grouped(uint32_t d_tmem, uint32_t a_tmem,
+                                               uint32_t b_saddr, bool acc) {
+  using G = BGeo<D>;
+#pragma unroll
+  for (int kk = 0; kk < G::KSTEPS_N; ++kk)
+    mma_ts_f16(d_tmem, a_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+               smem_desc(b_saddr + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_TS,
+               (acc || kk > 0) ? 1u : 0u);
 }
 
 // D = A[smem 128 x 128, MN-major] B[smem 128 x D, MN-major]
@@ -449,7 +468,7 @@ struct MainBars {
 constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256;
 
 template <int D, int MAP>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_main(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams p) {
@@ -467,7 +486,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t *sQD = smem + 2 * G::TILE_BYTES;              // [2 stages][Q, dO]
   uint8_t *sDS = smem + p.ds_off;                        // 128 x 128 bf16, MN-major
   float2 *tab = reinterpret_cast<float2 *>(smem + p.tab_off);   // [row][n]
-  float *cst = reinterpret_cast<float *>(smem + p.cst_off);     // [C_NUM][128]
+  float *cst = reinterpret_cast<float *>(smem + p.cst_off);     // [128][8]: C_* per row
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   MainBars bars;
   bars.kv_full = bp;
@@ -493,12 +512,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&bars.qd_empty[i], 1);
     }
     mbar_init(bars.sdp_full, 1);
-    mbar_init(bars.pds_full, 128);
+    mbar_init(bars.pds_full, kMainMapThreads);
     mbar_init(bars.dq_full, 1);
-    mbar_init(bars.dq_empty, 128);
+    mbar_init(bars.dq_empty, kMainMapThreads);
     mbar_init(bars.acc_full, 1);
     mbar_init(bars.drain, 1);
-    mbar_init(bars.cst_ready, 128);
+    mbar_init(bars.cst_ready, kMainMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
   }
@@ -553,8 +572,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = mbar_wait(bars.pds_full, n & 1, abort);
         if (!ok) break;
         tc_fence_after();
-        mma_tn<D>(tmem + T_DV, tmem + T_S, da, n > 0);     // dV += P^T dO
-        mma_tn<D>(tmem + T_DK, tmem + T_DP, qa, n > 0);    // dK += dS^T Q
+        mma_tn_grouped<D>(tmem + T_DV, tmem + T_S, da, n > 0);    // dV += P^T dO
+        mma_tn_grouped<D>(tmem + T_DK, tmem + T_DP, qa, n > 0);   // dK += dS^T Q
         if (n > 0) {
           ok = mbar_wait(bars.dq_empty, (n - 1) & 1, abort);
           if (!ok) break;
@@ -569,48 +588,49 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait(bars.drain, 0, abort);
     }
   } else if (warp >= 4) {
-    const int key = threadIdx.x - 128;                   // 0..127: TMEM lane, key row
+    const int g = (warp - 4) >> 2;                       // map group 0..3
+    const int key = (warp & 3) * 32 + (threadIdx.x & 31);  // TMEM lane, key row
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int kg = kt * 128 + key;
     const bool key_ok = kg < p.S;
     const float Kf = static_cast<float>(p.K);
     const int K1 = p.K + 1;
     const uint32_t ds_base = smem_u32(sDS);
+    const int col0 = 32 * g;                             // this group's query columns
+    const float4 *cst4 = reinterpret_cast<const float4 *>(cst);
     bool ok = true;
     for (int n = 0; n < nq && ok; ++n) {
       const int qt = i0 + n;
-      // ---- per-query-row constants of this tile: thread `key` fills row `key`
+      // ---- per-query-row constants of this tile: thread `key` serves row
+      // `key`; group 0 writes the scalars, the groups split the grid table
       {
         const int qg = qt * 128 + key;
         const size_t ri = static_cast<size_t>(bh) * p.S + min(qg, p.S - 1);
         const float *rw = p.rowws + ri * kRowWs;
         const float lse = p.LSE[ri];
-        float a = 0.0f, b = 0.0f, invs = 0.0f, e = 0.0f, hi = 0.0f;
+        float a = 0.0f, b = 0.0f, invs = 0.0f, e = 0.0f, invz = 0.0f;
         if (MAP == MAPB_EXACT) {
           e = lse * 1.4426950408889634f;
         } else {
-          hi = p.hi[ri];
+          const float hi = p.hi[ri];
           const RowMap rm = make_rowmap(hi, p.lo[ri], p.K, p.fixed_window != 0, p.window);
           a = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
           b = rm.degenerate ? Kf : rm.b;
           invs = rm.degenerate ? 0.0f : rm.inv;
           e = (p.surrogate == QSM_SURR_POST) ? rw[RW_LSESTAR] * 1.4426950408889634f
                                              : rm.hiL2E;
-          float gk = grid_value(rm, p.K, 0);
-          for (int m = 0; m <= p.K; ++m) {
+          for (int m = g; m <= p.K; m += 4) {
+            const float gk = grid_value(rm, p.K, m);
             const float gk1 = m < p.K ? grid_value(rm, p.K, m + 1) : gk;
             tab[key * K1 + m] = make_float2(gk, __fsub_rn(gk1, gk));
-            gk = gk1;
           }
-          cst[C_INVZ * 128 + key] = expf(hi - lse);
+          if (g == 0) invz = expf(hi - lse);
         }
-        if (MAP == MAPB_EXACT) cst[C_INVZ * 128 + key] = 0.0f;
-        cst[C_A * 128 + key] = a;
-        cst[C_B * 128 + key] = b;
-        cst[C_DELTA * 128 + key] = rw[RW_DELTA];
-        cst[C_E * 128 + key] = e;
-        cst[C_DSTAR * 128 + key] = rw[RW_DELTASTAR];
-        cst[C_INVS * 128 + key] = invs;
+        if (g == 0) {
+          float4 *c = reinterpret_cast<float4 *>(cst + key * 8);
+          c[0] = make_float4(a, b, invz, rw[RW_DELTA]);
+          c[1] = make_float4(e, rw[RW_DELTASTAR], invs, 0.0f);
+        }
       }
       // every row's constants are in place (a bounded wait, unlike bar.sync)
       mbar_arrive(bars.cst_ready);
@@ -621,74 +641,77 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const int qbase = qt * 128;
       const bool full = (qbase + 128 <= p.S) && (kt * 128 + 128 <= p.S) && (!p.causal || qt > kt);
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      {
         uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + T_S + 32 * cc, sv);
-        tmem_ld32(lane_base + T_DP + 32 * cc, dv);
+        tmem_ld32(lane_base + T_S + col0, sv);
+        tmem_ld32(lane_base + T_DP + col0, dv);
         tmem_wait_ld();
         reg_fence32(sv);
         reg_fence32(dv);
-        float pv[32], dsv[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = 32 * cc + i;
-          const int qg = qbase + col;
-          const bool valid = full || (key_ok && qg < p.S && (!p.causal || kg <= qg));
-          const float r = __uint_as_float(sv[i]);
-          const float dp = __uint_as_float(dv[i]);
-          const float delta = cst[C_DELTA * 128 + col];
-          float pw, ds;
-          if (MAP == MAPB_EXACT) {
-            pw = ex2_approx(__fmaf_rn(r, p.cL2E, -cst[C_E * 128 + col]));
-            ds = pw * (dp - delta);
-          } else {
-            const float invZ = cst[C_INVZ * 128 + col];
-            const float u = __fmaf_rn(r, cst[C_A * 128 + col], cst[C_B * 128 + col]);
-            const float uc = fminf(fmaxf(u, 0.0f), Kf);
-            const bool below = p.fixed_window && u < 0.0f;
-            float w, slope = 0.0f;
-            if (MAP == MAPB_HARD) {
-              const int m = static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
-              w = tab[col * K1 + m].x;
-            } else {
-              const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), Kf - 1.0f);
-              const int k = static_cast<int>(kf);
-              const float2 gd = tab[col * K1 + k];
-              w = __fmaf_rn(__fsub_rn(uc, kf), gd.y, gd.x);
-              slope = gd.y;
-            }
-            if (below && p.flush) w = 0.0f;
-            pw = w * invZ;
-            const float gw = (dp - delta) * invZ;
-            if (p.surrogate == QSM_SURR_NONE) {
-              ds = (MAP == MAPB_INTERP && !below) ? gw * slope * cst[C_INVS * 128 + col] : 0.0f;
-            } else if (p.surrogate == QSM_SURR_PRE) {
-              ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -cst[C_E * 128 + col]));
-            } else {
-              ds = ex2_approx(__fmaf_rn(r, p.cL2E, -cst[C_E * 128 + col])) *
-                   (dp - cst[C_DSTAR * 128 + col]);
-            }
-          }
-          pv[i] = valid ? pw : 0.0f;
-          dsv[i] = valid ? ds : 0.0f;
-        }
         uint32_t pp[16], dd[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          pp[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
-          dd[i] = pack_bf16x2(dsv[2 * i], dsv[2 * i + 1]);
+        for (int i2 = 0; i2 < 16; ++i2) {
+          float pv2[2], ds2[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int i = 2 * i2 + h;
+            const int col = col0 + i;
+            const int qg = qbase + col;
+            const bool valid = full || (key_ok && qg < p.S && (!p.causal || kg <= qg));
+            const float r = __uint_as_float(sv[i]);
+            const float dp = __uint_as_float(dv[i]);
+            const float4 c0 = cst4[2 * col], c1 = cst4[2 * col + 1];
+            const float delta = c0.w;
+            float pw, ds;
+            if (MAP == MAPB_EXACT) {
+              pw = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
+              ds = pw * (dp - delta);
+            } else {
+              const float invZ = c0.z;
+              const float u = __fmaf_rn(r, c0.x, c0.y);
+              const float uc = fminf(fmaxf(u, 0.0f), Kf);
+              const bool below = p.fixed_window && u < 0.0f;
+              float w, slope = 0.0f;
+              if (MAP == MAPB_HARD) {
+                const int m = static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+                w = tab[col * K1 + m].x;
+              } else {
+                const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), Kf - 1.0f);
+                const int k = static_cast<int>(kf);
+                const float2 gd = tab[col * K1 + k];
+                w = __fmaf_rn(__fsub_rn(uc, kf), gd.y, gd.x);
+                slope = gd.y;
+              }
+              if (below && p.flush) w = 0.0f;
+              pw = w * invZ;
+              const float gw = (dp - delta) * invZ;
+              if (p.surrogate == QSM_SURR_NONE) {
+                ds = (MAP == MAPB_INTERP && !below) ? gw * slope * c1.z : 0.0f;
+              } else if (p.surrogate == QSM_SURR_PRE) {
+                ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
+              } else {
+                ds = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x)) * (dp - c1.y);
+              }
+            }
+            pv2[h] = valid ? pw : 0.0f;
+            ds2[h] = valid ? ds : 0.0f;
+          }
+          pp[i2] = pack_bf16x2(pv2[0], pv2[1]);
+          dd[i2] = pack_bf16x2(ds2[0], ds2[1]);
         }
-        tmem_st16(lane_base + T_S + 16 * cc, pp);
-        tmem_st16(lane_base + T_DP + 16 * cc, dd);
+        // P^T and dS^T into the first 16 of this group's own TMEM columns
+        // (the other groups are still reading theirs)
+        tmem_st16(lane_base + T_S + col0, pp);
+        tmem_st16(lane_base + T_DP + col0, dd);
         // dS in shared memory as the MN-major A operand of dQ = dS K:
         // K index = key (row of 128 bytes per 64 queries), M = query
-        const uint32_t region = ds_base + (cc >> 1) * G::CHUNK_BYTES + key * 128;
+        const uint32_t region = ds_base + (g >> 1) * G::CHUNK_BYTES + key * 128;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t gran = ((cc & 1) * 4 + g) ^ (key & 7);
+        for (int gi = 0; gi < 4; ++gi) {
+          const uint32_t gran = ((g & 1) * 4 + gi) ^ (key & 7);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(region + gran * 16),
-                       "r"(dd[4 * g]), "r"(dd[4 * g + 1]), "r"(dd[4 * g + 2]), "r"(dd[4 * g + 3])
+                       "r"(dd[4 * gi]), "r"(dd[4 * gi + 1]), "r"(dd[4 * gi + 2]),
+                       "r"(dd[4 * gi + 3])
                        : "memory");
         }
       }
@@ -696,20 +719,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(bars.pds_full);
-      // ---- dQ tile (lane = query row) into the fp32 workspace
+      // ---- dQ tile (lane = query row) into the fp32 workspace: group g adds
+      // columns g*D/4 .. (g+1)*D/4 - 1
       ok = warp_all_b(mbar_wait(bars.dq_full, n & 1, abort));
       if (!ok) break;
       tc_fence_after();
       const int qrow = qbase + key;
-      float *dst = p.dqacc + (static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1)) * D;
-#pragma unroll 1
-      for (int dc = 0; dc < D / 32; ++dc) {
-        uint32_t v[32];
-        tmem_ld32_sync(lane_base + T_DQ + 32 * dc, v);
+      float *dst = p.dqacc + (static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1)) * D + g * (D / 4);
+      static_assert(D / 4 == 16, "dQ slice of one map group: 16 columns");
+      {
+        uint32_t v[16];
+        tmem_ld16_sync(lane_base + T_DQ + g * (D / 4), v);
         if (qrow < p.S) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            red_add_v4(dst + 32 * dc + 4 * i, __uint_as_float(v[4 * i]) * p.c,
+          for (int i = 0; i < 4; ++i)
+            red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]) * p.c,
                        __uint_as_float(v[4 * i + 1]) * p.c, __uint_as_float(v[4 * i + 2]) * p.c,
                        __uint_as_float(v[4 * i + 3]) * p.c);
         }
@@ -717,48 +741,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(bars.dq_empty);
     }
-    // ---- dK, dV of this key tile
+    // ---- dK, dV of this key tile: group g stores 32 columns, dK for g < 2
     if (ok && nq > 0) ok = warp_all_b(mbar_wait(bars.acc_full, 0, abort));
     if (ok) {
       tc_fence_after();
       const size_t krow = static_cast<size_t>(bh) * p.S + min(kg, p.S - 1);
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16 *out = (which == 0 ? p.dK : p.dV) + krow * D;
-        const float sc = which == 0 ? p.c : 1.0f;
-#pragma unroll 1
-        for (int dc = 0; dc < D / 32; ++dc) {
-          uint32_t v[32];
-          if (nq > 0) {
-            tmem_ld32_sync(lane_base + (which == 0 ? T_DK : T_DV) + 32 * dc, v);
-          } else {
+      static_assert(D == 64, "dK / dV slices: two groups of 32 columns each");
+      const int which = g >> 1, dc = g & 1;
+      __nv_bfloat16 *out = (which == 0 ? p.dK : p.dV) + krow * D;
+      const float sc = which == 0 ? p.c : 1.0f;
+      uint32_t v[32];
+      if (nq > 0) {
+        tmem_ld32_sync(lane_base + (which == 0 ? T_DK : T_DV) + 32 * dc, v);
+      } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
-          float x[32];
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      }
+      float x[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(v[i]) * sc;
-          if (which == 0 && p.dkcal != nullptr && key_ok) {
-            const float4 *cal = reinterpret_cast<const float4 *>(p.dkcal + krow * D + 32 * dc);
+      for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(v[i]) * sc;
+      if (which == 0 && p.dkcal != nullptr && key_ok) {
+        const float4 *cal = reinterpret_cast<const float4 *>(p.dkcal + krow * D + 32 * dc);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 c4 = cal[i];
-              x[4 * i] += c4.x;
-              x[4 * i + 1] += c4.y;
-              x[4 * i + 2] += c4.z;
-              x[4 * i + 3] += c4.w;
-            }
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-          if (key_ok) {
-            uint4 *d4 = reinterpret_cast<uint4 *>(out + 32 * dc);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
+        for (int i = 0; i < 8; ++i) {
+          const float4 c4 = cal[i];
+          x[4 * i] += c4.x;
+          x[4 * i + 1] += c4.y;
+          x[4 * i + 2] += c4.z;
+          x[4 * i + 3] += c4.w;
         }
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+      if (key_ok) {
+        uint4 *d4 = reinterpret_cast<uint4 *>(out + 32 * dc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       }
     }
   }
@@ -805,7 +825,7 @@ qsm_status launch_bwd_d(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
     p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + 4 * G::TILE_BYTES);
     p.tab_off = p.ds_off + 128 * 128 * 2;
     p.cst_off = static_cast<uint32_t>(p.tab_off + tab);
-    p.bar_off = static_cast<uint32_t>((p.cst_off + C_NUM * 128 * 4 + 15) & ~15u);
+    p.bar_off = static_cast<uint32_t>((p.cst_off + 128 * 8 * 4 + 15) & ~15u);
     size_t smem = 1024 + p.bar_off + 256;
     if (smem < 120 * 1024) smem = 120 * 1024;
     if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
@@ -815,7 +835,7 @@ qsm_status launch_bwd_d(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return QSM_ERR_CUDA;
-    kern<<<dim3(p.nkvt, BH), kBwdThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+    kern<<<dim3(p.nkvt, BH), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
     if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
   }
   return QSM_OK;
