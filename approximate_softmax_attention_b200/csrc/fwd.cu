@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -903,6 +904,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------- host
 
+constexpr int kMaxDevices = 64;
+
 template <int D, bool FP8, int MAP>
 static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv) {
@@ -951,9 +954,25 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
   auto kern = qsm_fwd_kernel<D, FP8, MAP>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return QSM_ERR_CUDA;
+  // Raising the kernel's dynamic shared memory limit is a driver round trip;
+  // this instantiation remembers, per device, the largest limit already set.
+  static std::atomic<int> smem_set[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QSM_ERR_CUDA;
+  const bool cached = dev >= 0 && dev < kMaxDevices &&
+                      smem_set[dev].load(std::memory_order_acquire) >= static_cast<int>(smem);
+  if (!cached) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return QSM_ERR_CUDA;
+    if (dev >= 0 && dev < kMaxDevices) {
+      int prev = smem_set[dev].load(std::memory_order_relaxed);
+      while (prev < static_cast<int>(smem) &&
+             !smem_set[dev].compare_exchange_weak(prev, static_cast<int>(smem),
+                                                  std::memory_order_acq_rel)) {
+      }
+    }
+  }
   dim3 grid(p.nqt * a.B * a.H);
   kern<<<grid, kThreads, smem, a.stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;

@@ -217,6 +217,15 @@ def test_full_size_s8k_fp8_sampled(name):
     _sampled_check(name, 5e-2, 5e-3, nheads=2, nrows=48)
 
 
+@pytest.mark.parametrize("name,tol_max,tol_mean", [("s16k_bf16_causal", 1e-2, 1e-3),
+                                                   ("s16k_fp8_causal", 5e-2, 5e-3)])
+def test_full_size_s16k_causal_sampled(name, tol_max, tol_mean):
+    """B=1, H=32, S=16384, D=128 causal, bf16 and e4m3: exact, Rowmax-PoT and
+    the K-interval sweep K in {4, 16} x {min-max, fixed window} x
+    {interpolation, hard rounding}, on sampled rows of two heads."""
+    _sampled_check(name, tol_max, tol_mean, nheads=2, nrows=24)
+
+
 def test_timeout_path_reports_status_and_context_survives():
     d = inputs.draw(1, 1, 256, 64, seed=1)
     q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
