@@ -15,10 +15,11 @@
 //
 // Kernels, in launch order on the caller's stream:
 //   1. qsm_bwd_delta      delta_r = dO_r . O_r (one warp per row)
-//   2. qsm_bwd_rows       one thread per query row sweeps S = Q K^T and
-//                         dP = dO V^T tiles (tcgen05) and accumulates dhi,
-//                         dlo and, for the post surrogate, LSE* and delta*
-//                         online (only when one of them is needed)
+//   2. qsm_bwd_rows       one thread per (query row, column quarter) sweeps
+//                         S = Q K^T and dP = dO V^T tiles (tcgen05) and
+//                         accumulates dhi, dlo and, for the post surrogate,
+//                         LSE* and delta* online; the quarters merge at the
+//                         end (only run when one of them is needed)
 //   3. qsm_bwd_calib      one warp per row: the calibration terms, rank one
 //                         per row, in fp32: dQ_r += c (dhi k_argmax + dlo
 //                         k_argmin), dKcal[argmax] += c dhi q_r, dKcal[argmin]
@@ -45,9 +46,9 @@ namespace qsm {
 
 namespace {
 
-constexpr int kBwdThreads = 256;        // rows kernel: warp 0 TMA, warp 1 MMA, warps 4-7 map
-// main kernel: warp 0 TMA, warp 1 MMA, warps 4-19 four map groups, group g
-// owning query columns 32g .. 32g+31 of every S^T / dP^T tile
+// rows and main kernels: warp 0 TMA, warp 1 MMA, warps 4-19 four map groups,
+// group g owning columns 32g .. 32g+31 of every S / dP (rows) or S^T / dP^T
+// (main) tile
 constexpr int kMainThreads = 640;
 constexpr int kMainMapThreads = 512;
 constexpr uint32_t kBwdTmemCols = 512;
@@ -207,15 +208,17 @@ struct RowBars {
   uint64_t *q_full;
   uint64_t *sd_full, *sd_empty;   // [2]
   uint64_t *drain;
+  uint64_t *tab_ready, *part_ready;   // single use: grid table built; partial sums written
   uint32_t *tmem_slot;
   int *abort;
 };
 
 // --------------------------------------------------------------- rows
-// One CTA per 128 query rows of one (b, h); thread = row.  Computes the
+// One CTA per 128 query rows of one (b, h); four map groups, thread = row,
+// group g taking columns 32g .. 32g+31 of every S / dP tile.  Computes the
 // calibration derivatives dhi, dlo and (post surrogate) LSE*, delta*.
 template <int D, int MAP>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_rows(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams p) {
@@ -239,7 +242,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   bars.sd_full = bars.q_full + 1;
   bars.sd_empty = bars.sd_full + 2;
   bars.drain = bars.sd_empty + 2;
-  bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
+  bars.tab_ready = bars.drain + 1;
+  bars.part_ready = bars.tab_ready + 1;
+  bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.part_ready + 1);
+  // per-row partial sums of the four groups: dhi, dlo, m*, l*, a* ([5][4][128])
+  float *part = reinterpret_cast<float *>(smem + p.cst_off);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
   const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -252,9 +259,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bars.q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.sd_full[i], 1);
-      mbar_init(&bars.sd_empty[i], 128);
+      mbar_init(&bars.sd_empty[i], kMainMapThreads);
     }
     mbar_init(bars.drain, 1);
+    mbar_init(bars.tab_ready, kMainMapThreads);
+    mbar_init(bars.part_ready, kMainMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
   }
@@ -320,7 +329,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait(bars.drain, 0, abort);
     }
   } else if (warp >= 4) {
-    const int row = threadIdx.x - 128;
+    const int g = (warp - 4) >> 2;                       // map group: columns 32g..32g+31
+    const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int qrow = qt * 128 + row;
     const bool row_ok = qrow < p.S;
@@ -335,101 +345,129 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float a_raw = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
     const float b_raw = rm.degenerate ? static_cast<float>(p.K) : rm.b;
     const float Kf = static_cast<float>(p.K);
+    const float invK = 1.0f / Kf;
     const float a_s = __fsub_rn(hi, rm.lo);        // hi - lo in score units
+    const float inv_a = rm.degenerate ? 0.0f : 1.0f / a_s;
+    const float slope_fw = -Kf / p.window;         // fixed window: d(coordinate)/d(hi) per slope
     const bool calib = !p.detach && !rm.degenerate;
     const bool post = p.surrogate == QSM_SURR_POST;
-    // this row's grid table column: (g_n, g_{n+1} - g_n), n = 0..K
-    {
-      float gk = grid_value(rm, p.K, 0);
-      for (int n = 0; n <= p.K; ++n) {
-        const float gk1 = n < p.K ? grid_value(rm, p.K, n + 1) : gk;
-        tab[n * 128 + row] = make_float2(gk, __fsub_rn(gk1, gk));
-        gk = gk1;
-      }
+    // this row's grid table column: (g_n, g_{n+1} - g_n), n = 0..K; the four
+    // groups build alternate entries
+    for (int n = g; n <= p.K; n += 4) {
+      const float gk = grid_value(rm, p.K, n);
+      const float gk1 = n < p.K ? grid_value(rm, p.K, n + 1) : gk;
+      tab[n * 128 + row] = make_float2(gk, __fsub_rn(gk1, gk));
     }
+    mbar_arrive(bars.tab_ready);
+    bool ok = warp_all_b(mbar_wait(bars.tab_ready, 0, abort));
     float dhi = 0.0f, dlo = 0.0f;
     float mstar = -INFINITY, lstar = 0.0f, astar = 0.0f;
     uint32_t cnt[2] = {0, 0};
-    bool ok = true;
+    const int c0 = 32 * g;
     for (int j = 0; j < nkv && ok; ++j) {
       const int b = j & 1;
       ok = warp_all_b(mbar_wait(&bars.sd_full[b], cnt[b] & 1, abort));
       ++cnt[b];
       if (!ok) break;
       tc_fence_after();
-      const int lim = L - 128 * j;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(lane_base + b * 256 + 32 * cc, sv);
-        tmem_ld32(lane_base + b * 256 + 128 + 32 * cc, dv);
-        tmem_wait_ld();
-        reg_fence32(sv);
-        reg_fence32(dv);
-        if (post) {
-          float cm = -INFINITY;
+      const int lim = L - 128 * j - c0;            // valid columns of this group
+      uint32_t sv[32], dv[32];
+      tmem_ld32(lane_base + b * 256 + c0, sv);
+      tmem_ld32(lane_base + b * 256 + 128 + c0, dv);
+      tmem_wait_ld();
+      reg_fence32(sv);
+      reg_fence32(dv);
+      // values in registers: hand the buffers back first
+      tc_fence_before();
+      mbar_arrive(&bars.sd_empty[b]);
+      if (post) {
+        float cm = -INFINITY;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * cc + i < lim) cm = fmaxf(cm, __uint_as_float(sv[i]) * p.c);
-          if (cm > mstar) {
-            const float sc = expf(mstar - cm);
-            lstar *= sc;
-            astar *= sc;
-            mstar = cm;
-          }
+        for (int i = 0; i < 32; ++i)
+          if (i < lim) cm = fmaxf(cm, __uint_as_float(sv[i]) * p.c);
+        if (cm > mstar) {
+          const float sc = expf(mstar - cm);
+          lstar *= sc;
+          astar *= sc;
+          mstar = cm;
+        }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (32 * cc + i < lim) {
-              const float e = expf(__uint_as_float(sv[i]) * p.c - mstar);
-              lstar += e;
-              astar = fmaf(e, __uint_as_float(dv[i]), astar);
-            }
+        for (int i = 0; i < 32; ++i) {
+          if (i < lim) {
+            const float e = expf(__uint_as_float(sv[i]) * p.c - mstar);
+            lstar += e;
+            astar = fmaf(e, __uint_as_float(dv[i]), astar);
           }
         }
-        if (calib && MAP != MAPB_EXACT) {
+      }
+      if (calib && MAP != MAPB_EXACT) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (32 * cc + i >= lim) continue;
-            const float r = __uint_as_float(sv[i]);
-            const float gw = (__uint_as_float(dv[i]) - delta) * invZ;
-            const float u = __fmaf_rn(r, a_raw, b_raw);
-            const float uc = fminf(fmaxf(u, 0.0f), Kf);
-            if (MAP == MAPB_HARD) {
-              if (!p.fixed_window) {
-                const int n =
-                    static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
-                const float g = tab[n * 128 + row].x;
-                const float t = gw * (static_cast<float>(n) - Kf) / Kf * g;
-                dhi += t;
-                dlo -= t;
-              }
-            } else {
-              const float kf = fminf(floorf(uc), Kf - 1.0f);
-              const int k = static_cast<int>(kf);
-              const float f = uc - kf;
-              const float2 gd = tab[k * 128 + row];
-              const float g0 = gd.x, slope = gd.y, g1 = gd.x + gd.y;
-              if (!p.fixed_window) {
-                const float mix = ((1.0f - f) * (Kf - kf) * g0 + f * (Kf - kf - 1.0f) * g1) / Kf;
-                dhi += gw * (-slope * uc / a_s - mix);
-                dlo += gw * (-slope * (Kf - uc) / a_s + mix);
-              } else if (u >= 0.0f) {
-                dhi += gw * (-slope * Kf / p.window);
-              }
+        for (int i = 0; i < 32; ++i) {
+          if (i >= lim) continue;
+          const float r = __uint_as_float(sv[i]);
+          const float gw = (__uint_as_float(dv[i]) - delta) * invZ;
+          const float u = __fmaf_rn(r, a_raw, b_raw);
+          const float uc = fminf(fmaxf(u, 0.0f), Kf);
+          if (MAP == MAPB_HARD) {
+            if (!p.fixed_window) {
+              const int n =
+                  static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+              const float gv = tab[n * 128 + row].x;
+              const float t = gw * (static_cast<float>(n) - Kf) * invK * gv;
+              dhi += t;
+              dlo -= t;
+            }
+          } else {
+            const float kf = fminf(floorf(uc), Kf - 1.0f);
+            const int k = static_cast<int>(kf);
+            const float f = uc - kf;
+            const float2 gd = tab[k * 128 + row];
+            const float g0 = gd.x, slope = gd.y, g1 = gd.x + gd.y;
+            if (!p.fixed_window) {
+              const float mix = ((1.0f - f) * (Kf - kf) * g0 + f * (Kf - kf - 1.0f) * g1) * invK;
+              dhi += gw * (-slope * uc * inv_a - mix);
+              dlo += gw * (-slope * (Kf - uc) * inv_a + mix);
+            } else if (u >= 0.0f) {
+              dhi += gw * (slope * slope_fw);
             }
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars.sd_empty[b]);
     }
-    if (ok && row_ok) {
-      float *w = p.rowws + ri * kRowWs;
-      w[RW_DHI] = calib ? dhi : 0.0f;
-      w[RW_DLO] = calib ? dlo : 0.0f;
+    // merge the four groups' partial sums (the online log-sum-exp of the post
+    // surrogate rescales each part to the common maximum)
+    part[(0 * 4 + g) * 128 + row] = dhi;
+    part[(1 * 4 + g) * 128 + row] = dlo;
+    part[(2 * 4 + g) * 128 + row] = mstar;
+    part[(3 * 4 + g) * 128 + row] = lstar;
+    part[(4 * 4 + g) * 128 + row] = astar;
+    mbar_arrive(bars.part_ready);
+    if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
+    if (ok && row_ok && g == 0) {
+      float sdhi = 0.0f, sdlo = 0.0f, M = -INFINITY;
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) {
+        sdhi += part[(0 * 4 + gg) * 128 + row];
+        sdlo += part[(1 * 4 + gg) * 128 + row];
+        M = fmaxf(M, part[(2 * 4 + gg) * 128 + row]);
+      }
+      float Ls = 0.0f, As = 0.0f;
       if (post) {
-        w[RW_LSESTAR] = mstar + logf(lstar);
-        w[RW_DELTASTAR] = astar / lstar;
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg) {
+          const float mg = part[(2 * 4 + gg) * 128 + row];
+          if (mg == -INFINITY) continue;             // a group with no valid column
+          const float sc = expf(mg - M);
+          Ls = fmaf(part[(3 * 4 + gg) * 128 + row], sc, Ls);
+          As = fmaf(part[(4 * 4 + gg) * 128 + row], sc, As);
+        }
+      }
+      float *w = p.rowws + ri * kRowWs;
+      w[RW_DHI] = calib ? sdhi : 0.0f;
+      w[RW_DLO] = calib ? sdlo : 0.0f;
+      if (post) {
+        w[RW_LSESTAR] = M + logf(Ls);
+        w[RW_DELTASTAR] = As / Ls;
       }
     }
   }
@@ -802,7 +840,8 @@ qsm_status launch_bwd_d(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
     const size_t tab = static_cast<size_t>(128) * (p.K + 1) * sizeof(float2);
     BwdParams r = p;
     r.tab_off = static_cast<uint32_t>(2 * G::TILE_BYTES + 4 * G::TILE_BYTES);
-    r.bar_off = static_cast<uint32_t>((r.tab_off + tab + 15) & ~static_cast<size_t>(15));
+    r.cst_off = static_cast<uint32_t>((r.tab_off + tab + 15) & ~static_cast<size_t>(15));
+    r.bar_off = static_cast<uint32_t>(r.cst_off + 5 * 4 * 128 * sizeof(float));
     size_t smem = 1024 + r.bar_off + 256;
     if (smem < 120 * 1024) smem = 120 * 1024;
     if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
@@ -810,7 +849,7 @@ qsm_status launch_bwd_d(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return QSM_ERR_CUDA;
-    kern<<<dim3(p.nqt, BH), kBwdThreads, smem, a.stream>>>(mq, mk, mv, mdo, r);
+    kern<<<dim3(p.nqt, BH), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, r);
     if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
   }
   if (p.dkcal != nullptr) {
