@@ -791,14 +791,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (leader) mma_commit(bar);
       __syncwarp();
     };
+    // Descriptors: the start-address field is the low 14 bits (address >> 4)
+    // and every operand lies below 256 KB, so an operand offset is added to a
+    // base descriptor instead of building each descriptor again.
+    const uint64_t qdesc = smem_desc(qaddr, 16, 1024);
+    const uint64_t kdesc = smem_desc(kvaddr0, 16, 1024);
+    const uint64_t vdesc = smem_desc(kvaddr0, G::CHUNK_BYTES, 1024);
     auto issue_qk = [&](int st, uint32_t col) {
-      const uint32_t ka = kvaddr0 + st * G::TILE_BYTES;
+      const uint64_t kd = kdesc + ((st * G::TILE_BYTES) >> 4);
 #pragma unroll
       for (int kk = 0; kk < G::KSTEPS_QK; ++kk) {
         const int e = kk * G::MMA_K;
         const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * G::ELEM;
-        const uint64_t ad = smem_desc(qaddr + off, 16, 1024);
-        const uint64_t bd = smem_desc(ka + off, 16, 1024);
+        const uint64_t ad = qdesc + (off >> 4);
+        const uint64_t bd = kd + (off >> 4);
         if (leader) {
           if (FP8)
             mma_ss_f8(tmem + col, ad, bd, G::IDESC_QK, kk > 0);
@@ -809,10 +815,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     auto issue_pv = [&](int st, uint32_t pcol, bool acc) {
-      const uint32_t va = kvaddr0 + st * G::TILE_BYTES;
+      const uint64_t vd = vdesc + ((st * G::TILE_BYTES) >> 4);
 #pragma unroll
       for (int kk = 0; kk < G::KSTEPS_PV; ++kk) {
-        const uint64_t bd = smem_desc(va + kk * G::MMA_K * 128, G::CHUNK_BYTES, 1024);
+        const uint64_t bd = vd + ((kk * G::MMA_K * 128) >> 4);
         // keys 64h .. 64h+63 of the tile sit, packed, from TMEM column 64h
         // (the map group owning that half writes its P into the first of
         // its own S columns): 8 columns per k-step
