@@ -410,16 +410,20 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           const float uc = fminf(fmaxf(u, 0.0f), Kf);
           if (MAP == MAPB_HARD) {
             if (!p.fixed_window) {
-              const int n =
-                  static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+              // nearest node from the bits of a magic-number add (no
+              // float <-> int conversion on the XU pipe)
+              const float tn = __fadd_rn(uc, kMagic);
+              const int n = static_cast<int>(__float_as_uint(tn) - kMagicBits);
               const float gv = tab[n * 128 + row].x;
-              const float t = gw * (static_cast<float>(n) - Kf) * invK * gv;
+              const float t = gw * (__fsub_rn(tn, kMagic) - Kf) * invK * gv;
               dhi += t;
               dlo -= t;
             }
           } else {
-            const float kf = fminf(floorf(uc), Kf - 1.0f);
-            const int k = static_cast<int>(kf);
+            // floor from a round-down add of 2^23 (exact for 0 <= uc <= K)
+            const float tf = __fadd_rd(uc, 8388608.0f);
+            const float kf = fminf(__fsub_rn(tf, 8388608.0f), Kf - 1.0f);
+            const int k = min(static_cast<int>(__float_as_uint(tf) - 0x4B000000u), p.K - 1);
             const float f = uc - kf;
             const float2 gd = tab[k * 128 + row];
             const float g0 = gd.x, slope = gd.y, g1 = gd.x + gd.y;
@@ -714,8 +718,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                 const int m = static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
                 w = tab[col * K1 + m].x;
               } else {
-                const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), Kf - 1.0f);
-                const int k = static_cast<int>(kf);
+                const float tf = __fadd_rd(uc, 8388608.0f);
+                const float kf = fminf(__fsub_rn(tf, 8388608.0f), Kf - 1.0f);
+                const int k = min(static_cast<int>(__float_as_uint(tf) - 0x4B000000u), p.K - 1);
                 const float2 gd = tab[col * K1 + k];
                 w = __fmaf_rn(__fsub_rn(uc, kf), gd.y, gd.x);
                 slope = gd.y;
