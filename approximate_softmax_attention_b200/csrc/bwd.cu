@@ -101,17 +101,6 @@ __device__ __forceinline__ void mma_nt(uint32_t d_tmem, uint32_t a_saddr, uint32
   }
 }
 
-// acc (+)= A[tmem, 128 x 128] B[smem, 128 x D, MN-major]
-template <int D>
-__device__ __forceinline__ void mma_tn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_saddr,
-                                       bool acc) {
-  using G = BGeo<D>;
-#pragma unroll
-  for (int kk = 0; kk < G::KSTEPS_N; ++kk)
-    mma_ts_f16(d_tmem, a_tmem + kk * 8, smem_desc(b_saddr + kk * 16 * 128, G::CHUNK_BYTES, 1024),
-               G::IDESC_TS, (acc || kk > 0) ? 1u : 0u);
-}
-
 // acc (+)= A[tmem, 128 x 128, group layout] B[smem, 128 x D, MN-major]: the
 // bf16 values of K-columns 32g .. 32g+31 of A sit in TMEM columns 32g ..
 // 32g+15 (each map group writes its P^T / dS^T into the first half of its own
@@ -484,16 +473,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 }
 
 // --------------------------------------------------------------- main
-enum Cst {
-  C_A = 0,      // coordinate = fma(r, a, b)  (raw accumulator units)
-  C_B,
-  C_INVZ,
-  C_DELTA,
-  C_E,          // exact: LSE*log2e; pre: hi*log2e; post: LSE* * log2e
-  C_DSTAR,      // post: delta*
-  C_INVS,       // K / (hi - lo): d(coordinate)/ds
-  C_NUM
-};
+// Per-query-row record of the main kernel (8 floats, read as two float4):
+//   [0] a, [1] b      grid coordinate = fma(r, a, b) (raw accumulator units)
+//   [2] 1/Z           K-interval normaliser (exact map: unused)
+//   [3] delta         dO . O
+//   [4] e             exact: LSE*log2e; pre: hi*log2e; post: LSE* * log2e
+//   [5] delta*        post surrogate: sum of softmax(s) dP
+//   [6] K / (hi - lo) d(coordinate)/ds
+//   [7] unused
 
 struct MainBars {
   uint64_t *kv_full;                // K_j, V_j
@@ -528,7 +515,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *sQD = smem + 2 * G::TILE_BYTES;              // [2 stages][Q, dO]
   uint8_t *sDS = smem + p.ds_off;                        // 128 x 128 bf16, MN-major
   float2 *tab = reinterpret_cast<float2 *>(smem + p.tab_off);   // [row][n]
-  float *cst = reinterpret_cast<float *>(smem + p.cst_off);     // [128][8]: C_* per row
+  float *cst = reinterpret_cast<float *>(smem + p.cst_off);     // [128][8]: one record per row
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   MainBars bars;
   bars.kv_full = bp;
