@@ -21,7 +21,7 @@ from oracle import spec
 from oracle import attention as A
 from approximate_softmax_attention_b200 import inputs, qsm
 
-from _helpers import boundary_distance_rows, err_stats
+from _helpers import boundary_distance_rows, err_stats, err_stats_bf16_out
 
 pytestmark = pytest.mark.gpu
 
@@ -174,6 +174,45 @@ def test_fwd_below_policy(below):
                               want_idx=True)
         mx, mean = err_stats(got["O"], ref["O"])
         assert mx <= 1e-2 and mean <= 1e-3, (mode, mx, mean)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("below", [0, 1])
+@pytest.mark.parametrize("floor", [6, 15])
+def test_fwd_pot_floor_wide_scores(dtype, below, floor):
+    """Rowmax-PoT with most keys past the exponent floor: a score scale of
+    6/sqrt(D) spreads a row over tens of e-folds, so O depends on every
+    floored weight (clamped to 2^-floor, or flushed to 0), with the decision
+    dump checked as well."""
+    S, D = 384 if dtype == "bf16" else 512, 128
+    d = inputs.draw(1, 2, S, D, seed=31, peaked=True, dtype=dtype)
+    scale = 6.0 / D ** 0.5
+    q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    dbg = torch.full((1, 2, S, S), -7, dtype=torch.int8, device=DEV)
+    O, LSE = qsm.attention_forward(q, k, v, True, qsm.MODE_ROWMAX_POT, 4, 0, 1, scale=scale,
+                                   q_descale=d["q_descale"], k_descale=d["k_descale"],
+                                   v_descale=d["v_descale"], pot_floor=floor,
+                                   below_policy=below, debug_idx=dbg)
+    torch.cuda.synchronize()
+    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], True, A.ROWMAX_POT, scale=scale,
+                          q_descale=d["q_descale"], k_descale=d["k_descale"],
+                          v_descale=d["v_descale"], pot_floor=floor, below_policy=below,
+                          want_idx=True)
+    idx = ref["idx"]
+    valid = idx != -1                      # -1 masked; -2 flushed
+    floored = (idx == -2) if below else (idx == floor)
+    # the case is the one it claims to be: most valid keys are at the floor
+    assert floored.sum() > 0.5 * valid.sum()
+    # the weight concentrates on each row's top keys, so |O| reaches ~4, where
+    # rounding the exact value to bf16 alone costs up to 0.0156: the max is
+    # taken net of that half-ulp (the reading the backward's tests use too)
+    mx, mean = err_stats_bf16_out(O.float().cpu().numpy(), ref["O"])
+    tol = 1e-2 if dtype == "bf16" else 5e-2
+    assert mx <= tol and mean <= (1e-3 if dtype == "bf16" else 5e-3), (mx, mean)
+    np.testing.assert_allclose(LSE.cpu().numpy(), ref["LSE"], atol=5e-3, rtol=1e-4)
+    got_idx = dbg.cpu().numpy()
+    agree = (got_idx == idx)[valid].mean()
+    assert agree >= 0.999, agree
 
 
 @pytest.mark.parametrize("causal", [False, True])
