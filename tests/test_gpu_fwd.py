@@ -176,6 +176,26 @@ def test_fwd_below_policy(below):
         assert mx <= 1e-2 and mean <= 1e-3, (mode, mx, mean)
 
 
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp8")])
+@pytest.mark.parametrize("K,calib,rounding", [(1, 0, 0), (1, 1, 1), (64, 0, 0), (64, 1, 0),
+                                              (64, 0, 1)])
+def test_fwd_kinterval_extreme_K(D, dtype, K, calib, rounding):
+    """K-interval with K = 1 (the interpolation table is one segment) and
+    K = 64 (the largest K the forward accepts; its interpolation table leaves
+    the bf16 D = 128 ring three shared-memory stages), causal, ragged S."""
+    S = 330
+    d = inputs.draw(1, 2, S, D, seed=50 + K + D, peaked=True, dtype=dtype)
+    got = _run_fwd(d, True, 1, K, calib, rounding, window=6.0, debug=True)
+    ref = _oracle(d, True, 1, K, calib, rounding, window=6.0, want_idx=True)
+    mx, mean = err_stats(got["O"], ref["O"])
+    if dtype == "bf16":
+        assert mx <= 1e-2 and mean <= 1e-3, (mx, mean)
+    else:
+        assert mx <= 5e-2, (mx, mean)
+    np.testing.assert_allclose(got["LSE"], ref["LSE"], atol=2e-3, rtol=1e-4)
+    _check_idx(d, got["idx"], ref["idx"], True, 1, K, calib, rounding, 6.0)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp8"])
 @pytest.mark.parametrize("below", [0, 1])
 @pytest.mark.parametrize("floor", [6, 15])
