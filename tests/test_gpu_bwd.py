@@ -72,6 +72,18 @@ def test_bwd_kinterval_small(S, causal, K, calib, rnd, surr, detach):
     _check(got, ref)
 
 
+@pytest.mark.parametrize("K", [1, 32])
+@pytest.mark.parametrize("calib,rnd", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("surr", [1, 2])
+def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
+    """K = 1 (one grid segment) and K = 32 (the largest K the backward
+    accepts), pre and post surrogate, calibration derivatives on."""
+    d = inputs.draw(1, 2, 256, 64, seed=90 + K, with_dO=True)
+    *got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
+    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0, dec=dec)
+    _check(got, ref)
+
+
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False), (77, True), (384, False)])
 def test_bwd_exact(S, causal):
     d = inputs.draw(1, 2, S, 64, seed=7 + S, with_dO=True)
