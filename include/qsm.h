@@ -98,10 +98,11 @@ typedef struct {
                              1: flush such weights to 0 */
   int detach_extrema;     /* backward: 1 drops the calibration derivatives */
   /* Row statistics [B,H,S], optional in the forward (written when non-NULL)
-   * and required by the K-interval backward: hi = row max of s, lo = row min
-   * of s (min-max) or hi - window, argmax/argmin = lowest key index of the
-   * row max / min.  Device pointers.  The exact map runs no statistics
-   * sweep: it writes row_hi only and leaves the other three untouched. */
+   * and required by the K-interval backward.  hi = row max of s.  lo = hi -
+   * window for fixed-window K-interval, else the row min of s.  argmax /
+   * argmin = lowest key index of the row max / min.  Device pointers.  Every
+   * map, the exact one included, runs the statistics sweep and writes each
+   * of the four that is non-NULL. */
   float *row_hi, *row_lo;
   int32_t *row_argmax, *row_argmin;
   /* Backward scratch, at least qsm_attn_bwd_workspace_size() bytes, device,
