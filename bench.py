@@ -6,15 +6,17 @@ Workload (one step): the forward of the B=4, H=16, S=2048, D=128 bf16 causal
 problem with peaked keys (1% of keys shifted +3 along a per-head unit
 direction), once per map: exact softmax, Rowmax-PoT, and K-interval K=16
 (min-max calibration, interpolation).  ``value`` is the step's algorithmic
-TFLOP/s (4*B*H*S^2*D per call, halved for causal; the statistics sweep of
-the approximate maps is not counted), whole job, inputs resident in HBM.
+TFLOP/s (4*B*H*S^2*D per call, halved for causal; the statistics sweep every
+map runs is not counted), whole job, inputs resident in HBM.
 Inputs rotate over three device copies (3 x 100 MB > the 126 MB L2), so no
 call starts with its operands in L2.
 
 The line also carries per-map TFLOP/s, the roofline of the dominant kernel
 (CUDA events on the launching stream), the oracle timed on the host cores on
 a bounded sample, an end-to-end number through host buffers, sampled SM
-clocks, and secondary per-map figures for the 8K / 16K problems.
+clocks, the host-side latency of one call per map, and secondary figures: per
+map at the 8K and 16K shapes, and the K-interval backward on the training
+shape.
 
 With --gpus N (launched under torchrun) every rank runs the same per-rank
 problem on its own GPU (data-parallel over independent batches; there is no
