@@ -205,8 +205,13 @@ qsm_status qsm_weight_map(const float *scores, const int32_t *valid_len, int row
   if (mode == QSM_MODE_KINTERVAL && (Kint < 1 || Kint > 64)) return QSM_ERR_INVALID_ARG;
   if (!finite_pos(o.window) || o.pot_floor < 0 || o.pot_floor > 126) return QSM_ERR_INVALID_ARG;
   if (o.below_policy != 0 && o.below_policy != 1) return QSM_ERR_INVALID_ARG;
+  if (!(o.scale == 0.0f || finite_pos(o.scale))) return QSM_ERR_INVALID_ARG;
+  if (!finite_pos(o.q_descale) || !finite_pos(o.k_descale)) return QSM_ERR_INVALID_ARG;
+  // the score scale folded into the map, formed as the forward forms it
+  const float c = (o.scale > 0.0f ? o.scale : 1.0f) * o.q_descale * o.k_descale;
+  if (!finite_pos(c)) return QSM_ERR_INVALID_ARG;
   MapArgs a{};
-  a.scores = scores; a.valid_len = valid_len; a.rows = rows; a.cols = cols;
+  a.scores = scores; a.c = c; a.valid_len = valid_len; a.rows = rows; a.cols = cols;
   a.mode = mode; a.Kint = Kint; a.calib = calibration; a.rounding = rounding;
   a.window = o.window; a.pot_floor = o.pot_floor; a.below_policy = o.below_policy;
   a.w = w; a.idx = idx; a.hi = hi; a.lo = lo;

@@ -42,8 +42,6 @@
 
 namespace qsm {
 
-enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
-
 struct FwdParams {
   int S, nqt, BH;
   int causal;
@@ -150,105 +148,6 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
   return b;
 }
 
-// Per-row constants of the fused map, with the score scale folded in: the
-// map consumes the raw fp32 accumulator r = q.k of the MMA.
-//   PoT:        x = fma(r, -c*log2e, hi*log2e), w = 2^-rne(min(x, cap)) * pscale
-//   K-interval: u = fma(r, c*K/(hi-lo), -lo*K/(hi-lo)); hard: g[rne(u)];
-//               interpolation: u d_k + c_k at k = floor(u) (grid values
-//               pre-multiplied by pscale).  Same decisions as the library's
-//               fp32 map up to the rounding of the folded scale.
-struct MapRow {
-  float a, b;        // coordinate = fma(r, a, b)
-  float cap, Kf, Km1;
-  float flush_t;     // PoT flush: kMagic + floor (t above it: exponent past the floor)
-  uint32_t tab;      // shared address bias of this row's table column
-  uint32_t pow_bias; // bits of pscale (PoT)
-};
-
-// Packed fp32 pairs (sm_100 f32x2 arithmetic: two IEEE round-to-nearest
-// (or round-down) operations per instruction, the same results as the
-// scalar forms).
-__device__ __forceinline__ uint64_t f2_bits(float2 a) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
-  return r;
-}
-__device__ __forceinline__ float2 f2_from(uint64_t r) {
-  float2 a;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
-  return a;
-}
-__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
-  return f2_from(r);
-}
-__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-  return f2_from(r);
-}
-__device__ __forceinline__ float2 add2_rd(float2 a, float2 b) {
-  uint64_t r;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
-  return f2_from(r);
-}
-
-// Weights of two scores (the map's arithmetic on a pair; FLUSH: Rowmax-PoT
-// with the below-floor policy "flush", exponents above the floor give 0).
-template <int MAP, bool FLUSH>
-__device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
-  const float2 x = fma2_rn(r, make_float2(m.a, m.a), make_float2(m.b, m.b));
-  if (MAP == MAP_POT) {
-    const float2 t =
-        add2_rn(make_float2(fminf(x.x, m.cap), fminf(x.y, m.cap)), make_float2(kMagic, kMagic));
-    // 2^-n * pscale from the exponent field: bits(t) = kMagicBits + n and
-    // kMagicBits << 23 == 0 (mod 2^32), so -(bits(t) << 23) == -(n << 23)
-    float2 w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + m.pow_bias),
-                           __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + m.pow_bias));
-    if (FLUSH) {
-      // t is kMagic + n exactly: n > floor  <=>  t > kMagic + floor
-      if (t.x > m.flush_t) w.x = 0.0f;
-      if (t.y > m.flush_t) w.y = 0.0f;
-    }
-    return w;
-  } else if (MAP == MAP_KI_HARD) {
-    // the clamp to [0, K] bounds the table index for every input (masked
-    // keys, ragged rows, near-degenerate rows, inf and NaN included)
-    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
-    const float2 t = add2_rn(u, make_float2(kMagic, kMagic));
-    return make_float2(lds_f32(__float_as_uint(t.x) * 512u + m.tab),
-                       lds_f32(__float_as_uint(t.y) * 512u + m.tab));
-  } else {
-    // interpolation as one FMA: w = g_k + (u - k) d_k = u d_k + c_k with
-    // c_k = g_k - k d_k; k = floor(u) in [0, K] (the clamp bounds the index)
-    // through a round-down add of 2^23; the table entry at k = K repeats
-    // k = K - 1, which is the interpolation's value at u = K
-    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
-    const float2 t = add2_rd(u, make_float2(8388608.0f, 8388608.0f));
-    const float2 c0 = lds_f32x2(__float_as_uint(t.x) * 1024u + m.tab);
-    const float2 c1 = lds_f32x2(__float_as_uint(t.y) * 1024u + m.tab);
-    return make_float2(__fmaf_rn(u.x, c0.y, c0.x), __fmaf_rn(u.y, c1.y, c1.x));
-  }
-}
-
-// Decision index of one element (debug dump only; same arithmetic).
-template <int MAP>
-__device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flush, int N) {
-  if (MAP == MAP_EXACT) return 0;
-  const float x = __fmaf_rn(r, m.a, m.b);
-  if (MAP == MAP_POT) {
-    const int n = static_cast<int>(__float_as_uint(__fadd_rn(fminf(x, m.cap), kMagic)) -
-                                   kMagicBits);
-    return (flush && n > N) ? -2 : n;
-  }
-  const float uc = fminf(fmaxf(x, 0.0f), m.Kf);
-  if (MAP == MAP_KI_HARD)
-    return static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
-  const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), m.Km1);
-  return static_cast<int>(kf);
-}
-
 // Weights of one 32-column chunk, packed for the PV MMA and stored to TMEM;
 // FULL: every column valid.  z holds eight partial row sums as four pairs.
 template <int MAP, bool FULL, bool FP8, bool FLUSH>
@@ -257,14 +156,7 @@ __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow 
                                           uint32_t taddr_pc) {
   auto wt = [&](int i) {          // weights of columns 2i, 2i+1
     const float2 r = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    float2 w = map_pair<MAP, FLUSH>(r, m);
-    if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
-      // fixed-window flush: coordinate below the window
-      if (flush_below) {
-        if (__fmaf_rn(r.x, m.a, m.b) < 0.0f) w.x = 0.0f;
-        if (__fmaf_rn(r.y, m.a, m.b) < 0.0f) w.y = 0.0f;
-      }
-    }
+    float2 w = pair_weights<MAP, FLUSH>(r, m, flush_below);
     if (!FULL) {
       w.x = (c0 + 2 * i < lim) ? w.x : 0.0f;
       w.y = (c0 + 2 * i + 1 < lim) ? w.y : 0.0f;
@@ -327,18 +219,6 @@ struct Xch {
 };
 constexpr size_t kXchBytes = kGroups * 128 * 16 + kGroups * 128 * 4;
 
-// Three-input fp32 maximum / minimum (one instruction on sm_100).
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float min3f(float a, float b, float c) {
-  float r;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // Scale this group's O columns, pack to bf16 and store the row's slice.
 template <int OC>
 __device__ __forceinline__ void o_store(uint32_t taddr, float oscale, __nv_bfloat16 *dst,
@@ -366,9 +246,8 @@ template <bool FULL, bool FP8>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], float cL2E, float mL2E, int c0,
                                           int lim, float2 (&z)[4], uint32_t taddr_pc) {
   auto e = [&](int i) {           // weights of columns 2i, 2i+1
-    const float2 x = fma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
-                             make_float2(cL2E, cL2E), make_float2(-mL2E, -mL2E));
-    float2 w = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+    float2 w = exact_pair(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                          cL2E, mL2E);
     if (!FULL) {
       w.x = (c0 + 2 * i < lim) ? w.x : 0.0f;
       w.y = (c0 + 2 * i + 1 < lim) ? w.y : 0.0f;
@@ -422,6 +301,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   bool ok = true;
   float rmax = -INFINITY, rmin = INFINITY;
   int amax = 0, amin = 0;
+  bool nan_seen = false;             // argument scan: a NaN score (comparisons skip it)
   const bool want_arg = p.amax != nullptr || p.amin != nullptr;
   const bool want_min =
       ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window) || p.lo != nullptr;
@@ -456,6 +336,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
             const int col = 128 * j + c_off + c0 + i;
             if (valid && x > rmax) { rmax = x; amax = col; }
             if (valid && x < rmin) { rmin = x; amin = col; }
+            nan_seen = nan_seen || (valid && x != x);
           }
         };
         scan(v0, 0);
@@ -465,11 +346,11 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
         for (int i = 0; i < 16; ++i) {
           const float a0 = __uint_as_float(v0[2 * i]), a1 = __uint_as_float(v0[2 * i + 1]);
           const float b0 = __uint_as_float(v1[2 * i]), b1 = __uint_as_float(v1[2 * i + 1]);
-          mx[i & 1] = max3f(mx[i & 1], a0, a1);
-          mx[2 + (i & 1)] = max3f(mx[2 + (i & 1)], b0, b1);
+          mx[i & 1] = max3n(mx[i & 1], a0, a1);
+          mx[2 + (i & 1)] = max3n(mx[2 + (i & 1)], b0, b1);
           if (want_min) {
-            mn[i & 1] = min3f(mn[i & 1], a0, a1);
-            mn[2 + (i & 1)] = min3f(mn[2 + (i & 1)], b0, b1);
+            mn[i & 1] = min3n(mn[i & 1], a0, a1);
+            mn[2 + (i & 1)] = min3n(mn[2 + (i & 1)], b0, b1);
           }
         }
       } else {
@@ -478,9 +359,9 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
           for (int i = 0; i < 16; ++i) {
             const float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
             const bool va = c0 + 2 * i < lim, vb = c0 + 2 * i + 1 < lim;
-            mx[k + (i & 1)] = max3f(mx[k + (i & 1)], va ? a0 : -INFINITY, vb ? a1 : -INFINITY);
+            mx[k + (i & 1)] = max3n(mx[k + (i & 1)], va ? a0 : -INFINITY, vb ? a1 : -INFINITY);
             if (want_min)
-              mn[k + (i & 1)] = min3f(mn[k + (i & 1)], va ? a0 : INFINITY, vb ? a1 : INFINITY);
+              mn[k + (i & 1)] = min3n(mn[k + (i & 1)], va ? a0 : INFINITY, vb ? a1 : INFINITY);
           }
         };
         red(v0, 0, 0);
@@ -492,8 +373,10 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
     // parity, whose phases may still be two or more behind)
     mbar_arrive(bars.st_done);
     if (!want_arg) {
-      rmax = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-      rmin = min3f(mn[0], mn[1], fminf(mn[2], mn[3]));
+      rmax = max3n(mx[0], mx[1], max3n(mx[2], mx[3], mx[3]));
+      rmin = min3n(mn[0], mn[1], min3n(mn[2], mn[3], mn[3]));
+    } else if (nan_seen) {
+      rmax = rmin = __int_as_float(0x7FFFFFFF);
     }
     // combine the four groups in a fixed order (ties: the lower key index), so
     // every group ends with the same row statistics
@@ -506,13 +389,19 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
       rmax = -INFINITY;
       rmin = INFINITY;
       amax = amin = 0;
+      bool nan_max = false, nan_min = false;
 #pragma unroll
       for (int gg = 0; gg < kGroups; ++gg) {
         const float4 o = xc.stats[gg * 128 + row];
         const int oamax = __float_as_int(o.z), oamin = __float_as_int(o.w);
         if (o.x > rmax || (o.x == rmax && oamax < amax)) { rmax = o.x; amax = oamax; }
         if (o.y < rmin || (o.y == rmin && oamin < amin)) { rmin = o.y; amin = oamin; }
+        nan_max = nan_max || o.x != o.x;
+        nan_min = nan_min || o.y != o.y;
       }
+      // a NaN score makes the row's statistics NaN (and its output NaN)
+      if (nan_max) rmax = __int_as_float(0x7FFFFFFF);
+      if (nan_min) rmin = __int_as_float(0x7FFFFFFF);
     }
   }
 
@@ -521,59 +410,25 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
 #pragma unroll
   for (int i = 0; i < 4; ++i) z[i] = make_float2(0.0f, 0.0f);
   float hi = 0.0f, lo = 0.0f;
-  MapRow mr;
-  mr.a = mr.b = 0.0f;
-  mr.cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
-  mr.Kf = static_cast<float>(p.K);
-  mr.Km1 = static_cast<float>(p.K - 1);
-  mr.tab = 0;
-  mr.pow_bias = __float_as_uint(p.pscale);
-  mr.flush_t = kMagic + static_cast<float>(p.pot_floor);
+  MapCall mc;
+  mc.K = p.K;
+  mc.fixed_window = p.fixed_window;
+  mc.flush = p.flush;
+  mc.pot_floor = p.pot_floor;
+  mc.c = p.c;
+  mc.cL2E = p.cL2E;
+  mc.window = p.window;
+  mc.pscale = p.pscale;
   const bool pot_flush = MAP == MAP_POT && p.flush;
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush &&
                            p.fixed_window;
-  const float mL2E = rmax * p.cL2E;                 // exact map: the anchor in log2 units
-  if (ok) {
-    hi = __fmul_rn(p.c, rmax);
-    lo = __fmul_rn(p.c, rmin);
-  }
-  if (MAP != MAP_EXACT && ok) {
-    RowMap rm = make_rowmap(hi, lo, p.K, p.fixed_window != 0, p.window);
-    if (MAP == MAP_POT) {
-      mr.a = -p.cL2E;
-      mr.b = rm.hiL2E;
-    } else {
-      mr.a = __fmul_rn(p.c, rm.inv);
-      mr.b = rm.b;
-      if (rm.degenerate) {           // every key sits at the top node
-        mr.a = 0.0f;
-        mr.b = mr.Kf;
-      }
-      lo = rm.lo;
-      const uint32_t tb = smem_u32(tab);
-      // the four groups build interleaved entries of this row's grid table
-      if (MAP == MAP_KI_HARD) {
-        for (int nn = g; nn <= p.K; nn += kGroups)
-          tab[nn * 128 + row] = grid_value(rm, p.K, nn) * p.pscale;
-        mr.tab = tb + row * 4 - kMagicBits * 512u;
-      } else {
-        // entries k = 0 .. K: (c_k, d_k) with d_k = g_{k+1} - g_k and
-        // c_k = g_k - k d_k; entry K repeats entry K - 1
-        for (int nn = g; nn <= p.K; nn += kGroups) {
-          const int k = nn < p.K ? nn : p.K - 1;
-          const float gk = grid_value(rm, p.K, k);
-          const float gk1 = grid_value(rm, p.K, k + 1);
-          const float d = __fsub_rn(gk1, gk) * p.pscale;
-          tab[(nn * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, gk * p.pscale);
-          tab[(nn * 128 + row) * 2 + 1] = d;
-        }
-        // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
-        mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
-      }
-      // the table is complete before any group reads it
-      mbar_arrive(bars.xstat);
-      ok = warp_all(mbar_wait(bars.xstat, 1, abort));
-    }
+  // the four groups build interleaved entries of this row's grid table
+  const MapRow mr = row_setup<MAP>(mc, rmax, rmin, tab, row, g, kGroups, hi, lo);
+  const float mL2E = mr.mL2E;                       // exact map: the anchor in log2 units
+  if ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && ok) {
+    // the table is complete before any group reads it
+    mbar_arrive(bars.xstat);
+    ok = warp_all(mbar_wait(bars.xstat, 1, abort));
   }
   int8_t *dbg_row = (p.dbg != nullptr && row_ok)
                         ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
@@ -634,12 +489,18 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   mbar_arrive(bars.xz);
   if (!warp_all(mbar_wait(bars.xz, 0, abort))) return;
   const float Z = (xc.zsum[row] + xc.zsum[128 + row]) + (xc.zsum[256 + row] + xc.zsum[384 + row]);
-  const float oscale = p.v_descale / Z;          // pscale cancels: P and Z both carry it
+  // a row whose maximum is NaN or +inf (or, for min-max calibration, whose
+  // minimum is -inf) has no defined weights: its O and LSE are NaN
+  const bool bad = !(fabsf(hi) <= 3.402823466e38f) ||
+                   ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && !p.fixed_window &&
+                    !(fabsf(lo) <= 3.402823466e38f));
+  const float qnan = __int_as_float(0x7FFFFFFF);
+  const float oscale = bad ? qnan : p.v_descale / Z;  // pscale cancels: P and Z both carry it
   o_store<OC>(lane_base + kOCol + g * OC, oscale,
               p.O + (static_cast<size_t>(bh) * p.S + qrow) * D + g * OC, row_ok);
   if (row_ok && g == 0) {
     const size_t ri = static_cast<size_t>(bh) * p.S + qrow;
-    p.LSE[ri] = hi + logf(Z / p.pscale);
+    p.LSE[ri] = bad ? qnan : hi + logf(Z / p.pscale);
     if (p.hi) p.hi[ri] = hi;
     if (p.lo) p.lo[ri] = lo;
     if (p.amax) p.amax[ri] = amax;

@@ -32,7 +32,8 @@ struct FwdArgs {
 qsm_status launch_fwd(const FwdArgs &a);
 
 struct MapArgs {
-  const float *scores;
+  const float *scores;     // raw products r; the score is c * r
+  float c;
   const int32_t *valid_len;
   int rows, cols;
   int mode, Kint, calib, rounding;

@@ -1,27 +1,43 @@
-// wmap.cuh -- the per-row weight maps on fp32 scores.
+// wmap.cuh -- the per-row weight maps, as the fused kernels evaluate them.
 //
 // K-interval attention ("Pretraining Transformers with Quantized Softmax in
 // Attention", abstract: exp approximated from K+1 grid values, per-row grid
 // calibration, interpolation versus hard rounding) and Rowmax-PoT
 // ("Approximating Softmax in Pretrained LLMs", abstract: power-of-two weights
-// anchored at each row maximum), in the library's fp32 operation order:
+// anchored at each row maximum), plus the exact map.  The fused forward and
+// the standalone map (qsm_weight_map) both call the functions below, so the
+// standalone map is a bit-exact window onto the forward's arithmetic.
 //
-//   PoT        x = fma(s, -log2e, hi*log2e); n = rne(min(x, cap)); w = 2^-n
-//   K-interval u = fma(s, inv, b) with inv = K/(hi-lo), b = -(lo*inv);
-//              uc = clamp(u, 0, K); hard: n = rne(uc), w = g[n];
-//              interp: k = min(floor(uc), K-1), f = uc - k,
-//                      w = fma(f, g[k+1] - g[k], g[k])
-//   grid       g[k] = own_exp(-(K-k) * step), step = (hi-lo)/K or W/K
+// Inputs are raw fp32 products r = q.k (the MMA accumulator); the score is
+// s = c r with c = scale * q_descale * k_descale, folded into one FMA:
 //
-// rne(x) = (x + 1.5*2^23) - 1.5*2^23.  Every operation is written with an
-// explicit round-to-nearest intrinsic, so the compiler cannot contract or
-// reorder it; the result is therefore reproducible bit for bit by any IEEE
-// fp32 implementation of the same sequence.
+//   row statistics  rmax, rmin over the valid r (NaN-propagating max / min);
+//                   hi = c*rmax, lo = c*rmin
+//   exact       x = fma(r, c*log2e, -(rmax * c*log2e));   w = ex2.approx(x)
+//   PoT         x = fma(r, -(c*log2e), hi*log2e); t = min(x, cap) + 1.5*2^23;
+//               n = bits(t) - bits(1.5*2^23); w = 2^-n from the exponent field
+//   K-interval  lc = lo (min-max) or hi - W; a = hi - lc; inv = K/a;
+//               x = fma(r, c*inv, -(lc*inv))  (x = K on a degenerate row);
+//               uc = min(max(x, 0), K)
+//               hard:   n = bits(uc + 1.5*2^23) - bits(1.5*2^23); w = g[n]
+//               interp: k = floor(uc) (a round-down add of 2^23), entry k of
+//                       (c_k, d_k) = (g_k - k d_k, g_{k+1} - g_k), entry K
+//                       repeating entry K-1; w = fma(uc, d_k, c_k)
+//   grid        g[k] = own_exp(-(K-k) * step), step = a/K or W/K
+//
+// Every operation is an explicit round-to-nearest (or round-down) intrinsic,
+// so the compiler can neither contract nor reorder it, and an IEEE fp32
+// restatement of the same sequence reproduces it bit for bit (the exact map's
+// ex2.approx excepted, which is the hardware's own approximation).
 #pragma once
 
 #include <cstdint>
 
+#include "sm100.cuh"
+
 namespace qsm {
+
+enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
 
 constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u;
@@ -57,7 +73,8 @@ __device__ __forceinline__ float own_exp(float x) {
   return __fmul_rn(p, __int_as_float((e + 127) << 23));
 }
 
-// Per-row constants of a map, computed once per row from its statistics.
+// Per-row constants of a K-interval grid, computed once per row from its
+// statistics (score units).
 struct RowMap {
   float hi;       // row max of s
   float lo;       // calibrated lower end (K-interval) / row min
@@ -68,7 +85,7 @@ struct RowMap {
   bool degenerate;
 };
 
-// hi, lo_obs: exact fp32 row max / min of s.
+// hi, lo_obs: fp32 row max / min of s.
 __device__ __forceinline__ RowMap make_rowmap(float hi, float lo_obs, int K, bool fixed_window,
                                               float window) {
   RowMap m;
@@ -90,42 +107,215 @@ __device__ __forceinline__ float grid_value(const RowMap &m, int K, int k) {
   return own_exp(__fmul_rn(-static_cast<float>(K - k), m.step));
 }
 
-// Rowmax-PoT: returns w and writes the exponent n (or -2 when flushed).
-// cap = N (clamp) or N + 1 (flush).
-__device__ __forceinline__ float pot_weight(float s, float hiL2E, float cap, int N, bool flush,
-                                            int &n_out) {
-  const float x = __fmaf_rn(s, -log2e_f(), hiL2E);
-  const float t = __fadd_rn(fminf(x, cap), kMagic);
-  const int n = static_cast<int>(__float_as_uint(t) - kMagicBits);
-  if (flush && n > N) {
-    n_out = -2;
-    return 0.0f;
+// ------------------------------------------------ packed fp32 pair arithmetic
+// sm_100 f32x2 instructions: two IEEE round-to-nearest (or round-down)
+// operations per instruction, the same results as the scalar forms.
+__device__ __forceinline__ uint64_t f2_bits(float2 a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a.x), "f"(a.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_from(uint64_t r) {
+  float2 a;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a.x), "=f"(a.y) : "l"(r));
+  return a;
+}
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return f2_from(r);
+}
+__device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(r);
+}
+__device__ __forceinline__ float2 add2_rd(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(r);
+}
+
+// NaN-propagating fp32 maximum / minimum of three (one instruction on
+// sm_100): a row with a NaN score gets NaN statistics.
+__device__ __forceinline__ float max3n(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3n(float a, float b, float c) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// ------------------------------------------------------------ fused map
+// Per-row constants of the fused map, with the score scale folded in: the
+// map consumes the raw fp32 accumulator r of the QK product.
+//   PoT:        x = fma(r, -c*log2e, hi*log2e), w = 2^-rne(min(x, cap)) * pscale
+//   K-interval: x = fma(r, c*K/(hi-lo), -lo*K/(hi-lo)); hard: g[rne(x)];
+//               interpolation: u d_k + c_k at k = floor(u) (grid values
+//               pre-multiplied by pscale)
+//   exact:      x = fma(r, c*log2e, -mL2E), w = 2^x
+struct MapRow {
+  float a, b;        // coordinate = fma(r, a, b)
+  float cap, Kf, Km1;
+  float flush_t;     // PoT flush: kMagic + floor (t above it: exponent past the floor)
+  float mL2E;        // exact map: the anchor rmax * c * log2e
+  uint32_t tab;      // shared address bias of this row's table column
+  uint32_t pow_bias; // bits of pscale (PoT)
+};
+
+// Constants of one call of a map.
+struct MapCall {
+  int K;
+  int fixed_window;
+  int flush;        // below_policy == 1
+  int pot_floor;
+  float c;          // score scale
+  float cL2E;       // c * log2(e)
+  float window;
+  float pscale;     // weights are produced as w * pscale (FP8 P: 64)
+};
+
+// Grid table layout: node n of the row in table column `row` (0..127) sits at
+// float offset n*128 + row (hard rounding: g_n * pscale) or float2 offset
+// n*128 + row (interpolation: (c_n, d_n) * pscale), n = 0..K.  Bytes needed:
+// (K+1) * 128 * 4 (hard) or * 8 (interpolation).
+__host__ __device__ constexpr int table_bytes_for(int map, int K) {
+  return map == MAP_KI_HARD ? (K + 1) * 128 * 4 : (map == MAP_KI_INTERP ? (K + 1) * 128 * 8 : 0);
+}
+
+// Set up the map constants of one row from its raw statistics and write
+// table entries n = n0, n0 + nstep, ... (<= K) of its grid column.  The
+// caller makes the whole column visible before any map_pair on it.  Writes
+// the row's hi (c*rmax) and calibrated lower end (K-interval) or row min.
+template <int MAP>
+__device__ __forceinline__ MapRow row_setup(const MapCall &mc, float rmax, float rmin, float *tab,
+                                            int row, int n0, int nstep, float &hi, float &lo) {
+  MapRow mr;
+  mr.a = mr.b = 0.0f;
+  mr.cap = static_cast<float>(mc.flush ? mc.pot_floor + 1 : mc.pot_floor);
+  mr.Kf = static_cast<float>(mc.K);
+  mr.Km1 = static_cast<float>(mc.K - 1);
+  mr.tab = 0;
+  mr.pow_bias = __float_as_uint(mc.pscale);
+  mr.flush_t = kMagic + static_cast<float>(mc.pot_floor);
+  mr.mL2E = __fmul_rn(rmax, mc.cL2E);
+  hi = __fmul_rn(mc.c, rmax);
+  lo = __fmul_rn(mc.c, rmin);
+  if (MAP == MAP_EXACT) return mr;
+  const RowMap rm = make_rowmap(hi, lo, mc.K, mc.fixed_window != 0, mc.window);
+  if (MAP == MAP_POT) {
+    mr.a = -mc.cL2E;
+    mr.b = rm.hiL2E;
+    return mr;
   }
-  n_out = n;
-  return __uint_as_float(0x3F800000u - (static_cast<uint32_t>(n) << 23));
+  mr.a = __fmul_rn(mc.c, rm.inv);
+  mr.b = rm.b;
+  if (rm.degenerate) {           // every key sits at the top node
+    mr.a = 0.0f;
+    mr.b = mr.Kf;
+  }
+  lo = rm.lo;
+  const uint32_t tb = smem_u32(tab);
+  if (MAP == MAP_KI_HARD) {
+    for (int nn = n0; nn <= mc.K; nn += nstep)
+      tab[nn * 128 + row] = __fmul_rn(grid_value(rm, mc.K, nn), mc.pscale);
+    // bits(rne(u) + kMagic) = kMagicBits + n  ->  table row n
+    mr.tab = tb + row * 4 - kMagicBits * 512u;
+  } else {
+    // entries k = 0 .. K: (c_k, d_k) with d_k = g_{k+1} - g_k and
+    // c_k = g_k - k d_k; entry K repeats entry K - 1
+    for (int nn = n0; nn <= mc.K; nn += nstep) {
+      const int k = nn < mc.K ? nn : mc.K - 1;
+      const float gk = grid_value(rm, mc.K, k);
+      const float gk1 = grid_value(rm, mc.K, k + 1);
+      const float d = __fmul_rn(__fsub_rn(gk1, gk), mc.pscale);
+      tab[(nn * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, __fmul_rn(gk, mc.pscale));
+      tab[(nn * 128 + row) * 2 + 1] = d;
+    }
+    // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
+    mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
+  }
+  return mr;
 }
 
-// K-interval grid coordinate before clamping.
-__device__ __forceinline__ float kint_u(float s, const RowMap &m, float Kf) {
-  return m.degenerate ? Kf : __fmaf_rn(s, m.inv, m.b);
+// Weights of two scores (the map's arithmetic on a pair; FLUSH: Rowmax-PoT
+// with the below-floor policy "flush", exponents above the floor give 0).
+template <int MAP, bool FLUSH>
+__device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
+  const float2 x = fma2_rn(r, make_float2(m.a, m.a), make_float2(m.b, m.b));
+  if (MAP == MAP_POT) {
+    const float2 t =
+        add2_rn(make_float2(fminf(x.x, m.cap), fminf(x.y, m.cap)), make_float2(kMagic, kMagic));
+    // 2^-n * pscale from the exponent field: bits(t) = kMagicBits + n and
+    // kMagicBits << 23 == 0 (mod 2^32), so -(bits(t) << 23) == -(n << 23)
+    float2 w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + m.pow_bias),
+                           __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + m.pow_bias));
+    if (FLUSH) {
+      // t is kMagic + n exactly: n > floor  <=>  t > kMagic + floor
+      if (t.x > m.flush_t) w.x = 0.0f;
+      if (t.y > m.flush_t) w.y = 0.0f;
+    }
+    return w;
+  } else if (MAP == MAP_KI_HARD) {
+    // the clamp to [0, K] bounds the table index for every input (masked
+    // keys, ragged rows, near-degenerate rows, inf and NaN included)
+    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
+    const float2 t = add2_rn(u, make_float2(kMagic, kMagic));
+    return make_float2(lds_f32(__float_as_uint(t.x) * 512u + m.tab),
+                       lds_f32(__float_as_uint(t.y) * 512u + m.tab));
+  } else {
+    // interpolation as one FMA: w = g_k + (u - k) d_k = u d_k + c_k with
+    // c_k = g_k - k d_k; k = floor(u) in [0, K] (the clamp bounds the index)
+    // through a round-down add of 2^23; the table entry at k = K repeats
+    // k = K - 1, which is the interpolation's value at u = K
+    const float2 u = make_float2(fminf(fmaxf(x.x, 0.0f), m.Kf), fminf(fmaxf(x.y, 0.0f), m.Kf));
+    const float2 t = add2_rd(u, make_float2(8388608.0f, 8388608.0f));
+    const float2 c0 = lds_f32x2(__float_as_uint(t.x) * 1024u + m.tab);
+    const float2 c1 = lds_f32x2(__float_as_uint(t.y) * 1024u + m.tab);
+    return make_float2(__fmaf_rn(u.x, c0.y, c0.x), __fmaf_rn(u.y, c1.y, c1.x));
+  }
 }
 
-// Hard rounding: nearest node of the clamped coordinate.
-__device__ __forceinline__ int kint_hard_node(float u, float Kf) {
-  const float uc = fminf(fmaxf(u, 0.0f), Kf);
-  return static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+// Weights of a pair with the K-interval fixed-window flush (coordinate below
+// the window -> 0) applied when flush_below.
+template <int MAP, bool FLUSH>
+__device__ __forceinline__ float2 pair_weights(float2 r, const MapRow &m, bool flush_below) {
+  float2 w = map_pair<MAP, FLUSH>(r, m);
+  if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
+    if (flush_below) {
+      if (__fmaf_rn(r.x, m.a, m.b) < 0.0f) w.x = 0.0f;
+      if (__fmaf_rn(r.y, m.a, m.b) < 0.0f) w.y = 0.0f;
+    }
+  }
+  return w;
 }
 
-// Interpolation: lower node k and fraction f of the clamped coordinate.
-__device__ __forceinline__ int kint_interp_node(float u, float Kf, float &f) {
-  const float uc = fminf(fmaxf(u, 0.0f), Kf);
-  const float kf = fminf(floorf(uc), __fsub_rn(Kf, 1.0f));
-  f = __fsub_rn(uc, kf);
-  return static_cast<int>(__float_as_uint(__fadd_rn(kf, kMagic)) - kMagicBits);
+// Exact weights of a pair against the anchor mL2E (log2 units).
+__device__ __forceinline__ float2 exact_pair(float2 r, float cL2E, float mL2E) {
+  const float2 x = fma2_rn(r, make_float2(cL2E, cL2E), make_float2(-mL2E, -mL2E));
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
-__device__ __forceinline__ float kint_interp_weight(float f, float g0, float g1) {
-  return __fmaf_rn(f, __fsub_rn(g1, g0), g0);
+// Decision index of one element (debug dump and the standalone map; the same
+// arithmetic as map_pair): PoT exponent (-2 flushed), hard node, lower node of
+// the interpolation, 0 for the exact map.
+template <int MAP>
+__device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flush, int N) {
+  if (MAP == MAP_EXACT) return 0;
+  const float x = __fmaf_rn(r, m.a, m.b);
+  if (MAP == MAP_POT) {
+    const int n = static_cast<int>(__float_as_uint(__fadd_rn(fminf(x, m.cap), kMagic)) -
+                                   kMagicBits);
+    return (flush && n > N) ? -2 : n;
+  }
+  const float uc = fminf(fmaxf(x, 0.0f), m.Kf);
+  if (MAP == MAP_KI_HARD)
+    return static_cast<int>(__float_as_uint(__fadd_rn(uc, kMagic)) - kMagicBits);
+  const float kf = fminf(__fsub_rn(__fadd_rd(uc, 8388608.0f), 8388608.0f), m.Km1);
+  return static_cast<int>(kf);
 }
 
 }  // namespace qsm

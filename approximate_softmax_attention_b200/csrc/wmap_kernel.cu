@@ -1,8 +1,14 @@
-// wmap_kernel.cu -- the weight map alone on given fp32 scores (the maps'
-// bit-exact test surface).  One warp per row: the row's max / min come from a
-// warp reduction (exact in fp32 whatever the order), the grid values from the
-// library's own exp, and every element goes through the same device functions
-// the fused forward uses (wmap.cuh).
+// wmap_kernel.cu -- the weight map alone on given fp32 raw products (the
+// maps' bit-exact test surface).
+//
+// It runs the fused forward's own device functions (wmap.cuh): row_setup
+// for the per-row constants and grid table, pair_weights / exact_pair for the
+// weights and map_raw_index for the decision index, on raw products r with
+// the score scale c folded in exactly as the forward folds it.  One thread
+// per row (the table layout keeps one column per row of a 128-row block),
+// columns taken in pairs as the forward takes them; the row statistics come
+// from a sequential NaN-propagating max / min, exact in fp32 whatever the
+// order.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -12,82 +18,90 @@
 
 namespace qsm {
 
-__global__ void __launch_bounds__(256)
-    qsm_weight_map_kernel(const float *__restrict__ s, const int32_t *__restrict__ vlen, int rows,
-                          int cols, int mode, int K, int fixed_window, int hard, float window,
-                          int pot_floor, int flush, float *__restrict__ w,
-                          int32_t *__restrict__ idx, float *__restrict__ hi_out,
-                          float *__restrict__ lo_out) {
-  extern __shared__ float tab[];                       // [warps][K+1]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (r >= rows) return;
-  const float *sr = s + static_cast<size_t>(r) * cols;
+namespace {
+
+constexpr int kRowsPerBlock = 128;
+
+template <int MAP, bool FLUSH>
+__global__ void __launch_bounds__(kRowsPerBlock)
+    qsm_weight_map_kernel(const float *__restrict__ r_in, const int32_t *__restrict__ vlen,
+                          int rows, int cols, MapCall mc, int below_flush,
+                          float *__restrict__ w, int32_t *__restrict__ idx,
+                          float *__restrict__ hi_out, float *__restrict__ lo_out) {
+  extern __shared__ float tab[];                       // [K+1][128] entries
+  const int row = threadIdx.x;
+  const int r = blockIdx.x * kRowsPerBlock + row;
+  if (r >= rows) return;                               // no block-wide barrier below
+  const float *rr = r_in + static_cast<size_t>(r) * cols;
   float *wr = w + static_cast<size_t>(r) * cols;
   int32_t *ir = idx ? idx + static_cast<size_t>(r) * cols : nullptr;
   int L = vlen[r];
   L = L < 1 ? 1 : (L > cols ? cols : L);
-  float hi = -INFINITY, lo = INFINITY;
-  for (int j = lane; j < L; j += 32) {
-    hi = fmaxf(hi, sr[j]);
-    lo = fminf(lo, sr[j]);
+  float rmax = -INFINITY, rmin = INFINITY;
+  for (int j = 0; j < L; ++j) {
+    rmax = max3n(rmax, rr[j], rr[j]);
+    rmin = min3n(rmin, rr[j], rr[j]);
   }
-  for (int o = 16; o > 0; o >>= 1) {
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-  }
-  float *g = tab + warp * (K + 1);
-  RowMap m = make_rowmap(hi, lo, K, fixed_window != 0, window);
-  if (mode == QSM_MODE_KINTERVAL) {
-    for (int k = lane; k <= K; k += 32) g[k] = grid_value(m, K, k);
-    __syncwarp();
-  }
-  const float Kf = static_cast<float>(K);
-  const float cap = static_cast<float>(flush ? pot_floor + 1 : pot_floor);
-  for (int j = lane; j < cols; j += 32) {
-    float wj = 0.0f;
-    int n = -1;
-    if (j < L) {
-      const float x = sr[j];
-      if (mode == QSM_MODE_EXACT) {
-        wj = own_exp(__fsub_rn(x, hi));
-        n = 0;
-      } else if (mode == QSM_MODE_ROWMAX_POT) {
-        wj = pot_weight(x, m.hiL2E, cap, pot_floor, flush != 0, n);
-      } else {
-        const float u = kint_u(x, m, Kf);
-        if (flush && fixed_window && u < 0.0f) {
-          wj = 0.0f;
-          n = -2;
-        } else if (hard) {
-          n = kint_hard_node(u, Kf);
-          wj = g[n];
-        } else {
-          float f;
-          n = kint_interp_node(u, Kf, f);
-          wj = kint_interp_weight(f, g[n], g[n + 1]);
-        }
+  float hi, lo;
+  // this thread owns table column `row` and writes all of it
+  const MapRow mr = row_setup<MAP>(mc, rmax, rmin, tab, row, 0, 1, hi, lo);
+  const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && below_flush != 0;
+  for (int j = 0; j < cols; j += 2) {
+    const bool v0 = j < L, v1 = j + 1 < L;
+    const float2 x = make_float2(rr[j], j + 1 < cols ? rr[j + 1] : 0.0f);
+    float2 wt;
+    if (MAP == MAP_EXACT)
+      wt = exact_pair(x, mc.cL2E, mr.mL2E);
+    else
+      wt = pair_weights<MAP, FLUSH>(x, mr, flush_below);
+    wr[j] = v0 ? wt.x : 0.0f;
+    if (j + 1 < cols) wr[j + 1] = v1 ? wt.y : 0.0f;
+    if (ir) {
+      for (int e = 0; e < 2 && j + e < cols; ++e) {
+        const float xe = e ? x.y : x.x;
+        int n = map_raw_index<MAP>(xe, mr, mc.flush != 0, mc.pot_floor);
+        if (flush_below && __fmaf_rn(xe, mr.a, mr.b) < 0.0f) n = -2;
+        ir[j + e] = (j + e < L) ? n : -1;
       }
     }
-    wr[j] = wj;
-    if (ir) ir[j] = n;
   }
-  if (lane == 0) {
-    if (hi_out) hi_out[r] = hi;
-    if (lo_out) lo_out[r] = (mode == QSM_MODE_KINTERVAL) ? m.lo : lo;
-  }
+  if (hi_out) hi_out[r] = hi;
+  if (lo_out) lo_out[r] = lo;
 }
 
-qsm_status launch_weight_map(const MapArgs &a) {
-  const int K = a.mode == QSM_MODE_KINTERVAL ? a.Kint : 1;
-  const int warps = 8;
-  const dim3 grid((a.rows + warps - 1) / warps);
-  const size_t smem = static_cast<size_t>(warps) * (K + 1) * sizeof(float);
-  qsm_weight_map_kernel<<<grid, warps * 32, smem, a.stream>>>(
-      a.scores, a.valid_len, a.rows, a.cols, a.mode, K, a.calib == QSM_CALIB_FIXED_WINDOW,
-      a.rounding == QSM_ROUND_HARD, a.window, a.pot_floor, a.below_policy == 1, a.w, a.idx, a.hi,
-      a.lo);
+template <int MAP, bool FLUSH>
+qsm_status launch_map_t(const MapArgs &a, const MapCall &mc) {
+  const size_t smem = static_cast<size_t>(table_bytes_for(MAP, mc.K));
+  auto kern = qsm_weight_map_kernel<MAP, FLUSH>;
+  // the largest table (interpolation, K = 64) needs 66.5 KB
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return QSM_ERR_CUDA;
+  const dim3 grid((a.rows + kRowsPerBlock - 1) / kRowsPerBlock);
+  kern<<<grid, kRowsPerBlock, smem, a.stream>>>(
+      a.scores, a.valid_len, a.rows, a.cols, mc,
+      a.below_policy == 1 && a.calib == QSM_CALIB_FIXED_WINDOW, a.w, a.idx, a.hi, a.lo);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+}
+
+}  // namespace
+
+qsm_status launch_weight_map(const MapArgs &a) {
+  MapCall mc;
+  mc.K = a.mode == QSM_MODE_KINTERVAL ? a.Kint : 1;
+  mc.fixed_window = a.calib == QSM_CALIB_FIXED_WINDOW;
+  mc.flush = a.below_policy == 1;
+  mc.pot_floor = a.pot_floor;
+  mc.c = a.c;
+  mc.cL2E = a.c * 1.4426950408889634f;
+  mc.window = a.window;
+  mc.pscale = 1.0f;
+  if (a.mode == QSM_MODE_EXACT) return launch_map_t<MAP_EXACT, false>(a, mc);
+  if (a.mode == QSM_MODE_ROWMAX_POT)
+    return mc.flush ? launch_map_t<MAP_POT, true>(a, mc) : launch_map_t<MAP_POT, false>(a, mc);
+  if (a.rounding == QSM_ROUND_HARD) return launch_map_t<MAP_KI_HARD, false>(a, mc);
+  return launch_map_t<MAP_KI_INTERP, false>(a, mc);
 }
 
 }  // namespace qsm

@@ -55,7 +55,9 @@ typedef enum {
 /* The weight map.
  *  EXACT:      w = exp(s - hi), i.e. softmax (the pages' reference path, the
  *              "old path" through the special-function unit in the wiki
- *              flowchart).  Evaluated with online rescaling.
+ *              flowchart).  Evaluated in two sweeps like the other maps: a
+ *              statistics sweep finds the row maximum, then the weights are
+ *              taken against it (no rescaling of O).
  *  KINTERVAL:  "approximates the exponential using K+1 grid values" (arXiv
  *              2609.33591, abstract).  Grid over [lo, hi] of the row's scores,
  *              step Delta = (hi - lo)/K, grid values g_k = exp(-(K-k) Delta);
@@ -172,9 +174,13 @@ size_t qsm_attn_bwd_workspace_size(int B, int H, int S, int D);
  * (for D = 64, about 30 000 query rows B*H*S), before any launch.
  *
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
- * Every call uses the same array, so calls whose work overlaps on a GPU
- * (different streams or host threads) race; serialise them. */
+ * that device current); make that first call before any stream capture.  The
+ * address is kept for the driver context current at that first call; a call
+ * under another context (after cudaDeviceReset, or with a non-primary
+ * context current) looks it up again, so make such a call before any capture
+ * as well.  Every call uses the same array, so calls whose work overlaps on a
+ * GPU (different streams or host threads) race; serialise them.  D outside
+ * {64, 128} returns QSM_ERR_UNSUPPORTED, as qsm_attn_bwd does. */
 qsm_status qsm_attn_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O,
                                 const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
                                 int B, int H, int S, int D, int causal, qsm_mode mode, int Kint,
@@ -182,17 +188,24 @@ qsm_status qsm_attn_bwd_noalloc(const void *Q, const void *K, const void *V, con
                                 qsm_surrogate surrogate, const qsm_opts *opts,
                                 qsm_stream_t stream);
 
-/* The weight map alone on given fp32 scores (bit-exact with the library's
- * fp32 specification of the maps).
- *  scores:    device [rows, cols] fp32.
+/* The weight map alone, on given fp32 raw products, through the fused
+ * forward's own per-element map code (row set-up, grid table, pair
+ * arithmetic, decision index): the bit-exact window onto the forward's
+ * weights.  The score of a product r is s = c * r with
+ * c = (opts->scale, or 1 when opts->scale is 0) * q_descale * k_descale,
+ * folded into one fused multiply-add exactly as the forward folds it.
+ * The exact map's 2^x is the hardware's approximate instruction (not
+ * bit-reproducible elsewhere); the other maps are.
+ *  scores:    device [rows, cols] fp32 raw products r.
  *  valid_len: device [rows] int32; keys 0..valid_len[r]-1 of row r are valid
  *             (1 <= valid_len[r] <= cols).
  *  w:         device [rows, cols] fp32 (written; 0 where masked).
  *  idx:       device [rows, cols] int32 (written; decision index as in
  *             opts->debug_idx), may be NULL.
- *  hi, lo:    device [rows] fp32 (written: row max; calibrated lower end for
- *             K-interval, row min otherwise), may be NULL.
- *  Uses opts->window, pot_floor, below_policy. */
+ *  hi, lo:    device [rows] fp32 (written: c * row max of r; calibrated lower
+ *             end for K-interval, c * row min otherwise), may be NULL.  A NaN
+ *             among a row's valid products makes both NaN.
+ *  Uses opts->scale, q_descale, k_descale, window, pot_floor, below_policy. */
 qsm_status qsm_weight_map(const float *scores, const int32_t *valid_len, int rows, int cols,
                           qsm_mode mode, int Kint, qsm_calib calibration,
                           qsm_rounding rounding, const qsm_opts *opts, float *w,

@@ -119,17 +119,31 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
     R, S = s.shape
     out = dict(hi=hi, lo=lo, argmax=amax, argmin=amin)
     idx = np.full((R, S), IDX_MASKED, dtype=np.int64)
+    # Non-finite scores (possible only with non-finite inputs): a row whose
+    # maximum is NaN or +inf, or (min-max calibration) whose minimum is -inf,
+    # has no defined weights and gets NaN ones; a -inf score in any other row
+    # takes the map's limit at s -> -inf (0, the PoT floor, or the clamp to
+    # the lowest grid value / the flush).
+    bad = ~np.isfinite(hi)
+    if mode == KINTERVAL and calib == MINMAX:
+        bad = bad | ~np.isfinite(lo)
+    badr = bad[:, None] & valid
     if mode == EXACT:
-        w = np.where(valid, np.exp(np.where(valid, s, 0.0) - hi[:, None]), 0.0)
+        with np.errstate(invalid="ignore"):
+            w = np.where(valid, np.exp(np.where(valid, s, 0.0) - hi[:, None]), 0.0)
+        w = np.where(badr, np.nan, w)
         idx[valid] = 0
         out.update(w=w, idx=idx, lo_cal=lo)
         return out
     if mode == ROWMAX_POT:
-        x = (hi[:, None] - np.where(valid, s, hi[:, None])) * LOG2E
+        with np.errstate(invalid="ignore"):
+            x = (hi[:, None] - np.where(valid, s, hi[:, None])) * LOG2E
+        x = np.where(badr, 0.0, x)
         n = np.rint(x)                               # round half to even
         flushed = valid & (n > pot_floor) if below_policy == 1 else np.zeros_like(valid)
         n = np.minimum(n, pot_floor)
         w = np.where(valid & ~flushed, np.exp2(-n), 0.0)
+        w = np.where(badr, np.nan, w)
         idx[valid] = n[valid].astype(np.int64)
         idx[flushed] = IDX_FLUSHED
         out.update(w=w, idx=idx, x=x, lo_cal=lo)
@@ -137,13 +151,14 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
     if mode != KINTERVAL:
         raise ValueError("unknown mode %r" % (mode,))
     lo_cal = lo if calib == MINMAX else hi - window
-    a = hi - lo_cal
-    delta = a / K
+    with np.errstate(invalid="ignore"):
+        a = hi - lo_cal
+    delta = np.where(bad, 1.0, a / K)
     g = kint_grid(K, delta)
-    degenerate = ~(a > 0)
+    degenerate = ~(a > 0) & ~bad
     with np.errstate(divide="ignore", invalid="ignore"):
         u_raw = (s - lo_cal[:, None]) / delta[:, None]
-    u_raw = np.where(degenerate[:, None], float(K), u_raw)
+    u_raw = np.where(degenerate[:, None] | bad[:, None], float(K), u_raw)
     u_raw = np.where(valid, u_raw, float(K))
     below = valid & (u_raw < 0)
     u = np.clip(u_raw, 0.0, float(K))
@@ -165,6 +180,7 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
         raise ValueError("unknown rounding %r" % (rounding,))
     flushed = below if (below_policy == 1 and calib == FIXED_WINDOW) else np.zeros_like(valid)
     w = np.where(valid & ~flushed, w, 0.0)
+    w = np.where(badr, np.nan, w)
     idx[valid] = kidx[valid]
     idx[flushed] = IDX_FLUSHED
     out.update(w=w, idx=idx, u=u, kidx=kidx, f=f, g=g, a=a, delta=delta,

@@ -2,8 +2,9 @@
  * fp32 weight-map specification, restated in plain C.
  *
  * TEST INFRASTRUCTURE ONLY: only tests/ (through oracle/spec.py) load this.
- * It shares no code with the CUDA path; the GPU map must reproduce its output
- * bit for bit on the same fp32 scores.
+ * It shares no code with the CUDA path; the GPU map (the fused forward's own
+ * per-element arithmetic, exposed as qsm_weight_map) must reproduce its
+ * output bit for bit on the same fp32 inputs.
  *
  * Compile with -O2 -ffp-contract=off and without -ffast-math: every a*b+c
  * below is two correctly rounded operations unless written as fmaf().
@@ -13,22 +14,29 @@
  * values, per-row calibration, interpolation vs hard rounding; "Approximating
  * Softmax in Pretrained LLMs", abstract: Rowmax-PoT, power-of-two weights
  * anchored at the row maximum).  The fp32 operation order is this library's
- * own specification (the pages fix none):
+ * own specification (the pages fix none).  Inputs are raw products r = q.k;
+ * the score is s = c*r with the scale c folded into one fused multiply-add:
  *
- *   hi = max s, lo_obs = min s over the valid keys (exact in fp32)
- *   EXACT      w = spec_exp(s - hi)
- *   ROWMAX_POT x = fmaf(s, -L2E, hi*L2E);  n = rne(min(x, N))  (clamp)
- *              or n = rne(min(x, N+1)), flushed when n > N      (flush)
+ *   rmax, rmin = max / min of r over the valid keys (a NaN propagates)
+ *   hi = c*rmax, lo_obs = c*rmin, cl2e = c*L2E
+ *   EXACT      x = fmaf(r, cl2e, -(rmax*cl2e)); w = 2^x  (the GPU evaluates
+ *              2^x with its approximate hardware instruction, so for EXACT
+ *              this file returns x, not w)
+ *   ROWMAX_POT x = fmaf(r, -cl2e, hi*L2E); n = rne(min(x, cap)) with
+ *              cap = N (clamp) or N+1 (flush, n > N gives w = 0);
  *              w = 2^-n built from exponent bits
- *   KINTERVAL  lo = lo_obs (min-max) or hi - W (fixed-window)
- *              a = hi - lo; degenerate when !(a > 0): u = K
- *              inv = K / a; b = -(lo*inv); u = fmaf(s, inv, b)
- *              flushed when below_policy == 1, fixed-window and u < 0
- *              uc = min(max(u, 0), K)
- *              step = a / K (min-max) or W / K (fixed-window)
- *              g[k] = spec_exp(-(K-k) * step), d[k] = g[k+1] - g[k]
+ *   KINTERVAL  lc = lo_obs (min-max) or hi - W (fixed-window); a = hi - lc;
+ *              degenerate when !(a > 0): coordinate x = K for every key;
+ *              else inv = K/a, b = -(lc*inv), x = fmaf(r, c*inv, b);
+ *              flushed when below_policy == 1, fixed-window and x < 0;
+ *              uc = min(max(x, 0), K);
+ *              step = a/K (min-max) or W/K (fixed-window),
+ *              g[k] = spec_exp(-(K-k) * step);
  *              hard   n = rne(uc), w = g[n]
- *              interp k = min(floor(uc), K-1), f = uc - k, w = fmaf(f, d[k], g[k])
+ *              interp k = floor(uc) (0..K); the table entry of node k holds
+ *                     d = g[k'+1] - g[k'] and e = fmaf(-k', d, g[k']) with
+ *                     k' = min(k, K-1); w = fmaf(uc, d, e); the decision
+ *                     index reported is k'
  *   rne(x) = (x + 1.5*2^23) - 1.5*2^23  (round half to even, |x| < 2^22)
  *
  *   spec_exp(x): Cody-Waite reduction x = n*ln2 + r with n = rne(x*log2 e),
@@ -75,39 +83,43 @@ float spec_exp(float x) {
     return p * bits2f((uint32_t)(e + 127) << 23);
 }
 
+/* NaN-propagating maximum / minimum (a NaN operand gives NaN). */
+static float nmax(float a, float b) { return (a != a || b != b) ? NAN : (b > a ? b : a); }
+static float nmin(float a, float b) { return (a != a || b != b) ? NAN : (b < a ? b : a); }
+
 /*
- * Map `rows` rows of `cols` fp32 scores.  valid_len[r] keys (a prefix) are
- * valid in row r.  Outputs w [rows*cols] (0 where masked) and idx
- * [rows*cols] (node / lower node / exponent; -1 masked, -2 flushed), and the
- * per-row hi and lo (lo = the calibrated lower end for K-interval, the observed
- * minimum otherwise).
+ * Map `rows` rows of `cols` raw products with score scale c.  valid_len[r]
+ * keys (a prefix) are valid in row r.  Outputs w [rows*cols] (0 where masked;
+ * for EXACT the exponent x of 2^x, see above) and idx [rows*cols] (node /
+ * lower node / exponent; -1 masked, -2 flushed), and the per-row hi = c*rmax
+ * and lo (the calibrated lower end for K-interval, c*rmin otherwise).
  */
-void spec_map_rows(const float *s, int rows, int cols, const int *valid_len,
+void spec_map_rows(const float *rin, int rows, int cols, const int *valid_len, float c,
                    int mode, int K, int calib, int rounding, float window,
                    int pot_floor, int below_policy, float *w, int *idx,
                    float *hi_out, float *lo_out) {
-    float g[257], d[257];
+    float g[130];
+    float cl2e = c * L2E;
     for (int r = 0; r < rows; ++r) {
-        const float *sr = s + (size_t)r * cols;
+        const float *rr = rin + (size_t)r * cols;
         float *wr = w + (size_t)r * cols;
         int *ir = idx + (size_t)r * cols;
         int L = valid_len[r];
-        float hi = -INFINITY, lo = INFINITY;
-        for (int j = 0; j < L; ++j) {
-            if (sr[j] > hi) hi = sr[j];
-            if (sr[j] < lo) lo = sr[j];
-        }
+        float rmax = -INFINITY, rmin = INFINITY;
+        for (int j = 0; j < L; ++j) { rmax = nmax(rmax, rr[j]); rmin = nmin(rmin, rr[j]); }
+        float hi = c * rmax, lo = c * rmin;
         for (int j = L; j < cols; ++j) { wr[j] = 0.0f; ir[j] = -1; }
         if (mode == MODE_EXACT) {
-            for (int j = 0; j < L; ++j) { wr[j] = spec_exp(sr[j] - hi); ir[j] = 0; }
+            float m = rmax * cl2e;
+            for (int j = 0; j < L; ++j) { wr[j] = fmaf(rr[j], cl2e, -m); ir[j] = 0; }
         } else if (mode == MODE_POT) {
-            float hl = hi * L2E;
+            float b = hi * L2E;
             float cap = below_policy ? (float)(pot_floor + 1) : (float)pot_floor;
             for (int j = 0; j < L; ++j) {
-                float x = fmaf(sr[j], -L2E, hl);
+                float x = fmaf(rr[j], -cl2e, b);
                 float t = fminf(x, cap) + MAGIC;
                 int32_t n = (int32_t)f2bits(t) - (int32_t)f2bits(MAGIC);
-                if (n > pot_floor) { wr[j] = 0.0f; ir[j] = -2; continue; }
+                if (below_policy && n > pot_floor) { wr[j] = 0.0f; ir[j] = -2; continue; }
                 wr[j] = bits2f((uint32_t)(127 - n) << 23);
                 ir[j] = n;
             }
@@ -118,25 +130,27 @@ void spec_map_rows(const float *s, int rows, int cols, const int *valid_len,
             float Kf = (float)K;
             float step = (calib == CAL_MINMAX) ? a / Kf : window / Kf;
             for (int k = 0; k <= K; ++k) g[k] = spec_exp(-(float)(K - k) * step);
-            for (int k = 0; k < K; ++k) d[k] = g[k + 1] - g[k];
             float inv = degenerate ? 0.0f : Kf / a;
             float b = -(lc * inv);
+            float ca = c * inv;
+            if (degenerate) { ca = 0.0f; b = Kf; }
             lo = lc;
             for (int j = 0; j < L; ++j) {
-                float u = degenerate ? Kf : fmaf(sr[j], inv, b);
-                if (below_policy == 1 && calib == CAL_FIXED && u < 0.0f) {
+                float x = fmaf(rr[j], ca, b);
+                if (below_policy == 1 && calib == CAL_FIXED && x < 0.0f) {
                     wr[j] = 0.0f; ir[j] = -2; continue;
                 }
-                float uc = fminf(fmaxf(u, 0.0f), Kf);
+                float uc = fminf(fmaxf(x, 0.0f), Kf);
                 if (rounding == RND_HARD) {
                     int32_t n = (int32_t)f2bits(uc + MAGIC) - (int32_t)f2bits(MAGIC);
                     wr[j] = g[n];
                     ir[j] = n;
                 } else {
-                    float kf = fminf(floorf(uc), Kf - 1.0f);
-                    float f = uc - kf;
-                    int k = (int)kf;
-                    wr[j] = fmaf(f, d[k], g[k]);
+                    int k = (int)floorf(uc);
+                    if (k > K - 1) k = K - 1;
+                    float d = g[k + 1] - g[k];
+                    float e = fmaf(-(float)k, d, g[k]);
+                    wr[j] = fmaf(uc, d, e);
                     ir[j] = k;
                 }
             }

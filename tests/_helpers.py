@@ -53,27 +53,42 @@ def err_stats(got, want):
     return float(d.max()), float(d.mean())
 
 
-def half_ulp_bf16(x):
-    """Half the bf16 spacing at |x| (8 significand bits)."""
+def bf16_step(x):
+    """The bf16 spacing at |x| (8 significand bits)."""
     a = np.abs(np.asarray(x, dtype=np.float64))
     e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
-    return 0.5 * 2.0 ** (e - 7)
+    return 2.0 ** (e - 7)
 
 
-def err_stats_bf16_out(got, want):
-    """(max, mean) of |got - want|, the max taken net of the half-ulp that
-    rounding the exact value to the bf16 output format may already cost."""
+def to_bf16(x):
+    """x rounded to bf16 (round to nearest even), as float64."""
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def check_bf16_output(got, want, tol_max=1e-2, tol_mean=1e-3, what=""):
+    """A bf16 kernel output against the fp64 oracle rounded to the same bf16
+    format: |got - bf16(want)| <= tol_max everywhere, except that where one
+    bf16 step exceeds tol_max (|want| >= 2) the two may sit on adjacent bf16
+    codes (two values a hair apart can round to neighbours); and the mean
+    |got - want| <= tol_mean."""
     g = np.asarray(got, dtype=np.float64)
     w = np.asarray(want, dtype=np.float64)
-    d = np.abs(g - w)
-    return float(np.max(d - half_ulp_bf16(w))), float(d.mean())
+    d = np.abs(g - to_bf16(w))
+    allow = np.maximum(tol_max, bf16_step(w))
+    worst = float(np.max(d / allow))
+    mean = float(np.abs(g - w).mean())
+    assert worst <= 1.0 and mean <= tol_mean, (what, float(d.max()), worst, mean)
+    return float(d.max()), mean
 
 
-def check_decisions(d, got_idx, causal, mode, K, calib, rounding, window, heads=None):
+def check_decisions(d, got_idx, causal, mode, K, calib, rounding, window, heads=None,
+                    row_block=1024):
     """Kernel decisions (the forward's debug dump) against fp64 rounding:
     agreement >= 99.9 % and every mismatch within 1e-3 of a boundary; masked
     keys read -1 (or the buffer's fill value -7 in key tiles the kernel never
-    visits)."""
+    visits).  ``got_idx`` is the [B,H,S,S] dump, or a dict {(b, h): [S,S]}
+    holding only the heads checked."""
     if mode == A.EXACT:
         return
     q = d["q"].double().numpy() * d["q_descale"]
@@ -83,16 +98,20 @@ def check_decisions(d, got_idx, causal, mode, K, calib, rounding, window, heads=
         heads = [(b, h) for b in range(B) for h in range(H)]
     total = bad = 0
     for (b, h) in heads:
-        s = (q[b, h] @ k[b, h].T) / math.sqrt(D)
-        valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal \
-            else np.ones((S, S), bool)
-        m = A._map_rows(s, valid, mode, K, calib, rounding, window, 15, 0)
-        ref = m["idx"]
-        dist = boundary_distance_rows(s, valid, mode, K, calib, rounding, window)
-        g = got_idx[b, h].astype(np.int64)
-        assert np.all((g[~valid] == -1) | (g[~valid] == -7))
-        mism = (g != ref) & valid
-        assert np.all(dist[mism] <= 1e-3), (b, h, np.argwhere(mism & (dist > 1e-3))[:5])
-        bad += int(mism.sum())
-        total += int(valid.sum())
+        g_all = got_idx[(b, h)] if isinstance(got_idx, dict) else got_idx[b, h]
+        for r0 in range(0, S, row_block):
+            rr = np.arange(r0, min(S, r0 + row_block))
+            s = (q[b, h, rr] @ k[b, h].T) / math.sqrt(D)
+            valid = (np.arange(S)[None, :] <= rr[:, None]) if causal \
+                else np.ones((len(rr), S), bool)
+            m = A._map_rows(s, valid, mode, K, calib, rounding, window, 15, 0)
+            ref = m["idx"]
+            dist = boundary_distance_rows(s, valid, mode, K, calib, rounding, window)
+            g = np.asarray(g_all[rr], dtype=np.int64)
+            assert np.all((g[~valid] == -1) | (g[~valid] == -7))
+            mism = (g != ref) & valid
+            assert np.all(dist[mism] <= 1e-3), (b, h, np.argwhere(mism & (dist > 1e-3))[:5])
+            bad += int(mism.sum())
+            total += int(valid.sum())
     assert bad <= 1e-3 * total, (bad, total)
+    return bad, total

@@ -128,3 +128,20 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         qsm._ptr(torch.zeros(4))
+
+
+def test_noalloc_status_matches_the_workspace_backward():
+    """qsm_attn_bwd_noalloc returns the status qsm_attn_bwd returns for the same
+    shape errors, before touching any device."""
+    L = qsm.lib()
+    o = qsm.qsm_opts_default()
+
+    def both(B, S, D):
+        a = L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, 1, S, D, 1,
+                           1, 4, 0, 1, 1, ctypes.byref(o), None)
+        b = L.qsm_attn_bwd_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, 1, S,
+                                   D, 1, 1, 4, 0, 1, 1, ctypes.byref(o), None)
+        return a, b
+    assert both(1, 128, 96) == (qsm.QSM_ERR_UNSUPPORTED, qsm.QSM_ERR_UNSUPPORTED)
+    assert both(0, 128, 64) == (qsm.QSM_ERR_INVALID_ARG, qsm.QSM_ERR_INVALID_ARG)
+    assert both(1, 0, 64) == (qsm.QSM_ERR_INVALID_ARG, qsm.QSM_ERR_INVALID_ARG)

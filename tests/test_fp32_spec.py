@@ -1,9 +1,11 @@
 """Pins for the C restatement of the fp32 weight-map specification.
 
-The fp32 spec is the bit-exact target of the GPU map.  Here it is checked
-against the fp64 oracle (itself pinned in test_oracle_pins.py): decisions
-agree except within a small distance of a rounding boundary (where fp32 and
-fp64 may legitimately round differently), and weights agree to fp32 accuracy.
+The fp32 spec is the bit-exact target of the GPU map (the fused forward's
+own per-element arithmetic on raw products r, with the score scale c folded
+into one fused multiply-add).  Here it is checked against the fp64 oracle
+(itself pinned in test_oracle_pins.py) on the scores s = c r: decisions agree
+except within a small distance of a rounding boundary (where fp32 and fp64
+may legitimately round differently), and weights agree to fp32 accuracy.
 Its own exp is checked against float64 exp over the range the grid uses.
 """
 
@@ -41,37 +43,56 @@ def _boundary_distance(s64, valid, mode, K, calib, rounding, W):
     return np.minimum(fr, 1 - fr)
 
 
-CASES = [(A.ROWMAX_POT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 1)] + \
+CASES = [(A.EXACT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 1)] + \
     [(A.KINTERVAL, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
     [(A.KINTERVAL, 4, 1, 1, 1), (A.KINTERVAL, 16, 1, 0, 1)]
 
+# score scales: none, 1/sqrt(128), and 1/sqrt(128) times two e4m3 descales
+SCALES = [1.0, 0.08838834764831845, 0.08838834764831845 * 0.0121 * 0.0098]
 
+
+@pytest.mark.parametrize("c", SCALES)
 @pytest.mark.parametrize("mode,K,calib,rounding,below", CASES)
-def test_spec_matches_fp64_oracle(mode, K, calib, rounding, below):
+def test_spec_matches_fp64_oracle(mode, K, calib, rounding, below, c):
     rng = np.random.default_rng(31 + K + 100 * mode + 10 * calib + rounding)
     R, S = 256, 300
-    s32 = (rng.normal(0, 3.0, size=(R, S))).astype(np.float32)
+    c32 = np.float32(c)
+    # raw products whose scores c*r spread like N(0, 3^2)
+    r32 = (rng.normal(0, 3.0, size=(R, S)) / float(c32)).astype(np.float32)
     vl = rng.integers(1, S + 1, size=R).astype(np.int32)
     vl[:4] = [1, 2, S, S]
     valid = np.arange(S)[None, :] < vl[:, None]
     W = 6.0
-    w32, idx32, hi32, lo32 = spec.spec_map(s32, vl, mode, K=K, calib=calib, rounding=rounding,
-                                           window=W, pot_floor=15, below_policy=below)
-    s64 = s32.astype(np.float64)
+    w32, idx32, hi32, lo32 = spec.spec_map(r32, vl, mode, K=K, calib=calib, rounding=rounding,
+                                           window=W, pot_floor=15, below_policy=below, c=c)
+    s64 = float(c32) * r32.astype(np.float64)
     w64, idx64, hi64, _ = oracle.weight_map(s64, valid, mode, K=K, calib=calib,
                                             rounding=rounding, window=W, pot_floor=15,
                                             below_policy=below)
-    assert np.array_equal(hi32.astype(np.float64), hi64)       # max is exact
+    # hi = c * max r rounded once to fp32
+    assert np.array_equal(hi32, hi64.astype(np.float32))
+    if mode == A.EXACT:
+        # the spec gives the exponent x of 2^x
+        w32 = np.exp2(w32.astype(np.float64)) * valid
     dist = _boundary_distance(s64, valid, mode, K, calib, rounding, W)
     agree = idx32 == idx64
     assert np.all(agree | (dist < 1e-4)), np.argwhere(~agree & (dist >= 1e-4))[:5]
     assert agree.mean() > 0.999
     ok = agree & valid
     # weights are anchored at 1 for the row max; fp32 evaluation of the grid
-    # coordinate carries an absolute error of a few ulp of |s * K / a|, which
-    # the interpolation slope (<= 1 per unit of u) carries into w
-    np.testing.assert_allclose(w32[ok], w64[ok], rtol=4e-6, atol=4e-6)
+    # coordinate (slope c*K/a rounded once, then one fused multiply-add)
+    # carries an absolute error of a few ulp of |r * c * K / a|, which the
+    # interpolation slope (<= 1 per unit of u) carries into w
+    np.testing.assert_allclose(w32[ok], w64[ok], rtol=4e-6, atol=8e-6)
     assert np.all(w32[~valid] == 0) and np.all(idx32[~valid] == -1)
+
+
+def test_spec_nan_propagates_to_the_row_statistics():
+    r = np.array([[1.0, np.nan, -2.0], [1.0, 0.5, -2.0]], np.float32)
+    vl = np.array([3, 3], np.int32)
+    _, _, hi, lo = spec.spec_map(r, vl, A.KINTERVAL, K=4, calib=A.MINMAX, rounding=A.HARD)
+    assert np.isnan(hi[0]) and np.isnan(lo[0])
+    assert hi[1] == 1.0 and lo[1] == -2.0
 
 
 def test_spec_pot_is_exact_power_of_two_and_one_at_max():

@@ -4,10 +4,17 @@ against the CPU oracle, through the C ABI.
 The rules are the oracle's ("Pretraining Transformers with Quantized Softmax
 in Attention", abstract: backward rules including calibration derivatives;
 straight-through surrogate before or after normalization), whose own pins
-are in test_oracle_bwd.py.  Tolerance (bf16 gradients): max abs <= 1e-2 beyond the rounding of the
-exact value to the bf16 output (gradients of the first keys of a causal row
-reach magnitudes above 4, where half a bf16 ulp alone is 0.0078-0.0156),
-mean abs <= 1e-3.
+are in test_oracle_bwd.py.  The oracle evaluates them at its own fp64
+rounding decisions; nothing from the GPU path enters it.  Tolerance (bf16
+gradients): against the oracle rounded to bf16, max abs <= 1e-2 (adjacent
+bf16 codes allowed where one bf16 step exceeds 1e-2: the first keys of a
+causal row reach |dV| > 4), mean abs <= 1e-3.
+
+Separately, and only as a labelled diagnostic that no gradient comparison
+uses, the kernel forward's own decisions are checked against fp64 rounding
+(>= 99.9 % agreement, every mismatch within 1e-3 of a boundary): where they
+differ, the oracle's gradients and the kernel's follow different frozen
+decisions, and the tolerance above covers that.
 """
 
 import numpy as np
@@ -17,36 +24,31 @@ import torch
 import oracle
 from approximate_softmax_attention_b200 import inputs, qsm
 
-from _helpers import check_decisions, err_stats_bf16_out
+from _helpers import check_bf16_output, check_decisions
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
 
 
-def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0):
+def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=False):
     q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
     B, H, S, D = q.shape
-    dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV)
+    dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV) if dump else None
     O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rnd, window=window,
                                        stats=True, debug_idx=dbg)
     dQ, dK, dV = qsm.attention_backward(q, k, v, O, dO, LSE, st, causal, mode, K, calib, rnd,
                                         surr, detach_extrema=detach, window=window)
     torch.cuda.synchronize()
-    return (dQ.float().cpu().numpy(), dK.float().cpu().numpy(), dV.float().cpu().numpy(),
-            dbg.cpu().numpy())
+    out = [dQ.float().cpu().numpy(), dK.float().cpu().numpy(), dV.float().cpu().numpy()]
+    return out, (dbg.cpu().numpy() if dump else None)
 
 
-def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None, dec=None):
-    """The oracle's backward, with the node decisions the kernel's forward
-    took (they agree with fp64 rounding except within 1e-3 of a boundary,
-    checked by check_decisions; the rules hold the forward's decisions
-    fixed, so the gradients are compared at those decisions)."""
-    if dec is not None and mode == 1:
-        check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads)
+def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None):
+    """The oracle's backward at its own fp64 decisions."""
     return oracle.attn_bwd(d["q"], d["k"], d["v"], d["dO"], causal, mode, K=K, calib=calib,
                            rounding=rnd, surrogate=surr, detach_extrema=detach, window=window,
-                           heads=heads, decisions=dec if mode == 1 else None)
+                           heads=heads)
 
 
 def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3):
@@ -55,8 +57,7 @@ def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3):
         if heads is not None:
             g = np.stack([g[b, h] for (b, h) in heads])
             r = np.stack([r[b, h] for (b, h) in heads])
-        mx, mean = err_stats_bf16_out(g, r)
-        assert mx <= tol_max and mean <= tol_mean, (name, mx, mean)
+        check_bf16_output(g, r, tol_max, tol_mean, what=name)
 
 
 COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
@@ -67,8 +68,8 @@ COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
 def test_bwd_kinterval_small(S, causal, K, calib, rnd, surr, detach):
     d = inputs.draw(1, 2, S, 64, seed=50 + S, with_dO=True)
-    *got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
-    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, dec=dec)
+    got, _ = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
+    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
     _check(got, ref)
 
 
@@ -79,15 +80,15 @@ def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
     """K = 1 (one grid segment) and K = 32 (the largest K the backward
     accepts), pre and post surrogate, calibration derivatives on."""
     d = inputs.draw(1, 2, 256, 64, seed=90 + K, with_dO=True)
-    *got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
-    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0, dec=dec)
+    got, _ = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
+    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0)
     _check(got, ref)
 
 
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False), (77, True), (384, False)])
 def test_bwd_exact(S, causal):
     d = inputs.draw(1, 2, S, 64, seed=7 + S, with_dO=True)
-    *got, _ = _run(d, causal, 0, 4, 0, 1, 0, False)
+    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False)
     ref = _oracle(d, causal, 0, 4, 0, 1, 0, False)
     _check(got, ref)
 
@@ -102,8 +103,20 @@ def test_bwd_training_shape_sampled(mode, K, calib, rnd, surr, detach):
     w = inputs.WORKLOADS["train_s1k"]
     d = inputs.draw_workload(w)
     heads = [(0, 0), (3, 7), (7, 11)]
-    *got, dec = _run(d, True, mode, K, calib, rnd, surr, detach)
-    ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads, dec=dec)
+    got, _ = _run(d, True, mode, K, calib, rnd, surr, detach)
+    ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads)
     _check(got, ref, heads=heads)
     for g in got:
         assert np.isfinite(g).all()
+
+
+@pytest.mark.parametrize("K,calib,rnd", [(4, 0, 1), (16, 0, 0), (4, 1, 1), (16, 1, 0)])
+def test_diagnostic_forward_decisions_of_the_backward_runs(K, calib, rnd):
+    """Diagnostic only (no gradient comparison uses it): the decisions the
+    kernel's forward takes on the backward's inputs agree with fp64 rounding
+    (>= 99.9 %, mismatches within 1e-3 of a boundary)."""
+    w = inputs.WORKLOADS["train_s1k"]
+    d = inputs.draw_workload(w)
+    heads = [(0, 0), (3, 7), (7, 11)]
+    _, dec = _run(d, True, 1, K, calib, rnd, 1, False, dump=True)
+    check_decisions(d, dec, True, 1, K, calib, rnd, 8.0, heads)

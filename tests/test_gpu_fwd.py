@@ -21,7 +21,7 @@ from oracle import spec
 from oracle import attention as A
 from approximate_softmax_attention_b200 import inputs, qsm
 
-from _helpers import boundary_distance_rows, err_stats, err_stats_bf16_out
+from _helpers import boundary_distance_rows, check_bf16_output, check_decisions, err_stats
 
 pytestmark = pytest.mark.gpu
 
@@ -38,37 +38,64 @@ MAP_CASES = [(0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1)] + \
     [(1, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
     [(1, 4, 1, 1, 1), (1, 16, 1, 0, 1)]
 
+# (scale, q_descale, k_descale) as the forward forms c = scale * qd * kd
+SCALES = [(1.0, 1.0, 1.0), (1.0 / math.sqrt(128.0), 1.0, 1.0),
+          (1.0 / math.sqrt(128.0), 0.0121, 0.0098)]
 
+
+def _c32(scale, qd, kd):
+    return float(np.float32(np.float32(np.float32(scale) * np.float32(qd)) * np.float32(kd)))
+
+
+@pytest.mark.parametrize("scales", SCALES)
 @pytest.mark.parametrize("mode,K,calib,rounding,below", MAP_CASES)
-def test_weight_map_bit_exact(mode, K, calib, rounding, below):
+def test_weight_map_bit_exact(mode, K, calib, rounding, below, scales):
+    """qsm_weight_map runs the fused forward's own per-element map (row set-up,
+    table, pair arithmetic, decision index) on raw products with the score
+    scale folded in; it must equal the C restatement bit for bit.  The exact
+    map's 2^x is the hardware approximation: checked against 2^x in fp64."""
     rows, cols = 300, 517
+    c = _c32(*scales)
     s = inputs.scores_fp32(rows, cols, seed=40 + K + 3 * mode + calib + 7 * rounding).numpy()
+    r = (s / c).astype(np.float32)                  # raw products of the same scores
     rng = np.random.default_rng(K + mode)
     vl = rng.integers(1, cols + 1, size=rows).astype(np.int32)
     vl[:3] = [1, 2, cols]
-    s[5, :] = 0.5                                   # degenerate row
-    # adversarial: scores placed on and next to node boundaries of row 6
-    hi, lo = s[6].max(), s[6].min()
+    r[5, :] = np.float32(0.5 / c)                   # degenerate row
+    # adversarial: products placed on and next to node boundaries of row 6
+    hi, lo = r[6].max(), r[6].min()
     step = (hi - lo) / K
     for i in range(40):
         base = lo + (i % (K + 1)) * step + (0.5 * step if rounding == 1 else 0.0)
         toward = (-np.inf, base, np.inf)[i % 3]
-        s[6, 10 + i] = np.nextafter(np.float32(base), np.float32(toward))
+        r[6, 10 + i] = np.nextafter(np.float32(base), np.float32(toward))
     window = 6.0
-    w_ref, i_ref, hi_ref, lo_ref = spec.spec_map(s, vl, mode, K=K, calib=calib,
+    w_ref, i_ref, hi_ref, lo_ref = spec.spec_map(r, vl, mode, K=K, calib=calib,
                                                  rounding=rounding, window=window,
-                                                 pot_floor=15, below_policy=below)
-    S = _gpu(torch.from_numpy(s))
+                                                 pot_floor=15, below_policy=below, c=c)
+    S = _gpu(torch.from_numpy(r))
     VL = _gpu(torch.from_numpy(vl))
     W = torch.empty_like(S)
     I = torch.empty(rows, cols, dtype=torch.int32, device=DEV)
     HI = torch.empty(rows, dtype=torch.float32, device=DEV)
     LO = torch.empty(rows, dtype=torch.float32, device=DEV)
-    opts = qsm.make_opts(window=window, pot_floor=15, below_policy=below)
+    opts = qsm.make_opts(window=window, pot_floor=15, below_policy=below, scale=scales[0],
+                         q_descale=scales[1], k_descale=scales[2])
     st = qsm.qsm_weight_map(S, VL, mode, K, calib, rounding, opts, W, I, HI, LO)
     assert st == qsm.QSM_OK
     torch.cuda.synchronize()
-    assert np.array_equal(W.cpu().numpy().view(np.uint32), w_ref.view(np.uint32))
+    got = W.cpu().numpy()
+    if mode == 0:
+        x = w_ref.astype(np.float64)
+        valid = np.arange(cols)[None, :] < vl[:, None]
+        want = np.where(valid, np.exp2(x), 0.0)
+        normal = want >= 2.0 ** -126
+        # ex2.approx: a few ulp of relative error; results below the normal
+        # range flush to zero
+        assert np.all(np.abs(got[normal] - want[normal]) <= 2.0 ** -21 * want[normal])
+        assert np.all(got[~normal] <= 2.0 ** -126)
+    else:
+        assert np.array_equal(got.view(np.uint32), w_ref.view(np.uint32))
     assert np.array_equal(I.cpu().numpy(), i_ref)
     assert np.array_equal(HI.cpu().numpy().view(np.uint32), hi_ref.view(np.uint32))
     assert np.array_equal(LO.cpu().numpy().view(np.uint32), lo_ref.view(np.uint32))
@@ -223,12 +250,12 @@ def test_fwd_pot_floor_wide_scores(dtype, below, floor):
     floored = (idx == -2) if below else (idx == floor)
     # the case is the one it claims to be: most valid keys are at the floor
     assert floored.sum() > 0.5 * valid.sum()
-    # the weight concentrates on each row's top keys, so |O| reaches ~4, where
-    # rounding the exact value to bf16 alone costs up to 0.0156: the max is
-    # taken net of that half-ulp (the reading the backward's tests use too)
-    mx, mean = err_stats_bf16_out(O.float().cpu().numpy(), ref["O"])
-    tol = 1e-2 if dtype == "bf16" else 5e-2
-    assert mx <= tol and mean <= (1e-3 if dtype == "bf16" else 5e-3), (mx, mean)
+    # the weight concentrates on each row's top keys, so |O| reaches ~4: the
+    # output is compared with the oracle rounded to bf16 (adjacent bf16 codes
+    # allowed where one step exceeds the tolerance)
+    check_bf16_output(O.float().cpu().numpy(), ref["O"],
+                      tol_max=1e-2 if dtype == "bf16" else 5e-2,
+                      tol_mean=1e-3 if dtype == "bf16" else 5e-3, what="O")
     np.testing.assert_allclose(LSE.cpu().numpy(), ref["LSE"], atol=5e-3, rtol=1e-4)
     got_idx = dbg.cpu().numpy()
     agree = (got_idx == idx)[valid].mean()
@@ -245,6 +272,70 @@ def test_fwd_fp8(causal, mode, K, calib, rounding):
     mx, mean = err_stats(got["O"], ref["O"])
     assert mx <= 5e-2, (mx, mean)
     _check_idx(d, got["idx"], ref["idx"], causal, mode, K, calib, rounding, 8.0)
+
+
+ALL_MAPS = [(0, 4, 0, 1), (2, 4, 0, 1), (1, 4, 0, 1), (1, 4, 0, 0), (1, 4, 1, 1), (1, 16, 1, 0)]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("mode,K,calib,rounding", ALL_MAPS)
+def test_fwd_degenerate_rows(dtype, mode, K, calib, rounding):
+    """Every key equal: each row's scores are all equal (hi == lo), so every
+    map gives uniform weights (the degenerate-row reading: all at the top node
+    / exponent 0) and O is the mean of the valid V rows."""
+    S, D = 200, 128
+    d = inputs.draw(1, 2, S, D, seed=11, dtype=dtype)
+    d["k"] = d["k"][:, :, :1, :].expand(1, 2, S, D).contiguous()
+    got = _run_fwd(d, True, mode, K, calib, rounding, debug=True)
+    ref = _oracle(d, True, mode, K, calib, rounding, want_idx=True)
+    mx, mean = err_stats(got["O"], ref["O"])
+    assert mx <= (1e-2 if dtype == "bf16" else 5e-2) and mean <= 1e-3, (mx, mean)
+    np.testing.assert_allclose(got["LSE"], ref["LSE"], atol=2e-3, rtol=1e-4)
+    if not (mode == 1 and calib == 1):           # fixed window: lo = hi - W
+        assert np.array_equal(got["hi"], got["lo"])
+    valid = ref["idx"] != -1
+    assert np.array_equal(got["idx"][valid], ref["idx"][valid])
+
+
+@pytest.mark.parametrize("mode,K,calib,rounding,below", [
+    (0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1), (1, 4, 1, 1, 0), (1, 4, 1, 0, 1),
+    (1, 16, 0, 0, 0), (1, 4, 0, 1, 0)])
+def test_fwd_nonfinite_scores(mode, K, calib, rounding, below):
+    """Non-finite inputs give non-finite scores.  Head 0: key 37 carries -inf
+    in the first component and every query a positive one, so its score is
+    -inf in every row that sees it; key 100 carries a NaN.  Head 1: key 150
+    carries +inf.  The forward must end normally and match the oracle's
+    reading: a -inf score takes the map's limit (0, the PoT floor, the lowest
+    grid value, or a flush to 0); rows whose maximum is NaN or +inf, or whose
+    min-max grid starts at -inf, give NaN O and LSE; other rows are
+    untouched."""
+    S, D = 256, 64
+    d = inputs.draw(1, 2, S, D, seed=12)
+    q = d["q"].float()
+    q[..., 0] = q[..., 0].abs() + 0.25
+    k = d["k"].float()
+    k[0, 0, 37, 0] = -float("inf")
+    k[0, 0, 100, 5] = float("nan")
+    k[0, 1, 150, 0] = float("inf")
+    d["q"], d["k"] = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    qq, kk, vv = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    O, LSE = qsm.attention_forward(qq, kk, vv, True, mode, K, calib, rounding, window=6.0,
+                                   below_policy=below)
+    torch.cuda.synchronize()
+    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], True, mode, K=K, calib=calib,
+                          rounding=rounding, window=6.0, below_policy=below)
+    got_O, got_L = O.float().cpu().numpy(), LSE.cpu().numpy()
+    assert np.array_equal(np.isnan(got_O), np.isnan(ref["O"]))
+    assert np.array_equal(np.isnan(got_L), np.isnan(ref["LSE"]))
+    fin = ~np.isnan(ref["O"])
+    # rows before key 37 (head 0) and before key 150 (head 1) are finite, later
+    # head-0 rows are finite exactly when the map defines a -inf score
+    assert fin[0, 0, :37].all() and fin[0, 1, :150].all() and np.isnan(ref["O"][0, 1, 150:]).all()
+    mx, mean = err_stats(got_O[fin], ref["O"][fin])
+    assert mx <= 1e-2 and mean <= 1e-3, (mx, mean)
+    finL = ~np.isnan(ref["LSE"])
+    np.testing.assert_allclose(got_L[finL], ref["LSE"][finL], atol=2e-3, rtol=1e-4)
 
 
 def _sampled_check(name, tol_max, tol_mean, nheads=3, nrows=96):
@@ -274,6 +365,39 @@ def test_full_size_s2k_bf16_causal_sampled():
 @pytest.mark.parametrize("name", ["s8k_fp8", "s8k_fp8_causal"])
 def test_full_size_s8k_fp8_sampled(name):
     _sampled_check(name, 5e-2, 5e-3, nheads=2, nrows=48)
+
+
+def test_full_size_s8k_bf16_sampled():
+    """B=2, H=16, S=8192, D=128 bf16 non-causal, peaked keys (the bf16 copy of
+    the 8K shape): exact, Rowmax-PoT, K-interval K=4 fixed-window hard."""
+    _sampled_check("s8k_bf16", 1e-2, 1e-3, nheads=2, nrows=48)
+
+
+@pytest.mark.parametrize("name,heads", [("s2k_bf16_causal", [(0, 0), (3, 15)]),
+                                        ("s8k_fp8", [(1, 9)]), ("s8k_fp8_causal", [(0, 4)]),
+                                        ("s8k_bf16", [(1, 13)])])
+def test_full_size_decisions(name, heads):
+    """Decision agreement of the fused forward with fp64 rounding at the full
+    sizes (>= 99.9 %, every mismatch within 1e-3 of a boundary), on whole
+    heads, launched with the full B x H grid (heaviest-first CTA order, the
+    full K/V ring and long sweeps included)."""
+    w = inputs.WORKLOADS[name]
+    d = inputs.draw_workload(w)
+    q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    B, H, S, D = q.shape
+    dbg = torch.empty((B, H, S, S), dtype=torch.int8, device=DEV)
+    for (mode, K, calib, rnd) in w.modes:
+        if mode == 0:
+            continue
+        dbg.fill_(-7)
+        qsm.attention_forward(q, k, v, w.causal, mode, K, calib, rnd,
+                              q_descale=d["q_descale"], k_descale=d["k_descale"],
+                              v_descale=d["v_descale"], debug_idx=dbg)
+        torch.cuda.synchronize()
+        got = {(b, h): dbg[b, h].cpu().numpy() for (b, h) in heads}
+        check_decisions(d, got, w.causal, mode, K, calib, rnd, 8.0, heads)
+    del dbg
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("name,tol_max,tol_mean", [("s16k_bf16_causal", 1e-2, 1e-3),

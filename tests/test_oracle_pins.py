@@ -297,3 +297,43 @@ def test_detach_does_not_change_forward():
         _, P1, O1 = A.attn_bwd_rows(s, valid, v, dO, A.KINTERVAL, 4, cal, rnd, A.SURR_PRE, False, 3.0)
         _, P2, O2 = A.attn_bwd_rows(s, valid, v, dO, A.KINTERVAL, 4, cal, rnd, A.SURR_PRE, True, 3.0)
         assert np.array_equal(P1, P2) and np.array_equal(O1, O2)
+
+
+def test_nonfinite_scores_take_the_maps_limits_or_poison_the_row():
+    """A -inf score takes each map's limit at s -> -inf (exact: 0; PoT: the
+    floor 2^-N, or 0 when flushed; fixed-window K-interval: the lowest grid
+    value g_0, or 0 when flushed); a row whose maximum is NaN or +inf, or
+    whose min-max grid would start at -inf, has NaN weights."""
+    e = math.exp
+    s = np.array([[0.0, -1.0, -np.inf, -2.0],
+                  [0.0, np.nan, -1.0, -2.0],
+                  [0.0, np.inf, -1.0, -2.0]])
+    valid = np.ones_like(s, dtype=bool)
+    w, _, _, _ = oracle.weight_map(s, valid, A.EXACT)
+    np.testing.assert_allclose(w[0], [1.0, e(-1), 0.0, e(-2)], rtol=1e-15)
+    assert np.isnan(w[1]).all() and np.isnan(w[2]).all()
+    w, idx, _, _ = oracle.weight_map(s, valid, A.ROWMAX_POT, pot_floor=15)
+    assert w[0].tolist() == [1.0, 0.5, 2.0 ** -15, 0.125] and idx[0, 2] == 15
+    assert np.isnan(w[1]).all() and np.isnan(w[2]).all()
+    w, idx, _, _ = oracle.weight_map(s, valid, A.ROWMAX_POT, pot_floor=15, below_policy=1)
+    assert w[0].tolist() == [1.0, 0.5, 0.0, 0.125] and idx[0, 2] == -2
+    # fixed window W = 8, K = 4: Delta = 2, g_k = e^{-2(4-k)}; -1 -> u = 3.5 -> 4 (ties to
+    # even), -2 -> u = 3, -inf -> clamped to u = 0
+    w, idx, _, _ = oracle.weight_map(s, valid, A.KINTERVAL, K=4, calib=A.FIXED_WINDOW,
+                                     rounding=A.HARD, window=8.0)
+    np.testing.assert_allclose(w[0], [1.0, 1.0, e(-8), e(-2)], rtol=1e-15)
+    assert idx[0].tolist() == [4, 4, 0, 3]
+    w, idx, _, _ = oracle.weight_map(s, valid, A.KINTERVAL, K=4, calib=A.FIXED_WINDOW,
+                                     rounding=A.INTERP, window=8.0, below_policy=1)
+    assert w[0, 2] == 0.0 and idx[0, 2] == -2
+    w, _, _, _ = oracle.weight_map(s, valid, A.KINTERVAL, K=4, calib=A.MINMAX, rounding=A.HARD)
+    assert np.isnan(w).all()
+    # the forward: head 0 holds a -inf key (finite output), head 1 a NaN key
+    # (every row NaN); D = 1 and q = 1, so the scores are the keys themselves
+    q = np.ones((1, 2, 4, 1))
+    k = np.array([[0.0, -1.0, -np.inf, -2.0], [0.0, np.nan, -1.0, -2.0]]).reshape(1, 2, 4, 1)
+    v = np.arange(8.0).reshape(1, 2, 4, 1)
+    res = oracle.attn_fwd(q, k, v, False, A.EXACT, scale=1.0)
+    p = np.array([1.0, e(-1), 0.0, e(-2)]) / (1 + e(-1) + e(-2))
+    np.testing.assert_allclose(res["O"][0, 0, :, 0], p @ v[0, 0, :, 0], rtol=1e-14)
+    assert np.isnan(res["O"][0, 1]).all() and np.isnan(res["LSE"][0, 1]).all()

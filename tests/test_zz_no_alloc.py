@@ -6,7 +6,8 @@ pool, a latency-critical loop that cannot take cudaMalloc's synchronisation):
 its scratch is a fixed array inside the library instead of a caller
 workspace.  Through the C ABI, two calls in a row must give what
 qsm_attn_bwd gives with a workspace, within the backward's tolerance (max
-abs 1e-2 beyond the bf16 output rounding, mean abs 1e-3); a shape whose
+abs 1e-2, adjacent bf16 codes allowed where one step exceeds it; mean abs
+1e-3); a shape whose
 scratch exceeds the array is refused before any launch.
 
 This file is collected last on purpose, and it is self-contained, so it
@@ -19,7 +20,7 @@ import torch
 
 from approximate_softmax_attention_b200 import inputs, qsm
 
-from _helpers import err_stats_bf16_out
+from _helpers import check_bf16_output
 
 pytestmark = pytest.mark.gpu
 
@@ -56,9 +57,8 @@ def test_noalloc_matches_workspace_backward_twice(mode, K, calib, rnd, surr, det
     for _ in range(2):
         got = _grads(qsm.qsm_attn_bwd_noalloc, q, k, v, O, dO, LSE, causal, mode, K, calib,
                      rnd, surr, noalloc_opts)
-        for g, r in zip(got, ref):
-            mx, mean = err_stats_bf16_out(g, r)
-            assert mx <= 1e-2 and mean <= 1e-3, (mx, mean)
+        for g, r, name in zip(got, ref, ("dQ", "dK", "dV")):
+            check_bf16_output(g, r, 1e-2, 1e-3, what=name)
 
 
 def test_noalloc_refuses_oversize_before_launch():
