@@ -20,7 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqsm.so")
 BUILD = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "fwd.cu", "wmap_kernel.cu", "bwd.cu", "bwd_noalloc.cu"]
+SOURCES = ["api.cu", "fwd.cu", "fwd_online.cu", "wmap_kernel.cu", "bwd.cu",
+           "bwd_noalloc.cu"]
 HEADERS = ["sm100.cuh", "wmap.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

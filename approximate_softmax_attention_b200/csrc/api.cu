@@ -71,6 +71,11 @@ qsm_status check_common(int B, int H, int S, int D, int causal, int mode, int Ki
   if (o.pot_floor < 0 || o.pot_floor > 126) return QSM_ERR_INVALID_ARG;
   if (o.below_policy != 0 && o.below_policy != 1) return QSM_ERR_INVALID_ARG;
   if (o.detach_extrema != 0 && o.detach_extrema != 1) return QSM_ERR_INVALID_ARG;
+  if (o.anchor != 0 && o.anchor != 1) return QSM_ERR_INVALID_ARG;
+  // the running anchor has no min-max form (the grid would follow the
+  // running minimum too)
+  if (o.anchor == 1 && mode == QSM_MODE_KINTERVAL && calib == QSM_CALIB_MINMAX)
+    return QSM_ERR_UNSUPPORTED;
   const float scale = o.scale > 0.0f ? o.scale : 1.0f / std::sqrt(static_cast<float>(D));
   *c = scale * o.q_descale * o.k_descale;
   if (!finite_pos(*c)) return QSM_ERR_INVALID_ARG;
@@ -148,7 +153,12 @@ qsm_status qsm_attn_fwd(const void *Q, const void *K, const void *V, void *O, fl
   a.debug_idx = o.debug_idx;
   a.status_dev = o.status_dev;
   a.debug_flags = o.debug_flags;
+  a.anchor = o.anchor;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
+  if (o.anchor == 1) {
+    if (o.row_argmax || o.row_argmin) return QSM_ERR_UNSUPPORTED;
+    return launch_fwd_online(a);
+  }
   return launch_fwd(a);
 }
 
@@ -164,6 +174,9 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
   if (st != QSM_OK) return st;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return QSM_ERR_INVALID_ARG;
   if (mode == QSM_MODE_ROWMAX_POT || o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
+  // the rules are derived for maps anchored at the final row statistics; the
+  // exact map is softmax under either anchor
+  if (o.anchor == 1 && mode != QSM_MODE_EXACT) return QSM_ERR_UNSUPPORTED;
   if (mode == QSM_MODE_KINTERVAL &&
       (!o.row_hi || !o.row_lo || !o.row_argmax || !o.row_argmin))
     return QSM_ERR_INVALID_ARG;

@@ -26,10 +26,12 @@ struct FwdArgs {
   int8_t *debug_idx;
   int32_t *status_dev;
   int debug_flags;
+  int anchor;
   cudaStream_t stream;
 };
 
-qsm_status launch_fwd(const FwdArgs &a);
+qsm_status launch_fwd(const FwdArgs &a);         // two sweeps (anchor 0)
+qsm_status launch_fwd_online(const FwdArgs &a);  // one sweep (anchor 1)
 
 struct MapArgs {
   const float *scores;     // raw products r; the score is c * r

@@ -25,6 +25,7 @@ CALIB_MINMAX, CALIB_FIXED_WINDOW = 0, 1
 ROUND_INTERP, ROUND_HARD = 0, 1
 SURR_NONE, SURR_PRE, SURR_POST = 0, 1, 2
 DTYPE_BF16, DTYPE_FP8_E4M3 = 0, 1
+ANCHOR_FINAL, ANCHOR_RUNNING = 0, 1
 
 EXPORTED = ("qsm_opts_default", "qsm_attn_fwd", "qsm_attn_bwd", "qsm_attn_bwd_workspace_size",
             "qsm_attn_bwd_noalloc", "qsm_weight_map", "qsm_status_string", "qsm_version")
@@ -52,6 +53,7 @@ class QsmOpts(ctypes.Structure):
         ("status_dev", ctypes.c_void_p),
         ("debug_idx", ctypes.c_void_p),
         ("debug_flags", ctypes.c_int),
+        ("anchor", ctypes.c_int),
     ]
 
 
@@ -198,10 +200,12 @@ def _check(status, where):
 def attention_forward(q, k, v, causal=False, mode=MODE_EXACT, Kint=4,
                       calibration=CALIB_MINMAX, rounding=ROUND_HARD, *, scale=None,
                       q_descale=1.0, k_descale=1.0, v_descale=1.0, window=8.0, pot_floor=15,
-                      below_policy=0, stats=False, debug_idx=None, stream=None):
+                      below_policy=0, stats=False, debug_idx=None, anchor=ANCHOR_FINAL,
+                      stream=None):
     """Allocate the outputs with torch and run ``qsm_attn_fwd``.
 
-    Returns (O, LSE) or (O, LSE, stats dict) with hi, lo, argmax, argmin.
+    Returns (O, LSE) or (O, LSE, stats dict) with hi, lo, argmax, argmin
+    (with ``anchor=ANCHOR_RUNNING``, the one-sweep form: hi and lo only).
     """
     B, H, S, D = q.shape
     dev = q.device
@@ -211,14 +215,15 @@ def attention_forward(q, k, v, causal=False, mode=MODE_EXACT, Kint=4,
     kw = dict(dtype=DTYPE_FP8_E4M3 if q.dtype == torch.float8_e4m3fn else DTYPE_BF16,
               scale=0.0 if scale is None else float(scale), q_descale=float(q_descale),
               k_descale=float(k_descale), v_descale=float(v_descale), window=float(window),
-              pot_floor=int(pot_floor), below_policy=int(below_policy))
+              pot_floor=int(pot_floor), below_policy=int(below_policy), anchor=int(anchor))
     if stats:
         st = dict(hi=torch.empty(B, H, S, dtype=torch.float32, device=dev),
-                  lo=torch.empty(B, H, S, dtype=torch.float32, device=dev),
-                  argmax=torch.empty(B, H, S, dtype=torch.int32, device=dev),
-                  argmin=torch.empty(B, H, S, dtype=torch.int32, device=dev))
-        kw.update(row_hi=st["hi"], row_lo=st["lo"], row_argmax=st["argmax"],
-                  row_argmin=st["argmin"])
+                  lo=torch.empty(B, H, S, dtype=torch.float32, device=dev))
+        kw.update(row_hi=st["hi"], row_lo=st["lo"])
+        if anchor == ANCHOR_FINAL:
+            st.update(argmax=torch.empty(B, H, S, dtype=torch.int32, device=dev),
+                      argmin=torch.empty(B, H, S, dtype=torch.int32, device=dev))
+            kw.update(row_argmax=st["argmax"], row_argmin=st["argmin"])
     if debug_idx is not None:
         kw["debug_idx"] = debug_idx
     opts = make_opts(**kw)

@@ -5,9 +5,12 @@
 
 Workload (one step, the default): the forward of the B=1, H=32, S=16384,
 D=128 causal problem with peaked keys (1% of keys shifted +3 along a per-head
-unit direction), in bf16 and in e4m3, once per map: exact softmax (two-sweep
-form), Rowmax-PoT, and K-interval K in {4, 16} x {min-max, fixed window} x
-{interpolation, hard rounding} -- 20 forwards.  ``value`` is the step's
+unit direction), in bf16 and in e4m3, once per map.  Maps anchored at the
+row's final statistics (two sweeps): exact softmax, Rowmax-PoT, and
+K-interval K in {4, 16} x {min-max, fixed window} x {interpolation, hard
+rounding}; maps anchored at the running maximum (one sweep, labels
+"_online"): the online softmax (the exact-exp comparator), Rowmax-PoT and the
+four fixed-window K-interval maps -- 32 forwards.  ``value`` is the step's
 algorithmic TFLOP/s (4*B*H*S^2*D per forward, halved for causal; the
 statistics sweep of the two-sweep maps is not counted), whole job, inputs
 resident in HBM.  Every input set (bf16 402 MB, e4m3 201 MB) is larger than
@@ -61,10 +64,26 @@ METRIC = ("attn fwd TFLOPS & % of B200 tensor peak per softmax mode, causal/non-
 
 
 def mode_label(m):
-    mode, K, cal, rnd = m
-    if mode == 1:
-        return "kinterval_K%d_%s_%s" % (K, CALIB_NAMES[cal], ROUND_NAMES[rnd])
-    return MODE_NAMES[mode]
+    mode, K, cal, rnd = m[:4]
+    anchor = m[4] if len(m) > 4 else 0
+    lab = ("kinterval_K%d_%s_%s" % (K, CALIB_NAMES[cal], ROUND_NAMES[rnd]) if mode == 1
+           else MODE_NAMES[mode])
+    return lab + ("_online" if anchor else "")
+
+
+def step_maps(w):
+    """The maps of one step on workload w: the workload's maps anchored at the
+    final row statistics (two sweeps), then the one-sweep forms anchored at
+    the running maximum: the online softmax (this build's exact-exp
+    comparator), Rowmax-PoT, and every fixed-window K-interval map of the
+    workload."""
+    maps = [tuple(m) + (0,) for m in w.modes]
+    maps.append((0, 4, 0, 0, 1))
+    maps.append((2, 4, 0, 0, 1))
+    for (mode, K, cal, rnd) in w.modes:
+        if mode == 1 and cal == 1:
+            maps.append((mode, K, cal, rnd, 1))
+    return maps
 
 
 def dtype_name(w):
@@ -243,7 +262,7 @@ def oracle_sample(workloads, budget_s=12.0, rows_per_map=256):
     import numpy as np
     import oracle
     from approximate_softmax_attention_b200 import inputs
-    cases = [(w, m) for w in workloads for m in w.modes]
+    cases = [(w, m) for w in workloads for m in step_maps(w)]
     per_case = budget_s / len(cases)
     done_flops, t_total, rows_done = 0.0, 0.0, 0
     draws = {}
@@ -252,15 +271,20 @@ def oracle_sample(workloads, budget_s=12.0, rows_per_map=256):
             draws[w.name] = inputs.draw(1, 1, w.S, w.D, seed=w.seed, peaked=w.peaked,
                                         dtype=w.dtype)
         d = draws[w.name]
-        mode, K, cal, rnd = m
+        mode, K, cal, rnd, anchor = m
         n = rows_per_map
         t_case = 0.0
         while True:
             rows = np.unique(np.linspace(0, w.S - 1, n).astype(np.int64))
+            kw = dict(q_descale=d["q_descale"], k_descale=d["k_descale"],
+                      v_descale=d["v_descale"], rows=rows, row_block=128)
             t0 = time.perf_counter()
-            oracle.attn_fwd(d["q"], d["k"], d["v"], w.causal, mode, K=K, calib=cal,
-                            rounding=rnd, q_descale=d["q_descale"], k_descale=d["k_descale"],
-                            v_descale=d["v_descale"], rows=rows, row_block=128)
+            if anchor and mode != 0:
+                oracle.attn_fwd_online(d["q"], d["k"], d["v"], w.causal, mode, K=K,
+                                       rounding=rnd, **kw)
+            else:
+                oracle.attn_fwd(d["q"], d["k"], d["v"], w.causal, mode, K=K, calib=cal,
+                                rounding=rnd, **kw)
             dt = time.perf_counter() - t0
             keys = (rows + 1).sum() if w.causal else len(rows) * w.S
             done_flops += 4.0 * w.D * float(keys)
@@ -317,21 +341,22 @@ class Problem:
         B, H, S, D = w.shape
         self.O = torch.empty(B, H, S, D, dtype=torch.bfloat16, device=dev)
         self.LSE = torch.empty(B, H, S, dtype=torch.float32, device=dev)
-        self.opts = qsm.make_opts(dtype=qsm.DTYPE_FP8_E4M3 if w.dtype == "fp8" else 0,
-                                  q_descale=d["q_descale"], k_descale=d["k_descale"],
-                                  v_descale=d["v_descale"])
-        self.modes = [m for m in w.modes if maps is None or mode_label(m) in maps]
+        self.opts = [qsm.make_opts(dtype=qsm.DTYPE_FP8_E4M3 if w.dtype == "fp8" else 0,
+                                   q_descale=d["q_descale"], k_descale=d["k_descale"],
+                                   v_descale=d["v_descale"], anchor=anchor)
+                     for anchor in (0, 1)]
+        self.modes = [m for m in step_maps(w) if maps is None or mode_label(m) in maps]
         self.qsm = qsm
         self.i = 0
 
     def call(self, m, stream, O=None, q=None, k=None, v=None):
-        mode, K, cal, rnd = m
+        mode, K, cal, rnd, anchor = m
         c = self.i % self.ncopy
         st = self.qsm.qsm_attn_fwd(q if q is not None else self.q[c],
                                    k if k is not None else self.k[c],
                                    v if v is not None else self.v[c],
                                    self.O if O is None else O, self.LSE, self.w.causal, mode, K,
-                                   cal, rnd, 0, self.opts, stream)
+                                   cal, rnd, 0, self.opts[anchor], stream)
         if st != 0:
             raise RuntimeError("qsm_attn_fwd: " + self.qsm.qsm_status_string(st))
         self.i += 1
@@ -666,7 +691,7 @@ def run_reference(args):
                                        "causal": w.causal, "dtype": dtype_name(w)}
                               for w in wls},
                    "maps": ["%s/%s" % (dtype_name(w), mode_label(m)) for w in wls
-                            for m in w.modes],
+                            for m in step_maps(w)],
                    "step": "a bounded sample of query rows of every (dtype, map) forward"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"],
                          "kind": "oracle", "sample": last["sample"]},

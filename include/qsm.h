@@ -121,6 +121,24 @@ typedef struct {
   int debug_flags;        /* test hooks, 0 in normal use; bit 0: the forward's
                              load warp issues no loads, so every consumer wait
                              runs out (exercises the timeout path) */
+  int anchor;             /* where the maps are anchored (default 0):
+                             0: at the row's final maximum (and minimum): a
+                                statistics sweep, then the weights -- the maps
+                                exactly as defined above;
+                             1: at the row's running maximum after each key
+                                tile of 128 keys, tiles in increasing key
+                                order, in one sweep (the form a one-sweep
+                                kernel such as the pages' FlashAttention-4
+                                patch can take; "Rowmax-H15 in FlashAttention-4
+                                on B200", wiki flowchart).  Earlier tiles are
+                                carried over by 2^-rne((a_t - a_{t-1}) log2 e)
+                                (Rowmax-PoT: every weight stays a power of two)
+                                or exp(a_{t-1} - a_t) (exact: softmax, the
+                                online softmax; K-interval: fixed-window
+                                calibration only, QSM_ERR_UNSUPPORTED for
+                                min-max).  Only row_hi / row_lo are written
+                                (row_argmax / row_argmin must be NULL), and the
+                                backward accepts it for the exact map only. */
 } qsm_opts;
 
 /* Fill *opts with the defaults listed above. */

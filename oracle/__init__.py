@@ -13,7 +13,10 @@ Contents
 --------
 ``attention``  fp64 NumPy restatement of the forward weight maps, the attention
                forward and the K-interval backward (one row at a time,
-               vectorised over rows only; no tiling, no online rescaling).
+               vectorised over rows only; no tiling, no online rescaling),
+               and the online-anchor maps (attn_fwd_online: the anchor of
+               each key tile is the running maximum after it, tiles in key
+               order -- a reading of the one-sweep kernel on the pages).
 ``fp32_spec``  a separately written C restatement of the fp32 weight-map
                specification (the op sequence the GPU map must reproduce bit
                for bit), loaded through ctypes.
@@ -40,5 +43,5 @@ from .attention import (  # noqa: F401
     SURR_NONE, SURR_PRE, SURR_POST,
     LOG2E,
     row_scores, row_stats, kint_grid, weight_map, attn_fwd, attn_bwd,
-    attn_bwd_rows,
+    attn_bwd_rows, attn_fwd_online,
 )

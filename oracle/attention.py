@@ -388,3 +388,141 @@ def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
             dK[b, h] += c * (ds.T @ q[b, h, rr])
             dV[b, h] += P.T @ dO[b, h, rr]
     return dict(dQ=dQ, dK=dK, dV=dV)
+
+
+# ---------------------------------------------------------------------------
+# Online-anchor maps (one sweep over key tiles)
+#
+# The pages' kernel is a patch to a one-sweep attention kernel ("Rowmax-H15 in
+# FlashAttention-4 on B200", wiki flowchart: QK tile -> row max (anchor) ->
+# power-of-two weights -> PV), which only knows the maximum of the keys it has
+# visited so far.  The pages do not state how such a kernel anchors its
+# weights; the reading coded here (the build's choice) anchors each key tile
+# at the running maximum of the row after that tile, in increasing key order,
+# and carries the earlier tiles' accumulators over by the factor the anchor's
+# move implies:
+#
+#   tiles t = 0, 1, ... of `tile` consecutive keys; a_t = max(a_{t-1}, max of
+#   the row's valid scores in tile t), a_{-1} = -inf (a tile with no valid key
+#   of the row changes nothing)
+#   Rowmax-PoT   k_t = rne((a_t - a_{t-1}) log2 e) (0 for the row's first
+#                tile); n_j = min(rne((a_t - s_j) log2 e), N) (or flushed past
+#                N); O <- O 2^-k_t + sum_j 2^-n_j v_j, Z <- Z 2^-k_t + sum 2^-n_j.
+#                Every weight stays a power of two.
+#   K-interval (fixed window only): the grid of tile t spans [a_t - W, a_t]
+#                (step W/K, values g_k = exp(-(K-k) W/K)); w_j read off it by
+#                interpolation or hard rounding as in the two-sweep map;
+#                O <- O exp(a_{t-1} - a_t) + sum_j w_j v_j, Z likewise.
+#   Exact        w_j = exp(s_j - a_t), rescaled by exp(a_{t-1} - a_t): the
+#                online softmax recursion, equal to softmax.
+#   O_r = O / Z * v_descale, LSE_r = a_last + ln Z.
+# Min-max calibration has no online form here: its grid depends on the
+# running minimum as well, so the grid would move with nearly every tile.
+# ---------------------------------------------------------------------------
+
+def attn_fwd_online(q, k, v, causal, mode, K=4, rounding=HARD, scale=None,
+                    q_descale=1.0, k_descale=1.0, v_descale=1.0, window=8.0,
+                    pot_floor=15, below_policy=0, tile=128, heads=None,
+                    rows=None, row_block=512, want_idx=False):
+    """Attention forward with the online-anchor maps (see the block comment
+    above); [B, H, S, D] inputs.  K-interval uses fixed-window calibration.
+    Returns the dict of attn_fwd (hi = the last anchor = the row maximum; lo =
+    hi - W for K-interval, the row minimum otherwise; argmax/argmin -1), with
+    ``idx`` the per-element decision against its tile's anchor."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    B, H, S, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    c = float(scale) * float(q_descale) * float(k_descale)
+    O = np.full((B, H, S, v.shape[-1]), np.nan)
+    LSE = np.full((B, H, S), np.nan)
+    HI = np.full((B, H, S), np.nan)
+    LO = np.full((B, H, S), np.nan)
+    IDX = np.full((B, H, S, S), IDX_MASKED, dtype=np.int8) if want_idx else None
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    row_list = np.arange(S) if rows is None else np.asarray(rows)
+    delta = window / K
+    g = np.exp(-(K - np.arange(K + 1, dtype=np.float64)) * delta)
+    for (b, h) in heads:
+        for i0 in range(0, len(row_list), row_block):
+            rr = row_list[i0:i0 + row_block]
+            s = c * (q[b, h, rr] @ k[b, h].T)
+            valid = (np.arange(S)[None, :] <= rr[:, None]) if causal \
+                else np.ones_like(s, dtype=bool)
+            R = len(rr)
+            a = np.full(R, -np.inf)
+            Z = np.zeros(R)
+            acc = np.zeros((R, v.shape[-1]))
+            idx = np.full((R, S), IDX_MASKED, dtype=np.int64)
+            for t0 in range(0, S, tile):
+                cols = slice(t0, min(S, t0 + tile))
+                st, vt = s[:, cols], valid[:, cols]
+                seen = vt.any(axis=1)
+                if not seen.any():
+                    continue
+                with np.errstate(invalid="ignore"):
+                    tmax = np.where(vt, st, -np.inf).max(axis=1, initial=-np.inf)
+                    # a NaN score of the tile makes the anchor NaN
+                    tmax = np.where(np.isnan(np.where(vt, st, 0.0)).any(axis=1), np.nan, tmax)
+                    a_new = np.where(seen, np.maximum(a, tmax), a)
+                    first = ~np.isfinite(a) & ~np.isnan(a)      # no key seen yet
+                    if mode == ROWMAX_POT:
+                        kt = np.where(first, 0.0, np.rint((a_new - a) * LOG2E))
+                        fac = np.exp2(-kt)
+                    else:
+                        fac = np.where(first, 1.0, np.exp(a - a_new))
+                fac = np.where(seen, fac, 1.0)
+                Z = Z * fac
+                acc = acc * fac[:, None]
+                with np.errstate(invalid="ignore"):
+                    if mode == EXACT:
+                        w = np.exp(np.where(vt, st, 0.0) - a_new[:, None])
+                        dec = np.zeros_like(st, dtype=np.int64)
+                    elif mode == ROWMAX_POT:
+                        x = (a_new[:, None] - np.where(vt, st, a_new[:, None])) * LOG2E
+                        x = np.where(np.isfinite(a_new)[:, None], x, 0.0)
+                        n = np.rint(x)
+                        fl = (n > pot_floor) if below_policy == 1 else np.zeros_like(vt)
+                        n = np.minimum(n, pot_floor)
+                        w = np.where(fl, 0.0, np.exp2(-n))
+                        dec = np.where(fl, IDX_FLUSHED, n).astype(np.int64)
+                    elif mode == KINTERVAL:
+                        lo_t = a_new - window
+                        u_raw = (np.where(vt, st, a_new[:, None]) - lo_t[:, None]) / delta
+                        u_raw = np.where(np.isfinite(a_new)[:, None], u_raw, float(K))
+                        below = u_raw < 0
+                        u = np.clip(u_raw, 0.0, float(K))
+                        if rounding == HARD:
+                            kk = np.rint(u).astype(np.int64)
+                            w = g[kk]
+                        else:
+                            kk = np.minimum(np.floor(u), K - 1).astype(np.int64)
+                            f = u - kk
+                            w = (1.0 - f) * g[kk] + f * g[kk + 1]
+                        fl = below if below_policy == 1 else np.zeros_like(vt)
+                        w = np.where(fl, 0.0, w)
+                        dec = np.where(fl, IDX_FLUSHED, kk)
+                    else:
+                        raise ValueError("unknown mode %r" % (mode,))
+                w = np.where(vt, w, 0.0)
+                Z = Z + w.sum(axis=1)
+                acc = acc + w @ v[b, h, cols]
+                idx[:, cols] = np.where(vt, dec, IDX_MASKED)
+                a = a_new
+            bad = ~np.isfinite(a)
+            with np.errstate(invalid="ignore", divide="ignore"):
+                O[b, h, rr] = np.where(bad[:, None], np.nan, acc / Z[:, None]) * float(v_descale)
+                LSE[b, h, rr] = np.where(bad, np.nan, a + np.log(Z))
+            HI[b, h, rr] = a
+            if mode == KINTERVAL:
+                LO[b, h, rr] = a - window
+            else:
+                LO[b, h, rr] = np.where(valid, s, np.inf).min(axis=1)
+            if want_idx:
+                IDX[b, h, rr] = idx.astype(np.int8)
+    res = dict(O=O, LSE=LSE, hi=HI, lo=LO, argmax=np.full((B, H, S), -1),
+               argmin=np.full((B, H, S), -1))
+    if want_idx:
+        res["idx"] = IDX
+    return res

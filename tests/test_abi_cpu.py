@@ -34,7 +34,9 @@ def test_status_strings_and_defaults():
     o = qsm.qsm_opts_default()
     assert (o.dtype, o.scale, o.window, o.pot_floor, o.below_policy) == (0, 0.0, 8.0, 15, 0)
     assert (o.q_descale, o.k_descale, o.v_descale) == (1.0, 1.0, 1.0)
-    assert ctypes.sizeof(qsm.QsmOpts) == 112
+    assert ctypes.sizeof(qsm.QsmOpts) == 112          # anchor fills the old tail padding
+    assert qsm.QsmOpts.anchor.offset == 108
+    assert o.anchor == 0
 
 
 FAKE = 1 << 20          # aligned, never dereferenced: every call below fails validation
@@ -69,6 +71,7 @@ def test_fwd_rejects_bad_arguments(kw, want):
     ("below_policy", 2, qsm.QSM_ERR_INVALID_ARG), ("scale", -1.0, qsm.QSM_ERR_INVALID_ARG),
     ("q_descale", 0.0, qsm.QSM_ERR_INVALID_ARG), ("dtype", 7, qsm.QSM_ERR_INVALID_ARG),
     ("dtype", 1, qsm.QSM_ERR_UNSUPPORTED),           # e4m3 needs D = 128
+    ("anchor", 2, qsm.QSM_ERR_INVALID_ARG),
 ])
 def test_fwd_rejects_bad_options(field, val, want):
     o = qsm.qsm_opts_default()
@@ -145,3 +148,21 @@ def test_noalloc_status_matches_the_workspace_backward():
     assert both(1, 128, 96) == (qsm.QSM_ERR_UNSUPPORTED, qsm.QSM_ERR_UNSUPPORTED)
     assert both(0, 128, 64) == (qsm.QSM_ERR_INVALID_ARG, qsm.QSM_ERR_INVALID_ARG)
     assert both(1, 0, 64) == (qsm.QSM_ERR_INVALID_ARG, qsm.QSM_ERR_INVALID_ARG)
+
+
+def test_running_anchor_refusals_before_launch():
+    """anchor = 1 (the one-sweep maps): no min-max K-interval form, no argument
+    statistics, and no backward except for the exact map."""
+    o = qsm.qsm_opts_default()
+    o.anchor = 1
+    assert _fwd(mode=1, calib=0, opts=o) == qsm.QSM_ERR_UNSUPPORTED
+    o.row_argmax = FAKE
+    assert _fwd(mode=2, opts=o) == qsm.QSM_ERR_UNSUPPORTED
+    L = qsm.lib()
+    o = qsm.qsm_opts_default()
+    o.anchor = 1
+    o.row_hi = o.row_lo = o.row_argmax = o.row_argmin = FAKE
+    o.workspace = FAKE
+    o.workspace_bytes = qsm.qsm_attn_bwd_workspace_size(1, 1, 128, 64)
+    assert L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64,
+                          1, 1, 4, 1, 1, 1, ctypes.byref(o), None) == qsm.QSM_ERR_UNSUPPORTED
