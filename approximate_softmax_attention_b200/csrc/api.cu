@@ -173,13 +173,14 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
                                o, &c);
   if (st != QSM_OK) return st;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return QSM_ERR_INVALID_ARG;
-  if (mode == QSM_MODE_ROWMAX_POT || o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
+  if (o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
   // the rules are derived for maps anchored at the final row statistics; the
   // exact map is softmax under either anchor
   if (o.anchor == 1 && mode != QSM_MODE_EXACT) return QSM_ERR_UNSUPPORTED;
   if (mode == QSM_MODE_KINTERVAL &&
       (!o.row_hi || !o.row_lo || !o.row_argmax || !o.row_argmin))
     return QSM_ERR_INVALID_ARG;
+  if (mode == QSM_MODE_ROWMAX_POT && !o.row_hi) return QSM_ERR_INVALID_ARG;
   const size_t need = bwd_workspace_bytes(B, H, S, D);
   if (!o.workspace || o.workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(o.workspace) & 255u))
@@ -190,7 +191,7 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
   a.B = B; a.H = H; a.S = S; a.D = D; a.causal = causal;
   a.mode = mode; a.Kint = Kint; a.calib = calibration; a.rounding = rounding;
   a.surrogate = surrogate; a.detach = o.detach_extrema;
-  a.c = c; a.window = o.window; a.below_policy = o.below_policy;
+  a.c = c; a.window = o.window; a.below_policy = o.below_policy; a.pot_floor = o.pot_floor;
   a.row_hi = o.row_hi; a.row_lo = o.row_lo;
   a.row_argmax = o.row_argmax; a.row_argmin = o.row_argmin;
   a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;

@@ -56,7 +56,7 @@ struct BwdArgs {
   int B, H, S, D, causal;
   int mode, Kint, calib, rounding, surrogate, detach;
   float c, window;
-  int below_policy;
+  int below_policy, pot_floor;
   const float *row_hi, *row_lo;
   const int32_t *row_argmax, *row_argmin;
   void *workspace;

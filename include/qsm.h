@@ -157,12 +157,19 @@ qsm_status qsm_attn_fwd(const void *Q, const void *K, const void *V, void *O, fl
                         qsm_calib calibration, qsm_rounding rounding,
                         qsm_surrogate surrogate, const qsm_opts *opts, qsm_stream_t stream);
 
-/* Backward of qsm_attn_fwd (bf16, EXACT or KINTERVAL).
+/* Backward of qsm_attn_fwd (bf16, D = 64): the exact map, K-interval
+ * attention (K <= 32) and Rowmax-PoT.
  *  Q, K, V, O, dO: device [B,H,S,D] bf16 (O = the forward's output).
  *  LSE:  device [B,H,S] fp32 from the forward.
  *  dQ, dK, dV: device [B,H,S,D] bf16 (written).
- *  K-interval needs opts->row_hi/row_lo/row_argmax/row_argmin from the forward
- *  and opts->workspace.  ROWMAX_POT and e4m3 return QSM_ERR_UNSUPPORTED. */
+ *  The rules are the exact gradients of the surrogate graphs with the
+ *  forward's rounding decisions frozen (see qsm_surrogate).  Rowmax-PoT's
+ *  backward is not derived on the pages; the same surrogates apply to it,
+ *  and with its exponents frozen a power-of-two weight has no derivative of
+ *  its own, nor a calibration term (QSM_SURR_NONE gives dQ = dK = 0).
+ *  K-interval needs opts->row_hi/row_lo/row_argmax/row_argmin from the
+ *  forward, Rowmax-PoT opts->row_hi; all need opts->workspace.  e4m3, D = 128
+ *  and K > 32 return QSM_ERR_UNSUPPORTED. */
 qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void *O,
                         const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
                         int B, int H, int S, int D, int causal, qsm_mode mode, int Kint,
@@ -189,7 +196,7 @@ size_t qsm_attn_bwd_workspace_size(int B, int H, int S, int D);
  * Arguments and results are those of qsm_attn_bwd; opts->workspace and
  * opts->workspace_bytes are ignored.  Returns QSM_ERR_INVALID_ARG when
  * qsm_attn_bwd_workspace_size(B, H, S, D) exceeds QSM_NOALLOC_SCRATCH_BYTES
- * (for D = 64, about 30 000 query rows B*H*S), before any launch.
+ * (for D = 64, about 28 000 query rows B*H*S), before any launch.
  *
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.  The

@@ -267,14 +267,18 @@ def attn_fwd(q, k, v, causal, mode, K=4, calib=MINMAX, rounding=HARD,
 
 def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
                   surrogate=SURR_NONE, detach_extrema=False, window=8.0,
-                  below_policy=0, frozen=None):
+                  below_policy=0, frozen=None, pot_floor=15):
     """Backward of one block of query rows against all keys.
 
     Returns (dS [R,S], P [R,S], O [R,D]): dS is dL/ds (before the factor c
     that maps it to dQ / dK), P the forward probabilities.  The rules are the
     exact gradients of the surrogate graphs named in the module docstring.
+    Rowmax-PoT (its backward is not derived on the pages; these are the same
+    surrogate graphs applied to it): with its exponents frozen a power-of-two
+    weight depends neither on its own score nor on the anchor, so only the
+    surrogate's direct term remains (none: dS = 0).
     """
-    m = _map_rows(s, valid, mode, K, calib, rounding, window, 15,
+    m = _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
                   below_policy, frozen)
     w = m["w"]
     Z = w.sum(axis=1)
@@ -287,8 +291,23 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
     rows = np.arange(R)
     if mode == EXACT:
         return np.where(valid, P * (dp - delta[:, None]), 0.0), P, O
+    if mode == ROWMAX_POT:
+        if surrogate == SURR_NONE:
+            ds = np.zeros_like(s)
+        elif surrogate == SURR_PRE:
+            e = np.where(valid, np.exp(np.where(valid, s, 0.0) - m["hi"][:, None]), 0.0)
+            ds = gw * e
+        elif surrogate == SURR_POST:
+            sm = np.where(valid, s, -np.inf)
+            ex = np.where(valid, np.exp(sm - sm.max(axis=1, keepdims=True)), 0.0)
+            pstar = ex / ex.sum(axis=1, keepdims=True)
+            dstar = (pstar * dp).sum(axis=1)
+            ds = np.where(valid, pstar * (dp - dstar[:, None]), 0.0)
+        else:
+            raise ValueError("unknown surrogate %r" % (surrogate,))
+        return ds, P, O
     if mode != KINTERVAL:
-        raise ValueError("backward is defined for EXACT and KINTERVAL only")
+        raise ValueError("backward is defined for EXACT, KINTERVAL and ROWMAX_POT")
 
     g, kidx, f, u = m["g"], m["kidx"], m["f"], m["u"]
     a, delta_grid = m["a"], m["delta"]
@@ -357,7 +376,7 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
 def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
              surrogate=SURR_NONE, detach_extrema=False, scale=None,
              window=8.0, below_policy=0, heads=None, row_block=512,
-             decisions=None):
+             decisions=None, pot_floor=15):
     """Gradients dQ, dK, dV [B,H,S,D] (float64) of the attention forward.
 
     ``heads`` restricts the work to a list of (b, h); other heads are NaN.
@@ -383,7 +402,8 @@ def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
             fz = None if decisions is None else np.asarray(decisions[b, h, rr], dtype=np.int64)
             ds, P, _ = attn_bwd_rows(s, valid, v[b, h], dO[b, h, rr], mode,
                                      K, calib, rounding, surrogate,
-                                     detach_extrema, window, below_policy, fz)
+                                     detach_extrema, window, below_policy, fz,
+                                     pot_floor)
             dQ[b, h, rr] = c * (ds @ k[b, h])
             dK[b, h] += c * (ds.T @ q[b, h, rr])
             dV[b, h] += P.T @ dO[b, h, rr]

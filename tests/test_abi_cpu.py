@@ -87,7 +87,7 @@ def test_bwd_rejects_bad_arguments():
         o.dtype = dtype
         return L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128,
                               128, 1, mode, 4, 0, 1, 1, ctypes.byref(o), None)
-    assert bwd(mode=2) == qsm.QSM_ERR_UNSUPPORTED           # PoT backward
+    assert bwd(mode=2) == qsm.QSM_ERR_INVALID_ARG           # PoT backward needs row_hi
     assert bwd(mode=1, dtype=1) == qsm.QSM_ERR_UNSUPPORTED  # e4m3 backward
     assert bwd(mode=1) == qsm.QSM_ERR_INVALID_ARG           # no row statistics
     o = qsm.qsm_opts_default()

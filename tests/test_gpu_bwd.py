@@ -120,3 +120,26 @@ def test_diagnostic_forward_decisions_of_the_backward_runs(K, calib, rnd):
     heads = [(0, 0), (3, 7), (7, 11)]
     _, dec = _run(d, True, 1, K, calib, rnd, 1, False, dump=True)
     check_decisions(d, dec, True, 1, K, calib, rnd, 8.0, heads)
+
+
+@pytest.mark.parametrize("surr", [0, 1, 2])
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
+def test_bwd_rowmax_pot(S, causal, surr):
+    """Rowmax-PoT under the surrogate rules (exponents frozen: none gives dQ =
+    dK = 0 and only dV; pre and post the surrogate's direct term)."""
+    d = inputs.draw(1, 2, S, 64, seed=70 + S, with_dO=True)
+    got, _ = _run(d, causal, 2, 4, 0, 1, surr, False)
+    ref = _oracle(d, causal, 2, 4, 0, 1, surr, False)
+    _check(got, ref)
+    if surr == 0:
+        assert np.abs(got[0]).max() == 0 and np.abs(got[1]).max() == 0
+
+
+@pytest.mark.parametrize("surr", [1, 2])
+def test_bwd_rowmax_pot_training_shape(surr):
+    w = inputs.WORKLOADS["train_s1k"]
+    d = inputs.draw_workload(w)
+    heads = [(1, 2), (6, 9)]
+    got, _ = _run(d, True, 2, 4, 0, 1, surr, False)
+    ref = _oracle(d, True, 2, 4, 0, 1, surr, False, heads=heads)
+    _check(got, ref, heads=heads)

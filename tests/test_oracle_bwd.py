@@ -212,3 +212,54 @@ def test_frozen_decisions_input(K, calib, rounding, surrogate):
                                  surrogate, False, W, c)
             fd = (lp - lm) / (2 * h)
             assert abs(fd - G[0, 0, a, d]) <= 1e-6 * max(1.0, abs(fd)), (name, a, d)
+
+
+def _pot_surrogate_loss(q, k, v, dO, n0, s0, hi0, surrogate, c):
+    """The Rowmax-PoT surrogate graphs with the exponents n0 frozen: none, w =
+    2^-n0 (constant); pre, w = 2^-n0 + exp(s - hi0) - exp(s0 - hi0); post, p =
+    2^-n0 normalised + softmax(s) - softmax(s0)."""
+    s = c * (q @ k.T)
+    w0 = np.exp2(-n0)
+    if surrogate == A.SURR_NONE:
+        p = w0 / w0.sum(1, keepdims=True)
+    elif surrogate == A.SURR_PRE:
+        w = w0 + np.exp(s - hi0[:, None]) - np.exp(s0 - hi0[:, None])
+        p = w / w.sum(1, keepdims=True)
+    else:
+        sm = np.exp(s - s.max(1, keepdims=True))
+        sm /= sm.sum(1, keepdims=True)
+        sm0 = np.exp(s0 - s0.max(1, keepdims=True))
+        sm0 /= sm0.sum(1, keepdims=True)
+        p = w0 / w0.sum(1, keepdims=True) + sm - sm0
+    return float((dO * (p @ v)).sum())
+
+
+@pytest.mark.parametrize("surrogate", [A.SURR_NONE, A.SURR_PRE, A.SURR_POST])
+def test_pot_backward_finite_differences(surrogate):
+    """Rowmax-PoT under the same surrogate rules: central differences of the
+    surrogate graph (exponents frozen, floor N = 4 so some weights sit on it)."""
+    rng = np.random.default_rng(7 + surrogate)
+    S, D = 9, 4
+    q, k, v, dO = (rng.normal(size=(S, D)) for _ in range(4))
+    c = 1.5 / math.sqrt(D)
+    res = oracle.attn_bwd(q[None, None], k[None, None], v[None, None], dO[None, None], False,
+                          A.ROWMAX_POT, surrogate=surrogate, scale=c, pot_floor=4)
+    s0 = c * (q @ k.T)
+    hi0 = s0.max(1)
+    n0 = np.minimum(np.rint((hi0[:, None] - s0) / math.log(2.0)), 4)
+    h = 1e-6
+    for name, X, G in (("q", q, res["dQ"]), ("k", k, res["dK"]), ("v", v, res["dV"])):
+        for (i, d) in [(0, 0), (3, 1), (5, 2), (8, 3), (2, 0)]:
+            args = {"q": q, "k": k, "v": v}
+            Xp = X.copy(); Xp[i, d] += h
+            Xm = X.copy(); Xm[i, d] -= h
+            args[name] = Xp
+            lp = _pot_surrogate_loss(args["q"], args["k"], args["v"], dO, n0, s0, hi0,
+                                     surrogate, c)
+            args[name] = Xm
+            lm = _pot_surrogate_loss(args["q"], args["k"], args["v"], dO, n0, s0, hi0,
+                                     surrogate, c)
+            np.testing.assert_allclose(G[0, 0, i, d], (lp - lm) / (2 * h), rtol=1e-6,
+                                       atol=1e-8)
+    if surrogate == A.SURR_NONE:
+        assert np.abs(res["dQ"]).max() == 0 and np.abs(res["dK"]).max() == 0
