@@ -45,6 +45,7 @@ qsm_opts defaults() {
   o.window = 8.0f;
   o.pot_floor = 15;
   o.below_policy = 0;
+  o.support = 4.0f;
   return o;
 }
 
@@ -56,7 +57,7 @@ qsm_status check_common(int B, int H, int S, int D, int causal, int mode, int Ki
   if (B < 1 || H < 1 || S < 1 || S > 65536) return QSM_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 65535) return QSM_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return QSM_ERR_INVALID_ARG;
-  if (mode < QSM_MODE_EXACT || mode > QSM_MODE_ROWMAX_POT) return QSM_ERR_INVALID_ARG;
+  if (mode < QSM_MODE_EXACT || mode > QSM_MODE_UNIFORM) return QSM_ERR_INVALID_ARG;
   if (calib != QSM_CALIB_MINMAX && calib != QSM_CALIB_FIXED_WINDOW) return QSM_ERR_INVALID_ARG;
   if (rounding != QSM_ROUND_INTERP && rounding != QSM_ROUND_HARD) return QSM_ERR_INVALID_ARG;
   if (surrogate < QSM_SURR_NONE || surrogate > QSM_SURR_POST) return QSM_ERR_INVALID_ARG;
@@ -72,6 +73,10 @@ qsm_status check_common(int B, int H, int S, int D, int causal, int mode, int Ki
   if (o.below_policy != 0 && o.below_policy != 1) return QSM_ERR_INVALID_ARG;
   if (o.detach_extrema != 0 && o.detach_extrema != 1) return QSM_ERR_INVALID_ARG;
   if (o.anchor != 0 && o.anchor != 1) return QSM_ERR_INVALID_ARG;
+  if (!(o.support >= 0.0f) || !std::isfinite(o.support)) return QSM_ERR_INVALID_ARG;
+  // the probes are defined against the final row maximum only
+  if (o.anchor == 1 && (mode == QSM_MODE_TRUNCATED || mode == QSM_MODE_UNIFORM))
+    return QSM_ERR_UNSUPPORTED;
   // the running anchor has no min-max form (the grid would follow the
   // running minimum too)
   if (o.anchor == 1 && mode == QSM_MODE_KINTERVAL && calib == QSM_CALIB_MINMAX)
@@ -148,6 +153,7 @@ qsm_status qsm_attn_fwd(const void *Q, const void *K, const void *V, void *O, fl
   a.window = o.window;
   a.pot_floor = o.pot_floor;
   a.below_policy = o.below_policy;
+  a.support = o.support;
   a.row_hi = o.row_hi; a.row_lo = o.row_lo;
   a.row_argmax = o.row_argmax; a.row_argmin = o.row_argmin;
   a.debug_idx = o.debug_idx;
@@ -174,6 +180,8 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
   if (st != QSM_OK) return st;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return QSM_ERR_INVALID_ARG;
   if (o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
+  // the probes are forward-only sensitivity studies
+  if (mode == QSM_MODE_TRUNCATED || mode == QSM_MODE_UNIFORM) return QSM_ERR_UNSUPPORTED;
   // the rules are derived for maps anchored at the final row statistics; the
   // exact map is softmax under either anchor
   if (o.anchor == 1 && mode != QSM_MODE_EXACT) return QSM_ERR_UNSUPPORTED;
@@ -212,9 +220,10 @@ qsm_status qsm_weight_map(const float *scores, const int32_t *valid_len, int row
   const qsm_opts o = opts ? *opts : defaults();
   if (!scores || !valid_len || !w) return QSM_ERR_INVALID_ARG;
   if (rows < 1 || cols < 1) return QSM_ERR_INVALID_ARG;
-  if (mode < QSM_MODE_EXACT || mode > QSM_MODE_ROWMAX_POT) return QSM_ERR_INVALID_ARG;
+  if (mode < QSM_MODE_EXACT || mode > QSM_MODE_UNIFORM) return QSM_ERR_INVALID_ARG;
   if (calibration != QSM_CALIB_MINMAX && calibration != QSM_CALIB_FIXED_WINDOW)
     return QSM_ERR_INVALID_ARG;
+  if (!(o.support >= 0.0f) || !std::isfinite(o.support)) return QSM_ERR_INVALID_ARG;
   if (rounding != QSM_ROUND_INTERP && rounding != QSM_ROUND_HARD) return QSM_ERR_INVALID_ARG;
   if (mode == QSM_MODE_KINTERVAL && (Kint < 1 || Kint > 64)) return QSM_ERR_INVALID_ARG;
   if (!finite_pos(o.window) || o.pot_floor < 0 || o.pot_floor > 126) return QSM_ERR_INVALID_ARG;
@@ -228,6 +237,7 @@ qsm_status qsm_weight_map(const float *scores, const int32_t *valid_len, int row
   a.scores = scores; a.c = c; a.valid_len = valid_len; a.rows = rows; a.cols = cols;
   a.mode = mode; a.Kint = Kint; a.calib = calibration; a.rounding = rounding;
   a.window = o.window; a.pot_floor = o.pot_floor; a.below_policy = o.below_policy;
+  a.support = o.support;
   a.w = w; a.idx = idx; a.hi = hi; a.lo = lo;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
   return launch_weight_map(a);

@@ -54,6 +54,7 @@ struct FwdParams {
   float window;
   float v_descale;
   float pscale;     // P is stored as w * pscale (FP8 approximate maps: 64)
+  float thr;        // probes: -(support width * log2e)
   int tab_stride;   // floats of grid table
   int num_stages;
   uint32_t table_off, bar_off, xch_off;
@@ -419,6 +420,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   mc.cL2E = p.cL2E;
   mc.window = p.window;
   mc.pscale = p.pscale;
+  mc.thr = p.thr;
   const bool pot_flush = MAP == MAP_POT && p.flush;
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush &&
                            p.fixed_window;
@@ -789,7 +791,10 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.c = a.c;
   p.cL2E = a.c * 1.4426950408889634f;
   p.window = a.window;
-  p.pscale = (FP8 && MAP != MAP_EXACT) ? 64.0f : 1.0f;
+  // P carries 64 w in e4m3 for the maps whose weights reach 2^-15 exactly
+  // (the exact and truncated maps keep w: ex2 values are not e4m3-exact anyway)
+  p.pscale = (FP8 && MAP != MAP_EXACT && MAP != MAP_TRUNC) ? 64.0f : 1.0f;
+  p.thr = -a.support * 1.4426950408889634f;
   p.v_descale = a.v_descale;
   p.O = static_cast<__nv_bfloat16 *>(a.O);
   p.LSE = a.LSE;
@@ -850,6 +855,8 @@ static qsm_status launch_d(const FwdArgs &a, const CUtensorMap &mq, const CUtens
                            const CUtensorMap &mv) {
   if (a.mode == QSM_MODE_EXACT) return launch_t<D, FP8, MAP_EXACT>(a, mq, mk, mv);
   if (a.mode == QSM_MODE_ROWMAX_POT) return launch_t<D, FP8, MAP_POT>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_TRUNCATED) return launch_t<D, FP8, MAP_TRUNC>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_UNIFORM) return launch_t<D, FP8, MAP_UNIFORM>(a, mq, mk, mv);
   if (a.rounding == QSM_ROUND_HARD) return launch_t<D, FP8, MAP_KI_HARD>(a, mq, mk, mv);
   return launch_t<D, FP8, MAP_KI_INTERP>(a, mq, mk, mv);
 }

@@ -236,6 +236,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   mc.cL2E = p.cL2E;
   mc.window = p.window;
   mc.pscale = p.pscale;
+  mc.thr = 0.0f;
   if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
     // the fixed-window grid values do not depend on the anchor: one table,
     // built once (the three groups take interleaved entries of each row)

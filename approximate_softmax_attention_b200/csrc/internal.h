@@ -21,6 +21,7 @@ struct FwdArgs {
   float v_descale;
   float window;
   int pot_floor, below_policy;
+  float support;    // probes: support width T (natural-log units of s)
   float *row_hi, *row_lo;
   int32_t *row_argmax, *row_argmin;
   int8_t *debug_idx;
@@ -41,6 +42,7 @@ struct MapArgs {
   int mode, Kint, calib, rounding;
   float window;
   int pot_floor, below_policy;
+  float support;
   float *w;
   int32_t *idx;
   float *hi, *lo;

@@ -24,6 +24,8 @@
 //                       (c_k, d_k) = (g_k - k d_k, g_{k+1} - g_k), entry K
 //                       repeating entry K-1; w = fma(uc, d_k, c_k)
 //   grid        g[k] = own_exp(-(K-k) * step), step = a/K or W/K
+//   probes      x as for the exact map; kept when x >= thr = -(T*log2e):
+//               truncated w = 2^x (ex2.approx), uniform w = 1; 0 when cut
 //
 // Every operation is an explicit round-to-nearest (or round-down) intrinsic,
 // so the compiler can neither contract nor reorder it, and an IEEE fp32
@@ -37,7 +39,12 @@
 
 namespace qsm {
 
-enum MapKind { MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3 };
+enum MapKind {
+  MAP_EXACT = 0, MAP_POT = 1, MAP_KI_HARD = 2, MAP_KI_INTERP = 3,
+  // the sensitivity probes: keys within the support width of the row
+  // maximum keep their exact weight (TRUNC) or weight 1 (UNIFORM), the rest 0
+  MAP_TRUNC = 4, MAP_UNIFORM = 5
+};
 
 constexpr float kMagic = 12582912.0f;                  // 1.5 * 2^23
 constexpr uint32_t kMagicBits = 0x4B400000u;
@@ -176,6 +183,7 @@ struct MapCall {
   float cL2E;       // c * log2(e)
   float window;
   float pscale;     // weights are produced as w * pscale (FP8 P: 64)
+  float thr;        // probes: the support threshold -(T * log2e)
 };
 
 // Grid table layout: node n of the row in table column `row` (0..127) sits at
@@ -205,6 +213,12 @@ __device__ __forceinline__ MapRow row_setup(const MapCall &mc, float rmax, float
   hi = __fmul_rn(mc.c, rmax);
   lo = __fmul_rn(mc.c, rmin);
   if (MAP == MAP_EXACT) return mr;
+  if (MAP == MAP_TRUNC || MAP == MAP_UNIFORM) {
+    mr.a = mc.cL2E;
+    mr.b = -mr.mL2E;
+    mr.cap = mc.thr;
+    return mr;
+  }
   const RowMap rm = make_rowmap(hi, lo, mc.K, mc.fixed_window != 0, mc.window);
   if (MAP == MAP_POT) {
     mr.a = -mc.cL2E;
@@ -246,7 +260,14 @@ __device__ __forceinline__ MapRow row_setup(const MapCall &mc, float rmax, float
 template <int MAP, bool FLUSH>
 __device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
   const float2 x = fma2_rn(r, make_float2(m.a, m.a), make_float2(m.b, m.b));
-  if (MAP == MAP_POT) {
+  if (MAP == MAP_TRUNC || MAP == MAP_UNIFORM) {
+    float2 w = (MAP == MAP_TRUNC) ? make_float2(ex2_approx(x.x), ex2_approx(x.y))
+                                  : make_float2(__uint_as_float(m.pow_bias),
+                                                __uint_as_float(m.pow_bias));
+    if (!(x.x >= m.cap)) w.x = 0.0f;
+    if (!(x.y >= m.cap)) w.y = 0.0f;
+    return w;
+  } else if (MAP == MAP_POT) {
     const float2 t =
         add2_rn(make_float2(fminf(x.x, m.cap), fminf(x.y, m.cap)), make_float2(kMagic, kMagic));
     // 2^-n * pscale from the exponent field: bits(t) = kMagicBits + n and
@@ -306,6 +327,7 @@ template <int MAP>
 __device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flush, int N) {
   if (MAP == MAP_EXACT) return 0;
   const float x = __fmaf_rn(r, m.a, m.b);
+  if (MAP == MAP_TRUNC || MAP == MAP_UNIFORM) return x >= m.cap ? 0 : -2;
   if (MAP == MAP_POT) {
     const int n = static_cast<int>(__float_as_uint(__fadd_rn(fminf(x, m.cap), kMagic)) -
                                    kMagicBits);

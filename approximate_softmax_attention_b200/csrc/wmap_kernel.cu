@@ -97,7 +97,10 @@ qsm_status launch_weight_map(const MapArgs &a) {
   mc.cL2E = a.c * 1.4426950408889634f;
   mc.window = a.window;
   mc.pscale = 1.0f;
+  mc.thr = -a.support * 1.4426950408889634f;
   if (a.mode == QSM_MODE_EXACT) return launch_map_t<MAP_EXACT, false>(a, mc);
+  if (a.mode == QSM_MODE_TRUNCATED) return launch_map_t<MAP_TRUNC, false>(a, mc);
+  if (a.mode == QSM_MODE_UNIFORM) return launch_map_t<MAP_UNIFORM, false>(a, mc);
   if (a.mode == QSM_MODE_ROWMAX_POT)
     return mc.flush ? launch_map_t<MAP_POT, true>(a, mc) : launch_map_t<MAP_POT, false>(a, mc);
   if (a.rounding == QSM_ROUND_HARD) return launch_map_t<MAP_KI_HARD, false>(a, mc);

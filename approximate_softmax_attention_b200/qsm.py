@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libqsm.so")
 
 # enums of include/qsm.h
 QSM_OK, QSM_ERR_INVALID_ARG, QSM_ERR_UNSUPPORTED, QSM_ERR_CUDA, QSM_ERR_TIMEOUT = range(5)
-MODE_EXACT, MODE_KINTERVAL, MODE_ROWMAX_POT = 0, 1, 2
+MODE_EXACT, MODE_KINTERVAL, MODE_ROWMAX_POT, MODE_TRUNCATED, MODE_UNIFORM = 0, 1, 2, 3, 4
 CALIB_MINMAX, CALIB_FIXED_WINDOW = 0, 1
 ROUND_INTERP, ROUND_HARD = 0, 1
 SURR_NONE, SURR_PRE, SURR_POST = 0, 1, 2
@@ -54,6 +54,7 @@ class QsmOpts(ctypes.Structure):
         ("debug_idx", ctypes.c_void_p),
         ("debug_flags", ctypes.c_int),
         ("anchor", ctypes.c_int),
+        ("support", ctypes.c_float),
     ]
 
 
@@ -201,7 +202,7 @@ def attention_forward(q, k, v, causal=False, mode=MODE_EXACT, Kint=4,
                       calibration=CALIB_MINMAX, rounding=ROUND_HARD, *, scale=None,
                       q_descale=1.0, k_descale=1.0, v_descale=1.0, window=8.0, pot_floor=15,
                       below_policy=0, stats=False, debug_idx=None, anchor=ANCHOR_FINAL,
-                      stream=None):
+                      support=4.0, stream=None):
     """Allocate the outputs with torch and run ``qsm_attn_fwd``.
 
     Returns (O, LSE) or (O, LSE, stats dict) with hi, lo, argmax, argmin
@@ -215,7 +216,8 @@ def attention_forward(q, k, v, causal=False, mode=MODE_EXACT, Kint=4,
     kw = dict(dtype=DTYPE_FP8_E4M3 if q.dtype == torch.float8_e4m3fn else DTYPE_BF16,
               scale=0.0 if scale is None else float(scale), q_descale=float(q_descale),
               k_descale=float(k_descale), v_descale=float(v_descale), window=float(window),
-              pot_floor=int(pot_floor), below_policy=int(below_policy), anchor=int(anchor))
+              pot_floor=int(pot_floor), below_policy=int(below_policy), anchor=int(anchor),
+              support=float(support))
     if stats:
         st = dict(hi=torch.empty(B, H, S, dtype=torch.float32, device=dev),
                   lo=torch.empty(B, H, S, dtype=torch.float32, device=dev))

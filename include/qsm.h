@@ -65,7 +65,20 @@ typedef enum {
  *  ROWMAX_POT: "coarse logarithmic weight representation anchored at each row
  *              maximum" (arXiv 2609.33586, abstract): n = round((hi-s) log2 e),
  *              clamped to pot_floor, w = 2^-n; w = 1 exactly at the row max. */
-typedef enum { QSM_MODE_EXACT = 0, QSM_MODE_KINTERVAL = 1, QSM_MODE_ROWMAX_POT = 2 } qsm_mode;
+typedef enum {
+  QSM_MODE_EXACT = 0,
+  QSM_MODE_KINTERVAL = 1,
+  QSM_MODE_ROWMAX_POT = 2,
+  /* The sensitivity probes of "Approximating Softmax in Pretrained LLMs"
+   * (abstract: the number of positions can be cut substantially, yet uniform
+   * weighting of them is damaging), read as maps on the same kernel: the kept
+   * positions are the valid keys within opts->support of the row maximum
+   * (s >= hi - support).  TRUNCATED: exp(s - hi) on them; UNIFORM: 1 on
+   * them; 0 on every other key.  Forward only, anchored at the final row
+   * maximum (two sweeps). */
+  QSM_MODE_TRUNCATED = 3,
+  QSM_MODE_UNIFORM = 4
+} qsm_mode;
 
 /* K-interval grid calibration ("per-row grid calibration", arXiv 2609.33591):
  *  MINMAX: lo = the row's minimum score.  FIXED_WINDOW: lo = hi - window. */
@@ -139,6 +152,8 @@ typedef struct {
                                 min-max).  Only row_hi / row_lo are written
                                 (row_argmax / row_argmin must be NULL), and the
                                 backward accepts it for the exact map only. */
+  float support;          /* probes (TRUNCATED, UNIFORM): the support width T
+                             in units of s, >= 0 (default 4) */
 } qsm_opts;
 
 /* Fill *opts with the defaults listed above. */

@@ -37,7 +37,7 @@ unpinned" here; at present there are none.
 """
 
 from .attention import (  # noqa: F401
-    EXACT, KINTERVAL, ROWMAX_POT,
+    EXACT, KINTERVAL, ROWMAX_POT, TRUNCATED, UNIFORM,
     MINMAX, FIXED_WINDOW,
     INTERP, HARD,
     SURR_NONE, SURR_PRE, SURR_POST,

@@ -59,6 +59,7 @@ import math
 import numpy as np
 
 EXACT, KINTERVAL, ROWMAX_POT = 0, 1, 2
+TRUNCATED, UNIFORM = 3, 4     # the sensitivity probes of paper B (see _map_rows)
 MINMAX, FIXED_WINDOW = 0, 1
 INTERP, HARD = 0, 1
 SURR_NONE, SURR_PRE, SURR_POST = 0, 1, 2
@@ -105,7 +106,7 @@ def kint_grid(K: int, delta: np.ndarray) -> np.ndarray:
 
 
 def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
-              below_policy, frozen=None):
+              below_policy, frozen=None, support=4.0):
     """Apply one weight map to a block of rows; returns a dict of per-row and
     per-element quantities (everything the backward needs, decisions frozen).
 
@@ -134,6 +135,22 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
         w = np.where(badr, np.nan, w)
         idx[valid] = 0
         out.update(w=w, idx=idx, lo_cal=lo)
+        return out
+    if mode in (TRUNCATED, UNIFORM):
+        # "Approximating Softmax in Pretrained LLMs", abstract: the number of
+        # positions can be cut substantially, yet uniform weighting of them
+        # is damaging.  Reading: the kept positions are the valid keys within
+        # `support` (natural-log units of s) of the row maximum; TRUNCATED
+        # keeps their exact weights exp(s - hi), UNIFORM gives each weight 1;
+        # every other key gets 0 (decision index -2).
+        with np.errstate(invalid="ignore"):
+            kept = valid & (s >= hi[:, None] - support)
+            e = np.exp(np.where(valid, s, 0.0) - hi[:, None])
+        w = np.where(kept, e if mode == TRUNCATED else 1.0, 0.0)
+        w = np.where(badr, np.nan, w)
+        idx[valid] = IDX_FLUSHED
+        idx[kept] = 0
+        out.update(w=w, idx=idx, lo_cal=lo, kept=kept)
         return out
     if mode == ROWMAX_POT:
         with np.errstate(invalid="ignore"):
@@ -190,17 +207,18 @@ def _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
 
 
 def weight_map(s, valid, mode, K=4, calib=MINMAX, rounding=HARD, window=8.0,
-               pot_floor=15, below_policy=0):
+               pot_floor=15, below_policy=0, support=4.0):
     """Weights and decision indices of one map on given scores.
 
     ``s``: [R, S] scores, ``valid``: [R, S] bool.  Returns (w, idx, hi, lo)
     where idx is the grid node (hard), the lower node (interp), the PoT
-    exponent, 0 for exact, -1 masked, -2 flushed.
+    exponent, 0 for exact and for a kept key of the probes, -1 masked, -2
+    flushed (or cut, for the probes).
     """
     s = np.asarray(s, dtype=np.float64)
     valid = np.asarray(valid, dtype=bool)
     m = _map_rows(s, valid, mode, K, calib, rounding, window, pot_floor,
-                  below_policy)
+                  below_policy, support=support)
     return m["w"], m["idx"], m["hi"], m["lo"]
 
 
@@ -214,7 +232,7 @@ def _as64(t):
 def attn_fwd(q, k, v, causal, mode, K=4, calib=MINMAX, rounding=HARD,
              scale=None, q_descale=1.0, k_descale=1.0, v_descale=1.0,
              window=8.0, pot_floor=15, below_policy=0, heads=None,
-             rows=None, row_block=512, want_idx=False):
+             rows=None, row_block=512, want_idx=False, support=4.0):
     """Attention forward, [B, H, S, D] inputs.
 
     Returns a dict with O [B,H,S,D], LSE/hi/lo [B,H,S] float64 and
@@ -248,7 +266,7 @@ def attn_fwd(q, k, v, causal, mode, K=4, calib=MINMAX, rounding=HARD,
                 valid = (np.arange(S)[None, :] <= rr[:, None]) if causal \
                     else np.ones_like(s, dtype=bool)
             m = _map_rows(s, valid, mode, K, calib, rounding, window,
-                          pot_floor, below_policy)
+                          pot_floor, below_policy, support=support)
             Z = m["w"].sum(axis=1)
             p = m["w"] / Z[:, None]
             O[b, h, rr] = (p @ v[b, h]) * float(v_descale)

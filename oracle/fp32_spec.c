@@ -37,6 +37,9 @@
  *                     d = g[k'+1] - g[k'] and e = fmaf(-k', d, g[k']) with
  *                     k' = min(k, K-1); w = fmaf(uc, d, e); the decision
  *                     index reported is k'
+ *   TRUNCATED  x as for EXACT; kept when x >= thr, thr = -(T*L2E) (T the
+ *              support width); returns x for a kept key and -inf otherwise
+ *   UNIFORM    the same kept test; w = 1 kept, 0 otherwise
  *   rne(x) = (x + 1.5*2^23) - 1.5*2^23  (round half to even, |x| < 2^22)
  *
  *   spec_exp(x): Cody-Waite reduction x = n*ln2 + r with n = rne(x*log2 e),
@@ -51,6 +54,8 @@
 #define MODE_EXACT 0
 #define MODE_KINTERVAL 1
 #define MODE_POT 2
+#define MODE_TRUNC 3
+#define MODE_UNIFORM 4
 #define CAL_MINMAX 0
 #define CAL_FIXED 1
 #define RND_INTERP 0
@@ -96,7 +101,7 @@ static float nmin(float a, float b) { return (a != a || b != b) ? NAN : (b < a ?
  */
 void spec_map_rows(const float *rin, int rows, int cols, const int *valid_len, float c,
                    int mode, int K, int calib, int rounding, float window,
-                   int pot_floor, int below_policy, float *w, int *idx,
+                   int pot_floor, int below_policy, float support, float *w, int *idx,
                    float *hi_out, float *lo_out) {
     float g[130];
     float cl2e = c * L2E;
@@ -112,6 +117,16 @@ void spec_map_rows(const float *rin, int rows, int cols, const int *valid_len, f
         if (mode == MODE_EXACT) {
             float m = rmax * cl2e;
             for (int j = 0; j < L; ++j) { wr[j] = fmaf(rr[j], cl2e, -m); ir[j] = 0; }
+        } else if (mode == MODE_TRUNC || mode == MODE_UNIFORM) {
+            float m = rmax * cl2e;
+            float thr = -(support * L2E);
+            for (int j = 0; j < L; ++j) {
+                float x = fmaf(rr[j], cl2e, -m);
+                int kept = x >= thr;
+                if (mode == MODE_TRUNC) wr[j] = kept ? x : -INFINITY;
+                else wr[j] = kept ? 1.0f : 0.0f;
+                ir[j] = kept ? 0 : -2;
+            }
         } else if (mode == MODE_POT) {
             float b = hi * L2E;
             float cap = below_policy ? (float)(pot_floor + 1) : (float)pot_floor;

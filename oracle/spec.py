@@ -35,7 +35,7 @@ def load():
         f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                       ctypes.c_float,
                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                      ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                      ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_float,
                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                       ctypes.c_void_p]
         e = lib.spec_exp_vec
@@ -53,11 +53,12 @@ def spec_exp(x) -> np.ndarray:
 
 
 def spec_map(s, valid_len, mode, K=4, calib=0, rounding=1, window=8.0,
-             pot_floor=15, below_policy=0, c=1.0):
+             pot_floor=15, below_policy=0, c=1.0, support=4.0):
     """fp32 map of [rows, cols] raw products ``s`` with score scale ``c``
     (score = c * s); returns (w, idx, hi, lo).  For the exact map ``w`` holds
     the exponent x of the weight 2^x (the GPU evaluates 2^x with its own
-    approximate instruction)."""
+    approximate instruction); for the truncated map it holds that exponent
+    for a kept key and -inf for a cut one."""
     s = np.ascontiguousarray(s, dtype=np.float32)
     rows, cols = s.shape
     vl = np.ascontiguousarray(valid_len, dtype=np.int32)
@@ -69,6 +70,6 @@ def spec_map(s, valid_len, mode, K=4, calib=0, rounding=1, window=8.0,
     load().spec_map_rows(s.ctypes.data, rows, cols, vl.ctypes.data, float(np.float32(c)),
                          int(mode),
                          int(K), int(calib), int(rounding), float(window),
-                         int(pot_floor), int(below_policy), w.ctypes.data,
+                         int(pot_floor), int(below_policy), float(support), w.ctypes.data,
                          idx.ctypes.data, hi.ctypes.data, lo.ctypes.data)
     return w, idx, hi, lo

@@ -34,8 +34,9 @@ def test_status_strings_and_defaults():
     o = qsm.qsm_opts_default()
     assert (o.dtype, o.scale, o.window, o.pot_floor, o.below_policy) == (0, 0.0, 8.0, 15, 0)
     assert (o.q_descale, o.k_descale, o.v_descale) == (1.0, 1.0, 1.0)
-    assert ctypes.sizeof(qsm.QsmOpts) == 112          # anchor fills the old tail padding
-    assert qsm.QsmOpts.anchor.offset == 108
+    assert ctypes.sizeof(qsm.QsmOpts) == 120
+    assert qsm.QsmOpts.anchor.offset == 108 and qsm.QsmOpts.support.offset == 112
+    assert o.support == 4.0
     assert o.anchor == 0
 
 
@@ -55,7 +56,7 @@ def _fwd(**kw):
 @pytest.mark.parametrize("kw,want", [
     (dict(B=0), qsm.QSM_ERR_INVALID_ARG), (dict(S=0), qsm.QSM_ERR_INVALID_ARG),
     (dict(S=70000), qsm.QSM_ERR_INVALID_ARG), (dict(D=96), qsm.QSM_ERR_UNSUPPORTED),
-    (dict(mode=3), qsm.QSM_ERR_INVALID_ARG), (dict(mode=1, Kint=0), qsm.QSM_ERR_INVALID_ARG),
+    (dict(mode=5), qsm.QSM_ERR_INVALID_ARG), (dict(mode=1, Kint=0), qsm.QSM_ERR_INVALID_ARG),
     (dict(mode=1, Kint=65), qsm.QSM_ERR_INVALID_ARG), (dict(calib=2), qsm.QSM_ERR_INVALID_ARG),
     (dict(rnd=5), qsm.QSM_ERR_INVALID_ARG), (dict(surr=3), qsm.QSM_ERR_INVALID_ARG),
     (dict(causal=2), qsm.QSM_ERR_INVALID_ARG), (dict(Q=0), qsm.QSM_ERR_INVALID_ARG),
@@ -72,6 +73,7 @@ def test_fwd_rejects_bad_arguments(kw, want):
     ("q_descale", 0.0, qsm.QSM_ERR_INVALID_ARG), ("dtype", 7, qsm.QSM_ERR_INVALID_ARG),
     ("dtype", 1, qsm.QSM_ERR_UNSUPPORTED),           # e4m3 needs D = 128
     ("anchor", 2, qsm.QSM_ERR_INVALID_ARG),
+    ("support", -1.0, qsm.QSM_ERR_INVALID_ARG), ("support", float("inf"), qsm.QSM_ERR_INVALID_ARG),
 ])
 def test_fwd_rejects_bad_options(field, val, want):
     o = qsm.qsm_opts_default()
@@ -166,3 +168,18 @@ def test_running_anchor_refusals_before_launch():
     o.workspace_bytes = qsm.qsm_attn_bwd_workspace_size(1, 1, 128, 64)
     assert L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64,
                           1, 1, 4, 1, 1, 1, ctypes.byref(o), None) == qsm.QSM_ERR_UNSUPPORTED
+
+
+def test_probe_refusals_before_launch():
+    """The probes are forward-only and anchored at the final row maximum."""
+    o = qsm.qsm_opts_default()
+    o.anchor = 1
+    assert _fwd(mode=3, opts=o) == qsm.QSM_ERR_UNSUPPORTED
+    L = qsm.lib()
+    o = qsm.qsm_opts_default()
+    o.row_hi = o.row_lo = o.row_argmax = o.row_argmin = FAKE
+    o.workspace = FAKE
+    o.workspace_bytes = qsm.qsm_attn_bwd_workspace_size(1, 1, 128, 64)
+    for mode in (3, 4):
+        assert L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64,
+                              1, mode, 4, 0, 1, 1, ctypes.byref(o), None) == qsm.QSM_ERR_UNSUPPORTED

@@ -9,6 +9,8 @@ may legitimately round differently), and weights agree to fp32 accuracy.
 Its own exp is checked against float64 exp over the range the grid uses.
 """
 
+import math
+
 import numpy as np
 import pytest
 
@@ -32,6 +34,8 @@ def _boundary_distance(s64, valid, mode, K, calib, rounding, W):
     coordinate to the nearest rounding boundary of its map."""
     hi = np.where(valid, s64, -np.inf).max(1, keepdims=True)
     lo = np.where(valid, s64, np.inf).min(1, keepdims=True)
+    if mode in (A.TRUNCATED, A.UNIFORM):
+        return np.abs(s64 - (hi - 4.0)) / math.log(2.0)
     if mode == A.ROWMAX_POT:
         x = (hi - s64) * A.LOG2E
         return np.abs(x - np.floor(x) - 0.5)
@@ -43,7 +47,8 @@ def _boundary_distance(s64, valid, mode, K, calib, rounding, W):
     return np.minimum(fr, 1 - fr)
 
 
-CASES = [(A.EXACT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 1)] + \
+CASES = [(A.EXACT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 0), (A.ROWMAX_POT, 4, 0, 1, 1),
+         (A.TRUNCATED, 4, 0, 1, 0), (A.UNIFORM, 4, 0, 1, 0)] + \
     [(A.KINTERVAL, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
     [(A.KINTERVAL, 4, 1, 1, 1), (A.KINTERVAL, 16, 1, 0, 1)]
 
@@ -71,9 +76,9 @@ def test_spec_matches_fp64_oracle(mode, K, calib, rounding, below, c):
                                             below_policy=below)
     # hi = c * max r rounded once to fp32
     assert np.array_equal(hi32, hi64.astype(np.float32))
-    if mode == A.EXACT:
-        # the spec gives the exponent x of 2^x
-        w32 = np.exp2(w32.astype(np.float64)) * valid
+    if mode in (A.EXACT, A.TRUNCATED):
+        # the spec gives the exponent x of 2^x (-inf for a cut key)
+        w32 = np.where(valid, np.exp2(w32.astype(np.float64)), 0.0)
     dist = _boundary_distance(s64, valid, mode, K, calib, rounding, W)
     agree = idx32 == idx64
     assert np.all(agree | (dist < 1e-4)), np.argwhere(~agree & (dist >= 1e-4))[:5]

@@ -34,7 +34,7 @@ def _gpu(x):
 
 # ------------------------------------------------------------ weight map
 
-MAP_CASES = [(0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1)] + \
+MAP_CASES = [(0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1), (3, 4, 0, 1, 0), (4, 4, 0, 1, 0)] + \
     [(1, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
     [(1, 4, 1, 1, 1), (1, 16, 1, 0, 1)]
 
@@ -85,7 +85,7 @@ def test_weight_map_bit_exact(mode, K, calib, rounding, below, scales):
     assert st == qsm.QSM_OK
     torch.cuda.synchronize()
     got = W.cpu().numpy()
-    if mode == 0:
+    if mode in (0, 3):
         x = w_ref.astype(np.float64)
         valid = np.arange(cols)[None, :] < vl[:, None]
         want = np.where(valid, np.exp2(x), 0.0)
@@ -94,6 +94,7 @@ def test_weight_map_bit_exact(mode, K, calib, rounding, below, scales):
         # range flush to zero
         assert np.all(np.abs(got[normal] - want[normal]) <= 2.0 ** -21 * want[normal])
         assert np.all(got[~normal] <= 2.0 ** -126)
+        assert np.all(got[np.isneginf(x)] == 0)          # cut keys of the truncated probe
     else:
         assert np.array_equal(got.view(np.uint32), w_ref.view(np.uint32))
     assert np.array_equal(I.cpu().numpy(), i_ref)
@@ -336,6 +337,43 @@ def test_fwd_nonfinite_scores(mode, K, calib, rounding, below):
     assert mx <= 1e-2 and mean <= 1e-3, (mx, mean)
     finL = ~np.isnan(ref["LSE"])
     np.testing.assert_allclose(got_L[finL], ref["LSE"][finL], atol=2e-3, rtol=1e-4)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("mode", [3, 4])
+@pytest.mark.parametrize("support", [0.0, 1.5, 4.0])
+@pytest.mark.parametrize("S,causal", [(200, False), (384, True)])
+def test_fwd_probe_maps(dtype, mode, support, S, causal):
+    """Support truncation (mode 3) and uniform weighting (mode 4) of the keys
+    within `support` of the row maximum, against the oracle, with decisions."""
+    d = inputs.draw(1, 2, S, 128, seed=60 + S, peaked=True, dtype=dtype)
+    q, k, v = _gpu(d["q"]), _gpu(d["k"]), _gpu(d["v"])
+    dbg = torch.full((1, 2, S, S), -7, dtype=torch.int8, device=DEV)
+    O, LSE = qsm.attention_forward(q, k, v, causal, mode, q_descale=d["q_descale"],
+                                   k_descale=d["k_descale"], v_descale=d["v_descale"],
+                                   support=support, debug_idx=dbg)
+    torch.cuda.synchronize()
+    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, q_descale=d["q_descale"],
+                          k_descale=d["k_descale"], v_descale=d["v_descale"], support=support,
+                          want_idx=True)
+    # a key within rounding of the support edge may land on either side
+    qq = d["q"].double().numpy() * d["q_descale"]
+    kk = d["k"].double().numpy() * d["k_descale"]
+    got_idx = dbg.cpu().numpy().astype(np.int64)
+    edge_rows = np.zeros((1, 2, S), bool)
+    for h in range(2):
+        s = (qq[0, h] @ kk[0, h].T) / math.sqrt(128)
+        valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal else np.ones((S, S), bool)
+        hi = np.where(valid, s, -np.inf).max(1, keepdims=True)
+        near = valid & (np.abs(s - (hi - support)) < 1e-4)
+        mism = (got_idx[0, h] != ref["idx"][0, h]) & valid
+        assert np.all(near[mism]), np.argwhere(mism & ~near)[:5]
+        edge_rows[0, h] = mism.any(1)
+    keep = ~edge_rows
+    tol = 1e-2 if dtype == "bf16" else 5e-2
+    mx, mean = err_stats(O.float().cpu().numpy()[keep], ref["O"][keep])
+    assert mx <= tol and mean <= tol / 10, (mx, mean)
+    np.testing.assert_allclose(LSE.cpu().numpy()[keep], ref["LSE"][keep], atol=2e-3, rtol=1e-4)
 
 
 def _sampled_check(name, tol_max, tol_mean, nheads=3, nrows=96):

@@ -18,6 +18,7 @@ import torch
 
 import oracle
 from oracle import attention as A
+from approximate_softmax_attention_b200 import inputs
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -337,3 +338,57 @@ def test_nonfinite_scores_take_the_maps_limits_or_poison_the_row():
     p = np.array([1.0, e(-1), 0.0, e(-2)]) / (1 + e(-1) + e(-2))
     np.testing.assert_allclose(res["O"][0, 0, :, 0], p @ v[0, 0, :, 0], rtol=1e-14)
     assert np.isnan(res["O"][0, 1]).all() and np.isnan(res["LSE"][0, 1]).all()
+
+
+def test_probe_maps_hand_row_and_limits():
+    """Support truncation and uniform weighting ("Approximating Softmax in
+    Pretrained LLMs", abstract: positions can be cut, uniform weighting of
+    them is damaging), read as: keep the keys within T of the row maximum,
+    with their exact weights or with weight 1."""
+    e = math.exp
+    s = np.array([[0.0, -1.0, -2.5, -4.0]])
+    valid = np.ones_like(s, dtype=bool)
+    w, idx, _, _ = oracle.weight_map(s, valid, A.TRUNCATED, support=2.6)
+    np.testing.assert_allclose(w[0], [1.0, e(-1), e(-2.5), 0.0], rtol=1e-15)
+    assert idx[0].tolist() == [0, 0, 0, -2]
+    w, idx, _, _ = oracle.weight_map(s, valid, A.UNIFORM, support=2.6)
+    assert w[0].tolist() == [1.0, 1.0, 1.0, 0.0]
+    # the boundary is inclusive: a key exactly T below the maximum is kept
+    w, _, _, _ = oracle.weight_map(s, valid, A.UNIFORM, support=2.5)
+    assert w[0].tolist() == [1.0, 1.0, 1.0, 0.0]
+    d = inputs.draw(1, 2, 96, 64, seed=21, peaked=True)
+    for causal in (False, True):
+        ex = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, A.EXACT)
+        tr = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, A.TRUNCATED, support=1e9)
+        np.testing.assert_allclose(tr["O"], ex["O"], atol=1e-14)
+        un = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, A.UNIFORM, support=1e9)
+        v = d["v"].double().numpy()
+        if causal:
+            mean = np.cumsum(v, axis=2) / np.arange(1, 97)[None, None, :, None]
+        else:
+            mean = np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+        np.testing.assert_allclose(un["O"], mean, atol=1e-13)
+        # T = 0 keeps the maximum only: O is the value row of the argmax
+        t0 = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, A.TRUNCATED, support=0.0)
+        am = ex["argmax"]
+        np.testing.assert_allclose(t0["O"], np.take_along_axis(v, am[..., None], axis=2),
+                                   atol=1e-14)
+
+
+def test_probe_maps_brute_force_and_monotone_support():
+    rng = np.random.default_rng(5)
+    for _ in range(30):
+        n = int(rng.integers(1, 8))
+        s = rng.normal(0, 2.0, (1, n))
+        T = float(rng.uniform(0, 4))
+        hi = s.max()
+        kept = [x >= hi - T for x in s[0]]
+        for mode in (A.TRUNCATED, A.UNIFORM):
+            w, _, _, _ = oracle.weight_map(s, np.ones_like(s, bool), mode, support=T)
+            want = [(math.exp(x - hi) if mode == A.TRUNCATED else 1.0) if k else 0.0
+                    for x, k in zip(s[0], kept)]
+            np.testing.assert_allclose(w[0], want, rtol=1e-15)
+    s = rng.normal(0, 2.0, (16, 40))
+    counts = [(oracle.weight_map(s, np.ones_like(s, bool), A.UNIFORM, support=T)[0] > 0).sum()
+              for T in (0.0, 0.5, 1.0, 2.0, 4.0, 100.0)]
+    assert counts == sorted(counts) and counts[0] == 16 and counts[-1] == s.size
