@@ -56,7 +56,7 @@ EXTRA_WORKLOADS = ("s8k_fp8", "s8k_bf16", "s8k_fp8_causal", "s2k_bf16_causal")
 MODE_NAMES = {0: "exact", 1: "kinterval", 2: "rowmax_pot"}
 CALIB_NAMES = {0: "minmax", 1: "fixed_window"}
 ROUND_NAMES = {0: "interp", 1: "hard"}
-KERNEL_SOURCE = os.path.join(ROOT, "approximate_softmax_attention_b200", "csrc", "fwd.cu")
+CSRC = os.path.join(ROOT, "approximate_softmax_attention_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fwd_traffic.json")
 L2_BYTES = 126 * 2 ** 20
 METRIC = ("attn fwd TFLOPS & % of B200 tensor peak per softmax mode, causal/non-causal "
@@ -230,16 +230,22 @@ class ClockSampler:
                 "samples": len(sm), "power_w_median": statistics.median(pw) if pw else None}
 
 
+def source_sha(name):
+    """sha256 prefix of a kernel source file (the key of the traffic records)."""
+    with open(os.path.join(CSRC, name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
 def traffic_for(workload_name, label):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    the current source of the kernel that ran the map (fwd_online.cu for the
+    one-sweep maps, fwd.cu otherwise); else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    with open(KERNEL_SOURCE, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:16]
-    if d.get("kernel_source_sha256_16") != h:
+    src = "fwd_online.cu" if label.endswith("_online") else "fwd.cu"
+    if d.get("sources", {}).get(src) != source_sha(src):
         return None
     e = d.get("entries", {}).get("%s/%s" % (workload_name, label))
     return None if e is None else e.get("dram_bytes_per_launch")
