@@ -15,17 +15,19 @@
 //               exp(a_{t-1} - a_t).
 //
 // One CTA per 128-row query tile (same grid and order as the two-sweep
-// kernel), 512 threads:
+// kernel), 640 threads:
 //   warp 0      TMA producer: Q once, then K and V tiles through a ring (K
 //               three tiles ahead of V).
 //   warp 1      QK issuer: S_j = Q K_j^T into TMEM buffer j % 3.
 //   warp 2      PV issuer: O += P_j V_j, P read from TMEM.
-//   warps 4-15  three map warpgroups; group g maps the key tiles j = g mod 3
+//   warps 4-7   the anchor warpgroup: one thread per query row sweeps every
+//               tile in key order, folds the tile's row maximum into the
+//               running maximum (in its own registers), decides the frame,
+//               publishes both for the tile, and rescales O when the frame
+//               moves (after PV(j-1) has landed, before PV(j)).
+//   warps 8-19  three map warpgroups; group g maps the key tiles j = g mod 3
 //               (buffer g), one thread per query row covering all 128 key
-//               columns.  The tiles' anchors form a chain through shared
-//               memory: the group of tile j takes the running maximum after
-//               tile j-1, folds in its tile's maximum and hands it on before
-//               it computes its weights.
+//               columns, against the anchor published for the tile.
 // TMEM: S / P buffers at columns 0, 128, 256; O at 384.
 //
 // Frames.  The accumulators are kept in a per-row frame `base` (log2 units)
@@ -88,7 +90,7 @@ struct OGeo {
   static constexpr uint32_t IDESC_PV = instr_desc(FMT, true, 128, D);
 };
 
-constexpr int kOnThreads = 512;     // control warpgroup + three map warpgroups
+constexpr int kOnThreads = 640;     // control, anchor and three map warpgroups
 constexpr int kOnGroups = 3;
 constexpr int kOnMapThreads = 128 * kOnGroups;
 constexpr int kOnBufs = 3;
@@ -106,13 +108,13 @@ struct OnBars {
   uint64_t *kv_full, *kv_empty;          // [stages]
   uint64_t *q_full;
   uint64_t *s_full, *p_full, *s_free;    // [kOnBufs]
-  uint64_t *chain;                       // [kOnBufs]: tile j's anchor handed on
+  uint64_t *anc_ready;                   // [kOnBufs]: tile j's anchor and frame published
   uint64_t *tab_ready;                   // the grid table is built
-  uint64_t *o_full, *drain, *zx;
+  uint64_t *o_full, *drain, *fin_ready, *zx;
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr int kOnFixedBars = 1 + 4 * kOnBufs + 1 + 3;
+constexpr int kOnFixedBars = 1 + 4 * kOnBufs + 1 + 4;
 
 __host__ __device__ constexpr size_t on_bar_bytes(int ns) {
   return ((2 * static_cast<size_t>(ns) + kOnFixedBars) * 8 + 8 + 15) & ~static_cast<size_t>(15);
@@ -127,48 +129,31 @@ __device__ __forceinline__ OnBars on_carve(uint8_t *base, int ns) {
   b.s_full = b.q_full + 1;
   b.p_full = b.s_full + kOnBufs;
   b.s_free = b.p_full + kOnBufs;
-  b.chain = b.s_free + kOnBufs;
-  b.tab_ready = b.chain + kOnBufs;
+  b.anc_ready = b.s_free + kOnBufs;
+  b.tab_ready = b.anc_ready + kOnBufs;
   b.o_full = b.tab_ready + 1;
   b.drain = b.o_full + 1;
-  b.zx = b.drain + 1;
+  b.fin_ready = b.drain + 1;
+  b.zx = b.fin_ready + 1;
   b.tmem_slot = reinterpret_cast<uint32_t *>(b.zx + 1);
   b.abort = reinterpret_cast<int *>(b.tmem_slot + 1);
   return b;
 }
 
-// Per-row state shared along the chain (shared memory, one slot per row).
+// Per-row state in shared memory: the anchor published for each buffer's
+// tile, the final values, and the map groups' row sums at the end.
 struct OnRows {
-  float *a;       // running maximum of the raw products r (anchor / c)
-  float *mn;      // running minimum of r (statistics output only)
-  float *base;    // the accumulators' frame (log2 units)
-  float *C;       // PoT: sum of the rounded anchor moves
-  float *zx;      // [kOnGroups][128] row sums at the end
+  float *a, *base, *C;     // [kOnBufs][128]: running max of r, frame, PoT move sum
+  float *fa, *fbase, *fC, *fmn;   // [128]: after the last tile (and the running min)
+  float *zx;               // [kOnGroups][128]
 };
-constexpr size_t kOnRowBytes = (4 + kOnGroups) * 128 * 4;
+constexpr size_t kOnRowBytes = (3 * kOnBufs + 4 + kOnGroups) * 128 * 4;
 
 __device__ __forceinline__ bool on_all(bool x) { return __all_sync(0xffffffffu, x); }
 __device__ __forceinline__ bool on_any(bool x) { return __any_sync(0xffffffffu, x); }
 
 __device__ __forceinline__ bool on_full_tile(const OnParams &p, int qi, int j) {
   return 128 * (j + 1) <= p.S && (!p.causal || j < qi);
-}
-
-// Pack and store the P of one 32-column chunk (chunk c of the tile) into the
-// buffer's columns c*16 (bf16) or c*8 (e4m3): columns this thread has read.
-template <bool FP8>
-__device__ __forceinline__ void store_p(uint32_t taddr, const float (&w)[32]) {
-  if (FP8) {
-    uint32_t pk[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) pk[i] = pack_e4m3x4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-    tmem_st8(taddr, pk);
-  } else {
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(w[2 * i], w[2 * i + 1]);
-    tmem_st16(taddr, pk);
-  }
 }
 
 // 2^(from - to), the factor that carries a value from one frame to another:
@@ -185,13 +170,14 @@ __device__ __forceinline__ float frame_factor(float from, float to) {
   return exp2f(d);
 }
 
-// Weights of one chunk into w[], masked, with the row sum accumulated.
-template <int MAP, bool FULL, bool FLUSH>
-__device__ __forceinline__ void on_weights(const uint32_t (&v)[32], const MapRow &mr, float cL2E,
-                                           float fr, bool flush_below, int c0, int lim,
-                                           float2 (&z)[4], float (&w)[32]) {
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
+// Weights of one 32-column chunk (masked), packed for the PV product and
+// stored into the buffer's columns c*16 (bf16) or c*8 (e4m3) -- columns this
+// thread has already read -- with the row sum accumulated.
+template <int MAP, bool FULL, bool FLUSH, bool FP8>
+__device__ __forceinline__ void on_chunk(const uint32_t (&v)[32], const MapRow &mr, float cL2E,
+                                         float fr, bool flush_below, int c0, int lim,
+                                         float2 (&z)[4], uint32_t taddr) {
+  auto wt = [&](int i) {
     const float2 r = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
     float2 x;
     if (MAP == MAP_EXACT) {
@@ -207,13 +193,134 @@ __device__ __forceinline__ void on_weights(const uint32_t (&v)[32], const MapRow
       x.y = (c0 + 2 * i + 1 < lim) ? x.y : 0.0f;
     }
     z[i & 3] = add2_rn(z[i & 3], x);
-    w[2 * i] = x.x;
-    w[2 * i + 1] = x.y;
+    return x;
+  };
+  if (FP8) {
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 a = wt(2 * i), b = wt(2 * i + 1);
+      pk[i] = pack_e4m3x4(a.x, a.y, b.x, b.y);
+    }
+    tmem_st8(taddr, pk);
+  } else {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float2 a = wt(i);
+      pk[i] = pack_bf16x2(a.x, a.y);
+    }
+    tmem_st16(taddr, pk);
   }
 }
 
+// The frame value F of a tile with running maximum a (raw units): the
+// anchor in log2 units (exact, K-interval); PoT keeps the integer sum of its
+// rounded moves, tracked by the caller.
+template <int MAP>
+__device__ __forceinline__ float anchor_l2e(const OnParams &p, float a) {
+  if (MAP == MAP_EXACT) return __fmul_rn(a, p.cL2E);
+  return __fmul_rn(__fmul_rn(p.c, a), log2e_f());
+}
+
+// The anchor warpgroup.  Thread `row` owns query row qi*128 + row and visits
+// every key tile in order: the tile's row maximum (and minimum) from TMEM, the
+// running maximum, the frame, the published slot for the tile's map group, and
+// the O rescale when the frame moves.
+template <int D, int MAP>
+__device__ __forceinline__ void on_anchor(const OnParams &p, const OnBars &bars, const OnRows &rs,
+                                          int row, uint32_t lane_base, int qi, int n,
+                                          volatile int *abort) {
+  const int qrow = qi * 128 + row;
+  const int L = p.causal ? min(qrow + 1, p.S) : p.S;
+  const bool want_min = p.lo != nullptr && MAP != MAP_KI_HARD && MAP != MAP_KI_INTERP;
+  float a = -INFINITY, mn = INFINITY, base = 0.0f, C = 0.0f, prev_l2e = 0.0f;
+  bool ok = true;
+  for (int j = 0; j < n && ok; ++j) {
+    const int b = j % kOnBufs;
+    ok = on_all(mbar_wait(&bars.s_full[b], (j / kOnBufs) & 1, abort));
+    if (!ok) break;
+    tc_fence_after();
+    const int lim = L - 128 * j;
+    const bool full = on_full_tile(p, qi, j);
+    const uint32_t sb = lane_base + b * 128;
+    float tmax = -INFINITY, tmin = INFINITY;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(sb + 64 * h, v0);
+      tmem_ld32(sb + 64 * h + 32, v1);
+      tmem_wait_ld();
+      reg_fence32(v0);
+      reg_fence32(v1);
+      if (full) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          tmax = max3n(tmax, __uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+          tmax = max3n(tmax, __uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          if (want_min) {
+            tmin = min3n(tmin, __uint_as_float(v0[2 * i]), __uint_as_float(v0[2 * i + 1]));
+            tmin = min3n(tmin, __uint_as_float(v1[2 * i]), __uint_as_float(v1[2 * i + 1]));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool o0 = 64 * h + i < lim, o1 = 64 * h + 32 + i < lim;
+          const float x0 = __uint_as_float(v0[i]), x1 = __uint_as_float(v1[i]);
+          tmax = max3n(tmax, o0 ? x0 : -INFINITY, o1 ? x1 : -INFINITY);
+          if (want_min) tmin = min3n(tmin, o0 ? x0 : INFINITY, o1 ? x1 : INFINITY);
+        }
+      }
+    }
+    // every row has a valid key in every tile it visits (key 0 in tile 0; a
+    // later tile below the diagonal is full); the NaN-propagating max keeps a
+    // NaN anchor NaN
+    const float an = (lim > 0) ? max3n(a, tmax, tmax) : a;
+    mn = min3n(mn, tmin, tmin);
+    const float l2e = anchor_l2e<MAP>(p, an);
+    if (MAP == MAP_POT && j > 0) C = __fadd_rn(C, rne_f(__fsub_rn(l2e, prev_l2e)));
+    const float F = (MAP == MAP_POT) ? C : l2e;
+    // move the frame to the anchor when the slack runs out (or on a NaN)
+    const float nb = (j == 0 || !(__fsub_rn(F, base) <= p.tau)) ? F : base;
+    const float resc = (j == 0 || nb == base) ? 1.0f : frame_factor<MAP>(base, nb);
+    rs.a[b * 128 + row] = an;
+    rs.base[b * 128 + row] = nb;
+    rs.C[b * 128 + row] = C;
+    mbar_arrive(&bars.anc_ready[b]);
+    if (j > 0 && on_any(resc != 1.0f)) {
+      // O to the new frame, after PV(j-1) has landed (PV(j) waits for this
+      // group's arrival below)
+      const int pj = j - 1;
+      ok = on_all(mbar_wait(&bars.s_free[pj % kOnBufs], (pj / kOnBufs) & 1, abort));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(lane_base + kOnOCol + 32 * c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * resc);
+        tmem_st32(lane_base + kOnOCol + 32 * c, v);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(&bars.p_full[b]);
+    a = an;
+    base = nb;
+    prev_l2e = l2e;
+  }
+  rs.fa[row] = a;
+  rs.fbase[row] = base;
+  rs.fC[row] = C;
+  rs.fmn[row] = mn;
+  mbar_arrive(bars.fin_ready);
+}
+
 // One map warpgroup.  Thread `row` owns query row qi*128 + row (TMEM lane
-// `row`) and maps key tiles j = g, g + 3, ... in S buffer g.
+// `row`) and maps key tiles j = g, g + 3, ... in S buffer g against the
+// anchor and frame the anchor group published for the tile.
 template <int D, bool FP8, int MAP>
 __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, const OnRows &rs,
                                        int g, int row, uint32_t lane_base, int qi, int n, int bh,
@@ -222,7 +329,6 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   const int qrow = qi * 128 + row;
   const bool row_ok = qrow < p.S;
   const int L = p.causal ? min(qrow + 1, p.S) : p.S;
-  const bool want_min = p.lo != nullptr && MAP != MAP_KI_HARD && MAP != MAP_KI_INTERP;
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush;
   const bool pot_flush = MAP == MAP_POT && p.flush;
   bool ok = true;
@@ -259,129 +365,54 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
     const int b = g;                                    // j % 3
     const uint32_t par = (j / kOnBufs) & 1;
     ok = on_all(mbar_wait(&bars.s_full[b], par, abort));
+    if (ok) ok = on_all(mbar_wait(&bars.anc_ready[b], par, abort));
     if (!ok) break;
     tc_fence_after();
-    const int lim = L - 128 * j;                        // valid columns of this row
+    const int lim = L - 128 * j;
     const bool full = on_full_tile(p, qi, j);
     const uint32_t sb = lane_base + b * 128;
-    // ---- pass A: the tile's row maximum (and minimum)
-    float tmax = -INFINITY, tmin = INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
-      tmem_ld32_sync(sb + 32 * c, v);
-      if (full) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          tmax = max3n(tmax, __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          if (want_min) tmin = min3n(tmin, __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = __uint_as_float(v[i]);
-          const bool ok_i = 32 * c + i < lim;
-          tmax = max3n(tmax, ok_i ? x : -INFINITY, ok_i ? x : -INFINITY);
-          if (want_min) tmin = min3n(tmin, ok_i ? x : INFINITY, ok_i ? x : INFINITY);
-        }
-      }
-    }
-    // ---- the chain: the anchor after tile j-1, then this tile's
-    float a_prev = -INFINITY, mn_prev = INFINITY, base = 0.0f, C = 0.0f;
-    if (j > 0) {
-      const int pj = j - 1;
-      ok = on_all(mbar_wait(&bars.chain[pj % kOnBufs], (pj / kOnBufs) & 1, abort));
-      if (!ok) break;
-      a_prev = rs.a[row];
-      mn_prev = rs.mn[row];
-      base = rs.base[row];
-      C = rs.C[row];
-    }
-    // a row with no valid key in this tile (never the case: key 0 is valid
-    // for every row and every later tile below the diagonal is full) keeps
-    // its anchor; the NaN-propagating max keeps a NaN anchor NaN
-    const float a = (lim > 0) ? max3n(a_prev, tmax, tmax) : a_prev;
-    const float mnr = min3n(mn_prev, tmin, tmin);
-    // frame value F of this tile's weights, and the new frame
-    float F;
+    const float a = rs.a[b * 128 + row];
+    const float base = rs.base[b * 128 + row];
     MapRow mr;
-    if (MAP == MAP_POT) {
+    float fr = 1.0f;                                    // K-interval frame factor
+    if (MAP == MAP_EXACT) {
+      mr.mL2E = base;
+    } else if (MAP == MAP_POT) {
       float hi_t, lo_t;
       mr = row_setup<MAP_POT>(mc, a, a, tab, row, 0, 1, hi_t, lo_t);
-      if (j > 0) {
-        float hip, lop;
-        const MapRow pm = row_setup<MAP_POT>(mc, a_prev, a_prev, tab, row, 0, 1, hip, lop);
-        // rounded anchor move, in whole powers of two
-        C = __fadd_rn(C, rne_f(__fsub_rn(mr.b, pm.b)));
-      }
-      F = C;
-    } else if (MAP == MAP_EXACT) {
-      F = __fmul_rn(a, p.cL2E);
-      mr.mL2E = F;
+      mr.pow_bias = __float_as_uint(p.pscale) +
+                    (static_cast<uint32_t>(static_cast<int>(__fsub_rn(rs.C[b * 128 + row], base)))
+                     << 23);
     } else {
+      // n0 = K + 1: no table entry is written (the table is shared and
+      // constant); this only forms the tile's coordinate map
       float hi_t, lo_t;
-      // n0 = K + 1: the per-tile set-up writes no table entry (the table is
-      // shared and constant); it only forms this tile's coordinate map
       mr = row_setup<MAP>(mc, a, a, tab, row, p.K + 1, 1, hi_t, lo_t);
-      F = __fmul_rn(__fmul_rn(p.c, a), log2e_f());
+      fr = exp2f(__fsub_rn(anchor_l2e<MAP>(p, a), base));
     }
-    // move the frame to the anchor when the slack runs out (or on a NaN)
-    const float new_base = (j == 0 || !(__fsub_rn(F, base) <= p.tau)) ? F : base;
-    const float resc = (j == 0 || new_base == base) ? 1.0f : frame_factor<MAP>(base, new_base);
-    rs.a[row] = a;
-    rs.mn[row] = mnr;
-    rs.base[row] = new_base;
-    rs.C[row] = C;
-    mbar_arrive(&bars.chain[j % kOnBufs]);
-    // ---- O rescale (rows whose frame moved), after PV(j-1) has landed
-    if (j > 0 && on_any(resc != 1.0f)) {
-      const int pj = j - 1;
-      ok = on_all(mbar_wait(&bars.s_free[pj % kOnBufs], (pj / kOnBufs) & 1, abort));
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(lane_base + kOnOCol + 32 * c, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * resc);
-        tmem_st32(lane_base + kOnOCol + 32 * c, v);
-      }
-      tmem_wait_st();
-    }
-    // this group's row sums into the new frame
-    if (zset && zbase != new_base) {
-      const float f = frame_factor<MAP>(zbase, new_base);
+    // this group's row sums into the tile's frame
+    if (zset && zbase != base) {
+      const float f = frame_factor<MAP>(zbase, base);
 #pragma unroll
       for (int i = 0; i < 4; ++i) z[i] = make_float2(z[i].x * f, z[i].y * f);
     }
-    zbase = new_base;
+    zbase = base;
     zset = true;
-    // ---- pass B: the weights against the anchor, in the frame
-    float fr = 1.0f;                                    // K-interval frame factor
-    if (MAP == MAP_POT)
-      mr.pow_bias = __float_as_uint(p.pscale) +
-                    (static_cast<uint32_t>(static_cast<int>(__fsub_rn(F, new_base))) << 23);
-    else if (MAP == MAP_EXACT)
-      mr.mL2E = new_base;
-    else
-      fr = exp2f(__fsub_rn(F, new_base));
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t v[32];
       tmem_ld32_sync(sb + 32 * c, v);
-      float w[32];
+      const uint32_t pc = sb + c * PCOLS;
       if (pot_flush) {
         if (full)
-          on_weights<MAP, true, true>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, w);
+          on_chunk<MAP, true, true, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
         else
-          on_weights<MAP, false, true>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, w);
+          on_chunk<MAP, false, true, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
       } else if (full) {
-        on_weights<MAP, true, false>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, w);
+        on_chunk<MAP, true, false, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
       } else {
-        on_weights<MAP, false, false>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, w);
+        on_chunk<MAP, false, false, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
       }
-      store_p<FP8>(sb + c * PCOLS, w);
       if (dbg_row != nullptr) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -402,13 +433,10 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
 
   // ---------------------------------------------------------- epilogue
   if (ok) ok = on_all(mbar_wait(bars.o_full, 0, abort));
-  if (ok && n > 0) {
-    const int lj = n - 1;                              // the last tile's hand-on
-    ok = on_all(mbar_wait(&bars.chain[lj % kOnBufs], (lj / kOnBufs) & 1, abort));
-  }
+  if (ok) ok = on_all(mbar_wait(bars.fin_ready, 0, abort));
   if (!ok) return;
   tc_fence_after();
-  const float a = rs.a[row], base = rs.base[row], Cf = rs.C[row];
+  const float a = rs.fa[row], base = rs.fbase[row], Cf = rs.fC[row];
   const float zg = ((z[0].x + z[0].y) + (z[1].x + z[1].y)) + ((z[2].x + z[2].y) + (z[3].x + z[3].y));
   rs.zx[g * 128 + row] =
       (zset && zg != 0.0f) ? (zbase == base ? zg : zg * frame_factor<MAP>(zbase, base)) : 0.0f;
@@ -418,9 +446,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   const float hi = __fmul_rn(p.c, a);
   // the final weights' frame: the last anchor (exact, K-interval) or the
   // sum of the anchor moves (PoT)
-  const float ref = (MAP == MAP_POT) ? Cf
-                    : (MAP == MAP_EXACT) ? __fmul_rn(a, p.cL2E)
-                                         : __fmul_rn(hi, log2e_f());
+  const float ref = (MAP == MAP_POT) ? Cf : anchor_l2e<MAP>(p, a);
   const bool bad = !(fabsf(hi) <= 3.402823466e38f);
   const float qnan = __int_as_float(0x7FFFFFFF);
   const float oscale = bad ? qnan : p.v_descale / Z;   // pscale and the frame cancel
@@ -443,7 +469,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
     p.LSE[ri] = bad ? qnan : hi + (logf(Z / p.pscale) + __fsub_rn(base, ref) * 0.6931471805599453f);
     if (p.hi) p.hi[ri] = hi;
     if (p.lo) p.lo[ri] = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP)
-                             ? __fsub_rn(hi, p.window) : __fmul_rn(p.c, rs.mn[row]);
+                             ? __fsub_rn(hi, p.window) : __fmul_rn(p.c, rs.fmn[row]);
   }
 }
 
@@ -474,10 +500,13 @@ __global__ void __launch_bounds__(kOnThreads, 1)
   OnRows rs;
   float *rowp = reinterpret_cast<float *>(smem + p.row_off);
   rs.a = rowp;
-  rs.mn = rowp + 128;
-  rs.base = rowp + 256;
-  rs.C = rowp + 384;
-  rs.zx = rowp + 512;
+  rs.base = rowp + kOnBufs * 128;
+  rs.C = rowp + 2 * kOnBufs * 128;
+  rs.fa = rowp + 3 * kOnBufs * 128;
+  rs.fbase = rs.fa + 128;
+  rs.fC = rs.fa + 256;
+  rs.fmn = rs.fa + 384;
+  rs.zx = rs.fa + 512;
   volatile int *abort = bars.abort;
   const int nkvt = (p.S + 127) / 128;
   const int n = p.causal ? min(nkvt, qi + 1) : nkvt;
@@ -490,13 +519,14 @@ __global__ void __launch_bounds__(kOnThreads, 1)
     mbar_init(bars.q_full, 1);
     for (int i = 0; i < kOnBufs; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.p_full[i], 128);
+      mbar_init(&bars.p_full[i], 256);           // the tile's map group + the anchor group
       mbar_init(&bars.s_free[i], 1);
-      mbar_init(&bars.chain[i], 128);
+      mbar_init(&bars.anc_ready[i], 128);
     }
     mbar_init(bars.tab_ready, kOnMapThreads);
     mbar_init(bars.o_full, 1);
     mbar_init(bars.drain, 2);
+    mbar_init(bars.fin_ready, 128);
     mbar_init(bars.zx, kOnMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
@@ -640,9 +670,12 @@ __global__ void __launch_bounds__(kOnThreads, 1)
     }
     commit(bars.drain);
     mbar_wait(bars.drain, 0, abort);
-  } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;
-    on_map<D, FP8, MAP>(p, bars, rs, g, threadIdx.x - 128 - g * 128,
+  } else if (warp >= 4 && warp < 8) {
+    on_anchor<D, MAP>(p, bars, rs, threadIdx.x - 128,
+                      tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, abort);
+  } else if (warp >= 8) {
+    const int g = (warp - 8) >> 2;
+    on_map<D, FP8, MAP>(p, bars, rs, g, threadIdx.x - 256 - g * 128,
                         tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh, sTab,
                         abort);
   }

@@ -416,7 +416,7 @@ def roofline_of(w, label, entry, pk):
             "traffic": traffic_for(w.name, label)}
 
 
-def energy_per_forward(prob, m, stream, dev_index, uuid=None, min_s=0.3):
+def energy_per_forward(prob, m, stream, dev_index, uuid=None, min_s=1.0):
     """Board energy per forward (J) from the NVML total-energy counter, read
     around a loop of forwards (read-only; on a shared machine other users'
     work on other GPUs does not enter this GPU's counter)."""
@@ -510,9 +510,12 @@ def run_ours(args):
         e2e = None if args.no_e2e else run_e2e(probs, owners, stream, dev, args, world)
         energy = None
         if not args.no_energy and rank == 0:
+            # exact and Rowmax-PoT, two-sweep and one-sweep, each dtype: the
+            # pages' comparison (board energy per forward at causal 16K)
             energy = {}
             for j, (p, m) in enumerate(owners):
-                energy[labels[j]] = energy_per_forward(p, m, stream, local, gpu_uuid(dev))
+                if m[0] in (0, 2):
+                    energy[labels[j]] = energy_per_forward(p, m, stream, local, gpu_uuid(dev))
         line = {
             "metric": METRIC,
             "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,

@@ -10,11 +10,14 @@ gradients): against the oracle rounded to bf16, max abs <= 1e-2 (adjacent
 bf16 codes allowed where one bf16 step exceeds 1e-2: the first keys of a
 causal row reach |dV| > 4), mean abs <= 1e-3.
 
-Separately, and only as a labelled diagnostic that no gradient comparison
-uses, the kernel forward's own decisions are checked against fp64 rounding
-(>= 99.9 % agreement, every mismatch within 1e-3 of a boundary): where they
-differ, the oracle's gradients and the kernel's follow different frozen
-decisions, and the tolerance above covers that.
+The kernel's forward takes its rounding decisions in fp32 and may round an
+element within rounding error of a grid node the other way (>= 99.9 %
+agreement, every mismatch within 1e-3 of a boundary: checked first).  Where
+it does, the two sides follow different frozen decisions: the element's own
+slope, and the row's calibration sums dhi / dlo, which land on the whole dQ
+row and on the dK rows of the row's argmax and argmin.  Those gradient rows
+(and the dK / dV rows of the flipped key) are left out of the comparison and
+counted; the oracle itself never sees the kernel's decisions.
 """
 
 import numpy as np
@@ -31,7 +34,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=False):
+def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True):
     q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
     B, H, S, D = q.shape
     dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV) if dump else None
@@ -51,13 +54,42 @@ def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None
                            heads=heads)
 
 
-def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3):
+def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads):
+    """Rows of dQ and of dK / dV touched by the kernel forward's decision
+    mismatches with fp64 rounding (after checking every mismatch lies within
+    1e-3 of a boundary); returns boolean [B,H,S] masks and the count."""
+    B, H, S, _ = d["q"].shape
+    dq = np.zeros((B, H, S), bool)
+    dkv = np.zeros((B, H, S), bool)
+    if mode != 1 or dec is None:
+        return dq, dkv, 0
+    check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads)
+    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, K=K, calib=calib, rounding=rnd,
+                          window=window, heads=heads, want_idx=True)
+    n = 0
+    for (b, h) in heads:
+        valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal \
+            else np.ones((S, S), bool)
+        mism = (dec[b, h].astype(np.int64) != ref["idx"][b, h].astype(np.int64)) & valid
+        rows, keys = np.nonzero(mism)
+        n += len(rows)
+        dq[b, h, rows] = True
+        dkv[b, h, keys] = True
+        dkv[b, h, ref["argmax"][b, h, rows]] = True
+        dkv[b, h, ref["argmin"][b, h, rows]] = True
+    return dq, dkv, n
+
+
+def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3, skip=None):
+    B, H, S, _ = got[0].shape
+    heads = heads or [(b, h) for b in range(B) for h in range(H)]
+    skip_q, skip_kv = skip if skip is not None else (np.zeros((B, H, S), bool),) * 2
     for g, name in zip(got, ("dQ", "dK", "dV")):
         r = ref[name]
-        if heads is not None:
-            g = np.stack([g[b, h] for (b, h) in heads])
-            r = np.stack([r[b, h] for (b, h) in heads])
-        check_bf16_output(g, r, tol_max, tol_mean, what=name)
+        keep = ~(skip_q if name == "dQ" else skip_kv)
+        gg = np.concatenate([g[b, h][keep[b, h]] for (b, h) in heads])
+        rr = np.concatenate([r[b, h][keep[b, h]] for (b, h) in heads])
+        check_bf16_output(gg, rr, tol_max, tol_mean, what=name)
 
 
 COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
@@ -68,9 +100,12 @@ COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
 def test_bwd_kinterval_small(S, causal, K, calib, rnd, surr, detach):
     d = inputs.draw(1, 2, S, 64, seed=50 + S, with_dO=True)
-    got, _ = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
+    got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
     ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
-    _check(got, ref)
+    heads = [(0, 0), (0, 1)]
+    fq, fkv, n = _flip_rows(d, dec, causal, 1, K, calib, rnd, 6.0, heads)
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
 
 
 @pytest.mark.parametrize("K", [1, 32])
@@ -80,15 +115,17 @@ def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
     """K = 1 (one grid segment) and K = 32 (the largest K the backward
     accepts), pre and post surrogate, calibration derivatives on."""
     d = inputs.draw(1, 2, 256, 64, seed=90 + K, with_dO=True)
-    got, _ = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
+    got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
     ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0)
-    _check(got, ref)
+    fq, fkv, n = _flip_rows(d, dec, True, 1, K, calib, rnd, 6.0, [(0, 0), (0, 1)])
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
 
 
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False), (77, True), (384, False)])
 def test_bwd_exact(S, causal):
     d = inputs.draw(1, 2, S, 64, seed=7 + S, with_dO=True)
-    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False)
+    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False, dump=False)
     ref = _oracle(d, causal, 0, 4, 0, 1, 0, False)
     _check(got, ref)
 
@@ -103,23 +140,14 @@ def test_bwd_training_shape_sampled(mode, K, calib, rnd, surr, detach):
     w = inputs.WORKLOADS["train_s1k"]
     d = inputs.draw_workload(w)
     heads = [(0, 0), (3, 7), (7, 11)]
-    got, _ = _run(d, True, mode, K, calib, rnd, surr, detach)
+    got, dec = _run(d, True, mode, K, calib, rnd, surr, detach)
     ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads)
-    _check(got, ref, heads=heads)
+    fq, fkv, n = _flip_rows(d, dec, True, mode, K, calib, rnd, 8.0, heads)
+    _check(got, ref, heads=heads, skip=(fq, fkv))
+    # the flips are rare: a few rows of the three heads checked
+    assert fq.sum() <= 0.01 * 3 * 1024, n
     for g in got:
         assert np.isfinite(g).all()
-
-
-@pytest.mark.parametrize("K,calib,rnd", [(4, 0, 1), (16, 0, 0), (4, 1, 1), (16, 1, 0)])
-def test_diagnostic_forward_decisions_of_the_backward_runs(K, calib, rnd):
-    """Diagnostic only (no gradient comparison uses it): the decisions the
-    kernel's forward takes on the backward's inputs agree with fp64 rounding
-    (>= 99.9 %, mismatches within 1e-3 of a boundary)."""
-    w = inputs.WORKLOADS["train_s1k"]
-    d = inputs.draw_workload(w)
-    heads = [(0, 0), (3, 7), (7, 11)]
-    _, dec = _run(d, True, 1, K, calib, rnd, 1, False, dump=True)
-    check_decisions(d, dec, True, 1, K, calib, rnd, 8.0, heads)
 
 
 @pytest.mark.parametrize("surr", [0, 1, 2])
@@ -128,7 +156,7 @@ def test_bwd_rowmax_pot(S, causal, surr):
     """Rowmax-PoT under the surrogate rules (exponents frozen: none gives dQ =
     dK = 0 and only dV; pre and post the surrogate's direct term)."""
     d = inputs.draw(1, 2, S, 64, seed=70 + S, with_dO=True)
-    got, _ = _run(d, causal, 2, 4, 0, 1, surr, False)
+    got, _ = _run(d, causal, 2, 4, 0, 1, surr, False, dump=False)
     ref = _oracle(d, causal, 2, 4, 0, 1, surr, False)
     _check(got, ref)
     if surr == 0:
@@ -140,6 +168,6 @@ def test_bwd_rowmax_pot_training_shape(surr):
     w = inputs.WORKLOADS["train_s1k"]
     d = inputs.draw_workload(w)
     heads = [(1, 2), (6, 9)]
-    got, _ = _run(d, True, 2, 4, 0, 1, surr, False)
+    got, _ = _run(d, True, 2, 4, 0, 1, surr, False, dump=False)
     ref = _oracle(d, True, 2, 4, 0, 1, surr, False, heads=heads)
     _check(got, ref, heads=heads)
