@@ -557,11 +557,16 @@ __device__ __forceinline__ void calib_elem(const BwdParams &p, float Kf, float i
     }
   } else if (MAP == MAPB_INTERP) {
     const float f = uc - kf;
-    const float g0 = gd.x, slope = gd.y, g1 = gd.x + gd.y;
+    const float slope = gd.y;
     if (!p.fixed_window) {
-      const float mix = ((1.0f - f) * (Kf - kf) * g0 + f * (Kf - kf - 1.0f) * g1) * invK;
-      dhi += gw * (-slope * uc * inv_a - mix);
-      dlo += gw * (-slope * (Kf - uc) * inv_a + mix);
+      // ((1-f)(K-k) g_k + f (K-k-1) g_{k+1}) / K = ((K-k) w - f g_{k+1}) / K
+      // with w = g_k + f (g_{k+1} - g_k) the interpolated weight
+      const float w = gd.x + f * slope;
+      const float mix = ((Kf - kf) * w - f * (gd.x + slope)) * invK;
+      const float ts = gw * slope * inv_a;
+      const float gm = gw * mix;
+      dhi += -ts * uc - gm;
+      dlo += -ts * (Kf - uc) + gm;
     } else if (u >= 0.0f) {
       dhi += gw * (slope * (-Kf / p.window));
     }
