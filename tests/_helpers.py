@@ -76,9 +76,12 @@ def check_bf16_output(got, want, tol_max=1e-2, tol_mean=1e-3, what=""):
     w = np.asarray(want, dtype=np.float64)
     d = np.abs(g - to_bf16(w))
     allow = np.maximum(tol_max, bf16_step(w))
-    worst = float(np.max(d / allow))
+    ratio = d / allow
+    worst = float(np.max(ratio))
     mean = float(np.abs(g - w).mean())
-    assert worst <= 1.0 and mean <= tol_mean, (what, float(d.max()), worst, mean)
+    at = np.unravel_index(int(np.argmax(ratio)), ratio.shape)
+    assert worst <= 1.0 and mean <= tol_mean, (what, float(d.max()), worst, mean, tuple(
+        int(i) for i in at), float(g[at]), float(w[at]), int((ratio > 1.0).sum()))
     return float(d.max()), mean
 
 

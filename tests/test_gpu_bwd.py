@@ -87,8 +87,9 @@ def _check(got, ref, heads=None, tol_max=1e-2, tol_mean=1e-3, skip=None):
     for g, name in zip(got, ("dQ", "dK", "dV")):
         r = ref[name]
         keep = ~(skip_q if name == "dQ" else skip_kv)
-        gg = np.concatenate([g[b, h][keep[b, h]] for (b, h) in heads])
-        rr = np.concatenate([r[b, h][keep[b, h]] for (b, h) in heads])
+        # rows kept, laid out [head, row, D] so a failure reports where it is
+        gg = np.stack([np.where(keep[b, h][:, None], g[b, h], 0.0) for (b, h) in heads])
+        rr = np.stack([np.where(keep[b, h][:, None], r[b, h], 0.0) for (b, h) in heads])
         check_bf16_output(gg, rr, tol_max, tol_mean, what=name)
 
 
