@@ -34,9 +34,9 @@
 // that follows the anchor lazily: the weights written to P are w * 2^(F -
 // base) with F the anchor's own frame value, and O (and the groups' row sums)
 // are rescaled only when F - base would exceed what the P format holds (exact
-// and K-interval: 2^8 in bf16, 2^8 / 2^1 in e4m3 with its 64x P scale; PoT,
-// whose frame value is the integer sum of its rounded anchor moves: 2^64 in
-// bf16, 2^2 in e4m3).  The result is the same up to rounding (PoT: exactly,
+// and K-interval: 2^8 in bf16; e4m3: 2^8 exact, 2^4 K-interval with a 16x P
+// scale; PoT, whose frame value is the integer sum of its rounded anchor
+// moves: 2^64 in bf16, 2^2 in e4m3 with its 64x P scale).  The result is the same up to rounding (PoT: exactly,
 // every factor being a power of two).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -706,15 +706,22 @@ qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMa
   p.cL2E = a.c * 1.4426950408889634f;
   p.window = a.window;
   p.v_descale = a.v_descale;
-  p.pscale = (FP8 && MAP != MAP_EXACT) ? 64.0f : 1.0f;
-  // frame slack (log2 units): P = w * pscale * 2^(F - base) must stay finite
-  // in the P format -- bf16 has fp32's range; e4m3 tops out at 448
-  if (MAP == MAP_POT)
+  // P scale and frame slack (log2 units): P = w * pscale * 2^(F - base) must
+  // stay finite in the P format -- bf16 has fp32's range; e4m3 tops out at
+  // 448.  e4m3 Rowmax-PoT keeps 64 (every weight down to 2^-15 exact) and so
+  // only 2^2 of slack; e4m3 K-interval takes 16 and 2^4 (its smallest
+  // fixed-window weight, e^-8 * 16, is an e4m3 subnormal with the ~6 %
+  // rounding e4m3 gives every weight)
+  if (MAP == MAP_POT) {
+    p.pscale = FP8 ? 64.0f : 1.0f;
     p.tau = FP8 ? 2.0f : 64.0f;
-  else if (MAP == MAP_EXACT)
+  } else if (MAP == MAP_EXACT) {
+    p.pscale = 1.0f;
     p.tau = 8.0f;
-  else
-    p.tau = FP8 ? 1.0f : 8.0f;
+  } else {
+    p.pscale = FP8 ? 16.0f : 1.0f;
+    p.tau = FP8 ? 4.0f : 8.0f;
+  }
   p.O = static_cast<__nv_bfloat16 *>(a.O);
   p.LSE = a.LSE;
   p.hi = a.row_hi;
