@@ -179,6 +179,11 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
                                o, &c);
   if (st != QSM_OK) return st;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return QSM_ERR_INVALID_ARG;
+  // rows are read and written as 16-byte vectors
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+      (reinterpret_cast<uintptr_t>(LSE) & 3u))
+    return QSM_ERR_INVALID_ARG;
   if (o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
   // the probes are forward-only sensitivity studies
   if (mode == QSM_MODE_TRUNCATED || mode == QSM_MODE_UNIFORM) return QSM_ERR_UNSUPPORTED;

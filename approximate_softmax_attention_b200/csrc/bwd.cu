@@ -1,7 +1,7 @@
-// bwd.cu -- backward of the fused attention for the exact map and K-interval
-// attention ("Pretraining Transformers with Quantized Softmax in Attention",
-// abstract: backward rules including calibration derivatives, and a
-// straight-through surrogate placed before or after normalization).
+// bwd.cu -- backward of the fused attention for the exact map, K-interval
+// attention and Rowmax-PoT ("Pretraining Transformers with Quantized Softmax
+// in Attention", abstract: backward rules including calibration derivatives,
+// and a straight-through surrogate placed before or after normalization).
 //
 // Rules (integer decisions of the forward frozen; gw_j = dL/dw_j =
 // (dp_j - delta)/Z with dp_j = dO.v_j, delta = dO.O):
@@ -12,28 +12,34 @@
 //   dlo = sum_j gw_j dF_j/dlo, which belong to ds at the row's argmax /
 //   argmin; they are applied as fp32 rank-one updates.
 //   dQ = c dS K, dK = c dS^T Q, dV = P^T dO.
+// Within one grid interval both calibration derivatives are affine in the
+// coordinate u: interpolation dF/dhi = A_k + B_k u and dF/dhi + dF/dlo =
+// -d_k K/(hi - lo); hard rounding dF/dhi = -dF/dlo = (n - K)/K g_n; fixed
+// window dF/dhi = -d_k K/W.  Each element therefore costs one table read and
+// at most three FMAs for them (the per-node coefficients are built once per
+// row).
 //
 // Kernels, in launch order on the caller's stream:
-//   1. qsm_bwd_delta  delta_r = dO_r . O_r (one warp per row)
-//   2. qsm_bwd_rows   post surrogate only: LSE* and delta* per query row
+//   1. qsm_bwd_rows   post surrogate only: LSE* and delta* per query row
 //                     (S and dP tiles swept once per query tile)
-//   3. qsm_bwd_prep   one thread per query row: the row's map constants and
-//                     its grid table (g_n, g_{n+1} - g_n), written once to
-//                     the workspace for both passes below
-//   4. qsm_bwd_dq     one CTA per 128-row query tile, sweeping the key tiles
-//                     in halves of 64 keys: S = Q K^T and dP = dO V^T into a
-//                     double-buffered TMEM pair, dS by the rule above into
-//                     shared memory, dQ += dS K in TMEM; the calibration sums
-//                     dhi, dlo accumulate per row; the epilogue adds the
-//                     rank-one terms to dQ (fp32) before its bf16 store and
-//                     scatters the dK ones into an fp32 buffer
-//   5. qsm_bwd_dkdv   one CTA per 128-key tile, sweeping the query tiles in
+//   2. qsm_bwd_dq     one CTA per 128-row query tile: each row's delta, map
+//                     constants and grid tables (the dK / dV pass's copies go
+//                     to the workspace), then the key tiles in halves of 64
+//                     keys: S = Q K^T and dP = dO V^T into a double-buffered
+//                     TMEM pair, dS by the rule above into shared memory,
+//                     dQ += dS K in TMEM; the calibration sums accumulate per
+//                     row; the epilogue adds the rank-one terms to dQ (fp32)
+//                     before its bf16 store and scatters the dK ones into an
+//                     fp32 buffer
+//   3. qsm_bwd_dkdv   one CTA per 128-key tile, sweeping the query tiles in
 //                     halves of 64 rows: S^T = K Q^T, dP^T = V dO^T into a
 //                     double-buffered TMEM pair, P^T and dS^T written back to
 //                     TMEM, dV += P^T dO and dK += dS^T Q in TMEM; dK gets the
 //                     fp32 calibration part before its bf16 store
 // Each pass recomputes its products, so no dQ partial sums cross CTAs; the
 // double buffers let the map of one half overlap the products of the next.
+// The element code is specialised per map, surrogate and calibration form,
+// so no per-element branch remains.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,39 +56,41 @@ namespace qsm {
 
 namespace {
 
-// rows pass: warp 0 TMA, warp 1 MMA, warps 4-19 four map groups, group g
-// owning columns 32g .. 32g+31 of every S / dP tile
+// warp 0 TMA, warps 1-2 MMA, warps 4-19 four map groups of 128 threads
 constexpr int kMainThreads = 640;
 constexpr int kMainMapThreads = 512;
 constexpr uint32_t kBwdTmemCols = 512;
 constexpr int kRowWs = 8;               // floats per row in the row workspace
-enum RowWs { RW_DELTA = 0, RW_DHI = 1, RW_DLO = 2, RW_LSESTAR = 3, RW_DELTASTAR = 4 };
+enum RowWs { RW_LSESTAR = 0, RW_DELTASTAR = 1 };
 constexpr int kBwdMaxK = 32;            // largest K the backward accepts
 constexpr int kCst = 8;                 // floats of one query row's map constants
+constexpr float kL2E = 1.4426950408889634f;
+
+constexpr int MAPB_EXACT = 0, MAPB_POT = 1, MAPB_HARD = 2, MAPB_INTERP = 3;
+constexpr int SURR_NONE = QSM_SURR_NONE, SURR_PRE = QSM_SURR_PRE, SURR_POST = QSM_SURR_POST;
+// calibration form of the dQ pass: none (detached, or fixed-window hard
+// rounding, whose weights do not move with hi), min-max, fixed window
+constexpr int CAL_OFF = 0, CAL_MINMAX = 1, CAL_FIXED = 2;
 
 struct BwdParams {
-  int S, nqt, nkvt;
+  int S, nqt, nkvt, BH;
   int causal;
-  int map;          // 0 exact, 1 Rowmax-PoT, 2 K-interval hard, 3 K-interval interp
-  int pot_floor;
-  int K, fixed_window, flush, surrogate, detach;
-  int calib;        // calibration terms on (K-interval, not detached)
-  int KT;           // float2 entries of one row's table in the workspace (K+1, even)
+  int hgroup;       // causal query-tile order: heads per group (see q_tile_order)
+  int K, fixed_window, flush, pot_floor;
+  int TS;           // floats of one query row's dK / dV pass table (a multiple of 4)
   float c, cL2E, window;
   const float *LSE, *hi, *lo;
   const int32_t *amax, *amin;
-  float *rowws;
-  float *cst;       // [rows][kCst] per query row: a, b, 1/Z, delta, e, delta*, inv, 1/(hi-lo)
-  float2 *tabg;     // [rows][KT] per query row: (g_n, g_{n+1} - g_n), n = 0..K
+  float *rowws;     // [rows][kRowWs]: LSE*, delta* (post surrogate)
+  float *cst;       // [rows][kCst]: a, b, 1/Z, -delta/Z, e0, delta_s, K/(hi-lo), 0
+  float *tabk;      // [rows][TS]: the dK / dV pass's grid table of each row
   float *dkcal;     // [rows][D] fp32 calibration part of dK (nullptr: none)
-  const __nv_bfloat16 *Q, *K_;
+  const __nv_bfloat16 *Q, *K_, *O, *dO;
   __nv_bfloat16 *dQ, *dK, *dV;
   int32_t *status;
   int num_stages;
-  uint32_t tab_off, cst_off, ds_off, bar_off, part_off, stage_bytes;
+  uint32_t tab_off, ds_off, bar_off, part_off, stage_bytes;
 };
-
-constexpr int MAPB_EXACT = 0, MAPB_POT = 1, MAPB_HARD = 2, MAPB_INTERP = 3;
 
 template <int D>
 struct BGeo {
@@ -125,29 +133,48 @@ __device__ __forceinline__ void mma_nt_half(uint32_t d_tmem, uint32_t a_saddr, u
   }
 }
 
-// --------------------------------------------------------------- delta
-__global__ void __launch_bounds__(256) qsm_bwd_delta(const __nv_bfloat16 *__restrict__ O,
-                                                     const __nv_bfloat16 *__restrict__ dO,
-                                                     float *__restrict__ rowws, long long rows,
-                                                     int D) {
-  const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  float acc = 0.0f;
-  for (int d = lane * 2; d < D; d += 64) {
-    const __nv_bfloat162 o = *reinterpret_cast<const __nv_bfloat162 *>(O + r * D + d);
-    const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162 *>(dO + r * D + d);
-    acc = fmaf(__bfloat162float(o.x), __bfloat162float(g.x), acc);
-    acc = fmaf(__bfloat162float(o.y), __bfloat162float(g.y), acc);
+// The (head, query tile) of a query-tile CTA on a 1-D grid of nqt * BH:
+// non-causal head after head; causal in groups of hgroup heads (their K / V
+// share L2), heaviest tiles first within a group.
+__device__ __forceinline__ void q_tile_order(const BwdParams &p, int &bh, int &qt) {
+  const int b = static_cast<int>(blockIdx.x);
+  if (p.causal) {
+    const int per = p.hgroup * p.nqt;
+    const int grp = b / per;
+    const int within = b - grp * per;
+    const int h0 = grp * p.hgroup;
+    const int gh = min(p.hgroup, p.BH - h0);
+    const int rank = within / gh;
+    bh = h0 + (within - rank * gh);
+    qt = p.nqt - 1 - rank;
+  } else {
+    qt = b % p.nqt;
+    bh = b / p.nqt;
   }
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) {
-    float *w = rowws + r * kRowWs;
-    w[RW_DELTA] = acc;
-    w[RW_DHI] = 0.0f;
-    w[RW_DLO] = 0.0f;
-    w[RW_LSESTAR] = 0.0f;
-    w[RW_DELTASTAR] = 0.0f;
+}
+
+// bf16 bit patterns to fp32 (exact).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b, float acc) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    acc = __fmaf_rn(bf_lo(aw[k]), bf_lo(bw[k]), acc);
+    acc = __fmaf_rn(bf_hi(aw[k]), bf_hi(bw[k]), acc);
+  }
+  return acc;
+}
+
+// Sixteen bf16 (two uint4) to fp32.
+__device__ __forceinline__ void bf16x16_to_f32(const uint4 *src, float (&x)[16]) {
+  const uint4 a = src[0], b = src[1];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    x[2 * k] = bf_lo(w[k]);
+    x[2 * k + 1] = bf_hi(w[k]);
   }
 }
 
@@ -157,16 +184,16 @@ struct RowBars {
   uint64_t *q_full;
   uint64_t *sd_full, *sd_empty;   // [2]
   uint64_t *drain;
-  uint64_t *tab_ready, *part_ready;   // single use: grid table built; partial sums written
+  uint64_t *part_ready;           // single use: partial sums written
   uint32_t *tmem_slot;
   int *abort;
 };
 
-// --------------------------------------------------------------- rows
 // One CTA per 128 query rows of one (b, h); four map groups, thread = row,
-// group g taking columns 32g .. 32g+31 of every S / dP tile.  Computes the
-// calibration derivatives dhi, dlo and (post surrogate) LSE*, delta*.
-template <int D, int MAP>
+// group g taking columns 32g .. 32g+31 of every S / dP tile.  The post
+// surrogate's row statistics: LSE* = log sum_j exp(s_j) and delta* =
+// sum_j p*_j dp_j, by an online log-sum-exp in log2 units.
+template <int D>
 __global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_rows(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -174,15 +201,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   using G = BGeo<D>;
   constexpr int NS = 4;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int qt = blockIdx.x;
+  int bh, qt;
+  q_tile_order(p, bh, qt);
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;
-  float2 *tab = reinterpret_cast<float2 *>(smem + p.tab_off);
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   RowBars bars;
   bars.kv_full = bp;
@@ -191,11 +216,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.sd_full = bars.q_full + 1;
   bars.sd_empty = bars.sd_full + 2;
   bars.drain = bars.sd_empty + 2;
-  bars.tab_ready = bars.drain + 1;
-  bars.part_ready = bars.tab_ready + 1;
+  bars.part_ready = bars.drain + 1;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.part_ready + 1);
-  // per-row partial sums of the four groups: dhi, dlo, m*, l*, a* ([5][4][128])
-  float *part = reinterpret_cast<float *>(smem + p.cst_off);
+  // per-row partial sums of the four groups: m2, l2, a2 ([3][4][128])
+  float *part = reinterpret_cast<float *>(smem + p.part_off);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
   const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -211,7 +235,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.sd_empty[i], kMainMapThreads);
     }
     mbar_init(bars.drain, 1);
-    mbar_init(bars.tab_ready, kMainMapThreads);
     mbar_init(bars.part_ready, kMainMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
@@ -285,32 +308,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const bool row_ok = qrow < p.S;
     const int L = p.causal ? min(qrow + 1, p.S) : p.S;
     const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-    const float delta = p.rowws[ri * kRowWs + RW_DELTA];
-    const float hi = p.hi[ri];
-    const float lo_in = p.lo != nullptr ? p.lo[ri] : hi;
-    const float Z = expf(p.LSE[ri] - hi);
-    const float invZ = 1.0f / Z;
-    const RowMap rm = make_rowmap(hi, lo_in, p.K, p.fixed_window != 0, p.window);
-    const float a_raw = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
-    const float b_raw = rm.degenerate ? static_cast<float>(p.K) : rm.b;
-    const float Kf = static_cast<float>(p.K);
-    const float invK = 1.0f / Kf;
-    const float a_s = __fsub_rn(hi, rm.lo);        // hi - lo in score units
-    const float inv_a = rm.degenerate ? 0.0f : 1.0f / a_s;
-    const float slope_fw = -Kf / p.window;         // fixed window: d(coordinate)/d(hi) per slope
-    const bool calib = !p.detach && !rm.degenerate;
-    const bool post = p.surrogate == QSM_SURR_POST;
-    // this row's grid table column: (g_n, g_{n+1} - g_n), n = 0..K; the four
-    // groups build alternate entries
-    for (int n = g; n <= p.K; n += 4) {
-      const float gk = grid_value(rm, p.K, n);
-      const float gk1 = n < p.K ? grid_value(rm, p.K, n + 1) : gk;
-      tab[n * 128 + row] = make_float2(gk, __fsub_rn(gk1, gk));
-    }
-    mbar_arrive(bars.tab_ready);
-    bool ok = warp_all_b(mbar_wait(bars.tab_ready, 0, abort));
-    float dhi = 0.0f, dlo = 0.0f;
-    float mstar = -INFINITY, lstar = 0.0f, astar = 0.0f;
+    // m2: running max of x = r c log2e; l2 = sum 2^(x - m2); a2 = sum 2^(x - m2) dp
+    float m2 = -INFINITY, l2 = 0.0f, a2 = 0.0f;
+    bool ok = true;
     uint32_t cnt[2] = {0, 0};
     const int c0 = 32 * g;
     for (int j = 0; j < nkv && ok; ++j) {
@@ -329,99 +329,49 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       // values in registers: hand the buffers back first
       tc_fence_before();
       mbar_arrive(&bars.sd_empty[b]);
-      if (post) {
-        float cm = -INFINITY;
+      float cm = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i < lim) cm = fmaxf(cm, __uint_as_float(sv[i]) * p.c);
-        if (cm > mstar) {
-          const float sc = expf(mstar - cm);
-          lstar *= sc;
-          astar *= sc;
-          mstar = cm;
-        }
+      for (int i = 0; i < 32; ++i)
+        if (i < lim) cm = fmaxf(cm, __fmul_rn(__uint_as_float(sv[i]), p.cL2E));
+      if (cm > m2) {
+        const float sc = ex2_approx(__fsub_rn(m2, cm));
+        l2 *= sc;
+        a2 *= sc;
+        m2 = cm;
+      }
+      if (m2 > -INFINITY) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i < lim) {
-            const float e = expf(__uint_as_float(sv[i]) * p.c - mstar);
-            lstar += e;
-            astar = fmaf(e, __uint_as_float(dv[i]), astar);
-          }
-        }
-      }
-      if (calib && MAP != MAPB_EXACT) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i >= lim) continue;
-          const float r = __uint_as_float(sv[i]);
-          const float gw = (__uint_as_float(dv[i]) - delta) * invZ;
-          const float u = __fmaf_rn(r, a_raw, b_raw);
-          const float uc = fminf(fmaxf(u, 0.0f), Kf);
-          if (MAP == MAPB_HARD) {
-            if (!p.fixed_window) {
-              // nearest node from the bits of a magic-number add (no
-              // float <-> int conversion on the XU pipe)
-              const float tn = __fadd_rn(uc, kMagic);
-              const int n = static_cast<int>(__float_as_uint(tn) - kMagicBits);
-              const float gv = tab[n * 128 + row].x;
-              const float t = gw * (__fsub_rn(tn, kMagic) - Kf) * invK * gv;
-              dhi += t;
-              dlo -= t;
-            }
-          } else {
-            // floor from a round-down add of 2^23 (exact for 0 <= uc <= K)
-            const float tf = __fadd_rd(uc, 8388608.0f);
-            const float kf = fminf(__fsub_rn(tf, 8388608.0f), Kf - 1.0f);
-            const int k = min(static_cast<int>(__float_as_uint(tf) - 0x4B000000u), p.K - 1);
-            const float f = uc - kf;
-            const float2 gd = tab[k * 128 + row];
-            const float g0 = gd.x, slope = gd.y, g1 = gd.x + gd.y;
-            if (!p.fixed_window) {
-              const float mix = ((1.0f - f) * (Kf - kf) * g0 + f * (Kf - kf - 1.0f) * g1) * invK;
-              dhi += gw * (-slope * uc * inv_a - mix);
-              dlo += gw * (-slope * (Kf - uc) * inv_a + mix);
-            } else if (u >= 0.0f) {
-              dhi += gw * (slope * slope_fw);
-            }
+            const float e = ex2_approx(__fmaf_rn(__uint_as_float(sv[i]), p.cL2E, -m2));
+            l2 += e;
+            a2 = __fmaf_rn(e, __uint_as_float(dv[i]), a2);
           }
         }
       }
     }
-    // merge the four groups' partial sums (the online log-sum-exp of the post
-    // surrogate rescales each part to the common maximum)
-    part[(0 * 4 + g) * 128 + row] = dhi;
-    part[(1 * 4 + g) * 128 + row] = dlo;
-    part[(2 * 4 + g) * 128 + row] = mstar;
-    part[(3 * 4 + g) * 128 + row] = lstar;
-    part[(4 * 4 + g) * 128 + row] = astar;
+    // merge the four groups' partial sums at their common maximum
+    part[(0 * 4 + g) * 128 + row] = m2;
+    part[(1 * 4 + g) * 128 + row] = l2;
+    part[(2 * 4 + g) * 128 + row] = a2;
     mbar_arrive(bars.part_ready);
     if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
     if (ok && row_ok && g == 0) {
-      float sdhi = 0.0f, sdlo = 0.0f, M = -INFINITY;
+      float M = -INFINITY;
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg) M = fmaxf(M, part[gg * 128 + row]);
+      float Ls = 0.0f, As = 0.0f;
 #pragma unroll
       for (int gg = 0; gg < 4; ++gg) {
-        sdhi += part[(0 * 4 + gg) * 128 + row];
-        sdlo += part[(1 * 4 + gg) * 128 + row];
-        M = fmaxf(M, part[(2 * 4 + gg) * 128 + row]);
-      }
-      float Ls = 0.0f, As = 0.0f;
-      if (post) {
-#pragma unroll
-        for (int gg = 0; gg < 4; ++gg) {
-          const float mg = part[(2 * 4 + gg) * 128 + row];
-          if (mg == -INFINITY) continue;             // a group with no valid column
-          const float sc = expf(mg - M);
-          Ls = fmaf(part[(3 * 4 + gg) * 128 + row], sc, Ls);
-          As = fmaf(part[(4 * 4 + gg) * 128 + row], sc, As);
-        }
+        const float mg = part[gg * 128 + row];
+        if (mg == -INFINITY) continue;             // a group with no valid column
+        const float sc = ex2_approx(__fsub_rn(mg, M));
+        Ls = __fmaf_rn(part[(4 + gg) * 128 + row], sc, Ls);
+        As = __fmaf_rn(part[(8 + gg) * 128 + row], sc, As);
       }
       float *w = p.rowws + ri * kRowWs;
-      w[RW_DHI] = calib ? sdhi : 0.0f;
-      w[RW_DLO] = calib ? sdlo : 0.0f;
-      if (post) {
-        w[RW_LSESTAR] = M + logf(Ls);
-        w[RW_DELTASTAR] = As / Ls;
-      }
+      w[RW_LSESTAR] = M * 0.6931471805599453f + logf(Ls);
+      w[RW_DELTASTAR] = As / Ls;
     }
   }
   __syncwarp();
@@ -432,145 +382,119 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   if (threadIdx.x == 0 && *bars.abort && p.status != nullptr) atomicExch(p.status, QSM_ERR_TIMEOUT);
 }
 
-// ------------------------------------------------------------------ prep
-// One thread per query row: the constants of the row's map, as the two
-// passes read them (cst), and its grid table (g_n, g_{n+1} - g_n).
-//   cst = a, b (coordinate = fma(r, a, b) on the raw product r), 1/Z,
-//         delta, e (exact: LSE log2e; pre: hi log2e; post: LSE* log2e),
-//         delta*, K/(hi-lo) (d coordinate / d score), 1/(hi-lo)
-__global__ void __launch_bounds__(256) qsm_bwd_prep(const BwdParams p, long long rows) {
-  const long long r = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
-  if (r >= rows) return;
-  const float *rw = p.rowws + r * kRowWs;
-  const float lse = p.LSE[r];
-  float c[kCst] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-  c[3] = rw[RW_DELTA];
-  if (p.map == MAPB_EXACT) {
-    c[4] = lse * 1.4426950408889634f;
-  } else if (p.map == MAPB_POT) {
-    // the forward's exponent coordinate x = fma(r, -c log2e, hi log2e)
-    const float hi = p.hi[r];
-    const float hiL2E = __fmul_rn(hi, log2e_f());
-    c[0] = -p.cL2E;
-    c[1] = hiL2E;
-    c[2] = expf(hi - lse);
-    c[4] = (p.surrogate == QSM_SURR_POST) ? rw[RW_LSESTAR] * 1.4426950408889634f : hiL2E;
-    c[5] = rw[RW_DELTASTAR];
-  } else {
-    const float hi = p.hi[r];
-    const RowMap rm = make_rowmap(hi, p.lo[r], p.K, p.fixed_window != 0, p.window);
-    c[0] = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
-    c[1] = rm.degenerate ? static_cast<float>(p.K) : rm.b;
-    c[2] = expf(hi - lse);                              // 1/Z, Z = exp(LSE - hi)
-    c[4] = (p.surrogate == QSM_SURR_POST) ? rw[RW_LSESTAR] * 1.4426950408889634f : rm.hiL2E;
-    c[5] = rw[RW_DELTASTAR];
-    c[6] = rm.degenerate ? 0.0f : rm.inv;
-    c[7] = rm.degenerate ? 0.0f : 1.0f / __fsub_rn(hi, rm.lo);
-    float2 *t = p.tabg + r * p.KT;
-    for (int n = 0; n <= p.K; ++n) {
-      const float gk = grid_value(rm, p.K, n);
-      const float gk1 = n < p.K ? grid_value(rm, p.K, n + 1) : gk;
-      t[n] = make_float2(gk, __fsub_rn(gk1, gk));
-    }
-  }
-  float4 *cd = reinterpret_cast<float4 *>(p.cst + r * kCst);
-  cd[0] = make_float4(c[0], c[1], c[2], c[3]);
-  cd[1] = make_float4(c[4], c[5], c[6], c[7]);
-}
+// ------------------------------------------------------------ row constants
+// The constants of one query row, as both passes use them (registers in the
+// dQ pass, the workspace copy cst in the dK / dV pass):
+//   a, b   coordinate u = fma(r, a, b) on the raw product r (PoT: the
+//          exponent coordinate, a = -c log2e, b = hi log2e)
+//   invZ   1/Z, Z = exp(LSE - hi)
+//   nDZ    -delta/Z, so that gw = fma(dp, invZ, nDZ)
+//   e0     the surrogate's exponent offset in log2 units: exact LSE log2e,
+//          pre hi log2e, post LSE* log2e (w* = 2^(r c log2e - e0))
+//   ds_    delta (exact) or delta* (post)
+//   kinv   K / (hi - lo): d coordinate / d score (0 for a degenerate row)
+struct RowC {
+  float a, b, invZ, nDZ, e0, ds_, kinv;
+  bool calib;       // the row takes calibration terms
+};
 
-// One element of the backward: returns the probability p = w / Z and writes
-// ds (the surrogate's dL/ds, before the factor c), the map's intermediate
-// values (for the calibration sums) and gw = dL/dw.  c0 = (a, b, 1/Z,
-// delta), c1 = (e, delta*, K/(hi-lo), 1/(hi-lo)); tab[n * ts] = (g_n, g_{n+1}
-// - g_n) of the element's query row.
-template <int MAP>
-__device__ __forceinline__ float bwd_elem(float r, float dp, const float4 &c0, const float4 &c1,
-                                          const float2 *tab, int ts, const BwdParams &p,
-                                          float Kf, float &ds, float &gw, float &u, float &uc,
-                                          float &kf, float2 &gd) {
+// Table layouts (K-interval).  Entry i of a row, interpolation, i = 0..K+1:
+// i = 0 the below-window entry (fixed window: weight g_0, or 0 when flushed,
+// no derivative; min-max: a copy of interval 0), i = k + 1 interval k =
+// 0..K-1, i = K + 1 a copy of interval K - 1 (u = K).  The index is
+// floor(clamp(u, -1, K)) + 1 from a round-down add of 1.5 * 2^23.  Hard
+// rounding: entry n = 0..K at rne(clamp(u, 0, K)).
+//   dQ pass (shared memory, [entry][128 rows]): interpolation with min-max
+//   calibration (A, B, d, 0); interpolation otherwise d; hard rounding with
+//   min-max calibration (n - K)/K g_n.
+//   dK / dV pass (workspace, [row][TS]): interpolation (e, d) pairs with
+//   w = fma(u, d, e); hard rounding g_n.
+template <int MAP, int SURR, int CAL>
+struct DqTab {
+  static constexpr bool KI = MAP == MAPB_HARD || MAP == MAPB_INTERP;
+  static constexpr bool ANY = KI && (CAL != CAL_OFF || (MAP == MAPB_INTERP && SURR == SURR_NONE));
+  static constexpr int ESZ = (MAP == MAPB_INTERP && CAL == CAL_MINMAX) ? 16 : 4;
+  static constexpr int STRIDE = ESZ * 128;
+  static constexpr int entries(int K) { return MAP == MAPB_INTERP ? K + 2 : K + 1; }
+  static constexpr size_t bytes(int K) {
+    return ANY ? static_cast<size_t>(entries(K)) * STRIDE : 0;
+  }
+};
+
+// Build this thread's row constants and its group's entries of the row's
+// tables (entries g, g + 4, ...), both for the dQ pass (shared memory at
+// tq_base) and, when row_ok, for the dK / dV pass (workspace).
+template <int MAP, int SURR, int CAL>
+__device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, int g, int row,
+                                              bool row_ok, uint32_t tq_base) {
+  using T = DqTab<MAP, SURR, CAL>;
+  RowC k;
+  k.a = k.b = k.invZ = k.nDZ = k.e0 = k.ds_ = k.kinv = 0.0f;
+  k.calib = false;
+  const float lse = p.LSE[ri];
   if (MAP == MAPB_EXACT) {
-    const float pw = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
-    ds = pw * (dp - c0.w);
-    gw = 0.0f;
-    return pw;
+    k.e0 = __fmul_rn(lse, kL2E);
+    return k;
   }
+  const float hi = p.hi[ri];
+  k.invZ = expf(__fsub_rn(hi, lse));
   if (MAP == MAPB_POT) {
-    // the forward's power-of-two weight (exponent frozen: no own-score or
-    // anchor derivative; only the surrogate's direct term)
-    const float x = __fmaf_rn(r, c0.x, c0.y);
-    const float cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
-    const float t = __fadd_rn(fminf(x, cap), kMagic);
-    float w = __uint_as_float(__float_as_uint(t) * 0xFF800000u + 0x3F800000u);
-    if (p.flush && t > kMagic + static_cast<float>(p.pot_floor)) w = 0.0f;
-    const float pw = w * c0.z;
-    gw = (dp - c0.w) * c0.z;
-    if (p.surrogate == QSM_SURR_NONE)
-      ds = 0.0f;
-    else if (p.surrogate == QSM_SURR_PRE)
-      ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
-    else
-      ds = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x)) * (dp - c1.y);
-    return pw;
-  }
-  u = __fmaf_rn(r, c0.x, c0.y);
-  uc = fminf(fmaxf(u, 0.0f), Kf);
-  const bool below = p.fixed_window && u < 0.0f;
-  float w, slope = 0.0f;
-  if (MAP == MAPB_HARD) {
-    // nearest node from the bits of a magic-number add
-    const float tn = __fadd_rn(uc, kMagic);
-    gd = tab[static_cast<int>(__float_as_uint(tn) - kMagicBits) * ts];
-    w = gd.x;
-    kf = __fsub_rn(tn, kMagic);
+    k.a = -p.cL2E;
+    k.b = __fmul_rn(hi, log2e_f());
+    k.e0 = k.b;
   } else {
-    // floor from a round-down add of 2^23 (exact for 0 <= uc <= K)
-    const float tf = __fadd_rd(uc, 8388608.0f);
-    kf = fminf(__fsub_rn(tf, 8388608.0f), Kf - 1.0f);
-    gd = tab[min(static_cast<int>(__float_as_uint(tf) - 0x4B000000u), p.K - 1) * ts];
-    w = __fmaf_rn(__fsub_rn(uc, kf), gd.y, gd.x);
-    slope = gd.y;
-  }
-  if (below && p.flush) w = 0.0f;
-  const float pw = w * c0.z;
-  gw = (dp - c0.w) * c0.z;
-  if (p.surrogate == QSM_SURR_NONE)
-    ds = (MAP == MAPB_INTERP && !below) ? gw * slope * c1.z : 0.0f;
-  else if (p.surrogate == QSM_SURR_PRE)
-    ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
-  else
-    ds = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x)) * (dp - c1.y);
-  return pw;
-}
-
-// Calibration sums of one element: dhi += gw dF/dhi, dlo += gw dF/dlo with s
-// and the decision held fixed (min-max hard: dF/dhi = -(K-n)/K w = -dF/dlo;
-// interpolation: the slope and mixing terms; fixed window: only hi moves).
-template <int MAP>
-__device__ __forceinline__ void calib_elem(const BwdParams &p, float Kf, float invK, float gw,
-                                           float u, float uc, float kf, float2 gd, float inv_a,
-                                           float &dhi, float &dlo) {
-  if (MAP == MAPB_HARD) {
-    if (!p.fixed_window) {
-      const float t = gw * (kf - Kf) * invK * gd.x;
-      dhi += t;
-      dlo -= t;
-    }
-  } else if (MAP == MAPB_INTERP) {
-    const float f = uc - kf;
-    const float slope = gd.y;
-    if (!p.fixed_window) {
-      // ((1-f)(K-k) g_k + f (K-k-1) g_{k+1}) / K = ((K-k) w - f g_{k+1}) / K
-      // with w = g_k + f (g_{k+1} - g_k) the interpolated weight
-      const float w = gd.x + f * slope;
-      const float mix = ((Kf - kf) * w - f * (gd.x + slope)) * invK;
-      const float ts = gw * slope * inv_a;
-      const float gm = gw * mix;
-      dhi += -ts * uc - gm;
-      dlo += -ts * (Kf - uc) + gm;
-    } else if (u >= 0.0f) {
-      dhi += gw * (slope * (-Kf / p.window));
+    const RowMap rm =
+        make_rowmap(hi, p.lo != nullptr ? p.lo[ri] : hi, p.K, p.fixed_window != 0, p.window);
+    k.a = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
+    k.b = rm.degenerate ? static_cast<float>(p.K) : rm.b;
+    k.e0 = rm.hiL2E;
+    k.kinv = rm.inv;
+    k.calib = CAL != CAL_OFF && !rm.degenerate;
+    const float Kf = static_cast<float>(p.K);
+    float *tk = p.tabk + ri * p.TS;
+    if (MAP == MAPB_INTERP) {
+      const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(hi, rm.lo));
+      for (int i = g; i <= p.K + 1; i += 4) {
+        float e, d, A = 0.0f, B = 0.0f;
+        if (i == 0 && p.fixed_window) {
+          e = p.flush ? 0.0f : grid_value(rm, p.K, 0);
+          d = 0.0f;
+        } else {
+          const int kk = min(max(i - 1, 0), p.K - 1);
+          const float gk = grid_value(rm, p.K, kk), gk1 = grid_value(rm, p.K, kk + 1);
+          const float kf = static_cast<float>(kk), kmk = static_cast<float>(p.K - kk);
+          d = __fsub_rn(gk1, gk);
+          e = __fmaf_rn(-kf, d, gk);
+          if (CAL == CAL_MINMAX) {
+            A = -__fdiv_rn(__fmaf_rn(kmk, e, __fmul_rn(kf, gk1)), Kf);
+            B = __fsub_rn(-__fmul_rn(d, inv_a), __fdiv_rn(__fsub_rn(__fmul_rn(kmk, d), gk1), Kf));
+          }
+        }
+        if (row_ok) {
+          tk[2 * i] = e;
+          tk[2 * i + 1] = d;
+        }
+        if (CAL == CAL_MINMAX)
+          sts_f32x4(tq_base + i * T::STRIDE + row * 16, make_float4(A, B, d, 0.0f));
+        else if (T::ANY)
+          sts_f32(tq_base + i * T::STRIDE + row * 4, d);
+      }
+    } else {
+      for (int n = g; n <= p.K; n += 4) {
+        const float gn = grid_value(rm, p.K, n);
+        if (row_ok) tk[n] = gn;
+        if (T::ANY)
+          sts_f32(tq_base + n * T::STRIDE + row * 4,
+                  __fmul_rn(__fdiv_rn(static_cast<float>(n - p.K), Kf), gn));
+      }
     }
   }
+  if (SURR == SURR_POST) {
+    const float *w = p.rowws + ri * kRowWs;
+    k.e0 = __fmul_rn(w[RW_LSESTAR], kL2E);
+    k.ds_ = w[RW_DELTASTAR];
+  }
+  return k;
 }
 
 // ----------------------------------------------------------------- dQ pass
@@ -589,25 +513,25 @@ struct DqBars {
 };
 constexpr uint32_t T_DQ = 256;
 
-template <int D, int MAP>
+template <int D, int MAP, int SURR, int CAL>
 __global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const BwdParams p) {
   using G = BGeo<D>;
+  using T = DqTab<MAP, SURR, CAL>;
   static_assert(D == 64, "dQ slices of the four map groups: 16 columns each");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y, qt = blockIdx.x;
+  int bh, qt;
+  q_tile_order(p, bh, qt);
   const int ns = p.num_stages;
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages of (K_j, V_j)
   uint8_t *sDS = smem + p.ds_off;                        // 2 x 128 rows x 128 bytes
-  float2 *tab = reinterpret_cast<float2 *>(smem + p.tab_off);   // [n][128]
-  float *part = reinterpret_cast<float *>(smem + p.part_off);   // [2][4][128]
+  float *part = reinterpret_cast<float *>(smem + p.part_off);   // [3][4][128]
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   DqBars bars;
   bars.kv_full = bp;
@@ -741,15 +665,36 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const bool row_ok = qrow < p.S;
     const int L = p.causal ? min(qrow + 1, p.S) : p.S;
     const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-    const float4 *cg = reinterpret_cast<const float4 *>(p.cst + ri * kCst);
-    const float4 c0 = cg[0], c1 = cg[1];
-    const float Kf = static_cast<float>(p.K), invK = 1.0f / Kf;
-    const bool calib = p.calib && c1.w != 0.0f;          // 1/(hi-lo) = 0: degenerate row
-    if (MAP == MAPB_HARD || MAP == MAPB_INTERP)
-      for (int n = g; n <= p.K; n += 4) tab[n * 128 + row] = p.tabg[ri * p.KT + n];
+    // ---- per-row setup: this group's share of delta = dO_r . O_r, the row
+    // constants and this group's table entries
+    {
+      const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
+      const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
+      part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
+    }
+    const uint32_t tq_base = smem_u32(smem + p.tab_off);
+    RowC kc = row_constants<MAP, SURR, CAL>(p, ri, g, row, row_ok, tq_base);
     mbar_arrive(bars.tab_ready);
     bool ok = warp_all_b(mbar_wait(bars.tab_ready, 0, abort));
-    float dhi = 0.0f, dlo = 0.0f;
+    const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
+    if (MAP == MAPB_EXACT) {
+      kc.ds_ = delta;
+    } else {
+      kc.nDZ = -__fmul_rn(delta, kc.invZ);
+    }
+    if (g == 0 && row_ok) {
+      float4 *cd = reinterpret_cast<float4 *>(p.cst + ri * kCst);
+      cd[0] = make_float4(kc.a, kc.b, kc.invZ, kc.nDZ);
+      cd[1] = make_float4(kc.e0, kc.ds_, kc.kinv, 0.0f);
+    }
+    // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) - bits(M)
+    // + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard),
+    // M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
+    const uint32_t tq_row = (MAP == MAPB_INTERP)
+                                ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
+                                : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
+    const float Kf = static_cast<float>(p.K);
+    float s1 = 0.0f, s2 = 0.0f;                          // calibration sums
     const uint32_t dsb = smem_u32(sDS);
     for (int h = 0; h < nh && ok; ++h) {
       const int j = h >> 1, e = h & 1, x = h & 1;
@@ -765,6 +710,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars.sdp_free[x]);                  // the pair can take half h + 2
       const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
+      const bool full = warp_all_b(lim >= 16);
       uint32_t dd[8];
 #pragma unroll
       for (int i2 = 0; i2 < 8; ++i2) {
@@ -772,13 +718,42 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const int i = 2 * i2 + t;
-          float ds, gw, u = 0.0f, uc = 0.0f, kf = 0.0f;
-          float2 gd = make_float2(0.0f, 0.0f);
-          (void)bwd_elem<MAP>(__uint_as_float(sv[i]), __uint_as_float(dv[i]), c0, c1,
-                              tab + row, 128, p, Kf, ds, gw, u, uc, kf, gd);
-          const bool valid = i < lim;
-          if ((MAP == MAPB_HARD || MAP == MAPB_INTERP) && calib && valid)
-            calib_elem<MAP>(p, Kf, invK, gw, u, uc, kf, gd, c1.w, dhi, dlo);
+          const bool valid = full || i < lim;
+          const float r = __uint_as_float(sv[i]), dp = __uint_as_float(dv[i]);
+          float ds;
+          if (MAP == MAPB_EXACT) {
+            ds = ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0)) * (dp - kc.ds_);
+          } else {
+            float gw = __fmaf_rn(dp, kc.invZ, kc.nDZ);
+            if (!valid) gw = 0.0f;
+            if (SURR == SURR_PRE)
+              ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0));
+            else if (SURR == SURR_POST)
+              ds = ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0)) * (dp - kc.ds_);
+            else
+              ds = 0.0f;
+            if (T::ANY) {
+              const float u = __fmaf_rn(r, kc.a, kc.b);
+              if (MAP == MAPB_INTERP) {
+                const float ucl = fminf(fmaxf(u, -1.0f), Kf);
+                const uint32_t ad = __float_as_uint(__fadd_rd(ucl, kMagic)) * T::STRIDE + tq_row;
+                if (CAL == CAL_MINMAX) {
+                  const float4 ab = lds_f32x4(ad);     // A, B, d
+                  s1 = __fmaf_rn(gw, __fmaf_rn(ab.y, ucl, ab.x), s1);
+                  s2 = __fmaf_rn(gw, ab.z, s2);
+                  if (SURR == SURR_NONE) ds = gw * ab.z * kc.kinv;
+                } else {
+                  const float d = lds_f32(ad);
+                  if (CAL == CAL_FIXED) s2 = __fmaf_rn(gw, d, s2);
+                  if (SURR == SURR_NONE) ds = gw * d * kc.kinv;
+                }
+              } else {
+                const float uc = fminf(fmaxf(u, 0.0f), Kf);
+                const uint32_t ad = __float_as_uint(__fadd_rn(uc, kMagic)) * T::STRIDE + tq_row;
+                s1 = __fmaf_rn(gw, lds_f32(ad), s1);
+              }
+            }
+          }
           d2[t] = valid ? ds : 0.0f;
         }
         dd[i2] = pack_bf16x2(d2[0], d2[1]);
@@ -801,43 +776,60 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_arrive(&bars.ds_full[x]);
     }
     // ---- epilogue: the row's calibration sums, dQ
-    part[(0 * 4 + g) * 128 + row] = dhi;
-    part[(1 * 4 + g) * 128 + row] = dlo;
+    part[(4 + g) * 128 + row] = s1;
+    part[(8 + g) * 128 + row] = s2;
     mbar_arrive(bars.part_ready);
     if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
     if (ok) ok = warp_all_b(mbar_wait(bars.dq_full, 0, abort));
     if (ok) {
       tc_fence_after();
-      const float tdhi = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
-      const float tdlo = (part[512 + row] + part[640 + row]) + (part[768 + row] + part[896 + row]);
       uint32_t v[16];
       tmem_ld16_sync(lane_base + T_DQ + 16 * g, v);
       float xq[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[i]) * p.c;
-      if (calib && row_ok) {
-        // rank-one calibration terms in fp32: dQ_r += c (dhi k_argmax + dlo k_argmin)
-        const size_t head = static_cast<size_t>(bh) * p.S;
-        const __nv_bfloat16 *ka = p.K_ + (head + p.amax[ri]) * D + 16 * g;
-        const __nv_bfloat16 *kb = p.K_ + (head + p.amin[ri]) * D + 16 * g;
-        const float sh = p.c * tdhi, sl = p.c * tdlo;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          xq[i] += sh * __bfloat162float(ka[i]) + sl * __bfloat162float(kb[i]);
-        // and dK_argmax += c dhi q_r, dK_argmin += c dlo q_r, into the fp32
-        // calibration part of dK (many rows can share one key: atomics)
-        const __nv_bfloat16 *qr = p.Q + ri * D + 16 * g;
-        float *da = p.dkcal + (head + p.amax[ri]) * D + 16 * g;
-        float *db = p.dkcal + (head + p.amin[ri]) * D + 16 * g;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float qv = __bfloat162float(qr[i]);
-          atomicAdd(da + i, sh * qv);
-          atomicAdd(db + i, sl * qv);
+      if (CAL != CAL_OFF && kc.calib && row_ok) {
+        const float S1 = (part[512 + row] + part[640 + row]) + (part[768 + row] + part[896 + row]);
+        const float S2 =
+            (part[1024 + row] + part[1152 + row]) + (part[1280 + row] + part[1408 + row]);
+        float dhi, dlo;
+        if (CAL == CAL_FIXED) {
+          dhi = -(Kf / p.window) * S2;
+          dlo = 0.0f;
+        } else if (MAP == MAPB_HARD) {
+          dhi = S1;
+          dlo = -S1;
+        } else {
+          dhi = S1;
+          dlo = -S1 - kc.kinv * S2;
         }
-        if (g == 0) {
-          p.rowws[ri * kRowWs + RW_DHI] = tdhi;
-          p.rowws[ri * kRowWs + RW_DLO] = tdlo;
+        // rank-one calibration terms in fp32: dQ_r += c (dhi k_argmax + dlo
+        // k_argmin), and dK_argmax += c dhi q_r, dK_argmin += c dlo q_r into
+        // the fp32 calibration part of dK (many rows can share a key: vector
+        // reductions)
+        const size_t head = static_cast<size_t>(bh) * p.S;
+        const float sh = p.c * dhi, sl = p.c * dlo;
+        float kx[16], qx[16];
+        bf16x16_to_f32(reinterpret_cast<const uint4 *>(p.K_ + (head + p.amax[ri]) * D + 16 * g),
+                       kx);
+        bf16x16_to_f32(reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g), qx);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
+        float *da = p.dkcal + (head + p.amax[ri]) * D + 16 * g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
+                                                sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
+        if (CAL == CAL_MINMAX) {
+          bf16x16_to_f32(
+              reinterpret_cast<const uint4 *>(p.K_ + (head + p.amin[ri]) * D + 16 * g), kx);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
+          float *db = p.dkcal + (head + p.amin[ri]) * D + 16 * g;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
+                                                  sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
         }
       }
       uint32_t pk[8];
@@ -875,7 +867,48 @@ struct KvBars {
 };
 constexpr uint32_t T_DV = 256, T_DK = 320;
 
-template <int D, int MAP>
+// One element of the dK / dV pass: the probability p = w / Z (returned) and
+// ds (the surrogate's dL/ds before the factor c).  c0 = (a, b, 1/Z,
+// -delta/Z), c1 = (e0, delta_s, K/(hi-lo), 0) of the element's query row;
+// trow the (biased) shared address of that row's table.
+template <int MAP, int SURR>
+__device__ __forceinline__ float kv_elem(float r, float dp, const float4 &c0, const float4 &c1,
+                                         uint32_t trow, const BwdParams &p, float Kf, float cap,
+                                         float flush_t, bool flush_below, float &ds) {
+  if (MAP == MAPB_EXACT) {
+    const float pw = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
+    ds = pw * (dp - c1.y);
+    return pw;
+  }
+  const float gw = __fmaf_rn(dp, c0.z, c0.w);
+  const float u = __fmaf_rn(r, c0.x, c0.y);
+  float w, dnone = 0.0f;
+  if (MAP == MAPB_POT) {
+    // the forward's power-of-two weight (exponent frozen: no own-score or
+    // anchor derivative; only the surrogate's direct term)
+    const float t = __fadd_rn(fminf(u, cap), kMagic);
+    w = __uint_as_float(__float_as_uint(t) * 0xFF800000u + 0x3F800000u);
+    if (p.flush && t > flush_t) w = 0.0f;
+  } else if (MAP == MAPB_HARD) {
+    const float uc = fminf(fmaxf(u, 0.0f), Kf);
+    w = lds_f32(__float_as_uint(__fadd_rn(uc, kMagic)) * 4u + trow);
+    if (flush_below && u < 0.0f) w = 0.0f;
+  } else {
+    const float ucl = fminf(fmaxf(u, -1.0f), Kf);
+    const float2 ed = lds_f32x2(__float_as_uint(__fadd_rd(ucl, kMagic)) * 8u + trow);
+    w = __fmaf_rn(ucl, ed.y, ed.x);
+    dnone = ed.y;
+  }
+  if (SURR == SURR_PRE)
+    ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
+  else if (SURR == SURR_POST)
+    ds = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x)) * (dp - c1.y);
+  else
+    ds = (MAP == MAPB_INTERP) ? gw * dnone * c1.z : 0.0f;
+  return w * c0.z;
+}
+
+template <int D, int MAP, int SURR>
 __global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_dkdv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -883,8 +916,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   using G = BGeo<D>;
   static_assert(D == 64, "dK / dV slices of the four map groups: 16 columns each");
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, kt = blockIdx.x;
   const int ns = p.num_stages;
@@ -951,8 +983,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         const int nrow = min(128, p.S - it * 128);
         const size_t r0 = static_cast<size_t>(bh) * p.S + static_cast<size_t>(it) * 128;
         const uint32_t cbytes = static_cast<uint32_t>(nrow) * kCst * 4;
-        const uint32_t tbytes =
-            (MAP == MAPB_EXACT || MAP == MAPB_POT) ? 0u : static_cast<uint32_t>(nrow) * p.KT * 8;
+        const uint32_t tbytes = static_cast<uint32_t>(nrow) * p.TS * 4;
         mbar_expect_tx(&bars.qd_full[st], 2 * G::TILE_BYTES + cbytes + tbytes);
         for (int ch = 0; ch < G::CHUNKS; ++ch) {
           tma_load_3d(s + ch * G::CHUNK_BYTES, &tmQ, &bars.qd_full[st], ch * G::EPC, it * 128, bh);
@@ -960,7 +991,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                       ch * G::EPC, it * 128, bh);
         }
         bulk_load(s + CST_OFF, p.cst + r0 * kCst, cbytes, &bars.qd_full[st]);
-        if (tbytes) bulk_load(s + TAB_OFF, p.tabg + r0 * p.KT, tbytes, &bars.qd_full[st]);
+        if (tbytes) bulk_load(s + TAB_OFF, p.tabk + r0 * p.TS, tbytes, &bars.qd_full[st]);
       }
       mbar_wait(bars.kv_full, 0, abort);
       for (int st = 0; st < ns && st < nq; ++st)
@@ -1031,6 +1062,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const int kg = kt * 128 + key;
     const bool key_ok = kg < p.S;
     const float Kf = static_cast<float>(p.K);
+    const float cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
+    const float flush_t = kMagic + static_cast<float>(p.pot_floor);
+    const bool flush_below = MAP == MAPB_HARD && p.flush && p.fixed_window;
+    // table entry bias: bits(M + floor(clamp(u, -1, K))) - bits(M) + 1 (interp)
+    // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), mod 2^32
+    const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - kMagicBits * 8u : 0u - kMagicBits * 4u;
     bool ok = true;
     for (int h = 0; h < nh && ok; ++h) {
       const int n = h >> 1, e = h & 1, x = h & 1;
@@ -1043,9 +1080,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       ok = warp_all_b(mbar_wait(&bars.sdp_full[x], (h >> 1) & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      const uint8_t *s = sSt + (n % ns) * SB;
-      const float4 *cst4 = reinterpret_cast<const float4 *>(s + CST_OFF);
-      const float2 *tabs = reinterpret_cast<const float2 *>(s + TAB_OFF);
+      const uint32_t st = smem_u32(sSt + (n % ns) * SB);
       uint32_t sv[16], dv[16];
       tmem_ld16(lane_base + 128 * x + 16 * g, sv);
       tmem_ld16(lane_base + 128 * x + 64 + 16 * g, dv);
@@ -1053,6 +1088,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       reg_fence16(sv);
       reg_fence16(dv);
       const int qbase = (i0 + n) * 128 + 64 * e + 16 * g;   // first query row of the slice
+      const int ql0 = 64 * e + 16 * g;                      // its row within the tile
+      // every element valid: the key exists, the slice's rows exist and (causal)
+      // lie at or below this key
+      const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
       uint32_t pp[8], dd[8];
 #pragma unroll
       for (int i2 = 0; i2 < 8; ++i2) {
@@ -1060,14 +1099,27 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const int i = 2 * i2 + t;
-          const int ql = 64 * e + 16 * g + i;              // query row within the tile
+          const int ql = ql0 + i;
           const int qg = qbase + i;
-          const bool valid = key_ok && qg < p.S && (!p.causal || kg <= qg);
-          const float4 c0 = cst4[2 * ql], c1 = cst4[2 * ql + 1];
-          float ds, gw, u, uc, kf;
-          float2 gd;
-          const float pw = bwd_elem<MAP>(__uint_as_float(sv[i]), __uint_as_float(dv[i]), c0, c1,
-                                         tabs + ql * p.KT, 1, p, Kf, ds, gw, u, uc, kf, gd);
+          const bool valid = full || (key_ok && qg < p.S && (!p.causal || kg <= qg));
+          const uint32_t ca = st + CST_OFF + ql * (kCst * 4);
+          // only the constants this map and surrogate read
+          const float4 c0 = (MAP == MAPB_EXACT) ? make_float4(0.0f, 0.0f, 0.0f, 0.0f)
+                                                : lds_f32x4(ca);
+          float4 c1 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (MAP == MAPB_EXACT || SURR == SURR_POST) {
+            const float2 t2 = lds_f32x2(ca + 16);
+            c1.x = t2.x;
+            c1.y = t2.y;
+          } else if (SURR == SURR_PRE) {
+            c1.x = lds_f32(ca + 16);
+          } else if (MAP == MAPB_INTERP) {
+            c1.z = lds_f32(ca + 24);
+          }
+          float ds;
+          const float pw = kv_elem<MAP, SURR>(__uint_as_float(sv[i]), __uint_as_float(dv[i]), c0,
+                                              c1, st + TAB_OFF + ql * (p.TS * 4) + tbias, p, Kf,
+                                              cap, flush_t, flush_below, ds);
           p2[t] = valid ? pw : 0.0f;
           d2[t] = valid ? ds : 0.0f;
         }
@@ -1148,80 +1200,92 @@ bool set_smem_once(F kern, int bytes, std::atomic<int> (&cache)[kMaxDevices]) {
 }
 
 constexpr size_t kMaxSmem = 232448;                      // 227 KB opt-in per CTA
+constexpr size_t kBarBytes = ((2 * 8 + 16) * 8 + 8 + 15) & ~static_cast<size_t>(15);
 
-template <int D, int MAP>
-qsm_status launch_passes(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
-                         const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
+template <int D, int MAP, int SURR, int CAL>
+qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const CUtensorMap &mk,
+                     const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  const int BH = a.B * a.H;
-  const size_t bar_bytes = ((2 * 8 + 16) * 8 + 8 + 15) & ~static_cast<size_t>(15);
-  {
-    // dQ pass: Q, dO, ns x (K, V), 2 dS buffers, table, partial sums, barriers
-    const size_t tab = static_cast<size_t>(p.K + 1) * 128 * sizeof(float2);
-    const size_t fixed = 1024 + 2 * G::TILE_BYTES + 2 * 128 * 128 + tab + 2 * 4 * 128 * 4 + bar_bytes;
-    int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
-    if (ns > 4) ns = 4;
-    if (ns < 2) return QSM_ERR_UNSUPPORTED;
-    BwdParams q = p;
-    q.num_stages = ns;
-    q.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
-    q.tab_off = q.ds_off + 2 * 128 * 128;
-    q.part_off = static_cast<uint32_t>(q.tab_off + tab);
-    q.bar_off = q.part_off + 2 * 4 * 128 * 4;
-    size_t smem = 1024 + q.bar_off + bar_bytes;
-    if (smem < 120 * 1024) smem = 120 * 1024;            // one CTA per SM (all of TMEM)
-    if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
-    auto kern = qsm_bwd_dq<D, MAP>;
-    static std::atomic<int> cache[kMaxDevices];
-    if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-    kern<<<dim3(p.nqt, BH), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, q);
-    if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
-  }
-  {
-    // dK/dV pass: K, V, ns x (Q, dO, constants, tables), barriers
-    const size_t tabb = (MAP == MAPB_EXACT || MAP == MAPB_POT) ? 0 : static_cast<size_t>(128) * p.KT * 8;
-    const size_t stage = (2 * G::TILE_BYTES + 128 * kCst * 4 + tabb + 1023) & ~static_cast<size_t>(1023);
-    const size_t fixed = 1024 + 2 * G::TILE_BYTES + bar_bytes;
-    int ns = static_cast<int>((kMaxSmem - fixed) / stage);
-    if (ns > 4) ns = 4;
-    if (ns < 2) return QSM_ERR_UNSUPPORTED;
-    BwdParams k = p;
-    k.num_stages = ns;
-    k.stage_bytes = static_cast<uint32_t>(stage);
-    k.bar_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * stage);
-    size_t smem = 1024 + k.bar_off + bar_bytes;
-    if (smem < 120 * 1024) smem = 120 * 1024;
-    if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
-    auto kern = qsm_bwd_dkdv<D, MAP>;
-    static std::atomic<int> cache[kMaxDevices];
-    if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-    kern<<<dim3(p.nkvt, BH), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, k);
-    if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
-  }
-  return QSM_OK;
+  // Q, dO, ns x (K, V), 2 dS buffers, table, partial sums, barriers
+  const size_t tab = (DqTab<MAP, SURR, CAL>::bytes(p.K) + 15) & ~static_cast<size_t>(15);
+  const size_t part = 3 * 4 * 128 * sizeof(float);
+  const size_t fixed = 1024 + 2 * G::TILE_BYTES + 2 * 128 * 128 + tab + part + kBarBytes;
+  int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
+  if (ns > 4) ns = 4;
+  if (ns < 2) return QSM_ERR_UNSUPPORTED;
+  p.num_stages = ns;
+  p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
+  p.tab_off = p.ds_off + 2 * 128 * 128;
+  p.part_off = static_cast<uint32_t>(p.tab_off + tab);
+  p.bar_off = static_cast<uint32_t>(p.part_off + part);
+  size_t smem = 1024 + p.bar_off + kBarBytes;
+  if (smem < 120 * 1024) smem = 120 * 1024;            // one CTA per SM (all of TMEM)
+  if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
+  auto kern = qsm_bwd_dq<D, MAP, SURR, CAL>;
+  static std::atomic<int> cache[kMaxDevices];
+  if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
+  kern<<<dim3(p.nqt * a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+}
+
+template <int D, int MAP, int SURR>
+qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
+                       const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
+  using G = BGeo<D>;
+  // K, V, ns x (Q, dO, constants, tables), barriers
+  const size_t stage =
+      (2 * G::TILE_BYTES + 128 * kCst * 4 + static_cast<size_t>(128) * p.TS * 4 + 1023) &
+      ~static_cast<size_t>(1023);
+  const size_t fixed = 1024 + 2 * G::TILE_BYTES + kBarBytes;
+  int ns = static_cast<int>((kMaxSmem - fixed) / stage);
+  if (ns > 4) ns = 4;
+  if (ns < 2) return QSM_ERR_UNSUPPORTED;
+  p.num_stages = ns;
+  p.stage_bytes = static_cast<uint32_t>(stage);
+  p.bar_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * stage);
+  size_t smem = 1024 + p.bar_off + kBarBytes;
+  if (smem < 120 * 1024) smem = 120 * 1024;
+  if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
+  auto kern = qsm_bwd_dkdv<D, MAP, SURR>;
+  static std::atomic<int> cache[kMaxDevices];
+  if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
+  kern<<<dim3(p.nkvt, a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+}
+
+template <int D, int MAP, int SURR, int CAL>
+qsm_status launch_passes(const BwdArgs &a, const BwdParams &p, const CUtensorMap &mq,
+                         const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
+  const qsm_status st = launch_dq<D, MAP, SURR, CAL>(a, p, mq, mk, mv, mdo);
+  if (st != QSM_OK) return st;
+  return launch_dkdv<D, MAP, SURR>(a, p, mq, mk, mv, mdo);
+}
+
+template <int D, int MAP, int CAL>
+qsm_status launch_by_surr(int surr, const BwdArgs &a, const BwdParams &p, const CUtensorMap &mq,
+                          const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
+  if (surr == SURR_PRE) return launch_passes<D, MAP, SURR_PRE, CAL>(a, p, mq, mk, mv, mdo);
+  if (surr == SURR_POST) return launch_passes<D, MAP, SURR_POST, CAL>(a, p, mq, mk, mv, mdo);
+  return launch_passes<D, MAP, SURR_NONE, CAL>(a, p, mq, mk, mv, mdo);
 }
 
 template <int D>
 qsm_status launch_rows(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
                        const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  const size_t tab = static_cast<size_t>(128) * (p.K + 1) * sizeof(float2);
-  BwdParams r = p;
-  r.tab_off = static_cast<uint32_t>(2 * G::TILE_BYTES + 4 * G::TILE_BYTES);
-  r.cst_off = static_cast<uint32_t>((r.tab_off + tab + 15) & ~static_cast<size_t>(15));
-  r.bar_off = static_cast<uint32_t>(r.cst_off + 5 * 4 * 128 * sizeof(float));
-  size_t smem = 1024 + r.bar_off + 256;
+  p.part_off = static_cast<uint32_t>(2 * G::TILE_BYTES + 4 * G::TILE_BYTES);
+  p.bar_off = static_cast<uint32_t>(p.part_off + 3 * 4 * 128 * sizeof(float));
+  size_t smem = 1024 + p.bar_off + 256;
   if (smem < 120 * 1024) smem = 120 * 1024;
   if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
-  auto kern = (p.map == MAPB_HARD) ? qsm_bwd_rows<D, MAPB_HARD> : qsm_bwd_rows<D, MAPB_INTERP>;
-  static std::atomic<int> cache_h[kMaxDevices], cache_i[kMaxDevices];
-  if (!set_smem_once(kern, static_cast<int>(smem), p.map == MAPB_HARD ? cache_h : cache_i))
-    return QSM_ERR_CUDA;
-  kern<<<dim3(p.nqt, a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, r);
+  auto kern = qsm_bwd_rows<D>;
+  static std::atomic<int> cache[kMaxDevices];
+  if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
+  kern<<<dim3(p.nqt * a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
-constexpr int kTabKT = (kBwdMaxK + 2) & ~1;              // table row stride in the workspace
+constexpr int kTabKT = (kBwdMaxK + 2) & ~1;              // float2 entries per row, workspace
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -1229,7 +1293,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 size_t bwd_workspace_bytes(int B, int H, int S, int D) {
   // fp32 calibration part of dK, then per query row: the row workspace, the
-  // map constants and the grid table; each part 256-byte aligned
+  // map constants and the dK / dV pass's grid table; each part 256-byte
+  // aligned
   const size_t rows = static_cast<size_t>(B) * H * S;
   return align256(rows * D * sizeof(float)) + align256(rows * kRowWs * sizeof(float)) +
          align256(rows * kCst * sizeof(float)) + align256(rows * kTabKT * sizeof(float2));
@@ -1239,22 +1304,25 @@ qsm_status launch_bwd(const BwdArgs &a) {
   if (a.D != 64) return QSM_ERR_UNSUPPORTED;          // TMEM schedule holds D = 64
   if (a.mode == QSM_MODE_KINTERVAL && a.Kint > kBwdMaxK) return QSM_ERR_UNSUPPORTED;
   const size_t rows = static_cast<size_t>(a.B) * a.H * a.S;
+  const int map = a.mode == QSM_MODE_EXACT       ? MAPB_EXACT
+                  : a.mode == QSM_MODE_ROWMAX_POT ? MAPB_POT
+                  : (a.rounding == QSM_ROUND_HARD ? MAPB_HARD : MAPB_INTERP);
   BwdParams p{};
   p.S = a.S;
   p.nqt = (a.S + 127) / 128;
   p.nkvt = p.nqt;
+  p.BH = a.B * a.H;
   p.causal = a.causal;
-  p.map = a.mode == QSM_MODE_EXACT       ? MAPB_EXACT
-          : a.mode == QSM_MODE_ROWMAX_POT ? MAPB_POT
-          : (a.rounding == QSM_ROUND_HARD ? MAPB_HARD : MAPB_INTERP);
+  p.hgroup = causal_head_group(a.S, a.D, false, p.BH);
   p.pot_floor = a.pot_floor;
   p.K = a.mode == QSM_MODE_KINTERVAL ? a.Kint : 1;
   p.fixed_window = a.calib == QSM_CALIB_FIXED_WINDOW;
   p.flush = a.below_policy == 1;
-  p.surrogate = a.surrogate;
-  p.detach = a.detach;
-  p.calib = a.mode == QSM_MODE_KINTERVAL && !a.detach;
-  p.KT = (p.K + 2) & ~1;
+  // the dK / dV pass's table row: interpolation K + 2 (e, d) pairs, hard
+  // rounding K + 1 grid values; a multiple of 4 floats (16-byte copies)
+  p.TS = map == MAPB_INTERP ? ((2 * (p.K + 2) + 3) & ~3)
+         : map == MAPB_HARD ? ((p.K + 1 + 3) & ~3)
+                            : 0;
   p.c = a.c;
   p.cL2E = a.c * 1.4426950408889634f;
   p.window = a.window;
@@ -1263,17 +1331,24 @@ qsm_status launch_bwd(const BwdArgs &a) {
   p.lo = a.row_lo;
   p.amax = a.row_argmax;
   p.amin = a.row_argmin;
+  // calibration form: none when detached, and for fixed-window hard rounding,
+  // whose grid does not move with hi
+  const bool calib = a.mode == QSM_MODE_KINTERVAL && !a.detach &&
+                     !(map == MAPB_HARD && p.fixed_window);
+  const int cal = !calib ? CAL_OFF : (p.fixed_window ? CAL_FIXED : CAL_MINMAX);
   uint8_t *ws = static_cast<uint8_t *>(a.workspace);
   const size_t o_dk = 0;
   const size_t o_rw = o_dk + align256(rows * a.D * sizeof(float));
   const size_t o_cst = o_rw + align256(rows * kRowWs * sizeof(float));
   const size_t o_tab = o_cst + align256(rows * kCst * sizeof(float));
-  p.dkcal = p.calib ? reinterpret_cast<float *>(ws + o_dk) : nullptr;
+  p.dkcal = calib ? reinterpret_cast<float *>(ws + o_dk) : nullptr;
   p.rowws = reinterpret_cast<float *>(ws + o_rw);
   p.cst = reinterpret_cast<float *>(ws + o_cst);
-  p.tabg = reinterpret_cast<float2 *>(ws + o_tab);
+  p.tabk = reinterpret_cast<float *>(ws + o_tab);
   p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
   p.K_ = static_cast<const __nv_bfloat16 *>(a.K);
+  p.O = static_cast<const __nv_bfloat16 *>(a.O);
+  p.dO = static_cast<const __nv_bfloat16 *>(a.dO);
   p.dQ = static_cast<__nv_bfloat16 *>(a.dQ);
   p.dK = static_cast<__nv_bfloat16 *>(a.dK);
   p.dV = static_cast<__nv_bfloat16 *>(a.dV);
@@ -1290,28 +1365,24 @@ qsm_status launch_bwd(const BwdArgs &a) {
   if (p.dkcal != nullptr &&
       cudaMemsetAsync(p.dkcal, 0, rows * a.D * sizeof(float), a.stream) != cudaSuccess)
     return QSM_ERR_CUDA;
-  const long long nrows = static_cast<long long>(rows);
-  qsm_bwd_delta<<<static_cast<unsigned>((nrows + 7) / 8), 256, 0, a.stream>>>(
-      static_cast<const __nv_bfloat16 *>(a.O), static_cast<const __nv_bfloat16 *>(a.dO), p.rowws,
-      nrows, a.D);
-  if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
-  if (a.mode != QSM_MODE_EXACT && a.surrogate == QSM_SURR_POST) {
-    // LSE* and delta* of the post surrogate (for Rowmax-PoT without the
-    // calibration sums, which it does not have)
-    BwdParams r = p;
-    if (p.map == MAPB_POT) {
-      r.map = MAPB_HARD;
-      r.detach = 1;
-    }
-    qsm_status st = launch_rows<64>(a, r, mq, mk, mv, mdo);
+  if (map != MAPB_EXACT && a.surrogate == QSM_SURR_POST) {
+    const qsm_status st = launch_rows<64>(a, p, mq, mk, mv, mdo);
     if (st != QSM_OK) return st;
   }
-  qsm_bwd_prep<<<static_cast<unsigned>((nrows + 255) / 256), 256, 0, a.stream>>>(p, nrows);
-  if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
-  if (p.map == MAPB_EXACT) return launch_passes<64, MAPB_EXACT>(a, p, mq, mk, mv, mdo);
-  if (p.map == MAPB_POT) return launch_passes<64, MAPB_POT>(a, p, mq, mk, mv, mdo);
-  if (p.map == MAPB_HARD) return launch_passes<64, MAPB_HARD>(a, p, mq, mk, mv, mdo);
-  return launch_passes<64, MAPB_INTERP>(a, p, mq, mk, mv, mdo);
+  const int surr = a.surrogate;
+  if (map == MAPB_EXACT)
+    return launch_passes<64, MAPB_EXACT, SURR_NONE, CAL_OFF>(a, p, mq, mk, mv, mdo);
+  if (map == MAPB_POT) return launch_by_surr<64, MAPB_POT, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
+  if (map == MAPB_HARD) {
+    if (cal == CAL_MINMAX)
+      return launch_by_surr<64, MAPB_HARD, CAL_MINMAX>(surr, a, p, mq, mk, mv, mdo);
+    return launch_by_surr<64, MAPB_HARD, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
+  }
+  if (cal == CAL_MINMAX)
+    return launch_by_surr<64, MAPB_INTERP, CAL_MINMAX>(surr, a, p, mq, mk, mv, mdo);
+  if (cal == CAL_FIXED)
+    return launch_by_surr<64, MAPB_INTERP, CAL_FIXED>(surr, a, p, mq, mk, mv, mdo);
+  return launch_by_surr<64, MAPB_INTERP, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
 }
 
 }  // namespace qsm

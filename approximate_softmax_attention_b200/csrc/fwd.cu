@@ -45,6 +45,7 @@ namespace qsm {
 struct FwdParams {
   int S, nqt, BH;
   int causal;
+  int hgroup;       // causal work order: heads per group (their K/V shares L2)
   int K;
   int fixed_window;
   int flush;        // below_policy == 1
@@ -516,17 +517,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using G = Geo<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   // Work order: non-causal CTAs sweep one head's query tiles after another
-  // (the running CTAs share few heads' K/V in L2); causal CTAs go heaviest
-  // first over all heads (longest-processing-time order, so the lightest
-  // tiles form the tail).
+  // (the running CTAs share few heads' K/V in L2); causal CTAs take groups of
+  // hgroup heads, whose K/V fit in L2 together, and within a group go
+  // heaviest first (longest-processing-time order, so the lightest tiles
+  // form each group's tail).
   int bh, qi;
   if (p.causal) {
-    const int rank = static_cast<int>(blockIdx.x) / p.BH;
-    bh = static_cast<int>(blockIdx.x) - rank * p.BH;
+    const int per = p.hgroup * p.nqt;
+    const int grp = static_cast<int>(blockIdx.x) / per;
+    const int within = static_cast<int>(blockIdx.x) - grp * per;
+    const int h0 = grp * p.hgroup;
+    const int gh = min(p.hgroup, p.BH - h0);
+    const int rank = within / gh;
+    bh = h0 + (within - rank * gh);
     qi = p.nqt - 1 - rank;
   } else {
     qi = static_cast<int>(blockIdx.x) % p.nqt;
@@ -784,6 +790,7 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   p.nqt = (a.S + 127) / 128;
   p.BH = a.B * a.H;
   p.causal = a.causal;
+  p.hgroup = causal_head_group(a.S, a.D, a.fp8, a.B * a.H);
   p.K = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) ? a.Kint : 1;
   p.fixed_window = a.calib == QSM_CALIB_FIXED_WINDOW;
   p.flush = a.below_policy == 1;

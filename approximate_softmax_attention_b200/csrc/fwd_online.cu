@@ -57,6 +57,7 @@ namespace {
 struct OnParams {
   int S, nqt, BH;
   int causal;
+  int hgroup;       // causal work order: heads per group (their K/V shares L2)
   int K;
   int flush;        // below_policy == 1
   int pot_floor;
@@ -480,13 +481,17 @@ __global__ void __launch_bounds__(kOnThreads, 1)
                           const __grid_constant__ CUtensorMap tmV, const OnParams p) {
   using G = OGeo<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5;
   int bh, qi;
   if (p.causal) {
-    const int rank = static_cast<int>(blockIdx.x) / p.BH;
-    bh = static_cast<int>(blockIdx.x) - rank * p.BH;
+    const int per = p.hgroup * p.nqt;
+    const int grp = static_cast<int>(blockIdx.x) / per;
+    const int within = static_cast<int>(blockIdx.x) - grp * per;
+    const int h0 = grp * p.hgroup;
+    const int gh = min(p.hgroup, p.BH - h0);
+    const int rank = within / gh;
+    bh = h0 + (within - rank * gh);
     qi = p.nqt - 1 - rank;
   } else {
     qi = static_cast<int>(blockIdx.x) % p.nqt;
@@ -699,6 +704,7 @@ qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMa
   p.nqt = (a.S + 127) / 128;
   p.BH = a.B * a.H;
   p.causal = a.causal;
+  p.hgroup = causal_head_group(a.S, a.D, a.fp8, a.B * a.H);
   p.K = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) ? a.Kint : 1;
   p.flush = a.below_policy == 1;
   p.pot_floor = a.pot_floor;

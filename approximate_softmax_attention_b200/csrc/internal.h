@@ -68,6 +68,17 @@ struct BwdArgs {
 };
 
 qsm_status launch_bwd(const BwdArgs &a);
+
+// Causal forward work order: heads per group, so that the K and V of one
+// group (2 S D bytes per element each head) stay within about 48 MB of the
+// 126 MB L2 while the running CTAs sweep them.
+inline int causal_head_group(int S, int D, bool fp8, int BH) {
+  const double kv = 2.0 * S * D * (fp8 ? 1 : 2);
+  int g = static_cast<int>((48.0 * 1024 * 1024) / kv);
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return g;
+}
 size_t bwd_workspace_bytes(int B, int H, int S, int D);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no

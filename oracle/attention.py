@@ -285,12 +285,15 @@ def attn_fwd(q, k, v, causal, mode, K=4, calib=MINMAX, rounding=HARD,
 
 def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
                   surrogate=SURR_NONE, detach_extrema=False, window=8.0,
-                  below_policy=0, frozen=None, pot_floor=15):
+                  below_policy=0, frozen=None, pot_floor=15, O_in=None):
     """Backward of one block of query rows against all keys.
 
     Returns (dS [R,S], P [R,S], O [R,D]): dS is dL/ds (before the factor c
     that maps it to dQ / dK), P the forward probabilities.  The rules are the
     exact gradients of the surrogate graphs named in the module docstring.
+    delta = dO . O is formed from O_in when given (the forward output a
+    caller stores and passes back, as the library's backward takes it), else
+    from this function's own O = P V.
     Rowmax-PoT (its backward is not derived on the pages; these are the same
     surrogate graphs applied to it): with its exponents frozen a power-of-two
     weight depends neither on its own score nor on the anchor, so only the
@@ -303,7 +306,7 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
     P = w / Z[:, None]
     O = P @ v
     dp = dO @ v.T                                   # dp_j = dO_r . v_j
-    delta = (dO * O).sum(axis=1)                    # sum_j p_j dp_j
+    delta = (dO * (O if O_in is None else O_in)).sum(axis=1)   # dO . O = sum_j p_j dp_j
     gw = np.where(valid, (dp - delta[:, None]) / Z[:, None], 0.0)   # dL/dw_j
     R = s.shape[0]
     rows = np.arange(R)
@@ -394,14 +397,18 @@ def attn_bwd_rows(s, valid, v, dO, mode, K=4, calib=MINMAX, rounding=HARD,
 def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
              surrogate=SURR_NONE, detach_extrema=False, scale=None,
              window=8.0, below_policy=0, heads=None, row_block=512,
-             decisions=None, pot_floor=15):
+             decisions=None, pot_floor=15, O=None):
     """Gradients dQ, dK, dV [B,H,S,D] (float64) of the attention forward.
 
     ``heads`` restricts the work to a list of (b, h); other heads are NaN.
     ``decisions`` (optional, [B,H,S,S] ints, the forward's per-element node
     decisions) freezes the K-interval decisions at those values.
+    ``O`` (optional, [B,H,S,D]) is the stored forward output the backward
+    forms delta = dO . O from, as the library's backward does with the O it
+    is given; by default the exact output P V.
     """
     q, k, v, dO = _as64(q), _as64(k), _as64(v), _as64(dO)
+    O_given = None if O is None else _as64(O)
     B, H, S, D = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(D)
@@ -421,7 +428,8 @@ def attn_bwd(q, k, v, dO, causal, mode, K=4, calib=MINMAX, rounding=HARD,
             ds, P, _ = attn_bwd_rows(s, valid, v[b, h], dO[b, h, rr], mode,
                                      K, calib, rounding, surrogate,
                                      detach_extrema, window, below_policy, fz,
-                                     pot_floor)
+                                     pot_floor,
+                                     None if O_given is None else O_given[b, h, rr])
             dQ[b, h, rr] = c * (ds @ k[b, h])
             dK[b, h] += c * (ds.T @ q[b, h, rr])
             dV[b, h] += P.T @ dO[b, h, rr]

@@ -18,6 +18,13 @@ slope, and the row's calibration sums dhi / dlo, which land on the whole dQ
 row and on the dK rows of the row's argmax and argmin.  Those gradient rows
 (and the dK / dV rows of the flipped key) are left out of the comparison and
 counted; the oracle itself never sees the kernel's decisions.
+
+Both backwards form delta = dO . O from the stored forward output they are
+given, as the library's backward does with the O a caller passes back.  Both
+get the same one: the oracle's own forward output rounded to bf16, the
+format the forward writes (a kernel O would bring a CUDA value into the
+oracle; an fp64 O on one side only would test bf16 storage, not the
+backward: on a short causal row it moves delta by several percent).
 """
 
 import numpy as np
@@ -27,19 +34,30 @@ import torch
 import oracle
 from approximate_softmax_attention_b200 import inputs, qsm
 
-from _helpers import check_bf16_output, check_decisions
+from _helpers import check_bf16_output, check_decisions, to_bf16
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda:0"
 
 
-def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True):
+def _stored_o(d, causal, mode, K, calib, rnd, window=8.0, heads=None):
+    """The oracle's forward (with its decision indices), whose O rounded to
+    bf16 both backwards take as the stored output."""
+    return oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, K=K, calib=calib, rounding=rnd,
+                           window=window, heads=heads, want_idx=True)
+
+
+def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True, O_store=None):
     q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
     B, H, S, D = q.shape
     dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV) if dump else None
     O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rnd, window=window,
                                        stats=True, debug_idx=dbg)
+    if O_store is not None:
+        # heads the oracle left out (NaN) keep the kernel's own output
+        Os = torch.from_numpy(np.asarray(O_store, dtype=np.float32)).to(DEV)
+        O = torch.where(torch.isnan(Os), O.float(), Os).to(torch.bfloat16).contiguous()
     dQ, dK, dV = qsm.attention_backward(q, k, v, O, dO, LSE, st, causal, mode, K, calib, rnd,
                                         surr, detach_extrema=detach, window=window)
     torch.cuda.synchronize()
@@ -47,25 +65,25 @@ def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True):
     return out, (dbg.cpu().numpy() if dump else None)
 
 
-def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None):
-    """The oracle's backward at its own fp64 decisions."""
+def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None, O_store=None):
+    """The oracle's backward at its own fp64 decisions, delta from the stored
+    (bf16) output."""
     return oracle.attn_bwd(d["q"], d["k"], d["v"], d["dO"], causal, mode, K=K, calib=calib,
                            rounding=rnd, surrogate=surr, detach_extrema=detach, window=window,
-                           heads=heads)
+                           heads=heads, O=None if O_store is None else to_bf16(O_store))
 
 
-def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads):
+def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads, ref):
     """Rows of dQ and of dK / dV touched by the kernel forward's decision
     mismatches with fp64 rounding (after checking every mismatch lies within
-    1e-3 of a boundary); returns boolean [B,H,S] masks and the count."""
+    1e-3 of a boundary); returns boolean [B,H,S] masks and the count.  ref:
+    the oracle's forward with its decision indices."""
     B, H, S, _ = d["q"].shape
     dq = np.zeros((B, H, S), bool)
     dkv = np.zeros((B, H, S), bool)
     if mode != 1 or dec is None:
         return dq, dkv, 0
     check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads)
-    ref = oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, K=K, calib=calib, rounding=rnd,
-                          window=window, heads=heads, want_idx=True)
     n = 0
     for (b, h) in heads:
         valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal \
@@ -101,10 +119,11 @@ COMBOS = [(K, c, r, s, det) for K in (4, 16) for c in (0, 1) for r in (0, 1)
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
 def test_bwd_kinterval_small(S, causal, K, calib, rnd, surr, detach):
     d = inputs.draw(1, 2, S, 64, seed=50 + S, with_dO=True)
-    got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
-    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0)
+    fwd = _stored_o(d, causal, 1, K, calib, rnd, window=6.0)
+    got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
+    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
     heads = [(0, 0), (0, 1)]
-    fq, fkv, n = _flip_rows(d, dec, causal, 1, K, calib, rnd, 6.0, heads)
+    fq, fkv, n = _flip_rows(d, dec, causal, 1, K, calib, rnd, 6.0, heads, fwd)
     _check(got, ref, skip=(fq, fkv))
     assert fq.sum() <= 0.02 * fq.size, n
 
@@ -116,9 +135,10 @@ def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
     """K = 1 (one grid segment) and K = 32 (the largest K the backward
     accepts), pre and post surrogate, calibration derivatives on."""
     d = inputs.draw(1, 2, 256, 64, seed=90 + K, with_dO=True)
-    got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0)
-    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0)
-    fq, fkv, n = _flip_rows(d, dec, True, 1, K, calib, rnd, 6.0, [(0, 0), (0, 1)])
+    fwd = _stored_o(d, True, 1, K, calib, rnd, window=6.0)
+    got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
+    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
+    fq, fkv, n = _flip_rows(d, dec, True, 1, K, calib, rnd, 6.0, [(0, 0), (0, 1)], fwd)
     _check(got, ref, skip=(fq, fkv))
     assert fq.sum() <= 0.02 * fq.size, n
 
@@ -126,8 +146,9 @@ def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
 @pytest.mark.parametrize("S,causal", [(256, True), (200, False), (77, True), (384, False)])
 def test_bwd_exact(S, causal):
     d = inputs.draw(1, 2, S, 64, seed=7 + S, with_dO=True)
-    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False, dump=False)
-    ref = _oracle(d, causal, 0, 4, 0, 1, 0, False)
+    fwd = _stored_o(d, causal, 0, 4, 0, 1)
+    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False, dump=False, O_store=fwd["O"])
+    ref = _oracle(d, causal, 0, 4, 0, 1, 0, False, O_store=fwd["O"])
     _check(got, ref)
 
 
@@ -141,9 +162,10 @@ def test_bwd_training_shape_sampled(mode, K, calib, rnd, surr, detach):
     w = inputs.WORKLOADS["train_s1k"]
     d = inputs.draw_workload(w)
     heads = [(0, 0), (3, 7), (7, 11)]
-    got, dec = _run(d, True, mode, K, calib, rnd, surr, detach)
-    ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads)
-    fq, fkv, n = _flip_rows(d, dec, True, mode, K, calib, rnd, 8.0, heads)
+    fwd = _stored_o(d, True, mode, K, calib, rnd, heads=heads)
+    got, dec = _run(d, True, mode, K, calib, rnd, surr, detach, O_store=fwd["O"])
+    ref = _oracle(d, True, mode, K, calib, rnd, surr, detach, heads=heads, O_store=fwd["O"])
+    fq, fkv, n = _flip_rows(d, dec, True, mode, K, calib, rnd, 8.0, heads, fwd)
     _check(got, ref, heads=heads, skip=(fq, fkv))
     # the flips are rare: a few rows of the three heads checked
     assert fq.sum() <= 0.01 * 3 * 1024, n
@@ -157,8 +179,9 @@ def test_bwd_rowmax_pot(S, causal, surr):
     """Rowmax-PoT under the surrogate rules (exponents frozen: none gives dQ =
     dK = 0 and only dV; pre and post the surrogate's direct term)."""
     d = inputs.draw(1, 2, S, 64, seed=70 + S, with_dO=True)
-    got, _ = _run(d, causal, 2, 4, 0, 1, surr, False, dump=False)
-    ref = _oracle(d, causal, 2, 4, 0, 1, surr, False)
+    fwd = _stored_o(d, causal, 2, 4, 0, 1)
+    got, _ = _run(d, causal, 2, 4, 0, 1, surr, False, dump=False, O_store=fwd["O"])
+    ref = _oracle(d, causal, 2, 4, 0, 1, surr, False, O_store=fwd["O"])
     _check(got, ref)
     if surr == 0:
         assert np.abs(got[0]).max() == 0 and np.abs(got[1]).max() == 0
@@ -169,6 +192,7 @@ def test_bwd_rowmax_pot_training_shape(surr):
     w = inputs.WORKLOADS["train_s1k"]
     d = inputs.draw_workload(w)
     heads = [(1, 2), (6, 9)]
-    got, _ = _run(d, True, 2, 4, 0, 1, surr, False, dump=False)
-    ref = _oracle(d, True, 2, 4, 0, 1, surr, False, heads=heads)
+    fwd = _stored_o(d, True, 2, 4, 0, 1, heads=heads)
+    got, _ = _run(d, True, 2, 4, 0, 1, surr, False, dump=False, O_store=fwd["O"])
+    ref = _oracle(d, True, 2, 4, 0, 1, surr, False, heads=heads, O_store=fwd["O"])
     _check(got, ref, heads=heads)

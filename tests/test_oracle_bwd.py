@@ -152,6 +152,36 @@ def test_exact_backward_is_autograd(causal):
 
 
 @pytest.mark.parametrize("causal", [False, True])
+def test_stored_output_enters_only_through_delta(causal):
+    """delta = dO . O is formed from the stored output when one is given.
+    Given the exact output it changes nothing; given O + E, delta moves by
+    dO . E per row, which for the exact map (dS = P (dP - delta)) moves dQ by
+    -c (dO . E) (P K) and dK by -c P^T ((dO . E) Q), and leaves dV alone."""
+    rng = np.random.default_rng(12)
+    B, H, S, D = 1, 1, 13, 8
+    q, k, v, dO = (rng.normal(size=(B, H, S, D)) for _ in range(4))
+    c = 1.0 / math.sqrt(D)
+    base = oracle.attn_bwd(q, k, v, dO, causal, A.EXACT)
+    O = oracle.attn_fwd(q, k, v, causal, A.EXACT)["O"]
+    same = oracle.attn_bwd(q, k, v, dO, causal, A.EXACT, O=O)
+    for n in ("dQ", "dK", "dV"):
+        np.testing.assert_allclose(same[n], base[n], rtol=1e-12, atol=1e-13)
+    E = 1e-3 * rng.normal(size=O.shape)
+    moved = oracle.attn_bwd(q, k, v, dO, causal, A.EXACT, O=O + E)
+    shift = (dO * E).sum(axis=-1)[0, 0]                       # [S]
+    s = c * (q[0, 0] @ k[0, 0].T)
+    if causal:
+        s = np.where(np.tril(np.ones((S, S), bool)), s, -np.inf)
+    P = np.exp(s - s.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(moved["dQ"][0, 0] - base["dQ"][0, 0],
+                               -c * shift[:, None] * (P @ k[0, 0]), rtol=1e-9, atol=1e-13)
+    np.testing.assert_allclose(moved["dK"][0, 0] - base["dK"][0, 0],
+                               -c * P.T @ (shift[:, None] * q[0, 0]), rtol=1e-9, atol=1e-13)
+    np.testing.assert_allclose(moved["dV"], base["dV"], rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("calib,rounding", [(0, 0), (0, 1), (1, 0), (1, 1)])
 def test_post_detached_is_softmax_backward_for_q_and_k(causal, calib, rounding):
     rng = np.random.default_rng(10)
