@@ -82,8 +82,8 @@ struct BwdParams {
   const float *LSE, *hi, *lo;
   const int32_t *amax, *amin;
   float *rowws;     // [rows][kRowWs]: LSE*, delta* (post surrogate)
-  float *cst;       // [rows][kCst]: a, b, 1/Z, -delta/Z, e0, delta_s, K/(hi-lo), 0
-  float *tabk;      // [rows][TS]: the dK / dV pass's grid table of each row
+  float *cst;       // [tile rows / 2][16]: row pairs' constants, interleaved (cst_index)
+  float *tabk;      // [tile rows][TS]: the dK / dV pass's grid table of each row
   float *dkcal;     // [rows][D] fp32 calibration part of dK (nullptr: none)
   const __nv_bfloat16 *Q, *K_, *O, *dO;
   __nv_bfloat16 *dQ, *dK, *dV;
@@ -398,6 +398,26 @@ struct RowC {
   bool calib;       // the row takes calibration terms
 };
 
+// Workspace rows are tile rows: (bh * nqt + qt) * 128 + row, so that every
+// query tile starts a row pair.  The constants of rows 2m and 2m + 1 sit
+// together, each field as a pair, so that one 16-byte load gives the packed
+// operands of two rows: [a a' b b' | invZ invZ' nDZ nDZ' | -e0 -e0' -ds_ -ds_'
+// | kinv kinv' 0 0] (16 floats).
+__device__ __forceinline__ size_t tile_row(const BwdParams &p, int bh, int qt, int row) {
+  return (static_cast<size_t>(bh) * p.nqt + qt) * 128 + row;
+}
+__device__ __forceinline__ void store_row_constants(const BwdParams &p, size_t trow, const RowC &k) {
+  float *c = p.cst + (trow >> 1) * 16 + (trow & 1);
+  c[0] = k.a;
+  c[2] = k.b;
+  c[4] = k.invZ;
+  c[6] = k.nDZ;
+  c[8] = -k.e0;
+  c[10] = -k.ds_;
+  c[12] = k.kinv;
+  c[14] = 0.0f;
+}
+
 // Table layouts (K-interval).  Entry i of a row, interpolation, i = 0..K+1:
 // i = 0 the below-window entry (fixed window: weight g_0, or 0 when flushed,
 // no derivative; min-max: a copy of interval 0), i = k + 1 interval k =
@@ -425,8 +445,8 @@ struct DqTab {
 // tables (entries g, g + 4, ...), both for the dQ pass (shared memory at
 // tq_base) and, when row_ok, for the dK / dV pass (workspace).
 template <int MAP, int SURR, int CAL>
-__device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, int g, int row,
-                                              bool row_ok, uint32_t tq_base) {
+__device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, size_t trow, int g,
+                                              int row, bool row_ok, uint32_t tq_base) {
   using T = DqTab<MAP, SURR, CAL>;
   RowC k;
   k.a = k.b = k.invZ = k.nDZ = k.e0 = k.ds_ = k.kinv = 0.0f;
@@ -451,7 +471,7 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, int
     k.kinv = rm.inv;
     k.calib = CAL != CAL_OFF && !rm.degenerate;
     const float Kf = static_cast<float>(p.K);
-    float *tk = p.tabk + ri * p.TS;
+    float *tk = p.tabk + trow * p.TS;
     if (MAP == MAPB_INTERP) {
       const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(hi, rm.lo));
       for (int i = g; i <= p.K + 1; i += 4) {
@@ -495,6 +515,77 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, int
     k.ds_ = w[RW_DELTASTAR];
   }
   return k;
+}
+
+__device__ __forceinline__ float2 ex2_pair(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
+// The dQ pass's per-row values for the element loop.
+struct DqK {
+  float a, b, invZ, nDZ, ne0, nds, kinv, cL2E, Kf;
+  uint32_t tq_row;   // biased shared address of this row's dQ-pass table
+};
+
+// dS of one 16-key slice of a row (bf16 pairs into dd) and the calibration
+// sums, two elements per packed fp32 operation.  FULL: every key valid.
+template <int MAP, int SURR, int CAL, bool FULL>
+__device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
+                                         const DqK &k, int lim, uint32_t (&dd)[8], float2 &s1,
+                                         float2 &s2) {
+  using T = DqTab<MAP, SURR, CAL>;
+  const float2 cl2 = make_float2(k.cL2E, k.cL2E), ne0 = make_float2(k.ne0, k.ne0);
+  const float2 nds = make_float2(k.nds, k.nds);
+  const float2 mg = make_float2(kMagic, kMagic);
+#pragma unroll
+  for (int i2 = 0; i2 < 8; ++i2) {
+    const float2 r = make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1]));
+    const float2 dp = make_float2(__uint_as_float(dv[2 * i2]), __uint_as_float(dv[2 * i2 + 1]));
+    const bool v0 = FULL || 2 * i2 < lim, v1 = FULL || 2 * i2 + 1 < lim;
+    float2 ds = make_float2(0.0f, 0.0f);
+    if (MAP == MAPB_EXACT) {
+      ds = mul2_rn(ex2_pair(fma2_rn(r, cl2, ne0)), add2_rn(dp, nds));
+    } else {
+      float2 gw = fma2_rn(dp, make_float2(k.invZ, k.invZ), make_float2(k.nDZ, k.nDZ));
+      if (!v0) gw.x = 0.0f;
+      if (!v1) gw.y = 0.0f;
+      if (SURR == SURR_PRE)
+        ds = mul2_rn(gw, ex2_pair(fma2_rn(r, cl2, ne0)));
+      else if (SURR == SURR_POST)
+        ds = mul2_rn(ex2_pair(fma2_rn(r, cl2, ne0)), add2_rn(dp, nds));
+      if (T::ANY) {
+        const float2 u = fma2_rn(r, make_float2(k.a, k.a), make_float2(k.b, k.b));
+        if (MAP == MAPB_INTERP) {
+          const float2 uc = make_float2(fminf(fmaxf(u.x, -1.0f), k.Kf), fminf(fmaxf(u.y, -1.0f), k.Kf));
+          const float2 t = add2_rd(uc, mg);
+          const uint32_t ad0 = __float_as_uint(t.x) * T::STRIDE + k.tq_row;
+          const uint32_t ad1 = __float_as_uint(t.y) * T::STRIDE + k.tq_row;
+          float2 d;
+          if (CAL == CAL_MINMAX) {
+            const float4 e0 = lds_f32x4(ad0), e1 = lds_f32x4(ad1);     // A, B, d
+            s1 = fma2_rn(gw, make_float2(__fmaf_rn(e0.y, uc.x, e0.x), __fmaf_rn(e1.y, uc.y, e1.x)),
+                         s1);
+            d = make_float2(e0.z, e1.z);
+            s2 = fma2_rn(gw, d, s2);
+          } else {
+            d = make_float2(lds_f32(ad0), lds_f32(ad1));
+            if (CAL == CAL_FIXED) s2 = fma2_rn(gw, d, s2);
+          }
+          if (SURR == SURR_NONE) ds = mul2_rn(mul2_rn(gw, d), make_float2(k.kinv, k.kinv));
+        } else {
+          const float2 uc = make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
+          const float2 t = add2_rn(uc, mg);
+          s1 = fma2_rn(gw,
+                       make_float2(lds_f32(__float_as_uint(t.x) * T::STRIDE + k.tq_row),
+                                   lds_f32(__float_as_uint(t.y) * T::STRIDE + k.tq_row)),
+                       s1);
+        }
+      }
+    }
+    if (!v0) ds.x = 0.0f;
+    if (!v1) ds.y = 0.0f;
+    dd[i2] = pack_bf16x2(ds.x, ds.y);
+  }
 }
 
 // ----------------------------------------------------------------- dQ pass
@@ -673,7 +764,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
     }
     const uint32_t tq_base = smem_u32(smem + p.tab_off);
-    RowC kc = row_constants<MAP, SURR, CAL>(p, ri, g, row, row_ok, tq_base);
+    const size_t trow = tile_row(p, bh, qt, row);
+    RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, tq_base);
     mbar_arrive(bars.tab_ready);
     bool ok = warp_all_b(mbar_wait(bars.tab_ready, 0, abort));
     const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
@@ -682,19 +774,25 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     } else {
       kc.nDZ = -__fmul_rn(delta, kc.invZ);
     }
-    if (g == 0 && row_ok) {
-      float4 *cd = reinterpret_cast<float4 *>(p.cst + ri * kCst);
-      cd[0] = make_float4(kc.a, kc.b, kc.invZ, kc.nDZ);
-      cd[1] = make_float4(kc.e0, kc.ds_, kc.kinv, 0.0f);
-    }
+    if (g == 0 && row_ok) store_row_constants(p, trow, kc);
     // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) - bits(M)
     // + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard),
     // M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
-    const uint32_t tq_row = (MAP == MAPB_INTERP)
-                                ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
-                                : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
-    const float Kf = static_cast<float>(p.K);
-    float s1 = 0.0f, s2 = 0.0f;                          // calibration sums
+    DqK dk;
+    dk.a = kc.a;
+    dk.b = kc.b;
+    dk.invZ = kc.invZ;
+    dk.nDZ = kc.nDZ;
+    dk.ne0 = -kc.e0;
+    dk.nds = -kc.ds_;
+    dk.kinv = kc.kinv;
+    dk.cL2E = p.cL2E;
+    dk.Kf = static_cast<float>(p.K);
+    dk.tq_row = (MAP == MAPB_INTERP)
+                    ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
+                    : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
+    const float Kf = dk.Kf;
+    float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
     const uint32_t dsb = smem_u32(sDS);
     for (int h = 0; h < nh && ok; ++h) {
       const int j = h >> 1, e = h & 1, x = h & 1;
@@ -710,54 +808,11 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars.sdp_free[x]);                  // the pair can take half h + 2
       const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
-      const bool full = warp_all_b(lim >= 16);
       uint32_t dd[8];
-#pragma unroll
-      for (int i2 = 0; i2 < 8; ++i2) {
-        float d2[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int i = 2 * i2 + t;
-          const bool valid = full || i < lim;
-          const float r = __uint_as_float(sv[i]), dp = __uint_as_float(dv[i]);
-          float ds;
-          if (MAP == MAPB_EXACT) {
-            ds = ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0)) * (dp - kc.ds_);
-          } else {
-            float gw = __fmaf_rn(dp, kc.invZ, kc.nDZ);
-            if (!valid) gw = 0.0f;
-            if (SURR == SURR_PRE)
-              ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0));
-            else if (SURR == SURR_POST)
-              ds = ex2_approx(__fmaf_rn(r, p.cL2E, -kc.e0)) * (dp - kc.ds_);
-            else
-              ds = 0.0f;
-            if (T::ANY) {
-              const float u = __fmaf_rn(r, kc.a, kc.b);
-              if (MAP == MAPB_INTERP) {
-                const float ucl = fminf(fmaxf(u, -1.0f), Kf);
-                const uint32_t ad = __float_as_uint(__fadd_rd(ucl, kMagic)) * T::STRIDE + tq_row;
-                if (CAL == CAL_MINMAX) {
-                  const float4 ab = lds_f32x4(ad);     // A, B, d
-                  s1 = __fmaf_rn(gw, __fmaf_rn(ab.y, ucl, ab.x), s1);
-                  s2 = __fmaf_rn(gw, ab.z, s2);
-                  if (SURR == SURR_NONE) ds = gw * ab.z * kc.kinv;
-                } else {
-                  const float d = lds_f32(ad);
-                  if (CAL == CAL_FIXED) s2 = __fmaf_rn(gw, d, s2);
-                  if (SURR == SURR_NONE) ds = gw * d * kc.kinv;
-                }
-              } else {
-                const float uc = fminf(fmaxf(u, 0.0f), Kf);
-                const uint32_t ad = __float_as_uint(__fadd_rn(uc, kMagic)) * T::STRIDE + tq_row;
-                s1 = __fmaf_rn(gw, lds_f32(ad), s1);
-              }
-            }
-          }
-          d2[t] = valid ? ds : 0.0f;
-        }
-        dd[i2] = pack_bf16x2(d2[0], d2[1]);
-      }
+      if (warp_all_b(lim >= 16))
+        dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
+      else
+        dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
       if (h >= 2) {
         ok = warp_all_b(mbar_wait(&bars.ds_free[x], ((h >> 1) - 1) & 1, abort));
         if (!ok) break;
@@ -776,8 +831,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_arrive(&bars.ds_full[x]);
     }
     // ---- epilogue: the row's calibration sums, dQ
-    part[(4 + g) * 128 + row] = s1;
-    part[(8 + g) * 128 + row] = s2;
+    part[(4 + g) * 128 + row] = s1.x + s1.y;
+    part[(8 + g) * 128 + row] = s2.x + s2.y;
     mbar_arrive(bars.part_ready);
     if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
     if (ok) ok = warp_all_b(mbar_wait(bars.dq_full, 0, abort));
@@ -867,45 +922,82 @@ struct KvBars {
 };
 constexpr uint32_t T_DV = 256, T_DK = 320;
 
-// One element of the dK / dV pass: the probability p = w / Z (returned) and
-// ds (the surrogate's dL/ds before the factor c).  c0 = (a, b, 1/Z,
-// -delta/Z), c1 = (e0, delta_s, K/(hi-lo), 0) of the element's query row;
-// trow the (biased) shared address of that row's table.
-template <int MAP, int SURR>
-__device__ __forceinline__ float kv_elem(float r, float dp, const float4 &c0, const float4 &c1,
-                                         uint32_t trow, const BwdParams &p, float Kf, float cap,
-                                         float flush_t, bool flush_below, float &ds) {
-  if (MAP == MAPB_EXACT) {
-    const float pw = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
-    ds = pw * (dp - c1.y);
-    return pw;
+// The dK / dV pass's per-thread values for the element loop.
+struct KvK {
+  float cL2E, Kf, cap, flush_t;
+  bool flush, flush_below;
+};
+
+// P^T and dS^T of one key against a 16-row query slice (bf16 pairs into pp,
+// dd), two rows per packed fp32 operation.  cb: shared address of the
+// slice's first row pair of constants (64 bytes a pair, see
+// store_row_constants); tr: biased shared address of the slice's first row
+// table, ts its row stride in bytes; vmask: valid rows (bit i) unless FULL.
+template <int MAP, int SURR, bool FULL>
+__device__ __forceinline__ void kv_slice(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
+                                         uint32_t cb, uint32_t tr, uint32_t ts, const KvK &k,
+                                         uint32_t vmask, uint32_t (&pp)[8], uint32_t (&dd)[8]) {
+  const float2 cl2 = make_float2(k.cL2E, k.cL2E);
+  const float2 mg = make_float2(kMagic, kMagic);
+#pragma unroll
+  for (int i2 = 0; i2 < 8; ++i2) {
+    const float2 r = make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1]));
+    const float2 dp = make_float2(__uint_as_float(dv[2 * i2]), __uint_as_float(dv[2 * i2 + 1]));
+    const uint32_t c = cb + i2 * 64;
+    const uint32_t t0 = tr + (2 * i2) * ts, t1 = t0 + ts;
+    float2 pw, ds = make_float2(0.0f, 0.0f);
+    if (MAP == MAPB_EXACT) {
+      const float4 c2 = lds_f32x4(c + 32);                 // -e0 pair, -delta pair
+      pw = ex2_pair(fma2_rn(r, cl2, make_float2(c2.x, c2.y)));
+      ds = mul2_rn(pw, add2_rn(dp, make_float2(c2.z, c2.w)));
+    } else {
+      const float4 c0 = lds_f32x4(c);                      // a pair, b pair
+      const float4 c1 = lds_f32x4(c + 16);                 // 1/Z pair, -delta/Z pair
+      const float2 iz = make_float2(c1.x, c1.y);
+      const float2 gw = fma2_rn(dp, iz, make_float2(c1.z, c1.w));
+      const float2 u = fma2_rn(r, make_float2(c0.x, c0.y), make_float2(c0.z, c0.w));
+      float2 w, dn = make_float2(0.0f, 0.0f);
+      if (MAP == MAPB_POT) {
+        // the forward's power-of-two weight (exponent frozen: no own-score or
+        // anchor derivative; only the surrogate's direct term)
+        const float2 t = add2_rn(make_float2(fminf(u.x, k.cap), fminf(u.y, k.cap)), mg);
+        w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + 0x3F800000u),
+                        __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + 0x3F800000u));
+        if (k.flush && t.x > k.flush_t) w.x = 0.0f;
+        if (k.flush && t.y > k.flush_t) w.y = 0.0f;
+      } else if (MAP == MAPB_HARD) {
+        const float2 uc = make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
+        const float2 t = add2_rn(uc, mg);
+        w = make_float2(lds_f32(__float_as_uint(t.x) * 4u + t0),
+                        lds_f32(__float_as_uint(t.y) * 4u + t1));
+        if (k.flush_below && u.x < 0.0f) w.x = 0.0f;
+        if (k.flush_below && u.y < 0.0f) w.y = 0.0f;
+      } else {
+        const float2 uc = make_float2(fminf(fmaxf(u.x, -1.0f), k.Kf), fminf(fmaxf(u.y, -1.0f), k.Kf));
+        const float2 t = add2_rd(uc, mg);
+        const float2 e0 = lds_f32x2(__float_as_uint(t.x) * 8u + t0);
+        const float2 e1 = lds_f32x2(__float_as_uint(t.y) * 8u + t1);
+        w = make_float2(__fmaf_rn(uc.x, e0.y, e0.x), __fmaf_rn(uc.y, e1.y, e1.x));
+        dn = make_float2(e0.y, e1.y);
+      }
+      pw = mul2_rn(w, iz);
+      if (SURR == SURR_PRE) {
+        ds = mul2_rn(gw, ex2_pair(fma2_rn(r, cl2, lds_f32x2(c + 32))));
+      } else if (SURR == SURR_POST) {
+        const float4 c2 = lds_f32x4(c + 32);               // -e0 pair, -delta* pair
+        ds = mul2_rn(ex2_pair(fma2_rn(r, cl2, make_float2(c2.x, c2.y))),
+                     add2_rn(dp, make_float2(c2.z, c2.w)));
+      } else if (MAP == MAPB_INTERP) {
+        ds = mul2_rn(mul2_rn(gw, dn), lds_f32x2(c + 48));    // K/(hi - lo) pair
+      }
+    }
+    if (!FULL) {
+      if (!((vmask >> (2 * i2)) & 1u)) pw.x = ds.x = 0.0f;
+      if (!((vmask >> (2 * i2 + 1)) & 1u)) pw.y = ds.y = 0.0f;
+    }
+    pp[i2] = pack_bf16x2(pw.x, pw.y);
+    dd[i2] = pack_bf16x2(ds.x, ds.y);
   }
-  const float gw = __fmaf_rn(dp, c0.z, c0.w);
-  const float u = __fmaf_rn(r, c0.x, c0.y);
-  float w, dnone = 0.0f;
-  if (MAP == MAPB_POT) {
-    // the forward's power-of-two weight (exponent frozen: no own-score or
-    // anchor derivative; only the surrogate's direct term)
-    const float t = __fadd_rn(fminf(u, cap), kMagic);
-    w = __uint_as_float(__float_as_uint(t) * 0xFF800000u + 0x3F800000u);
-    if (p.flush && t > flush_t) w = 0.0f;
-  } else if (MAP == MAPB_HARD) {
-    const float uc = fminf(fmaxf(u, 0.0f), Kf);
-    w = lds_f32(__float_as_uint(__fadd_rn(uc, kMagic)) * 4u + trow);
-    if (flush_below && u < 0.0f) w = 0.0f;
-  } else {
-    const float ucl = fminf(fmaxf(u, -1.0f), Kf);
-    const float2 ed = lds_f32x2(__float_as_uint(__fadd_rd(ucl, kMagic)) * 8u + trow);
-    w = __fmaf_rn(ucl, ed.y, ed.x);
-    dnone = ed.y;
-  }
-  if (SURR == SURR_PRE)
-    ds = gw * ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x));
-  else if (SURR == SURR_POST)
-    ds = ex2_approx(__fmaf_rn(r, p.cL2E, -c1.x)) * (dp - c1.y);
-  else
-    ds = (MAP == MAPB_INTERP) ? gw * dnone * c1.z : 0.0f;
-  return w * c0.z;
 }
 
 template <int D, int MAP, int SURR>
@@ -978,12 +1070,11 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         if (n >= ns) ok = mbar_wait(&bars.qd_empty[st], ((n / ns) - 1) & 1, abort);
         if (!ok) break;
         uint8_t *s = sSt + st * SB;
-        // the constants and tables of the tile's rows that exist (a ragged last
-        // tile copies fewer; its missing rows are never valid)
-        const int nrow = min(128, p.S - it * 128);
-        const size_t r0 = static_cast<size_t>(bh) * p.S + static_cast<size_t>(it) * 128;
-        const uint32_t cbytes = static_cast<uint32_t>(nrow) * kCst * 4;
-        const uint32_t tbytes = static_cast<uint32_t>(nrow) * p.TS * 4;
+        // the constants and tables of the tile's 128 tile rows (rows past S in
+        // a ragged last tile are never valid)
+        const size_t r0 = (static_cast<size_t>(bh) * p.nqt + it) * 128;
+        const uint32_t cbytes = 128u * kCst * 4;
+        const uint32_t tbytes = 128u * static_cast<uint32_t>(p.TS) * 4;
         mbar_expect_tx(&bars.qd_full[st], 2 * G::TILE_BYTES + cbytes + tbytes);
         for (int ch = 0; ch < G::CHUNKS; ++ch) {
           tma_load_3d(s + ch * G::CHUNK_BYTES, &tmQ, &bars.qd_full[st], ch * G::EPC, it * 128, bh);
@@ -1061,10 +1152,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int kg = kt * 128 + key;
     const bool key_ok = kg < p.S;
-    const float Kf = static_cast<float>(p.K);
-    const float cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
-    const float flush_t = kMagic + static_cast<float>(p.pot_floor);
-    const bool flush_below = MAP == MAPB_HARD && p.flush && p.fixed_window;
+    KvK kk;
+    kk.cL2E = p.cL2E;
+    kk.Kf = static_cast<float>(p.K);
+    kk.cap = static_cast<float>(p.flush ? p.pot_floor + 1 : p.pot_floor);
+    kk.flush_t = kMagic + static_cast<float>(p.pot_floor);
+    kk.flush = p.flush != 0;
+    kk.flush_below = MAP == MAPB_HARD && p.flush && p.fixed_window;
     // table entry bias: bits(M + floor(clamp(u, -1, K))) - bits(M) + 1 (interp)
     // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), mod 2^32
     const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - kMagicBits * 8u : 0u - kMagicBits * 4u;
@@ -1092,39 +1186,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       // every element valid: the key exists, the slice's rows exist and (causal)
       // lie at or below this key
       const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
+      const uint32_t cb = st + CST_OFF + ql0 * (kCst * 4);
+      const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
+      const uint32_t tr = st + TAB_OFF + ql0 * tsb + tbias;
       uint32_t pp[8], dd[8];
+      if (full) {
+        kv_slice<MAP, SURR, true>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
+      } else {
+        uint32_t vmask = 0;
 #pragma unroll
-      for (int i2 = 0; i2 < 8; ++i2) {
-        float p2[2], d2[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int i = 2 * i2 + t;
-          const int ql = ql0 + i;
-          const int qg = qbase + i;
-          const bool valid = full || (key_ok && qg < p.S && (!p.causal || kg <= qg));
-          const uint32_t ca = st + CST_OFF + ql * (kCst * 4);
-          // only the constants this map and surrogate read
-          const float4 c0 = (MAP == MAPB_EXACT) ? make_float4(0.0f, 0.0f, 0.0f, 0.0f)
-                                                : lds_f32x4(ca);
-          float4 c1 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (MAP == MAPB_EXACT || SURR == SURR_POST) {
-            const float2 t2 = lds_f32x2(ca + 16);
-            c1.x = t2.x;
-            c1.y = t2.y;
-          } else if (SURR == SURR_PRE) {
-            c1.x = lds_f32(ca + 16);
-          } else if (MAP == MAPB_INTERP) {
-            c1.z = lds_f32(ca + 24);
-          }
-          float ds;
-          const float pw = kv_elem<MAP, SURR>(__uint_as_float(sv[i]), __uint_as_float(dv[i]), c0,
-                                              c1, st + TAB_OFF + ql * (p.TS * 4) + tbias, p, Kf,
-                                              cap, flush_t, flush_below, ds);
-          p2[t] = valid ? pw : 0.0f;
-          d2[t] = valid ? ds : 0.0f;
-        }
-        pp[i2] = pack_bf16x2(p2[0], p2[1]);
-        dd[i2] = pack_bf16x2(d2[0], d2[1]);
+        for (int i = 0; i < 16; ++i)
+          vmask |= (key_ok && qbase + i < p.S && (!p.causal || kg <= qbase + i)) ? (1u << i) : 0u;
+        kv_slice<MAP, SURR, false>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
       }
       tmem_st8(lane_base + 128 * x + 16 * g, pp);
       tmem_st8(lane_base + 128 * x + 64 + 16 * g, dd);
@@ -1292,12 +1365,13 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 }  // namespace
 
 size_t bwd_workspace_bytes(int B, int H, int S, int D) {
-  // fp32 calibration part of dK, then per query row: the row workspace, the
-  // map constants and the dK / dV pass's grid table; each part 256-byte
-  // aligned
+  // fp32 calibration part of dK and the row workspace per query row, then
+  // per tile row (each head's rows padded to whole 128-row tiles) the map
+  // constants and the dK / dV pass's grid table; each part 256-byte aligned
   const size_t rows = static_cast<size_t>(B) * H * S;
+  const size_t trows = static_cast<size_t>(B) * H * ((S + 127) / 128) * 128;
   return align256(rows * D * sizeof(float)) + align256(rows * kRowWs * sizeof(float)) +
-         align256(rows * kCst * sizeof(float)) + align256(rows * kTabKT * sizeof(float2));
+         align256(trows * kCst * sizeof(float)) + align256(trows * kTabKT * sizeof(float2));
 }
 
 qsm_status launch_bwd(const BwdArgs &a) {
@@ -1340,7 +1414,8 @@ qsm_status launch_bwd(const BwdArgs &a) {
   const size_t o_dk = 0;
   const size_t o_rw = o_dk + align256(rows * a.D * sizeof(float));
   const size_t o_cst = o_rw + align256(rows * kRowWs * sizeof(float));
-  const size_t o_tab = o_cst + align256(rows * kCst * sizeof(float));
+  const size_t trows = static_cast<size_t>(p.BH) * p.nqt * 128;
+  const size_t o_tab = o_cst + align256(trows * kCst * sizeof(float));
   p.dkcal = calib ? reinterpret_cast<float *>(ws + o_dk) : nullptr;
   p.rowws = reinterpret_cast<float *>(ws + o_rw);
   p.cst = reinterpret_cast<float *>(ws + o_cst);

@@ -152,13 +152,13 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base, int ns) {
 
 // Weights of one 32-column chunk, packed for the PV MMA and stored to TMEM;
 // FULL: every column valid.  z holds eight partial row sums as four pairs.
-template <int MAP, bool FULL, bool FP8, bool FLUSH>
+template <int MAP, bool FULL, bool FP8, bool FLUSH, bool SAT>
 __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow &m, int c0,
                                           int lim, bool flush_below, float2 (&z)[4],
                                           uint32_t taddr_pc) {
   auto wt = [&](int i) {          // weights of columns 2i, 2i+1
     const float2 r = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-    float2 w = pair_weights<MAP, FLUSH>(r, m, flush_below);
+    float2 w = pair_weights<MAP, FLUSH, SAT>(r, m, flush_below);
     if (!FULL) {
       w.x = (c0 + 2 * i < lim) ? w.x : 0.0f;
       w.y = (c0 + 2 * i + 1 < lim) ? w.y : 0.0f;
@@ -186,7 +186,7 @@ __device__ __forceinline__ void map_chunk(const uint32_t (&v)[32], const MapRow 
 }
 
 // Decision dump of one chunk (debug option).
-template <int MAP>
+template <int MAP, bool SAT>
 __device__ __forceinline__ void debug_chunk(int8_t *dbg_row, const uint32_t (&v)[32],
                                             const MapRow &m, int kv0, int c0, int lim,
                                             const FwdParams &p, bool flush_below) {
@@ -194,7 +194,7 @@ __device__ __forceinline__ void debug_chunk(int8_t *dbg_row, const uint32_t (&v)
   for (int i = 0; i < 32; ++i) {
     if (dbg_row != nullptr && kv0 + i < p.S) {
       const float r = __uint_as_float(v[i]);
-      int n = map_raw_index<MAP>(r, m, p.flush != 0, p.pot_floor);
+      int n = map_raw_index<MAP, SAT>(r, m, p.flush != 0, p.pot_floor);
       if (flush_below && __fmaf_rn(r, m.a, m.b) < 0.0f) n = -2;
       dbg_row[kv0 + i] = static_cast<int8_t>((c0 + i < lim) ? n : -1);
     }
@@ -289,7 +289,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], float cL2E, f
 // (and minimum, arguments) over all keys, then the main sweep maps each score
 // against those final values.  For the exact map this is softmax against the
 // true row maximum, with no online rescaling of O.
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, int g, int row,
                                          uint32_t lane_base, int qi, int n, int bh, float *tab,
                                          const Xch &xc, volatile int *abort) {
@@ -423,6 +423,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   mc.pscale = p.pscale;
   mc.thr = p.thr;
   const bool pot_flush = MAP == MAP_POT && p.flush;
+
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush &&
                            p.fixed_window;
   // the four groups build interleaved entries of this row's grid table
@@ -465,16 +466,21 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
       } else {
         if (pot_flush) {
           if (full)
-            map_chunk<MAP, true, FP8, true>(v, mr, 32 * c, lim, false, z, pc);
+            map_chunk<MAP, true, FP8, true, false>(v, mr, 32 * c, lim, false, z, pc);
           else
-            map_chunk<MAP, false, FP8, true>(v, mr, 32 * c, lim, false, z, pc);
+            map_chunk<MAP, false, FP8, true, false>(v, mr, 32 * c, lim, false, z, pc);
+        } else if (KSAT) {
+          if (full)
+            map_chunk<MAP, true, FP8, false, true>(v, mr, 32 * c, lim, flush_below, z, pc);
+          else
+            map_chunk<MAP, false, FP8, false, true>(v, mr, 32 * c, lim, flush_below, z, pc);
         } else if (full) {
-          map_chunk<MAP, true, FP8, false>(v, mr, 32 * c, lim, flush_below, z, pc);
+          map_chunk<MAP, true, FP8, false, false>(v, mr, 32 * c, lim, flush_below, z, pc);
         } else {
-          map_chunk<MAP, false, FP8, false>(v, mr, 32 * c, lim, flush_below, z, pc);
+          map_chunk<MAP, false, FP8, false, false>(v, mr, 32 * c, lim, flush_below, z, pc);
         }
         if (p.dbg != nullptr)
-          debug_chunk<MAP>(dbg_row, v, mr, 128 * j + c_off + 32 * c, 32 * c, lim, p,
+          debug_chunk<MAP, KSAT>(dbg_row, v, mr, 128 * j + c_off + 32 * c, 32 * c, lim, p,
                            flush_below);
       }
     }
@@ -511,7 +517,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   }
 }
 
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 __global__ void __launch_bounds__(kThreads, 1)
     qsm_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -764,7 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(bars.drain, 0, abort);
   } else if (warp >= 4) {
     const int g = (warp - 4) >> 2;                 // map group 0..3
-    map_half<D, FP8, MAP>(p, bars, g, threadIdx.x - 128 - g * 128,
+    map_half<D, FP8, MAP, KSAT>(p, bars, g, threadIdx.x - 128 - g * 128,
                            tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh,
                            sTab, xc, abort);
   }
@@ -781,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 constexpr int kMaxDevices = 64;
 
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv) {
   using G = Geo<D, FP8>;
@@ -832,7 +838,7 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   if (smem < 120 * 1024) smem = 120 * 1024;
   if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
-  auto kern = qsm_fwd_kernel<D, FP8, MAP>;
+  auto kern = qsm_fwd_kernel<D, FP8, MAP, KSAT>;
   // Raising the kernel's dynamic shared memory limit is a driver round trip;
   // this instantiation remembers, per device, the largest limit already set.
   static std::atomic<int> smem_set[kMaxDevices];
@@ -860,12 +866,17 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
 template <int D, bool FP8>
 static qsm_status launch_d(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv) {
-  if (a.mode == QSM_MODE_EXACT) return launch_t<D, FP8, MAP_EXACT>(a, mq, mk, mv);
-  if (a.mode == QSM_MODE_ROWMAX_POT) return launch_t<D, FP8, MAP_POT>(a, mq, mk, mv);
-  if (a.mode == QSM_MODE_TRUNCATED) return launch_t<D, FP8, MAP_TRUNC>(a, mq, mk, mv);
-  if (a.mode == QSM_MODE_UNIFORM) return launch_t<D, FP8, MAP_UNIFORM>(a, mq, mk, mv);
-  if (a.rounding == QSM_ROUND_HARD) return launch_t<D, FP8, MAP_KI_HARD>(a, mq, mk, mv);
-  return launch_t<D, FP8, MAP_KI_INTERP>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_EXACT) return launch_t<D, FP8, MAP_EXACT, false>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_ROWMAX_POT) return launch_t<D, FP8, MAP_POT, false>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_TRUNCATED) return launch_t<D, FP8, MAP_TRUNC, false>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_UNIFORM) return launch_t<D, FP8, MAP_UNIFORM, false>(a, mq, mk, mv);
+  // K-interval: K a power of two takes the saturating coordinate (map_pair)
+  const bool p2 = k_pow2(a.Kint);
+  if (a.rounding == QSM_ROUND_HARD)
+    return p2 ? launch_t<D, FP8, MAP_KI_HARD, true>(a, mq, mk, mv)
+              : launch_t<D, FP8, MAP_KI_HARD, false>(a, mq, mk, mv);
+  return p2 ? launch_t<D, FP8, MAP_KI_INTERP, true>(a, mq, mk, mv)
+            : launch_t<D, FP8, MAP_KI_INTERP, false>(a, mq, mk, mv);
 }
 
 qsm_status launch_fwd(const FwdArgs &a) {

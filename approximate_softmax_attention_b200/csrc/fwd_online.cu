@@ -174,7 +174,7 @@ __device__ __forceinline__ float frame_factor(float from, float to) {
 // Weights of one 32-column chunk (masked), packed for the PV product and
 // stored into the buffer's columns c*16 (bf16) or c*8 (e4m3) -- columns this
 // thread has already read -- with the row sum accumulated.
-template <int MAP, bool FULL, bool FLUSH, bool FP8>
+template <int MAP, bool FULL, bool FLUSH, bool FP8, bool SAT = false>
 __device__ __forceinline__ void on_chunk(const uint32_t (&v)[32], const MapRow &mr, float cL2E,
                                          float fr, bool flush_below, int c0, int lim,
                                          float2 (&z)[4], uint32_t taddr) {
@@ -186,7 +186,7 @@ __device__ __forceinline__ void on_chunk(const uint32_t (&v)[32], const MapRow &
     } else if (MAP == MAP_POT) {
       x = map_pair<MAP_POT, FLUSH>(r, mr);
     } else {
-      x = pair_weights<MAP, false>(r, mr, flush_below);
+      x = pair_weights<MAP, false, SAT>(r, mr, flush_below);
       x = make_float2(__fmul_rn(x.x, fr), __fmul_rn(x.y, fr));
     }
     if (!FULL) {
@@ -322,7 +322,7 @@ __device__ __forceinline__ void on_anchor(const OnParams &p, const OnBars &bars,
 // One map warpgroup.  Thread `row` owns query row qi*128 + row (TMEM lane
 // `row`) and maps key tiles j = g, g + 3, ... in S buffer g against the
 // anchor and frame the anchor group published for the tile.
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, const OnRows &rs,
                                        int g, int row, uint32_t lane_base, int qi, int n, int bh,
                                        float *tab, volatile int *abort) {
@@ -332,6 +332,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   const int L = p.causal ? min(qrow + 1, p.S) : p.S;
   const bool flush_below = (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && p.flush;
   const bool pot_flush = MAP == MAP_POT && p.flush;
+
   bool ok = true;
 
   MapCall mc;
@@ -409,6 +410,11 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
           on_chunk<MAP, true, true, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
         else
           on_chunk<MAP, false, true, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
+      } else if (KSAT) {
+        if (full)
+          on_chunk<MAP, true, false, FP8, true>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
+        else
+          on_chunk<MAP, false, false, FP8, true>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
       } else if (full) {
         on_chunk<MAP, true, false, FP8>(v, mr, p.cL2E, fr, flush_below, 32 * c, lim, z, pc);
       } else {
@@ -420,7 +426,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
           const int kv = 128 * j + 32 * c + i;
           if (kv < p.S) {
             const float r = __uint_as_float(v[i]);
-            int d = map_raw_index<MAP>(r, mr, p.flush != 0, p.pot_floor);
+            int d = map_raw_index<MAP, KSAT>(r, mr, p.flush != 0, p.pot_floor);
             if (flush_below && __fmaf_rn(r, mr.a, mr.b) < 0.0f) d = -2;
             dbg_row[kv] = static_cast<int8_t>((32 * c + i < lim) ? d : -1);
           }
@@ -474,7 +480,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   }
 }
 
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 __global__ void __launch_bounds__(kOnThreads, 1)
     qsm_fwd_online_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -680,7 +686,7 @@ __global__ void __launch_bounds__(kOnThreads, 1)
                       tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, abort);
   } else if (warp >= 8) {
     const int g = (warp - 8) >> 2;
-    on_map<D, FP8, MAP>(p, bars, rs, g, threadIdx.x - 256 - g * 128,
+    on_map<D, FP8, MAP, KSAT>(p, bars, rs, g, threadIdx.x - 256 - g * 128,
                         tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh, sTab,
                         abort);
   }
@@ -695,7 +701,7 @@ __global__ void __launch_bounds__(kOnThreads, 1)
 
 constexpr int kMaxDevices = 64;
 
-template <int D, bool FP8, int MAP>
+template <int D, bool FP8, int MAP, bool KSAT>
 qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                        const CUtensorMap &mv) {
   using G = OGeo<D, FP8>;
@@ -751,7 +757,7 @@ qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMa
   if (smem < 120 * 1024) smem = 120 * 1024;            // one CTA per SM (all of TMEM)
   if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
-  auto kern = qsm_fwd_online_kernel<D, FP8, MAP>;
+  auto kern = qsm_fwd_online_kernel<D, FP8, MAP, KSAT>;
   static std::atomic<int> smem_set[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QSM_ERR_CUDA;
@@ -776,10 +782,15 @@ qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMa
 template <int D, bool FP8>
 qsm_status launch_on_d(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                        const CUtensorMap &mv) {
-  if (a.mode == QSM_MODE_EXACT) return launch_on_t<D, FP8, MAP_EXACT>(a, mq, mk, mv);
-  if (a.mode == QSM_MODE_ROWMAX_POT) return launch_on_t<D, FP8, MAP_POT>(a, mq, mk, mv);
-  if (a.rounding == QSM_ROUND_HARD) return launch_on_t<D, FP8, MAP_KI_HARD>(a, mq, mk, mv);
-  return launch_on_t<D, FP8, MAP_KI_INTERP>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_EXACT) return launch_on_t<D, FP8, MAP_EXACT, false>(a, mq, mk, mv);
+  if (a.mode == QSM_MODE_ROWMAX_POT) return launch_on_t<D, FP8, MAP_POT, false>(a, mq, mk, mv);
+  // K-interval: K a power of two takes the saturating coordinate (map_pair)
+  const bool p2 = k_pow2(a.Kint);
+  if (a.rounding == QSM_ROUND_HARD)
+    return p2 ? launch_on_t<D, FP8, MAP_KI_HARD, true>(a, mq, mk, mv)
+              : launch_on_t<D, FP8, MAP_KI_HARD, false>(a, mq, mk, mv);
+  return p2 ? launch_on_t<D, FP8, MAP_KI_INTERP, true>(a, mq, mk, mv)
+            : launch_on_t<D, FP8, MAP_KI_INTERP, false>(a, mq, mk, mv);
 }
 
 }  // namespace

@@ -137,6 +137,11 @@ __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return f2_from(r);
 }
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return f2_from(r);
+}
 __device__ __forceinline__ float2 add2_rd(float2 a, float2 b) {
   uint64_t r;
   asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_bits(a)), "l"(f2_bits(b)));
@@ -165,7 +170,8 @@ __device__ __forceinline__ float min3n(float a, float b, float c) {
 //               pre-multiplied by pscale)
 //   exact:      x = fma(r, c*log2e, -mL2E), w = 2^x
 struct MapRow {
-  float a, b;        // coordinate = fma(r, a, b)
+  float a, b;        // coordinate = fma(r, a, b) (K-interval, K = 2^m: both / K)
+  float mk;          // K-interval, K = 2^m: 1.5 * 2^23 / K
   float cap, Kf, Km1;
   float flush_t;     // PoT flush: kMagic + floor (t above it: exponent past the floor)
   float mL2E;        // exact map: the anchor rmax * c * log2e
@@ -186,10 +192,15 @@ struct MapCall {
   float thr;        // probes: the support threshold -(T * log2e)
 };
 
+// K a power of two: the K-interval coordinate can be formed already divided
+// by K and clamped by one saturating FMA (see map_pair).
+__host__ __device__ constexpr bool k_pow2(int K) { return K > 0 && (K & (K - 1)) == 0; }
+
 // Grid table layout: node n of the row in table column `row` (0..127) sits at
 // float offset n*128 + row (hard rounding: g_n * pscale) or float2 offset
-// n*128 + row (interpolation: (c_n, d_n) * pscale), n = 0..K.  Bytes needed:
-// (K+1) * 128 * 4 (hard) or * 8 (interpolation).
+// n*128 + row (interpolation: (c_n, d_n) * pscale, d_n further times K when
+// K is a power of two), n = 0..K.  Bytes needed: (K+1) * 128 * 4 (hard) or
+// * 8 (interpolation).
 __host__ __device__ constexpr int table_bytes_for(int map, int K) {
   return map == MAP_KI_HARD ? (K + 1) * 128 * 4 : (map == MAP_KI_INTERP ? (K + 1) * 128 * 8 : 0);
 }
@@ -203,6 +214,7 @@ __device__ __forceinline__ MapRow row_setup(const MapCall &mc, float rmax, float
                                             int row, int n0, int nstep, float &hi, float &lo) {
   MapRow mr;
   mr.a = mr.b = 0.0f;
+  mr.mk = kMagic;
   mr.cap = static_cast<float>(mc.flush ? mc.pot_floor + 1 : mc.pot_floor);
   mr.Kf = static_cast<float>(mc.K);
   mr.Km1 = static_cast<float>(mc.K - 1);
@@ -232,33 +244,68 @@ __device__ __forceinline__ MapRow row_setup(const MapCall &mc, float rmax, float
     mr.b = mr.Kf;
   }
   lo = rm.lo;
+  // K = 2^m: the coordinate is kept divided by K (a / K and b / K are exact;
+  // its sign, which the below-window flush tests, is unchanged), and 1.5 *
+  // 2^23 / K has a unit in the last place of exactly 1 / K over [M/K, M/K + 1]
+  const bool sat = k_pow2(mc.K);
+  const float invK = sat ? 1.0f / mr.Kf : 1.0f;
+  mr.a = __fmul_rn(mr.a, invK);
+  mr.b = __fmul_rn(mr.b, invK);
+  mr.mk = __fmul_rn(kMagic, invK);
+  const uint32_t mkbits = __float_as_uint(mr.mk);
   const uint32_t tb = smem_u32(tab);
   if (MAP == MAP_KI_HARD) {
     for (int nn = n0; nn <= mc.K; nn += nstep)
       tab[nn * 128 + row] = __fmul_rn(grid_value(rm, mc.K, nn), mc.pscale);
-    // bits(rne(u) + kMagic) = kMagicBits + n  ->  table row n
-    mr.tab = tb + row * 4 - kMagicBits * 512u;
+    // bits(rne(u) + kMagic) = kMagicBits + n  ->  table row n (scaled:
+    // bits(rne(u)/K + M/K) = bits(M/K) + n)
+    mr.tab = tb + row * 4 - (sat ? mkbits : kMagicBits) * 512u;
   } else {
     // entries k = 0 .. K: (c_k, d_k) with d_k = g_{k+1} - g_k and
-    // c_k = g_k - k d_k; entry K repeats entry K - 1
+    // c_k = g_k - k d_k; entry K repeats entry K - 1.  K a power of two:
+    // d_k is stored times K (exact), for w = (u/K) (K d_k) + c_k
     for (int nn = n0; nn <= mc.K; nn += nstep) {
       const int k = nn < mc.K ? nn : mc.K - 1;
       const float gk = grid_value(rm, mc.K, k);
       const float gk1 = grid_value(rm, mc.K, k + 1);
       const float d = __fmul_rn(__fsub_rn(gk1, gk), mc.pscale);
       tab[(nn * 128 + row) * 2 + 0] = __fmaf_rn(-static_cast<float>(k), d, __fmul_rn(gk, mc.pscale));
-      tab[(nn * 128 + row) * 2 + 1] = d;
+      tab[(nn * 128 + row) * 2 + 1] = sat ? __fmul_rn(d, mr.Kf) : d;
     }
-    // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k
-    mr.tab = tb + row * 8 - 0x4B000000u * 1024u;
+    // floor bits: bits(2^23 + k) = 0x4B000000 + k  ->  table row k (scaled:
+    // bits(floor_K(u/K) + M/K) = bits(M/K) + k)
+    mr.tab = tb + row * 8 - (sat ? mkbits : 0x4B000000u) * 1024u;
   }
   return mr;
 }
 
+// fma with the result clamped to [0, 1] (NaN gives 0), one instruction.
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  return __saturatef(__fmaf_rn(a, b, c));
+}
+
 // Weights of two scores (the map's arithmetic on a pair; FLUSH: Rowmax-PoT
 // with the below-floor policy "flush", exponents above the floor give 0).
-template <int MAP, bool FLUSH>
+// SAT (K-interval, K = 2^m, the row set up for it): the clamped coordinate
+// is formed as v = sat(fma(r, a/K, b/K)) = clamp(u, 0, K) / K, exactly
+// (scaling by a power of two commutes with rounding), so the node index,
+// the rounding and the interpolated weight are bit-identical to the unscaled
+// form's, for one instruction instead of an FMA and two clamps.  Callers
+// take SAT exactly when k_pow2(K), as row_setup does.
+template <int MAP, bool FLUSH, bool SAT = false>
 __device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
+  if ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && SAT) {
+    const float2 v = make_float2(fma_sat(r.x, m.a, m.b), fma_sat(r.y, m.a, m.b));
+    if (MAP == MAP_KI_HARD) {
+      const float2 t = add2_rn(v, make_float2(m.mk, m.mk));
+      return make_float2(lds_f32(__float_as_uint(t.x) * 512u + m.tab),
+                         lds_f32(__float_as_uint(t.y) * 512u + m.tab));
+    }
+    const float2 t = add2_rd(v, make_float2(m.mk, m.mk));
+    const float2 c0 = lds_f32x2(__float_as_uint(t.x) * 1024u + m.tab);
+    const float2 c1 = lds_f32x2(__float_as_uint(t.y) * 1024u + m.tab);
+    return make_float2(__fmaf_rn(v.x, c0.y, c0.x), __fmaf_rn(v.y, c1.y, c1.x));
+  }
   const float2 x = fma2_rn(r, make_float2(m.a, m.a), make_float2(m.b, m.b));
   if (MAP == MAP_TRUNC || MAP == MAP_UNIFORM) {
     float2 w = (MAP == MAP_TRUNC) ? make_float2(ex2_approx(x.x), ex2_approx(x.y))
@@ -302,9 +349,9 @@ __device__ __forceinline__ float2 map_pair(float2 r, const MapRow &m) {
 
 // Weights of a pair with the K-interval fixed-window flush (coordinate below
 // the window -> 0) applied when flush_below.
-template <int MAP, bool FLUSH>
+template <int MAP, bool FLUSH, bool SAT = false>
 __device__ __forceinline__ float2 pair_weights(float2 r, const MapRow &m, bool flush_below) {
-  float2 w = map_pair<MAP, FLUSH>(r, m);
+  float2 w = map_pair<MAP, FLUSH, SAT>(r, m);
   if (MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) {
     if (flush_below) {
       if (__fmaf_rn(r.x, m.a, m.b) < 0.0f) w.x = 0.0f;
@@ -323,7 +370,7 @@ __device__ __forceinline__ float2 exact_pair(float2 r, float cL2E, float mL2E) {
 // Decision index of one element (debug dump and the standalone map; the same
 // arithmetic as map_pair): PoT exponent (-2 flushed), hard node, lower node of
 // the interpolation, 0 for the exact map.
-template <int MAP>
+template <int MAP, bool SAT = false>
 __device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flush, int N) {
   if (MAP == MAP_EXACT) return 0;
   const float x = __fmaf_rn(r, m.a, m.b);
@@ -332,6 +379,14 @@ __device__ __forceinline__ int map_raw_index(float r, const MapRow &m, bool flus
     const int n = static_cast<int>(__float_as_uint(__fadd_rn(fminf(x, m.cap), kMagic)) -
                                    kMagicBits);
     return (flush && n > N) ? -2 : n;
+  }
+  if (SAT) {
+    // the row was set up with the coordinate divided by K (map_pair's SAT)
+    const float v = fma_sat(r, m.a, m.b);
+    const uint32_t mb = __float_as_uint(m.mk);
+    if (MAP == MAP_KI_HARD) return static_cast<int>(__float_as_uint(__fadd_rn(v, m.mk)) - mb);
+    return min(static_cast<int>(__float_as_uint(__fadd_rd(v, m.mk)) - mb),
+               static_cast<int>(m.Km1));
   }
   const float uc = fminf(fmaxf(x, 0.0f), m.Kf);
   if (MAP == MAP_KI_HARD)

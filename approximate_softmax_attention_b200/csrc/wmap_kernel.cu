@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kRowsPerBlock)
     float2 wt;
     if (MAP == MAP_EXACT)
       wt = exact_pair(x, mc.cL2E, mr.mL2E);
+    else if ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && k_pow2(mc.K))
+      wt = pair_weights<MAP, FLUSH, true>(x, mr, flush_below);   // as the fused forward
     else
       wt = pair_weights<MAP, FLUSH>(x, mr, flush_below);
     wr[j] = v0 ? wt.x : 0.0f;
@@ -59,7 +61,9 @@ __global__ void __launch_bounds__(kRowsPerBlock)
     if (ir) {
       for (int e = 0; e < 2 && j + e < cols; ++e) {
         const float xe = e ? x.y : x.x;
-        int n = map_raw_index<MAP>(xe, mr, mc.flush != 0, mc.pot_floor);
+        int n = ((MAP == MAP_KI_HARD || MAP == MAP_KI_INTERP) && k_pow2(mc.K))
+                    ? map_raw_index<MAP, true>(xe, mr, mc.flush != 0, mc.pot_floor)
+                    : map_raw_index<MAP, false>(xe, mr, mc.flush != 0, mc.pot_floor);
         if (flush_below && __fmaf_rn(xe, mr.a, mr.b) < 0.0f) n = -2;
         ir[j + e] = (j + e < L) ? n : -1;
       }

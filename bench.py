@@ -230,10 +230,68 @@ class ClockSampler:
                 "samples": len(sm), "power_w_median": statistics.median(pw) if pw else None}
 
 
+KERNEL_HEADERS = ("wmap.cuh", "sm100.cuh", "internal.h")
+
+
 def source_sha(name):
-    """sha256 prefix of a kernel source file (the key of the traffic records)."""
-    with open(os.path.join(CSRC, name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 prefix of a kernel source file and the headers it includes (the
+    key of the traffic records)."""
+    h = hashlib.sha256()
+    for n in (name,) + KERNEL_HEADERS:
+        with open(os.path.join(CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def record_traffic(csv_path, workload):
+    """Write the DRAM bytes of one forward step into the traffic records
+    (profiles/fwd_traffic.json), from an ncu CSV of `bench.py --part fwd
+    --workload W` that captured exactly one step's launches (-s warmup*n -c n)
+    with dram__bytes_read.sum, dram__bytes_write.sum, gpu__time_duration.sum.
+    Entries of other workloads are kept only while their kernel sources are
+    unchanged."""
+    import csv
+    import io
+    from approximate_softmax_attention_b200 import inputs
+    names = HEADLINE.get(workload, (workload,))
+    order = [(w.name, mode_label(m)) for w in (inputs.WORKLOADS[n] for n in names)
+             for m in step_maps(w)]
+    txt = open(csv_path).read()
+    rows = list(csv.DictReader(io.StringIO(txt[txt.find('"ID"'):])))
+    per = {}
+    for r in rows:
+        d = per.setdefault(int(r["ID"]), {"kernel": r["Kernel Name"]})
+        d[r["Metric Name"]] = float(r["Metric Value"].replace(",", ""))
+    launches = [per[i] for i in sorted(per)]
+    if len(launches) != len(order):
+        raise SystemExit("expected %d launches (one step), found %d" % (len(order), len(launches)))
+    srcs = {n: source_sha(n) for n in ("fwd.cu", "fwd_online.cu")}
+    old = {}
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            old = json.load(f)
+    keep = {}
+    if old.get("sources") == srcs:
+        keep = {k: v for k, v in old.get("entries", {}).items()
+                if not any(k.startswith(n + "/") for n in names)}
+    for (wname, label), d in zip(order, launches):
+        online = label.endswith("_online")
+        if ("qsm_fwd_online_kernel" in d["kernel"]) != online:
+            raise SystemExit("launch order does not match the step: %s vs %s" % (label, d["kernel"]))
+        rd, wr = d["dram__bytes_read.sum"], d["dram__bytes_write.sum"]
+        keep["%s/%s" % (wname, label)] = {
+            "dram_bytes_per_launch": int(rd + wr), "dram_read": int(rd), "dram_write": int(wr),
+            "ncu_duration_ns": int(d["gpu__time_duration.sum"])}
+    out = {"sources": srcs,
+           "source": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,"
+                     "gpu__time_duration.sum --clock-control none -k regex:qsm_fwd -s <warm-up "
+                     "launches> -c <one step> on python bench.py --part fwd --workload <W> "
+                     "--steps 1 --warmup <w>; recorded by bench.py --record-traffic",
+           "entries": dict(sorted(keep.items()))}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(out, f, indent=1)
+        f.write("\n")
+    print("recorded %d launches of %s into %s" % (len(order), workload, TRAFFIC_FILE))
 
 
 def traffic_for(workload_name, label):
@@ -405,7 +463,8 @@ def map_entry(w, ms, pk):
 
 def roofline_of(w, label, entry, pk):
     burst, sust, src = pk[dtype_name(w)]
-    return {"bound": "tensor", "kernel": "qsm_fwd_kernel (%s, %s)" % (w.name, label),
+    kern = "qsm_fwd_online_kernel" if label.endswith("_online") else "qsm_fwd_kernel"
+    return {"bound": "tensor", "kernel": "%s (%s, %s)" % (kern, w.name, label),
             "achieved": entry["tflops"], "peak": round(burst, 1), "unit": "TFLOP/s",
             "frac": round(entry["tflops"] / burst, 4),
             "peak_sustained": round(sust, 1),
@@ -726,12 +785,17 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=100.0)
     ap.add_argument("--bwd-reps", type=int, default=10)
+    ap.add_argument("--record-traffic", metavar="CSV", default=None,
+                    help="write an ncu DRAM capture of one --part fwd step of --workload into "
+                         "the traffic records and exit (no GPU needed)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.part != "all":
         args.no_e2e = args.no_energy = args.no_cpu_baseline = True
-    if args.impl == "reference":
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.workload)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -35,7 +35,7 @@ def _gpu(x):
 # ------------------------------------------------------------ weight map
 
 MAP_CASES = [(0, 4, 0, 1, 0), (2, 4, 0, 1, 0), (2, 4, 0, 1, 1), (3, 4, 0, 1, 0), (4, 4, 0, 1, 0)] + \
-    [(1, K, c, r, 0) for K in (1, 4, 16, 64) for c in (0, 1) for r in (0, 1)] + \
+    [(1, K, c, r, 0) for K in (1, 3, 4, 12, 16, 64) for c in (0, 1) for r in (0, 1)] + \
     [(1, 4, 1, 1, 1), (1, 16, 1, 0, 1)]
 
 # (scale, q_descale, k_descale) as the forward forms c = scale * qd * kd
@@ -206,11 +206,12 @@ def test_fwd_below_policy(below):
 
 @pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "bf16"), (128, "fp8")])
 @pytest.mark.parametrize("K,calib,rounding", [(1, 0, 0), (1, 1, 1), (64, 0, 0), (64, 1, 0),
-                                              (64, 0, 1)])
+                                              (64, 0, 1), (12, 0, 0), (12, 1, 1)])
 def test_fwd_kinterval_extreme_K(D, dtype, K, calib, rounding):
-    """K-interval with K = 1 (the interpolation table is one segment) and
+    """K-interval with K = 1 (the interpolation table is one segment),
     K = 64 (the largest K the forward accepts; its interpolation table leaves
-    the bf16 D = 128 ring three shared-memory stages), causal, ragged S."""
+    the bf16 D = 128 ring three shared-memory stages) and K = 12 (not a power
+    of two: the unscaled clamp path), causal, ragged S."""
     S = 330
     d = inputs.draw(1, 2, S, D, seed=50 + K + D, peaked=True, dtype=dtype)
     got = _run_fwd(d, True, 1, K, calib, rounding, window=6.0, debug=True)

@@ -137,7 +137,8 @@ def _compare(d, got, ref, causal, mode, tol_max, tol_mean, heads=None, rows=None
 
 
 ONLINE_MAPS = [(A.EXACT, 4, 1), (A.ROWMAX_POT, 4, 1), (A.KINTERVAL, 4, A.HARD),
-               (A.KINTERVAL, 16, A.INTERP), (A.KINTERVAL, 4, A.INTERP)]
+               (A.KINTERVAL, 16, A.INTERP), (A.KINTERVAL, 4, A.INTERP),
+               (A.KINTERVAL, 12, A.INTERP), (A.KINTERVAL, 6, A.HARD)]
 
 
 @pytest.mark.parametrize("S,D,causal", [(1, 64, False), (77, 64, True), (200, 128, False),
