@@ -59,6 +59,10 @@ namespace {
 // warp 0 TMA, warps 1-2 MMA, warps 4-19 four map groups of 128 threads
 constexpr int kMainThreads = 640;
 constexpr int kMainMapThreads = 512;
+// The dQ and dK/dV passes keep three halves in flight (TMEM buffers, and dS
+// tiles in the dQ pass): a buffer's round trip through the products that
+// read it and refill it overlaps the map of the two halves in between.
+constexpr int kHalfBufs = 3;
 constexpr uint32_t kBwdTmemCols = 512;
 constexpr int kRowWs = 8;               // floats per row in the row workspace
 enum RowWs { RW_LSESTAR = 0, RW_DELTASTAR = 1 };
@@ -591,18 +595,18 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
 // ----------------------------------------------------------------- dQ pass
 // One CTA per 128-row query tile of one (b, h); thread = query row (TMEM
 // lane); the key tiles are taken in halves of 64 keys, half h in TMEM pair
-// x = h & 1 (S at 128x, dP at 128x + 64) and shared dS buffer x; map group g
-// owns keys 16g .. 16g+15 of each half.  dQ accumulates at TMEM column 256.
+// x = h mod 3 (S at 128x, dP at 128x + 64) and shared dS buffer x; map group
+// g owns keys 16g .. 16g+15 of each half.  dQ accumulates at TMEM column 384.
 struct DqBars {
   uint64_t *kv_full, *kv_empty;       // [ns]: K_j, V_j
   uint64_t *q_full;                   // Q, dO
-  uint64_t *sdp_full, *sdp_free;      // [2]
-  uint64_t *ds_full, *ds_free;        // [2]
+  uint64_t *sdp_full, *sdp_free;      // [kHalfBufs]
+  uint64_t *ds_full, *ds_free;        // [kHalfBufs]
   uint64_t *dq_full, *tab_ready, *part_ready, *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr uint32_t T_DQ = 256;
+constexpr uint32_t T_DQ = 384;
 
 template <int D, int MAP, int SURR, int CAL>
 __global__ void __launch_bounds__(kMainThreads, 1)
@@ -621,7 +625,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages of (K_j, V_j)
-  uint8_t *sDS = smem + p.ds_off;                        // 2 x 128 rows x 128 bytes
+  uint8_t *sDS = smem + p.ds_off;                        // 3 x 128 rows x 128 bytes
   float *part = reinterpret_cast<float *>(smem + p.part_off);   // [3][4][128]
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   DqBars bars;
@@ -629,10 +633,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.kv_empty = bp + ns;
   bars.q_full = bp + 2 * ns;
   bars.sdp_full = bars.q_full + 1;
-  bars.sdp_free = bars.sdp_full + 2;
-  bars.ds_full = bars.sdp_free + 2;
-  bars.ds_free = bars.ds_full + 2;
-  bars.dq_full = bars.ds_free + 2;
+  bars.sdp_free = bars.sdp_full + kHalfBufs;
+  bars.ds_full = bars.sdp_free + kHalfBufs;
+  bars.ds_free = bars.ds_full + kHalfBufs;
+  bars.dq_full = bars.ds_free + kHalfBufs;
   bars.tab_ready = bars.dq_full + 1;
   bars.part_ready = bars.tab_ready + 1;
   bars.drain = bars.part_ready + 1;
@@ -648,7 +652,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.kv_empty[i], 1);
     }
     mbar_init(bars.q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kHalfBufs; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.sdp_free[i], kMainMapThreads);
       mbar_init(&bars.ds_full[i], kMainMapThreads);
@@ -693,20 +697,20 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_wait(&bars.kv_full[st], (((nkv - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair h & 1
+    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair h mod 3
     if (lane == 0) {
       bool ok = mbar_wait(bars.q_full, 0, abort);
       tc_fence_after();
       const uint32_t qa = smem_u32(sQ), da = smem_u32(sdO), kva = smem_u32(sKV);
       for (int h = 0; h < nh && ok; ++h) {
-        const int j = h >> 1, e = h & 1, x = h & 1;
+        const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
         if (e == 0) {
           ok = mbar_wait(&bars.kv_full[j % ns], (j / ns) & 1, abort);
           if (!ok) break;
           tc_fence_after();
         }
-        if (h >= 2) {
-          ok = mbar_wait(&bars.sdp_free[x], ((h >> 1) - 1) & 1, abort);
+        if (u >= 1) {
+          ok = mbar_wait(&bars.sdp_free[x], (u - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
         }
@@ -724,14 +728,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       const uint32_t kva = smem_u32(sKV), dsa = smem_u32(sDS);
       for (int h = 0; h < nh && ok; ++h) {
-        const int j = h >> 1, e = h & 1, x = h & 1;
+        const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
         if (e == 0) {
           // K_j has landed (this warp reads it too; the stage cannot refill
           // before this warp's own release below)
           ok = mbar_wait(&bars.kv_full[j % ns], (j / ns) & 1, abort);
           if (!ok) break;
         }
-        ok = mbar_wait(&bars.ds_full[x], (h >> 1) & 1, abort);
+        ok = mbar_wait(&bars.ds_full[x], u & 1, abort);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kb = kva + (j % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
@@ -795,8 +799,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
     const uint32_t dsb = smem_u32(sDS);
     for (int h = 0; h < nh && ok; ++h) {
-      const int j = h >> 1, e = h & 1, x = h & 1;
-      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], (h >> 1) & 1, abort));
+      const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
+      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
       if (!ok) break;
       tc_fence_after();
       uint32_t sv[16], dv[16];
@@ -806,15 +810,16 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       reg_fence16(sv);
       reg_fence16(dv);
       tc_fence_before();
-      mbar_arrive(&bars.sdp_free[x]);                  // the pair can take half h + 2
+      mbar_arrive(&bars.sdp_free[x]);                  // the pair can take half h + 3
       const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
       uint32_t dd[8];
       if (warp_all_b(lim >= 16))
         dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
       else
         dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
-      if (h >= 2) {
-        ok = warp_all_b(mbar_wait(&bars.ds_free[x], ((h >> 1) - 1) & 1, abort));
+      if (u >= 1) {
+        // the dQ product of half h - 3 has read dS buffer x
+        ok = warp_all_b(mbar_wait(&bars.ds_free[x], (u - 1) & 1, abort));
         if (!ok) break;
       }
       // dS row-major (K-major operand), 128-byte swizzle: this group's 16
@@ -907,20 +912,21 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 
 // --------------------------------------------------------------- dK/dV pass
 // One CTA per 128-key tile of one (b, h); thread = key (TMEM lane); the
-// query tiles are taken in halves of 64 rows, half h in TMEM pair x = h & 1
-// (S^T at 128x, dP^T at 128x + 64); map group g owns queries 16g .. 16g+15 of
+// query tiles are taken in halves of 64 rows, half h in TMEM pair x = h mod 3
+// (S^T at 128x, dP^T at 128x + 64); map group g owns rows 16g .. 16g+15 of
 // each half and writes its P^T and dS^T (bf16) into the first 8 of its own 16
-// columns, which the dV / dK products read as their TMEM A operand.  A ring
-// stage holds Q_i, dO_i and the tile's per-row constants and grid tables.
+// columns, which the dV / dK products (dV at TMEM column 384, dK at 448) read
+// as their TMEM A operand.  A ring stage holds Q_i, dO_i and the tile's
+// per-row constants and grid tables.
 struct KvBars {
   uint64_t *qd_full, *qd_empty;       // [ns]
   uint64_t *kv_full;                  // K, V once
-  uint64_t *sdp_full, *pds_full, *s_free;   // [2]
+  uint64_t *sdp_full, *pds_full, *s_free;   // [kHalfBufs]
   uint64_t *acc_full, *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr uint32_t T_DV = 256, T_DK = 320;
+constexpr uint32_t T_DV = 384, T_DK = 448;
 
 // The dK / dV pass's per-thread values for the element loop.
 struct KvK {
@@ -1024,9 +1030,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.qd_empty = bp + ns;
   bars.kv_full = bp + 2 * ns;
   bars.sdp_full = bars.kv_full + 1;
-  bars.pds_full = bars.sdp_full + 2;
-  bars.s_free = bars.pds_full + 2;
-  bars.acc_full = bars.s_free + 2;
+  bars.pds_full = bars.sdp_full + kHalfBufs;
+  bars.s_free = bars.pds_full + kHalfBufs;
+  bars.acc_full = bars.s_free + kHalfBufs;
   bars.drain = bars.acc_full + 1;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
@@ -1041,7 +1047,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.qd_empty[i], 1);
     }
     mbar_init(bars.kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kHalfBufs; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.pds_full[i], kMainMapThreads);
       mbar_init(&bars.s_free[i], 1);
@@ -1089,21 +1095,21 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_wait(&bars.qd_full[st], (((nq - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair h & 1, once
-    // the dV / dK products of half h - 2 have read it
+    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair h mod 3,
+    // once the dV / dK products of half h - 3 have read it
     if (lane == 0) {
       bool ok = mbar_wait(bars.kv_full, 0, abort);
       tc_fence_after();
       const uint32_t ka = smem_u32(sK), va = smem_u32(sV), sa = smem_u32(sSt);
       for (int h = 0; h < nh && ok; ++h) {
-        const int n = h >> 1, e = h & 1, x = h & 1;
+        const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
         if (e == 0) {
           ok = mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort);
           if (!ok) break;
           tc_fence_after();
         }
-        if (h >= 2) {
-          ok = mbar_wait(&bars.s_free[x], ((h >> 1) - 1) & 1, abort);
+        if (u >= 1) {
+          ok = mbar_wait(&bars.s_free[x], (u - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
         }
@@ -1121,12 +1127,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       const uint32_t sa = smem_u32(sSt);
       for (int h = 0; h < nh && ok; ++h) {
-        const int n = h >> 1, e = h & 1, x = h & 1;
+        const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
         if (e == 0) {
           ok = mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort);
           if (!ok) break;
         }
-        ok = mbar_wait(&bars.pds_full[x], (h >> 1) & 1, abort);
+        ok = mbar_wait(&bars.pds_full[x], u & 1, abort);
         if (!ok) break;
         tc_fence_after();
         const uint32_t qb = sa + (n % ns) * SB + e * 64 * 128;
@@ -1163,15 +1169,16 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), mod 2^32
     const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - kMagicBits * 8u : 0u - kMagicBits * 4u;
     bool ok = true;
+    const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
     for (int h = 0; h < nh && ok; ++h) {
-      const int n = h >> 1, e = h & 1, x = h & 1;
+      const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
       if (e == 0) {
         // the stage's constants and tables have landed (the stage cannot
         // refill before this tile's products, which wait for these threads)
         ok = warp_all_b(mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort));
         if (!ok) break;
       }
-      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], (h >> 1) & 1, abort));
+      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
       if (!ok) break;
       tc_fence_after();
       const uint32_t st = smem_u32(sSt + (n % ns) * SB);
@@ -1187,7 +1194,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       // lie at or below this key
       const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
       const uint32_t cb = st + CST_OFF + ql0 * (kCst * 4);
-      const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
       const uint32_t tr = st + TAB_OFF + ql0 * tsb + tbias;
       uint32_t pp[8], dd[8];
       if (full) {
@@ -1273,22 +1279,23 @@ bool set_smem_once(F kern, int bytes, std::atomic<int> (&cache)[kMaxDevices]) {
 }
 
 constexpr size_t kMaxSmem = 232448;                      // 227 KB opt-in per CTA
-constexpr size_t kBarBytes = ((2 * 8 + 16) * 8 + 8 + 15) & ~static_cast<size_t>(15);
+constexpr size_t kBarBytes = ((2 * 8 + 24) * 8 + 8 + 15) & ~static_cast<size_t>(15);
 
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  // Q, dO, ns x (K, V), 2 dS buffers, table, partial sums, barriers
+  // Q, dO, ns x (K, V), kHalfBufs dS buffers, table, partial sums, barriers
   const size_t tab = (DqTab<MAP, SURR, CAL>::bytes(p.K) + 15) & ~static_cast<size_t>(15);
   const size_t part = 3 * 4 * 128 * sizeof(float);
-  const size_t fixed = 1024 + 2 * G::TILE_BYTES + 2 * 128 * 128 + tab + part + kBarBytes;
+  const size_t fixed =
+      1024 + 2 * G::TILE_BYTES + kHalfBufs * 128 * 128 + tab + part + kBarBytes;
   int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
   if (ns > 4) ns = 4;
   if (ns < 2) return QSM_ERR_UNSUPPORTED;
   p.num_stages = ns;
   p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
-  p.tab_off = p.ds_off + 2 * 128 * 128;
+  p.tab_off = p.ds_off + kHalfBufs * 128 * 128;
   p.part_off = static_cast<uint32_t>(p.tab_off + tab);
   p.bar_off = static_cast<uint32_t>(p.part_off + part);
   size_t smem = 1024 + p.bar_off + kBarBytes;
