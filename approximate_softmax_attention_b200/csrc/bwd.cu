@@ -79,7 +79,7 @@ constexpr int CAL_OFF = 0, CAL_MINMAX = 1, CAL_FIXED = 2;
 struct BwdParams {
   int S, nqt, nkvt, BH;
   int causal;
-  int hgroup;       // causal query-tile order: heads per group (see q_tile_order)
+  int hgroup;       // causal query-tile order: heads per group (see q_tile_of)
   int K, fixed_window, flush, pot_floor;
   int TS;           // floats of one query row's dK / dV pass table (a multiple of 4)
   float c, cL2E, window;
@@ -137,11 +137,10 @@ __device__ __forceinline__ void mma_nt_half(uint32_t d_tmem, uint32_t a_saddr, u
   }
 }
 
-// The (head, query tile) of a query-tile CTA on a 1-D grid of nqt * BH:
-// non-causal head after head; causal in groups of hgroup heads (their K / V
-// share L2), heaviest tiles first within a group.
-__device__ __forceinline__ void q_tile_order(const BwdParams &p, int &bh, int &qt) {
-  const int b = static_cast<int>(blockIdx.x);
+// The (head, query tile) of query tile number b of nqt * BH: non-causal
+// head after head; causal in groups of hgroup heads (their K / V share L2),
+// heaviest tiles first within a group.
+__device__ __forceinline__ void q_tile_of(const BwdParams &p, int b, int &bh, int &qt) {
   if (p.causal) {
     const int per = p.hgroup * p.nqt;
     const int grp = b / per;
@@ -154,6 +153,24 @@ __device__ __forceinline__ void q_tile_order(const BwdParams &p, int &bh, int &q
   } else {
     qt = b % p.nqt;
     bh = b / p.nqt;
+  }
+}
+
+// The (head, key tile) of key tile number b of nkvt * BH: non-causal head
+// after head; causal in groups of hgroup heads, heaviest (lowest) key tiles
+// first within a group.
+__device__ __forceinline__ void kv_tile_of(const BwdParams &p, int b, int &bh, int &kt) {
+  if (p.causal) {
+    const int per = p.hgroup * p.nkvt;
+    const int grp = b / per;
+    const int within = b - grp * per;
+    const int h0 = grp * p.hgroup;
+    const int gh = min(p.hgroup, p.BH - h0);
+    kt = within / gh;
+    bh = h0 + (within - kt * gh);
+  } else {
+    kt = b % p.nkvt;
+    bh = b / p.nkvt;
   }
 }
 
@@ -171,8 +188,8 @@ __device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b, float acc) {
   return acc;
 }
 
-// Sixteen bf16 (two uint4) to fp32.
-__device__ __forceinline__ void bf16x16_to_f32(const uint4 *src, float (&x)[16]) {
+// Sixteen bf16 (two uint4, already loaded) to fp32.
+__device__ __forceinline__ void bf16x16_to_f32(const uint4 (&src)[2], float (&x)[16]) {
   const uint4 a = src[0], b = src[1];
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -208,7 +225,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int bh, qt;
-  q_tile_order(p, bh, qt);
+  q_tile_of(p, static_cast<int>(blockIdx.x), bh, qt);
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;
@@ -593,16 +610,20 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
 }
 
 // ----------------------------------------------------------------- dQ pass
-// One CTA per 128-row query tile of one (b, h); thread = query row (TMEM
-// lane); the key tiles are taken in halves of 64 keys, half h in TMEM pair
-// x = h mod 3 (S at 128x, dP at 128x + 64) and shared dS buffer x; map group
-// g owns keys 16g .. 16g+15 of each half.  dQ accumulates at TMEM column 384.
+// Persistent: one CTA per SM takes the 128-row query tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ... in the heaviest-first order; thread = query row
+// (TMEM lane); the key tiles are taken in halves of 64 keys, half number hc
+// (counted across tiles) in TMEM pair x = hc mod 3 (S at 128x, dP at 128x +
+// 64) and shared dS buffer x; map group g owns keys 16g .. 16g+15 of each
+// half.  dQ accumulates at TMEM column 384 and is read out before the next
+// tile's first dQ product.
 struct DqBars {
   uint64_t *kv_full, *kv_empty;       // [ns]: K_j, V_j
-  uint64_t *q_full;                   // Q, dO
+  uint64_t *q_full, *q_free;          // Q, dO of the current tile
   uint64_t *sdp_full, *sdp_free;      // [kHalfBufs]
   uint64_t *ds_full, *ds_free;        // [kHalfBufs]
-  uint64_t *dq_full, *tab_ready, *part_ready, *drain;
+  uint64_t *dq_full, *dq_free;        // the tile's dQ complete / read out of TMEM
+  uint64_t *tab_ready, *part_ready, *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
@@ -619,8 +640,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int bh, qt;
-  q_tile_order(p, bh, qt);
+  const int ntiles = p.nqt * p.BH;
+  const int step = static_cast<int>(gridDim.x);
   const int ns = p.num_stages;
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
@@ -632,19 +653,19 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.kv_full = bp;
   bars.kv_empty = bp + ns;
   bars.q_full = bp + 2 * ns;
-  bars.sdp_full = bars.q_full + 1;
+  bars.q_free = bars.q_full + 1;
+  bars.sdp_full = bars.q_free + 1;
   bars.sdp_free = bars.sdp_full + kHalfBufs;
   bars.ds_full = bars.sdp_free + kHalfBufs;
   bars.ds_free = bars.ds_full + kHalfBufs;
   bars.dq_full = bars.ds_free + kHalfBufs;
-  bars.tab_ready = bars.dq_full + 1;
+  bars.dq_free = bars.dq_full + 1;
+  bars.tab_ready = bars.dq_free + 1;
   bars.part_ready = bars.tab_ready + 1;
   bars.drain = bars.part_ready + 1;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
-  const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
-  const int nh = 2 * nkv;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
@@ -652,6 +673,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.kv_empty[i], 1);
     }
     mbar_init(bars.q_full, 1);
+    mbar_init(bars.q_free, 1);
     for (int i = 0; i < kHalfBufs; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.sdp_free[i], kMainMapThreads);
@@ -659,6 +681,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.ds_free[i], 1);
     }
     mbar_init(bars.dq_full, 1);
+    mbar_init(bars.dq_free, kMainMapThreads);
     mbar_init(bars.tab_ready, kMainMapThreads);
     mbar_init(bars.part_ready, kMainMapThreads);
     mbar_init(bars.drain, 2);
@@ -671,53 +694,79 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
+  // Tiles of this CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ... of the
+  // heaviest-first order (persistent: the next tile's loads and first
+  // products overlap this tile's epilogue).  Every role walks the same
+  // sequence; the ring position `it` and the half counter `hc` run on across
+  // tiles, and per-tile barriers take the tile's own parity k & 1.
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(bars.q_full, 2 * G::TILE_BYTES);
-      for (int ch = 0; ch < G::CHUNKS; ++ch) {
-        tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qt * 128, bh);
-        tma_load_3d(sdO + ch * G::CHUNK_BYTES, &tmdO, bars.q_full, ch * G::EPC, qt * 128, bh);
-      }
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j % ns;
-        if (j >= ns) ok = mbar_wait(&bars.kv_empty[st], ((j / ns) - 1) & 1, abort);
+      int it = 0, k = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        // Q, dO of the previous tile are no longer read
+        if (k >= 1) ok = mbar_wait(bars.q_free, (k - 1) & 1, abort);
         if (!ok) break;
-        uint8_t *kdst = sKV + st * 2 * G::TILE_BYTES;
-        mbar_expect_tx(&bars.kv_full[st], 2 * G::TILE_BYTES);
+        mbar_expect_tx(bars.q_full, 2 * G::TILE_BYTES);
         for (int ch = 0; ch < G::CHUNKS; ++ch) {
-          tma_load_3d(kdst + ch * G::CHUNK_BYTES, &tmK, &bars.kv_full[st], ch * G::EPC, j * 128, bh);
-          tma_load_3d(kdst + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmV, &bars.kv_full[st],
-                      ch * G::EPC, j * 128, bh);
+          tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qt * 128, bh);
+          tma_load_3d(sdO + ch * G::CHUNK_BYTES, &tmdO, bars.q_full, ch * G::EPC, qt * 128, bh);
+        }
+        for (int j = 0; j < nkv && ok; ++j, ++it) {
+          const int st = it % ns;
+          if (it >= ns) ok = mbar_wait(&bars.kv_empty[st], ((it / ns) - 1) & 1, abort);
+          if (!ok) break;
+          uint8_t *kdst = sKV + st * 2 * G::TILE_BYTES;
+          mbar_expect_tx(&bars.kv_full[st], 2 * G::TILE_BYTES);
+          for (int ch = 0; ch < G::CHUNKS; ++ch) {
+            tma_load_3d(kdst + ch * G::CHUNK_BYTES, &tmK, &bars.kv_full[st], ch * G::EPC,
+                        j * 128, bh);
+            tma_load_3d(kdst + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmV, &bars.kv_full[st],
+                        ch * G::EPC, j * 128, bh);
+          }
         }
       }
-      // every load issued must land before the CTA may exit
-      mbar_wait(bars.q_full, 0, abort);
-      for (int st = 0; st < ns && st < nkv; ++st)
-        mbar_wait(&bars.kv_full[st], (((nkv - st + ns - 1) / ns) - 1) & 1, abort);
+      // every load issued must land before the CTA may exit: the last Q / dO
+      // load and the latest fill of each ring stage
+      if (k >= 1) mbar_wait(bars.q_full, (k - 1) & 1, abort);
+      for (int st = 0; st < ns && st < it; ++st)
+        mbar_wait(&bars.kv_full[st], (((it - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair h mod 3
+    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair hc mod 3
     if (lane == 0) {
-      bool ok = mbar_wait(bars.q_full, 0, abort);
-      tc_fence_after();
+      bool ok = true;
+      int it0 = 0, hc = 0, k = 0;
       const uint32_t qa = smem_u32(sQ), da = smem_u32(sdO), kva = smem_u32(sKV);
-      for (int h = 0; h < nh && ok; ++h) {
-        const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-        if (e == 0) {
-          ok = mbar_wait(&bars.kv_full[j % ns], (j / ns) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        ok = mbar_wait(bars.q_full, k & 1, abort);
+        tc_fence_after();
+        for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
+          const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+          const int itj = it0 + j;
+          if (e == 0) {
+            ok = mbar_wait(&bars.kv_full[itj % ns], (itj / ns) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (u >= 1) {
+            ok = mbar_wait(&bars.sdp_free[x], (u - 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint32_t kb = kva + (itj % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
+          mma_nt_half<D>(tmem + 128 * x, qa, kb);
+          mma_nt_half<D>(tmem + 128 * x + 64, da, kb + G::TILE_BYTES);
+          mma_commit(&bars.sdp_full[x]);
         }
-        if (u >= 1) {
-          ok = mbar_wait(&bars.sdp_free[x], (u - 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        const uint32_t kb = kva + (j % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
-        mma_nt_half<D>(tmem + 128 * x, qa, kb);
-        mma_nt_half<D>(tmem + 128 * x + 64, da, kb + G::TILE_BYTES);
-        mma_commit(&bars.sdp_full[x]);
+        if (ok) mma_commit(bars.q_free);                // the tile's Q, dO are read
+        it0 += nkv;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -726,29 +775,39 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // dQ += dS_h K_h (dS K-major in shared memory, K as an MN-major operand)
     if (lane == 0) {
       bool ok = true;
+      int it0 = 0, hc = 0, k = 0;
       const uint32_t kva = smem_u32(sKV), dsa = smem_u32(sDS);
-      for (int h = 0; h < nh && ok; ++h) {
-        const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-        if (e == 0) {
-          // K_j has landed (this warp reads it too; the stage cannot refill
-          // before this warp's own release below)
-          ok = mbar_wait(&bars.kv_full[j % ns], (j / ns) & 1, abort);
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
+          const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+          const int itj = it0 + j;
+          if (e == 0) {
+            // K_j has landed (this warp reads it too; the stage cannot refill
+            // before this warp's own release below)
+            ok = mbar_wait(&bars.kv_full[itj % ns], (itj / ns) & 1, abort);
+            if (!ok) break;
+          }
+          ok = mbar_wait(&bars.ds_full[x], u & 1, abort);
+          // the previous tile's dQ has been read out of TMEM
+          if (ok && h == 0 && k >= 1) ok = mbar_wait(bars.dq_free, (k - 1) & 1, abort);
           if (!ok) break;
-        }
-        ok = mbar_wait(&bars.ds_full[x], u & 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kb = kva + (j % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
-        const uint32_t ab = dsa + x * 128 * 128;
+          tc_fence_after();
+          const uint32_t kb = kva + (itj % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
+          const uint32_t ab = dsa + x * 128 * 128;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss_f16(tmem + T_DQ, smem_desc(ab + kk * 32, 16, 1024),
-                     smem_desc(kb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN,
-                     (h > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars.ds_free[x]);
-        if (e == 1) mma_commit(&bars.kv_empty[j % ns]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss_f16(tmem + T_DQ, smem_desc(ab + kk * 32, 16, 1024),
+                       smem_desc(kb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN,
+                       (h > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.ds_free[x]);
+          if (e == 1) mma_commit(&bars.kv_empty[itj % ns]);
+        }
+        if (ok) mma_commit(bars.dq_full);
+        it0 += nkv;
       }
-      if (ok) mma_commit(bars.dq_full);
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
     }
@@ -756,99 +815,133 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const int g = (warp - 4) >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int qrow = qt * 128 + row;
-    const bool row_ok = qrow < p.S;
-    const int L = p.causal ? min(qrow + 1, p.S) : p.S;
-    const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-    // ---- per-row setup: this group's share of delta = dO_r . O_r, the row
-    // constants and this group's table entries
-    {
-      const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
-      const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
-      part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
-    }
     const uint32_t tq_base = smem_u32(smem + p.tab_off);
-    const size_t trow = tile_row(p, bh, qt, row);
-    RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, tq_base);
-    mbar_arrive(bars.tab_ready);
-    bool ok = warp_all_b(mbar_wait(bars.tab_ready, 0, abort));
-    const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
-    if (MAP == MAPB_EXACT) {
-      kc.ds_ = delta;
-    } else {
-      kc.nDZ = -__fmul_rn(delta, kc.invZ);
-    }
-    if (g == 0 && row_ok) store_row_constants(p, trow, kc);
-    // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) - bits(M)
-    // + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard),
-    // M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
-    DqK dk;
-    dk.a = kc.a;
-    dk.b = kc.b;
-    dk.invZ = kc.invZ;
-    dk.nDZ = kc.nDZ;
-    dk.ne0 = -kc.e0;
-    dk.nds = -kc.ds_;
-    dk.kinv = kc.kinv;
-    dk.cL2E = p.cL2E;
-    dk.Kf = static_cast<float>(p.K);
-    dk.tq_row = (MAP == MAPB_INTERP)
-                    ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
-                    : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
-    const float Kf = dk.Kf;
-    float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
     const uint32_t dsb = smem_u32(sDS);
-    for (int h = 0; h < nh && ok; ++h) {
-      const int j = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
+    const float Kf = static_cast<float>(p.K);
+    bool ok = true;
+    int hc = 0, k = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      int bh, qt;
+      q_tile_of(p, t, bh, qt);
+      const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+      const int qrow = qt * 128 + row;
+      const bool row_ok = qrow < p.S;
+      const int L = p.causal ? min(qrow + 1, p.S) : p.S;
+      const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
+      // ---- per-row setup: this group's share of delta = dO_r . O_r, the
+      // row constants and this group's table entries
+      {
+        const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
+        const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
+        part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
+      }
+      const size_t trow = tile_row(p, bh, qt, row);
+      RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, tq_base);
+      mbar_arrive(bars.tab_ready);
+      ok = warp_all_b(mbar_wait(bars.tab_ready, k & 1, abort));
       if (!ok) break;
-      tc_fence_after();
-      uint32_t sv[16], dv[16];
-      tmem_ld16(lane_base + 128 * x + 16 * g, sv);
-      tmem_ld16(lane_base + 128 * x + 64 + 16 * g, dv);
-      tmem_wait_ld();
-      reg_fence16(sv);
-      reg_fence16(dv);
-      tc_fence_before();
-      mbar_arrive(&bars.sdp_free[x]);                  // the pair can take half h + 3
-      const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
-      uint32_t dd[8];
-      if (warp_all_b(lim >= 16))
-        dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
-      else
-        dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
-      if (u >= 1) {
-        // the dQ product of half h - 3 has read dS buffer x
-        ok = warp_all_b(mbar_wait(&bars.ds_free[x], (u - 1) & 1, abort));
+      const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
+      if (MAP == MAPB_EXACT) {
+        kc.ds_ = delta;
+      } else {
+        kc.nDZ = -__fmul_rn(delta, kc.invZ);
+      }
+      if (g == 0 && row_ok) store_row_constants(p, trow, kc);
+      // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) -
+      // bits(M) + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M)
+      // (hard), M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
+      DqK dk;
+      dk.a = kc.a;
+      dk.b = kc.b;
+      dk.invZ = kc.invZ;
+      dk.nDZ = kc.nDZ;
+      dk.ne0 = -kc.e0;
+      dk.nds = -kc.ds_;
+      dk.kinv = kc.kinv;
+      dk.cL2E = p.cL2E;
+      dk.Kf = Kf;
+      dk.tq_row = (MAP == MAPB_INTERP)
+                      ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
+                      : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
+      float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
+      for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
+        const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+        ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
         if (!ok) break;
-      }
-      // dS row-major (K-major operand), 128-byte swizzle: this group's 16
-      // keys are granules 2g, 2g + 1 of the row
-      const uint32_t rowa = dsb + x * 128 * 128 + row * 128;
+        tc_fence_after();
+        uint32_t sv[16], dv[16];
+        tmem_ld16(lane_base + 128 * x + 16 * g, sv);
+        tmem_ld16(lane_base + 128 * x + 64 + 16 * g, dv);
+        tmem_wait_ld();
+        reg_fence16(sv);
+        reg_fence16(dv);
+        tc_fence_before();
+        mbar_arrive(&bars.sdp_free[x]);                // the pair can take half hc + 3
+        const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
+        uint32_t dd[8];
+        if (warp_all_b(lim >= 16))
+          dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
+        else
+          dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
+        if (u >= 1) {
+          // the dQ product of half hc - 3 has read dS buffer x
+          ok = warp_all_b(mbar_wait(&bars.ds_free[x], (u - 1) & 1, abort));
+          if (!ok) break;
+        }
+        // dS row-major (K-major operand), 128-byte swizzle: this group's 16
+        // keys are granules 2g, 2g + 1 of the row
+        const uint32_t rowa = dsb + x * 128 * 128 + row * 128;
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        const uint32_t gran = static_cast<uint32_t>((2 * g + gi) ^ (row & 7));
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + gran * 16),
-                     "r"(dd[4 * gi]), "r"(dd[4 * gi + 1]), "r"(dd[4 * gi + 2]), "r"(dd[4 * gi + 3])
-                     : "memory");
+        for (int gi = 0; gi < 2; ++gi) {
+          const uint32_t gran = static_cast<uint32_t>((2 * g + gi) ^ (row & 7));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + gran * 16),
+                       "r"(dd[4 * gi]), "r"(dd[4 * gi + 1]), "r"(dd[4 * gi + 2]),
+                       "r"(dd[4 * gi + 3])
+                       : "memory");
+        }
+        fence_async_smem();
+        mbar_arrive(&bars.ds_full[x]);
       }
-      fence_async_smem();
-      mbar_arrive(&bars.ds_full[x]);
-    }
-    // ---- epilogue: the row's calibration sums, dQ
-    part[(4 + g) * 128 + row] = s1.x + s1.y;
-    part[(8 + g) * 128 + row] = s2.x + s2.y;
-    mbar_arrive(bars.part_ready);
-    if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
-    if (ok) ok = warp_all_b(mbar_wait(bars.dq_full, 0, abort));
-    if (ok) {
+      if (!ok) break;
+      // ---- epilogue: the row's calibration sums, dQ.  The key rows of the
+      // row's argmax / argmin and its own query row are fetched first, so
+      // their latency overlaps the waits for the other groups and the last
+      // product.
+      const bool cal_row = CAL != CAL_OFF && kc.calib && row_ok;
+      const size_t head = static_cast<size_t>(bh) * p.S;
+      int amx = 0, amn = 0;
+      uint4 kaw[2] = {}, kbw[2] = {}, qw[2] = {};
+      if (cal_row) {
+        amx = p.amax[ri];
+        const uint4 *ka = reinterpret_cast<const uint4 *>(p.K_ + (head + amx) * D + 16 * g);
+        const uint4 *qr = reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g);
+        kaw[0] = ka[0];
+        kaw[1] = ka[1];
+        qw[0] = qr[0];
+        qw[1] = qr[1];
+        if (CAL == CAL_MINMAX) {
+          amn = p.amin[ri];
+          const uint4 *kb = reinterpret_cast<const uint4 *>(p.K_ + (head + amn) * D + 16 * g);
+          kbw[0] = kb[0];
+          kbw[1] = kb[1];
+        }
+      }
+      part[(4 + g) * 128 + row] = s1.x + s1.y;
+      part[(8 + g) * 128 + row] = s2.x + s2.y;
+      mbar_arrive(bars.part_ready);
+      ok = warp_all_b(mbar_wait(bars.part_ready, k & 1, abort));
+      if (ok) ok = warp_all_b(mbar_wait(bars.dq_full, k & 1, abort));
+      if (!ok) break;
       tc_fence_after();
       uint32_t v[16];
       tmem_ld16_sync(lane_base + T_DQ + 16 * g, v);
+      // dQ is in registers: the next tile's dQ products may start
+      tc_fence_before();
+      mbar_arrive(bars.dq_free);
       float xq[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[i]) * p.c;
-      if (CAL != CAL_OFF && kc.calib && row_ok) {
+      if (cal_row) {
         const float S1 = (part[512 + row] + part[640 + row]) + (part[768 + row] + part[896 + row]);
         const float S2 =
             (part[1024 + row] + part[1152 + row]) + (part[1280 + row] + part[1408 + row]);
@@ -865,27 +958,24 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         }
         // rank-one calibration terms in fp32: dQ_r += c (dhi k_argmax + dlo
         // k_argmin), and dK_argmax += c dhi q_r, dK_argmin += c dlo q_r into
-        // the fp32 calibration part of dK (many rows can share a key: vector
+        // the fp32 calibration part of dK (rows can share a key: vector
         // reductions)
-        const size_t head = static_cast<size_t>(bh) * p.S;
         const float sh = p.c * dhi, sl = p.c * dlo;
         float kx[16], qx[16];
-        bf16x16_to_f32(reinterpret_cast<const uint4 *>(p.K_ + (head + p.amax[ri]) * D + 16 * g),
-                       kx);
-        bf16x16_to_f32(reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g), qx);
+        bf16x16_to_f32(kaw, kx);
+        bf16x16_to_f32(qw, qx);
 #pragma unroll
         for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
-        float *da = p.dkcal + (head + p.amax[ri]) * D + 16 * g;
+        float *da = p.dkcal + (head + amx) * D + 16 * g;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
                                                 sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
         if (CAL == CAL_MINMAX) {
-          bf16x16_to_f32(
-              reinterpret_cast<const uint4 *>(p.K_ + (head + p.amin[ri]) * D + 16 * g), kx);
+          bf16x16_to_f32(kbw, kx);
 #pragma unroll
           for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
-          float *db = p.dkcal + (head + p.amin[ri]) * D + 16 * g;
+          float *db = p.dkcal + (head + amn) * D + 16 * g;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
@@ -911,8 +1001,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 }
 
 // --------------------------------------------------------------- dK/dV pass
-// One CTA per 128-key tile of one (b, h); thread = key (TMEM lane); the
-// query tiles are taken in halves of 64 rows, half h in TMEM pair x = h mod 3
+// Persistent: one CTA per SM takes the 128-key tiles in the heaviest-first
+// order; thread = key (TMEM lane); the query tiles are taken in halves of 64
+// rows, half number hc (counted across tiles) in TMEM pair x = hc mod 3
 // (S^T at 128x, dP^T at 128x + 64); map group g owns rows 16g .. 16g+15 of
 // each half and writes its P^T and dS^T (bf16) into the first 8 of its own 16
 // columns, which the dV / dK products (dV at TMEM column 384, dK at 448) read
@@ -920,9 +1011,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 // per-row constants and grid tables.
 struct KvBars {
   uint64_t *qd_full, *qd_empty;       // [ns]
-  uint64_t *kv_full;                  // K, V once
+  uint64_t *kv_full, *kv_free;        // K, V of the current tile
   uint64_t *sdp_full, *pds_full, *s_free;   // [kHalfBufs]
-  uint64_t *acc_full, *drain;
+  uint64_t *acc_full, *acc_free;      // the tile's dV, dK complete / read out of TMEM
+  uint64_t *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
@@ -1016,7 +1108,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y, kt = blockIdx.x;
+  const int ntiles = p.nkvt * p.BH;
+  const int step = static_cast<int>(gridDim.x);
   const int ns = p.num_stages;
   uint8_t *sK = smem;
   uint8_t *sV = smem + G::TILE_BYTES;
@@ -1029,17 +1122,16 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.qd_full = bp;
   bars.qd_empty = bp + ns;
   bars.kv_full = bp + 2 * ns;
-  bars.sdp_full = bars.kv_full + 1;
+  bars.kv_free = bars.kv_full + 1;
+  bars.sdp_full = bars.kv_free + 1;
   bars.pds_full = bars.sdp_full + kHalfBufs;
   bars.s_free = bars.pds_full + kHalfBufs;
   bars.acc_full = bars.s_free + kHalfBufs;
-  bars.drain = bars.acc_full + 1;
+  bars.acc_free = bars.acc_full + 1;
+  bars.drain = bars.acc_free + 1;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
-  const int i0 = p.causal ? kt : 0;                      // first query tile
-  const int nq = p.nqt - i0;
-  const int nh = 2 * nq;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ns; ++i) {
@@ -1047,12 +1139,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.qd_empty[i], 1);
     }
     mbar_init(bars.kv_full, 1);
+    mbar_init(bars.kv_free, 1);
     for (int i = 0; i < kHalfBufs; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.pds_full[i], kMainMapThreads);
       mbar_init(&bars.s_free[i], 1);
     }
     mbar_init(bars.acc_full, 1);
+    mbar_init(bars.acc_free, kMainMapThreads);
     mbar_init(bars.drain, 2);
     *bars.abort = 0;
     fence_mbar_init();
@@ -1063,60 +1157,85 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
+  // Tiles of this CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ... of the
+  // heaviest-first key-tile order (persistent, as the dQ pass); the ring
+  // position and the half counter run on across tiles.
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(bars.kv_full, 2 * G::TILE_BYTES);
-      for (int ch = 0; ch < G::CHUNKS; ++ch) {
-        tma_load_3d(sK + ch * G::CHUNK_BYTES, &tmK, bars.kv_full, ch * G::EPC, kt * 128, bh);
-        tma_load_3d(sV + ch * G::CHUNK_BYTES, &tmV, bars.kv_full, ch * G::EPC, kt * 128, bh);
-      }
       bool ok = true;
-      for (int n = 0; n < nq && ok; ++n) {
-        const int st = n % ns, it = i0 + n;
-        if (n >= ns) ok = mbar_wait(&bars.qd_empty[st], ((n / ns) - 1) & 1, abort);
+      int rc = 0, k = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, kt;
+        kv_tile_of(p, t, bh, kt);
+        const int i0 = p.causal ? kt : 0;                // first query tile
+        const int nq = p.nqt - i0;
+        // K, V of the previous tile are no longer read
+        if (k >= 1) ok = mbar_wait(bars.kv_free, (k - 1) & 1, abort);
         if (!ok) break;
-        uint8_t *s = sSt + st * SB;
-        // the constants and tables of the tile's 128 tile rows (rows past S in
-        // a ragged last tile are never valid)
-        const size_t r0 = (static_cast<size_t>(bh) * p.nqt + it) * 128;
-        const uint32_t cbytes = 128u * kCst * 4;
-        const uint32_t tbytes = 128u * static_cast<uint32_t>(p.TS) * 4;
-        mbar_expect_tx(&bars.qd_full[st], 2 * G::TILE_BYTES + cbytes + tbytes);
+        mbar_expect_tx(bars.kv_full, 2 * G::TILE_BYTES);
         for (int ch = 0; ch < G::CHUNKS; ++ch) {
-          tma_load_3d(s + ch * G::CHUNK_BYTES, &tmQ, &bars.qd_full[st], ch * G::EPC, it * 128, bh);
-          tma_load_3d(s + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmdO, &bars.qd_full[st],
-                      ch * G::EPC, it * 128, bh);
+          tma_load_3d(sK + ch * G::CHUNK_BYTES, &tmK, bars.kv_full, ch * G::EPC, kt * 128, bh);
+          tma_load_3d(sV + ch * G::CHUNK_BYTES, &tmV, bars.kv_full, ch * G::EPC, kt * 128, bh);
         }
-        bulk_load(s + CST_OFF, p.cst + r0 * kCst, cbytes, &bars.qd_full[st]);
-        if (tbytes) bulk_load(s + TAB_OFF, p.tabk + r0 * p.TS, tbytes, &bars.qd_full[st]);
+        for (int n = 0; n < nq && ok; ++n, ++rc) {
+          const int st = rc % ns, qi = i0 + n;
+          if (rc >= ns) ok = mbar_wait(&bars.qd_empty[st], ((rc / ns) - 1) & 1, abort);
+          if (!ok) break;
+          uint8_t *s = sSt + st * SB;
+          // the constants and tables of the tile's 128 tile rows (rows past S
+          // in a ragged last tile are never valid)
+          const size_t r0 = (static_cast<size_t>(bh) * p.nqt + qi) * 128;
+          const uint32_t cbytes = 128u * kCst * 4;
+          const uint32_t tbytes = 128u * static_cast<uint32_t>(p.TS) * 4;
+          mbar_expect_tx(&bars.qd_full[st], 2 * G::TILE_BYTES + cbytes + tbytes);
+          for (int ch = 0; ch < G::CHUNKS; ++ch) {
+            tma_load_3d(s + ch * G::CHUNK_BYTES, &tmQ, &bars.qd_full[st], ch * G::EPC, qi * 128,
+                        bh);
+            tma_load_3d(s + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmdO, &bars.qd_full[st],
+                        ch * G::EPC, qi * 128, bh);
+          }
+          bulk_load(s + CST_OFF, p.cst + r0 * kCst, cbytes, &bars.qd_full[st]);
+          if (tbytes) bulk_load(s + TAB_OFF, p.tabk + r0 * p.TS, tbytes, &bars.qd_full[st]);
+        }
       }
-      mbar_wait(bars.kv_full, 0, abort);
-      for (int st = 0; st < ns && st < nq; ++st)
-        mbar_wait(&bars.qd_full[st], (((nq - st + ns - 1) / ns) - 1) & 1, abort);
+      // every load issued must land before the CTA may exit
+      if (k >= 1) mbar_wait(bars.kv_full, (k - 1) & 1, abort);
+      for (int st = 0; st < ns && st < rc; ++st)
+        mbar_wait(&bars.qd_full[st], (((rc - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair h mod 3,
-    // once the dV / dK products of half h - 3 have read it
+    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair hc mod 3,
+    // once the dV / dK products of half hc - 3 have read it
     if (lane == 0) {
-      bool ok = mbar_wait(bars.kv_full, 0, abort);
-      tc_fence_after();
+      bool ok = true;
+      int rc0 = 0, hc = 0, k = 0;
       const uint32_t ka = smem_u32(sK), va = smem_u32(sV), sa = smem_u32(sSt);
-      for (int h = 0; h < nh && ok; ++h) {
-        const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-        if (e == 0) {
-          ok = mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, kt;
+        kv_tile_of(p, t, bh, kt);
+        const int nq = p.nqt - (p.causal ? kt : 0);
+        ok = mbar_wait(bars.kv_full, k & 1, abort);
+        tc_fence_after();
+        for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
+          const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+          const int rn = rc0 + n;
+          if (e == 0) {
+            ok = mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          if (u >= 1) {
+            ok = mbar_wait(&bars.s_free[x], (u - 1) & 1, abort);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint32_t qb = sa + (rn % ns) * SB + e * 64 * 128;
+          mma_nt_half<D>(tmem + 128 * x, ka, qb);
+          mma_nt_half<D>(tmem + 128 * x + 64, va, qb + G::TILE_BYTES);
+          mma_commit(&bars.sdp_full[x]);
         }
-        if (u >= 1) {
-          ok = mbar_wait(&bars.s_free[x], (u - 1) & 1, abort);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        const uint32_t qb = sa + (n % ns) * SB + e * 64 * 128;
-        mma_nt_half<D>(tmem + 128 * x, ka, qb);
-        mma_nt_half<D>(tmem + 128 * x + 64, va, qb + G::TILE_BYTES);
-        mma_commit(&bars.sdp_full[x]);
+        if (ok) mma_commit(bars.kv_free);               // the tile's K, V are read
+        rc0 += nq;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -1125,30 +1244,40 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // dV += P^T_h dO_h and dK += dS^T_h Q_h (A from TMEM, B MN-major)
     if (lane == 0) {
       bool ok = true;
+      int rc0 = 0, hc = 0, k = 0;
       const uint32_t sa = smem_u32(sSt);
-      for (int h = 0; h < nh && ok; ++h) {
-        const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-        if (e == 0) {
-          ok = mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort);
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, kt;
+        kv_tile_of(p, t, bh, kt);
+        const int nq = p.nqt - (p.causal ? kt : 0);
+        for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
+          const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+          const int rn = rc0 + n;
+          if (e == 0) {
+            ok = mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort);
+            if (!ok) break;
+          }
+          ok = mbar_wait(&bars.pds_full[x], u & 1, abort);
+          // the previous tile's dV, dK have been read out of TMEM
+          if (ok && h == 0 && k >= 1) ok = mbar_wait(bars.acc_free, (k - 1) & 1, abort);
           if (!ok) break;
-        }
-        ok = mbar_wait(&bars.pds_full[x], u & 1, abort);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t qb = sa + (n % ns) * SB + e * 64 * 128;
-        const uint32_t db = qb + G::TILE_BYTES;
+          tc_fence_after();
+          const uint32_t qb = sa + (rn % ns) * SB + e * 64 * 128;
+          const uint32_t db = qb + G::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t acc = (h > 0 || kk > 0) ? 1u : 0u;
-          mma_ts_f16(tmem + T_DV, tmem + 128 * x + 16 * kk,
-                     smem_desc(db + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
-          mma_ts_f16(tmem + T_DK, tmem + 128 * x + 64 + 16 * kk,
-                     smem_desc(qb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = (h > 0 || kk > 0) ? 1u : 0u;
+            mma_ts_f16(tmem + T_DV, tmem + 128 * x + 16 * kk,
+                       smem_desc(db + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
+            mma_ts_f16(tmem + T_DK, tmem + 128 * x + 64 + 16 * kk,
+                       smem_desc(qb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
+          }
+          mma_commit(&bars.s_free[x]);
+          if (e == 1) mma_commit(&bars.qd_empty[rn % ns]);
         }
-        mma_commit(&bars.s_free[x]);
-        if (e == 1) mma_commit(&bars.qd_empty[n % ns]);
+        if (ok) mma_commit(bars.acc_full);
+        rc0 += nq;
       }
-      if (ok) mma_commit(bars.acc_full);
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
     }
@@ -1156,8 +1285,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const int g = (warp - 4) >> 2;
     const int key = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int kg = kt * 128 + key;
-    const bool key_ok = kg < p.S;
     KvK kk;
     kk.cL2E = p.cL2E;
     kk.Kf = static_cast<float>(p.K);
@@ -1168,76 +1295,100 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // table entry bias: bits(M + floor(clamp(u, -1, K))) - bits(M) + 1 (interp)
     // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), mod 2^32
     const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - kMagicBits * 8u : 0u - kMagicBits * 4u;
-    bool ok = true;
     const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
-    for (int h = 0; h < nh && ok; ++h) {
-      const int n = h >> 1, e = h & 1, x = h % kHalfBufs, u = h / kHalfBufs;
-      if (e == 0) {
-        // the stage's constants and tables have landed (the stage cannot
-        // refill before this tile's products, which wait for these threads)
-        ok = warp_all_b(mbar_wait(&bars.qd_full[n % ns], (n / ns) & 1, abort));
+    bool ok = true;
+    int rc0 = 0, hc = 0, k = 0;
+    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      int bh, kt;
+      kv_tile_of(p, t, bh, kt);
+      const int i0 = p.causal ? kt : 0;                  // first query tile
+      const int nq = p.nqt - i0;
+      const int kg = kt * 128 + key;
+      const bool key_ok = kg < p.S;
+      for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
+        const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+        const int rn = rc0 + n;
+        if (e == 0) {
+          // the stage's constants and tables have landed (the stage cannot
+          // refill before this tile's products, which wait for these threads)
+          ok = warp_all_b(mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort));
+          if (!ok) break;
+        }
+        ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
         if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sSt + (rn % ns) * SB);
+        uint32_t sv[16], dv[16];
+        tmem_ld16(lane_base + 128 * x + 16 * g, sv);
+        tmem_ld16(lane_base + 128 * x + 64 + 16 * g, dv);
+        tmem_wait_ld();
+        reg_fence16(sv);
+        reg_fence16(dv);
+        const int qbase = (i0 + n) * 128 + 64 * e + 16 * g;   // first query row of the slice
+        const int ql0 = 64 * e + 16 * g;                      // its row within the tile
+        // every element valid: the key exists, the slice's rows exist and
+        // (causal) lie at or below this key
+        const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
+        const uint32_t cb = st + CST_OFF + ql0 * (kCst * 4);
+        const uint32_t tr = st + TAB_OFF + ql0 * tsb + tbias;
+        uint32_t pp[8], dd[8];
+        if (full) {
+          kv_slice<MAP, SURR, true>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
+        } else {
+          uint32_t vmask = 0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            vmask |= (key_ok && qbase + i < p.S && (!p.causal || kg <= qbase + i)) ? (1u << i) : 0u;
+          kv_slice<MAP, SURR, false>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
+        }
+        tmem_st8(lane_base + 128 * x + 16 * g, pp);
+        tmem_st8(lane_base + 128 * x + 64 + 16 * g, dd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars.pds_full[x]);
       }
-      ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
+      if (!ok) break;
+      rc0 += nq;
+      // the key's fp32 calibration part of dK (written by the dQ pass) is
+      // fetched before the wait for the tile's last products
+      const size_t krow = static_cast<size_t>(bh) * p.S + min(kg, p.S - 1);
+      float4 cal[4] = {};
+      if (p.dkcal != nullptr && key_ok) {
+        const float4 *c4 = reinterpret_cast<const float4 *>(p.dkcal + krow * D + 16 * g);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) cal[i] = c4[i];
+      }
+      ok = warp_all_b(mbar_wait(bars.acc_full, k & 1, abort));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t st = smem_u32(sSt + (n % ns) * SB);
-      uint32_t sv[16], dv[16];
-      tmem_ld16(lane_base + 128 * x + 16 * g, sv);
-      tmem_ld16(lane_base + 128 * x + 64 + 16 * g, dv);
+      uint32_t v[16], w[16];
+      tmem_ld16(lane_base + T_DV + 16 * g, v);
+      tmem_ld16(lane_base + T_DK + 16 * g, w);
       tmem_wait_ld();
-      reg_fence16(sv);
-      reg_fence16(dv);
-      const int qbase = (i0 + n) * 128 + 64 * e + 16 * g;   // first query row of the slice
-      const int ql0 = 64 * e + 16 * g;                      // its row within the tile
-      // every element valid: the key exists, the slice's rows exist and (causal)
-      // lie at or below this key
-      const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
-      const uint32_t cb = st + CST_OFF + ql0 * (kCst * 4);
-      const uint32_t tr = st + TAB_OFF + ql0 * tsb + tbias;
-      uint32_t pp[8], dd[8];
-      if (full) {
-        kv_slice<MAP, SURR, true>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
-      } else {
-        uint32_t vmask = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          vmask |= (key_ok && qbase + i < p.S && (!p.causal || kg <= qbase + i)) ? (1u << i) : 0u;
-        kv_slice<MAP, SURR, false>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
-      }
-      tmem_st8(lane_base + 128 * x + 16 * g, pp);
-      tmem_st8(lane_base + 128 * x + 64 + 16 * g, dd);
-      tmem_wait_st();
+      reg_fence16(v);
+      reg_fence16(w);
+      // dV, dK are in registers: the next tile's products may start
       tc_fence_before();
-      mbar_arrive(&bars.pds_full[x]);
-    }
-    if (ok) ok = warp_all_b(mbar_wait(bars.acc_full, 0, abort));
-    if (ok) {
-      tc_fence_after();
-      const size_t krow = static_cast<size_t>(bh) * p.S + min(kg, p.S - 1);
-      uint32_t v[16];
-      tmem_ld16_sync(lane_base + T_DV + 16 * g, v);
+      mbar_arrive(bars.acc_free);
       uint32_t pk[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+      for (int i = 0; i < 8; ++i)
+        pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
       if (key_ok) {
         uint4 *d4 = reinterpret_cast<uint4 *>(p.dV + krow * D + 16 * g);
         d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
-      tmem_ld16_sync(lane_base + T_DK + 16 * g, v);
       float xk[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xk[i] = __uint_as_float(v[i]) * p.c;
+      for (int i = 0; i < 16; ++i) xk[i] = __uint_as_float(w[i]) * p.c;
       if (p.dkcal != nullptr && key_ok) {
-        const float4 *cal = reinterpret_cast<const float4 *>(p.dkcal + krow * D + 16 * g);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float4 c4 = cal[i];
-          xk[4 * i] += c4.x;
-          xk[4 * i + 1] += c4.y;
-          xk[4 * i + 2] += c4.z;
-          xk[4 * i + 3] += c4.w;
+          xk[4 * i] += cal[i].x;
+          xk[4 * i + 1] += cal[i].y;
+          xk[4 * i + 2] += cal[i].z;
+          xk[4 * i + 3] += cal[i].w;
         }
       }
 #pragma unroll
@@ -1279,6 +1430,23 @@ bool set_smem_once(F kern, int bytes, std::atomic<int> (&cache)[kMaxDevices]) {
 }
 
 constexpr size_t kMaxSmem = 232448;                      // 227 KB opt-in per CTA
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool in = dev >= 0 && dev < kMaxDevices;
+  if (in) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (in) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 constexpr size_t kBarBytes = ((2 * 8 + 24) * 8 + 8 + 15) & ~static_cast<size_t>(15);
 
 template <int D, int MAP, int SURR, int CAL>
@@ -1304,7 +1472,10 @@ qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const
   auto kern = qsm_bwd_dq<D, MAP, SURR, CAL>;
   static std::atomic<int> cache[kMaxDevices];
   if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-  kern<<<dim3(p.nqt * a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+  // persistent: one CTA per SM walks the query tiles
+  const int ntiles = p.nqt * a.B * a.H;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  kern<<<dim3(grid), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
@@ -1329,7 +1500,10 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
   auto kern = qsm_bwd_dkdv<D, MAP, SURR>;
   static std::atomic<int> cache[kMaxDevices];
   if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-  kern<<<dim3(p.nkvt, a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+  // persistent: one CTA per SM walks the key tiles
+  const int ntiles = p.nkvt * a.B * a.H;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  kern<<<dim3(grid), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
