@@ -88,12 +88,14 @@ struct BwdParams {
   float *rowws;     // [rows][kRowWs]: LSE*, delta* (post surrogate)
   float *cst;       // [tile rows / 2][16]: row pairs' constants, interleaved (cst_index)
   float *tabk;      // [tile rows][TS]: the dK / dV pass's grid table of each row
+  uint8_t *tabq;    // [query tiles][tabq_tile bytes]: the dQ pass's table of each tile
   float *dkcal;     // [rows][D] fp32 calibration part of dK (nullptr: none)
   const __nv_bfloat16 *Q, *K_, *O, *dO;
   __nv_bfloat16 *dQ, *dK, *dV;
   int32_t *status;
   int num_stages;
-  uint32_t tab_off, ds_off, bar_off, part_off, stage_bytes;
+  uint32_t tabq_tile;   // bytes of one tile's dQ-pass table (0: none)
+  uint32_t tab_off, ds_off, bar_off, part_off, stage_bytes, cst_off;
 };
 
 template <int D>
@@ -423,7 +425,8 @@ struct RowC {
 // query tile starts a row pair.  The constants of rows 2m and 2m + 1 sit
 // together, each field as a pair, so that one 16-byte load gives the packed
 // operands of two rows: [a a' b b' | invZ invZ' nDZ nDZ' | -e0 -e0' -ds_ -ds_'
-// | kinv kinv' 0 0] (16 floats).
+// | kinv kinv' cal cal'] (16 floats; cal = 1 when the row takes calibration
+// terms, else 0).
 __device__ __forceinline__ size_t tile_row(const BwdParams &p, int bh, int qt, int row) {
   return (static_cast<size_t>(bh) * p.nqt + qt) * 128 + row;
 }
@@ -436,7 +439,7 @@ __device__ __forceinline__ void store_row_constants(const BwdParams &p, size_t t
   c[8] = -k.e0;
   c[10] = -k.ds_;
   c[12] = k.kinv;
-  c[14] = 0.0f;
+  c[14] = k.calib ? 1.0f : 0.0f;
 }
 
 // Table layouts (K-interval).  Entry i of a row, interpolation, i = 0..K+1:
@@ -538,6 +541,54 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, siz
   return k;
 }
 
+// ----------------------------------------------------------- row prep
+// One CTA per 128-row query tile, four threads per row (group g owns
+// columns 16g .. 16g+15 of delta = dO_r . O_r and table entries g, g + 4,
+// ...): each row's delta, map constants and grid tables, written to the
+// workspace -- the constants (both passes), the dK / dV pass's table per
+// row, and the dQ pass's table per tile in its shared-memory layout, which
+// the dQ pass copies in with one bulk load per tile.  Rows past S in a
+// ragged last tile take the last row's values, so every workspace entry of a
+// tile is defined.
+template <int D, int MAP, int SURR, int CAL>
+__global__ void __launch_bounds__(kMainMapThreads)
+    qsm_bwd_prep(const BwdParams p) {
+  using T = DqTab<MAP, SURR, CAL>;
+  static_assert(D == 64, "delta slices of the four groups: 16 columns each");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_align1024(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = warp >> 2;
+  const int row = (warp & 3) * 32 + lane;
+  const int tix = static_cast<int>(blockIdx.x);         // bh * nqt + qt
+  const int bh = tix / p.nqt, qt = tix - bh * p.nqt;
+  const int qrow = qt * 128 + row;
+  const bool row_ok = qrow < p.S;
+  const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
+  const size_t tbytes = T::bytes(p.K);
+  float *part = reinterpret_cast<float *>(smem + ((tbytes + 15) & ~static_cast<size_t>(15)));
+  {
+    const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
+    const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
+    part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
+  }
+  const size_t trow = tile_row(p, bh, qt, row);
+  RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, smem_u32(smem));
+  __syncthreads();
+  const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
+  if (MAP == MAPB_EXACT)
+    kc.ds_ = delta;
+  else
+    kc.nDZ = -__fmul_rn(delta, kc.invZ);
+  if (!row_ok) kc.calib = false;
+  if (g == 0) store_row_constants(p, trow, kc);
+  if (T::ANY) {
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(smem);
+    uint4 *d4 = reinterpret_cast<uint4 *>(p.tabq + static_cast<size_t>(tix) * p.tabq_tile);
+    for (size_t i = threadIdx.x; i < tbytes / 16; i += kMainMapThreads) d4[i] = s4[i];
+  }
+}
+
 __device__ __forceinline__ float2 ex2_pair(float2 x) {
   return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
@@ -615,19 +666,33 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
 // (TMEM lane); the key tiles are taken in halves of 64 keys, half number hc
 // (counted across tiles) in TMEM pair x = hc mod 3 (S at 128x, dP at 128x +
 // 64) and shared dS buffer x; map group g owns keys 16g .. 16g+15 of each
-// half.  dQ accumulates at TMEM column 384 and is read out before the next
-// tile's first dQ product.
+// half.  The row constants and the table of a tile come from the prep kernel
+// (warp 3 copies them in).  dQ of tile k accumulates in TMEM buffer k mod 2
+// (columns 384 + 64 (k mod 2)), and the map threads read it out after the
+// halves of tile k + 1: by then every map thread has finished tile k, so
+// the read-out waits for no straggler and the products of tile k + 1 run
+// meanwhile.
 struct DqBars {
   uint64_t *kv_full, *kv_empty;       // [ns]: K_j, V_j
   uint64_t *q_full, *q_free;          // Q, dO of the current tile
   uint64_t *sdp_full, *sdp_free;      // [kHalfBufs]
   uint64_t *ds_full, *ds_free;        // [kHalfBufs]
-  uint64_t *dq_full, *dq_free;        // the tile's dQ complete / read out of TMEM
-  uint64_t *tab_ready, *part_ready, *drain;
+  uint64_t *dq_full, *dq_free;        // [2]: a tile's dQ complete / read out of TMEM
+  uint64_t *tab_full, *tab_free;      // the tile's constants and table
+  uint64_t *part_ready, *part_free;   // [2]: a tile's calibration sums written / read
+  uint64_t *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
 constexpr uint32_t T_DQ = 384;
+
+// The calibration state of a finished tile that its read-out needs: the
+// tile, the row's argmax / argmin key (amx < 0: no calibration terms) and
+// K/(hi - lo).
+struct DqPrev {
+  int t, amx, amn;
+  float kinv;
+};
 
 template <int D, int MAP, int SURR, int CAL>
 __global__ void __launch_bounds__(kMainThreads, 1)
@@ -647,7 +712,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *sdO = smem + G::TILE_BYTES;
   uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages of (K_j, V_j)
   uint8_t *sDS = smem + p.ds_off;                        // 3 x 128 rows x 128 bytes
-  float *part = reinterpret_cast<float *>(smem + p.part_off);   // [3][4][128]
+  uint8_t *sCst = smem + p.cst_off;                      // 64 row pairs x 16 floats
+  float *part = reinterpret_cast<float *>(smem + p.part_off);   // [2][2][4][128]
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   DqBars bars;
   bars.kv_full = bp;
@@ -659,10 +725,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.ds_full = bars.sdp_free + kHalfBufs;
   bars.ds_free = bars.ds_full + kHalfBufs;
   bars.dq_full = bars.ds_free + kHalfBufs;
-  bars.dq_free = bars.dq_full + 1;
-  bars.tab_ready = bars.dq_free + 1;
-  bars.part_ready = bars.tab_ready + 1;
-  bars.drain = bars.part_ready + 1;
+  bars.dq_free = bars.dq_full + 2;
+  bars.tab_full = bars.dq_free + 2;
+  bars.tab_free = bars.tab_full + 1;
+  bars.part_ready = bars.tab_free + 1;
+  bars.part_free = bars.part_ready + 2;
+  bars.drain = bars.part_free + 2;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
@@ -680,10 +748,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_init(&bars.ds_full[i], kMainMapThreads);
       mbar_init(&bars.ds_free[i], 1);
     }
-    mbar_init(bars.dq_full, 1);
-    mbar_init(bars.dq_free, kMainMapThreads);
-    mbar_init(bars.tab_ready, kMainMapThreads);
-    mbar_init(bars.part_ready, kMainMapThreads);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars.dq_full[i], 1);
+      mbar_init(&bars.dq_free[i], kMainMapThreads);
+      mbar_init(&bars.part_ready[i], kMainMapThreads);
+      mbar_init(&bars.part_free[i], kMainMapThreads);
+    }
+    mbar_init(bars.tab_full, 1);
+    mbar_init(bars.tab_free, kMainMapThreads);
     mbar_init(bars.drain, 2);
     *bars.abort = 0;
     fence_mbar_init();
@@ -696,9 +768,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 
   // Tiles of this CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ... of the
   // heaviest-first order (persistent: the next tile's loads and first
-  // products overlap this tile's epilogue).  Every role walks the same
+  // products overlap this tile's last halves).  Every role walks the same
   // sequence; the ring position `it` and the half counter `hc` run on across
-  // tiles, and per-tile barriers take the tile's own parity k & 1.
+  // tiles, and per-tile barriers take the tile's own parity.
   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
@@ -773,6 +845,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     }
   } else if (warp == 2) {
     // dQ += dS_h K_h (dS K-major in shared memory, K as an MN-major operand)
+    // into TMEM buffer k mod 2
     if (lane == 0) {
       bool ok = true;
       int it0 = 0, hc = 0, k = 0;
@@ -781,6 +854,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        const uint32_t dq = tmem + T_DQ + 64 * (k & 1);
         for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
           const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
           const int itj = it0 + j;
@@ -791,35 +865,159 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             if (!ok) break;
           }
           ok = mbar_wait(&bars.ds_full[x], u & 1, abort);
-          // the previous tile's dQ has been read out of TMEM
-          if (ok && h == 0 && k >= 1) ok = mbar_wait(bars.dq_free, (k - 1) & 1, abort);
+          // the buffer's previous tile (k - 2) has been read out of TMEM
+          if (ok && h == 0 && k >= 2) ok = mbar_wait(&bars.dq_free[k & 1], ((k >> 1) - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = kva + (itj % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
           const uint32_t ab = dsa + x * 128 * 128;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss_f16(tmem + T_DQ, smem_desc(ab + kk * 32, 16, 1024),
+            mma_ss_f16(dq, smem_desc(ab + kk * 32, 16, 1024),
                        smem_desc(kb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN,
                        (h > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.ds_free[x]);
           if (e == 1) mma_commit(&bars.kv_empty[itj % ns]);
         }
-        if (ok) mma_commit(bars.dq_full);
+        if (ok) mma_commit(&bars.dq_full[k & 1]);
         it0 += nkv;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
+    }
+  } else if (warp == 3) {
+    // the tile's row constants and dQ-pass table (prep kernel output), once
+    // every map thread is done with the previous tile's
+    if (lane == 0) {
+      bool ok = true;
+      int k = 0;
+      const uint32_t cbytes = 128u * kCst * 4;
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        if (k >= 1) ok = mbar_wait(bars.tab_free, (k - 1) & 1, abort);
+        if (!ok) break;
+        const size_t tix = static_cast<size_t>(bh) * p.nqt + qt;
+        mbar_expect_tx(bars.tab_full, cbytes + p.tabq_tile);
+        bulk_load(sCst, p.cst + tix * 128 * kCst, cbytes, bars.tab_full);
+        if (p.tabq_tile)
+          bulk_load(smem + p.tab_off, p.tabq + tix * p.tabq_tile, p.tabq_tile, bars.tab_full);
+      }
+      // every load issued must land before the CTA may exit
+      if (k >= 1) mbar_wait(bars.tab_full, (k - 1) & 1, abort);
     }
   } else if (warp >= 4) {
     const int g = (warp - 4) >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t tq_base = smem_u32(smem + p.tab_off);
+    // this row's constants: field f at ca + 8 f (row pairs interleaved)
+    const uint32_t ca = smem_u32(sCst) + (row >> 1) * 64 + (row & 1) * 4;
+    const float *cstf = reinterpret_cast<const float *>(sCst) + (row >> 1) * 16 + (row & 1);
     const uint32_t dsb = smem_u32(sDS);
     const float Kf = static_cast<float>(p.K);
+    // Read-out of a finished tile (position kp in this CTA's sequence, tile
+    // t): dQ out of TMEM buffer kp mod 2, the rank-one calibration terms in
+    // fp32 -- dQ_r += c (dhi k_argmax + dlo k_argmin), and dK_argmax += c dhi
+    // q_r, dK_argmin += c dlo q_r into the fp32 calibration part of dK (rows
+    // can share a key: vector reductions) -- and the bf16 store.  amx < 0:
+    // the row takes no calibration terms.
+    auto read_out = [&](int t, int kp, int amx, int amn, float kinv) -> bool {
+      const int x = kp & 1;
+      const uint32_t ph = static_cast<uint32_t>(kp >> 1) & 1u;
+      int bh, qt;
+      q_tile_of(p, t, bh, qt);
+      const int qrow = qt * 128 + row;
+      const size_t head = static_cast<size_t>(bh) * p.S;
+      const size_t ri = head + min(qrow, p.S - 1);
+      const bool cal_row = CAL != CAL_OFF && amx >= 0;
+      // the key rows and the query row are fetched before the waits
+      uint4 kaw[2] = {}, kbw[2] = {}, qw[2] = {};
+      if (cal_row) {
+        const uint4 *ka = reinterpret_cast<const uint4 *>(p.K_ + (head + amx) * D + 16 * g);
+        const uint4 *qr = reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g);
+        kaw[0] = ka[0];
+        kaw[1] = ka[1];
+        qw[0] = qr[0];
+        qw[1] = qr[1];
+        if (CAL == CAL_MINMAX) {
+          const uint4 *kb = reinterpret_cast<const uint4 *>(p.K_ + (head + amn) * D + 16 * g);
+          kbw[0] = kb[0];
+          kbw[1] = kb[1];
+        }
+      }
+      bool rok = warp_all_b(mbar_wait(&bars.part_ready[x], ph, abort));
+      if (rok) rok = warp_all_b(mbar_wait(&bars.dq_full[x], ph, abort));
+      if (!rok) return false;
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16_sync(lane_base + T_DQ + 64 * x + 16 * g, v);
+      // the accumulator is in registers: tile kp + 2 may take the buffer
+      tc_fence_before();
+      mbar_arrive(&bars.dq_free[x]);
+      // the row's calibration derivatives from the four groups' sums; they
+      // are computed (the loaded sums consumed) before the buffer's release
+      float sh = 0.0f, sl = 0.0f;
+      if (cal_row) {
+        const float *pp = part + x * 1024;
+        const float S1 = (pp[row] + pp[128 + row]) + (pp[256 + row] + pp[384 + row]);
+        const float S2 = (pp[512 + row] + pp[640 + row]) + (pp[768 + row] + pp[896 + row]);
+        float dhi, dlo;
+        if (CAL == CAL_FIXED) {
+          dhi = -(Kf / p.window) * S2;
+          dlo = 0.0f;
+        } else if (MAP == MAPB_HARD) {
+          dhi = S1;
+          dlo = -S1;
+        } else {
+          dhi = S1;
+          dlo = -S1 - kinv * S2;
+        }
+        sh = p.c * dhi;
+        sl = p.c * dlo;
+      }
+      asm volatile("" ::"f"(sh), "f"(sl) : "memory");
+      mbar_arrive(&bars.part_free[x]);
+      float xq[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[i]) * p.c;
+      if (cal_row) {
+        float kx[16], qx[16];
+        bf16x16_to_f32(kaw, kx);
+        bf16x16_to_f32(qw, qx);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
+        float *da = p.dkcal + (head + amx) * D + 16 * g;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
+                                                sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
+        if (CAL == CAL_MINMAX) {
+          bf16x16_to_f32(kbw, kx);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
+          float *db = p.dkcal + (head + amn) * D + 16 * g;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
+                                                  sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
+        }
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(xq[2 * i], xq[2 * i + 1]);
+      if (qrow < p.S) {
+        uint4 *d4 = reinterpret_cast<uint4 *>(p.dQ + ri * D + 16 * g);
+        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      return true;
+    };
+
     bool ok = true;
     int hc = 0, k = 0;
+    int pv_amx = -1, pv_amn = 0;        // the previous tile's read-out state
+    float pv_kinv = 0.0f;
     for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
       int bh, qt;
       q_tile_of(p, t, bh, qt);
@@ -828,36 +1026,19 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const bool row_ok = qrow < p.S;
       const int L = p.causal ? min(qrow + 1, p.S) : p.S;
       const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-      // ---- per-row setup: this group's share of delta = dO_r . O_r, the
-      // row constants and this group's table entries
-      {
-        const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
-        const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
-        part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
-      }
-      const size_t trow = tile_row(p, bh, qt, row);
-      RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, tq_base);
-      mbar_arrive(bars.tab_ready);
-      ok = warp_all_b(mbar_wait(bars.tab_ready, k & 1, abort));
+      ok = warp_all_b(mbar_wait(bars.tab_full, k & 1, abort));
       if (!ok) break;
-      const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
-      if (MAP == MAPB_EXACT) {
-        kc.ds_ = delta;
-      } else {
-        kc.nDZ = -__fmul_rn(delta, kc.invZ);
-      }
-      if (g == 0 && row_ok) store_row_constants(p, trow, kc);
       // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) -
       // bits(M) + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M)
       // (hard), M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
       DqK dk;
-      dk.a = kc.a;
-      dk.b = kc.b;
-      dk.invZ = kc.invZ;
-      dk.nDZ = kc.nDZ;
-      dk.ne0 = -kc.e0;
-      dk.nds = -kc.ds_;
-      dk.kinv = kc.kinv;
+      dk.a = lds_f32(ca);
+      dk.b = lds_f32(ca + 8);
+      dk.invZ = lds_f32(ca + 16);
+      dk.nDZ = lds_f32(ca + 24);
+      dk.ne0 = lds_f32(ca + 32);
+      dk.nds = lds_f32(ca + 40);
+      dk.kinv = lds_f32(ca + 48);
       dk.cL2E = p.cL2E;
       dk.Kf = Kf;
       dk.tq_row = (MAP == MAPB_INTERP)
@@ -903,94 +1084,44 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_arrive(&bars.ds_full[x]);
       }
       if (!ok) break;
-      // ---- epilogue: the row's calibration sums, dQ.  The key rows of the
-      // row's argmax / argmin and its own query row are fetched first, so
-      // their latency overlaps the waits for the other groups and the last
-      // product.
-      const bool cal_row = CAL != CAL_OFF && kc.calib && row_ok;
-      const size_t head = static_cast<size_t>(bh) * p.S;
-      int amx = 0, amn = 0;
-      uint4 kaw[2] = {}, kbw[2] = {}, qw[2] = {};
-      if (cal_row) {
+      // The tile's constants and table are no longer read.  The next bulk copy
+      // (async proxy) overwrites them, so every value read from them is
+      // consumed by an instruction ahead of the release -- the sums the last
+      // table reads feed, the calibration flag (a load whose result is still
+      // in flight is not ordered by the arrive) -- and a proxy fence orders
+      // those reads before the copy.
+      const bool calib = CAL != CAL_OFF && row_ok && cstf[14] != 0.0f;
+      asm volatile("" ::"f"(s1.x), "f"(s1.y), "f"(s2.x), "f"(s2.y), "r"(calib ? 1 : 0)
+                   : "memory");
+      fence_async_smem();
+      mbar_arrive(bars.tab_free);
+      // this row's argmax / argmin key, needed at the tile's read-out (after
+      // the next tile's halves)
+      int amx = -1, amn = 0;
+      if (calib) {
         amx = p.amax[ri];
-        const uint4 *ka = reinterpret_cast<const uint4 *>(p.K_ + (head + amx) * D + 16 * g);
-        const uint4 *qr = reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g);
-        kaw[0] = ka[0];
-        kaw[1] = ka[1];
-        qw[0] = qr[0];
-        qw[1] = qr[1];
-        if (CAL == CAL_MINMAX) {
-          amn = p.amin[ri];
-          const uint4 *kb = reinterpret_cast<const uint4 *>(p.K_ + (head + amn) * D + 16 * g);
-          kbw[0] = kb[0];
-          kbw[1] = kb[1];
-        }
+        if (CAL == CAL_MINMAX) amn = p.amin[ri];
       }
-      part[(4 + g) * 128 + row] = s1.x + s1.y;
-      part[(8 + g) * 128 + row] = s2.x + s2.y;
-      mbar_arrive(bars.part_ready);
-      ok = warp_all_b(mbar_wait(bars.part_ready, k & 1, abort));
-      if (ok) ok = warp_all_b(mbar_wait(bars.dq_full, k & 1, abort));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16_sync(lane_base + T_DQ + 16 * g, v);
-      // dQ is in registers: the next tile's dQ products may start
-      tc_fence_before();
-      mbar_arrive(bars.dq_free);
-      float xq[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[i]) * p.c;
-      if (cal_row) {
-        const float S1 = (part[512 + row] + part[640 + row]) + (part[768 + row] + part[896 + row]);
-        const float S2 =
-            (part[1024 + row] + part[1152 + row]) + (part[1280 + row] + part[1408 + row]);
-        float dhi, dlo;
-        if (CAL == CAL_FIXED) {
-          dhi = -(Kf / p.window) * S2;
-          dlo = 0.0f;
-        } else if (MAP == MAPB_HARD) {
-          dhi = S1;
-          dlo = -S1;
-        } else {
-          dhi = S1;
-          dlo = -S1 - kc.kinv * S2;
-        }
-        // rank-one calibration terms in fp32: dQ_r += c (dhi k_argmax + dlo
-        // k_argmin), and dK_argmax += c dhi q_r, dK_argmin += c dlo q_r into
-        // the fp32 calibration part of dK (rows can share a key: vector
-        // reductions)
-        const float sh = p.c * dhi, sl = p.c * dlo;
-        float kx[16], qx[16];
-        bf16x16_to_f32(kaw, kx);
-        bf16x16_to_f32(qw, qx);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
-        float *da = p.dkcal + (head + amx) * D + 16 * g;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
-                                                sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
-        if (CAL == CAL_MINMAX) {
-          bf16x16_to_f32(kbw, kx);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
-          float *db = p.dkcal + (head + amn) * D + 16 * g;
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
-                                                  sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
-        }
+      // the calibration sums, once the buffer's previous tile (k - 2) has been
+      // read out
+      if (k >= 2) {
+        ok = warp_all_b(mbar_wait(&bars.part_free[k & 1], ((k >> 1) - 1) & 1, abort));
+        if (!ok) break;
       }
-      uint32_t pk[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(xq[2 * i], xq[2 * i + 1]);
-      if (row_ok) {
-        uint4 *d4 = reinterpret_cast<uint4 *>(p.dQ + ri * D + 16 * g);
-        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      float *pp = part + (k & 1) * 1024;
+      pp[g * 128 + row] = s1.x + s1.y;
+      pp[512 + g * 128 + row] = s2.x + s2.y;
+      mbar_arrive(&bars.part_ready[k & 1]);
+      if (k >= 1 && !read_out(t - step, k - 1, pv_amx, pv_amn, pv_kinv)) {
+        ok = false;
+        break;
       }
+      pv_amx = amx;
+      pv_amn = amn;
+      pv_kinv = dk.kinv;
     }
+    if (ok && k >= 1) read_out(static_cast<int>(blockIdx.x) + (k - 1) * step, k - 1, pv_amx,
+                               pv_amn, pv_kinv);
   }
   __syncwarp();
   tc_fence_before();
@@ -1447,23 +1578,26 @@ int sm_count() {
   if (in) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
-constexpr size_t kBarBytes = ((2 * 8 + 24) * 8 + 8 + 15) & ~static_cast<size_t>(15);
+constexpr size_t kBarBytes = ((2 * 8 + 26) * 8 + 8 + 15) & ~static_cast<size_t>(15);
 
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  // Q, dO, ns x (K, V), kHalfBufs dS buffers, table, partial sums, barriers
-  const size_t tab = (DqTab<MAP, SURR, CAL>::bytes(p.K) + 15) & ~static_cast<size_t>(15);
-  const size_t part = 3 * 4 * 128 * sizeof(float);
+  // Q, dO, ns x (K, V), kHalfBufs dS buffers, constants, table, two tiles'
+  // calibration sums, barriers
+  const size_t tab = (static_cast<size_t>(p.tabq_tile) + 15) & ~static_cast<size_t>(15);
+  const size_t cst = 128 * kCst * sizeof(float);
+  const size_t part = 2 * 2 * 4 * 128 * sizeof(float);
   const size_t fixed =
-      1024 + 2 * G::TILE_BYTES + kHalfBufs * 128 * 128 + tab + part + kBarBytes;
+      1024 + 2 * G::TILE_BYTES + kHalfBufs * 128 * 128 + cst + tab + part + kBarBytes;
   int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
   if (ns > 4) ns = 4;
   if (ns < 2) return QSM_ERR_UNSUPPORTED;
   p.num_stages = ns;
   p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
-  p.tab_off = p.ds_off + kHalfBufs * 128 * 128;
+  p.cst_off = p.ds_off + kHalfBufs * 128 * 128;
+  p.tab_off = static_cast<uint32_t>(p.cst_off + cst);
   p.part_off = static_cast<uint32_t>(p.tab_off + tab);
   p.bar_off = static_cast<uint32_t>(p.part_off + part);
   size_t smem = 1024 + p.bar_off + kBarBytes;
@@ -1508,9 +1642,27 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
 }
 
 template <int D, int MAP, int SURR, int CAL>
-qsm_status launch_passes(const BwdArgs &a, const BwdParams &p, const CUtensorMap &mq,
+qsm_status launch_prep(const BwdArgs &a, const BwdParams &p) {
+  // the tile's dQ-pass table, then the four groups' delta parts
+  const size_t smem =
+      1024 + ((static_cast<size_t>(p.tabq_tile) + 15) & ~static_cast<size_t>(15)) +
+      4 * 128 * sizeof(float);
+  if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
+  auto kern = qsm_bwd_prep<D, MAP, SURR, CAL>;
+  static std::atomic<int> cache[kMaxDevices];
+  if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
+  kern<<<dim3(p.nqt * a.B * a.H), kMainMapThreads, smem, a.stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+}
+
+template <int D, int MAP, int SURR, int CAL>
+qsm_status launch_passes(const BwdArgs &a, const BwdParams &p0, const CUtensorMap &mq,
                          const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
-  const qsm_status st = launch_dq<D, MAP, SURR, CAL>(a, p, mq, mk, mv, mdo);
+  BwdParams p = p0;
+  p.tabq_tile = static_cast<uint32_t>(DqTab<MAP, SURR, CAL>::bytes(p.K));
+  qsm_status st = launch_prep<D, MAP, SURR, CAL>(a, p);
+  if (st != QSM_OK) return st;
+  st = launch_dq<D, MAP, SURR, CAL>(a, p, mq, mk, mv, mdo);
   if (st != QSM_OK) return st;
   return launch_dkdv<D, MAP, SURR>(a, p, mq, mk, mv, mdo);
 }
@@ -1540,6 +1692,9 @@ qsm_status launch_rows(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
 }
 
 constexpr int kTabKT = (kBwdMaxK + 2) & ~1;              // float2 entries per row, workspace
+// bytes of one query tile's dQ-pass table at the largest K (interpolation
+// with min-max calibration: K + 2 entries of 16 bytes per row)
+constexpr size_t kTabQTile = static_cast<size_t>(kBwdMaxK + 2) * 16 * 128;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -1548,11 +1703,14 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 size_t bwd_workspace_bytes(int B, int H, int S, int D) {
   // fp32 calibration part of dK and the row workspace per query row, then
   // per tile row (each head's rows padded to whole 128-row tiles) the map
-  // constants and the dK / dV pass's grid table; each part 256-byte aligned
+  // constants and the dK / dV pass's grid table, and per query tile the dQ
+  // pass's table; each part 256-byte aligned
   const size_t rows = static_cast<size_t>(B) * H * S;
-  const size_t trows = static_cast<size_t>(B) * H * ((S + 127) / 128) * 128;
+  const size_t tiles = static_cast<size_t>(B) * H * ((S + 127) / 128);
+  const size_t trows = tiles * 128;
   return align256(rows * D * sizeof(float)) + align256(rows * kRowWs * sizeof(float)) +
-         align256(trows * kCst * sizeof(float)) + align256(trows * kTabKT * sizeof(float2));
+         align256(trows * kCst * sizeof(float)) + align256(trows * kTabKT * sizeof(float2)) +
+         align256(tiles * kTabQTile);
 }
 
 qsm_status launch_bwd(const BwdArgs &a) {
@@ -1597,10 +1755,12 @@ qsm_status launch_bwd(const BwdArgs &a) {
   const size_t o_cst = o_rw + align256(rows * kRowWs * sizeof(float));
   const size_t trows = static_cast<size_t>(p.BH) * p.nqt * 128;
   const size_t o_tab = o_cst + align256(trows * kCst * sizeof(float));
+  const size_t o_tabq = o_tab + align256(trows * kTabKT * sizeof(float2));
   p.dkcal = calib ? reinterpret_cast<float *>(ws + o_dk) : nullptr;
   p.rowws = reinterpret_cast<float *>(ws + o_rw);
   p.cst = reinterpret_cast<float *>(ws + o_cst);
   p.tabk = reinterpret_cast<float *>(ws + o_tab);
+  p.tabq = ws + o_tabq;
   p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
   p.K_ = static_cast<const __nv_bfloat16 *>(a.K);
   p.O = static_cast<const __nv_bfloat16 *>(a.O);
