@@ -465,13 +465,10 @@ struct DqTab {
   }
 };
 
-// Build this thread's row constants and its group's entries of the row's
-// tables (entries g, g + 4, ...), both for the dQ pass (shared memory at
-// tq_base) and, when row_ok, for the dK / dV pass (workspace).
+// The constants of one query row before delta is known, and (K-interval) its
+// grid map.
 template <int MAP, int SURR, int CAL>
-__device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, size_t trow, int g,
-                                              int row, bool row_ok, uint32_t tq_base) {
-  using T = DqTab<MAP, SURR, CAL>;
+__device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, RowMap &rm) {
   RowC k;
   k.a = k.b = k.invZ = k.nDZ = k.e0 = k.ds_ = k.kinv = 0.0f;
   k.calib = false;
@@ -487,51 +484,12 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, siz
     k.b = __fmul_rn(hi, log2e_f());
     k.e0 = k.b;
   } else {
-    const RowMap rm =
-        make_rowmap(hi, p.lo != nullptr ? p.lo[ri] : hi, p.K, p.fixed_window != 0, p.window);
+    rm = make_rowmap(hi, p.lo != nullptr ? p.lo[ri] : hi, p.K, p.fixed_window != 0, p.window);
     k.a = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
     k.b = rm.degenerate ? static_cast<float>(p.K) : rm.b;
     k.e0 = rm.hiL2E;
     k.kinv = rm.inv;
     k.calib = CAL != CAL_OFF && !rm.degenerate;
-    const float Kf = static_cast<float>(p.K);
-    float *tk = p.tabk + trow * p.TS;
-    if (MAP == MAPB_INTERP) {
-      const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(hi, rm.lo));
-      for (int i = g; i <= p.K + 1; i += 4) {
-        float e, d, A = 0.0f, B = 0.0f;
-        if (i == 0 && p.fixed_window) {
-          e = p.flush ? 0.0f : grid_value(rm, p.K, 0);
-          d = 0.0f;
-        } else {
-          const int kk = min(max(i - 1, 0), p.K - 1);
-          const float gk = grid_value(rm, p.K, kk), gk1 = grid_value(rm, p.K, kk + 1);
-          const float kf = static_cast<float>(kk), kmk = static_cast<float>(p.K - kk);
-          d = __fsub_rn(gk1, gk);
-          e = __fmaf_rn(-kf, d, gk);
-          if (CAL == CAL_MINMAX) {
-            A = -__fdiv_rn(__fmaf_rn(kmk, e, __fmul_rn(kf, gk1)), Kf);
-            B = __fsub_rn(-__fmul_rn(d, inv_a), __fdiv_rn(__fsub_rn(__fmul_rn(kmk, d), gk1), Kf));
-          }
-        }
-        if (row_ok) {
-          tk[2 * i] = e;
-          tk[2 * i + 1] = d;
-        }
-        if (CAL == CAL_MINMAX)
-          sts_f32x4(tq_base + i * T::STRIDE + row * 16, make_float4(A, B, d, 0.0f));
-        else if (T::ANY)
-          sts_f32(tq_base + i * T::STRIDE + row * 4, d);
-      }
-    } else {
-      for (int n = g; n <= p.K; n += 4) {
-        const float gn = grid_value(rm, p.K, n);
-        if (row_ok) tk[n] = gn;
-        if (T::ANY)
-          sts_f32(tq_base + n * T::STRIDE + row * 4,
-                  __fmul_rn(__fdiv_rn(static_cast<float>(n - p.K), Kf), gn));
-      }
-    }
   }
   if (SURR == SURR_POST) {
     const float *w = p.rowws + ri * kRowWs;
@@ -541,52 +499,112 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, siz
   return k;
 }
 
+// The grid tables of one row (K-interval): the dK / dV pass's row tk (TS
+// floats) and the dQ pass's entries, entry i at byte tq + i * STRIDE.  The
+// grid values g_k are formed first, all independent (the loop is unrolled
+// to the largest K, guarded by K), and each serves the two intervals it
+// bounds; x/K is a product with 1/K when K is a power of two (exact, so the
+// same value).
+template <int MAP, int SURR, int CAL>
+__device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm, float *tk,
+                                           uint8_t *tq) {
+  using T = DqTab<MAP, SURR, CAL>;
+  const int K = p.K;
+  const float Kf = static_cast<float>(K);
+  const bool p2 = (K & (K - 1)) == 0;
+  const float rK = 1.0f / Kf;
+  auto divK = [&](float x) { return p2 ? __fmul_rn(x, rK) : __fdiv_rn(x, Kf); };
+  float gv[kBwdMaxK + 1];
+#pragma unroll
+  for (int n = 0; n <= kBwdMaxK; ++n) gv[n] = n <= K ? grid_value(rm, K, n) : 0.0f;
+  if (MAP == MAPB_INTERP) {
+    const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(rm.hi, rm.lo));
+    auto put = [&](int i, float e, float d, float A, float B) {
+      *reinterpret_cast<float2 *>(tk + 2 * i) = make_float2(e, d);
+      if (CAL == CAL_MINMAX)
+        *reinterpret_cast<float4 *>(tq + i * T::STRIDE) = make_float4(A, B, d, 0.0f);
+      else if (T::ANY)
+        *reinterpret_cast<float *>(tq + i * T::STRIDE) = d;
+    };
+    // below the window: fixed window g_0 (0 when flushed), no derivative
+    if (p.fixed_window) put(0, p.flush ? 0.0f : gv[0], 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int kk = 0; kk < kBwdMaxK; ++kk) {
+      if (kk < K) {
+        const float gk = gv[kk], gk1 = gv[kk + 1];
+        const float kf = static_cast<float>(kk), kmk = static_cast<float>(K - kk);
+        const float d = __fsub_rn(gk1, gk);
+        const float e = __fmaf_rn(-kf, d, gk);
+        float A = 0.0f, B = 0.0f;
+        if (CAL == CAL_MINMAX) {
+          A = -divK(__fmaf_rn(kmk, e, __fmul_rn(kf, gk1)));
+          B = __fsub_rn(-__fmul_rn(d, inv_a), divK(__fsub_rn(__fmul_rn(kmk, d), gk1)));
+        }
+        put(kk + 1, e, d, A, B);
+        if (kk == 0 && !p.fixed_window) put(0, e, d, A, B);   // min-max: below = interval 0
+        if (kk == K - 1) put(K + 1, e, d, A, B);              // u = K: interval K - 1
+      }
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n <= kBwdMaxK; ++n) {
+      if (n <= K) {
+        tk[n] = gv[n];
+        if (T::ANY)
+          *reinterpret_cast<float *>(tq + n * T::STRIDE) =
+              __fmul_rn(divK(static_cast<float>(n - K)), gv[n]);
+      }
+    }
+  }
+}
+
 // ----------------------------------------------------------- row prep
-// One CTA per 128-row query tile, four threads per row (group g owns
-// columns 16g .. 16g+15 of delta = dO_r . O_r and table entries g, g + 4,
-// ...): each row's delta, map constants and grid tables, written to the
-// workspace -- the constants (both passes), the dK / dV pass's table per
-// row, and the dQ pass's table per tile in its shared-memory layout, which
-// the dQ pass copies in with one bulk load per tile.  Rows past S in a
-// ragged last tile take the last row's values, so every workspace entry of a
-// tile is defined.
+// One CTA of 128 threads per query tile, thread = row: each row's delta =
+// dO_r . O_r, map constants and grid tables, written to the workspace -- the
+// constants (both passes), the dK / dV pass's table per row and the dQ
+// pass's table per tile in its shared-memory layout (entry-major, so the
+// rows of a warp store one contiguous run), which the dQ pass copies in with
+// one bulk load per tile.  Rows past S in a ragged last tile take the last
+// row's values, so every workspace entry of a tile is defined.
 template <int D, int MAP, int SURR, int CAL>
-__global__ void __launch_bounds__(kMainMapThreads)
+__global__ void __launch_bounds__(128, 4)
     qsm_bwd_prep(const BwdParams p) {
   using T = DqTab<MAP, SURR, CAL>;
-  static_assert(D == 64, "delta slices of the four groups: 16 columns each");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = smem_align1024(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = warp >> 2;
-  const int row = (warp & 3) * 32 + lane;
+  static_assert(D == 64, "delta in four 16-column parts");
+  const int row = threadIdx.x;
   const int tix = static_cast<int>(blockIdx.x);         // bh * nqt + qt
   const int bh = tix / p.nqt, qt = tix - bh * p.nqt;
   const int qrow = qt * 128 + row;
   const bool row_ok = qrow < p.S;
   const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-  const size_t tbytes = T::bytes(p.K);
-  float *part = reinterpret_cast<float *>(smem + ((tbytes + 15) & ~static_cast<size_t>(15)));
+  // delta in four 16-column parts, summed pairwise
+  float part[4];
   {
-    const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D + 16 * g);
-    const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D + 16 * g);
-    part[g * 128 + row] = dot_bf16x8(o4[1], d4[1], dot_bf16x8(o4[0], d4[0], 0.0f));
+    const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D);
+    const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D);
+    uint4 ov[8], dv[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      ov[i] = o4[i];
+      dv[i] = d4[i];
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      part[g] = dot_bf16x8(ov[2 * g + 1], dv[2 * g + 1], dot_bf16x8(ov[2 * g], dv[2 * g], 0.0f));
   }
-  const size_t trow = tile_row(p, bh, qt, row);
-  RowC kc = row_constants<MAP, SURR, CAL>(p, ri, trow, g, row, row_ok, smem_u32(smem));
-  __syncthreads();
-  const float delta = (part[row] + part[128 + row]) + (part[256 + row] + part[384 + row]);
+  const float delta = (part[0] + part[1]) + (part[2] + part[3]);
+  RowMap rm{};
+  RowC kc = row_constants<MAP, SURR, CAL>(p, ri, rm);
   if (MAP == MAPB_EXACT)
     kc.ds_ = delta;
   else
     kc.nDZ = -__fmul_rn(delta, kc.invZ);
   if (!row_ok) kc.calib = false;
-  if (g == 0) store_row_constants(p, trow, kc);
-  if (T::ANY) {
-    const uint4 *s4 = reinterpret_cast<const uint4 *>(smem);
-    uint4 *d4 = reinterpret_cast<uint4 *>(p.tabq + static_cast<size_t>(tix) * p.tabq_tile);
-    for (size_t i = threadIdx.x; i < tbytes / 16; i += kMainMapThreads) d4[i] = s4[i];
-  }
+  const size_t trow = tile_row(p, bh, qt, row);
+  store_row_constants(p, trow, kc);
+  if (MAP == MAPB_HARD || MAP == MAPB_INTERP)
+    row_tables<MAP, SURR, CAL>(p, rm, p.tabk + trow * p.TS,
+                               p.tabq + static_cast<size_t>(tix) * p.tabq_tile + row * T::ESZ);
 }
 
 __device__ __forceinline__ float2 ex2_pair(float2 x) {
@@ -1643,15 +1661,7 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
 
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_prep(const BwdArgs &a, const BwdParams &p) {
-  // the tile's dQ-pass table, then the four groups' delta parts
-  const size_t smem =
-      1024 + ((static_cast<size_t>(p.tabq_tile) + 15) & ~static_cast<size_t>(15)) +
-      4 * 128 * sizeof(float);
-  if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
-  auto kern = qsm_bwd_prep<D, MAP, SURR, CAL>;
-  static std::atomic<int> cache[kMaxDevices];
-  if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-  kern<<<dim3(p.nqt * a.B * a.H), kMainMapThreads, smem, a.stream>>>(p);
+  qsm_bwd_prep<D, MAP, SURR, CAL><<<dim3(p.nqt * a.B * a.H), 128, 0, a.stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
