@@ -201,64 +201,79 @@ __device__ __forceinline__ void bf16x16_to_f32(const uint4 (&src)[2], float (&x)
   }
 }
 
+__device__ __forceinline__ float2 ex2_pair(float2 x) {
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
 // ----------------------------------------------------------------- rows
 struct RowBars {
-  uint64_t *kv_full, *kv_empty;   // [ns]
-  uint64_t *q_full;
-  uint64_t *sd_full, *sd_empty;   // [2]
+  uint64_t *kv_full, *kv_empty;       // [ns]: K_j, V_j
+  uint64_t *q_full, *q_free;          // Q, dO of the current tile
+  uint64_t *sdp_full, *sdp_free;      // [2]: S, dP of a key tile
+  uint64_t *part_ready, *part_free;   // [2]: a tile's partial sums written / read
   uint64_t *drain;
-  uint64_t *part_ready;           // single use: partial sums written
   uint32_t *tmem_slot;
   int *abort;
 };
 
-// One CTA per 128 query rows of one (b, h); four map groups, thread = row,
-// group g taking columns 32g .. 32g+31 of every S / dP tile.  The post
-// surrogate's row statistics: LSE* = log sum_j exp(s_j) and delta* =
-// sum_j p*_j dp_j, by an online log-sum-exp in log2 units.
+// The post surrogate's row statistics: LSE* = log sum_j exp(s_j) and delta*
+// = sum_j p*_j dp_j.  The forward's row maximum hi bounds every score, so the
+// sums are taken at the fixed offset hi (no running maximum, no rescaling):
+// L = sum_j 2^(x_j), A = sum_j 2^(x_j) dp_j with x_j = (s_j - hi) log2 e, and
+// LSE* = hi + ln L, delta* = A / L.
+// Persistent like the dQ pass: one CTA per SM takes the query tiles t =
+// blockIdx.x, blockIdx.x + gridDim.x, ...; S = Q K^T and dP = dO V^T of whole
+// 128-key tiles (products of N = 128: the map here is light, so the products
+// set the pace) in TMEM pair n mod 2 (n counting key tiles across query
+// tiles; S at 256 (n mod 2), dP 128 columns on); thread = query row, map
+// group g owning keys 32g .. 32g+31 of each tile.  A query tile's sums go
+// through shared memory (buffer k mod 2), and the group-0 threads combine
+// them after the next tile's key tiles.
 template <int D>
 __global__ void __launch_bounds__(kMainThreads, 1)
     qsm_bwd_rows(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams p) {
   using G = BGeo<D>;
-  constexpr int NS = 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int bh, qt;
-  q_tile_of(p, static_cast<int>(blockIdx.x), bh, qt);
+  const int ntiles = p.nqt * p.BH;
+  const int step = static_cast<int>(gridDim.x);
+  const int ns = p.num_stages;
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
-  uint8_t *sKV = smem + 2 * G::TILE_BYTES;
+  uint8_t *sKV = smem + 2 * G::TILE_BYTES;              // ns stages of (K_j, V_j)
+  float *part = reinterpret_cast<float *>(smem + p.part_off);   // [2][2][4][128]
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   RowBars bars;
   bars.kv_full = bp;
-  bars.kv_empty = bp + NS;
-  bars.q_full = bp + 2 * NS;
-  bars.sd_full = bars.q_full + 1;
-  bars.sd_empty = bars.sd_full + 2;
-  bars.drain = bars.sd_empty + 2;
-  bars.part_ready = bars.drain + 1;
-  bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.part_ready + 1);
-  // per-row partial sums of the four groups: m2, l2, a2 ([3][4][128])
-  float *part = reinterpret_cast<float *>(smem + p.part_off);
+  bars.kv_empty = bp + ns;
+  bars.q_full = bp + 2 * ns;
+  bars.q_free = bars.q_full + 1;
+  bars.sdp_full = bars.q_free + 1;
+  bars.sdp_free = bars.sdp_full + 2;
+  bars.part_ready = bars.sdp_free + 2;
+  bars.part_free = bars.part_ready + 2;
+  bars.drain = bars.part_free + 2;
+  bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
   bars.abort = reinterpret_cast<int *>(bars.tmem_slot + 1);
   volatile int *abort = bars.abort;
-  const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
+    for (int i = 0; i < ns; ++i) {
       mbar_init(&bars.kv_full[i], 1);
       mbar_init(&bars.kv_empty[i], 1);
     }
     mbar_init(bars.q_full, 1);
+    mbar_init(bars.q_free, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.sd_full[i], 1);
-      mbar_init(&bars.sd_empty[i], kMainMapThreads);
+      mbar_init(&bars.sdp_full[i], 1);
+      mbar_init(&bars.sdp_free[i], kMainMapThreads);
+      mbar_init(&bars.part_ready[i], kMainMapThreads);
+      mbar_init(&bars.part_free[i], kMainMapThreads);
     }
     mbar_init(bars.drain, 1);
-    mbar_init(bars.part_ready, kMainMapThreads);
     *bars.abort = 0;
     fence_mbar_init();
   }
@@ -270,132 +285,165 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(bars.q_full, 2 * G::TILE_BYTES);
-      for (int ch = 0; ch < G::CHUNKS; ++ch) {
-        tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qt * 128, bh);
-        tma_load_3d(sdO + ch * G::CHUNK_BYTES, &tmdO, bars.q_full, ch * G::EPC, qt * 128, bh);
-      }
-      int it = 0;
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        for (int w = 0; w < 2 && ok; ++w) {
-          const int st = it % NS;
-          if (it >= NS) ok = mbar_wait(&bars.kv_empty[st], ((it / NS) & 1) ^ 1, abort);
+      int it = 0, k = 0;
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        // Q, dO of the previous tile are no longer read
+        if (k >= 1) ok = mbar_wait(bars.q_free, (k - 1) & 1, abort);
+        if (!ok) break;
+        mbar_expect_tx(bars.q_full, 2 * G::TILE_BYTES);
+        for (int ch = 0; ch < G::CHUNKS; ++ch) {
+          tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qt * 128, bh);
+          tma_load_3d(sdO + ch * G::CHUNK_BYTES, &tmdO, bars.q_full, ch * G::EPC, qt * 128, bh);
+        }
+        for (int j = 0; j < nkv && ok; ++j, ++it) {
+          const int st = it % ns;
+          if (it >= ns) ok = mbar_wait(&bars.kv_empty[st], ((it / ns) - 1) & 1, abort);
           if (!ok) break;
-          mbar_expect_tx(&bars.kv_full[st], G::TILE_BYTES);
-          for (int ch = 0; ch < G::CHUNKS; ++ch)
-            tma_load_3d(sKV + st * G::TILE_BYTES + ch * G::CHUNK_BYTES, w ? &tmV : &tmK,
-                        &bars.kv_full[st], ch * G::EPC, j * 128, bh);
-          ++it;
+          uint8_t *kdst = sKV + st * 2 * G::TILE_BYTES;
+          mbar_expect_tx(&bars.kv_full[st], 2 * G::TILE_BYTES);
+          for (int ch = 0; ch < G::CHUNKS; ++ch) {
+            tma_load_3d(kdst + ch * G::CHUNK_BYTES, &tmK, &bars.kv_full[st], ch * G::EPC,
+                        j * 128, bh);
+            tma_load_3d(kdst + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmV, &bars.kv_full[st],
+                        ch * G::EPC, j * 128, bh);
+          }
         }
       }
-      mbar_wait(bars.q_full, 0, abort);
-      for (int st = 0; st < NS && st < it; ++st)
-        mbar_wait(&bars.kv_full[st], (((it - st + NS - 1) / NS) - 1) & 1, abort);
+      // every load issued must land before the CTA may exit
+      if (k >= 1) mbar_wait(bars.q_full, (k - 1) & 1, abort);
+      for (int st = 0; st < ns && st < it; ++st)
+        mbar_wait(&bars.kv_full[st], (((it - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
+    // S = Q K_j^T and dP = dO V_j^T of key tile j into TMEM pair n mod 2,
+    // once the map threads have read the pair's previous use
     if (lane == 0) {
-      bool ok = mbar_wait(bars.q_full, 0, abort);
-      tc_fence_after();
-      int it = 0;
+      bool ok = true;
+      int it0 = 0, k = 0;
       const uint32_t qa = smem_u32(sQ), da = smem_u32(sdO), kva = smem_u32(sKV);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int b = j & 1, use = j >> 1;
-        if (use >= 1) {
-          ok = mbar_wait(&bars.sd_empty[b], (use - 1) & 1, abort);
+      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+        int bh, qt;
+        q_tile_of(p, t, bh, qt);
+        const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+        ok = mbar_wait(bars.q_full, k & 1, abort);
+        tc_fence_after();
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int n = it0 + j, x = n & 1, u = n >> 1;
+          ok = mbar_wait(&bars.kv_full[n % ns], (n / ns) & 1, abort);
+          if (ok && u >= 1) ok = mbar_wait(&bars.sdp_free[x], (u - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
+          const uint32_t kb = kva + (n % ns) * 2 * G::TILE_BYTES;
+          mma_nt<D>(tmem + 256 * x, qa, kb);
+          mma_nt<D>(tmem + 256 * x + 128, da, kb + G::TILE_BYTES);
+          mma_commit(&bars.sdp_full[x]);
+          mma_commit(&bars.kv_empty[n % ns]);
         }
-        const int ks = it % NS;
-        ok = mbar_wait(&bars.kv_full[ks], (it / NS) & 1, abort);
-        ++it;
-        const int vs = it % NS;
-        ok = ok && mbar_wait(&bars.kv_full[vs], (it / NS) & 1, abort);
-        ++it;
-        if (!ok) break;
-        tc_fence_after();
-        mma_nt<D>(tmem + b * 256, qa, kva + ks * G::TILE_BYTES);
-        mma_nt<D>(tmem + b * 256 + 128, da, kva + vs * G::TILE_BYTES);
-        mma_commit(&bars.sd_full[b]);
-        mma_commit(&bars.kv_empty[ks]);
-        mma_commit(&bars.kv_empty[vs]);
+        if (ok) mma_commit(bars.q_free);                // the tile's Q, dO are read
+        it0 += nkv;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
     }
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;                       // map group: columns 32g..32g+31
+    const int g = (warp - 4) >> 2;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int qrow = qt * 128 + row;
-    const bool row_ok = qrow < p.S;
-    const int L = p.causal ? min(qrow + 1, p.S) : p.S;
-    const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-    // m2: running max of x = r c log2e; l2 = sum 2^(x - m2); a2 = sum 2^(x - m2) dp
-    float m2 = -INFINITY, l2 = 0.0f, a2 = 0.0f;
-    bool ok = true;
-    uint32_t cnt[2] = {0, 0};
-    const int c0 = 32 * g;
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int b = j & 1;
-      ok = warp_all_b(mbar_wait(&bars.sd_full[b], cnt[b] & 1, abort));
-      ++cnt[b];
-      if (!ok) break;
-      tc_fence_after();
-      const int lim = L - 128 * j - c0;            // valid columns of this group
-      uint32_t sv[32], dv[32];
-      tmem_ld32(lane_base + b * 256 + c0, sv);
-      tmem_ld32(lane_base + b * 256 + 128 + c0, dv);
-      tmem_wait_ld();
-      reg_fence32(sv);
-      reg_fence32(dv);
-      // values in registers: hand the buffers back first
-      tc_fence_before();
-      mbar_arrive(&bars.sd_empty[b]);
-      float cm = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i < lim) cm = fmaxf(cm, __fmul_rn(__uint_as_float(sv[i]), p.cL2E));
-      if (cm > m2) {
-        const float sc = ex2_approx(__fsub_rn(m2, cm));
-        l2 *= sc;
-        a2 *= sc;
-        m2 = cm;
-      }
-      if (m2 > -INFINITY) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (i < lim) {
-            const float e = ex2_approx(__fmaf_rn(__uint_as_float(sv[i]), p.cL2E, -m2));
-            l2 += e;
-            a2 = __fmaf_rn(e, __uint_as_float(dv[i]), a2);
+    const float2 cl2 = make_float2(p.cL2E, p.cL2E);
+    // A finished tile (position kp, tile t): the group-0 thread of each row
+    // combines the four groups' sums; every map thread then releases the
+    // buffer.
+    auto finish = [&](int t, int kp, float hi) -> bool {
+      const int x = kp & 1;
+      bool rok = true;
+      if (g == 0) {
+        rok = warp_all_b(mbar_wait(&bars.part_ready[x], static_cast<uint32_t>(kp >> 1) & 1u, abort));
+        if (rok) {
+          int bh, qt;
+          q_tile_of(p, t, bh, qt);
+          const int qrow = qt * 128 + row;
+          const float *pp = part + x * 1024;
+          const float Ls = (pp[row] + pp[128 + row]) + (pp[256 + row] + pp[384 + row]);
+          const float As = (pp[512 + row] + pp[640 + row]) + (pp[768 + row] + pp[896 + row]);
+          // the loaded sums are consumed before the release
+          asm volatile("" ::"f"(Ls), "f"(As) : "memory");
+          if (qrow < p.S) {
+            float *w = p.rowws + (static_cast<size_t>(bh) * p.S + qrow) * kRowWs;
+            w[RW_LSESTAR] = hi + logf(Ls);
+            w[RW_DELTASTAR] = As / Ls;
           }
         }
       }
-    }
-    // merge the four groups' partial sums at their common maximum
-    part[(0 * 4 + g) * 128 + row] = m2;
-    part[(1 * 4 + g) * 128 + row] = l2;
-    part[(2 * 4 + g) * 128 + row] = a2;
-    mbar_arrive(bars.part_ready);
-    if (ok) ok = warp_all_b(mbar_wait(bars.part_ready, 0, abort));
-    if (ok && row_ok && g == 0) {
-      float M = -INFINITY;
+      mbar_arrive(&bars.part_free[x]);
+      return rok;
+    };
+    auto row_hi = [&](int t) -> float {
+      int bh, qt;
+      q_tile_of(p, t, bh, qt);
+      return p.hi[static_cast<size_t>(bh) * p.S + min(qt * 128 + row, p.S - 1)];
+    };
+    bool ok = true;
+    int n = 0, k = 0;
+    float pv_hi = 0.0f;
+    float hi_next = static_cast<int>(blockIdx.x) < ntiles ? row_hi(blockIdx.x) : 0.0f;
+    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      int bh, qt;
+      q_tile_of(p, t, bh, qt);
+      const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
+      const int qrow = qt * 128 + row;
+      const int L = p.causal ? min(qrow + 1, p.S) : p.S;
+      const float hi = hi_next;
+      if (t + step < ntiles) hi_next = row_hi(t + step);     // consumed a tile later
+      const float hl = __fmul_rn(hi, log2e_f());
+      const float2 nh = make_float2(-hl, -hl);
+      float2 l2 = make_float2(0.0f, 0.0f), a2 = make_float2(0.0f, 0.0f);
+      for (int j = 0; j < nkv && ok; ++j, ++n) {
+        const int x = n & 1, u = n >> 1;
+        ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sv[32], dv[32];
+        tmem_ld32(lane_base + 256 * x + 32 * g, sv);
+        tmem_ld32(lane_base + 256 * x + 128 + 32 * g, dv);
+        tmem_wait_ld();
+        reg_fence32(sv);
+        reg_fence32(dv);
+        tc_fence_before();
+        mbar_arrive(&bars.sdp_free[x]);                // the pair can take key tile n + 2
+        const int lim = L - (128 * j + 32 * g);        // valid keys of this slice
 #pragma unroll
-      for (int gg = 0; gg < 4; ++gg) M = fmaxf(M, part[gg * 128 + row]);
-      float Ls = 0.0f, As = 0.0f;
-#pragma unroll
-      for (int gg = 0; gg < 4; ++gg) {
-        const float mg = part[gg * 128 + row];
-        if (mg == -INFINITY) continue;             // a group with no valid column
-        const float sc = ex2_approx(__fsub_rn(mg, M));
-        Ls = __fmaf_rn(part[(4 + gg) * 128 + row], sc, Ls);
-        As = __fmaf_rn(part[(8 + gg) * 128 + row], sc, As);
+        for (int i2 = 0; i2 < 16; ++i2) {
+          const float2 r = make_float2(__uint_as_float(sv[2 * i2]), __uint_as_float(sv[2 * i2 + 1]));
+          const float2 dp =
+              make_float2(__uint_as_float(dv[2 * i2]), __uint_as_float(dv[2 * i2 + 1]));
+          float2 ev = ex2_pair(fma2_rn(r, cl2, nh));
+          if (2 * i2 >= lim) ev.x = 0.0f;
+          if (2 * i2 + 1 >= lim) ev.y = 0.0f;
+          l2 = add2_rn(l2, ev);
+          a2 = fma2_rn(ev, dp, a2);
+        }
       }
-      float *w = p.rowws + ri * kRowWs;
-      w[RW_LSESTAR] = M * 0.6931471805599453f + logf(Ls);
-      w[RW_DELTASTAR] = As / Ls;
+      if (!ok) break;
+      // this tile's sums, once the buffer's previous tile (k - 2) is combined
+      if (k >= 2) {
+        ok = warp_all_b(mbar_wait(&bars.part_free[k & 1], ((k >> 1) - 1) & 1, abort));
+        if (!ok) break;
+      }
+      float *pp = part + (k & 1) * 1024;
+      pp[g * 128 + row] = l2.x + l2.y;
+      pp[512 + g * 128 + row] = a2.x + a2.y;
+      mbar_arrive(&bars.part_ready[k & 1]);
+      if (k >= 1 && !finish(t - step, k - 1, pv_hi)) {
+        ok = false;
+        break;
+      }
+      pv_hi = hi;
     }
+    if (ok && k >= 1) finish(static_cast<int>(blockIdx.x) + (k - 1) * step, k - 1, pv_hi);
   }
   __syncwarp();
   tc_fence_before();
@@ -605,10 +653,6 @@ __global__ void __launch_bounds__(128, 4)
   if (MAP == MAPB_HARD || MAP == MAPB_INTERP)
     row_tables<MAP, SURR, CAL>(p, rm, p.tabk + trow * p.TS,
                                p.tabq + static_cast<size_t>(tix) * p.tabq_tile + row * T::ESZ);
-}
-
-__device__ __forceinline__ float2 ex2_pair(float2 x) {
-  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
 }
 
 // The dQ pass's per-row values for the element loop.
@@ -1689,15 +1733,25 @@ template <int D>
 qsm_status launch_rows(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
                        const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  p.part_off = static_cast<uint32_t>(2 * G::TILE_BYTES + 4 * G::TILE_BYTES);
-  p.bar_off = static_cast<uint32_t>(p.part_off + 3 * 4 * 128 * sizeof(float));
-  size_t smem = 1024 + p.bar_off + 256;
-  if (smem < 120 * 1024) smem = 120 * 1024;
+  // Q, dO, ns x (K, V), two tiles' partial sums, barriers
+  const size_t part = 2 * 2 * 4 * 128 * sizeof(float);
+  const size_t fixed = 1024 + 2 * G::TILE_BYTES + part + kBarBytes;
+  int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
+  if (ns > 4) ns = 4;
+  if (ns < 2) return QSM_ERR_UNSUPPORTED;
+  p.num_stages = ns;
+  p.part_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
+  p.bar_off = static_cast<uint32_t>(p.part_off + part);
+  size_t smem = 1024 + p.bar_off + kBarBytes;
+  if (smem < 120 * 1024) smem = 120 * 1024;            // one CTA per SM (all of TMEM)
   if (smem > kMaxSmem) return QSM_ERR_UNSUPPORTED;
   auto kern = qsm_bwd_rows<D>;
   static std::atomic<int> cache[kMaxDevices];
   if (!set_smem_once(kern, static_cast<int>(smem), cache)) return QSM_ERR_CUDA;
-  kern<<<dim3(p.nqt * a.B * a.H), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
+  // persistent: one CTA per SM walks the query tiles
+  const int ntiles = p.nqt * a.B * a.H;
+  const int grid = ntiles < sm_count() ? ntiles : sm_count();
+  kern<<<dim3(grid), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
