@@ -20,24 +20,28 @@
 // row).
 //
 // Kernels, in launch order on the caller's stream:
-//   1. qsm_bwd_rows   post surrogate only: LSE* and delta* per query row
-//                     (S and dP tiles swept once per query tile)
-//   2. qsm_bwd_dq     one CTA per 128-row query tile: each row's delta, map
-//                     constants and grid tables (the dK / dV pass's copies go
-//                     to the workspace), then the key tiles in halves of 64
-//                     keys: S = Q K^T and dP = dO V^T into a double-buffered
-//                     TMEM pair, dS by the rule above into shared memory,
-//                     dQ += dS K in TMEM; the calibration sums accumulate per
-//                     row; the epilogue adds the rank-one terms to dQ (fp32)
-//                     before its bf16 store and scatters the dK ones into an
-//                     fp32 buffer
-//   3. qsm_bwd_dkdv   one CTA per 128-key tile, sweeping the query tiles in
-//                     halves of 64 rows: S^T = K Q^T, dP^T = V dO^T into a
-//                     double-buffered TMEM pair, P^T and dS^T written back to
-//                     TMEM, dV += P^T dO and dK += dS^T Q in TMEM; dK gets the
-//                     fp32 calibration part before its bf16 store
+//   1. qsm_bwd_rows   post surrogate only: LSE* and delta* per query row, sums
+//                     of 2^((s - hi) log2 e) at the forward's row maximum over
+//                     whole S and dP tiles (persistent)
+//   2. qsm_bwd_prep   one CTA per query tile, thread = row: delta = dO . O, the
+//                     map constants and grid tables of both passes, into the
+//                     workspace
+//   3. qsm_bwd_dq     persistent, one CTA per SM over the query tiles: a tile's
+//                     constants and table copied in, then the key tiles in
+//                     halves of 64 keys: S = Q K^T and dP = dO V^T into one of
+//                     three TMEM pairs, dS by the rule above into shared
+//                     memory, dQ += dS K in TMEM (two accumulators, by tile
+//                     parity); the calibration sums accumulate per row.  A
+//                     tile's dQ is read out after the next tile's halves: the
+//                     rank-one terms are added to dQ (fp32) before its bf16
+//                     store and the dK ones are scattered into an fp32 buffer
+//   4. qsm_bwd_dkdv   persistent over the key tiles, sweeping the query tiles
+//                     in halves of 64 rows: S^T = K Q^T, dP^T = V dO^T into one
+//                     of three TMEM pairs, P^T and dS^T written back to TMEM,
+//                     dV += P^T dO and dK += dS^T Q in TMEM; dK gets the fp32
+//                     calibration part before its bf16 store
 // Each pass recomputes its products, so no dQ partial sums cross CTAs; the
-// double buffers let the map of one half overlap the products of the next.
+// buffered halves let the map of one half overlap the products of the next.
 // The element code is specialised per map, surrogate and calibration form,
 // so no per-element branch remains.
 #include <cuda.h>

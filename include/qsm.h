@@ -211,7 +211,7 @@ size_t qsm_attn_bwd_workspace_size(int B, int H, int S, int D);
  * Arguments and results are those of qsm_attn_bwd; opts->workspace and
  * opts->workspace_bytes are ignored.  Returns QSM_ERR_INVALID_ARG when
  * qsm_attn_bwd_workspace_size(B, H, S, D) exceeds QSM_NOALLOC_SCRATCH_BYTES
- * (for D = 64, about 28 000 query rows B*H*S), before any launch.
+ * (for D = 64, about 14 700 query rows B*H*S), before any launch.
  *
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.  The
