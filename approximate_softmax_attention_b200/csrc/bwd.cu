@@ -130,15 +130,18 @@ __device__ __forceinline__ void mma_nt(uint32_t d_tmem, uint32_t a_saddr, uint32
 }
 
 // Half tile: D[128 x 64] = A[128 x D] B[64 x D]^T, both K-major (B: 64 rows
-// of a 128-row tile, the start of a 1024-byte swizzle atom).
-template <int D>
+// at the start of a 1024-byte swizzle atom).  A is a whole 128-row tile
+// (64-column chunks 16 KB apart); B's chunks sit BCH bytes apart (16 KB
+// within a whole tile, 8 KB in a 64-row stage).
+template <int D, int BCH = 128 * 128>
 __device__ __forceinline__ void mma_nt_half(uint32_t d_tmem, uint32_t a_saddr, uint32_t b_saddr) {
   using G = BGeo<D>;
 #pragma unroll
   for (int kk = 0; kk < G::KSTEPS_D; ++kk) {
     const int e = kk * 16;
-    const uint32_t off = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * 2;
-    mma_ss_f16(d_tmem, smem_desc(a_saddr + off, 16, 1024), smem_desc(b_saddr + off, 16, 1024),
+    const uint32_t offa = (e / G::EPC) * G::CHUNK_BYTES + (e % G::EPC) * 2;
+    const uint32_t offb = (e / G::EPC) * BCH + (e % G::EPC) * 2;
+    mma_ss_f16(d_tmem, smem_desc(a_saddr + offa, 16, 1024), smem_desc(b_saddr + offb, 16, 1024),
                G::IDESC_H, kk > 0);
   }
 }
@@ -622,27 +625,33 @@ template <int D, int MAP, int SURR, int CAL>
 __global__ void __launch_bounds__(128, 4)
     qsm_bwd_prep(const BwdParams p) {
   using T = DqTab<MAP, SURR, CAL>;
-  static_assert(D == 64, "delta in four 16-column parts");
+  static_assert(D == 64 || D == 128, "delta in four D/4-column parts");
   const int row = threadIdx.x;
   const int tix = static_cast<int>(blockIdx.x);         // bh * nqt + qt
   const int bh = tix / p.nqt, qt = tix - bh * p.nqt;
   const int qrow = qt * 128 + row;
   const bool row_ok = qrow < p.S;
   const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-  // delta in four 16-column parts, summed pairwise
+  // delta in four D/4-column parts (each a running sum over its 8-column
+  // chunks), summed pairwise
+  constexpr int CPP = D / 32;                             // 8-column chunks per part
   float part[4];
   {
     const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D);
     const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D);
-    uint4 ov[8], dv[8];
+    uint4 ov[D / 8], dv[D / 8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < D / 8; ++i) {
       ov[i] = o4[i];
       dv[i] = d4[i];
     }
 #pragma unroll
-    for (int g = 0; g < 4; ++g)
-      part[g] = dot_bf16x8(ov[2 * g + 1], dv[2 * g + 1], dot_bf16x8(ov[2 * g], dv[2 * g], 0.0f));
+    for (int g = 0; g < 4; ++g) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int c = 0; c < CPP; ++c) acc = dot_bf16x8(ov[CPP * g + c], dv[CPP * g + c], acc);
+      part[g] = acc;
+    }
   }
   const float delta = (part[0] + part[1]) + (part[2] + part[3]);
   RowMap rm{};
@@ -741,8 +750,8 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
 struct DqBars {
   uint64_t *kv_full, *kv_empty;       // [ns]: K_j, V_j
   uint64_t *q_full, *q_free;          // Q, dO of the current tile
-  uint64_t *sdp_full, *sdp_free;      // [kHalfBufs]
-  uint64_t *ds_full, *ds_free;        // [kHalfBufs]
+  uint64_t *sdp_full, *sdp_free;      // [HB]
+  uint64_t *ds_full, *ds_free;        // [HB]
   uint64_t *dq_full, *dq_free;        // [2]: a tile's dQ complete / read out of TMEM
   uint64_t *tab_full, *tab_free;      // the tile's constants and table
   uint64_t *part_ready, *part_free;   // [2]: a tile's calibration sums written / read
@@ -750,7 +759,19 @@ struct DqBars {
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr uint32_t T_DQ = 384;
+// Geometry of the dQ pass: D = 64 keeps three TMEM pairs and whole key
+// tiles per ring stage; D = 128 (accumulators of 128 columns) two pairs and
+// half key tiles (64 keys) per stage.
+template <int D>
+struct DqGeo {
+  static constexpr int HB = D > 64 ? 2 : 3;          // TMEM S / dP pairs, dS buffers
+  static constexpr int KROWS = D > 64 ? 64 : 128;    // key rows per ring stage
+  static constexpr int HPU = KROWS / 64;             // halves per stage
+  static constexpr int KBYTES = KROWS * D * 2;       // the K (or V) rows of a stage
+  static constexpr int KCHUNK = KROWS * 128;         // bytes between their 64-column chunks
+  static constexpr uint32_t T_DQ = HB * 128;         // dQ accumulators: T_DQ + D (k mod 2)
+  static constexpr int DG = D / 4;                   // dQ columns per map group
+};
 
 // The calibration state of a finished tile that its read-out needs: the
 // tile, the row's argmax / argmin key (amx < 0: no calibration terms) and
@@ -767,7 +788,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                const BwdParams p) {
   using G = BGeo<D>;
   using T = DqTab<MAP, SURR, CAL>;
-  static_assert(D == 64, "dQ slices of the four map groups: 16 columns each");
+  using QG = DqGeo<D>;
+  static_assert(D == 64 || D == 128, "dQ slices of the four map groups: D / 4 columns");
+  constexpr int HB = QG::HB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -787,10 +810,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.q_full = bp + 2 * ns;
   bars.q_free = bars.q_full + 1;
   bars.sdp_full = bars.q_free + 1;
-  bars.sdp_free = bars.sdp_full + kHalfBufs;
-  bars.ds_full = bars.sdp_free + kHalfBufs;
-  bars.ds_free = bars.ds_full + kHalfBufs;
-  bars.dq_full = bars.ds_free + kHalfBufs;
+  bars.sdp_free = bars.sdp_full + HB;
+  bars.ds_full = bars.sdp_free + HB;
+  bars.ds_free = bars.ds_full + HB;
+  bars.dq_full = bars.ds_free + HB;
   bars.dq_free = bars.dq_full + 2;
   bars.tab_full = bars.dq_free + 2;
   bars.tab_free = bars.tab_full + 1;
@@ -808,7 +831,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     }
     mbar_init(bars.q_full, 1);
     mbar_init(bars.q_free, 1);
-    for (int i = 0; i < kHalfBufs; ++i) {
+    for (int i = 0; i < HB; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.sdp_free[i], kMainMapThreads);
       mbar_init(&bars.ds_full[i], kMainMapThreads);
@@ -853,17 +876,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           tma_load_3d(sQ + ch * G::CHUNK_BYTES, &tmQ, bars.q_full, ch * G::EPC, qt * 128, bh);
           tma_load_3d(sdO + ch * G::CHUNK_BYTES, &tmdO, bars.q_full, ch * G::EPC, qt * 128, bh);
         }
-        for (int j = 0; j < nkv && ok; ++j, ++it) {
+        // one stage per KROWS keys (K / V tensor maps of KROWS-row boxes)
+        for (int j = 0; j < nkv * (128 / QG::KROWS) && ok; ++j, ++it) {
           const int st = it % ns;
           if (it >= ns) ok = mbar_wait(&bars.kv_empty[st], ((it / ns) - 1) & 1, abort);
           if (!ok) break;
-          uint8_t *kdst = sKV + st * 2 * G::TILE_BYTES;
-          mbar_expect_tx(&bars.kv_full[st], 2 * G::TILE_BYTES);
+          uint8_t *kdst = sKV + st * 2 * QG::KBYTES;
+          mbar_expect_tx(&bars.kv_full[st], 2 * QG::KBYTES);
           for (int ch = 0; ch < G::CHUNKS; ++ch) {
-            tma_load_3d(kdst + ch * G::CHUNK_BYTES, &tmK, &bars.kv_full[st], ch * G::EPC,
-                        j * 128, bh);
-            tma_load_3d(kdst + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmV, &bars.kv_full[st],
-                        ch * G::EPC, j * 128, bh);
+            tma_load_3d(kdst + ch * QG::KCHUNK, &tmK, &bars.kv_full[st], ch * G::EPC,
+                        j * QG::KROWS, bh);
+            tma_load_3d(kdst + QG::KBYTES + ch * QG::KCHUNK, &tmV, &bars.kv_full[st],
+                        ch * G::EPC, j * QG::KROWS, bh);
           }
         }
       }
@@ -874,7 +898,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_wait(&bars.kv_full[st], (((it - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair hc mod 3
+    // S = Q K_h^T and dP = dO V_h^T of half h into TMEM pair hc mod HB
     if (lane == 0) {
       bool ok = true;
       int it0 = 0, hc = 0, k = 0;
@@ -886,8 +910,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         ok = mbar_wait(bars.q_full, k & 1, abort);
         tc_fence_after();
         for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
-          const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
-          const int itj = it0 + j;
+          const int e = h % QG::HPU, x = hc % HB, u = hc / HB;
+          const int itj = it0 + h / QG::HPU;                // the half's stage
           if (e == 0) {
             ok = mbar_wait(&bars.kv_full[itj % ns], (itj / ns) & 1, abort);
             if (!ok) break;
@@ -898,13 +922,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             if (!ok) break;
             tc_fence_after();
           }
-          const uint32_t kb = kva + (itj % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
-          mma_nt_half<D>(tmem + 128 * x, qa, kb);
-          mma_nt_half<D>(tmem + 128 * x + 64, da, kb + G::TILE_BYTES);
+          const uint32_t kb = kva + (itj % ns) * 2 * QG::KBYTES + e * 64 * 128;
+          mma_nt_half<D, QG::KCHUNK>(tmem + 128 * x, qa, kb);
+          mma_nt_half<D, QG::KCHUNK>(tmem + 128 * x + 64, da, kb + QG::KBYTES);
           mma_commit(&bars.sdp_full[x]);
         }
         if (ok) mma_commit(bars.q_free);                // the tile's Q, dO are read
-        it0 += nkv;
+        it0 += 2 * nkv / QG::HPU;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -920,10 +944,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
-        const uint32_t dq = tmem + T_DQ + 64 * (k & 1);
+        const uint32_t dq = tmem + QG::T_DQ + D * (k & 1);
         for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
-          const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
-          const int itj = it0 + j;
+          const int e = h % QG::HPU, x = hc % HB, u = hc / HB;
+          const int itj = it0 + h / QG::HPU;                // the half's stage
           if (e == 0) {
             // K_j has landed (this warp reads it too; the stage cannot refill
             // before this warp's own release below)
@@ -935,18 +959,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           if (ok && h == 0 && k >= 2) ok = mbar_wait(&bars.dq_free[k & 1], ((k >> 1) - 1) & 1, abort);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kb = kva + (itj % ns) * 2 * G::TILE_BYTES + e * 64 * 128;
+          const uint32_t kb = kva + (itj % ns) * 2 * QG::KBYTES + e * 64 * 128;
           const uint32_t ab = dsa + x * 128 * 128;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss_f16(dq, smem_desc(ab + kk * 32, 16, 1024),
-                       smem_desc(kb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN,
+                       smem_desc(kb + kk * 16 * 128, QG::KCHUNK, 1024), G::IDESC_MN,
                        (h > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.ds_free[x]);
-          if (e == 1) mma_commit(&bars.kv_empty[itj % ns]);
+          if (e == QG::HPU - 1) mma_commit(&bars.kv_empty[itj % ns]);
         }
         if (ok) mma_commit(&bars.dq_full[k & 1]);
-        it0 += nkv;
+        it0 += 2 * nkv / QG::HPU;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -989,6 +1013,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // can share a key: vector reductions) -- and the bf16 store.  amx < 0:
     // the row takes no calibration terms.
     auto read_out = [&](int t, int kp, int amx, int amn, float kinv) -> bool {
+      constexpr int NP = D / 64;                         // 16-column pieces of the slice
       const int x = kp & 1;
       const uint32_t ph = static_cast<uint32_t>(kp >> 1) & 1u;
       int bh, qt;
@@ -997,27 +1022,36 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const size_t head = static_cast<size_t>(bh) * p.S;
       const size_t ri = head + min(qrow, p.S - 1);
       const bool cal_row = CAL != CAL_OFF && amx >= 0;
-      // the key rows and the query row are fetched before the waits
+      // the key rows and the query row of a piece (the first one before the
+      // waits)
       uint4 kaw[2] = {}, kbw[2] = {}, qw[2] = {};
-      if (cal_row) {
-        const uint4 *ka = reinterpret_cast<const uint4 *>(p.K_ + (head + amx) * D + 16 * g);
-        const uint4 *qr = reinterpret_cast<const uint4 *>(p.Q + ri * D + 16 * g);
-        kaw[0] = ka[0];
-        kaw[1] = ka[1];
-        qw[0] = qr[0];
-        qw[1] = qr[1];
-        if (CAL == CAL_MINMAX) {
-          const uint4 *kb = reinterpret_cast<const uint4 *>(p.K_ + (head + amn) * D + 16 * g);
-          kbw[0] = kb[0];
-          kbw[1] = kb[1];
+      auto gather = [&](int c0) {
+        if (cal_row) {
+          const uint4 *ka = reinterpret_cast<const uint4 *>(p.K_ + (head + amx) * D + c0);
+          const uint4 *qr = reinterpret_cast<const uint4 *>(p.Q + ri * D + c0);
+          kaw[0] = ka[0];
+          kaw[1] = ka[1];
+          qw[0] = qr[0];
+          qw[1] = qr[1];
+          if (CAL == CAL_MINMAX) {
+            const uint4 *kb = reinterpret_cast<const uint4 *>(p.K_ + (head + amn) * D + c0);
+            kbw[0] = kb[0];
+            kbw[1] = kb[1];
+          }
         }
-      }
+      };
+      gather(QG::DG * g);
       bool rok = warp_all_b(mbar_wait(&bars.part_ready[x], ph, abort));
       if (rok) rok = warp_all_b(mbar_wait(&bars.dq_full[x], ph, abort));
       if (!rok) return false;
       tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16_sync(lane_base + T_DQ + 64 * x + 16 * g, v);
+      uint32_t v[NP][16];
+#pragma unroll
+      for (int pc = 0; pc < NP; ++pc)
+        tmem_ld16(lane_base + QG::T_DQ + D * x + QG::DG * g + 16 * pc, v[pc]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int pc = 0; pc < NP; ++pc) reg_fence16(v[pc]);
       // the accumulator is in registers: tile kp + 2 may take the buffer
       tc_fence_before();
       mbar_arrive(&bars.dq_free[x]);
@@ -1044,38 +1078,43 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       }
       asm volatile("" ::"f"(sh), "f"(sl) : "memory");
       mbar_arrive(&bars.part_free[x]);
-      float xq[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[i]) * p.c;
-      if (cal_row) {
-        float kx[16], qx[16];
-        bf16x16_to_f32(kaw, kx);
-        bf16x16_to_f32(qw, qx);
+      for (int pc = 0; pc < NP; ++pc) {
+        const int c0 = QG::DG * g + 16 * pc;
+        if (pc > 0) gather(c0);
+        float xq[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
-        float *da = p.dkcal + (head + amx) * D + 16 * g;
+        for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[pc][i]) * p.c;
+        if (cal_row) {
+          float kx[16], qx[16];
+          bf16x16_to_f32(kaw, kx);
+          bf16x16_to_f32(qw, qx);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
-                                                sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
-        if (CAL == CAL_MINMAX) {
-          bf16x16_to_f32(kbw, kx);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
-          float *db = p.dkcal + (head + amn) * D + 16 * g;
+          for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sh, kx[i], xq[i]);
+          float *da = p.dkcal + (head + amx) * D + c0;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
-                                                  sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
-        }
-      }
-      uint32_t pk[8];
+            red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
+                                                  sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
+          if (CAL == CAL_MINMAX) {
+            bf16x16_to_f32(kbw, kx);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(xq[2 * i], xq[2 * i + 1]);
-      if (qrow < p.S) {
-        uint4 *d4 = reinterpret_cast<uint4 *>(p.dQ + ri * D + 16 * g);
-        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            for (int i = 0; i < 16; ++i) xq[i] = __fmaf_rn(sl, kx[i], xq[i]);
+            float *db = p.dkcal + (head + amn) * D + c0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
+                                                    sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
+          }
+        }
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(xq[2 * i], xq[2 * i + 1]);
+        if (qrow < p.S) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(p.dQ + ri * D + c0);
+          d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
       return true;
     };
@@ -1112,7 +1151,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                       : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
       float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
       for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
-        const int j = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
+        const int j = h >> 1, e = h & 1, x = hc % HB, u = hc / HB;
         ok = warp_all_b(mbar_wait(&bars.sdp_full[x], u & 1, abort));
         if (!ok) break;
         tc_fence_after();
@@ -1200,22 +1239,66 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 // --------------------------------------------------------------- dK/dV pass
 // Persistent: one CTA per SM takes the 128-key tiles in the heaviest-first
 // order; thread = key (TMEM lane); the query tiles are taken in halves of 64
-// rows, half number hc (counted across tiles) in TMEM pair x = hc mod 3
+// rows, half number hc (counted across tiles) in TMEM pair x = hc mod HB
 // (S^T at 128x, dP^T at 128x + 64); map group g owns rows 16g .. 16g+15 of
 // each half and writes its P^T and dS^T (bf16) into the first 8 of its own 16
-// columns, which the dV / dK products (dV at TMEM column 384, dK at 448) read
-// as their TMEM A operand.  A ring stage holds Q_i, dO_i and the tile's
-// per-row constants and grid tables.
+// columns, which the dV / dK products (dV at TMEM column T_DV, dK at T_DK)
+// read as their TMEM A operand.  A ring stage holds Q, dO rows and their
+// per-row constants and grid tables: a whole query tile at D = 64 (three
+// pairs), a half tile at D = 128, whose accumulators take twice the TMEM
+// columns (two pairs) and whose tiles twice the shared memory.
 struct KvBars {
   uint64_t *qd_full, *qd_empty;       // [ns]
   uint64_t *kv_full, *kv_free;        // K, V of the current tile
-  uint64_t *sdp_full, *pds_full, *s_free;   // [kHalfBufs]
+  uint64_t *sdp_full, *pds_full, *s_free;   // [HB]
   uint64_t *acc_full, *acc_free;      // the tile's dV, dK complete / read out of TMEM
   uint64_t *drain;
   uint32_t *tmem_slot;
   int *abort;
 };
-constexpr uint32_t T_DV = 384, T_DK = 448;
+template <int D>
+struct KvGeo {
+  static constexpr int HB = D > 64 ? 2 : 3;          // TMEM S^T / dP^T pairs
+  static constexpr int SROWS = D > 64 ? 64 : 128;    // query rows per ring stage
+  static constexpr int HPU = SROWS / 64;             // halves per stage
+  static constexpr int QBYTES = SROWS * D * 2;       // the Q (or dO) rows of a stage
+  static constexpr int QCHUNK = SROWS * 128;         // bytes between their 64-column chunks
+  static constexpr uint32_t T_DV = HB * 128, T_DK = T_DV + D;
+  static constexpr int DG = D / 4;                   // dV / dK columns per map group
+};
+
+// Sixteen fp32 TMEM values, times scale, to bf16 at d4 (two 16-byte stores);
+// with cal, its sixteen fp32 values are added first.
+__device__ __forceinline__ void store_bf16x16(uint4 *d4, const uint32_t (&v)[16], float scale) {
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * scale, __uint_as_float(v[2 * i + 1]) * scale);
+  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+__device__ __forceinline__ void store_bf16x16_cal(uint4 *d4, const uint32_t (&v)[16], float scale,
+                                                  const float *cal) {
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(v[i]) * scale;
+  if (cal != nullptr) {
+    const float4 *c4 = reinterpret_cast<const float4 *>(cal);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 c = c4[i];
+      x[4 * i] += c.x;
+      x[4 * i + 1] += c.y;
+      x[4 * i + 2] += c.z;
+      x[4 * i + 3] += c.w;
+    }
+  }
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+  d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
 
 // The dK / dV pass's per-thread values for the element loop.
 struct KvK {
@@ -1301,7 +1384,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                  const BwdParams p) {
   using G = BGeo<D>;
-  static_assert(D == 64, "dK / dV slices of the four map groups: 16 columns each");
+  using KG = KvGeo<D>;
+  static_assert(D == 64 || D == 128, "dK / dV slices of the four map groups: D / 4 columns");
+  constexpr int HB = KG::HB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1312,8 +1397,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *sV = smem + G::TILE_BYTES;
   uint8_t *sSt = smem + 2 * G::TILE_BYTES;              // ns stages: Q, dO, cst, tab
   const uint32_t SB = p.stage_bytes;
-  const uint32_t CST_OFF = 2 * G::TILE_BYTES;
-  const uint32_t TAB_OFF = CST_OFF + 128 * kCst * 4;
+  const uint32_t CST_OFF = 2 * KG::QBYTES;
+  const uint32_t TAB_OFF = CST_OFF + KG::SROWS * kCst * 4;
   uint64_t *bp = reinterpret_cast<uint64_t *>(smem + p.bar_off);
   KvBars bars;
   bars.qd_full = bp;
@@ -1321,9 +1406,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   bars.kv_full = bp + 2 * ns;
   bars.kv_free = bars.kv_full + 1;
   bars.sdp_full = bars.kv_free + 1;
-  bars.pds_full = bars.sdp_full + kHalfBufs;
-  bars.s_free = bars.pds_full + kHalfBufs;
-  bars.acc_full = bars.s_free + kHalfBufs;
+  bars.pds_full = bars.sdp_full + HB;
+  bars.s_free = bars.pds_full + HB;
+  bars.acc_full = bars.s_free + HB;
   bars.acc_free = bars.acc_full + 1;
   bars.drain = bars.acc_free + 1;
   bars.tmem_slot = reinterpret_cast<uint32_t *>(bars.drain + 1);
@@ -1337,7 +1422,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     }
     mbar_init(bars.kv_full, 1);
     mbar_init(bars.kv_free, 1);
-    for (int i = 0; i < kHalfBufs; ++i) {
+    for (int i = 0; i < HB; ++i) {
       mbar_init(&bars.sdp_full[i], 1);
       mbar_init(&bars.pds_full[i], kMainMapThreads);
       mbar_init(&bars.s_free[i], 1);
@@ -1374,22 +1459,23 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           tma_load_3d(sK + ch * G::CHUNK_BYTES, &tmK, bars.kv_full, ch * G::EPC, kt * 128, bh);
           tma_load_3d(sV + ch * G::CHUNK_BYTES, &tmV, bars.kv_full, ch * G::EPC, kt * 128, bh);
         }
-        for (int n = 0; n < nq && ok; ++n, ++rc) {
-          const int st = rc % ns, qi = i0 + n;
+        // one stage per SROWS query rows (Q / dO tensor maps of SROWS-row boxes)
+        for (int n = 0; n < nq * (128 / KG::SROWS) && ok; ++n, ++rc) {
+          const int st = rc % ns;
+          const int row0 = (i0 * 128) + n * KG::SROWS;     // first query row of the stage
           if (rc >= ns) ok = mbar_wait(&bars.qd_empty[st], ((rc / ns) - 1) & 1, abort);
           if (!ok) break;
           uint8_t *s = sSt + st * SB;
-          // the constants and tables of the tile's 128 tile rows (rows past S
-          // in a ragged last tile are never valid)
-          const size_t r0 = (static_cast<size_t>(bh) * p.nqt + qi) * 128;
-          const uint32_t cbytes = 128u * kCst * 4;
-          const uint32_t tbytes = 128u * static_cast<uint32_t>(p.TS) * 4;
-          mbar_expect_tx(&bars.qd_full[st], 2 * G::TILE_BYTES + cbytes + tbytes);
+          // the constants and tables of the stage's tile rows (rows past S in
+          // a ragged last tile are never valid)
+          const size_t r0 = static_cast<size_t>(bh) * p.nqt * 128 + row0;
+          const uint32_t cbytes = KG::SROWS * kCst * 4;
+          const uint32_t tbytes = KG::SROWS * static_cast<uint32_t>(p.TS) * 4;
+          mbar_expect_tx(&bars.qd_full[st], 2 * KG::QBYTES + cbytes + tbytes);
           for (int ch = 0; ch < G::CHUNKS; ++ch) {
-            tma_load_3d(s + ch * G::CHUNK_BYTES, &tmQ, &bars.qd_full[st], ch * G::EPC, qi * 128,
-                        bh);
-            tma_load_3d(s + G::TILE_BYTES + ch * G::CHUNK_BYTES, &tmdO, &bars.qd_full[st],
-                        ch * G::EPC, qi * 128, bh);
+            tma_load_3d(s + ch * KG::QCHUNK, &tmQ, &bars.qd_full[st], ch * G::EPC, row0, bh);
+            tma_load_3d(s + KG::QBYTES + ch * KG::QCHUNK, &tmdO, &bars.qd_full[st], ch * G::EPC,
+                        row0, bh);
           }
           bulk_load(s + CST_OFF, p.cst + r0 * kCst, cbytes, &bars.qd_full[st]);
           if (tbytes) bulk_load(s + TAB_OFF, p.tabk + r0 * p.TS, tbytes, &bars.qd_full[st]);
@@ -1401,8 +1487,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_wait(&bars.qd_full[st], (((rc - st + ns - 1) / ns) - 1) & 1, abort);
     }
   } else if (warp == 1) {
-    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair hc mod 3,
-    // once the dV / dK products of half hc - 3 have read it
+    // S^T = K Q_h^T and dP^T = V dO_h^T of half h into TMEM pair hc mod HB,
+    // once the dV / dK products of half hc - HB have read it
     if (lane == 0) {
       bool ok = true;
       int rc0 = 0, hc = 0, k = 0;
@@ -1414,8 +1500,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         ok = mbar_wait(bars.kv_full, k & 1, abort);
         tc_fence_after();
         for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
-          const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
-          const int rn = rc0 + n;
+          const int e = h % KG::HPU, x = hc % HB, u = hc / HB;
+          const int rn = rc0 + h / KG::HPU;                 // the half's stage
           if (e == 0) {
             ok = mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort);
             if (!ok) break;
@@ -1427,12 +1513,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             tc_fence_after();
           }
           const uint32_t qb = sa + (rn % ns) * SB + e * 64 * 128;
-          mma_nt_half<D>(tmem + 128 * x, ka, qb);
-          mma_nt_half<D>(tmem + 128 * x + 64, va, qb + G::TILE_BYTES);
+          mma_nt_half<D, KG::QCHUNK>(tmem + 128 * x, ka, qb);
+          mma_nt_half<D, KG::QCHUNK>(tmem + 128 * x + 64, va, qb + KG::QBYTES);
           mma_commit(&bars.sdp_full[x]);
         }
         if (ok) mma_commit(bars.kv_free);               // the tile's K, V are read
-        rc0 += nq;
+        rc0 += 2 * nq / KG::HPU;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -1448,8 +1534,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         kv_tile_of(p, t, bh, kt);
         const int nq = p.nqt - (p.causal ? kt : 0);
         for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
-          const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
-          const int rn = rc0 + n;
+          const int e = h % KG::HPU, x = hc % HB, u = hc / HB;
+          const int rn = rc0 + h / KG::HPU;                 // the half's stage
           if (e == 0) {
             ok = mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort);
             if (!ok) break;
@@ -1460,20 +1546,20 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t qb = sa + (rn % ns) * SB + e * 64 * 128;
-          const uint32_t db = qb + G::TILE_BYTES;
+          const uint32_t db = qb + KG::QBYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (h > 0 || kk > 0) ? 1u : 0u;
-            mma_ts_f16(tmem + T_DV, tmem + 128 * x + 16 * kk,
-                       smem_desc(db + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
-            mma_ts_f16(tmem + T_DK, tmem + 128 * x + 64 + 16 * kk,
-                       smem_desc(qb + kk * 16 * 128, G::CHUNK_BYTES, 1024), G::IDESC_MN, acc);
+            mma_ts_f16(tmem + KG::T_DV, tmem + 128 * x + 16 * kk,
+                       smem_desc(db + kk * 16 * 128, KG::QCHUNK, 1024), G::IDESC_MN, acc);
+            mma_ts_f16(tmem + KG::T_DK, tmem + 128 * x + 64 + 16 * kk,
+                       smem_desc(qb + kk * 16 * 128, KG::QCHUNK, 1024), G::IDESC_MN, acc);
           }
           mma_commit(&bars.s_free[x]);
-          if (e == 1) mma_commit(&bars.qd_empty[rn % ns]);
+          if (e == KG::HPU - 1) mma_commit(&bars.qd_empty[rn % ns]);
         }
         if (ok) mma_commit(bars.acc_full);
-        rc0 += nq;
+        rc0 += 2 * nq / KG::HPU;
       }
       mma_commit(bars.drain);
       mbar_wait(bars.drain, 0, abort);
@@ -1503,9 +1589,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const int kg = kt * 128 + key;
       const bool key_ok = kg < p.S;
       for (int h = 0; h < 2 * nq && ok; ++h, ++hc) {
-        const int n = h >> 1, e = h & 1, x = hc % kHalfBufs, u = hc / kHalfBufs;
-        const int rn = rc0 + n;
-        if (e == 0) {
+        const int n = h >> 1, e = h & 1, x = hc % HB, u = hc / HB;
+        const int rn = rc0 + h / KG::HPU;                   // the half's stage
+        if (h % KG::HPU == 0) {
           // the stage's constants and tables have landed (the stage cannot
           // refill before this tile's products, which wait for these threads)
           ok = warp_all_b(mbar_wait(&bars.qd_full[rn % ns], (rn / ns) & 1, abort));
@@ -1522,7 +1608,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         reg_fence16(sv);
         reg_fence16(dv);
         const int qbase = (i0 + n) * 128 + 64 * e + 16 * g;   // first query row of the slice
-        const int ql0 = 64 * e + 16 * g;                      // its row within the tile
+        const int ql0 = 64 * (h % KG::HPU) + 16 * g;          // its row within the stage
         // every element valid: the key exists, the slice's rows exist and
         // (causal) lie at or below this key
         const bool full = warp_all_b(key_ok && qbase + 15 < p.S && (!p.causal || kg <= qbase));
@@ -1545,7 +1631,42 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_arrive(&bars.pds_full[x]);
       }
       if (!ok) break;
-      rc0 += nq;
+      rc0 += 2 * nq / KG::HPU;
+      if constexpr (D > 64) {
+        // D = 128: 32 columns a group, dV read out first, then dK
+        if (!warp_all_b(mbar_wait(bars.acc_full, k & 1, abort))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const size_t krow = static_cast<size_t>(bh) * p.S + min(kg, p.S - 1);
+        uint32_t v0[16], v1[16];
+        tmem_ld16(lane_base + KG::T_DV + KG::DG * g, v0);
+        tmem_ld16(lane_base + KG::T_DV + KG::DG * g + 16, v1);
+        tmem_wait_ld();
+        reg_fence16(v0);
+        reg_fence16(v1);
+        if (key_ok) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(p.dV + krow * D + KG::DG * g);
+          store_bf16x16(d4, v0, 1.0f);
+          store_bf16x16(d4 + 2, v1, 1.0f);
+        }
+        tmem_ld16(lane_base + KG::T_DK + KG::DG * g, v0);
+        tmem_ld16(lane_base + KG::T_DK + KG::DG * g + 16, v1);
+        tmem_wait_ld();
+        reg_fence16(v0);
+        reg_fence16(v1);
+        // dV, dK are in registers: the next tile's products may start
+        tc_fence_before();
+        mbar_arrive(bars.acc_free);
+        if (key_ok) {
+          const float *cal = p.dkcal != nullptr ? p.dkcal + krow * D + KG::DG * g : nullptr;
+          uint4 *d4 = reinterpret_cast<uint4 *>(p.dK + krow * D + KG::DG * g);
+          store_bf16x16_cal(d4, v0, p.c, cal);
+          store_bf16x16_cal(d4 + 2, v1, p.c, cal != nullptr ? cal + 16 : nullptr);
+        }
+        continue;
+      }
       // the key's fp32 calibration part of dK (written by the dQ pass) is
       // fetched before the wait for the tile's last products
       const size_t krow = static_cast<size_t>(bh) * p.S + min(kg, p.S - 1);
@@ -1559,8 +1680,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       if (!ok) break;
       tc_fence_after();
       uint32_t v[16], w[16];
-      tmem_ld16(lane_base + T_DV + 16 * g, v);
-      tmem_ld16(lane_base + T_DK + 16 * g, w);
+      tmem_ld16(lane_base + KG::T_DV + 16 * g, v);
+      tmem_ld16(lane_base + KG::T_DK + 16 * g, w);
       tmem_wait_ld();
       reg_fence16(v);
       reg_fence16(w);
@@ -1646,23 +1767,31 @@ int sm_count() {
 }
 constexpr size_t kBarBytes = ((2 * 8 + 26) * 8 + 8 + 15) & ~static_cast<size_t>(15);
 
+// The backward's tensor maps: whole 128-row tiles, and the row boxes the
+// passes stage by (the same at D = 64; 64 rows at D = 128).
+struct alignas(64) BwdMaps {
+  CUtensorMap q, k, v, dO;
+  CUtensorMap q_stage, k_stage, v_stage, dO_stage;
+};
+
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  // Q, dO, ns x (K, V), kHalfBufs dS buffers, constants, table, two tiles'
+  using QG = DqGeo<D>;
+  // Q, dO, ns x (K, V rows), HB dS buffers, constants, table, two tiles'
   // calibration sums, barriers
   const size_t tab = (static_cast<size_t>(p.tabq_tile) + 15) & ~static_cast<size_t>(15);
   const size_t cst = 128 * kCst * sizeof(float);
   const size_t part = 2 * 2 * 4 * 128 * sizeof(float);
   const size_t fixed =
-      1024 + 2 * G::TILE_BYTES + kHalfBufs * 128 * 128 + cst + tab + part + kBarBytes;
-  int ns = static_cast<int>((kMaxSmem - fixed) / (2 * G::TILE_BYTES));
+      1024 + 2 * G::TILE_BYTES + QG::HB * 128 * 128 + cst + tab + part + kBarBytes;
+  int ns = static_cast<int>((kMaxSmem - fixed) / (2 * QG::KBYTES));
   if (ns > 4) ns = 4;
-  if (ns < 2) return QSM_ERR_UNSUPPORTED;
+  if (ns < (D > 64 ? 1 : 2)) return QSM_ERR_UNSUPPORTED;
   p.num_stages = ns;
-  p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * G::TILE_BYTES);
-  p.cst_off = p.ds_off + kHalfBufs * 128 * 128;
+  p.ds_off = static_cast<uint32_t>(2 * G::TILE_BYTES + ns * 2 * QG::KBYTES);
+  p.cst_off = p.ds_off + QG::HB * 128 * 128;
   p.tab_off = static_cast<uint32_t>(p.cst_off + cst);
   p.part_off = static_cast<uint32_t>(p.tab_off + tab);
   p.bar_off = static_cast<uint32_t>(p.part_off + part);
@@ -1683,10 +1812,11 @@ template <int D, int MAP, int SURR>
 qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
                        const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
   using G = BGeo<D>;
-  // K, V, ns x (Q, dO, constants, tables), barriers
-  const size_t stage =
-      (2 * G::TILE_BYTES + 128 * kCst * 4 + static_cast<size_t>(128) * p.TS * 4 + 1023) &
-      ~static_cast<size_t>(1023);
+  using KG = KvGeo<D>;
+  // K, V, ns x (Q, dO rows, their constants and tables), barriers
+  const size_t stage = (2 * KG::QBYTES + KG::SROWS * kCst * 4 +
+                        static_cast<size_t>(KG::SROWS) * p.TS * 4 + 1023) &
+                       ~static_cast<size_t>(1023);
   const size_t fixed = 1024 + 2 * G::TILE_BYTES + kBarBytes;
   int ns = static_cast<int>((kMaxSmem - fixed) / stage);
   if (ns > 4) ns = 4;
@@ -1714,23 +1844,23 @@ qsm_status launch_prep(const BwdArgs &a, const BwdParams &p) {
 }
 
 template <int D, int MAP, int SURR, int CAL>
-qsm_status launch_passes(const BwdArgs &a, const BwdParams &p0, const CUtensorMap &mq,
-                         const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
+qsm_status launch_passes(const BwdArgs &a, const BwdParams &p0, const BwdMaps &m) {
   BwdParams p = p0;
   p.tabq_tile = static_cast<uint32_t>(DqTab<MAP, SURR, CAL>::bytes(p.K));
   qsm_status st = launch_prep<D, MAP, SURR, CAL>(a, p);
   if (st != QSM_OK) return st;
-  st = launch_dq<D, MAP, SURR, CAL>(a, p, mq, mk, mv, mdo);
+  // the dQ pass stages K, V by KROWS-row boxes, the dK / dV pass Q, dO by
+  // SROWS-row boxes
+  st = launch_dq<D, MAP, SURR, CAL>(a, p, m.q, m.k_stage, m.v_stage, m.dO);
   if (st != QSM_OK) return st;
-  return launch_dkdv<D, MAP, SURR>(a, p, mq, mk, mv, mdo);
+  return launch_dkdv<D, MAP, SURR>(a, p, m.q_stage, m.k, m.v, m.dO_stage);
 }
 
 template <int D, int MAP, int CAL>
-qsm_status launch_by_surr(int surr, const BwdArgs &a, const BwdParams &p, const CUtensorMap &mq,
-                          const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mdo) {
-  if (surr == SURR_PRE) return launch_passes<D, MAP, SURR_PRE, CAL>(a, p, mq, mk, mv, mdo);
-  if (surr == SURR_POST) return launch_passes<D, MAP, SURR_POST, CAL>(a, p, mq, mk, mv, mdo);
-  return launch_passes<D, MAP, SURR_NONE, CAL>(a, p, mq, mk, mv, mdo);
+qsm_status launch_by_surr(int surr, const BwdArgs &a, const BwdParams &p, const BwdMaps &m) {
+  if (surr == SURR_PRE) return launch_passes<D, MAP, SURR_PRE, CAL>(a, p, m);
+  if (surr == SURR_POST) return launch_passes<D, MAP, SURR_POST, CAL>(a, p, m);
+  return launch_passes<D, MAP, SURR_NONE, CAL>(a, p, m);
 }
 
 template <int D>
@@ -1766,6 +1896,26 @@ constexpr size_t kTabQTile = static_cast<size_t>(kBwdMaxK + 2) * 16 * 128;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The post surrogate's row pass, then the passes of the map, surrogate and
+// calibration form.
+template <int D>
+qsm_status launch_maps(const BwdArgs &a, const BwdParams &p, int map, int cal, const BwdMaps &m) {
+  if (map != MAPB_EXACT && a.surrogate == QSM_SURR_POST) {
+    const qsm_status st = launch_rows<D>(a, p, m.q, m.k, m.v, m.dO);
+    if (st != QSM_OK) return st;
+  }
+  const int surr = a.surrogate;
+  if (map == MAPB_EXACT) return launch_passes<D, MAPB_EXACT, SURR_NONE, CAL_OFF>(a, p, m);
+  if (map == MAPB_POT) return launch_by_surr<D, MAPB_POT, CAL_OFF>(surr, a, p, m);
+  if (map == MAPB_HARD) {
+    if (cal == CAL_MINMAX) return launch_by_surr<D, MAPB_HARD, CAL_MINMAX>(surr, a, p, m);
+    return launch_by_surr<D, MAPB_HARD, CAL_OFF>(surr, a, p, m);
+  }
+  if (cal == CAL_MINMAX) return launch_by_surr<D, MAPB_INTERP, CAL_MINMAX>(surr, a, p, m);
+  if (cal == CAL_FIXED) return launch_by_surr<D, MAPB_INTERP, CAL_FIXED>(surr, a, p, m);
+  return launch_by_surr<D, MAPB_INTERP, CAL_OFF>(surr, a, p, m);
+}
+
 }  // namespace
 
 size_t bwd_workspace_bytes(int B, int H, int S, int D) {
@@ -1782,7 +1932,7 @@ size_t bwd_workspace_bytes(int B, int H, int S, int D) {
 }
 
 qsm_status launch_bwd(const BwdArgs &a) {
-  if (a.D != 64) return QSM_ERR_UNSUPPORTED;          // TMEM schedule holds D = 64
+  if (a.D != 64 && a.D != 128) return QSM_ERR_UNSUPPORTED;
   if (a.mode == QSM_MODE_KINTERVAL && a.Kint > kBwdMaxK) return QSM_ERR_UNSUPPORTED;
   const size_t rows = static_cast<size_t>(a.B) * a.H * a.S;
   const int map = a.mode == QSM_MODE_EXACT       ? MAPB_EXACT
@@ -1838,35 +1988,23 @@ qsm_status launch_bwd(const BwdArgs &a) {
   p.dV = static_cast<__nv_bfloat16 *>(a.dV);
   p.status = a.status_dev;
 
-  alignas(64) CUtensorMap mq, mk, mv, mdo;
+  BwdMaps m;
   const int bh = a.B * a.H;
-  if (!make_tmap_3d(&mq, a.Q, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&mk, a.K, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&mv, a.V, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&mdo, a.dO, false, a.D, a.S, bh, 128))
+  const int srows = a.D > 64 ? 64 : 128;               // the passes' stage boxes
+  if (!make_tmap_3d(&m.q, a.Q, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.k, a.K, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.v, a.V, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.dO, a.dO, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.q_stage, a.Q, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.k_stage, a.K, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.v_stage, a.V, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.dO_stage, a.dO, false, a.D, a.S, bh, srows))
     return QSM_ERR_CUDA;
 
   if (p.dkcal != nullptr &&
       cudaMemsetAsync(p.dkcal, 0, rows * a.D * sizeof(float), a.stream) != cudaSuccess)
     return QSM_ERR_CUDA;
-  if (map != MAPB_EXACT && a.surrogate == QSM_SURR_POST) {
-    const qsm_status st = launch_rows<64>(a, p, mq, mk, mv, mdo);
-    if (st != QSM_OK) return st;
-  }
-  const int surr = a.surrogate;
-  if (map == MAPB_EXACT)
-    return launch_passes<64, MAPB_EXACT, SURR_NONE, CAL_OFF>(a, p, mq, mk, mv, mdo);
-  if (map == MAPB_POT) return launch_by_surr<64, MAPB_POT, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
-  if (map == MAPB_HARD) {
-    if (cal == CAL_MINMAX)
-      return launch_by_surr<64, MAPB_HARD, CAL_MINMAX>(surr, a, p, mq, mk, mv, mdo);
-    return launch_by_surr<64, MAPB_HARD, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
-  }
-  if (cal == CAL_MINMAX)
-    return launch_by_surr<64, MAPB_INTERP, CAL_MINMAX>(surr, a, p, mq, mk, mv, mdo);
-  if (cal == CAL_FIXED)
-    return launch_by_surr<64, MAPB_INTERP, CAL_FIXED>(surr, a, p, mq, mk, mv, mdo);
-  return launch_by_surr<64, MAPB_INTERP, CAL_OFF>(surr, a, p, mq, mk, mv, mdo);
+  return a.D == 64 ? launch_maps<64>(a, p, map, cal, m) : launch_maps<128>(a, p, map, cal, m);
 }
 
 }  // namespace qsm

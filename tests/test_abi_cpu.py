@@ -104,7 +104,7 @@ def test_bwd_rejects_bad_arguments():
 
 def test_bwd_refuses_unsupported_shapes_before_launch():
     # complete arguments (statistics and a large enough workspace) for shapes
-    # the backward's TMEM schedule and table do not cover: D = 128, K > 32
+    # the backward's grid tables do not cover: K > 32, at either D
     L = qsm.lib()
     o = qsm.qsm_opts_default()
     o.row_hi = o.row_lo = o.row_argmax = o.row_argmin = FAKE
@@ -114,7 +114,7 @@ def test_bwd_refuses_unsupported_shapes_before_launch():
         o.workspace_bytes = qsm.qsm_attn_bwd_workspace_size(1, 1, 128, D)
         return L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128,
                               D, 1, 1, Kint, 0, 1, 1, ctypes.byref(o), None)
-    assert bwd(128, 4) == qsm.QSM_ERR_UNSUPPORTED
+    assert bwd(128, 33) == qsm.QSM_ERR_UNSUPPORTED
     assert bwd(64, 33) == qsm.QSM_ERR_UNSUPPORTED
 
 

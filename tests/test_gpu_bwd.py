@@ -1,5 +1,5 @@
-"""GPU parity of the backward (K-interval and exact maps, bf16, D = 64)
-against the CPU oracle, through the C ABI.
+"""GPU parity of the backward (K-interval, exact and Rowmax-PoT maps, bf16,
+D = 64 and 128) against the CPU oracle, through the C ABI.
 
 The rules are the oracle's ("Pretraining Transformers with Quantized Softmax
 in Attention", abstract: backward rules including calibration derivatives;
@@ -196,3 +196,63 @@ def test_bwd_rowmax_pot_training_shape(surr):
     got, _ = _run(d, True, 2, 4, 0, 1, surr, False, dump=False, O_store=fwd["O"])
     ref = _oracle(d, True, 2, 4, 0, 1, surr, False, heads=heads, O_store=fwd["O"])
     _check(got, ref, heads=heads)
+
+
+# ------------------------------------------------------------------ D = 128
+# Head dimension 128: two TMEM pairs and half-tile ring stages in both passes
+# (64-row Q / dO stages in the dK / dV pass, 64-key K / V stages in the dQ
+# pass), 32-column slices per map group in the read-outs.
+
+D128_COMBOS = [(4, 0, 1, 1, False), (16, 0, 0, 2, False), (4, 1, 1, 0, False),
+               (16, 1, 0, 1, False), (16, 0, 0, 0, True), (32, 0, 0, 1, False),
+               (4, 0, 0, 2, True)]
+
+
+@pytest.mark.parametrize("K,calib,rnd,surr,detach", D128_COMBOS)
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False), (333, True)])
+def test_bwd_kinterval_d128(S, causal, K, calib, rnd, surr, detach):
+    d = inputs.draw(1, 2, S, 128, seed=130 + S, with_dO=True)
+    fwd = _stored_o(d, causal, 1, K, calib, rnd, window=6.0)
+    got, dec = _run(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
+    ref = _oracle(d, causal, 1, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
+    heads = [(0, 0), (0, 1)]
+    fq, fkv, n = _flip_rows(d, dec, causal, 1, K, calib, rnd, 6.0, heads, fwd)
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
+
+
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
+def test_bwd_exact_d128(S, causal):
+    d = inputs.draw(1, 2, S, 128, seed=170 + S, with_dO=True)
+    fwd = _stored_o(d, causal, 0, 4, 0, 1)
+    got, _ = _run(d, causal, 0, 4, 0, 1, 0, False, dump=False, O_store=fwd["O"])
+    ref = _oracle(d, causal, 0, 4, 0, 1, 0, False, O_store=fwd["O"])
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("surr", [1, 2])
+def test_bwd_rowmax_pot_d128(surr):
+    d = inputs.draw(1, 2, 256, 128, seed=190 + surr, with_dO=True)
+    fwd = _stored_o(d, True, 2, 4, 0, 1)
+    got, _ = _run(d, True, 2, 4, 0, 1, surr, False, dump=False, O_store=fwd["O"])
+    ref = _oracle(d, True, 2, 4, 0, 1, surr, False, O_store=fwd["O"])
+    _check(got, ref)
+
+
+@pytest.mark.parametrize("mode,K,calib,rnd,surr", [(1, 16, 0, 0, 1), (1, 4, 0, 1, 2),
+                                                   (1, 16, 1, 0, 2)])
+def test_bwd_d128_many_tiles(mode, K, calib, rnd, surr):
+    """More query and key tiles than SMs (B2 H48 S512 causal: 384 tiles), so
+    every persistent CTA takes several tiles through the rings; the oracle
+    checks three whole heads."""
+    d = inputs.draw(2, 48, 512, 128, seed=211 + K, with_dO=True)
+    heads = [(0, 0), (1, 17), (1, 47)]
+    fwd = _stored_o(d, True, mode, K, calib, rnd, heads=heads)
+    got, dec = _run(d, True, mode, K, calib, rnd, surr, False, O_store=fwd["O"])
+    ref = _oracle(d, True, mode, K, calib, rnd, surr, False, heads=heads, O_store=fwd["O"])
+    fq, fkv, n = _flip_rows(d, dec, True, mode, K, calib, rnd, 8.0, heads, fwd)
+    _check(got, ref, heads=heads, skip=(fq, fkv))
+    assert fq.sum() <= 0.01 * 3 * 512, n
+    for g in got:
+        assert np.isfinite(g).all()
+
