@@ -184,7 +184,6 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
       (reinterpret_cast<uintptr_t>(LSE) & 3u))
     return QSM_ERR_INVALID_ARG;
-  if (o.dtype != QSM_BF16) return QSM_ERR_UNSUPPORTED;
   // the probes are forward-only sensitivity studies
   if (mode == QSM_MODE_TRUNCATED || mode == QSM_MODE_UNIFORM) return QSM_ERR_UNSUPPORTED;
   // the rules are derived for maps anchored at the final row statistics; the
@@ -205,6 +204,9 @@ qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void 
   a.mode = mode; a.Kint = Kint; a.calib = calibration; a.rounding = rounding;
   a.surrogate = surrogate; a.detach = o.detach_extrema;
   a.c = c; a.window = o.window; a.below_policy = o.below_policy; a.pot_floor = o.pot_floor;
+  a.fp8 = o.dtype == QSM_FP8_E4M3;
+  a.scale = o.scale > 0.0f ? o.scale : 1.0f / std::sqrt(static_cast<float>(D));
+  a.q_descale = o.q_descale; a.k_descale = o.k_descale; a.v_descale = o.v_descale;
   a.row_hi = o.row_hi; a.row_lo = o.row_lo;
   a.row_argmax = o.row_argmax; a.row_argmin = o.row_argmin;
   a.workspace = o.workspace; a.workspace_bytes = o.workspace_bytes;

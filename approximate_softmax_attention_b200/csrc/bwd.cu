@@ -46,6 +46,7 @@
 // so no per-element branch remains.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -87,6 +88,8 @@ struct BwdParams {
   int K, fixed_window, flush, pot_floor;
   int TS;           // floats of one query row's dK / dV pass table (a multiple of 4)
   float c, cL2E, window;
+  float gq, gk;     // gradient scales: dQ = gq dS K, dK = gk dS^T Q (c, or for
+                    // e4m3 the score scale with one descale each: see launch_bwd)
   const float *LSE, *hi, *lo;
   const int32_t *amax, *amin;
   float *rowws;     // [rows][kRowWs]: LSE*, delta* (post surrogate)
@@ -613,6 +616,35 @@ __device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm,
   }
 }
 
+// ------------------------------------------------------------- e4m3 inputs
+// The backward of an e4m3 forward runs on bf16 copies: the Q and K codes as
+// they are (every e4m3 value is a bf16 value, so the recomputed scores are the
+// forward's), the V codes times v_descale (rounded to bf16; dP = dO V~^T
+// needs V~ itself).  Eight elements a thread step, as 8-byte loads and
+// 16-byte stores.
+__device__ __forceinline__ uint4 e4m3x8_to_bf16(uint2 w, float scale) {
+  __nv_fp8x4_e4m3 lo, hi;
+  lo.__x = w.x;
+  hi.__x = w.y;
+  const float4 a = static_cast<float4>(lo), b = static_cast<float4>(hi);
+  return make_uint4(pack_bf16x2(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale)),
+                    pack_bf16x2(__fmul_rn(a.z, scale), __fmul_rn(a.w, scale)),
+                    pack_bf16x2(__fmul_rn(b.x, scale), __fmul_rn(b.y, scale)),
+                    pack_bf16x2(__fmul_rn(b.z, scale), __fmul_rn(b.w, scale)));
+}
+
+__global__ void __launch_bounds__(256)
+    qsm_bwd_dequant(const uint2 *__restrict__ q8, const uint2 *__restrict__ k8,
+                    const uint2 *__restrict__ v8, uint4 *qb, uint4 *kb, uint4 *vb, size_t n8,
+                    float v_descale) {
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    qb[i] = e4m3x8_to_bf16(q8[i], 1.0f);
+    kb[i] = e4m3x8_to_bf16(k8[i], 1.0f);
+    vb[i] = e4m3x8_to_bf16(v8[i], v_descale);
+  }
+}
+
 // ----------------------------------------------------------- row prep
 // One CTA of 128 threads per query tile, thread = row: each row's delta =
 // dO_r . O_r, map constants and grid tables, written to the workspace -- the
@@ -1057,7 +1089,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       mbar_arrive(&bars.dq_free[x]);
       // the row's calibration derivatives from the four groups' sums; they
       // are computed (the loaded sums consumed) before the buffer's release
-      float sh = 0.0f, sl = 0.0f;
+      float sh = 0.0f, sl = 0.0f, shk = 0.0f, slk = 0.0f;   // dQ side, dK side
       if (cal_row) {
         const float *pp = part + x * 1024;
         const float S1 = (pp[row] + pp[128 + row]) + (pp[256 + row] + pp[384 + row]);
@@ -1073,10 +1105,12 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           dhi = S1;
           dlo = -S1 - kinv * S2;
         }
-        sh = p.c * dhi;
-        sl = p.c * dlo;
+        sh = p.gq * dhi;
+        sl = p.gq * dlo;
+        shk = p.gk * dhi;
+        slk = p.gk * dlo;
       }
-      asm volatile("" ::"f"(sh), "f"(sl) : "memory");
+      asm volatile("" ::"f"(sh), "f"(sl), "f"(shk), "f"(slk) : "memory");
       mbar_arrive(&bars.part_free[x]);
 #pragma unroll
       for (int pc = 0; pc < NP; ++pc) {
@@ -1084,7 +1118,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         if (pc > 0) gather(c0);
         float xq[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[pc][i]) * p.c;
+        for (int i = 0; i < 16; ++i) xq[i] = __uint_as_float(v[pc][i]) * p.gq;
         if (cal_row) {
           float kx[16], qx[16];
           bf16x16_to_f32(kaw, kx);
@@ -1094,8 +1128,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           float *da = p.dkcal + (head + amx) * D + c0;
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            red_add_f32x4(da + 4 * i, make_float4(sh * qx[4 * i], sh * qx[4 * i + 1],
-                                                  sh * qx[4 * i + 2], sh * qx[4 * i + 3]));
+            red_add_f32x4(da + 4 * i, make_float4(shk * qx[4 * i], shk * qx[4 * i + 1],
+                                                  shk * qx[4 * i + 2], shk * qx[4 * i + 3]));
           if (CAL == CAL_MINMAX) {
             bf16x16_to_f32(kbw, kx);
 #pragma unroll
@@ -1103,8 +1137,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
             float *db = p.dkcal + (head + amn) * D + c0;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              red_add_f32x4(db + 4 * i, make_float4(sl * qx[4 * i], sl * qx[4 * i + 1],
-                                                    sl * qx[4 * i + 2], sl * qx[4 * i + 3]));
+              red_add_f32x4(db + 4 * i, make_float4(slk * qx[4 * i], slk * qx[4 * i + 1],
+                                                    slk * qx[4 * i + 2], slk * qx[4 * i + 3]));
           }
         }
         uint32_t pk[8];
@@ -1662,8 +1696,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         if (key_ok) {
           const float *cal = p.dkcal != nullptr ? p.dkcal + krow * D + KG::DG * g : nullptr;
           uint4 *d4 = reinterpret_cast<uint4 *>(p.dK + krow * D + KG::DG * g);
-          store_bf16x16_cal(d4, v0, p.c, cal);
-          store_bf16x16_cal(d4 + 2, v1, p.c, cal != nullptr ? cal + 16 : nullptr);
+          store_bf16x16_cal(d4, v0, p.gk, cal);
+          store_bf16x16_cal(d4 + 2, v1, p.gk, cal != nullptr ? cal + 16 : nullptr);
         }
         continue;
       }
@@ -1699,7 +1733,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       }
       float xk[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) xk[i] = __uint_as_float(w[i]) * p.c;
+      for (int i = 0; i < 16; ++i) xk[i] = __uint_as_float(w[i]) * p.gk;
       if (p.dkcal != nullptr && key_ok) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -1926,9 +1960,11 @@ size_t bwd_workspace_bytes(int B, int H, int S, int D) {
   const size_t rows = static_cast<size_t>(B) * H * S;
   const size_t tiles = static_cast<size_t>(B) * H * ((S + 127) / 128);
   const size_t trows = tiles * 128;
+  // (D = 128: bf16 copies of e4m3 Q, K, V)
+  const size_t deq = D == 128 ? 3 * align256(rows * D * 2) : 0;
   return align256(rows * D * sizeof(float)) + align256(rows * kRowWs * sizeof(float)) +
          align256(trows * kCst * sizeof(float)) + align256(trows * kTabKT * sizeof(float2)) +
-         align256(tiles * kTabQTile);
+         align256(tiles * kTabQTile) + deq;
 }
 
 qsm_status launch_bwd(const BwdArgs &a) {
@@ -1956,6 +1992,11 @@ qsm_status launch_bwd(const BwdArgs &a) {
                             : 0;
   p.c = a.c;
   p.cL2E = a.c * 1.4426950408889634f;
+  // gradients with respect to the tensors the scores are formed from: Q, K
+  // (bf16), or q_descale Q, k_descale K (e4m3), whose bf16 copies hold the
+  // codes, so dQ = scale k_descale dS K and dK = scale q_descale dS^T Q
+  p.gq = a.fp8 ? a.scale * a.k_descale : a.c;
+  p.gk = a.fp8 ? a.scale * a.q_descale : a.c;
   p.window = a.window;
   p.LSE = a.LSE;
   p.hi = a.row_hi;
@@ -1974,13 +2015,33 @@ qsm_status launch_bwd(const BwdArgs &a) {
   const size_t trows = static_cast<size_t>(p.BH) * p.nqt * 128;
   const size_t o_tab = o_cst + align256(trows * kCst * sizeof(float));
   const size_t o_tabq = o_tab + align256(trows * kTabKT * sizeof(float2));
+  const size_t o_deq = o_tabq + align256(static_cast<size_t>(p.BH) * p.nqt * kTabQTile);
   p.dkcal = calib ? reinterpret_cast<float *>(ws + o_dk) : nullptr;
   p.rowws = reinterpret_cast<float *>(ws + o_rw);
   p.cst = reinterpret_cast<float *>(ws + o_cst);
   p.tabk = reinterpret_cast<float *>(ws + o_tab);
   p.tabq = ws + o_tabq;
-  p.Q = static_cast<const __nv_bfloat16 *>(a.Q);
-  p.K_ = static_cast<const __nv_bfloat16 *>(a.K);
+  const void *Qp = a.Q, *Kp = a.K, *Vp = a.V;
+  if (a.fp8) {
+    if (a.D != 128) return QSM_ERR_UNSUPPORTED;
+    const size_t part = align256(rows * a.D * 2);
+    uint4 *qb = reinterpret_cast<uint4 *>(ws + o_deq);
+    uint4 *kb = reinterpret_cast<uint4 *>(ws + o_deq + part);
+    uint4 *vb = reinterpret_cast<uint4 *>(ws + o_deq + 2 * part);
+    const size_t n8 = rows * a.D / 8;
+    const size_t want = (n8 + 255) / 256;
+    const int grid = static_cast<int>(want < 8 * 148 ? want : 8 * 148);
+    qsm_bwd_dequant<<<grid, 256, 0, a.stream>>>(static_cast<const uint2 *>(a.Q),
+                                                 static_cast<const uint2 *>(a.K),
+                                                 static_cast<const uint2 *>(a.V), qb, kb, vb, n8,
+                                                 a.v_descale);
+    if (cudaGetLastError() != cudaSuccess) return QSM_ERR_CUDA;
+    Qp = qb;
+    Kp = kb;
+    Vp = vb;
+  }
+  p.Q = static_cast<const __nv_bfloat16 *>(Qp);
+  p.K_ = static_cast<const __nv_bfloat16 *>(Kp);
   p.O = static_cast<const __nv_bfloat16 *>(a.O);
   p.dO = static_cast<const __nv_bfloat16 *>(a.dO);
   p.dQ = static_cast<__nv_bfloat16 *>(a.dQ);
@@ -1991,13 +2052,13 @@ qsm_status launch_bwd(const BwdArgs &a) {
   BwdMaps m;
   const int bh = a.B * a.H;
   const int srows = a.D > 64 ? 64 : 128;               // the passes' stage boxes
-  if (!make_tmap_3d(&m.q, a.Q, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&m.k, a.K, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&m.v, a.V, false, a.D, a.S, bh, 128) ||
+  if (!make_tmap_3d(&m.q, Qp, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.k, Kp, false, a.D, a.S, bh, 128) ||
+      !make_tmap_3d(&m.v, Vp, false, a.D, a.S, bh, 128) ||
       !make_tmap_3d(&m.dO, a.dO, false, a.D, a.S, bh, 128) ||
-      !make_tmap_3d(&m.q_stage, a.Q, false, a.D, a.S, bh, srows) ||
-      !make_tmap_3d(&m.k_stage, a.K, false, a.D, a.S, bh, srows) ||
-      !make_tmap_3d(&m.v_stage, a.V, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.q_stage, Qp, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.k_stage, Kp, false, a.D, a.S, bh, srows) ||
+      !make_tmap_3d(&m.v_stage, Vp, false, a.D, a.S, bh, srows) ||
       !make_tmap_3d(&m.dO_stage, a.dO, false, a.D, a.S, bh, srows))
     return QSM_ERR_CUDA;
 

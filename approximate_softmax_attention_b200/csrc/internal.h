@@ -58,6 +58,10 @@ struct BwdArgs {
   int B, H, S, D, causal;
   int mode, Kint, calib, rounding, surrogate, detach;
   float c, window;
+  // e4m3 inputs (D = 128): Q, K, V hold codes that stand for q_descale Q,
+  // k_descale K, v_descale V; scale is the score scale before the descales
+  int fp8;
+  float scale, q_descale, k_descale, v_descale;
   int below_policy, pot_floor;
   const float *row_hi, *row_lo;
   const int32_t *row_argmax, *row_argmin;

@@ -240,20 +240,24 @@ def default_scale(D):
 
 def attention_backward(q, k, v, O, dO, LSE, stats, causal=False, mode=MODE_KINTERVAL, Kint=4,
                        calibration=CALIB_MINMAX, rounding=ROUND_HARD, surrogate=SURR_NONE, *,
-                       detach_extrema=False, scale=None, window=8.0, below_policy=0,
-                       workspace=None, stream=None):
-    """Allocate dQ, dK, dV (and the workspace, unless given) with torch and run
-    ``qsm_attn_bwd``.  ``stats`` is the dict returned by attention_forward(...,
-    stats=True)."""
+                       detach_extrema=False, scale=None, q_descale=1.0, k_descale=1.0,
+                       v_descale=1.0, window=8.0, below_policy=0, workspace=None, stream=None):
+    """Allocate dQ, dK, dV (bf16; and the workspace, unless given) with torch
+    and run ``qsm_attn_bwd``.  ``stats`` is the dict returned by
+    attention_forward(..., stats=True).  With e4m3 q, k, v (and their
+    descales, as given to the forward) the gradients are those of
+    q_descale q, k_descale k, v_descale v."""
     B, H, S, D = q.shape
     dev = q.device
-    dQ = torch.empty_like(q)
-    dK = torch.empty_like(k)
-    dV = torch.empty_like(v)
+    dQ = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    dK = torch.empty(k.shape, dtype=torch.bfloat16, device=dev)
+    dV = torch.empty(v.shape, dtype=torch.bfloat16, device=dev)
     need = qsm_attn_bwd_workspace_size(B, H, S, D)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    kw = dict(scale=0.0 if scale is None else float(scale), window=float(window),
+    kw = dict(dtype=DTYPE_FP8_E4M3 if q.dtype == torch.float8_e4m3fn else DTYPE_BF16,
+              scale=0.0 if scale is None else float(scale), q_descale=float(q_descale),
+              k_descale=float(k_descale), v_descale=float(v_descale), window=float(window),
               below_policy=int(below_policy), detach_extrema=int(bool(detach_extrema)),
               workspace=workspace, workspace_bytes=int(workspace.numel()))
     if stats is not None:

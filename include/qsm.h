@@ -172,26 +172,34 @@ qsm_status qsm_attn_fwd(const void *Q, const void *K, const void *V, void *O, fl
                         qsm_calib calibration, qsm_rounding rounding,
                         qsm_surrogate surrogate, const qsm_opts *opts, qsm_stream_t stream);
 
-/* Backward of qsm_attn_fwd (bf16, D = 64): the exact map, K-interval
+/* Backward of qsm_attn_fwd (D = 64 or 128): the exact map, K-interval
  * attention (K <= 32) and Rowmax-PoT.
- *  Q, K, V, O, dO: device [B,H,S,D] bf16 (O = the forward's output).
+ *  Q, K, V: device [B,H,S,D] as given to the forward: bf16, or (D = 128)
+ *        e4m3 with the forward's opts->q_descale/k_descale/v_descale.
+ *  O, dO: device [B,H,S,D] bf16 (O = the forward's output).
  *  LSE:  device [B,H,S] fp32 from the forward.
- *  dQ, dK, dV: device [B,H,S,D] bf16 (written).
+ *  dQ, dK, dV: device [B,H,S,D] bf16 (written): the gradients with respect
+ *        to the tensors the forward's scores and output are formed from --
+ *        Q, K, V for bf16; q_descale Q, k_descale K, v_descale V for e4m3,
+ *        whose codes are copied to bf16 in the workspace (Q and K exactly, so
+ *        the recomputed scores are the forward's; V times v_descale, rounded
+ *        to bf16) before the bf16 passes run.
  *  The rules are the exact gradients of the surrogate graphs with the
  *  forward's rounding decisions frozen (see qsm_surrogate).  Rowmax-PoT's
  *  backward is not derived on the pages; the same surrogates apply to it,
  *  and with its exponents frozen a power-of-two weight has no derivative of
  *  its own, nor a calibration term (QSM_SURR_NONE gives dQ = dK = 0).
  *  K-interval needs opts->row_hi/row_lo/row_argmax/row_argmin from the
- *  forward, Rowmax-PoT opts->row_hi; all need opts->workspace.  e4m3, D = 128
- *  and K > 32 return QSM_ERR_UNSUPPORTED. */
+ *  forward, Rowmax-PoT opts->row_hi; all need opts->workspace.  e4m3 at
+ *  D = 64 and K > 32 return QSM_ERR_UNSUPPORTED. */
 qsm_status qsm_attn_bwd(const void *Q, const void *K, const void *V, const void *O,
                         const void *dO, const float *LSE, void *dQ, void *dK, void *dV,
                         int B, int H, int S, int D, int causal, qsm_mode mode, int Kint,
                         qsm_calib calibration, qsm_rounding rounding,
                         qsm_surrogate surrogate, const qsm_opts *opts, qsm_stream_t stream);
 
-/* Bytes of opts->workspace that qsm_attn_bwd needs for this shape. */
+/* Bytes of opts->workspace that qsm_attn_bwd needs for this shape (at
+ * D = 128 including room for bf16 copies of e4m3 Q, K, V). */
 size_t qsm_attn_bwd_workspace_size(int B, int H, int S, int D);
 
 /* Size of the library's own backward scratch array (16 MiB). */

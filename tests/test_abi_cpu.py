@@ -90,7 +90,11 @@ def test_bwd_rejects_bad_arguments():
         return L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128,
                               128, 1, mode, 4, 0, 1, 1, ctypes.byref(o), None)
     assert bwd(mode=2) == qsm.QSM_ERR_INVALID_ARG           # PoT backward needs row_hi
-    assert bwd(mode=1, dtype=1) == qsm.QSM_ERR_UNSUPPORTED  # e4m3 backward
+    assert bwd(mode=1, dtype=1) == qsm.QSM_ERR_INVALID_ARG  # e4m3 (D = 128): no statistics
+    o64 = qsm.qsm_opts_default()
+    o64.dtype = 1
+    assert L.qsm_attn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 1,
+                          1, 4, 0, 1, 1, ctypes.byref(o64), None) == qsm.QSM_ERR_UNSUPPORTED
     assert bwd(mode=1) == qsm.QSM_ERR_INVALID_ARG           # no row statistics
     o = qsm.qsm_opts_default()
     o.row_hi = o.row_lo = o.row_argmax = o.row_argmin = FAKE

@@ -256,3 +256,50 @@ def test_bwd_d128_many_tiles(mode, K, calib, rnd, surr):
     for g in got:
         assert np.isfinite(g).all()
 
+
+
+# ----------------------------------------------------------------- e4m3
+# The backward of an e4m3 forward (D = 128): gradients with respect to
+# q_descale Q, k_descale K, v_descale V, which the oracle takes as its inputs
+# (exact in float64).
+
+def _run_fp8(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, O_store=None):
+    q, k, v = (d[n].to(DEV).contiguous() for n in ("q", "k", "v"))
+    dO = d["dO"].to(DEV).contiguous()
+    B, H, S, D = q.shape
+    desc = dict(q_descale=d["q_descale"], k_descale=d["k_descale"], v_descale=d["v_descale"])
+    dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV)
+    O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rnd, window=window,
+                                       stats=True, debug_idx=dbg, **desc)
+    if O_store is not None:
+        Os = torch.from_numpy(np.asarray(O_store, dtype=np.float32)).to(DEV)
+        O = torch.where(torch.isnan(Os), O.float(), Os).to(torch.bfloat16).contiguous()
+    dQ, dK, dV = qsm.attention_backward(q, k, v, O, dO, LSE, st, causal, mode, K, calib, rnd,
+                                        surr, detach_extrema=detach, window=window, **desc)
+    torch.cuda.synchronize()
+    return [x.float().cpu().numpy() for x in (dQ, dK, dV)], dbg.cpu().numpy()
+
+
+def _real(d):
+    """The tensors the e4m3 codes stand for, in float64."""
+    f = lambda t, s: t.to(torch.float32).double().numpy() * float(s)
+    return dict(d, q=f(d["q"], d["q_descale"]), k=f(d["k"], d["k_descale"]),
+                v=f(d["v"], d["v_descale"]), q_descale=1.0, k_descale=1.0, v_descale=1.0)
+
+
+@pytest.mark.parametrize("mode,K,calib,rnd,surr,detach",
+                         [(1, 4, 0, 1, 1, False), (1, 16, 0, 0, 2, False),
+                          (1, 16, 1, 0, 0, False), (1, 4, 1, 1, 2, True), (0, 4, 0, 1, 0, False),
+                          (2, 4, 0, 1, 1, False)])
+@pytest.mark.parametrize("S,causal", [(256, True), (200, False)])
+def test_bwd_fp8(S, causal, mode, K, calib, rnd, surr, detach):
+    d = inputs.draw(1, 2, S, 128, seed=240 + S, dtype="fp8", with_dO=True)
+    dr = _real(d)
+    fwd = _stored_o(dr, causal, mode, K, calib, rnd, window=6.0)
+    got, dec = _run_fp8(d, causal, mode, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
+    ref = _oracle(dr, causal, mode, K, calib, rnd, surr, detach, window=6.0, O_store=fwd["O"])
+    # (the decision check decodes the e4m3 codes with their descales itself)
+    fq, fkv, n = _flip_rows(d, dec if mode == 1 else None, causal, mode, K, calib, rnd, 6.0,
+                            [(0, 0), (0, 1)], fwd)
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
