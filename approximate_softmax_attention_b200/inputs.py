@@ -78,6 +78,12 @@ WORKLOADS = {
                           with_dO=True,
                           modes=((1, 4, 0, 1), (1, 16, 0, 0), (1, 4, 1, 1),
                                  (1, 16, 1, 0))),
+    # the backward at head dimension 128 (the forward workloads' D), bf16 and
+    # for an e4m3 forward: the training shape's rows with half the heads
+    "train_s1k_d128": Workload("train_s1k_d128", 8, 6, 1024, 128, "bf16", True, 5, False,
+                               with_dO=True, modes=((1, 4, 0, 1), (1, 16, 1, 0))),
+    "train_s1k_d128_fp8": Workload("train_s1k_d128_fp8", 8, 6, 1024, 128, "fp8", True, 5,
+                                   False, with_dO=True, modes=((1, 4, 0, 1), (1, 16, 1, 0))),
 }
 
 

@@ -610,6 +610,9 @@ def run_ours(args):
     if args.part in ("all", "bwd") and not args.no_extra and rank == 0:
         extras["train_s1k_bwd"] = run_backward(dev, qsm, inputs, stream, pk,
                                                reps=args.bwd_reps)
+        for wn in ("train_s1k_d128", "train_s1k_d128_fp8"):
+            extras[wn + "_bwd"] = run_backward(dev, qsm, inputs, stream, pk,
+                                               reps=args.bwd_reps, workload=wn)
 
     cpu = None
     if line is not None and rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -700,27 +703,32 @@ def run_extra_forwards(dev, qsm, inputs, stream, pk):
     return extras
 
 
-def run_backward(dev, qsm, inputs, stream, pk, reps=10):
+def run_backward(dev, qsm, inputs, stream, pk, reps=10, workload="train_s1k"):
     """Training shape: forward with statistics, then the backward (2.5 x the
-    forward's algorithmic FLOPs), per (map, surrogate)."""
+    forward's algorithmic FLOPs), per (map, surrogate).  An e4m3 workload runs
+    the backward of its e4m3 forward (bf16 passes, FLOPs counted the same)."""
     import torch
-    tw = inputs.WORKLOADS["train_s1k"]
+    tw = inputs.WORKLOADS[workload]
     td = inputs.draw_workload(tw)
     tq, tk, tv, tdo = (td[n].to(dev) for n in ("q", "k", "v", "dO"))
+    desc = dict(q_descale=td["q_descale"], k_descale=td["k_descale"],
+                v_descale=td["v_descale"])
     ws = torch.empty(qsm.qsm_attn_bwd_workspace_size(*tw.shape), dtype=torch.uint8, device=dev)
     res = {}
     for (mode, K, cal, rnd) in tw.modes:
         for surr in (qsm.SURR_PRE, qsm.SURR_POST):
-            O_, L_, st_ = qsm.attention_forward(tq, tk, tv, True, mode, K, cal, rnd, stats=True)
+            O_, L_, st_ = qsm.attention_forward(tq, tk, tv, True, mode, K, cal, rnd, stats=True,
+                                                **desc)
             fn = (lambda: qsm.attention_backward(tq, tk, tv, O_, tdo, L_, st_, True, mode, K,
-                                                 cal, rnd, surr, workspace=ws))
+                                                 cal, rnd, surr, workspace=ws, **desc))
             per, _ = time_calls([fn], stream, reps, 3)
             ms = sum(per[0]) / len(per[0])
             tf = 2.5 * fwd_flops(tw) / (ms * 1e-3) / 1e12
             lab = "%s_%s" % (mode_label((mode, K, cal, rnd)), {1: "pre", 2: "post"}[surr])
             res[lab] = {"bwd_ms": round(ms, 4), "bwd_tflops": round(tf, 1),
                         "frac_of_bf16_peak": round(tf / pk["bf16"][0], 4)}
-    return {"shape": list(tw.shape), "dtype": "bf16", "causal": True,
+    return {"shape": list(tw.shape), "dtype": "bf16" if tw.dtype == "bf16" else
+            "e4m3 inputs, bf16 passes", "causal": True,
             "flops": "2.5 x 4*B*H*S^2*D/2", "per_mode": res}
 
 
