@@ -288,8 +288,10 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], float cL2E, f
 // Every map runs two sweeps: the statistics sweep finds the row's maximum
 // (and minimum, arguments) over all keys, then the main sweep maps each score
 // against those final values.  For the exact map this is softmax against the
-// true row maximum, with no online rescaling of O.
-template <int D, bool FP8, int MAP, bool KSAT>
+// true row maximum, with no online rescaling of O.  DBG: the kernel writes
+// the decision dump (a separate instantiation, so that the dump's code takes
+// no registers from the ordinary one).
+template <int D, bool FP8, int MAP, bool KSAT, bool DBG>
 __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, int g, int row,
                                          uint32_t lane_base, int qi, int n, int bh, float *tab,
                                          const Xch &xc, volatile int *abort) {
@@ -434,7 +436,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
     mbar_arrive(bars.xstat);
     ok = warp_all(mbar_wait(bars.xstat, 1, abort));
   }
-  int8_t *dbg_row = (p.dbg != nullptr && row_ok)
+  int8_t *dbg_row = (DBG && p.dbg != nullptr && row_ok)
                         ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
                         : nullptr;
 
@@ -479,7 +481,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
         } else {
           map_chunk<MAP, false, FP8, false, false>(v, mr, 32 * c, lim, flush_below, z, pc);
         }
-        if (p.dbg != nullptr)
+        if (DBG && p.dbg != nullptr)
           debug_chunk<MAP, KSAT>(dbg_row, v, mr, 128 * j + c_off + 32 * c, 32 * c, lim, p,
                            flush_below);
       }
@@ -517,7 +519,7 @@ __device__ __forceinline__ void map_half(const FwdParams &p, const Bars &bars, i
   }
 }
 
-template <int D, bool FP8, int MAP, bool KSAT>
+template <int D, bool FP8, int MAP, bool KSAT, bool DBG>
 __global__ void __launch_bounds__(kThreads, 1)
     qsm_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -770,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(bars.drain, 0, abort);
   } else if (warp >= 4) {
     const int g = (warp - 4) >> 2;                 // map group 0..3
-    map_half<D, FP8, MAP, KSAT>(p, bars, g, threadIdx.x - 128 - g * 128,
+    map_half<D, FP8, MAP, KSAT, DBG>(p, bars, g, threadIdx.x - 128 - g * 128,
                            tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh,
                            sTab, xc, abort);
   }
@@ -838,23 +840,25 @@ static qsm_status launch_t(const FwdArgs &a, const CUtensorMap &mq, const CUtens
   if (smem < 120 * 1024) smem = 120 * 1024;
   if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
-  auto kern = qsm_fwd_kernel<D, FP8, MAP, KSAT>;
+  // the decision dump, when asked for, runs in its own instantiation
+  const int dbg = p.dbg != nullptr ? 1 : 0;
+  auto kern = dbg ? qsm_fwd_kernel<D, FP8, MAP, KSAT, true> : qsm_fwd_kernel<D, FP8, MAP, KSAT, false>;
   // Raising the kernel's dynamic shared memory limit is a driver round trip;
   // this instantiation remembers, per device, the largest limit already set.
-  static std::atomic<int> smem_set[kMaxDevices];
+  static std::atomic<int> smem_set[2][kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QSM_ERR_CUDA;
   const bool cached = dev >= 0 && dev < kMaxDevices &&
-                      smem_set[dev].load(std::memory_order_acquire) >= static_cast<int>(smem);
+                      smem_set[dbg][dev].load(std::memory_order_acquire) >= static_cast<int>(smem);
   if (!cached) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return QSM_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices) {
-      int prev = smem_set[dev].load(std::memory_order_relaxed);
+      int prev = smem_set[dbg][dev].load(std::memory_order_relaxed);
       while (prev < static_cast<int>(smem) &&
-             !smem_set[dev].compare_exchange_weak(prev, static_cast<int>(smem),
-                                                  std::memory_order_acq_rel)) {
+             !smem_set[dbg][dev].compare_exchange_weak(prev, static_cast<int>(smem),
+                                                       std::memory_order_acq_rel)) {
       }
     }
   }

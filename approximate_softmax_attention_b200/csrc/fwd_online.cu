@@ -321,8 +321,10 @@ __device__ __forceinline__ void on_anchor(const OnParams &p, const OnBars &bars,
 
 // One map warpgroup.  Thread `row` owns query row qi*128 + row (TMEM lane
 // `row`) and maps key tiles j = g, g + 3, ... in S buffer g against the
-// anchor and frame the anchor group published for the tile.
-template <int D, bool FP8, int MAP, bool KSAT>
+// anchor and frame the anchor group published for the tile.  DBG: the
+// kernel writes the decision dump (a separate instantiation, so that the
+// dump's code takes no registers from the ordinary one).
+template <int D, bool FP8, int MAP, bool KSAT, bool DBG>
 __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, const OnRows &rs,
                                        int g, int row, uint32_t lane_base, int qi, int n, int bh,
                                        float *tab, volatile int *abort) {
@@ -359,7 +361,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   for (int i = 0; i < 4; ++i) z[i] = make_float2(0.0f, 0.0f);
   float zbase = 0.0f;                  // frame of this group's row sums
   bool zset = false;
-  int8_t *dbg_row = (p.dbg != nullptr && row_ok)
+  int8_t *dbg_row = (DBG && p.dbg != nullptr && row_ok)
                         ? p.dbg + (static_cast<size_t>(bh) * p.S + qrow) * p.S
                         : nullptr;
 
@@ -480,7 +482,7 @@ __device__ __forceinline__ void on_map(const OnParams &p, const OnBars &bars, co
   }
 }
 
-template <int D, bool FP8, int MAP, bool KSAT>
+template <int D, bool FP8, int MAP, bool KSAT, bool DBG>
 __global__ void __launch_bounds__(kOnThreads, 1)
     qsm_fwd_online_kernel(const __grid_constant__ CUtensorMap tmQ,
                           const __grid_constant__ CUtensorMap tmK,
@@ -686,7 +688,7 @@ __global__ void __launch_bounds__(kOnThreads, 1)
                       tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, abort);
   } else if (warp >= 8) {
     const int g = (warp - 8) >> 2;
-    on_map<D, FP8, MAP, KSAT>(p, bars, rs, g, threadIdx.x - 256 - g * 128,
+    on_map<D, FP8, MAP, KSAT, DBG>(p, bars, rs, g, threadIdx.x - 256 - g * 128,
                         tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), qi, n, bh, sTab,
                         abort);
   }
@@ -757,21 +759,24 @@ qsm_status launch_on_t(const FwdArgs &a, const CUtensorMap &mq, const CUtensorMa
   if (smem < 120 * 1024) smem = 120 * 1024;            // one CTA per SM (all of TMEM)
   if (smem > max_smem) return QSM_ERR_UNSUPPORTED;
 
-  auto kern = qsm_fwd_online_kernel<D, FP8, MAP, KSAT>;
-  static std::atomic<int> smem_set[kMaxDevices];
+  // the decision dump, when asked for, runs in its own instantiation
+  const int dbg = p.dbg != nullptr ? 1 : 0;
+  auto kern = dbg ? qsm_fwd_online_kernel<D, FP8, MAP, KSAT, true>
+                  : qsm_fwd_online_kernel<D, FP8, MAP, KSAT, false>;
+  static std::atomic<int> smem_set[2][kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QSM_ERR_CUDA;
   const bool cached = dev >= 0 && dev < kMaxDevices &&
-                      smem_set[dev].load(std::memory_order_acquire) >= static_cast<int>(smem);
+                      smem_set[dbg][dev].load(std::memory_order_acquire) >= static_cast<int>(smem);
   if (!cached) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return QSM_ERR_CUDA;
     if (dev >= 0 && dev < kMaxDevices) {
-      int prev = smem_set[dev].load(std::memory_order_relaxed);
+      int prev = smem_set[dbg][dev].load(std::memory_order_relaxed);
       while (prev < static_cast<int>(smem) &&
-             !smem_set[dev].compare_exchange_weak(prev, static_cast<int>(smem),
-                                                  std::memory_order_acq_rel)) {
+             !smem_set[dbg][dev].compare_exchange_weak(prev, static_cast<int>(smem),
+                                                       std::memory_order_acq_rel)) {
       }
     }
   }
