@@ -186,6 +186,18 @@ __device__ __forceinline__ void kv_tile_of(const BwdParams &p, int b, int &bh, i
   }
 }
 
+// Tile number of this CTA's round k in a persistent pass: the heaviest-first
+// tile list is dealt out in rounds of gridDim.x tiles, in block order in the
+// even rounds and in reverse block order in the odd ones, so that the CTA
+// that takes a round's heaviest tile takes the lightest of the next (dealing
+// in block order every round leaves the low blocks the heaviest tile of each
+// round).  Strictly increasing in k: the first number >= the tile count ends
+// the CTA's sequence.
+__device__ __forceinline__ int cta_tile(int k) {
+  const int g = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  return k * g + ((k & 1) ? g - 1 - b : b);
+}
+
 // bf16 bit patterns to fp32 (exact).
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -231,8 +243,8 @@ struct RowBars {
 // sums are taken at the fixed offset hi (no running maximum, no rescaling):
 // L = sum_j 2^(x_j), A = sum_j 2^(x_j) dp_j with x_j = (s_j - hi) log2 e, and
 // LSE* = hi + ln L, delta* = A / L.
-// Persistent like the dQ pass: one CTA per SM takes the query tiles t =
-// blockIdx.x, blockIdx.x + gridDim.x, ...; S = Q K^T and dP = dO V^T of whole
+// Persistent like the dQ pass: one CTA per SM takes the query tiles
+// cta_tile(0), cta_tile(1), ...; S = Q K^T and dP = dO V^T of whole
 // 128-key tiles (products of N = 128: the map here is light, so the products
 // set the pace) in TMEM pair n mod 2 (n counting key tiles across query
 // tiles; S at 256 (n mod 2), dP 128 columns on); thread = query row, map
@@ -249,7 +261,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = p.nqt * p.BH;
-  const int step = static_cast<int>(gridDim.x);
   const int ns = p.num_stages;
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int it = 0, k = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -335,7 +346,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int it0 = 0, k = 0;
       const uint32_t qa = smem_u32(sQ), da = smem_u32(sdO), kva = smem_u32(sKV);
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -399,15 +410,16 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     bool ok = true;
     int n = 0, k = 0;
     float pv_hi = 0.0f;
-    float hi_next = static_cast<int>(blockIdx.x) < ntiles ? row_hi(blockIdx.x) : 0.0f;
-    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+    float hi_next = cta_tile(0) < ntiles ? row_hi(cta_tile(0)) : 0.0f;
+    for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
       int bh, qt;
       q_tile_of(p, t, bh, qt);
       const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
       const int qrow = qt * 128 + row;
       const int L = p.causal ? min(qrow + 1, p.S) : p.S;
       const float hi = hi_next;
-      if (t + step < ntiles) hi_next = row_hi(t + step);     // consumed a tile later
+      const int t_next = cta_tile(k + 1);
+      if (t_next < ntiles) hi_next = row_hi(t_next);          // consumed a tile later
       const float hl = __fmul_rn(hi, log2e_f());
       const float2 nh = make_float2(-hl, -hl);
       float2 l2 = make_float2(0.0f, 0.0f), a2 = make_float2(0.0f, 0.0f);
@@ -447,13 +459,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       pp[g * 128 + row] = l2.x + l2.y;
       pp[512 + g * 128 + row] = a2.x + a2.y;
       mbar_arrive(&bars.part_ready[k & 1]);
-      if (k >= 1 && !finish(t - step, k - 1, pv_hi)) {
+      if (k >= 1 && !finish(cta_tile(k - 1), k - 1, pv_hi)) {
         ok = false;
         break;
       }
       pv_hi = hi;
     }
-    if (ok && k >= 1) finish(static_cast<int>(blockIdx.x) + (k - 1) * step, k - 1, pv_hi);
+    if (ok && k >= 1) finish(cta_tile(k - 1), k - 1, pv_hi);
   }
   __syncwarp();
   tc_fence_before();
@@ -768,8 +780,8 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
 }
 
 // ----------------------------------------------------------------- dQ pass
-// Persistent: one CTA per SM takes the 128-row query tiles t = blockIdx.x,
-// blockIdx.x + gridDim.x, ... in the heaviest-first order; thread = query row
+// Persistent: one CTA per SM takes the 128-row query tiles cta_tile(0),
+// cta_tile(1), ... of the heaviest-first order; thread = query row
 // (TMEM lane); the key tiles are taken in halves of 64 keys, half number hc
 // (counted across tiles) in TMEM pair x = hc mod 3 (S at 128x, dP at 128x +
 // 64) and shared dS buffer x; map group g owns keys 16g .. 16g+15 of each
@@ -827,7 +839,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = p.nqt * p.BH;
-  const int step = static_cast<int>(gridDim.x);
   const int ns = p.num_stages;
   uint8_t *sQ = smem;
   uint8_t *sdO = smem + G::TILE_BYTES;
@@ -887,8 +898,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
-  // Tiles of this CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ... of the
-  // heaviest-first order (persistent: the next tile's loads and first
+  // Tiles of this CTA: cta_tile(0), cta_tile(1), ... of the heaviest-first
+  // order (persistent: the next tile's loads and first
   // products overlap this tile's last halves).  Every role walks the same
   // sequence; the ring position `it` and the half counter `hc` run on across
   // tiles, and per-tile barriers take the tile's own parity.
@@ -896,7 +907,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int it = 0, k = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -935,7 +946,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int it0 = 0, hc = 0, k = 0;
       const uint32_t qa = smem_u32(sQ), da = smem_u32(sdO), kva = smem_u32(sKV);
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -972,7 +983,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int it0 = 0, hc = 0, k = 0;
       const uint32_t kva = smem_u32(sKV), dsa = smem_u32(sDS);
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -1014,7 +1025,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int k = 0;
       const uint32_t cbytes = 128u * kCst * 4;
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, qt;
         q_tile_of(p, t, bh, qt);
         if (k >= 1) ok = mbar_wait(bars.tab_free, (k - 1) & 1, abort);
@@ -1157,7 +1168,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     int hc = 0, k = 0;
     int pv_amx = -1, pv_amn = 0;        // the previous tile's read-out state
     float pv_kinv = 0.0f;
-    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+    for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
       int bh, qt;
       q_tile_of(p, t, bh, qt);
       const int nkv = p.causal ? min(p.nkvt, qt + 1) : p.nkvt;
@@ -1251,7 +1262,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       pp[g * 128 + row] = s1.x + s1.y;
       pp[512 + g * 128 + row] = s2.x + s2.y;
       mbar_arrive(&bars.part_ready[k & 1]);
-      if (k >= 1 && !read_out(t - step, k - 1, pv_amx, pv_amn, pv_kinv)) {
+      if (k >= 1 && !read_out(cta_tile(k - 1), k - 1, pv_amx, pv_amn, pv_kinv)) {
         ok = false;
         break;
       }
@@ -1259,7 +1270,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       pv_amn = amn;
       pv_kinv = dk.kinv;
     }
-    if (ok && k >= 1) read_out(static_cast<int>(blockIdx.x) + (k - 1) * step, k - 1, pv_amx,
+    if (ok && k >= 1) read_out(cta_tile(k - 1), k - 1, pv_amx,
                                pv_amn, pv_kinv);
   }
   __syncwarp();
@@ -1425,7 +1436,6 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   uint8_t *smem = smem_align1024(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntiles = p.nkvt * p.BH;
-  const int step = static_cast<int>(gridDim.x);
   const int ns = p.num_stages;
   uint8_t *sK = smem;
   uint8_t *sV = smem + G::TILE_BYTES;
@@ -1473,14 +1483,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
 
-  // Tiles of this CTA: t = blockIdx.x, blockIdx.x + gridDim.x, ... of the
-  // heaviest-first key-tile order (persistent, as the dQ pass); the ring
+  // Tiles of this CTA: cta_tile(0), cta_tile(1), ... of the heaviest-first
+  // key-tile order (persistent, as the dQ pass); the ring
   // position and the half counter run on across tiles.
   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
       int rc = 0, k = 0;
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, kt;
         kv_tile_of(p, t, bh, kt);
         const int i0 = p.causal ? kt : 0;                // first query tile
@@ -1527,7 +1537,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int rc0 = 0, hc = 0, k = 0;
       const uint32_t ka = smem_u32(sK), va = smem_u32(sV), sa = smem_u32(sSt);
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, kt;
         kv_tile_of(p, t, bh, kt);
         const int nq = p.nqt - (p.causal ? kt : 0);
@@ -1563,7 +1573,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       bool ok = true;
       int rc0 = 0, hc = 0, k = 0;
       const uint32_t sa = smem_u32(sSt);
-      for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+      for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
         int bh, kt;
         kv_tile_of(p, t, bh, kt);
         const int nq = p.nqt - (p.causal ? kt : 0);
@@ -1615,7 +1625,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
     bool ok = true;
     int rc0 = 0, hc = 0, k = 0;
-    for (int t = blockIdx.x; t < ntiles && ok; t += step, ++k) {
+    for (int t = cta_tile(k); t < ntiles && ok; t = cta_tile(++k)) {
       int bh, kt;
       kv_tile_of(p, t, bh, kt);
       const int i0 = p.causal ? kt : 0;                  // first query tile
