@@ -23,9 +23,10 @@
 //   1. qsm_bwd_rows   post surrogate only: LSE* and delta* per query row, sums
 //                     of 2^((s - hi) log2 e) at the forward's row maximum over
 //                     whole S and dP tiles (persistent)
-//   2. qsm_bwd_prep   one CTA per query tile, thread = row: delta = dO . O, the
-//                     map constants and grid tables of both passes, into the
-//                     workspace
+//   2. qsm_bwd_prep   one CTA per query tile, two or four threads a row: delta =
+//                     dO . O, the map constants and grid tables of both
+//                     passes, into the workspace; zeroes the tile's rows of
+//                     the fp32 calibration part of dK
 //   3. qsm_bwd_dq     persistent, one CTA per SM over the query tiles: a tile's
 //                     constants and table copied in, then the key tiles in
 //                     halves of 64 keys: S = Q K^T and dP = dO V^T into one of
@@ -569,14 +570,14 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, Row
   return k;
 }
 
-// The grid tables of one row (K-interval): the dK / dV pass's row tk (TS
-// floats) and the dQ pass's entries, entry i at byte tq + i * STRIDE.  The
-// grid values g_k are formed first, all independent (the loop is unrolled
-// to the largest K, guarded by K), and each serves the two intervals it
-// bounds; x/K is a product with 1/K when K is a power of two (exact, so the
-// same value).
-template <int MAP, int SURR, int CAL>
-__device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm, float *tk,
+// The grid tables of one row (K-interval), the part of thread q = 0..NQ-1
+// of the row's NQ: the dK / dV pass's row tk (TS floats) and the dQ pass's
+// entries, entry i at byte tq + i * STRIDE.  Thread q takes the intervals
+// (interpolation) or grid values (hard rounding) k = q, q + NQ, ... and
+// forms the grid values it needs itself; x/K is a product with 1/K when K
+// is a power of two (exact, so the same value).
+template <int MAP, int SURR, int CAL, int NQ>
+__device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm, int q, float *tk,
                                            uint8_t *tq) {
   using T = DqTab<MAP, SURR, CAL>;
   const int K = p.K;
@@ -584,9 +585,6 @@ __device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm,
   const bool p2 = (K & (K - 1)) == 0;
   const float rK = 1.0f / Kf;
   auto divK = [&](float x) { return p2 ? __fmul_rn(x, rK) : __fdiv_rn(x, Kf); };
-  float gv[kBwdMaxK + 1];
-#pragma unroll
-  for (int n = 0; n <= kBwdMaxK; ++n) gv[n] = n <= K ? grid_value(rm, K, n) : 0.0f;
   if (MAP == MAPB_INTERP) {
     const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(rm.hi, rm.lo));
     auto put = [&](int i, float e, float d, float A, float B) {
@@ -596,34 +594,33 @@ __device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm,
       else if (T::ANY)
         *reinterpret_cast<float *>(tq + i * T::STRIDE) = d;
     };
-    // below the window: fixed window g_0 (0 when flushed), no derivative
-    if (p.fixed_window) put(0, p.flush ? 0.0f : gv[0], 0.0f, 0.0f, 0.0f);
-#pragma unroll
-    for (int kk = 0; kk < kBwdMaxK; ++kk) {
-      if (kk < K) {
-        const float gk = gv[kk], gk1 = gv[kk + 1];
-        const float kf = static_cast<float>(kk), kmk = static_cast<float>(K - kk);
-        const float d = __fsub_rn(gk1, gk);
-        const float e = __fmaf_rn(-kf, d, gk);
-        float A = 0.0f, B = 0.0f;
-        if (CAL == CAL_MINMAX) {
-          A = -divK(__fmaf_rn(kmk, e, __fmul_rn(kf, gk1)));
-          B = __fsub_rn(-__fmul_rn(d, inv_a), divK(__fsub_rn(__fmul_rn(kmk, d), gk1)));
-        }
-        put(kk + 1, e, d, A, B);
-        if (kk == 0 && !p.fixed_window) put(0, e, d, A, B);   // min-max: below = interval 0
-        if (kk == K - 1) put(K + 1, e, d, A, B);              // u = K: interval K - 1
+    for (int kk = q; kk < K; kk += NQ) {
+      const float gk = grid_value(rm, K, kk), gk1 = grid_value(rm, K, kk + 1);
+      const float kf = static_cast<float>(kk), kmk = static_cast<float>(K - kk);
+      const float d = __fsub_rn(gk1, gk);
+      const float e = __fmaf_rn(-kf, d, gk);
+      float A = 0.0f, B = 0.0f;
+      if (CAL == CAL_MINMAX) {
+        A = -divK(__fmaf_rn(kmk, e, __fmul_rn(kf, gk1)));
+        B = __fsub_rn(-__fmul_rn(d, inv_a), divK(__fsub_rn(__fmul_rn(kmk, d), gk1)));
       }
+      put(kk + 1, e, d, A, B);
+      if (kk == 0) {
+        // below the window: fixed window g_0 (0 when flushed), no
+        // derivative; min-max: interval 0
+        if (p.fixed_window)
+          put(0, p.flush ? 0.0f : gk, 0.0f, 0.0f, 0.0f);
+        else
+          put(0, e, d, A, B);
+      }
+      if (kk == K - 1) put(K + 1, e, d, A, B);            // u = K: interval K - 1
     }
   } else {
-#pragma unroll
-    for (int n = 0; n <= kBwdMaxK; ++n) {
-      if (n <= K) {
-        tk[n] = gv[n];
-        if (T::ANY)
-          *reinterpret_cast<float *>(tq + n * T::STRIDE) =
-              __fmul_rn(divK(static_cast<float>(n - K)), gv[n]);
-      }
+    for (int n = q; n <= K; n += NQ) {
+      const float g = grid_value(rm, K, n);
+      tk[n] = g;
+      if (T::ANY)
+        *reinterpret_cast<float *>(tq + n * T::STRIDE) = __fmul_rn(divK(static_cast<float>(n - K)), g);
     }
   }
 }
@@ -658,58 +655,90 @@ __global__ void __launch_bounds__(256)
 }
 
 // ----------------------------------------------------------- row prep
-// One CTA of 128 threads per query tile, thread = row: each row's delta =
-// dO_r . O_r, map constants and grid tables, written to the workspace -- the
-// constants (both passes), the dK / dV pass's table per row and the dQ
-// pass's table per tile in its shared-memory layout (entry-major, so the
-// rows of a warp store one contiguous run), which the dQ pass copies in with
-// one bulk load per tile.  Rows past S in a ragged last tile take the last
-// row's values, so every workspace entry of a tile is defined.
+// One CTA of 128 NQ threads per query tile, NQ threads a row (thread q of
+// row r is thread 128 q + r; NQ = 4 for interpolation, whose tables are the
+// longest, else 2): each row's delta = dO_r . O_r (four D/4-column parts,
+// 4/NQ of them a thread), map constants and grid tables (thread q every
+// NQ-th entry), written to the workspace -- the constants (both
+// passes), the dK / dV pass's table per row (staged in shared memory, then
+// copied out as one contiguous run per tile) and the dQ pass's table per
+// tile in its shared-memory layout (entry-major, so the rows of a warp store
+// one contiguous run), which the dQ pass copies in with one bulk load per
+// tile.  The tile's rows of the fp32 calibration part of dK are zeroed here,
+// ahead of the dQ pass's reductions into them.  Rows past S in a ragged last
+// tile take the last row's values, so every workspace entry of a tile is
+// defined.
+constexpr int kTabKRow = 2 * ((kBwdMaxK + 2) & ~1);     // floats: the widest table row (TS)
+template <int MAP>
+constexpr int prep_split() { return MAP == MAPB_INTERP ? 4 : 2; }
+
 template <int D, int MAP, int SURR, int CAL>
-__global__ void __launch_bounds__(128, 4)
+__global__ void __launch_bounds__(128 * prep_split<MAP>())
     qsm_bwd_prep(const BwdParams p) {
   using T = DqTab<MAP, SURR, CAL>;
+  constexpr int NQ = prep_split<MAP>(), NT = 128 * NQ;
   static_assert(D == 64 || D == 128, "delta in four D/4-column parts");
-  const int row = threadIdx.x;
+  constexpr bool KI = MAP == MAPB_HARD || MAP == MAPB_INTERP;
+  __shared__ float dpart[4][128];
+  __shared__ __align__(16) float tks[KI ? 128 * kTabKRow : 4];
+  const int row = threadIdx.x & 127, q = threadIdx.x >> 7;
   const int tix = static_cast<int>(blockIdx.x);         // bh * nqt + qt
   const int bh = tix / p.nqt, qt = tix - bh * p.nqt;
   const int qrow = qt * 128 + row;
   const bool row_ok = qrow < p.S;
   const size_t ri = static_cast<size_t>(bh) * p.S + min(qrow, p.S - 1);
-  // delta in four D/4-column parts (each a running sum over its 8-column
-  // chunks), summed pairwise
-  constexpr int CPP = D / 32;                             // 8-column chunks per part
-  float part[4];
   {
+    // this thread's parts of delta (parts q, q + NQ, ...), each a running
+    // sum over its 8-column chunks
+    constexpr int CPP = D / 32;                           // 8-column chunks per part
+    constexpr int PPT = 4 / NQ;                           // parts per thread
     const uint4 *o4 = reinterpret_cast<const uint4 *>(p.O + ri * D);
     const uint4 *d4 = reinterpret_cast<const uint4 *>(p.dO + ri * D);
-    uint4 ov[D / 8], dv[D / 8];
+    uint4 ov[PPT][CPP], dv[PPT][CPP];
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      ov[i] = o4[i];
-      dv[i] = d4[i];
-    }
+    for (int j = 0; j < PPT; ++j)
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
+      for (int c = 0; c < CPP; ++c) {
+        ov[j][c] = o4[CPP * (q + NQ * j) + c];
+        dv[j][c] = d4[CPP * (q + NQ * j) + c];
+      }
+#pragma unroll
+    for (int j = 0; j < PPT; ++j) {
       float acc = 0.0f;
 #pragma unroll
-      for (int c = 0; c < CPP; ++c) acc = dot_bf16x8(ov[CPP * g + c], dv[CPP * g + c], acc);
-      part[g] = acc;
+      for (int c = 0; c < CPP; ++c) acc = dot_bf16x8(ov[j][c], dv[j][c], acc);
+      dpart[q + NQ * j][row] = acc;
     }
   }
-  const float delta = (part[0] + part[1]) + (part[2] + part[3]);
+  if (p.dkcal != nullptr) {
+    const int nrow = min(128, p.S - qt * 128);
+    float4 *z = reinterpret_cast<float4 *>(p.dkcal + (static_cast<size_t>(bh) * p.S + qt * 128) * D);
+    for (int i = static_cast<int>(threadIdx.x); i < nrow * (D / 4); i += NT)
+      z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
   RowMap rm{};
   RowC kc = row_constants<MAP, SURR, CAL>(p, ri, rm);
-  if (MAP == MAPB_EXACT)
-    kc.ds_ = delta;
-  else
-    kc.nDZ = -__fmul_rn(delta, kc.invZ);
-  if (!row_ok) kc.calib = false;
-  const size_t trow = tile_row(p, bh, qt, row);
-  store_row_constants(p, trow, kc);
-  if (MAP == MAPB_HARD || MAP == MAPB_INTERP)
-    row_tables<MAP, SURR, CAL>(p, rm, p.tabk + trow * p.TS,
+  if (KI)
+    row_tables<MAP, SURR, CAL, NQ>(p, rm, q, tks + row * p.TS,
                                p.tabq + static_cast<size_t>(tix) * p.tabq_tile + row * T::ESZ);
+  __syncthreads();
+  if (q == 0) {
+    const float delta = (dpart[0][row] + dpart[1][row]) + (dpart[2][row] + dpart[3][row]);
+    if (MAP == MAPB_EXACT)
+      kc.ds_ = delta;
+    else
+      kc.nDZ = -__fmul_rn(delta, kc.invZ);
+    if (!row_ok) kc.calib = false;
+    store_row_constants(p, tile_row(p, bh, qt, row), kc);
+  }
+  if (KI) {
+    // the tile's table rows are contiguous in the workspace (TS a multiple
+    // of four floats): 16-byte copies
+    const int n4 = 32 * p.TS;
+    const float4 *src = reinterpret_cast<const float4 *>(tks);
+    float4 *dst = reinterpret_cast<float4 *>(p.tabk + static_cast<size_t>(tix) * 128 * p.TS);
+    for (int i = static_cast<int>(threadIdx.x); i < n4; i += NT) dst[i] = src[i];
+  }
 }
 
 // The dQ pass's per-row values for the element loop.
@@ -1883,7 +1912,8 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
 
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_prep(const BwdArgs &a, const BwdParams &p) {
-  qsm_bwd_prep<D, MAP, SURR, CAL><<<dim3(p.nqt * a.B * a.H), 128, 0, a.stream>>>(p);
+  qsm_bwd_prep<D, MAP, SURR, CAL><<<dim3(p.nqt * a.B * a.H), 128 * prep_split<MAP>(), 0,
+                                    a.stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
@@ -2072,9 +2102,7 @@ qsm_status launch_bwd(const BwdArgs &a) {
       !make_tmap_3d(&m.dO_stage, a.dO, false, a.D, a.S, bh, srows))
     return QSM_ERR_CUDA;
 
-  if (p.dkcal != nullptr &&
-      cudaMemsetAsync(p.dkcal, 0, rows * a.D * sizeof(float), a.stream) != cudaSuccess)
-    return QSM_ERR_CUDA;
+  // (the prep kernel zeroes the calibration part of dK, p.dkcal)
   return a.D == 64 ? launch_maps<64>(a, p, map, cal, m) : launch_maps<128>(a, p, map, cal, m);
 }
 
