@@ -476,16 +476,27 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   if (threadIdx.x == 0 && *bars.abort && p.status != nullptr) atomicExch(p.status, QSM_ERR_TIMEOUT);
 }
 
+// The dK / dV pass evaluates the coordinate in the saturating form
+// (fma_sat on the coordinate divided by K) when K = 2^m, unless the
+// below-window flush or the no-surrogate rule needs what the saturation
+// hides (the coordinate's sign, the below-window entry's zero derivative).
+// The prep kernel lays the pass's table out for the same choice.
+template <int SURR>
+__device__ __forceinline__ bool kv_sat(const BwdParams &p) {
+  return SURR != SURR_NONE && k_pow2(p.K) && p.flush == 0;
+}
+
 // ------------------------------------------------------------ row constants
 // The constants of one query row, as both passes use them (registers in the
 // dQ pass, the workspace copy cst in the dK / dV pass):
 //   a, b   coordinate u = fma(r, a, b) on the raw product r (PoT: the
-//          exponent coordinate, a = -c log2e, b = hi log2e)
+//          exponent coordinate, a = -c log2e, b = hi log2e); K-interval
+//          with K = 2^m: a / K and b / K (exact), for the saturating form
 //   invZ   1/Z, Z = exp(LSE - hi)
 //   nDZ    -delta/Z, so that gw = fma(dp, invZ, nDZ)
 //   e0     the surrogate's exponent offset in log2 units: exact LSE log2e,
 //          pre hi log2e, post LSE* log2e (w* = 2^(r c log2e - e0))
-//   ds_    delta (exact) or delta* (post)
+//   ds_    delta (exact, no surrogate) or delta* (post)
 //   kinv   K / (hi - lo): d coordinate / d score (0 for a degenerate row)
 struct RowC {
   float a, b, invZ, nDZ, e0, ds_, kinv;
@@ -522,8 +533,10 @@ __device__ __forceinline__ void store_row_constants(const BwdParams &p, size_t t
 //   dQ pass (shared memory, [entry][128 rows]): interpolation with min-max
 //   calibration (A, B, d, 0); interpolation otherwise d; hard rounding with
 //   min-max calibration (n - K)/K g_n.
-//   dK / dV pass (workspace, [row][TS]): interpolation (e, d) pairs with
-//   w = fma(u, d, e); hard rounding g_n.
+//   dK / dV pass (workspace, [row][TS]), times 1/Z (so that the lookup is P
+//   itself): interpolation (e, d) pairs with P = fma(u, d, e), on the
+//   saturating path (kv_sat) (e, K d) with P = fma(u / K, K d, e); hard
+//   rounding g_n.
 template <int MAP, int SURR, int CAL>
 struct DqTab {
   static constexpr bool KI = MAP == MAPB_HARD || MAP == MAPB_INTERP;
@@ -558,6 +571,13 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, Row
     rm = make_rowmap(hi, p.lo != nullptr ? p.lo[ri] : hi, p.K, p.fixed_window != 0, p.window);
     k.a = rm.degenerate ? 0.0f : __fmul_rn(p.c, rm.inv);
     k.b = rm.degenerate ? static_cast<float>(p.K) : rm.b;
+    if (k_pow2(p.K)) {
+      // K = 2^m: kept divided by K (exact), the coordinate of the saturating
+      // form fma_sat(r, a, b) = clamp(u, 0, K) / K
+      const float invK = 1.0f / static_cast<float>(p.K);
+      k.a = __fmul_rn(k.a, invK);
+      k.b = __fmul_rn(k.b, invK);
+    }
     k.e0 = rm.hiL2E;
     k.kinv = rm.inv;
     k.calib = CAL != CAL_OFF && !rm.degenerate;
@@ -577,18 +597,20 @@ __device__ __forceinline__ RowC row_constants(const BwdParams &p, size_t ri, Row
 // forms the grid values it needs itself; x/K is a product with 1/K when K
 // is a power of two (exact, so the same value).
 template <int MAP, int SURR, int CAL, int NQ>
-__device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm, int q, float *tk,
-                                           uint8_t *tq) {
+__device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm, float invZ, int q,
+                                           float *tk, uint8_t *tq) {
   using T = DqTab<MAP, SURR, CAL>;
   const int K = p.K;
   const float Kf = static_cast<float>(K);
+  const bool sat = kv_sat<SURR>(p);
   const bool p2 = (K & (K - 1)) == 0;
   const float rK = 1.0f / Kf;
   auto divK = [&](float x) { return p2 ? __fmul_rn(x, rK) : __fdiv_rn(x, Kf); };
   if (MAP == MAPB_INTERP) {
     const float inv_a = rm.degenerate ? 0.0f : __fdiv_rn(1.0f, __fsub_rn(rm.hi, rm.lo));
     auto put = [&](int i, float e, float d, float A, float B) {
-      *reinterpret_cast<float2 *>(tk + 2 * i) = make_float2(e, d);
+      *reinterpret_cast<float2 *>(tk + 2 * i) =
+          make_float2(__fmul_rn(e, invZ), __fmul_rn(sat ? __fmul_rn(d, Kf) : d, invZ));
       if (CAL == CAL_MINMAX)
         *reinterpret_cast<float4 *>(tq + i * T::STRIDE) = make_float4(A, B, d, 0.0f);
       else if (T::ANY)
@@ -618,7 +640,7 @@ __device__ __forceinline__ void row_tables(const BwdParams &p, const RowMap &rm,
   } else {
     for (int n = q; n <= K; n += NQ) {
       const float g = grid_value(rm, K, n);
-      tk[n] = g;
+      tk[n] = __fmul_rn(g, invZ);
       if (T::ANY)
         *reinterpret_cast<float *>(tq + n * T::STRIDE) = __fmul_rn(divK(static_cast<float>(n - K)), g);
     }
@@ -719,15 +741,13 @@ __global__ void __launch_bounds__(128 * prep_split<MAP>())
   RowMap rm{};
   RowC kc = row_constants<MAP, SURR, CAL>(p, ri, rm);
   if (KI)
-    row_tables<MAP, SURR, CAL, NQ>(p, rm, q, tks + row * p.TS,
+    row_tables<MAP, SURR, CAL, NQ>(p, rm, kc.invZ, q, tks + row * p.TS,
                                p.tabq + static_cast<size_t>(tix) * p.tabq_tile + row * T::ESZ);
   __syncthreads();
   if (q == 0) {
     const float delta = (dpart[0][row] + dpart[1][row]) + (dpart[2][row] + dpart[3][row]);
-    if (MAP == MAPB_EXACT)
-      kc.ds_ = delta;
-    else
-      kc.nDZ = -__fmul_rn(delta, kc.invZ);
+    if (MAP == MAPB_EXACT || SURR == SURR_NONE) kc.ds_ = delta;
+    if (MAP != MAPB_EXACT) kc.nDZ = -__fmul_rn(delta, kc.invZ);
     if (!row_ok) kc.calib = false;
     store_row_constants(p, tile_row(p, bh, qt, row), kc);
   }
@@ -744,12 +764,15 @@ __global__ void __launch_bounds__(128 * prep_split<MAP>())
 // The dQ pass's per-row values for the element loop.
 struct DqK {
   float a, b, invZ, nDZ, ne0, nds, kinv, cL2E, Kf;
+  float mk;          // hard rounding, K = 2^m: 1.5 * 2^23 / K
   uint32_t tq_row;   // biased shared address of this row's dQ-pass table
 };
 
 // dS of one 16-key slice of a row (bf16 pairs into dd) and the calibration
-// sums, two elements per packed fp32 operation.  FULL: every key valid.
-template <int MAP, int SURR, int CAL, bool FULL>
+// sums, two elements per packed fp32 operation.  FULL: every key valid.  SAT
+// (hard rounding, K = 2^m): the node from the saturating coordinate, rne of
+// fma_sat(r, a/K, b/K) at a unit of 1/K -- rne(clamp(u, 0, K)), the same node.
+template <int MAP, int SURR, int CAL, bool FULL, bool SAT = false>
 __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
                                          const DqK &k, int lim, uint32_t (&dd)[8], float2 &s1,
                                          float2 &s2) {
@@ -793,8 +816,15 @@ __device__ __forceinline__ void dq_slice(const uint32_t (&sv)[16], const uint32_
           }
           if (SURR == SURR_NONE) ds = mul2_rn(mul2_rn(gw, d), make_float2(k.kinv, k.kinv));
         } else {
-          const float2 uc = make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
-          const float2 t = add2_rn(uc, mg);
+          float2 t;
+          if (SAT) {
+            t = add2_rn(make_float2(fma_sat(r.x, k.a, k.b), fma_sat(r.y, k.a, k.b)),
+                        make_float2(k.mk, k.mk));
+          } else {
+            const float2 uc =
+                make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
+            t = add2_rn(uc, mg);
+          }
           s1 = fma2_rn(gw,
                        make_float2(lds_f32(__float_as_uint(t.x) * T::STRIDE + k.tq_row),
                                    lds_f32(__float_as_uint(t.y) * T::STRIDE + k.tq_row)),
@@ -1209,10 +1239,18 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       if (!ok) break;
       // table addresses: the entry is bits(M + floor(clamp(u, -1, K))) -
       // bits(M) + 1 (interpolation) or bits(M + rne(clamp(u, 0, K))) - bits(M)
-      // (hard), M = 1.5 * 2^23; the address arithmetic wraps mod 2^32
+      // (hard), M = 1.5 * 2^23 -- on the saturating path bits(M/K + v) -
+      // bits(M/K); the address arithmetic wraps mod 2^32.  The stored a, b
+      // are divided by K when K = 2^m: interpolation takes them back (exact).
       DqK dk;
+      const bool kp2 = k_pow2(p.K);
+      const bool hsat = MAP == MAPB_HARD && kp2;        // hard rounding: saturating form
       dk.a = lds_f32(ca);
       dk.b = lds_f32(ca + 8);
+      if (MAP == MAPB_INTERP && kp2) {
+        dk.a = __fmul_rn(dk.a, Kf);
+        dk.b = __fmul_rn(dk.b, Kf);
+      }
       dk.invZ = lds_f32(ca + 16);
       dk.nDZ = lds_f32(ca + 24);
       dk.ne0 = lds_f32(ca + 32);
@@ -1220,9 +1258,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       dk.kinv = lds_f32(ca + 48);
       dk.cL2E = p.cL2E;
       dk.Kf = Kf;
+      dk.mk = hsat ? __fmul_rn(kMagic, 1.0f / Kf) : kMagic;
       dk.tq_row = (MAP == MAPB_INTERP)
                       ? tq_base + row * T::ESZ - kMagicBits * T::STRIDE + T::STRIDE
-                      : tq_base + row * T::ESZ - kMagicBits * T::STRIDE;
+                      : tq_base + row * T::ESZ - __float_as_uint(dk.mk) * T::STRIDE;
       float2 s1 = make_float2(0.0f, 0.0f), s2 = make_float2(0.0f, 0.0f);   // calibration sums
       for (int h = 0; h < 2 * nkv && ok; ++h, ++hc) {
         const int j = h >> 1, e = h & 1, x = hc % HB, u = hc / HB;
@@ -1239,10 +1278,23 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         mbar_arrive(&bars.sdp_free[x]);                // the pair can take half hc + 3
         const int lim = L - (128 * j + 64 * e + 16 * g);  // valid keys of this slice
         uint32_t dd[8];
-        if (warp_all_b(lim >= 16))
+        const bool full = warp_all_b(lim >= 16);
+        if constexpr (MAP == MAPB_HARD) {
+          if (hsat) {
+            if (full)
+              dq_slice<MAP, SURR, CAL, true, true>(sv, dv, dk, lim, dd, s1, s2);
+            else
+              dq_slice<MAP, SURR, CAL, false, true>(sv, dv, dk, lim, dd, s1, s2);
+          } else if (full) {
+            dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
+          } else {
+            dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
+          }
+        } else if (full) {
           dq_slice<MAP, SURR, CAL, true>(sv, dv, dk, lim, dd, s1, s2);
-        else
+        } else {
           dq_slice<MAP, SURR, CAL, false>(sv, dv, dk, lim, dd, s1, s2);
+        }
         if (u >= 1) {
           // the dQ product of half hc - 3 has read dS buffer x
           ok = warp_all_b(mbar_wait(&bars.ds_free[x], (u - 1) & 1, abort));
@@ -1377,6 +1429,8 @@ __device__ __forceinline__ void store_bf16x16_cal(uint4 *d4, const uint32_t (&v)
 // The dK / dV pass's per-thread values for the element loop.
 struct KvK {
   float cL2E, Kf, cap, flush_t;
+  float Ksc;         // K when K = 2^m (the stored a, b are divided by it), else 1
+  float mk;          // saturating form: 1.5 * 2^23 / K
   bool flush, flush_below;
 };
 
@@ -1385,7 +1439,12 @@ struct KvK {
 // slice's first row pair of constants (64 bytes a pair, see
 // store_row_constants); tr: biased shared address of the slice's first row
 // table, ts its row stride in bytes; vmask: valid rows (bit i) unless FULL.
-template <int MAP, int SURR, bool FULL>
+// The K-interval tables hold the weights times 1/Z, so a lookup gives P.
+// SAT (kv_sat): the coordinate divided by K in one saturating FMA, v =
+// clamp(u, 0, K) / K; the node or interval from v + 1.5 * 2^23 / K, whose
+// unit is 1 / K (the same node or interval as from u), and interpolation's
+// P = fma(v, K d, e) with K d in the table.
+template <int MAP, int SURR, bool FULL, bool SAT>
 __device__ __forceinline__ void kv_slice(const uint32_t (&sv)[16], const uint32_t (&dv)[16],
                                          uint32_t cb, uint32_t tr, uint32_t ts, const KvK &k,
                                          uint32_t vmask, uint32_t (&pp)[8], uint32_t (&dd)[8]) {
@@ -1404,43 +1463,67 @@ __device__ __forceinline__ void kv_slice(const uint32_t (&sv)[16], const uint32_
       ds = mul2_rn(pw, add2_rn(dp, make_float2(c2.z, c2.w)));
     } else {
       const float4 c0 = lds_f32x4(c);                      // a pair, b pair
-      const float4 c1 = lds_f32x4(c + 16);                 // 1/Z pair, -delta/Z pair
-      const float2 iz = make_float2(c1.x, c1.y);
-      const float2 gw = fma2_rn(dp, iz, make_float2(c1.z, c1.w));
-      const float2 u = fma2_rn(r, make_float2(c0.x, c0.y), make_float2(c0.z, c0.w));
-      float2 w, dn = make_float2(0.0f, 0.0f);
+      float4 c1 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);    // 1/Z pair, -delta/Z pair
+      if (MAP == MAPB_POT || SURR == SURR_PRE) c1 = lds_f32x4(c + 16);
+      float2 dn = make_float2(0.0f, 0.0f);
       if (MAP == MAPB_POT) {
         // the forward's power-of-two weight (exponent frozen: no own-score or
         // anchor derivative; only the surrogate's direct term)
+        const float2 u = fma2_rn(r, make_float2(c0.x, c0.y), make_float2(c0.z, c0.w));
         const float2 t = add2_rn(make_float2(fminf(u.x, k.cap), fminf(u.y, k.cap)), mg);
-        w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + 0x3F800000u),
-                        __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + 0x3F800000u));
+        float2 w = make_float2(__uint_as_float(__float_as_uint(t.x) * 0xFF800000u + 0x3F800000u),
+                               __uint_as_float(__float_as_uint(t.y) * 0xFF800000u + 0x3F800000u));
         if (k.flush && t.x > k.flush_t) w.x = 0.0f;
         if (k.flush && t.y > k.flush_t) w.y = 0.0f;
-      } else if (MAP == MAPB_HARD) {
-        const float2 uc = make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
-        const float2 t = add2_rn(uc, mg);
-        w = make_float2(lds_f32(__float_as_uint(t.x) * 4u + t0),
-                        lds_f32(__float_as_uint(t.y) * 4u + t1));
-        if (k.flush_below && u.x < 0.0f) w.x = 0.0f;
-        if (k.flush_below && u.y < 0.0f) w.y = 0.0f;
+        pw = mul2_rn(w, make_float2(c1.x, c1.y));
+      } else if (SAT) {
+        const float2 v = make_float2(fma_sat(r.x, c0.x, c0.z), fma_sat(r.y, c0.y, c0.w));
+        const float2 mk = make_float2(k.mk, k.mk);
+        if (MAP == MAPB_HARD) {
+          const float2 t = add2_rn(v, mk);
+          pw = make_float2(lds_f32(__float_as_uint(t.x) * 4u + t0),
+                           lds_f32(__float_as_uint(t.y) * 4u + t1));
+        } else {
+          const float2 t = add2_rd(v, mk);
+          const float2 e0 = lds_f32x2(__float_as_uint(t.x) * 8u + t0);
+          const float2 e1 = lds_f32x2(__float_as_uint(t.y) * 8u + t1);
+          pw = make_float2(__fmaf_rn(v.x, e0.y, e0.x), __fmaf_rn(v.y, e1.y, e1.x));
+        }
       } else {
-        const float2 uc = make_float2(fminf(fmaxf(u.x, -1.0f), k.Kf), fminf(fmaxf(u.y, -1.0f), k.Kf));
-        const float2 t = add2_rd(uc, mg);
-        const float2 e0 = lds_f32x2(__float_as_uint(t.x) * 8u + t0);
-        const float2 e1 = lds_f32x2(__float_as_uint(t.y) * 8u + t1);
-        w = make_float2(__fmaf_rn(uc.x, e0.y, e0.x), __fmaf_rn(uc.y, e1.y, e1.x));
-        dn = make_float2(e0.y, e1.y);
+        // u itself: the stored a, b times Ksc (exact)
+        const float2 ks = make_float2(k.Ksc, k.Ksc);
+        const float2 u = fma2_rn(r, mul2_rn(make_float2(c0.x, c0.y), ks),
+                                 mul2_rn(make_float2(c0.z, c0.w), ks));
+        if (MAP == MAPB_HARD) {
+          const float2 uc =
+              make_float2(fminf(fmaxf(u.x, 0.0f), k.Kf), fminf(fmaxf(u.y, 0.0f), k.Kf));
+          const float2 t = add2_rn(uc, mg);
+          pw = make_float2(lds_f32(__float_as_uint(t.x) * 4u + t0),
+                           lds_f32(__float_as_uint(t.y) * 4u + t1));
+          if (k.flush_below && u.x < 0.0f) pw.x = 0.0f;
+          if (k.flush_below && u.y < 0.0f) pw.y = 0.0f;
+        } else {
+          const float2 uc =
+              make_float2(fminf(fmaxf(u.x, -1.0f), k.Kf), fminf(fmaxf(u.y, -1.0f), k.Kf));
+          const float2 t = add2_rd(uc, mg);
+          const float2 e0 = lds_f32x2(__float_as_uint(t.x) * 8u + t0);
+          const float2 e1 = lds_f32x2(__float_as_uint(t.y) * 8u + t1);
+          pw = make_float2(__fmaf_rn(uc.x, e0.y, e0.x), __fmaf_rn(uc.y, e1.y, e1.x));
+          dn = make_float2(e0.y, e1.y);                    // d / Z
+        }
       }
-      pw = mul2_rn(w, iz);
       if (SURR == SURR_PRE) {
+        const float2 gw =
+            fma2_rn(dp, make_float2(c1.x, c1.y), make_float2(c1.z, c1.w));
         ds = mul2_rn(gw, ex2_pair(fma2_rn(r, cl2, lds_f32x2(c + 32))));
       } else if (SURR == SURR_POST) {
         const float4 c2 = lds_f32x4(c + 32);               // -e0 pair, -delta* pair
         ds = mul2_rn(ex2_pair(fma2_rn(r, cl2, make_float2(c2.x, c2.y))),
                      add2_rn(dp, make_float2(c2.z, c2.w)));
       } else if (MAP == MAPB_INTERP) {
-        ds = mul2_rn(mul2_rn(gw, dn), lds_f32x2(c + 48));    // K/(hi - lo) pair
+        // (dp - delta) d / Z K / (hi - lo)
+        const float4 c2 = lds_f32x4(c + 32);               // -delta pair at z, w
+        ds = mul2_rn(mul2_rn(add2_rn(dp, make_float2(c2.z, c2.w)), dn), lds_f32x2(c + 48));
       }
     }
     if (!FULL) {
@@ -1648,9 +1731,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     kk.flush_t = kMagic + static_cast<float>(p.pot_floor);
     kk.flush = p.flush != 0;
     kk.flush_below = MAP == MAPB_HARD && p.flush && p.fixed_window;
+    kk.Ksc = k_pow2(p.K) ? kk.Kf : 1.0f;
+    kk.mk = __fmul_rn(kMagic, 1.0f / kk.Ksc);
+    const bool sat = (MAP == MAPB_HARD || MAP == MAPB_INTERP) && kv_sat<SURR>(p);
     // table entry bias: bits(M + floor(clamp(u, -1, K))) - bits(M) + 1 (interp)
-    // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), mod 2^32
-    const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - kMagicBits * 8u : 0u - kMagicBits * 4u;
+    // or bits(M + rne(clamp(u, 0, K))) - bits(M) (hard), M = 1.5 * 2^23; on
+    // the saturating path M / K and v in place of M and u; mod 2^32
+    const uint32_t mbits = sat ? __float_as_uint(kk.mk) : kMagicBits;
+    const uint32_t tbias = (MAP == MAPB_INTERP) ? 8u - mbits * 8u : 0u - mbits * 4u;
     const uint32_t tsb = static_cast<uint32_t>(p.TS) * 4u;
     bool ok = true;
     int rc0 = 0, hc = 0, k = 0;
@@ -1688,14 +1776,21 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         const uint32_t cb = st + CST_OFF + ql0 * (kCst * 4);
         const uint32_t tr = st + TAB_OFF + ql0 * tsb + tbias;
         uint32_t pp[8], dd[8];
+        constexpr bool KI = MAP == MAPB_HARD || MAP == MAPB_INTERP;
         if (full) {
-          kv_slice<MAP, SURR, true>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
+          if (KI && sat)
+            kv_slice<MAP, SURR, true, KI>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
+          else
+            kv_slice<MAP, SURR, true, false>(sv, dv, cb, tr, tsb, kk, 0u, pp, dd);
         } else {
           uint32_t vmask = 0;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             vmask |= (key_ok && qbase + i < p.S && (!p.causal || kg <= qbase + i)) ? (1u << i) : 0u;
-          kv_slice<MAP, SURR, false>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
+          if (KI && sat)
+            kv_slice<MAP, SURR, false, KI>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
+          else
+            kv_slice<MAP, SURR, false, false>(sv, dv, cb, tr, tsb, kk, vmask, pp, dd);
         }
         tmem_st8(lane_base + 128 * x + 16 * g, pp);
         tmem_st8(lane_base + 128 * x + 64 + 16 * g, dd);
