@@ -86,12 +86,13 @@ def check_bf16_output(got, want, tol_max=1e-2, tol_mean=1e-3, what=""):
 
 
 def check_decisions(d, got_idx, causal, mode, K, calib, rounding, window, heads=None,
-                    row_block=1024):
+                    row_block=1024, below_policy=0):
     """Kernel decisions (the forward's debug dump) against fp64 rounding:
     agreement >= 99.9 % and every mismatch within 1e-3 of a boundary; masked
     keys read -1 (or the buffer's fill value -7 in key tiles the kernel never
     visits).  ``got_idx`` is the [B,H,S,S] dump, or a dict {(b, h): [S,S]}
-    holding only the heads checked."""
+    holding only the heads checked.  below_policy 1: flushed keys read -2 on
+    both sides."""
     if mode == A.EXACT:
         return
     q = d["q"].double().numpy() * d["q_descale"]
@@ -107,7 +108,7 @@ def check_decisions(d, got_idx, causal, mode, K, calib, rounding, window, heads=
             s = (q[b, h, rr] @ k[b, h].T) / math.sqrt(D)
             valid = (np.arange(S)[None, :] <= rr[:, None]) if causal \
                 else np.ones((len(rr), S), bool)
-            m = A._map_rows(s, valid, mode, K, calib, rounding, window, 15, 0)
+            m = A._map_rows(s, valid, mode, K, calib, rounding, window, 15, below_policy)
             ref = m["idx"]
             dist = boundary_distance_rows(s, valid, mode, K, calib, rounding, window)
             g = np.asarray(g_all[rr], dtype=np.int64)

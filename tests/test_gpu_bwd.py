@@ -41,39 +41,43 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _stored_o(d, causal, mode, K, calib, rnd, window=8.0, heads=None):
+def _stored_o(d, causal, mode, K, calib, rnd, window=8.0, heads=None, below=0):
     """The oracle's forward (with its decision indices), whose O rounded to
     bf16 both backwards take as the stored output."""
     return oracle.attn_fwd(d["q"], d["k"], d["v"], causal, mode, K=K, calib=calib, rounding=rnd,
-                           window=window, heads=heads, want_idx=True)
+                           window=window, heads=heads, want_idx=True, below_policy=below)
 
 
-def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True, O_store=None):
+def _run(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, dump=True, O_store=None,
+         below=0):
     q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
     B, H, S, D = q.shape
     dbg = torch.full((B, H, S, S), -1, dtype=torch.int8, device=DEV) if dump else None
     O, LSE, st = qsm.attention_forward(q, k, v, causal, mode, K, calib, rnd, window=window,
-                                       stats=True, debug_idx=dbg)
+                                       stats=True, debug_idx=dbg, below_policy=below)
     if O_store is not None:
         # heads the oracle left out (NaN) keep the kernel's own output
         Os = torch.from_numpy(np.asarray(O_store, dtype=np.float32)).to(DEV)
         O = torch.where(torch.isnan(Os), O.float(), Os).to(torch.bfloat16).contiguous()
     dQ, dK, dV = qsm.attention_backward(q, k, v, O, dO, LSE, st, causal, mode, K, calib, rnd,
-                                        surr, detach_extrema=detach, window=window)
+                                        surr, detach_extrema=detach, window=window,
+                                        below_policy=below)
     torch.cuda.synchronize()
     out = [dQ.float().cpu().numpy(), dK.float().cpu().numpy(), dV.float().cpu().numpy()]
     return out, (dbg.cpu().numpy() if dump else None)
 
 
-def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None, O_store=None):
+def _oracle(d, causal, mode, K, calib, rnd, surr, detach, window=8.0, heads=None, O_store=None,
+            below=0):
     """The oracle's backward at its own fp64 decisions, delta from the stored
     (bf16) output."""
     return oracle.attn_bwd(d["q"], d["k"], d["v"], d["dO"], causal, mode, K=K, calib=calib,
                            rounding=rnd, surrogate=surr, detach_extrema=detach, window=window,
-                           heads=heads, O=None if O_store is None else to_bf16(O_store))
+                           below_policy=below, heads=heads,
+                           O=None if O_store is None else to_bf16(O_store))
 
 
-def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads, ref):
+def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads, ref, below=0):
     """Rows of dQ and of dK / dV touched by the kernel forward's decision
     mismatches with fp64 rounding (after checking every mismatch lies within
     1e-3 of a boundary); returns boolean [B,H,S] masks and the count.  ref:
@@ -83,7 +87,7 @@ def _flip_rows(d, dec, causal, mode, K, calib, rnd, window, heads, ref):
     dkv = np.zeros((B, H, S), bool)
     if mode != 1 or dec is None:
         return dq, dkv, 0
-    check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads)
+    check_decisions(d, dec, causal, mode, K, calib, rnd, window, heads, below_policy=below)
     n = 0
     for (b, h) in heads:
         valid = (np.arange(S)[None, :] <= np.arange(S)[:, None]) if causal \
@@ -139,6 +143,39 @@ def test_bwd_kinterval_extreme_K(K, calib, rnd, surr):
     got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
     ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
     fq, fkv, n = _flip_rows(d, dec, True, 1, K, calib, rnd, 6.0, [(0, 0), (0, 1)], fwd)
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
+
+
+@pytest.mark.parametrize("K", [3, 12])
+@pytest.mark.parametrize("calib,rnd", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("surr", [1, 2])
+def test_bwd_kinterval_non_pow2_K(K, calib, rnd, surr):
+    """K not a power of two: the passes evaluate the clamped coordinate itself
+    (the saturating form needs K = 2^m), pre and post surrogate."""
+    d = inputs.draw(1, 2, 256, 64, seed=130 + K, with_dO=True)
+    fwd = _stored_o(d, True, 1, K, calib, rnd, window=6.0)
+    got, dec = _run(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
+    ref = _oracle(d, True, 1, K, calib, rnd, surr, False, window=6.0, O_store=fwd["O"])
+    fq, fkv, n = _flip_rows(d, dec, True, 1, K, calib, rnd, 6.0, [(0, 0), (0, 1)], fwd)
+    _check(got, ref, skip=(fq, fkv))
+    assert fq.sum() <= 0.02 * fq.size, n
+
+
+@pytest.mark.parametrize("K", [4, 5])
+@pytest.mark.parametrize("rnd", [0, 1])
+@pytest.mark.parametrize("surr", [0, 1, 2])
+def test_bwd_kinterval_below_flush(K, rnd, surr):
+    """Fixed window with the below-window flush (below_policy = 1, keys below
+    hi - W weigh 0): a window of 2.5 puts a large share of the keys below it.
+    The passes take the clamped coordinate here, whose sign marks them."""
+    W = 2.5
+    d = inputs.draw(1, 2, 256, 64, seed=140 + K, with_dO=True)
+    fwd = _stored_o(d, True, 1, K, 1, rnd, window=W, below=1)
+    got, dec = _run(d, True, 1, K, 1, rnd, surr, False, window=W, O_store=fwd["O"], below=1)
+    ref = _oracle(d, True, 1, K, 1, rnd, surr, False, window=W, O_store=fwd["O"], below=1)
+    assert (fwd["idx"] == -2).sum() > 0.05 * (fwd["idx"] != -1).sum()   # flushed share
+    fq, fkv, n = _flip_rows(d, dec, True, 1, K, 1, rnd, W, [(0, 0), (0, 1)], fwd, below=1)
     _check(got, ref, skip=(fq, fkv))
     assert fq.sum() <= 0.02 * fq.size, n
 
