@@ -187,7 +187,7 @@ __device__ __forceinline__ void on_chunk(const uint32_t (&v)[32], const MapRow &
       x = map_pair<MAP_POT, FLUSH>(r, mr);
     } else {
       x = pair_weights<MAP, false, SAT>(r, mr, flush_below);
-      x = make_float2(__fmul_rn(x.x, fr), __fmul_rn(x.y, fr));
+      x = mul2_rn(x, make_float2(fr, fr));           // into the group's frame
     }
     if (!FULL) {
       x.x = (c0 + 2 * i < lim) ? x.x : 0.0f;
