@@ -703,6 +703,8 @@ __global__ void __launch_bounds__(128 * prep_split<MAP>())
   constexpr bool KI = MAP == MAPB_HARD || MAP == MAPB_INTERP;
   __shared__ float dpart[4][128];
   __shared__ __align__(16) float tks[KI ? 128 * kTabKRow : 4];
+  // the dQ pass may start its prologue once every CTA of this grid runs
+  grid_dep_launch();
   const int row = threadIdx.x & 127, q = threadIdx.x >> 7;
   const int tix = static_cast<int>(blockIdx.x);         // bh * nqt + qt
   const int bh = tix / p.nqt, qt = tix - bh * p.nqt;
@@ -956,6 +958,11 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
+  // The prologue above may overlap the prep kernel's last CTAs; its
+  // constants and tables (and the e4m3 path's bf16 copies) are complete from
+  // here on.  Then the dK/dV pass may start on the SMs this grid frees.
+  grid_dep_wait();
+  grid_dep_launch();
 
   // Tiles of this CTA: cta_tile(0), cta_tile(1), ... of the heaviest-first
   // order (persistent: the next tile's loads and first
@@ -1800,6 +1807,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       }
       if (!ok) break;
       rc0 += 2 * nq / KG::HPU;
+      // the dQ pass (whose fp32 calibration part of dK the read-out adds)
+      // has completed: this pass may have started on the SMs it freed
+      if (k == 0) grid_dep_wait();
       if constexpr (D > 64) {
         // D = 128: 32 columns a group, dV read out first, then dK
         if (!warp_all_b(mbar_wait(bars.acc_full, k & 1, abort))) {
@@ -1886,6 +1896,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       }
     }
   }
+  grid_dep_wait();                                    // no-op once waited
   __syncwarp();
   tc_fence_before();
   __syncthreads();
@@ -1942,6 +1953,26 @@ struct alignas(64) BwdMaps {
   CUtensorMap q_stage, k_stage, v_stage, dO_stage;
 };
 
+// A persistent pass launched with programmatic stream serialization: its
+// CTAs may start (prologue, then grid_dep_wait) while the previous kernel on
+// the stream finishes, once every CTA of that kernel has issued
+// grid_dep_launch or exited.
+template <typename... Args>
+cudaError_t launch_dependent(void (*kern)(Args...), int grid, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kMainThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, const CUtensorMap &mdo) {
@@ -1972,8 +2003,8 @@ qsm_status launch_dq(const BwdArgs &a, BwdParams p, const CUtensorMap &mq, const
   // persistent: one CTA per SM walks the query tiles
   const int ntiles = p.nqt * a.B * a.H;
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
-  kern<<<dim3(grid), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
-  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+  return launch_dependent(kern, grid, smem, a.stream, mq, mk, mv, mdo, p) == cudaSuccess ? QSM_OK
+                                                                           : QSM_ERR_CUDA;
 }
 
 template <int D, int MAP, int SURR>
@@ -2001,8 +2032,8 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
   // persistent: one CTA per SM walks the key tiles
   const int ntiles = p.nkvt * a.B * a.H;
   const int grid = ntiles < sm_count() ? ntiles : sm_count();
-  kern<<<dim3(grid), kMainThreads, smem, a.stream>>>(mq, mk, mv, mdo, p);
-  return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
+  return launch_dependent(kern, grid, smem, a.stream, mq, mk, mv, mdo, p) == cudaSuccess ? QSM_OK
+                                                                           : QSM_ERR_CUDA;
 }
 
 template <int D, int MAP, int SURR, int CAL>
