@@ -304,6 +304,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *bars.tmem_slot;
+  // the prep kernel (launched as a dependent at D = 64) may start on the SMs
+  // this grid frees; it waits for this grid before reading LSE* and delta*
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -741,6 +744,9 @@ __global__ void __launch_bounds__(128 * prep_split<MAP>())
       z[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
   RowMap rm{};
+  // post surrogate at D = 64: launched as a dependent of the row pass, whose
+  // LSE* and delta* the constants read (a no-op for a plain launch)
+  if (SURR == SURR_POST) grid_dep_wait();
   RowC kc = row_constants<MAP, SURR, CAL>(p, ri, rm);
   if (KI)
     row_tables<MAP, SURR, CAL, NQ>(p, rm, kc.invZ, q, tks + row * p.TS,
@@ -1953,16 +1959,16 @@ struct alignas(64) BwdMaps {
   CUtensorMap q_stage, k_stage, v_stage, dO_stage;
 };
 
-// A persistent pass launched with programmatic stream serialization: its
-// CTAs may start (prologue, then grid_dep_wait) while the previous kernel on
-// the stream finishes, once every CTA of that kernel has issued
-// grid_dep_launch or exited.
+// A kernel launched with programmatic stream serialization: its CTAs may
+// start (prologue, then grid_dep_wait) while the previous kernel on the
+// stream finishes, once every CTA of that kernel has issued grid_dep_launch
+// or exited.
 template <typename... Args>
-cudaError_t launch_dependent(void (*kern)(Args...), int grid, size_t smem, cudaStream_t stream,
-                             Args... args) {
+cudaError_t launch_dependent_block(void (*kern)(Args...), int grid, int block, size_t smem,
+                                   cudaStream_t stream, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kMainThreads);
+  cfg.blockDim = dim3(block);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1971,6 +1977,12 @@ cudaError_t launch_dependent(void (*kern)(Args...), int grid, size_t smem, cudaS
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+// The persistent passes (640 threads).
+template <typename... Args>
+cudaError_t launch_dependent(void (*kern)(Args...), int grid, size_t smem, cudaStream_t stream,
+                             Args... args) {
+  return launch_dependent_block(kern, grid, kMainThreads, smem, stream, args...);
 }
 
 template <int D, int MAP, int SURR, int CAL>
@@ -2038,8 +2050,18 @@ qsm_status launch_dkdv(const BwdArgs &a, BwdParams p, const CUtensorMap &mq,
 
 template <int D, int MAP, int SURR, int CAL>
 qsm_status launch_prep(const BwdArgs &a, const BwdParams &p) {
-  qsm_bwd_prep<D, MAP, SURR, CAL><<<dim3(p.nqt * a.B * a.H), 128 * prep_split<MAP>(), 0,
-                                    a.stream>>>(p);
+  const int grid = p.nqt * a.B * a.H, block = 128 * prep_split<MAP>();
+  if (SURR == SURR_POST && D == 64) {
+    // behind the row pass, as its dependent (it waits before the row
+    // constants).  Measured against the plain launch on one box: +0.3-2.5 %
+    // for the D = 64 post-surrogate calls, but -5 to -7 % at D = 128 with
+    // min-max calibration, so D = 128 keeps the plain launch.
+    return launch_dependent_block(qsm_bwd_prep<D, MAP, SURR, CAL>, grid, block, 0, a.stream, p) ==
+                   cudaSuccess
+               ? QSM_OK
+               : QSM_ERR_CUDA;
+  }
+  qsm_bwd_prep<D, MAP, SURR, CAL><<<dim3(grid), block, 0, a.stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? QSM_OK : QSM_ERR_CUDA;
 }
 
