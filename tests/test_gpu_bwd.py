@@ -340,3 +340,37 @@ def test_bwd_fp8(S, causal, mode, K, calib, rnd, surr, detach):
                             [(0, 0), (0, 1)], fwd)
     _check(got, ref, skip=(fq, fkv))
     assert fq.sum() <= 0.02 * fq.size, n
+
+
+@pytest.mark.parametrize("surr", [1, 2])
+@pytest.mark.parametrize("D", [64, 128])
+def test_bwd_back_to_back_shared_workspace(surr, D):
+    """Backward calls queued back to back on one stream, sharing one
+    workspace, without a synchronisation between them (within a call the
+    passes after the first start as programmatic dependents of the kernel
+    before them): every call's gradients equal those of the same call run
+    alone, bit for bit.  Fixed-window hard rounding has no calibration term,
+    so no fp32 reductions and the results are deterministic."""
+    K, calib, rnd, W = 4, 1, 1, 6.0
+    runs = []
+    for seed in (160, 161):
+        d = inputs.draw(1, 4, 512, D, seed=seed + D, with_dO=True)
+        q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
+        O, LSE, st = qsm.attention_forward(q, k, v, True, 1, K, calib, rnd, window=W, stats=True)
+        runs.append((q, k, v, O, dO, LSE, st))
+
+    def bwd(x, ws=None):
+        q, k, v, O, dO, LSE, st = x
+        return qsm.attention_backward(q, k, v, O, dO, LSE, st, True, 1, K, calib, rnd, surr,
+                                      window=W, workspace=ws)
+
+    alone = []
+    for x in runs:
+        alone.append(bwd(x))
+        torch.cuda.synchronize()
+    ws = torch.empty(qsm.qsm_attn_bwd_workspace_size(1, 4, 512, D), dtype=torch.uint8, device=DEV)
+    queued = [bwd(runs[i % 2], ws) for i in range(6)]
+    torch.cuda.synchronize()
+    for i, got in enumerate(queued):
+        for g, r, name in zip(got, alone[i % 2], ("dQ", "dK", "dV")):
+            assert torch.equal(g, r), (i, name)
