@@ -374,3 +374,43 @@ def test_bwd_back_to_back_shared_workspace(surr, D):
     for i, got in enumerate(queued):
         for g, r, name in zip(got, alone[i % 2], ("dQ", "dK", "dV")):
             assert torch.equal(g, r), (i, name)
+
+
+def _align256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_bwd_post_row_statistics(D):
+    """The post surrogate's row pass against plain fp64 softmax statistics:
+    LSE*_r = log sum_j exp(s_rj) and delta*_r = sum_j softmax(s_r)_j dO_r.v_j
+    over the valid keys.  White box: the pass writes them to the backward
+    workspace at byte offset align256(B H S D 4) (after the fp32 calibration
+    part of dK), 8 floats a row, LSE* first, then delta*.  The bound is the
+    fp32 sums' (and the exponentials') error, far below what the gradient
+    tolerances can see: LSE* within 5e-6, and delta* -- a signed sum, whose
+    error scales with sum_j p_j |dp_j| rather than with delta* itself --
+    within 5e-6 of that scale (both measure below 1e-6 here)."""
+    B, H, S = 1, 4, 512
+    d = inputs.draw(B, H, S, D, seed=170 + D, with_dO=True)
+    q, k, v, dO = (d[n].to(DEV).contiguous() for n in ("q", "k", "v", "dO"))
+    O, LSE, st = qsm.attention_forward(q, k, v, True, 1, 4, 1, 1, window=6.0, stats=True)
+    ws = torch.zeros(qsm.qsm_attn_bwd_workspace_size(B, H, S, D), dtype=torch.uint8, device=DEV)
+    qsm.attention_backward(q, k, v, O, dO, LSE, st, True, 1, 4, 1, 1, 2, window=6.0, workspace=ws)
+    torch.cuda.synchronize()
+    off = _align256(B * H * S * D * 4)
+    rw = ws[off:off + B * H * S * 8 * 4].view(torch.float32).view(B, H, S, 8).cpu().numpy()
+    q64, k64, v64, g64 = (d[n].double().numpy() for n in ("q", "k", "v", "dO"))
+    s = np.einsum("bhid,bhjd->bhij", q64, k64) / np.sqrt(D)
+    s = np.where(np.tril(np.ones((S, S), bool)), s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    Lsum = e.sum(axis=-1)
+    lse = m[..., 0] + np.log(Lsum)
+    dp = np.einsum("bhid,bhjd->bhij", g64, v64)
+    delta = (e * dp).sum(axis=-1) / Lsum
+    scale = (e * np.abs(dp)).sum(axis=-1) / Lsum
+    err_l = np.abs(rw[..., 0] - lse).max()
+    err_d = (np.abs(rw[..., 1] - delta) / scale).max()
+    assert err_l <= 5e-6, err_l
+    assert err_d <= 5e-6, err_d
